@@ -1,0 +1,209 @@
+"""fp64 CPU oracle for the routing-weighted SiTU-GLU -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path
+(``ffn_gated_activation_b200``) never imports it, and it never imports the
+product path: the two share no code.
+
+The arithmetic lives in ``situ_oracle.c`` (plain C, IEEE double, one element
+at a time); this module only builds that file with gcc and marshals numpy
+arrays through ctypes.
+
+Sources followed (see the C file for the per-function citations):
+  * Megatron-LM PR #6673 "[Dev] Add SiTU-GLU through Transformer Engine",
+    section "Activation": T_g = b1 tanh(G/b1) sigmoid(G), T_u = b2 tanh(U/b2),
+    Y = T_g T_u.
+  * NeMo AutoModel API, kimi_k3.situ: `_situ_fwd_core` (Y = situ(g) up(u0) w,
+    optional linear beta), `_situ_bwd_core` (analytic d_g, d_u and the
+    routing-weight reduction), `_WeightedSiTUFunction` (gate/up halves).
+
+Every function is pinned by tests/test_oracle_pins.py; no function here is
+"parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "situ_oracle.c")
+LIBRARY = os.path.join(_HERE, "libsitu_oracle.so")
+
+DTYPE_BF16 = 0
+DTYPE_F32 = 1
+RW_ROW = 0
+RW_SCALAR = 1
+
+# gcc flags: plain IEEE double, no fast-math, no contraction into FMA, so the
+# arithmetic is exactly what the C source spells out.
+CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math"]
+
+
+def build(output: str = LIBRARY, mutant: int = 0, force: bool = False) -> str:
+    """Compile situ_oracle.c with gcc into ``output``.  ``mutant`` > 0 builds a
+    copy with the planted mistake number ``mutant`` (used only by the pin tests
+    to show the pins reject it).  Rebuilds when the source is newer."""
+    if (not force and os.path.exists(output)
+            and os.path.getmtime(output) >= os.path.getmtime(SOURCE)):
+        return output
+    tmp = output + f".tmp{os.getpid()}"
+    cmd = ["gcc", *CFLAGS, f"-DSITU_ORACLE_MUTANT={int(mutant)}", SOURCE, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, output)
+    return output
+
+
+_I64 = ctypes.c_int64
+_INT = ctypes.c_int
+_DBL = ctypes.c_double
+_VP = ctypes.c_void_p
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(_VP)
+
+
+def _dtype_code(a: np.ndarray) -> int:
+    if a.dtype == np.uint16:
+        return DTYPE_BF16  # raw bf16 bit patterns
+    if a.dtype == np.float32:
+        return DTYPE_F32
+    raise TypeError(f"oracle inputs are bf16 bit patterns (uint16) or float32, got {a.dtype}")
+
+
+@dataclass
+class BackwardResult:
+    dg: np.ndarray   # [nrows, inter] float64, dL/dG
+    du: np.ndarray   # [nrows, inter] float64, dL/dU
+    dw: np.ndarray   # [nrows] float64, per-row routing-weight gradient
+    cg: np.ndarray   # [nrows, inter] float64, uncancelled magnitude of dG
+    sw: np.ndarray   # [nrows] float64, sum of |go T_g T_u| per row
+
+
+class Oracle:
+    """ctypes handle on one build of situ_oracle.c (the oracle, or a mutant)."""
+
+    def __init__(self, path: str = LIBRARY):
+        self.path = path
+        lib = ctypes.CDLL(path)
+        lib.situ_oracle_gate.argtypes = [_DBL, _DBL, ctypes.POINTER(_DBL), ctypes.POINTER(_DBL), ctypes.POINTER(_DBL)]
+        lib.situ_oracle_gate.restype = None
+        lib.situ_oracle_up.argtypes = [_DBL, _INT, _DBL, ctypes.POINTER(_DBL), ctypes.POINTER(_DBL)]
+        lib.situ_oracle_up.restype = None
+        lib.situ_oracle_gate_n.argtypes = [_I64, _VP, _DBL, _VP, _VP, _VP]
+        lib.situ_oracle_gate_n.restype = None
+        lib.situ_oracle_up_n.argtypes = [_I64, _VP, _INT, _DBL, _VP, _VP]
+        lib.situ_oracle_up_n.restype = None
+        lib.situ_oracle_fwd.argtypes = [_INT, _VP, _I64, _I64, _VP, _I64, _INT, _VP, _INT, _I64,
+                                        _DBL, _INT, _DBL, _VP]
+        lib.situ_oracle_fwd.restype = _INT
+        lib.situ_oracle_bwd.argtypes = [_INT, _VP, _I64, _I64, _VP, _I64, _INT, _VP, _INT, _I64,
+                                        _DBL, _INT, _DBL, _VP, _I64, _VP, _VP, _VP, _VP, _VP]
+        lib.situ_oracle_bwd.restype = _INT
+        lib.situ_oracle_dw_scalar.argtypes = [_INT, _VP, _I64, _I64, _I64, _DBL, _INT, _DBL, _VP, _I64,
+                                              ctypes.POINTER(_DBL), ctypes.POINTER(_DBL)]
+        lib.situ_oracle_dw_scalar.restype = _INT
+        lib.situ_oracle_mutant_id.restype = _INT
+        self._lib = lib
+        self.mutant_id = lib.situ_oracle_mutant_id()
+
+    # -- scalar branches -----------------------------------------------------
+    def gate(self, g, beta):
+        """T_g, T_g' and the uncancelled magnitude of T_g' at each g (float64)."""
+        g = np.ascontiguousarray(np.atleast_1d(np.asarray(g, dtype=np.float64)))
+        t, d, m = (np.empty_like(g) for _ in range(3))
+        self._lib.situ_oracle_gate_n(g.size, _ptr(g), float(beta), _ptr(t), _ptr(d), _ptr(m))
+        return t, d, m
+
+    def up(self, u, linear_beta):
+        """T_u and T_u' at each u; linear_beta None means T_u = u."""
+        u = np.ascontiguousarray(np.atleast_1d(np.asarray(u, dtype=np.float64)))
+        t, d = np.empty_like(u), np.empty_like(u)
+        has = linear_beta is not None
+        self._lib.situ_oracle_up_n(u.size, _ptr(u), int(has), float(linear_beta if has else 0.0),
+                                   _ptr(t), _ptr(d))
+        return t, d
+
+    # -- rows ------------------------------------------------------------------
+    @staticmethod
+    def _rows(rows, n_all):
+        if rows is None:
+            return None, n_all
+        r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        if r.size and (r.min() < 0 or r.max() >= n_all):
+            raise IndexError("row index out of range")
+        return r, r.size
+
+    def fwd(self, gate_up, rw, beta, linear_beta=None, rows=None, rw_mode=RW_ROW, inter=None):
+        """Y (float64, [nrows, inter]) for the selected rows of gate_up [T, >= 2I].
+        rw is float32 or bf16 bits: [T] / [T, 1] (row mode) or one value (scalar)."""
+        gate_up = np.ascontiguousarray(gate_up)
+        T, width = gate_up.shape
+        inter = width // 2 if inter is None else int(inter)
+        r, n = self._rows(rows, T)
+        rw_c = np.ascontiguousarray(rw).reshape(-1)
+        y = np.empty((n, inter), dtype=np.float64)
+        has = linear_beta is not None
+        rc = self._lib.situ_oracle_fwd(_dtype_code(gate_up), _ptr(gate_up), width, inter, _ptr(r), n,
+                                       _dtype_code(rw_c), _ptr(rw_c), int(rw_mode), 1,
+                                       float(beta), int(has), float(linear_beta if has else 0.0), _ptr(y))
+        if rc != 0:
+            raise ValueError("oracle fwd rejected its arguments")
+        return y
+
+    def bwd(self, gate_up, rw, grad_out, beta, linear_beta=None, rows=None, rw_mode=RW_ROW, inter=None):
+        """Analytic backward for the selected rows; grad_out is [T, >= I] in
+        gate_up's dtype.  Returns a BackwardResult of float64 arrays."""
+        gate_up = np.ascontiguousarray(gate_up)
+        grad_out = np.ascontiguousarray(grad_out)
+        if grad_out.dtype != gate_up.dtype:
+            raise TypeError("grad_out must have gate_up's dtype")
+        T, width = gate_up.shape
+        inter = width // 2 if inter is None else int(inter)
+        r, n = self._rows(rows, T)
+        rw_c = np.ascontiguousarray(rw).reshape(-1)
+        dg = np.empty((n, inter)); du = np.empty((n, inter)); cg = np.empty((n, inter))
+        dw = np.empty(n); sw = np.empty(n)
+        has = linear_beta is not None
+        rc = self._lib.situ_oracle_bwd(_dtype_code(gate_up), _ptr(gate_up), width, inter, _ptr(r), n,
+                                       _dtype_code(rw_c), _ptr(rw_c), int(rw_mode), 1,
+                                       float(beta), int(has), float(linear_beta if has else 0.0),
+                                       _ptr(grad_out), grad_out.shape[1],
+                                       _ptr(dg), _ptr(du), _ptr(dw), _ptr(cg), _ptr(sw))
+        if rc != 0:
+            raise ValueError("oracle bwd rejected its arguments")
+        return BackwardResult(dg=dg, du=du, dw=dw, cg=cg, sw=sw)
+
+    def dw_scalar(self, gate_up, grad_out, beta, linear_beta=None, inter=None):
+        """Gradient of one routing weight broadcast to all rows: (total, sum of |terms|)."""
+        gate_up = np.ascontiguousarray(gate_up)
+        grad_out = np.ascontiguousarray(grad_out)
+        T, width = gate_up.shape
+        inter = width // 2 if inter is None else int(inter)
+        total, mag = _DBL(), _DBL()
+        has = linear_beta is not None
+        rc = self._lib.situ_oracle_dw_scalar(_dtype_code(gate_up), _ptr(gate_up), width, inter, T,
+                                             float(beta), int(has), float(linear_beta if has else 0.0),
+                                             _ptr(grad_out), grad_out.shape[1],
+                                             ctypes.byref(total), ctypes.byref(mag))
+        if rc != 0:
+            raise ValueError("oracle dw_scalar rejected its arguments")
+        return total.value, mag.value
+
+
+_DEFAULT = None
+
+
+def load(path: str | None = None) -> Oracle:
+    """The oracle (built on first use if the shared object is missing or stale)."""
+    global _DEFAULT
+    if path is not None:
+        return Oracle(path)
+    if _DEFAULT is None:
+        build()
+        _DEFAULT = Oracle(LIBRARY)
+    return _DEFAULT

@@ -1,0 +1,341 @@
+"""Pins for the fp64 oracle (CPU only).
+
+The oracle is the definition the CUDA path is checked against, so it is
+itself checked here against things other than itself:
+
+  * 50-digit mpmath values of the two branch functions, and mpmath's
+    numerical derivative of them (independent of the analytic derivative);
+  * exact identities that follow from sigmoid(x) + sigmoid(-x) = 1:
+        T_g(g) - T_g(-g) = beta tanh(g / beta)
+        T_g(g) + T_g(-g) = beta tanh(g / beta) tanh(g / 2);
+  * the SwiGLU limit beta, beta_L -> infinity against torch's library SiLU
+    and its autograd derivative ("unary F.silu is not equivalent" -- the
+    Megatron-LM PR #6673 "Design" list -- holds only at finite beta);
+  * central finite differences of the oracle's own forward;
+  * torch float64 autograd of the formula for whole rows (independent
+    derivatives, strided rows, both dtypes, both routing-weight modes);
+  * special rows (G = 0, U = 0) whose gradients have closed forms;
+  * brute-force compensated sums for the routing-weight gradient.
+
+Each pin is a plain function of an oracle handle.  ``test_mutant_rejected``
+rebuilds situ_oracle.c with each planted mistake (-DSITU_ORACLE_MUTANT=n: a
+dropped term, a wrong sign, a transposed operand, swapped halves, an ignored
+stride, ...) and checks that at least one pin rejects it.
+"""
+import math
+import os
+
+import mpmath
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+mpmath.mp.dps = 50
+RNG_SEED = 12345
+
+
+# ---- high-precision restatements (mpmath, 50 digits) --------------------------
+
+def _mp_gate(g, beta):
+    g = mpmath.mpf(g)
+    return beta * mpmath.tanh(g / beta) / (1 + mpmath.exp(-g))
+
+
+def _mp_up(u, lb):
+    return lb * mpmath.tanh(mpmath.mpf(u) / lb)
+
+
+def _mp_diff(f, x):
+    """mpmath's numerical derivative at 400 working digits: enough that a slope
+    as small as 1e-174 next to function values near 1 keeps its double digits."""
+    with mpmath.workdps(400):
+        return float(mpmath.diff(f, mpmath.mpf(x)))
+
+
+def _close(a, b, rtol, atol=0.0):
+    return abs(a - b) <= rtol * abs(b) + atol
+
+
+# ---- pins ------------------------------------------------------------------------
+
+def pin_gate_values_mpmath(o):
+    """T_g and T_g' against 50-digit values, including saturation at |g| = 20, 60
+    (the fixed-value coverage asked for in the Megatron-LM PR #6673 review)."""
+    pts = [0.0, 0.5, -0.5, 1.0, -1.0, 4.0, -4.0, 20.0, -20.0, 60.0, -60.0, 7.3, -7.3,
+           1e-6, -1e-6, -1.2187557268720125, 2.5e-3, -33.0]
+    for beta in (1.0, 4.0, 16.0):
+        t, d, m = o.gate(pts, beta)
+        for k, g in enumerate(pts):
+            ref = float(_mp_gate(g, beta))
+            assert _close(t[k], ref, 4e-15, 1e-300), (beta, g, t[k], ref)
+            dref = _mp_diff(lambda x: _mp_gate(x, beta), g)
+            assert abs(d[k] - dref) <= 1e-14 * m[k] + 1e-300, (beta, g, d[k], dref)
+
+
+def pin_up_values_mpmath(o):
+    """T_u and T_u' against 50-digit values, including the beta_L soft cap."""
+    pts = [0.0, 1.0, -1.0, 25.0, -25.0, 60.0, -60.0, 1e-3, 200.0, -3.75]
+    for lb in (25.0, 1.0, 1000.0):
+        t, d = o.up(pts, lb)
+        for k, u in enumerate(pts):
+            ref = float(_mp_up(u, lb))
+            assert _close(t[k], ref, 4e-15, 1e-300), (lb, u, t[k], ref)
+            dref = _mp_diff(lambda x: _mp_up(x, lb), u)
+            assert _close(d[k], dref, 1e-14, 1e-300), (lb, u, d[k], dref)
+
+
+def pin_gate_parity_identities(o):
+    """sigmoid(x) + sigmoid(-x) = 1 and sigmoid(x) - sigmoid(-x) = tanh(x/2)
+    give the odd and even parts of T_g in closed form."""
+    rng = np.random.default_rng(RNG_SEED)
+    g = np.concatenate([rng.normal(0.0, 3.0, 400), rng.uniform(-70, 70, 100)])
+    for beta in (0.5, 1.0, 4.0, 16.0):
+        tp, _, _ = o.gate(g, beta)
+        tn, _, _ = o.gate(-g, beta)
+        scale = np.abs(tp) + np.abs(tn)
+        odd = np.array([beta * math.tanh(x / beta) for x in g])
+        even = np.array([beta * math.tanh(x / beta) * math.tanh(x / 2.0) for x in g])
+        assert np.all(np.abs((tp - tn) - odd) <= 1e-14 * scale + 1e-300)
+        assert np.all(np.abs((tp + tn) - even) <= 1e-14 * scale + 1e-300)
+
+
+def pin_gate_special_points(o):
+    """T_g(0) = 0 and T_g'(0) = 1/2 exactly; for beta = 4, T_g' vanishes at the
+    single negative minimum G* (found by mpmath) and T_g is smallest there."""
+    for beta in (1.0, 4.0, 16.0):
+        t, d, _ = o.gate([0.0], beta)
+        assert t[0] == 0.0 and d[0] == 0.5
+    g_star = float(mpmath.findroot(lambda x: mpmath.diff(lambda y: _mp_gate(y, 4.0), x), -1.2))
+    assert abs(g_star - (-1.2187557268720125)) < 1e-12
+    t, d, m = o.gate([g_star, g_star - 1e-3, g_star + 1e-3], 4.0)
+    assert abs(d[0]) <= 1e-15 * m[0]
+    assert t[1] > t[0] and t[2] > t[0]
+
+
+def pin_bounds_and_sign(o):
+    """|T_g| <= beta with the sign of g; |T_u| <= min(|u|, beta_L) with the sign of u."""
+    rng = np.random.default_rng(RNG_SEED + 1)
+    x = np.concatenate([rng.normal(0, 4, 500), rng.uniform(-100, 100, 200)])
+    for beta in (1.0, 4.0, 16.0):
+        t, _, _ = o.gate(x, beta)
+        assert np.all(np.abs(t) <= beta)
+        assert np.all(np.sign(t) == np.sign(x))
+    for lb in (1.0, 25.0):
+        t, _ = o.up(x, lb)
+        assert np.all(np.abs(t) <= np.minimum(np.abs(x), lb))
+        assert np.all(np.sign(t) == np.sign(x))
+    t, _ = o.up([60.0, -60.0], 25.0)
+    assert t[0] < 25.0 and t[1] > -25.0
+
+
+def pin_swiglu_limit(o):
+    """As beta, beta_L -> infinity, T_g -> SiLU(g) = g sigmoid(g) and T_u -> u:
+    compare with torch's SiLU and its autograd derivative in float64."""
+    rng = np.random.default_rng(RNG_SEED + 2)
+    g = rng.normal(0, 3, 300)
+    gt = torch.tensor(g, dtype=torch.float64, requires_grad=True)
+    silu = torch.nn.functional.silu(gt)
+    (dsilu,) = torch.autograd.grad(silu.sum(), gt)
+    t, d, _ = o.gate(g, 1e12)
+    np.testing.assert_allclose(t, silu.detach().numpy(), rtol=1e-12, atol=1e-300)
+    np.testing.assert_allclose(d, dsilu.numpy(), rtol=1e-11, atol=1e-14)
+    tu, du = o.up(g, 1e12)
+    np.testing.assert_allclose(tu, g, rtol=1e-12)
+    np.testing.assert_allclose(du, 1.0, rtol=1e-12)
+
+
+def pin_linear_beta_none(o):
+    """Without a linear beta the up branch is the identity, exactly."""
+    rng = np.random.default_rng(RNG_SEED + 3)
+    u = rng.normal(0, 10, 200)
+    t, d = o.up(u, None)
+    assert np.array_equal(t, u) and np.all(d == 1.0)
+
+
+def pin_finite_differences(o):
+    """Central differences of the oracle's forward against its analytic derivatives."""
+    rng = np.random.default_rng(RNG_SEED + 4)
+    x = np.concatenate([rng.normal(0, 3, 200), rng.uniform(-40, 40, 50)])
+    h = 1e-5 * np.maximum(1.0, np.abs(x))
+    for beta in (1.0, 4.0, 16.0):
+        tp, _, _ = o.gate(x + h, beta)
+        tm, _, _ = o.gate(x - h, beta)
+        _, d, m = o.gate(x, beta)
+        fd = (tp - tm) / (2 * h)
+        assert np.all(np.abs(fd - d) <= 1e-7 * (m + np.abs(fd)) + 1e-12), beta
+    for lb in (1.0, 25.0):
+        tp, _ = o.up(x + h, lb)
+        tm, _ = o.up(x - h, lb)
+        _, d = o.up(x, lb)
+        fd = (tp - tm) / (2 * h)
+        assert np.all(np.abs(fd - d) <= 1e-7 * np.abs(fd) + 1e-12), lb
+
+
+def _torch_rows(gu, rw, go, inter, beta, lb, scalar):
+    """float64 torch statement of the chain, differentiated by autograd."""
+    G = torch.tensor(gu[:, :inter], dtype=torch.float64, requires_grad=True)
+    U = torch.tensor(gu[:, inter:2 * inter], dtype=torch.float64, requires_grad=True)
+    W = torch.tensor(rw, dtype=torch.float64, requires_grad=True)
+    GO = torch.tensor(go[:, :inter], dtype=torch.float64)
+    tg = beta * torch.tanh(G / beta) * torch.sigmoid(G)
+    tu = U if lb is None else lb * torch.tanh(U / lb)
+    Y = tg * tu * (W if scalar else W[:, None])
+    (Y * GO).sum().backward()
+    return Y.detach().numpy(), G.grad.numpy(), U.grad.numpy(), W.grad.numpy()
+
+
+def _as_f64(a):
+    return workloads.bf16_bits_to_f32(a).astype(np.float64) if a.dtype == np.uint16 else a.astype(np.float64)
+
+
+def pin_torch_autograd_rows(o):
+    """Whole rows (padded row stride, bf16 and fp32 storage, row-aligned and
+    scalar routing weights, with and without a linear beta) against float64
+    autograd of the formula."""
+    rng = np.random.default_rng(RNG_SEED + 5)
+    T, I, pad = 5, 16, 3
+    for dtype in ("bf16", "f32"):
+        for lb in (25.0, 1.5, None):
+            for scalar in (False, True):
+                raw = rng.normal(0, 3, (T, 2 * I + pad)).astype(np.float32)
+                raw[0, 2] = 45.0
+                raw[1, I + 4] = -60.0
+                raw_go = rng.normal(0, 1, (T, I + pad)).astype(np.float32)
+                if dtype == "bf16":
+                    gu, go = workloads.f32_to_bf16_bits(raw), workloads.f32_to_bf16_bits(raw_go)
+                else:
+                    gu, go = raw, raw_go
+                rw = (rng.uniform(0.1, 1.0, 1 if scalar else T)).astype(np.float32)
+                mode = oracle.RW_SCALAR if scalar else oracle.RW_ROW
+                beta = 4.0
+                Y, dG, dU, dW = _torch_rows(_as_f64(gu), rw.astype(np.float64), _as_f64(go),
+                                             I, beta, lb, scalar)
+                y = o.fwd(gu, rw, beta, lb, rw_mode=mode, inter=I)
+                b = o.bwd(gu, rw, go, beta, lb, rw_mode=mode, inter=I)
+                np.testing.assert_allclose(y, Y, rtol=1e-13, atol=1e-300)
+                np.testing.assert_allclose(b.dg, dG, rtol=1e-12, atol=1e-13 * np.abs(dG).max())
+                np.testing.assert_allclose(b.du, dU, rtol=1e-12, atol=1e-13 * np.abs(dU).max())
+                if scalar:
+                    total, _ = o.dw_scalar(gu, go, beta, lb, inter=I)
+                    assert _close(total, dW[0], 1e-12, 1e-13 * b.sw.sum())
+                else:
+                    np.testing.assert_allclose(b.dw, dW, rtol=1e-12, atol=1e-13 * b.sw.max())
+
+
+def pin_special_rows(o):
+    """A zero gate column gives Y = 0, dU = 0, dG = go w T_u / 2; a zero up
+    column gives Y = 0, dG = 0, dU = go w T_g (sech^2(0) = 1)."""
+    I = 8
+    g_vals = np.array([1.5, -2.0, 3.0, -0.75, 5.0, -6.0, 0.0, 0.0], dtype=np.float32)
+    u_vals = np.array([0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 2.5, -1.25], dtype=np.float32)
+    gu = np.concatenate([g_vals, u_vals])[None, :]
+    go = np.array([[0.5, -1.0, 2.0, 1.5, -0.25, 3.0, -2.0, 0.75]], dtype=np.float32)
+    rw = np.array([0.625], dtype=np.float32)
+    w = 0.625
+    for lb in (25.0, None):
+        y = o.fwd(gu, rw, 4.0, lb, inter=I)
+        b = o.bwd(gu, rw, go, 4.0, lb, inter=I)
+        tg, _, _ = o.gate(g_vals.astype(np.float64), 4.0)
+        tu, _ = o.up(u_vals.astype(np.float64), lb)
+        assert np.all(y == 0.0)
+        # up column zero (first six): dG = 0, dU = go w T_g
+        assert np.all(b.dg[0, :6] == 0.0)
+        np.testing.assert_allclose(b.du[0, :6], go[0, :6] * w * tg[:6], rtol=1e-15)
+        # gate column zero (last two): dU = 0, dG = go w T_u / 2
+        assert np.all(b.du[0, 6:] == 0.0)
+        np.testing.assert_allclose(b.dg[0, 6:], go[0, 6:] * w * tu[6:] / 2.0, rtol=1e-15)
+
+
+def pin_dw_bruteforce(o):
+    """The row-aligned routing-weight gradient is sum_i go * Y / w (Y is linear
+    in w), summed here with math.fsum; the broadcast-scalar gradient is the
+    sum of those over every row."""
+    rng = np.random.default_rng(RNG_SEED + 6)
+    T, I = 6, 40
+    gu = workloads.f32_to_bf16_bits(rng.normal(0, 2, (T, 2 * I)).astype(np.float32))
+    go = workloads.f32_to_bf16_bits(rng.normal(0, 1, (T, I)).astype(np.float32))
+    rw = rng.uniform(0.2, 1.0, T).astype(np.float32)
+    y = o.fwd(gu, rw, 4.0, 25.0)
+    b = o.bwd(gu, rw, go, 4.0, 25.0)
+    gof = _as_f64(go)
+    for r in range(T):
+        ref = math.fsum((gof[r] * y[r] / float(rw[r])).tolist())
+        assert _close(b.dw[r], ref, 1e-13, 1e-15 * b.sw[r]), (r, b.dw[r], ref)
+        assert _close(b.sw[r], math.fsum(np.abs(gof[r] * y[r] / float(rw[r])).tolist()), 1e-13)
+    total, mag = o.dw_scalar(gu, go, 4.0, 25.0)
+    assert _close(total, math.fsum(b.dw.tolist()), 1e-13, 1e-15 * mag)
+
+
+def pin_bf16_loading(o):
+    """bf16 bit patterns decode exactly: the same values given as float32
+    produce identical results."""
+    rng = np.random.default_rng(RNG_SEED + 7)
+    f = rng.normal(0, 4, (3, 24)).astype(np.float32)
+    bits = workloads.f32_to_bf16_bits(f)
+    exact = workloads.bf16_bits_to_f32(bits)
+    go_bits = workloads.f32_to_bf16_bits(rng.normal(0, 1, (3, 12)).astype(np.float32))
+    rw = np.array([0.5, 1.0, 0.25], dtype=np.float32)
+    assert np.array_equal(o.fwd(bits, rw, 4.0, 25.0), o.fwd(exact, rw, 4.0, 25.0))
+    b1 = o.bwd(bits, rw, go_bits, 4.0, 25.0)
+    b2 = o.bwd(exact, rw, workloads.bf16_bits_to_f32(go_bits), 4.0, 25.0)
+    assert np.array_equal(b1.dg, b2.dg) and np.array_equal(b1.dw, b2.dw)
+    one = np.array([[0x3F80, 0x3F80]], dtype=np.uint16)  # G = U = 1.0
+    y = o.fwd(one, np.array([1.0], dtype=np.float32), 4.0, 25.0)
+    assert _close(y[0, 0], float(_mp_gate(1.0, 4.0) * _mp_up(1.0, 25.0)), 4e-15)
+
+
+PINS = [
+    pin_gate_values_mpmath,
+    pin_up_values_mpmath,
+    pin_gate_parity_identities,
+    pin_gate_special_points,
+    pin_bounds_and_sign,
+    pin_swiglu_limit,
+    pin_linear_beta_none,
+    pin_finite_differences,
+    pin_torch_autograd_rows,
+    pin_special_rows,
+    pin_dw_bruteforce,
+    pin_bf16_loading,
+]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
+def test_pin(pin, oracle_lib):
+    assert oracle_lib.mutant_id == 0
+    pin(oracle_lib)
+
+
+# Planted mistakes compiled into situ_oracle.c under -DSITU_ORACLE_MUTANT=n.
+MUTANTS = {
+    1: "dropped product-rule term in T_g'",
+    2: "wrong sign of the second T_g' term",
+    3: "u * beta_L instead of u / beta_L",
+    4: "sigmoid(-g) instead of sigmoid(g)",
+    5: "routing weight dropped from Y",
+    6: "dG uses T_g where T_u belongs",
+    7: "dU uses T_u where T_g belongs",
+    8: "gate and up halves swapped",
+    9: "upstream gradient dropped from d_w",
+    10: "linear beta ignored",
+    11: "sech^2 with exp(-|a|) instead of exp(-2|a|)",
+    12: "row stride ignored",
+}
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS), ids=[f"m{k}" for k in sorted(MUTANTS)])
+def test_mutant_rejected(mutant, tmp_path):
+    path = oracle.build(output=os.path.join(tmp_path, f"libsitu_oracle_m{mutant}.so"),
+                        mutant=mutant, force=True)
+    o = oracle.Oracle(path)
+    assert o.mutant_id == mutant
+    caught = []
+    for pin in PINS:
+        try:
+            pin(o)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin rejects mutant {mutant} ({MUTANTS[mutant]})"

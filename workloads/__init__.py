@@ -1,0 +1,223 @@
+"""Seeded synthetic inputs for the SiTU-GLU workloads.
+
+This module holds no SiTU arithmetic: it draws the inputs (gate_up, routing
+weights, grad_out) that both the CUDA path and the fp64 oracle consume, so
+that the two are compared on bit-identical data.  It imports neither of them.
+
+Generation is deterministic and independent of threading: every tensor is cut
+into blocks of ``BLOCK_ROWS`` rows and each block draws from its own numpy
+``PCG64`` stream seeded by ``SeedSequence([seed, tensor_id, block])``.
+Normals are numpy's ``standard_normal``; values are rounded to the storage
+dtype with round-to-nearest-even (float64 -> float32 -> bf16).
+
+The five workloads restate the synthetic configurations the measurements are
+quoted on (tiny, dense FFN, routed MoE expert rows, fp32 beta sweep with no
+linear clamp, large).  No dataset is involved.
+"""
+from __future__ import annotations
+
+import os
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass
+
+import numpy as np
+
+BLOCK_ROWS = 64
+
+TENSOR_GATE_UP = 1
+TENSOR_ROUTING = 2
+TENSOR_GRAD_OUT = 3
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One synthetic workload.  Standard deviations are the N(0, s) scale."""
+
+    index: int
+    name: str
+    dtype: str            # "bf16" or "f32": gate_up, output, grad_out, d_gate_up
+    tokens: int           # rows T
+    inter: int            # intermediate size I (gate_up is [T, 2I])
+    g_std: float
+    u_std: float
+    outlier_p: float      # probability an entry is replaced by +-U(lo, hi)
+    outlier_lo: float
+    outlier_hi: float
+    rw_kind: str          # "uniform" U(0,1), "ones", or "topk_softmax"
+    go_std: float
+    betas: tuple          # gate betas to run (the sweep has several)
+    linear_beta: float | None
+    seed: int
+    experts: int = 0      # topk_softmax only: experts per token
+    topk: int = 0         # topk_softmax only: weights kept per token
+
+    @property
+    def elem_bytes(self) -> int:
+        return 2 if self.dtype == "bf16" else 4
+
+    def fwd_bytes(self) -> int:
+        """Algorithmic HBM bytes of one forward: read gate_up and w, write Y."""
+        return self.tokens * (2 * self.inter * self.elem_bytes + 4 + self.inter * self.elem_bytes)
+
+    def bwd_bytes(self) -> int:
+        """Algorithmic HBM bytes of one backward: read gate_up, grad_out and w,
+        write d_gate_up and d_w."""
+        s = self.elem_bytes
+        return self.tokens * (2 * self.inter * s + self.inter * s + 4 + 2 * self.inter * s + 4)
+
+    def describe(self) -> str:
+        return (f"{self.name}: gate_up {self.dtype} [{self.tokens}, {2 * self.inter}] "
+                f"(I={self.inter}), beta={list(self.betas)}, linear_beta={self.linear_beta}")
+
+
+WORKLOADS = (
+    Workload(0, "tiny", "bf16", 256, 512, 1.0, 1.0, 0.0, 0.0, 0.0, "uniform", 1.0,
+             (4.0,), 25.0, seed=0),
+    Workload(1, "dense_ffn", "bf16", 4096, 3072, 2.0, 1.0, 0.0, 0.0, 0.0, "ones", 0.1,
+             (4.0,), 25.0, seed=1),
+    Workload(2, "routed_moe", "bf16", 32768, 2048, 3.0, 3.0, 0.01, 20.0, 60.0, "topk_softmax", 1.0,
+             (4.0,), 25.0, seed=2, experts=384, topk=8),
+    Workload(3, "beta_sweep_f32", "f32", 16384, 4096, 1.5, 1.5, 0.0, 0.0, 0.0, "uniform", 1.0,
+             (1.0, 4.0, 16.0), None, seed=3),
+    Workload(4, "large", "bf16", 131072, 4096, 2.0, 2.0, 0.0, 0.0, 0.0, "uniform", 0.05,
+             (4.0,), 25.0, seed=4),
+)
+
+
+def workload(index: int) -> Workload:
+    return WORKLOADS[index]
+
+
+# ---- rounding to the storage dtype ------------------------------------------
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bf16 (nearest, ties to even); returns the bf16
+    bit patterns as uint16.  Inputs here are finite."""
+    bits = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    rounding = np.uint32(0x7FFF) + ((bits >> np.uint32(16)) & np.uint32(1))
+    return ((bits + rounding) >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to float32."""
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def _store(values: np.ndarray, dtype: str) -> np.ndarray:
+    f32 = values.astype(np.float32)
+    return f32_to_bf16_bits(f32) if dtype == "bf16" else f32
+
+
+# ---- per-block streams ---------------------------------------------------------
+
+def _rng(seed: int, tensor_id: int, block: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, tensor_id, block])))
+
+
+def _threads() -> int:
+    return max(1, min(16, os.cpu_count() or 1))
+
+
+def _fill_blocks(rows: int, fill_block, n_threads: int | None = None) -> None:
+    blocks = (rows + BLOCK_ROWS - 1) // BLOCK_ROWS
+    n_threads = n_threads or _threads()
+    if blocks <= 2 or n_threads == 1:
+        for b in range(blocks):
+            fill_block(b)
+        return
+    with ThreadPoolExecutor(max_workers=n_threads) as pool:
+        list(pool.map(fill_block, range(blocks)))
+
+
+def _gate_up_block(wl: Workload, tokens: int, inter: int, b: int) -> np.ndarray:
+    # Always a whole block of draws, so that a row's values do not depend on T.
+    r0 = b * BLOCK_ROWS
+    n = BLOCK_ROWS
+    rng = _rng(wl.seed, TENSOR_GATE_UP, b)
+    v = rng.standard_normal((n, 2 * inter))
+    v[:, :inter] *= wl.g_std
+    v[:, inter:] *= wl.u_std
+    if wl.outlier_p > 0.0:
+        hit = rng.random((n, 2 * inter)) < wl.outlier_p
+        sign = np.where(rng.random((n, 2 * inter)) < 0.5, -1.0, 1.0)
+        mag = rng.uniform(wl.outlier_lo, wl.outlier_hi, size=(n, 2 * inter))
+        v = np.where(hit, sign * mag, v)
+    return v[:min(BLOCK_ROWS, tokens - r0)]
+
+
+def gate_up(wl: Workload, tokens: int | None = None, inter: int | None = None) -> np.ndarray:
+    """gate_up [T, 2I]: gate half ~ N(0, g_std), up half ~ N(0, u_std), with the
+    workload's outliers; bf16 bit patterns (uint16) or float32."""
+    tokens = wl.tokens if tokens is None else tokens
+    inter = wl.inter if inter is None else inter
+    out = np.empty((tokens, 2 * inter), dtype=np.uint16 if wl.dtype == "bf16" else np.float32)
+
+    def fill(b):
+        r0 = b * BLOCK_ROWS
+        blk = _gate_up_block(wl, tokens, inter, b)
+        out[r0:r0 + blk.shape[0]] = _store(blk, wl.dtype)
+
+    _fill_blocks(tokens, fill)
+    return out
+
+
+def grad_out(wl: Workload, tokens: int | None = None, inter: int | None = None) -> np.ndarray:
+    """grad_out [T, I] ~ N(0, go_std) in the workload's dtype."""
+    tokens = wl.tokens if tokens is None else tokens
+    inter = wl.inter if inter is None else inter
+    out = np.empty((tokens, inter), dtype=np.uint16 if wl.dtype == "bf16" else np.float32)
+
+    def fill(b):
+        r0 = b * BLOCK_ROWS
+        n = min(BLOCK_ROWS, tokens - r0)
+        v = _rng(wl.seed, TENSOR_GRAD_OUT, b).standard_normal((BLOCK_ROWS, inter))[:n] * wl.go_std
+        out[r0:r0 + n] = _store(v, wl.dtype)
+
+    _fill_blocks(tokens, fill)
+    return out
+
+
+def routing_weights(wl: Workload, tokens: int | None = None) -> np.ndarray:
+    """Row-aligned routing weights [T] float32.
+
+    "uniform": U(0, 1).  "ones": 1.0.  "topk_softmax": rows are token-major
+    expert assignments (row = token * topk + k); per token, ``experts``
+    N(0, 1) logits, softmax over all experts, then the ``topk`` largest
+    probabilities in descending order (ties to the lower expert index), not
+    renormalised."""
+    tokens = wl.tokens if tokens is None else tokens
+    if wl.rw_kind == "ones":
+        return np.ones(tokens, dtype=np.float32)
+    if wl.rw_kind == "uniform":
+        out = np.empty(tokens, dtype=np.float32)
+
+        def fill(b):
+            r0 = b * BLOCK_ROWS
+            n = min(BLOCK_ROWS, tokens - r0)
+            out[r0:r0 + n] = _rng(wl.seed, TENSOR_ROUTING, b).random(BLOCK_ROWS)[:n].astype(np.float32)
+
+        _fill_blocks(tokens, fill, n_threads=1)
+        return out
+    if wl.rw_kind == "topk_softmax":
+        k, e = wl.topk, wl.experts
+        n_tok = (tokens + k - 1) // k
+        probs = np.empty((n_tok, k), dtype=np.float64)
+        for b in range((n_tok + BLOCK_ROWS - 1) // BLOCK_ROWS):
+            t0 = b * BLOCK_ROWS
+            n = min(BLOCK_ROWS, n_tok - t0)
+            logits = _rng(wl.seed, TENSOR_ROUTING, b).standard_normal((BLOCK_ROWS, e))[:n]
+            z = np.exp(logits - logits.max(axis=1, keepdims=True))
+            p = z / z.sum(axis=1, keepdims=True)
+            order = np.argsort(-p, axis=1, kind="stable")[:, :k]
+            probs[t0:t0 + n] = np.take_along_axis(p, order, axis=1)
+        return probs.reshape(-1)[:tokens].astype(np.float32)
+    raise ValueError(f"unknown routing-weight kind {wl.rw_kind!r}")
+
+
+def inputs(wl: Workload, tokens: int | None = None, inter: int | None = None) -> dict:
+    """All three inputs of a workload: gate_up, routing_weights [T], grad_out."""
+    return {
+        "gate_up": gate_up(wl, tokens, inter),
+        "routing_weights": routing_weights(wl, tokens),
+        "grad_out": grad_out(wl, tokens, inter),
+    }
