@@ -1,0 +1,131 @@
+"""ctypes declarations of libsitu_glu.so, one Python callable per C entry point.
+
+Every function here has the name, argument order and meaning of its
+declaration in include/situ_glu.h (pointers are passed as integers).  Nothing
+is computed in Python.  The library is loaded on first use; if it has not been
+built the call raises ``NativeLibraryError`` -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+from . import _build
+
+SITU_OK = 0
+SITU_ERR_INVALID_ARG = 1
+SITU_ERR_UNSUPPORTED = 2
+SITU_ERR_MISALIGNED = 3
+SITU_ERR_CUDA = 4
+
+SITU_DTYPE_BF16 = 0
+SITU_DTYPE_F32 = 1
+
+SITU_RW_ROW = 0
+SITU_RW_SCALAR = 1
+SITU_RW_NONE = 2
+
+ABI_VERSION = 1
+
+# Entry points declared in include/situ_glu.h: name -> (restype, argtypes).
+_I64, _INT, _DBL, _VP, _SZ = ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_void_p, ctypes.c_size_t
+SIGNATURES = {
+    "situ_glu_fwd": (_INT, [_VP, _INT, _I64, _I64, _I64, _VP, _INT, _INT, _I64, _DBL, _INT, _DBL,
+                            _VP, _I64, _VP]),
+    "situ_glu_bwd": (_INT, [_VP, _INT, _I64, _I64, _I64, _VP, _INT, _INT, _I64, _DBL, _INT, _DBL,
+                            _VP, _I64, _VP, _I64, _VP, _I64, _VP, _SZ, _VP]),
+    "situ_glu_bwd_workspace_bytes": (_SZ, [_I64, _INT, _INT]),
+    "situ_glu_status_string": (ctypes.c_char_p, [_INT]),
+    "situ_glu_last_error": (ctypes.c_char_p, []),
+    "situ_glu_abi_version": (_INT, []),
+    "situ_glu_set_max_ctas": (_INT, [_INT]),
+}
+
+
+class NativeLibraryError(RuntimeError):
+    """The native library is missing, stale or does not match this binding."""
+
+
+class SituError(RuntimeError):
+    """A non-OK status returned by the library."""
+
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}: {detail}")
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def library_path() -> str:
+    return os.environ.get("SITU_GLU_LIBRARY", _build.LIBRARY)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (loaded once, on first use)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            path = library_path()
+            if not os.path.exists(path):
+                raise NativeLibraryError(
+                    f"{path} is not built; run `python -m ffn_gated_activation_b200._build` "
+                    "(or __graft_entry__.build()) -- there is no fallback implementation")
+            handle = ctypes.CDLL(path)
+            for name, (restype, argtypes) in SIGNATURES.items():
+                fn = getattr(handle, name)
+                fn.restype = restype
+                fn.argtypes = argtypes
+            if handle.situ_glu_abi_version() != ABI_VERSION:
+                raise NativeLibraryError(f"{path}: ABI {handle.situ_glu_abi_version()} != {ABI_VERSION}")
+            _lib = handle
+    return _lib
+
+
+def situ_glu_fwd(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride,
+                 beta, has_linear_beta, linear_beta, out, out_row_stride, stream) -> int:
+    return lib().situ_glu_fwd(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode,
+                              rw_stride, beta, has_linear_beta, linear_beta, out, out_row_stride, stream)
+
+
+def situ_glu_bwd(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride,
+                 beta, has_linear_beta, linear_beta, grad_out, grad_out_row_stride, d_gate_up,
+                 d_gate_up_row_stride, d_rw, d_rw_stride, workspace, workspace_bytes, stream) -> int:
+    return lib().situ_glu_bwd(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode,
+                              rw_stride, beta, has_linear_beta, linear_beta, grad_out,
+                              grad_out_row_stride, d_gate_up, d_gate_up_row_stride, d_rw, d_rw_stride,
+                              workspace, workspace_bytes, stream)
+
+
+def situ_glu_bwd_workspace_bytes(tokens, rw_mode, want_drw) -> int:
+    return lib().situ_glu_bwd_workspace_bytes(tokens, rw_mode, want_drw)
+
+
+def situ_glu_status_string(status) -> str:
+    return lib().situ_glu_status_string(status).decode()
+
+
+def situ_glu_last_error() -> str:
+    return lib().situ_glu_last_error().decode()
+
+
+def situ_glu_abi_version() -> int:
+    return lib().situ_glu_abi_version()
+
+
+def situ_glu_set_max_ctas(max_ctas) -> int:
+    return lib().situ_glu_set_max_ctas(max_ctas)
+
+
+def status_string(status: int) -> str:
+    return situ_glu_status_string(status)
+
+
+def check(status: int, where: str) -> None:
+    """Raise SituError for a non-OK status, with the library's own detail."""
+    if status != SITU_OK:
+        raise SituError(status, where, situ_glu_last_error())

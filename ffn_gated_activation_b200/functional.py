@@ -1,0 +1,199 @@
+"""Tensor-level binding: marshals torch tensors into the C ABI of libsitu_glu.so.
+
+PyTorch supplies device memory and the current stream; every step of the
+computation runs in the library's kernels.  The autograd function follows the
+contract of NeMo AutoModel's kimi_k3.situ `_WeightedSiTUFunction`: the forward
+saves only the low-precision inputs (gate_up and routing_weights in their own
+dtypes), the backward recomputes the fp32 chain and returns
+(d_gate_up, d_routing_weights or None, None, None).
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import abi
+
+# Kimi-K3 defaults (Megatron-LM PR #6673, "Activation": beta1 = 4, beta2 = 25;
+# the Kimi-K3 config.json: activation_situ_beta 4.0, activation_situ_linear_beta 25.0).
+DEFAULT_BETA = 4.0
+DEFAULT_LINEAR_BETA = 25.0
+
+_DTYPES = {torch.bfloat16: abi.SITU_DTYPE_BF16, torch.float32: abi.SITU_DTYPE_F32}
+
+
+def _dtype_code(t: torch.Tensor, what: str) -> int:
+    try:
+        return _DTYPES[t.dtype]
+    except KeyError:
+        raise TypeError(f"{what} must be bfloat16 or float32, got {t.dtype}") from None
+
+
+def _check_beta(beta, linear_beta):
+    # Megatron-LM PR #6673 "Design": SiTU-GLU betas must be finite and positive.
+    if not (isinstance(beta, (int, float)) and math.isfinite(beta) and beta > 0):
+        raise ValueError(f"beta must be a finite positive number, got {beta!r}")
+    if linear_beta is not None and not (isinstance(linear_beta, (int, float))
+                                        and math.isfinite(linear_beta) and linear_beta > 0):
+        raise ValueError(f"linear_beta must be None or a finite positive number, got {linear_beta!r}")
+
+
+def _rows(gate_up: torch.Tensor):
+    """gate_up [..., 2I] -> (2-D view [T, 2I], leading shape, I)."""
+    if gate_up.device.type != "cuda":
+        raise ValueError("gate_up must be a CUDA tensor")
+    if gate_up.dim() < 1 or gate_up.shape[-1] % 2:
+        raise ValueError(f"gate_up's last dimension must be 2 * intermediate, got {tuple(gate_up.shape)}")
+    inter = gate_up.shape[-1] // 2
+    lead = tuple(gate_up.shape[:-1])
+    g2 = gate_up.reshape(-1, 2 * inter)
+    if g2.stride(1) != 1 or (g2.shape[0] > 1 and g2.stride(0) < 2 * inter):
+        g2 = g2.contiguous()
+    return g2, lead, inter
+
+
+def routing_mode(gate_up_lead: tuple, routing_weights):
+    """Classify routing_weights against gate_up's leading shape (NeMo
+    `_situ_rw_is_row_aligned`): returns (mode, flat view or None).
+
+    None -> unweighted; one element -> broadcast scalar; shape [..., 1] with
+    gate_up's leading dimensions -> row-aligned.  Other broadcastable shapes
+    are not implemented (NotImplementedError)."""
+    if routing_weights is None:
+        return abi.SITU_RW_NONE, None
+    rw = routing_weights
+    if rw.numel() == 1:
+        return abi.SITU_RW_SCALAR, rw.reshape(1)
+    if rw.dim() >= 1 and tuple(rw.shape[:-1]) == gate_up_lead and rw.shape[-1] == 1:
+        return abi.SITU_RW_ROW, rw.reshape(-1)
+    if tuple(rw.shape) == gate_up_lead:
+        return abi.SITU_RW_ROW, rw.reshape(-1)
+    raise NotImplementedError(
+        f"routing_weights of shape {tuple(rw.shape)} against gate_up rows {gate_up_lead}: only "
+        "row-aligned [..., 1], a single broadcast value, or None are implemented")
+
+
+def _stream_handle(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def situ_glu_fwd(gate_up: torch.Tensor, routing_weights, beta: float = DEFAULT_BETA,
+                 linear_beta: float | None = DEFAULT_LINEAR_BETA, out: torch.Tensor | None = None,
+                 stream=None) -> torch.Tensor:
+    """Y = T_g(G) * T_u(U) * w for gate_up [..., 2I]; returns [..., I] in gate_up's dtype."""
+    _check_beta(beta, linear_beta)
+    g2, lead, inter = _rows(gate_up)
+    dtype = _dtype_code(g2, "gate_up")
+    mode, rw = routing_mode(lead, routing_weights)
+    if rw is not None:
+        if rw.device != g2.device:
+            raise ValueError("routing_weights must be on gate_up's device")
+        rw_dtype = _dtype_code(rw, "routing_weights")
+    else:
+        rw_dtype = abi.SITU_DTYPE_F32
+    if out is None:
+        out = torch.empty(lead + (inter,), dtype=gate_up.dtype, device=gate_up.device)
+    o2 = out.view(-1, inter)
+    tokens = g2.shape[0]
+    st = abi.situ_glu_fwd(g2.data_ptr(), dtype, tokens, inter, g2.stride(0) if tokens > 1 else 2 * inter,
+                          rw.data_ptr() if rw is not None else None, rw_dtype, mode,
+                          rw.stride(0) if rw is not None else 1,
+                          float(beta), int(linear_beta is not None),
+                          float(linear_beta) if linear_beta is not None else 0.0,
+                          o2.data_ptr(), o2.stride(0) if tokens > 1 else inter, _stream_handle(stream))
+    abi.check(st, "situ_glu_fwd")
+    return out
+
+
+def situ_glu_bwd(gate_up: torch.Tensor, routing_weights, grad_out: torch.Tensor,
+                 beta: float = DEFAULT_BETA, linear_beta: float | None = DEFAULT_LINEAR_BETA,
+                 want_drw: bool = True, d_gate_up: torch.Tensor | None = None,
+                 d_rw: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                 stream=None):
+    """Analytic backward.  Returns (d_gate_up [..., 2I], d_routing_weights shaped
+    like routing_weights, or None when not wanted / unweighted)."""
+    _check_beta(beta, linear_beta)
+    g2, lead, inter = _rows(gate_up)
+    dtype = _dtype_code(g2, "gate_up")
+    if grad_out.dtype != gate_up.dtype:
+        raise TypeError("grad_out must have gate_up's dtype")
+    if tuple(grad_out.shape) != lead + (inter,):
+        raise ValueError(f"grad_out shape {tuple(grad_out.shape)} != {lead + (inter,)}")
+    go2 = grad_out.reshape(-1, inter)
+    if go2.stride(1) != 1 or (go2.shape[0] > 1 and go2.stride(0) < inter):
+        go2 = go2.contiguous()
+    mode, rw = routing_mode(lead, routing_weights)
+    rw_dtype = _dtype_code(rw, "routing_weights") if rw is not None else abi.SITU_DTYPE_F32
+    want = bool(want_drw) and rw is not None
+    if d_gate_up is None:
+        d_gate_up = torch.empty(lead + (2 * inter,), dtype=gate_up.dtype, device=gate_up.device)
+    dg2 = d_gate_up.view(-1, 2 * inter)
+    d_rw_flat = None
+    if want:
+        if d_rw is None:
+            d_rw = torch.empty(routing_weights.shape, dtype=routing_weights.dtype, device=gate_up.device)
+        d_rw_flat = d_rw.view(-1)
+    tokens = g2.shape[0]
+    ws_bytes = abi.situ_glu_bwd_workspace_bytes(tokens, mode, int(want))
+    if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=gate_up.device)
+    st = abi.situ_glu_bwd(g2.data_ptr(), dtype, tokens, inter, g2.stride(0) if tokens > 1 else 2 * inter,
+                          rw.data_ptr() if rw is not None else None, rw_dtype, mode,
+                          rw.stride(0) if rw is not None else 1,
+                          float(beta), int(linear_beta is not None),
+                          float(linear_beta) if linear_beta is not None else 0.0,
+                          go2.data_ptr(), go2.stride(0) if tokens > 1 else inter,
+                          dg2.data_ptr(), dg2.stride(0) if tokens > 1 else 2 * inter,
+                          d_rw_flat.data_ptr() if d_rw_flat is not None else None,
+                          d_rw_flat.stride(0) if d_rw_flat is not None else 1,
+                          workspace.data_ptr() if ws_bytes else None, ws_bytes,
+                          _stream_handle(stream))
+    abi.check(st, "situ_glu_bwd")
+    return d_gate_up, (d_rw if want else None)
+
+
+class WeightedSiTUFunction(torch.autograd.Function):
+    """Routing-weighted SiTU-GLU with the analytic fused backward.
+
+    Saves only gate_up and routing_weights (NeMo `_WeightedSiTUFunction`:
+    "saves only the low-precision inputs"); backward returns
+    (d_gate_up, d_routing_weights, None, None)."""
+
+    @staticmethod
+    def forward(ctx, gate_up, routing_weights, beta, linear_beta):
+        out = situ_glu_fwd(gate_up, routing_weights, beta, linear_beta)
+        if routing_weights is None:
+            ctx.save_for_backward(gate_up)
+        else:
+            ctx.save_for_backward(gate_up, routing_weights)
+        ctx.has_rw = routing_weights is not None
+        ctx.beta = beta
+        ctx.linear_beta = linear_beta
+        return out
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        saved = ctx.saved_tensors
+        gate_up = saved[0]
+        rw = saved[1] if ctx.has_rw else None
+        want_drw = ctx.has_rw and ctx.needs_input_grad[1]
+        d_gate_up, d_rw = situ_glu_bwd(gate_up, rw, grad_out, ctx.beta, ctx.linear_beta,
+                                       want_drw=want_drw)
+        return d_gate_up, d_rw, None, None
+
+
+def weighted_situ(gate_up: torch.Tensor, routing_weights, beta: float = DEFAULT_BETA,
+                  linear_beta: float | None = DEFAULT_LINEAR_BETA) -> torch.Tensor:
+    """Apply SiTU-GLU and routing weights to gate_up [..., 2 * intermediate]
+    (NeMo `_weighted_situ`): gate in the first half, up in the second.
+    routing_weights: [..., 1] row-aligned, one broadcast value, or None."""
+    return WeightedSiTUFunction.apply(gate_up, routing_weights, beta, linear_beta)
+
+
+def situlu(gate_up: torch.Tensor, beta: float = DEFAULT_BETA,
+           linear_beta: float | None = DEFAULT_LINEAR_BETA) -> torch.Tensor:
+    """Unweighted SiTU-GLU (Megatron-LM PR #6673 "Design": the `situlu`
+    pointwise reference / TE SiTUGLU op), on the same kernels."""
+    return WeightedSiTUFunction.apply(gate_up, None, beta, linear_beta)

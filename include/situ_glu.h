@@ -1,0 +1,176 @@
+/*
+ * situ_glu.h -- C ABI of the B200 (sm_100a) routing-weighted SiTU-GLU library
+ * (libsitu_glu.so).
+ *
+ * The operation (Megatron-LM PR #6673 "[Dev] Add SiTU-GLU through Transformer
+ * Engine", section "Activation"; NeMo AutoModel API
+ * nemo_automodel.components.models.kimi_k3.situ, `_situ_fwd_core`):
+ *
+ *     G = gate_up[:, 0:I]          (gate half, first)
+ *     U = gate_up[:, I:2I]         (up half, second)
+ *     T_g = beta * tanh(G / beta) * sigmoid(G)
+ *     T_u = linear_beta * tanh(U / linear_beta)      (T_u = U without a linear beta)
+ *     Y   = T_g * T_u * w          (w: routing weight of the row)
+ *
+ * and its analytic backward (NeMo `_situ_bwd_core`,
+ * `_WeightedSiTUFunction.backward`), which recomputes the fp32 chain from the
+ * saved low-precision inputs only:
+ *
+ *     dG  = go * w * T_u * T_g'
+ *     dU  = go * w * T_g * T_u'
+ *     d_w = sum over the I columns of go * T_g * T_u     (per row)
+ *
+ * Conventions shared by every entry point:
+ *   - All functions are extern "C", never throw, and are thread-safe.
+ *   - Matrices are row-major with an explicit row stride in ELEMENTS.  Leading
+ *     batch dimensions are flattened into `tokens` by the caller.
+ *   - All tensor pointers are DEVICE pointers on the CUDA device that is
+ *     current on the calling thread.  The caller owns every buffer; the
+ *     library allocates nothing and keeps no state except a cached SM count
+ *     per device and the launch cap set by situ_glu_set_max_ctas().
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream) and the call returns without synchronising.  Errors raised while
+ *     the kernels run surface at the caller's next synchronisation.
+ *   - Arguments are validated on the host before anything is launched; on any
+ *     non-OK status nothing was enqueued and no output was touched.
+ *     situ_glu_last_error() then describes the failure.
+ *   - Arithmetic is fp32 in registers; each output is rounded once,
+ *     round-to-nearest-even, to its storage dtype.
+ */
+#ifndef SITU_GLU_H_
+#define SITU_GLU_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SITU_GLU_ABI_VERSION 1
+
+typedef enum situ_status {
+  SITU_OK = 0,
+  SITU_ERR_INVALID_ARG = 1, /* NULL pointer, bad size, stride, beta, enum or aliasing */
+  SITU_ERR_UNSUPPORTED = 2, /* a valid request this build does not implement          */
+  SITU_ERR_MISALIGNED = 3,  /* a base address or row pitch is not 16-byte aligned     */
+  SITU_ERR_CUDA = 4         /* the CUDA runtime reported an error at launch           */
+} situ_status_t;
+
+/* Storage dtype of a tensor.  bf16 = IEEE binary32 truncated to its upper 16
+ * bits (the torch.bfloat16 layout). */
+typedef enum situ_dtype {
+  SITU_DTYPE_BF16 = 0,
+  SITU_DTYPE_F32 = 1
+} situ_dtype_t;
+
+/* How the routing weights line up with the rows (NeMo `_situ_rw_is_row_aligned`
+ * and `_WeightedSiTUFunction.forward`, parameter routing_weights: "row-aligned
+ * with shape [..., k] matching gate_up's leading dimensions (typically
+ * [tokens, 1]) or broadcastable against them"). */
+typedef enum situ_rw_mode {
+  SITU_RW_ROW = 0,    /* one weight per row: w[row * rw_stride], gradient per row   */
+  SITU_RW_SCALAR = 1, /* one weight for every row: w[0]                             */
+  SITU_RW_NONE = 2    /* unweighted SiTU-GLU (w = 1; Megatron-LM PR #6673 "Design":
+                         the TE SiTUGLU op / `situlu`).  rw and d_rw must be NULL. */
+} situ_rw_mode_t;
+
+/*
+ * Forward: out[r, i] = T_g(G[r, i]) * T_u(U[r, i]) * w[r].
+ * Defined by: Megatron-LM PR #6673, section "Activation" (T_g, T_u, Y);
+ * NeMo kimi_k3.situ `_situ_fwd_core` ("situ(g) * up(u0) * w") and
+ * `_WeightedSiTUFunction.forward` (gate first half, up second half;
+ * optional linear_beta).
+ *
+ *   gate_up            [tokens, >= 2*inter] in `dtype`, row pitch gate_up_row_stride
+ *                      elements.  Read only.
+ *   dtype              SITU_DTYPE_BF16 or SITU_DTYPE_F32 (also the dtype of out).
+ *   tokens             rows, >= 0.  0 returns SITU_OK and launches nothing.
+ *   inter              I, > 0.  inter * sizeof(dtype) must be a multiple of 16
+ *                      (bf16: I % 8 == 0, fp32: I % 4 == 0).
+ *   rw, rw_dtype       routing weights (bf16 or fp32), laid out per rw_mode;
+ *                      rw_stride (elements, >= 0; 0 repeats w[0] on every row,
+ *                      as an expanded tensor does) is used by SITU_RW_ROW only.
+ *   beta               gate beta, finite and > 0 (Megatron-LM PR #6673
+ *                      "Design": finite positive betas).  Kimi-K3 default 4.
+ *   has_linear_beta    0: T_u = U.  1: linear_beta is used, finite and > 0
+ *                      (Kimi-K3 default 25).
+ *   out                [tokens, >= inter] in `dtype`, row pitch out_row_stride
+ *                      elements.  Written; must not overlap any input.
+ *   stream             cudaStream_t.
+ * Alignment: gate_up and out 16-byte aligned, row pitches multiples of 16
+ * bytes; rw aligned to its element size.  Otherwise SITU_ERR_MISALIGNED.
+ */
+situ_status_t situ_glu_fwd(const void *gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
+                           int64_t gate_up_row_stride,
+                           const void *rw, situ_dtype_t rw_dtype, situ_rw_mode_t rw_mode,
+                           int64_t rw_stride,
+                           double beta, int has_linear_beta, double linear_beta,
+                           void *out, int64_t out_row_stride,
+                           void *stream);
+
+/*
+ * Backward: recomputes T_g, T_u and their derivatives in fp32 from gate_up and
+ * rw (the only saved inputs: NeMo `_WeightedSiTUFunction`, "saves only the
+ * low-precision inputs") and writes, in one pass over HBM,
+ *   d_gate_up[r, 0:I]  = go * w * T_u * T_g'
+ *   d_gate_up[r, I:2I] = go * w * T_g * T_u'
+ *   d_rw               = sum over columns of go * T_g * T_u: per row for
+ *                        SITU_RW_ROW; summed over every row as well for
+ *                        SITU_RW_SCALAR (autograd's sum to the weight's shape).
+ * Defined by: NeMo kimi_k3.situ `_situ_bwd_core` (d_g, d_u, red; want_drw)
+ * and `_WeightedSiTUFunction.backward` (returns d_gate_up, d_routing_weights).
+ *
+ *   grad_out           [tokens, >= inter] in `dtype`, row pitch grad_out_row_stride.
+ *   d_gate_up          [tokens, >= 2*inter] in `dtype`, row pitch
+ *                      d_gate_up_row_stride.  Written; must not overlap any input.
+ *   d_rw               NULL: the routing-weight gradient is not wanted and no
+ *                      reduction runs (`want_drw` = false).  Otherwise in
+ *                      rw_dtype: element r at d_rw[r * d_rw_stride] (row mode)
+ *                      or one element (scalar mode).  Must be NULL for
+ *                      SITU_RW_NONE.
+ *   workspace          scratch for SITU_RW_SCALAR with d_rw != NULL: at least
+ *                      situ_glu_bwd_workspace_bytes() bytes, 16-byte aligned,
+ *                      device memory owned by the caller, contents ignored on
+ *                      entry and undefined on exit.  May be NULL when that
+ *                      query returns 0.
+ * Other arguments as for situ_glu_fwd.  Per-row reductions run in a fixed
+ * order, so every output is bitwise reproducible for a given build and shape,
+ * whatever the launch size.
+ */
+situ_status_t situ_glu_bwd(const void *gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
+                           int64_t gate_up_row_stride,
+                           const void *rw, situ_dtype_t rw_dtype, situ_rw_mode_t rw_mode,
+                           int64_t rw_stride,
+                           double beta, int has_linear_beta, double linear_beta,
+                           const void *grad_out, int64_t grad_out_row_stride,
+                           void *d_gate_up, int64_t d_gate_up_row_stride,
+                           void *d_rw, int64_t d_rw_stride,
+                           void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+/* Bytes of workspace situ_glu_bwd needs: tokens * 4 rounded up to 256 for
+ * SITU_RW_SCALAR with want_drw != 0, otherwise 0.  Negative tokens give 0. */
+size_t situ_glu_bwd_workspace_bytes(int64_t tokens, situ_rw_mode_t rw_mode, int want_drw);
+
+/* Static, human-readable name of a status code. */
+const char *situ_glu_status_string(situ_status_t status);
+
+/* Description of the most recent non-OK status returned on the calling thread
+ * ("" if none).  The pointer stays valid until the thread's next call. */
+const char *situ_glu_last_error(void);
+
+/* SITU_GLU_ABI_VERSION of the built library. */
+int situ_glu_abi_version(void);
+
+/* Upper bound on the CTAs of each launch (0 = automatic: SM count times the
+ * CTAs per SM the occupancy calculator allows).  Results do not depend on it;
+ * it exists for tuning and to check that.  Process-wide; returns the previous
+ * value, or -1 (and changes nothing) for a negative argument. */
+int situ_glu_set_max_ctas(int max_ctas);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* SITU_GLU_H_ */

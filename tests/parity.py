@@ -1,0 +1,184 @@
+"""Shared helpers of the GPU parity tests: device upload/download of the seeded
+inputs, guarded output buffers, direct calls through the C ABI, and the
+tolerance rule.
+
+Tolerance rule (derived from the arithmetic; the oracle value ``ref`` is the
+unrounded fp64 result):
+  * bf16 outputs (Y, dG, dU): |y - ref| <= 2^-8 |ref| + 1e-6, or y is one of the
+    two bf16 values that bracket ref (a faithful rounding: an fp32 chain whose
+    error is far below a bf16 ulp can still round a value that sits next to a
+    rounding midpoint to the other neighbour).
+  * fp32 outputs (Y, dU): |y - ref| <= 1e-5 |ref| + 1e-30.
+  * dG, both dtypes: the bound above plus 2^-18 * C_G, where C_G is the
+    uncancelled magnitude |go w T_u| (|sech^2 sigmoid| + |beta tanh sigmoid
+    (1 - sigmoid)|).  The two terms of T_g' cancel at a beta-dependent
+    G* < 0 (G* = -1.21876 for beta = 4); there the fp32 rounding of each term,
+    not the result, sets the error.
+  * d_w: |d - ref| <= 1e-4 |ref| + 2^-18 * S, S = sum_i |go T_g T_u| (the
+    rounding of a long fp32 sum scales with the sum of magnitudes).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import workloads
+from ffn_gated_activation_b200 import abi
+
+BF16_REL = 2.0 ** -8
+BF16_ABS = 1e-6
+F32_REL = 1e-5
+F32_ABS = 1e-30
+CANCEL = 2.0 ** -18
+DW_REL = 1e-4
+
+SENTINEL = 0xA5
+GUARD_BYTES = 4096
+
+
+# ---- device transfer -----------------------------------------------------------
+
+def to_device(a: np.ndarray, device) -> torch.Tensor:
+    if a.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def to_host(t: torch.Tensor) -> np.ndarray:
+    """Exact copy back: bf16 as uint16 bit patterns, fp32 as float32."""
+    t = t.detach()
+    if t.dtype == torch.bfloat16:
+        return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    return t.contiguous().cpu().numpy()
+
+
+def as_f64(a: np.ndarray) -> np.ndarray:
+    return workloads.bf16_bits_to_f32(a).astype(np.float64) if a.dtype == np.uint16 else a.astype(np.float64)
+
+
+def dtype_code(t: torch.Tensor) -> int:
+    return abi.SITU_DTYPE_BF16 if t.dtype == torch.bfloat16 else abi.SITU_DTYPE_F32
+
+
+# ---- guarded buffers ---------------------------------------------------------------
+
+class Guarded:
+    """An output buffer [rows, pitch] with GUARD_BYTES of sentinel bytes on each
+    side; ``view`` is the [rows, width] window the kernel may write.  check()
+    asserts that no byte outside the window changed (guards and row gaps)."""
+
+    def __init__(self, rows: int, width: int, pitch: int, dtype, device):
+        self.es = torch.empty((), dtype=dtype).element_size()
+        g = GUARD_BYTES // self.es
+        self.g, self.rows, self.width, self.pitch = g, rows, width, pitch
+        self.buf = torch.empty(2 * g + max(rows * pitch, 1), dtype=dtype, device=device)
+        self.buf.view(torch.uint8).fill_(SENTINEL)
+        self.mat = self.buf[g:g + rows * pitch].view(rows, pitch) if rows else self.buf[g:g]
+        self.view = self.mat[:, :width] if rows else self.mat
+
+    def ptr(self) -> int:
+        return self.buf[self.g:].data_ptr()
+
+    def check(self):
+        b = self.buf.view(torch.uint8)
+        gb = self.g * self.es
+        assert torch.all(b[:gb] == SENTINEL), "write before the output buffer"
+        assert torch.all(b[gb + self.rows * self.pitch * self.es:] == SENTINEL), "write past the output buffer"
+        if self.rows and self.pitch > self.width:
+            gap = self.mat[:, self.width:].contiguous().view(torch.uint8)
+            assert torch.all(gap == SENTINEL), "write into the row padding"
+
+
+# ---- direct C-ABI calls ---------------------------------------------------------------
+
+def call_fwd(gu: torch.Tensor, inter: int, rw, rw_mode: int, beta: float, lb, out: Guarded,
+             rw_stride: int = 1, stream: int = 0) -> int:
+    tokens = gu.shape[0]
+    rw_ptr = rw.data_ptr() if rw is not None else None
+    rw_dt = dtype_code(rw) if rw is not None else abi.SITU_DTYPE_F32
+    return abi.situ_glu_fwd(gu.data_ptr(), dtype_code(gu), tokens, inter, gu.stride(0),
+                            rw_ptr, rw_dt, rw_mode, rw_stride, float(beta), int(lb is not None),
+                            float(lb or 0.0), out.ptr(), out.pitch, stream)
+
+
+def call_bwd(gu: torch.Tensor, inter: int, rw, rw_mode: int, beta: float, lb, go: torch.Tensor,
+             dgu: Guarded, d_rw=None, rw_stride: int = 1, d_rw_stride: int = 1, workspace=None,
+             stream: int = 0) -> int:
+    tokens = gu.shape[0]
+    rw_ptr = rw.data_ptr() if rw is not None else None
+    rw_dt = dtype_code(rw) if rw is not None else abi.SITU_DTYPE_F32
+    ws_bytes = abi.situ_glu_bwd_workspace_bytes(tokens, rw_mode, int(d_rw is not None))
+    ws_ptr = None
+    if ws_bytes:
+        if workspace is None:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=gu.device)
+        ws_ptr = workspace.data_ptr()
+    return abi.situ_glu_bwd(gu.data_ptr(), dtype_code(gu), tokens, inter, gu.stride(0),
+                            rw_ptr, rw_dt, rw_mode, rw_stride, float(beta), int(lb is not None),
+                            float(lb or 0.0), go.data_ptr(), go.stride(0),
+                            dgu.ptr(), dgu.pitch,
+                            d_rw.data_ptr() if d_rw is not None else None, d_rw_stride,
+                            ws_ptr, ws_bytes, stream)
+
+
+# ---- tolerance ------------------------------------------------------------------------
+
+def _bf16_key(bits: np.ndarray) -> np.ndarray:
+    b = bits.astype(np.int32)
+    return np.where(b & 0x8000, -(b & 0x7FFF), b & 0x7FFF)
+
+
+def _bf16_from_key(k: np.ndarray) -> np.ndarray:
+    return np.where(k >= 0, k, 0x8000 | (-k)).astype(np.uint16)
+
+
+def bf16_faithful(bits: np.ndarray, ref: np.ndarray) -> np.ndarray:
+    """True where the bf16 value ``bits`` is one of the two bf16 neighbours of ref."""
+    y = as_f64(bits)
+    k = _bf16_key(bits)
+    up, down = ref > y, ref < y
+    toward = as_f64(_bf16_from_key(np.where(up, k + 1, np.where(down, k - 1, k))))
+    return (y == ref) | (up & (toward >= ref)) | (down & (toward <= ref))
+
+
+def check_output(name: str, got: np.ndarray, ref: np.ndarray, cancel_scale: np.ndarray | None = None):
+    """Assert the tolerance rule elementwise; returns a small report dict."""
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    y = as_f64(got)
+    err = np.abs(y - ref)
+    extra = CANCEL * cancel_scale if cancel_scale is not None else 0.0
+    if got.dtype == np.uint16:
+        strict = err <= BF16_REL * np.abs(ref) + BF16_ABS
+        ok = strict | bf16_faithful(got, ref) | (err <= BF16_REL * np.abs(ref) + BF16_ABS + extra)
+    else:
+        strict = err <= F32_REL * np.abs(ref) + F32_ABS
+        ok = strict | (err <= F32_REL * np.abs(ref) + F32_ABS + extra)
+    # equal values (equal infinities included) and NaN against NaN agree
+    ok |= (y == ref) | (np.isnan(y) & np.isnan(ref))
+    bad = np.flatnonzero(~ok)
+    if bad.size:
+        i = bad[0]
+        cs = cancel_scale.reshape(-1)[i] if cancel_scale is not None else 0.0
+        raise AssertionError(f"{name}: {bad.size} of {ok.size} elements out of tolerance; first at flat "
+                             f"index {i}: got {y.reshape(-1)[i]!r}, oracle {ref.reshape(-1)[i]!r}, "
+                             f"cancel scale {cs!r}")
+    fin = np.isfinite(ref) & np.isfinite(y)
+    rel = err[fin] / np.maximum(np.abs(ref[fin]), 1e-300)
+    strict |= ~fin
+    return {"n": int(ok.size), "extra_clause": int((~strict).sum()), "max_rel": float(np.max(rel, initial=0.0))}
+
+
+def check_dw(name: str, got: np.ndarray, ref: np.ndarray, mag: np.ndarray):
+    y = as_f64(got).reshape(-1)
+    ref = np.asarray(ref, dtype=np.float64).reshape(-1)
+    mag = np.asarray(mag, dtype=np.float64).reshape(-1)
+    tol = DW_REL * np.abs(ref) + CANCEL * mag
+    if got.dtype == np.uint16:  # a bf16 weight gradient is also rounded once
+        tol = tol + BF16_REL * np.abs(ref)
+    bad = np.flatnonzero(~((np.abs(y - ref) <= tol) | (y == ref) | (np.isnan(y) & np.isnan(ref))))
+    if bad.size:
+        i = bad[0]
+        raise AssertionError(f"{name}: {bad.size} of {y.size} rows out of tolerance; first row {i}: "
+                             f"got {y[i]!r}, oracle {ref[i]!r}, sum |terms| {mag[i]!r}")
+    strict = np.abs(y - ref) <= DW_REL * np.abs(ref)
+    return {"n": int(y.size), "extra_clause": int((~strict).sum())}

@@ -1,0 +1,196 @@
+"""The C-ABI boundary on the CPU: the library loads, exports every entry point
+include/situ_glu.h declares, and rejects bad arguments on the host before
+any CUDA call (no GPU is touched by these tests)."""
+import json
+import os
+import re
+import subprocess
+
+import pytest
+
+from ffn_gated_activation_b200 import abi
+import ffn_gated_activation_b200 as pkg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+           if f.endswith(".h")]
+
+BF16, F32 = abi.SITU_DTYPE_BF16, abi.SITU_DTYPE_F32
+ROW, SCALAR, NONE = abi.SITU_RW_ROW, abi.SITU_RW_SCALAR, abi.SITU_RW_NONE
+OK, INVALID, UNSUP, MISAL = abi.SITU_OK, abi.SITU_ERR_INVALID_ARG, abi.SITU_ERR_UNSUPPORTED, abi.SITU_ERR_MISALIGNED
+
+# Fake, well-separated, 256-byte-aligned device addresses: validation never
+# dereferences them.
+GU, RW, OUT, GO, DGU, DRW, WS = (0x1000_0000 * k for k in range(1, 8))
+
+
+def declared_functions():
+    names = set()
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(situ_glu_\w+)\s*\(", text, flags=re.M))
+    return names
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    assert {"situ_glu_fwd", "situ_glu_bwd", "situ_glu_bwd_workspace_bytes", "situ_glu_status_string",
+            "situ_glu_last_error", "situ_glu_abi_version", "situ_glu_set_max_ctas"} <= names
+
+
+def test_library_exports_every_declared_symbol(native_lib_path):
+    out = subprocess.run(["nm", "-D", "--defined-only", native_lib_path], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = declared_functions() - exported
+    assert not missing, f"declared but not exported: {sorted(missing)}"
+    lib = abi.lib()
+    for name in declared_functions():
+        getattr(lib, name)  # resolvable through ctypes
+
+
+def test_binding_covers_the_header_exactly():
+    assert set(abi.SIGNATURES) == declared_functions()
+    for name in abi.SIGNATURES:
+        assert hasattr(abi, name), f"binding lacks a Python function named {name}"
+
+
+def test_version_and_status_strings(native_lib_path):
+    assert abi.situ_glu_abi_version() == abi.ABI_VERSION == 1
+    assert abi.situ_glu_status_string(OK) == "SITU_OK"
+    assert abi.situ_glu_status_string(MISAL) == "SITU_ERR_MISALIGNED"
+    assert abi.situ_glu_status_string(99) == "SITU_ERR_UNKNOWN"
+
+
+def test_workspace_query(native_lib_path):
+    assert abi.situ_glu_bwd_workspace_bytes(1000, ROW, 1) == 0
+    assert abi.situ_glu_bwd_workspace_bytes(1000, SCALAR, 0) == 0
+    assert abi.situ_glu_bwd_workspace_bytes(1000, SCALAR, 1) == 4096
+    assert abi.situ_glu_bwd_workspace_bytes(64, SCALAR, 1) == 256
+    assert abi.situ_glu_bwd_workspace_bytes(0, SCALAR, 1) == 0
+    assert abi.situ_glu_bwd_workspace_bytes(-5, SCALAR, 1) == 0
+
+
+def test_max_ctas_knob(native_lib_path):
+    prev = abi.situ_glu_set_max_ctas(7)
+    assert abi.situ_glu_set_max_ctas(prev) == 7
+    assert abi.situ_glu_set_max_ctas(-1) == -1
+
+
+def fwd(**kw):
+    a = dict(gate_up=GU, dtype=BF16, tokens=16, inter=64, gate_up_row_stride=128, rw=RW, rw_dtype=F32,
+             rw_mode=ROW, rw_stride=1, beta=4.0, has_linear_beta=1, linear_beta=25.0, out=OUT,
+             out_row_stride=64, stream=None)
+    a.update(kw)
+    return abi.situ_glu_fwd(**a)
+
+
+def bwd(**kw):
+    a = dict(gate_up=GU, dtype=BF16, tokens=16, inter=64, gate_up_row_stride=128, rw=RW, rw_dtype=F32,
+             rw_mode=ROW, rw_stride=1, beta=4.0, has_linear_beta=1, linear_beta=25.0, grad_out=GO,
+             grad_out_row_stride=64, d_gate_up=DGU, d_gate_up_row_stride=128, d_rw=DRW, d_rw_stride=1,
+             workspace=None, workspace_bytes=0, stream=None)
+    a.update(kw)
+    return abi.situ_glu_bwd(**a)
+
+
+FWD_CASES = [
+    ("bad dtype", dict(dtype=7), INVALID),
+    ("bad rw_mode", dict(rw_mode=9), INVALID),
+    ("bad rw_dtype", dict(rw_dtype=3), INVALID),
+    ("negative tokens", dict(tokens=-1), INVALID),
+    ("zero inter", dict(inter=0), INVALID),
+    ("huge inter", dict(inter=1 << 29, gate_up_row_stride=1 << 30, out_row_stride=1 << 29), UNSUP),
+    ("beta zero", dict(beta=0.0), INVALID),
+    ("beta negative", dict(beta=-4.0), INVALID),
+    ("beta inf", dict(beta=float("inf")), INVALID),
+    ("beta nan", dict(beta=float("nan")), INVALID),
+    ("has_linear_beta not 0/1", dict(has_linear_beta=2), INVALID),
+    ("linear beta zero", dict(linear_beta=0.0), INVALID),
+    ("linear beta nan", dict(linear_beta=float("nan")), INVALID),
+    ("gate_up stride short", dict(gate_up_row_stride=127), INVALID),
+    ("out stride short", dict(out_row_stride=63), INVALID),
+    ("rw NULL in row mode", dict(rw=None), INVALID),
+    ("rw given when unweighted", dict(rw_mode=NONE), INVALID),
+    ("negative rw stride", dict(rw_stride=-1), INVALID),
+    ("inter not a 16-byte multiple", dict(inter=12, gate_up_row_stride=24, out_row_stride=12), MISAL),
+    ("gate_up NULL", dict(gate_up=None), INVALID),
+    ("out NULL", dict(out=None), INVALID),
+    ("gate_up misaligned", dict(gate_up=GU + 8), MISAL),
+    ("out misaligned", dict(out=OUT + 2), MISAL),
+    ("gate_up pitch misaligned", dict(gate_up_row_stride=132), MISAL),
+    ("rw misaligned", dict(rw=RW + 2), MISAL),
+    ("out overlaps gate_up", dict(out=GU + 256), INVALID),
+    ("out overlaps rw", dict(out=RW - 16 * 64 * 2 + 16), INVALID),
+    ("extent overflow", dict(tokens=1 << 40, gate_up_row_stride=1 << 40), INVALID),
+]
+
+
+@pytest.mark.parametrize("name,kw,status", FWD_CASES, ids=[c[0] for c in FWD_CASES])
+def test_fwd_rejects(name, kw, status, native_lib_path):
+    assert fwd(**kw) == status
+    assert abi.situ_glu_last_error() != ""
+
+
+BWD_CASES = [
+    ("grad_out stride short", dict(grad_out_row_stride=63), INVALID),
+    ("d_gate_up stride short", dict(d_gate_up_row_stride=100), INVALID),
+    ("d_rw when unweighted", dict(rw=None, rw_mode=NONE), INVALID),
+    ("d_rw stride zero", dict(d_rw_stride=0), INVALID),
+    ("scalar without workspace", dict(rw_mode=SCALAR), INVALID),
+    ("scalar workspace short", dict(rw_mode=SCALAR, workspace=WS, workspace_bytes=32), INVALID),
+    ("scalar workspace misaligned", dict(rw_mode=SCALAR, workspace=WS + 4, workspace_bytes=256), MISAL),
+    ("grad_out NULL", dict(grad_out=None), INVALID),
+    ("d_gate_up NULL", dict(d_gate_up=None), INVALID),
+    ("grad_out misaligned", dict(grad_out=GO + 4), MISAL),
+    ("d_rw misaligned", dict(d_rw=DRW + 1), MISAL),
+    ("d_gate_up overlaps grad_out", dict(d_gate_up=GO), INVALID),
+    ("d_gate_up overlaps gate_up", dict(d_gate_up=GU + 2048), INVALID),
+    ("d_rw overlaps d_gate_up", dict(d_rw=DGU + 64), INVALID),
+    ("d_rw overlaps rw", dict(d_rw=RW), INVALID),
+    ("workspace overlaps grad_out", dict(rw_mode=SCALAR, workspace=GO, workspace_bytes=256), INVALID),
+    ("beta negative", dict(beta=-1.0), INVALID),
+]
+
+
+@pytest.mark.parametrize("name,kw,status", BWD_CASES, ids=[c[0] for c in BWD_CASES])
+def test_bwd_rejects(name, kw, status, native_lib_path):
+    assert bwd(**kw) == status
+    assert abi.situ_glu_last_error() != ""
+
+
+def test_zero_tokens_launch_nothing(native_lib_path):
+    assert fwd(tokens=0, gate_up=None, out=None, rw=None) == OK
+    assert bwd(tokens=0, gate_up=None, grad_out=None, d_gate_up=None, d_rw=None) == OK
+    assert abi.situ_glu_last_error() == ""
+
+
+def test_binding_routing_modes():
+    import torch
+    from ffn_gated_activation_b200.functional import routing_mode
+    lead = (4, 6)
+    assert routing_mode(lead, None)[0] == NONE
+    assert routing_mode(lead, torch.tensor(0.5))[0] == SCALAR
+    assert routing_mode(lead, torch.ones(1, 1, 1))[0] == SCALAR
+    m, flat = routing_mode(lead, torch.ones(4, 6, 1))
+    assert m == ROW and flat.shape == (24,)
+    assert routing_mode(lead, torch.ones(4, 6))[0] == ROW
+    with pytest.raises(NotImplementedError):
+        routing_mode(lead, torch.ones(4, 6, 8))
+
+
+def test_binding_validates_betas():
+    from ffn_gated_activation_b200.functional import _check_beta
+    _check_beta(4.0, 25.0)
+    _check_beta(4.0, None)
+    for bad in ((0.0, 25.0), (float("inf"), None), (4.0, -1.0), (4.0, float("nan"))):
+        with pytest.raises(ValueError):
+            _check_beta(*bad)
+
+
+def test_defaults_match_the_pages():
+    golden = json.load(open(os.path.join(ROOT, "tests", "golden", "situ_defaults.json")))
+    assert pkg.DEFAULT_BETA == golden["beta"]["value"]
+    assert pkg.DEFAULT_LINEAR_BETA == golden["linear_beta"]["value"]
+    assert golden["moe_intermediate_size"]["value"] == 3072
