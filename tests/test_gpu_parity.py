@@ -150,8 +150,9 @@ def test_special_values(cuda_device):
         gu_h, rw32, go_h = case_inputs(dtype, T, I, seed=77)
         vals = np.array(specials, dtype=np.float32)
         vals_st = workloads.f32_to_bf16_bits(vals) if dtype == "bf16" else vals
+        base = gu_h
         for beta, lb in ((4.0, 25.0), (16.0, None), (1.0, 2.0)):
-            gu_h = gu_h.copy()
+            gu_h = base.copy()
             for r in range(T):
                 gu_h[r, :len(specials)] = np.roll(vals_st, r)           # gate column specials
                 if lb is not None:  # without a clamp, U = 3e38 overflows fp32 but not the oracle
