@@ -38,6 +38,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "situ_glu.h"
 
@@ -47,8 +48,9 @@ namespace {
 // Device helpers
 // ---------------------------------------------------------------------------
 
-constexpr float kNegLog2e = -1.4426950408889634f;  // -log2(e)
-constexpr int kMaxThreads = 256;                   // CTA size ceiling
+constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kMaxThreads = 256;  // CTA size ceiling
 constexpr int kVecBytes = 16;
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -61,6 +63,22 @@ __device__ __forceinline__ float rcp_approx(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Hardware tanh (MUFU).  Its relative error (about 2^-11) is far below half a
+// bf16 ulp (2^-9 relative), so it is used only where the result is rounded to
+// bf16 and nothing is accumulated from it: the up branch of the bf16 forward.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// max() that propagates NaN (a NaN input must give a NaN output).
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
 }
 
 // Read-only streaming load (no L1 allocation) and evict-first store: every
@@ -79,64 +97,119 @@ __device__ __forceinline__ void st_stream(void* p, const uint4& v) {
                : "memory");
 }
 
-// Storage types.  A 16-byte vector holds 8 bf16 or 4 fp32 values.
+// Packed fp32 pairs: sm_100 executes one f32x2 add/mul/fma per issue slot.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 splat(float a) { return make_float2(a, a); }
+
+__device__ __forceinline__ float2 ex2_neg2(float2 y) {  // (2^-y.x, 2^-y.y)
+  return make_float2(ex2_approx(-y.x), ex2_approx(-y.y));
+}
+__device__ __forceinline__ float2 rcp2(float2 a) { return make_float2(rcp_approx(a.x), rcp_approx(a.y)); }
+
+// A pair of input elements as fp32 bit patterns (bf16 widened exactly).
+struct Bits2 {
+  uint32_t lo, hi;
+};
+
+__device__ __forceinline__ float2 as_f2(Bits2 b) { return make_float2(__uint_as_float(b.lo), __uint_as_float(b.hi)); }
+__device__ __forceinline__ float2 abs_f2(Bits2 b) {
+  return make_float2(__uint_as_float(b.lo & 0x7fffffffu), __uint_as_float(b.hi & 0x7fffffffu));
+}
+// x with its sign bit flipped where the sign bit of `s` is set.
+__device__ __forceinline__ float xor_sign(float x, uint32_t s) {
+  return __uint_as_float(__float_as_uint(x) ^ (s & 0x80000000u));
+}
+__device__ __forceinline__ float2 xor_sign2(float2 x, Bits2 s) { return make_float2(xor_sign(x.x, s.lo), xor_sign(x.y, s.hi)); }
+// s negative ? a : b, element-wise on the sign bit of s.
+__device__ __forceinline__ float2 select_neg2(Bits2 s, float2 a, float2 b) {
+  const uint32_t m0 = static_cast<uint32_t>(static_cast<int32_t>(s.lo) >> 31);
+  const uint32_t m1 = static_cast<uint32_t>(static_cast<int32_t>(s.hi) >> 31);
+  return make_float2(__uint_as_float((__float_as_uint(a.x) & m0) | (__float_as_uint(b.x) & ~m0)),
+                     __uint_as_float((__float_as_uint(a.y) & m1) | (__float_as_uint(b.y) & ~m1)));
+}
+
+// Storage types.  A 16-byte vector holds 8 bf16 or 4 fp32 values, i.e. 4 or 2
+// pairs.  Pair p of a vector is (element 2p, element 2p + 1).
 struct Bf16 {
-  static constexpr int kPerVec = 8;
-  __device__ __forceinline__ static void unpack(const uint4& v, float (&f)[8]) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      f[2 * k] = __uint_as_float(w[k] << 16);           // element 2k: low half
-      f[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);  // element 2k+1: high half
-    }
+  static constexpr int kPairs = 4;
+  __device__ __forceinline__ static Bits2 pair(const uint4& v, int p) {
+    const uint32_t w = p == 0 ? v.x : p == 1 ? v.y : p == 2 ? v.z : v.w;
+    return {w << 16, w & 0xffff0000u};
   }
-  __device__ __forceinline__ static uint4 pack(const float (&f)[8]) {
-    uint32_t w[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k)  // cvt packs its first source into the high half
-      asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[k]) : "f"(f[2 * k + 1]), "f"(f[2 * k]));
-    return make_uint4(w[0], w[1], w[2], w[3]);
+  __device__ __forceinline__ static uint32_t pack(float2 f) {
+    uint32_t r;  // cvt packs its first source into the high half
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(f.y), "f"(f.x));
+    return r;
+  }
+  __device__ __forceinline__ static void put(uint4& v, int p, float2 f) {
+    const uint32_t w = pack(f);
+    if (p == 0) v.x = w; else if (p == 1) v.y = w; else if (p == 2) v.z = w; else v.w = w;
   }
 };
 
 struct F32 {
-  static constexpr int kPerVec = 4;
-  __device__ __forceinline__ static void unpack(const uint4& v, float (&f)[4]) {
-    f[0] = __uint_as_float(v.x);
-    f[1] = __uint_as_float(v.y);
-    f[2] = __uint_as_float(v.z);
-    f[3] = __uint_as_float(v.w);
+  static constexpr int kPairs = 2;
+  __device__ __forceinline__ static Bits2 pair(const uint4& v, int p) {
+    return p == 0 ? Bits2{v.x, v.y} : Bits2{v.z, v.w};
   }
-  __device__ __forceinline__ static uint4 pack(const float (&f)[4]) {
-    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
-                      __float_as_uint(f[3]));
+  __device__ __forceinline__ static void put(uint4& v, int p, float2 f) {
+    if (p == 0) {
+      v.x = __float_as_uint(f.x);
+      v.y = __float_as_uint(f.y);
+    } else {
+      v.z = __float_as_uint(f.x);
+      v.w = __float_as_uint(f.y);
+    }
   }
 };
 
-// 1 - exp(-x) for x >= 0, given E = ex2 approximation of exp(-x).  Where x is
-// small, 1 - E cancels; there the Taylor series x - x^2/2 + x^3/6 - ... is
-// used.  bf16 outputs: series to x^4 below x = 1/16 (truncation < 2^-22
-// relative; 1 - E above it is within ~2^-19).  fp32 outputs: series to x^6
-// below x = 1/4 (truncation < 2^-24; 1 - E above it within ~2^-21).
+// 1 - 2^-y, given E = 2^-y from the MUFU.  Where |y| is small, 1 - E cancels;
+// there the Taylor series of 1 - exp(-x) in x = y ln 2 is used, written in y:
+//   sum_k (-1)^(k+1) (ln 2)^k y^k / k!.
+// bf16 outputs: terms to y^4 for |x| < 1/16 (truncation below 2^-22 relative;
+// 1 - E above it within about 2^-19).  fp32 outputs: terms to y^6 for
+// |x| < 1/4 (truncation below 2^-24; 1 - E above it within about 2^-21).
+// Valid for either sign of y.
 template <typename S>
-__device__ __forceinline__ float one_minus_exp_neg(float x, float E);
+struct Series;
 
 template <>
-__device__ __forceinline__ float one_minus_exp_neg<Bf16>(float x, float E) {
-  float p = fmaf(x, -1.0f / 24.0f, 1.0f / 6.0f);
-  p = fmaf(p, x, -0.5f);
-  p = fmaf(p, x, 1.0f);
-  return x < 0.0625f ? p * x : 1.0f - E;
-}
+struct Series<Bf16> {
+  static constexpr float kYmax = 0.0625f / kLn2;
+  __device__ __forceinline__ static float2 eval(float2 y) {
+    const float c1 = kLn2, c2 = -kLn2 * kLn2 / 2.0f, c3 = kLn2 * kLn2 * kLn2 / 6.0f,
+                c4 = -kLn2 * kLn2 * kLn2 * kLn2 / 24.0f;
+    float2 p = fma2(y, splat(c4), splat(c3));
+    p = fma2(p, y, splat(c2));
+    p = fma2(p, y, splat(c1));
+    return mul2(p, y);
+  }
+};
 
 template <>
-__device__ __forceinline__ float one_minus_exp_neg<F32>(float x, float E) {
-  float p = fmaf(x, -1.0f / 720.0f, 1.0f / 120.0f);
-  p = fmaf(p, x, -1.0f / 24.0f);
-  p = fmaf(p, x, 1.0f / 6.0f);
-  p = fmaf(p, x, -0.5f);
-  p = fmaf(p, x, 1.0f);
-  return x < 0.25f ? p * x : 1.0f - E;
+struct Series<F32> {
+  static constexpr float kYmax = 0.25f / kLn2;
+  __device__ __forceinline__ static float2 eval(float2 y) {
+    const float l = kLn2;
+    const float c1 = l, c2 = -l * l / 2.0f, c3 = l * l * l / 6.0f, c4 = -l * l * l * l / 24.0f,
+                c5 = l * l * l * l * l / 120.0f, c6 = -l * l * l * l * l * l / 720.0f;
+    float2 p = fma2(y, splat(c6), splat(c5));
+    p = fma2(p, y, splat(c4));
+    p = fma2(p, y, splat(c3));
+    p = fma2(p, y, splat(c2));
+    p = fma2(p, y, splat(c1));
+    return mul2(p, y);
+  }
+};
+
+template <typename S>
+__device__ __forceinline__ float2 one_minus_exp2_neg(float2 y, float2 E) {
+  const float2 series = Series<S>::eval(y);
+  const float2 direct = add2(splat(1.0f), make_float2(-E.x, -E.y));
+  return make_float2(fabsf(y.x) < Series<S>::kYmax ? series.x : direct.x,
+                     fabsf(y.y) < Series<S>::kYmax ? series.y : direct.y);
 }
 
 // How the two gate exponentials relate for the given beta.
@@ -148,90 +221,147 @@ enum GateMode : int {
 };
 
 struct Coeffs {
-  float beta;      // gate beta
-  float lb;        // linear beta (unused without one)
-  float neg_kt;    // -2 log2(e) / beta: E_t = 2^(|g| neg_kt)
-  float xt_scale;  // 2 / beta: series argument x_t = 2|g| / beta
-  float neg_ku;    // -2 log2(e) / beta_L
-  float xu_scale;  // 2 / beta_L
-  float bb;        // beta * beta_L (beta without a linear beta)
+  float beta;    // gate beta
+  float lb;      // linear beta (1 without one)
+  float inv_lb;  // 1 / linear beta
+  float kt;      // 2 log2(e) / beta:    E_t = 2^-(|g| kt)
+  float ku;      // 2 log2(e) / beta_L:  E_u = 2^-(|u| ku)
+  float bb;      // beta * beta_L (beta without a linear beta)
 };
 
-struct GateExp {
-  float Et;   // exp(-2|g|/beta)
-  float Es;   // exp(-|g|)
-  float emt;  // 1 - Et, accurate
+// Exponentials of the gate: E_t = 2^-y with y = |g| kt (or g kt, signed form)
+// and E_s = exp(-|g|) (exp(-g)).  `y` must already hold the scaled argument.
+template <int GATE>
+__device__ __forceinline__ void gate_exps(float2 y, float2& Et, float2& Es) {
+  if (GATE == kGateSquare) {
+    Et = ex2_neg2(y);
+    Es = mul2(Et, Et);
+  } else if (GATE == kGateEqual) {
+    Et = ex2_neg2(y);
+    Es = Et;
+  } else if (GATE == kGateRoot) {  // kt = 2 log2(e): E_s = 2^-(y/2), E_t = E_s^2
+    Es = ex2_neg2(mul2(y, splat(0.5f)));
+    Et = mul2(Es, Es);
+  } else {
+    Et = ex2_neg2(y);
+    Es = make_float2(0.0f, 0.0f);  // set by the caller from its own argument
+  }
+}
+
+// ---- forward, bf16 storage ------------------------------------------------
+// Signed form: with H = exp(-2g/beta) and Hs = exp(-g) (g of either sign),
+//   tanh(g/beta) = (1 - H) / (1 + H),  sigmoid(g) = 1 / (1 + Hs),
+//   T_g = beta (1 - H) / ((1 + H)(1 + Hs)),
+// so neither a sign select nor |g| is needed.  The exponent argument is
+// clamped at 2^126 (a NaN passes through); when (1 + H)(1 + Hs) overflows the
+// reciprocal is 0 and T_g flushes to 0, which happens only where
+// |T_g| < 4 exp(-59) -- below the bf16 output's absolute resolution of the
+// tolerance.  The up branch uses the MUFU tanh (see tanh_approx).
+template <int GATE, bool HAS_LB>
+__device__ __forceinline__ float2 fwd_pair_bf16(Bits2 gb, Bits2 ub, float2 wbb, const Coeffs& c) {
+  const float2 g = as_f2(gb);
+  float2 y = mul2(g, splat(c.kt));
+  y = make_float2(max_nan(y.x, -126.0f), max_nan(y.y, -126.0f));
+  float2 H, Hs;
+  gate_exps<GATE>(y, H, Hs);
+  if (GATE == kGateGeneric) {
+    float2 ys = mul2(g, splat(kLog2e));
+    Hs = ex2_neg2(make_float2(max_nan(ys.x, -126.0f), max_nan(ys.y, -126.0f)));
+  }
+  const float2 em = one_minus_exp2_neg<Bf16>(y, H);
+  const float2 den = mul2(add2(splat(1.0f), H), add2(splat(1.0f), Hs));
+  float2 t;  // T_u / beta_L (or U)
+  if (HAS_LB) {
+    const float2 a = mul2(as_f2(ub), splat(c.inv_lb));
+    t = make_float2(tanh_approx(a.x), tanh_approx(a.y));
+  } else {
+    t = as_f2(ub);
+  }
+  return mul2(mul2(em, t), mul2(rcp2(den), wbb));
+}
+
+// ---- |g| form (fp32 forward and every backward) ---------------------------
+// E_t = exp(-2|g|/beta) <= 1 and E_s = exp(-|g|) <= 1, so no intermediate can
+// overflow; the sign of g enters through selects and sign flips.
+struct GateAbs {
+  float2 Et, Es, emt;  // emt = 1 - Et, accurate
 };
 
 template <int GATE, typename S>
-__device__ __forceinline__ GateExp gate_exp(float g, const Coeffs& c) {
-  const float ag = fabsf(g);
-  GateExp r;
-  if (GATE == kGateSquare) {
-    r.Et = ex2_approx(ag * c.neg_kt);
-    r.Es = r.Et * r.Et;
-  } else if (GATE == kGateEqual) {
-    r.Et = ex2_approx(ag * c.neg_kt);
-    r.Es = r.Et;
-  } else if (GATE == kGateRoot) {
-    r.Es = ex2_approx(ag * kNegLog2e);
-    r.Et = r.Es * r.Es;
-  } else {
-    r.Et = ex2_approx(ag * c.neg_kt);
-    r.Es = ex2_approx(ag * kNegLog2e);
-  }
-  r.emt = one_minus_exp_neg<S>(ag * c.xt_scale, r.Et);
+__device__ __forceinline__ GateAbs gate_abs(Bits2 gb, const Coeffs& c) {
+  const float2 ag = abs_f2(gb);
+  const float2 y = mul2(ag, splat(c.kt));
+  GateAbs r;
+  gate_exps<GATE>(y, r.Et, r.Es);
+  if (GATE == kGateGeneric) r.Es = ex2_neg2(mul2(ag, splat(kLog2e)));
+  r.emt = one_minus_exp2_neg<S>(y, r.Et);
   return r;
 }
 
-// Forward of one element.  wbb = w * beta * beta_L (w * beta without one).
-template <int GATE, bool HAS_LB, typename S>
-__device__ __forceinline__ float situ_fwd_elem(float g, float u, float wbb, const Coeffs& c) {
-  const GateExp e = gate_exp<GATE, S>(g, c);
-  const float sig = g < 0.0f ? e.Es : 1.0f;    // sigmoid(g) * (1 + E_s)
-  float num = copysignf(e.emt, g) * sig;        // T_g * (1 + E_t)(1 + E_s) / beta
-  float den = (1.0f + e.Et) * (1.0f + e.Es);
-  if (HAS_LB) {
-    const float au = fabsf(u);
-    const float Eu = ex2_approx(au * c.neg_ku);
-    const float emu = one_minus_exp_neg<S>(au * c.xu_scale, Eu);
-    num *= copysignf(emu, u);                   // T_u * (1 + E_u) / beta_L
-    den *= 1.0f + Eu;
-  } else {
-    num *= u;
-  }
-  return num * wbb * rcp_approx(den);
+template <typename S>
+__device__ __forceinline__ float2 up_emu(Bits2 ub, const Coeffs& c, float2& Eu) {
+  const float2 y = mul2(abs_f2(ub), splat(c.ku));
+  Eu = ex2_neg2(y);
+  return one_minus_exp2_neg<S>(y, Eu);
 }
 
-// Backward of one element: writes dG, dU and returns go * T_g * T_u.
+// fp32 forward of a pair.  Y = w beta beta_L s_g s_u (1 - E_t) sig (1 - E_u)
+// / ((1 + E_t)(1 + E_s)(1 + E_u)), sig = 1 (g >= 0) or E_s (g < 0).
 template <int GATE, bool HAS_LB, typename S>
-__device__ __forceinline__ float situ_bwd_elem(float g, float u, float go, float gow, const Coeffs& c,
-                                               float& dg, float& du) {
-  const GateExp e = gate_exp<GATE, S>(g, c);
-  const float sig = g < 0.0f ? e.Es : 1.0f;
-  const float tb = c.beta * copysignf(e.emt, g);  // beta tanh(g/beta) (1 + E_t)
-  const float tg = tb * sig;                        // T_g * A
-  const float opt = 1.0f + e.Et, ops = 1.0f + e.Es;
-  const float A = opt * ops;
-  // T_g' A^2 = [sech^2(g/beta) sigmoid(g)] A^2 + [beta tanh(g/beta) sigmoid(1 - sigmoid)] A^2
-  //          = 4 E_t sig (1 + E_s)            + tb (1 + E_t) E_s
-  const float ng = 4.0f * e.Et * sig * ops + tb * opt * e.Es;
+__device__ __forceinline__ float2 fwd_pair_abs(Bits2 gb, Bits2 ub, float2 wbb, const Coeffs& c) {
+  const GateAbs e = gate_abs<GATE, S>(gb, c);
+  const float2 sig = select_neg2(gb, e.Es, splat(1.0f));
+  float2 num = mul2(e.emt, sig);
+  float2 den = mul2(add2(splat(1.0f), e.Et), add2(splat(1.0f), e.Es));
   if (HAS_LB) {
-    const float au = fabsf(u);
-    const float Eu = ex2_approx(au * c.neg_ku);
-    const float tu = c.lb * copysignf(one_minus_exp_neg<S>(au * c.xu_scale, Eu), u);  // T_u * B
-    const float B = 1.0f + Eu;
-    const float AB = A * B;
-    const float R = rcp_approx(AB * AB);  // 1 / (A^2 B^2)
-    dg = gow * tu * ng * (B * R);          // go w T_u T_g'
-    du = gow * tg * (4.0f * Eu) * (A * R);  // go w T_g sech^2(u / beta_L)
-    return go * tg * tu * (AB * R);        // go T_g T_u
+    float2 Eu;
+    const float2 emu = up_emu<S>(ub, c, Eu);
+    num = mul2(num, emu);
+    den = mul2(den, add2(splat(1.0f), Eu));
+    // sign of the product: s_g s_u
+    const Bits2 s = {gb.lo ^ ub.lo, gb.hi ^ ub.hi};
+    return xor_sign2(mul2(num, mul2(rcp2(den), wbb)), s);
+  }
+  num = mul2(num, abs_f2(ub));
+  const Bits2 s = {gb.lo ^ ub.lo, gb.hi ^ ub.hi};
+  return xor_sign2(mul2(num, mul2(rcp2(den), wbb)), s);
+}
+
+// Backward of a pair.  With A = (1 + E_t)(1 + E_s), B = 1 + E_u (1 without a
+// linear beta), tb = beta tanh(g/beta) (1 + E_t) and sig as above:
+//   T_g  = tb sig / A
+//   T_g' = [4 E_t sig (1 + E_s) + tb (1 + E_t) E_s] / A^2
+//          (sech^2(g/beta) sigmoid + beta tanh sigmoid (1 - sigmoid), each over A^2)
+//   T_u  = tu / B,  T_u' = 4 E_u / B^2,  tu = beta_L s_u (1 - E_u)
+// and one reciprocal R = 1 / (A B)^2 serves every quotient.  Returns dG, dU;
+// adds go T_g T_u to acc.
+template <int GATE, bool HAS_LB, typename S>
+__device__ __forceinline__ void bwd_pair(Bits2 gb, Bits2 ub, float2 go, float2 gow, const Coeffs& c, float2& dg,
+                                         float2& du, float2& acc) {
+  const GateAbs e = gate_abs<GATE, S>(gb, c);
+  const float2 sig = select_neg2(gb, e.Es, splat(1.0f));
+  const float2 opt = add2(splat(1.0f), e.Et), ops = add2(splat(1.0f), e.Es);
+  const float2 A = mul2(opt, ops);
+  const float2 tb = mul2(xor_sign2(e.emt, gb), splat(c.beta));
+  const float2 tg = mul2(tb, sig);
+  const float2 ng = fma2(mul2(mul2(e.Et, sig), ops), splat(4.0f), mul2(mul2(tb, opt), e.Es));
+  if (HAS_LB) {
+    float2 Eu;
+    const float2 emu = up_emu<S>(ub, c, Eu);
+    const float2 tu = mul2(xor_sign2(emu, ub), splat(c.lb));
+    const float2 B = add2(splat(1.0f), Eu);
+    const float2 AB = mul2(A, B);
+    const float2 R = rcp2(mul2(AB, AB));
+    dg = mul2(mul2(gow, tu), mul2(ng, mul2(B, R)));
+    du = mul2(mul2(gow, tg), mul2(mul2(Eu, splat(4.0f)), mul2(A, R)));
+    acc = fma2(mul2(go, tg), mul2(tu, mul2(AB, R)), acc);
   } else {
-    const float R = rcp_approx(A * A);
-    dg = gow * u * ng * R;
-    const float AR = A * R;                // 1 / A
-    du = gow * tg * AR;
-    return go * tg * u * AR;
+    const float2 u = as_f2(ub);
+    const float2 R = rcp2(mul2(A, A));
+    const float2 AR = mul2(A, R);
+    dg = mul2(mul2(gow, u), mul2(ng, R));
+    du = mul2(gow, mul2(tg, AR));
+    acc = fma2(mul2(go, tg), mul2(u, AR), acc);
   }
 }
 
@@ -274,6 +404,10 @@ __device__ __forceinline__ float block_sum(float v, float* slot) {
 // ---------------------------------------------------------------------------
 // Kernels
 // ---------------------------------------------------------------------------
+// One CTA works on one row at a time and strides over rows.  Thread t handles
+// the 16-byte vectors t, t + nt, t + 2 nt, ... of each half row, two at a time
+// (both loads are issued before any arithmetic), so each thread keeps two
+// vectors of every input in flight.
 
 struct FwdArgs {
   const char* gate_up;
@@ -288,20 +422,39 @@ struct FwdArgs {
 };
 
 template <typename S, int GATE, bool HAS_LB>
+__device__ __forceinline__ uint4 fwd_vec(const uint4& gv, const uint4& uv, float2 wbb, const Coeffs& c) {
+  uint4 o;
+#pragma unroll
+  for (int p = 0; p < S::kPairs; ++p) {
+    float2 y;
+    if constexpr (std::is_same<S, Bf16>::value)
+      y = fwd_pair_bf16<GATE, HAS_LB>(S::pair(gv, p), S::pair(uv, p), wbb, c);
+    else
+      y = fwd_pair_abs<GATE, HAS_LB, S>(S::pair(gv, p), S::pair(uv, p), wbb, c);
+    S::put(o, p, y);
+  }
+  return o;
+}
+
+template <typename S, int GATE, bool HAS_LB>
 __global__ void __launch_bounds__(kMaxThreads) situ_glu_fwd_kernel(const FwdArgs a) {
-  constexpr int N = S::kPerVec;
+  const int nt = blockDim.x;
   for (int64_t row = blockIdx.x; row < a.tokens; row += gridDim.x) {
     const char* gu = a.gate_up + row * a.gu_pitch;
     char* out = a.out + row * a.out_pitch;
-    const float wbb = load_rw(a.rw, row) * a.c.bb;
-    for (int j = threadIdx.x; j < a.vpr; j += blockDim.x) {
-      const int off = j * kVecBytes;
-      float g[N], u[N], y[N];
-      S::unpack(ld_stream(gu + off), g);
-      S::unpack(ld_stream(gu + a.half_bytes + off), u);
-#pragma unroll
-      for (int k = 0; k < N; ++k) y[k] = situ_fwd_elem<GATE, HAS_LB, S>(g[k], u[k], wbb, a.c);
-      st_stream(out + off, S::pack(y));
+    const float2 wbb = splat(load_rw(a.rw, row) * a.c.bb);
+    for (int j = threadIdx.x; j < a.vpr; j += 2 * nt) {
+      const int j2 = j + nt;
+      const bool two = j2 < a.vpr;
+      const uint4 g0 = ld_stream(gu + j * kVecBytes);
+      const uint4 u0 = ld_stream(gu + a.half_bytes + j * kVecBytes);
+      uint4 g1 = make_uint4(0, 0, 0, 0), u1 = g1;
+      if (two) {
+        g1 = ld_stream(gu + j2 * kVecBytes);
+        u1 = ld_stream(gu + a.half_bytes + j2 * kVecBytes);
+      }
+      st_stream(out + j * kVecBytes, fwd_vec<S, GATE, HAS_LB>(g0, u0, wbb, a.c));
+      if (two) st_stream(out + j2 * kVecBytes, fwd_vec<S, GATE, HAS_LB>(g1, u1, wbb, a.c));
     }
   }
 }
@@ -333,30 +486,53 @@ __device__ __forceinline__ void store_rw_grad(void* base, int64_t idx, int bf16,
 }
 
 template <typename S, int GATE, bool HAS_LB>
+__device__ __forceinline__ void bwd_vec(const uint4& gv, const uint4& uv, const uint4& gov, float w,
+                                        const Coeffs& c, uint4& dgv, uint4& duv, float2& acc) {
+#pragma unroll
+  for (int p = 0; p < S::kPairs; ++p) {
+    const float2 go = as_f2(S::pair(gov, p));
+    float2 dg, du;
+    bwd_pair<GATE, HAS_LB, S>(S::pair(gv, p), S::pair(uv, p), go, mul2(go, splat(w)), c, dg, du, acc);
+    S::put(dgv, p, dg);
+    S::put(duv, p, du);
+  }
+}
+
+template <typename S, int GATE, bool HAS_LB>
 __global__ void __launch_bounds__(kMaxThreads) situ_glu_bwd_kernel(const BwdArgs a) {
-  constexpr int N = S::kPerVec;
   __shared__ float red[2][kMaxThreads / 32];
+  const int nt = blockDim.x;
   int parity = 0;
   for (int64_t row = blockIdx.x; row < a.tokens; row += gridDim.x) {
     const char* gu = a.gate_up + row * a.gu_pitch;
     const char* go_row = a.grad_out + row * a.go_pitch;
     char* dgu = a.d_gate_up + row * a.dgu_pitch;
     const float w = load_rw(a.rw, row);
-    float acc = 0.0f;
-    for (int j = threadIdx.x; j < a.vpr; j += blockDim.x) {
-      const int off = j * kVecBytes;
-      float g[N], u[N], go[N], dg[N], du[N];
-      S::unpack(ld_stream(gu + off), g);
-      S::unpack(ld_stream(gu + a.half_bytes + off), u);
-      S::unpack(ld_stream(go_row + off), go);
-#pragma unroll
-      for (int k = 0; k < N; ++k)
-        acc += situ_bwd_elem<GATE, HAS_LB, S>(g[k], u[k], go[k], go[k] * w, a.c, dg[k], du[k]);
-      st_stream(dgu + off, S::pack(dg));
-      st_stream(dgu + a.half_bytes + off, S::pack(du));
+    float2 acc = make_float2(0.0f, 0.0f);
+    for (int j = threadIdx.x; j < a.vpr; j += 2 * nt) {
+      const int j2 = j + nt;
+      const bool two = j2 < a.vpr;
+      const uint4 g0 = ld_stream(gu + j * kVecBytes);
+      const uint4 u0 = ld_stream(gu + a.half_bytes + j * kVecBytes);
+      const uint4 o0 = ld_stream(go_row + j * kVecBytes);
+      uint4 g1 = make_uint4(0, 0, 0, 0), u1 = g1, o1 = g1;
+      if (two) {
+        g1 = ld_stream(gu + j2 * kVecBytes);
+        u1 = ld_stream(gu + a.half_bytes + j2 * kVecBytes);
+        o1 = ld_stream(go_row + j2 * kVecBytes);
+      }
+      uint4 dg, du;
+      bwd_vec<S, GATE, HAS_LB>(g0, u0, o0, w, a.c, dg, du, acc);
+      st_stream(dgu + j * kVecBytes, dg);
+      st_stream(dgu + a.half_bytes + j * kVecBytes, du);
+      if (two) {  // zero inputs contribute exactly 0 to acc, but skip them anyway
+        bwd_vec<S, GATE, HAS_LB>(g1, u1, o1, w, a.c, dg, du, acc);
+        st_stream(dgu + j2 * kVecBytes, dg);
+        st_stream(dgu + a.half_bytes + j2 * kVecBytes, du);
+      }
     }
     if (a.want_drw) {  // uniform over the launch
-      const float total = block_sum(acc, red[parity]);
+      const float total = block_sum(acc.x + acc.y, red[parity]);
       parity ^= 1;
       if (threadIdx.x == 0) {
         if (a.rw.mode == SITU_RW_SCALAR)
@@ -477,21 +653,22 @@ situ_status_t check_common(situ_dtype_t dtype, int64_t tokens, int64_t inter, in
     return fail(SITU_ERR_MISALIGNED, "inter * element size (%lld bytes) is not a multiple of 16",
                 (long long)(inter * es));
 
-  const double kLog2e = 1.4426950408889634;
+  const double kLog2eD = 1.4426950408889634;
   c->beta = static_cast<float>(beta);
-  c->neg_kt = static_cast<float>(-2.0 * kLog2e / beta);
-  c->xt_scale = static_cast<float>(2.0 / beta);
+  c->kt = static_cast<float>(2.0 * kLog2eD / beta);
   c->lb = has_lb ? static_cast<float>(lb) : 1.0f;
-  c->neg_ku = has_lb ? static_cast<float>(-2.0 * kLog2e / lb) : 0.0f;
-  c->xu_scale = has_lb ? static_cast<float>(2.0 / lb) : 0.0f;
+  c->inv_lb = has_lb ? static_cast<float>(1.0 / lb) : 1.0f;
+  c->ku = has_lb ? static_cast<float>(2.0 * kLog2eD / lb) : 0.0f;
   c->bb = static_cast<float>(has_lb ? beta * lb : beta);
   *gate_mode = beta == 4.0 ? kGateSquare : beta == 2.0 ? kGateEqual : beta == 1.0 ? kGateRoot : kGateGeneric;
   return SITU_OK;
 }
 
+// Threads per CTA: enough that each thread handles two 16-byte vectors of a
+// half row (one pass of the kernel's two-vector body), at most kMaxThreads.
 int choose_threads(int vpr) {
-  const int per_thread = (vpr + kMaxThreads - 1) / kMaxThreads;
-  const int nt = (vpr + per_thread - 1) / per_thread;
+  const int passes = (vpr + 2 * kMaxThreads - 1) / (2 * kMaxThreads);
+  const int nt = (vpr + 2 * passes - 1) / (2 * passes);
   return (nt + 31) / 32 * 32;
 }
 
