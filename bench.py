@@ -411,6 +411,7 @@ def run_ours(args):
             "e2e": e2e,
             "gpu_launches": launches_per_step * K,
             "clocks": clocks.summary(),
+            "device_status": pkg.abi.situ_glu_device_status(0),
             "device": torch.cuda.get_device_name(dev),
         }
         print(json.dumps(line), flush=True)

@@ -40,6 +40,8 @@ SIGNATURES = {
     "situ_glu_last_error": (ctypes.c_char_p, []),
     "situ_glu_abi_version": (_INT, []),
     "situ_glu_set_max_ctas": (_INT, [_INT]),
+    "situ_glu_set_load_path": (_INT, [_INT]),
+    "situ_glu_device_status": (_INT, [_INT]),
 }
 
 
@@ -119,6 +121,14 @@ def situ_glu_abi_version() -> int:
 
 def situ_glu_set_max_ctas(max_ctas) -> int:
     return lib().situ_glu_set_max_ctas(max_ctas)
+
+
+def situ_glu_set_load_path(path) -> int:
+    return lib().situ_glu_set_load_path(path)
+
+
+def situ_glu_device_status(clear) -> int:
+    return lib().situ_glu_device_status(clear)
 
 
 def status_string(status: int) -> str:

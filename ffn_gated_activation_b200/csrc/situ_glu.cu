@@ -277,7 +277,9 @@ __device__ __forceinline__ float2 fwd_pair_bf16(Bits2 gb, Bits2 ub, float2 wbb, 
   } else {
     t = as_f2(ub);
   }
-  return mul2(mul2(em, t), mul2(rcp2(den), wbb));
+  // em / den = T_g / beta lies in [-1, 1]: form it first so that a huge |1 - H|
+  // meets its zero reciprocal before it can meet a large U.
+  return mul2(mul2(em, rcp2(den)), mul2(t, wbb));
 }
 
 // ---- |g| form (fp32 forward and every backward) ---------------------------
@@ -557,6 +559,244 @@ __global__ void __launch_bounds__(kFinalizeThreads)
 }
 
 // ---------------------------------------------------------------------------
+// TMA-staged kernels (the default path)
+// ---------------------------------------------------------------------------
+// Warp 0 of each CTA is a producer: one lane streams chunks of rows from HBM
+// into a ring of shared-memory stages with 1-D bulk copies (cp.async.bulk,
+// completion counted in bytes on the stage's "full" mbarrier).  The other
+// warps are consumers: they wait on "full", read their 16-byte vectors from
+// shared memory, compute in registers, store the outputs straight to global
+// memory, and release the stage on its "empty" mbarrier.  The bytes in flight
+// are set by the ring, not by registers, so the consumers keep every register
+// for arithmetic.  A CTA visits rows blockIdx.x, blockIdx.x + gridDim.x, ...
+// and, within a row, its chunks in order; producer and consumers derive the
+// same sequence, so no work queue is needed.
+//
+// Every wait is bounded (kWaitLimitNs of %globaltimer).  A wait that expires
+// sets g_device_status; a consumer then stops waiting and computing but keeps
+// the control flow (so the consumer-only named barrier cannot strand anyone),
+// and the producer waits, again bounded, for the copies it issued before it
+// returns.
+
+constexpr int kMaxStages = 8;
+constexpr int kMaxConsumers = 256;
+#ifndef SITU_RING_BYTES
+#define SITU_RING_BYTES (32 * 1024)
+#endif
+constexpr int kRingBytes = SITU_RING_BYTES;  // shared-memory ring per CTA
+constexpr int kHeaderBytes = 256;      // mbarriers + reduction slots
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr int kStatusWaitExpired = 1;
+
+__device__ int g_device_status = 0;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for the phase of parity `parity` to complete; false once the limit expires.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
+  if (mbar_try_wait(b, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  while (!mbar_try_wait(b, parity))
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+  return true;
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ uint4 lds16(const unsigned char* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ void consumer_bar(int n) { asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory"); }
+
+struct StreamArgs {
+  const char* gate_up;
+  int64_t gu_pitch;  // bytes
+  const char* grad_out;  // backward only
+  int64_t go_pitch;
+  char* out;  // forward: Y; backward: d_gate_up
+  int64_t out_pitch;
+  RwArgs rw;
+  void* d_rw;
+  int64_t d_rw_stride;
+  float* partials;
+  int want_drw;
+  int64_t tokens;
+  int half_bytes;   // inter * element size
+  int vpr;          // 16-byte vectors per half row
+  int chunk_v;      // vectors per half row per chunk (the last chunk may be shorter)
+  int nchunks;      // chunks per row
+  int stages;       // ring stages
+  int stage_bytes;  // bytes per stage (inputs x chunk_v x 16, rounded to 128)
+  Coeffs c;
+};
+
+template <typename S, int GATE, bool HAS_LB, bool BWD>
+__device__ __forceinline__ void tma_stream_body(const StreamArgs& a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  constexpr int kInputs = BWD ? 3 : 2;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + kMaxStages;
+  float* red = reinterpret_cast<float*>(empty + kMaxStages);  // [2][kMaxConsumers / 32]
+  unsigned char* ring = smem + kHeaderBytes;
+  const int nc = blockDim.x - 32;
+  const int chunk_bytes = a.chunk_v * kVecBytes;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], nc / 32);
+    }
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (threadIdx.x < 32) {  // ---- producer warp: one lane issues the copies
+    if (threadIdx.x != 0) return;
+    int64_t k = 0;
+    bool ok = true;
+    for (int64_t row = blockIdx.x; ok && row < a.tokens; row += gridDim.x) {
+      const char* gu = a.gate_up + row * a.gu_pitch;
+      const char* go = BWD ? a.grad_out + row * a.go_pitch : nullptr;
+      for (int ch = 0; ch < a.nchunks; ++ch, ++k) {
+        const int s = static_cast<int>(k % a.stages);
+        const int64_t use = k / a.stages;
+        if (use > 0 && !mbar_wait(&empty[s], static_cast<uint32_t>((use - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        const int v0 = ch * a.chunk_v;
+        const uint32_t bytes = static_cast<uint32_t>(min(a.chunk_v, a.vpr - v0)) * kVecBytes;
+        unsigned char* st = ring + s * a.stage_bytes;
+        mbar_arrive_expect_tx(&full[s], bytes * kInputs);
+        bulk_load(st, gu + v0 * kVecBytes, bytes, &full[s]);
+        bulk_load(st + chunk_bytes, gu + a.half_bytes + v0 * kVecBytes, bytes, &full[s]);
+        if (BWD) bulk_load(st + 2 * chunk_bytes, go + v0 * kVecBytes, bytes, &full[s]);
+      }
+    }
+    if (!ok) {  // drain: the last copy issued into each stage must land before the CTA exits
+      atomicExch(&g_device_status, kStatusWaitExpired);
+      for (int s = 0; s < a.stages && s < k; ++s) {
+        const int64_t last_use = (k - 1 - s) / a.stages;
+        mbar_wait(&full[s], static_cast<uint32_t>(last_use & 1));
+      }
+    }
+    return;
+  }
+
+  // ---- consumer warps
+  const int ctid = threadIdx.x - 32;
+  const int lane = threadIdx.x & 31;
+  int64_t k = 0;
+  int parity = 0;
+  bool ok = true;
+  for (int64_t row = blockIdx.x; row < a.tokens; row += gridDim.x) {
+    const float w = load_rw(a.rw, row);
+    const float2 wbb = splat(w * a.c.bb);
+    char* out = a.out + row * a.out_pitch;
+    float2 acc = make_float2(0.0f, 0.0f);
+    for (int ch = 0; ch < a.nchunks; ++ch, ++k) {
+      const int s = static_cast<int>(k % a.stages);
+      const int64_t use = k / a.stages;
+      if (ok && !mbar_wait(&full[s], static_cast<uint32_t>(use & 1))) {
+        ok = false;
+        atomicExch(&g_device_status, kStatusWaitExpired);
+      }
+      if (!ok) continue;
+      const unsigned char* st = ring + s * a.stage_bytes;
+      const int v0 = ch * a.chunk_v;
+      const int nv = min(a.chunk_v, a.vpr - v0);
+      for (int v = ctid; v < nv; v += 2 * nc) {
+        const int v2 = v + nc;
+        const bool two = v2 < nv;
+        const uint4 g0 = lds16(st + v * kVecBytes);
+        const uint4 u0 = lds16(st + chunk_bytes + v * kVecBytes);
+        uint4 g1 = make_uint4(0, 0, 0, 0), u1 = g1;
+        if (two) {
+          g1 = lds16(st + v2 * kVecBytes);
+          u1 = lds16(st + chunk_bytes + v2 * kVecBytes);
+        }
+        char* o0 = out + (v0 + v) * kVecBytes;
+        char* o1 = out + (v0 + v2) * kVecBytes;
+        if constexpr (BWD) {
+          const uint4 q0 = lds16(st + 2 * chunk_bytes + v * kVecBytes);
+          const uint4 q1 = two ? lds16(st + 2 * chunk_bytes + v2 * kVecBytes) : make_uint4(0, 0, 0, 0);
+          uint4 dg, du;
+          bwd_vec<S, GATE, HAS_LB>(g0, u0, q0, w, a.c, dg, du, acc);
+          st_stream(o0, dg);
+          st_stream(o0 + a.half_bytes, du);
+          if (two) {
+            bwd_vec<S, GATE, HAS_LB>(g1, u1, q1, w, a.c, dg, du, acc);
+            st_stream(o1, dg);
+            st_stream(o1 + a.half_bytes, du);
+          }
+        } else {
+          st_stream(o0, fwd_vec<S, GATE, HAS_LB>(g0, u0, wbb, a.c));
+          if (two) st_stream(o1, fwd_vec<S, GATE, HAS_LB>(g1, u1, wbb, a.c));
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    if (BWD && a.want_drw) {  // fixed-order sum over the consumer threads
+      float v = acc.x + acc.y;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      float* slot = red + parity * (kMaxConsumers / 32);
+      if (lane == 0) slot[ctid >> 5] = v;
+      consumer_bar(nc);
+      if (ctid < 32) {
+        float t = ctid < nc / 32 ? slot[ctid] : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (ctid == 0 && ok) {
+          if (a.rw.mode == SITU_RW_SCALAR)
+            a.partials[row] = t;
+          else
+            store_rw_grad(a.d_rw, row * a.d_rw_stride, a.rw.bf16, t);
+        }
+      }
+      parity ^= 1;
+    }
+  }
+}
+
+template <typename S, int GATE, bool HAS_LB>
+__global__ void __launch_bounds__(kMaxConsumers + 32) situ_glu_fwd_tma_kernel(const StreamArgs a) {
+  tma_stream_body<S, GATE, HAS_LB, false>(a);
+}
+
+template <typename S, int GATE, bool HAS_LB>
+__global__ void __launch_bounds__(kMaxConsumers + 32) situ_glu_bwd_tma_kernel(const StreamArgs a) {
+  tma_stream_body<S, GATE, HAS_LB, true>(a);
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 
@@ -672,12 +912,12 @@ int choose_threads(int vpr) {
   return (nt + 31) / 32 * 32;
 }
 
-situ_status_t launch_grid(const void* kernel, int threads, int64_t tokens, int* grid) {
+situ_status_t launch_grid(const void* kernel, int threads, int smem, int64_t tokens, int* grid) {
   int sms = 0;
   situ_status_t st = device_sm_count(&sms);
   if (st != SITU_OK) return st;
   int per_sm = 0;
-  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0);
+  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem);
   if (err != cudaSuccess || per_sm <= 0)
     return fail(SITU_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(err));
   int64_t g = static_cast<int64_t>(sms) * per_sm;
@@ -686,6 +926,98 @@ situ_status_t launch_grid(const void* kernel, int threads, int64_t tokens, int* 
   if (g > tokens) g = tokens;
   *grid = static_cast<int>(g);
   return SITU_OK;
+}
+
+situ_status_t check_launch(const char* what);
+
+std::atomic<int> g_load_path{0};  // 0: TMA ring (default), 1: direct vector loads
+
+// Ring geometry of the TMA-staged kernels for a half row of `vpr` vectors and
+// `inputs` streamed inputs (2 forward, 3 backward).
+struct Geometry {
+  int chunk_v, nchunks, consumers, stage_bytes, stages, smem;
+};
+
+Geometry stream_geometry(int vpr, int inputs) {
+  Geometry g;
+  const int balanced = (vpr + 2 * kMaxConsumers - 1) / (2 * kMaxConsumers);
+  g.chunk_v = (vpr + balanced - 1) / balanced;        // <= 2 * kMaxConsumers
+  g.nchunks = (vpr + g.chunk_v - 1) / g.chunk_v;      // every chunk holds >= 1 vector
+  g.consumers = ((g.chunk_v + 1) / 2 + 31) / 32 * 32;
+  g.stage_bytes = (g.chunk_v * kVecBytes * inputs + 127) / 128 * 128;
+  g.stages = kRingBytes / g.stage_bytes;
+  if (g.stages > kMaxStages) g.stages = kMaxStages;
+  if (g.stages < 2) g.stages = 2;
+  g.smem = kHeaderBytes + g.stages * g.stage_bytes;
+  return g;
+}
+
+// Opt a kernel in to more than 48 KB of dynamic shared memory, once per
+// (device, kernel, size).
+situ_status_t ensure_smem(const void* kernel, int bytes) {
+  struct Entry {
+    int dev;
+    const void* kernel;
+    int bytes;
+  };
+  static std::mutex mu;
+  static Entry seen[256];
+  static int n_seen = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaGetDevice failed");
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n_seen; ++i)
+    if (seen[i].dev == dev && seen[i].kernel == kernel && seen[i].bytes >= bytes) return SITU_OK;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(err));
+  if (n_seen < 256) seen[n_seen++] = {dev, kernel, bytes};
+  return SITU_OK;
+}
+
+using StreamKernel = void (*)(StreamArgs);
+
+template <typename S, int GATE, bool LB, bool BWD>
+StreamKernel stream_kernel() {
+  if constexpr (BWD)
+    return situ_glu_bwd_tma_kernel<S, GATE, LB>;
+  else
+    return situ_glu_fwd_tma_kernel<S, GATE, LB>;
+}
+
+template <typename S, bool LB, bool BWD>
+StreamKernel pick_stream_gate(int gate) {
+  switch (gate) {
+    case kGateSquare: return stream_kernel<S, kGateSquare, LB, BWD>();
+    case kGateEqual: return stream_kernel<S, kGateEqual, LB, BWD>();
+    case kGateRoot: return stream_kernel<S, kGateRoot, LB, BWD>();
+    default: return stream_kernel<S, kGateGeneric, LB, BWD>();
+  }
+}
+
+template <bool BWD>
+StreamKernel pick_stream(situ_dtype_t dtype, int gate, bool lb) {
+  if (dtype == SITU_DTYPE_BF16)
+    return lb ? pick_stream_gate<Bf16, true, BWD>(gate) : pick_stream_gate<Bf16, false, BWD>(gate);
+  return lb ? pick_stream_gate<F32, true, BWD>(gate) : pick_stream_gate<F32, false, BWD>(gate);
+}
+
+// Launch the TMA-staged kernel for the arguments in `a`.
+template <bool BWD>
+situ_status_t launch_stream(StreamArgs& a, situ_dtype_t dtype, int gate, bool lb, cudaStream_t stream) {
+  const Geometry g = stream_geometry(a.vpr, BWD ? 3 : 2);
+  a.chunk_v = g.chunk_v;
+  a.nchunks = g.nchunks;
+  a.stages = g.stages;
+  a.stage_bytes = g.stage_bytes;
+  StreamKernel k = pick_stream<BWD>(dtype, gate, lb);
+  situ_status_t st = ensure_smem(reinterpret_cast<const void*>(k), g.smem);
+  if (st != SITU_OK) return st;
+  const int threads = g.consumers + 32;
+  int grid = 0;
+  st = launch_grid(reinterpret_cast<const void*>(k), threads, g.smem, a.tokens, &grid);
+  if (st != SITU_OK) return st;
+  k<<<grid, threads, g.smem, stream>>>(a);
+  return check_launch(BWD ? "situ_glu_bwd" : "situ_glu_fwd");
 }
 
 situ_status_t check_launch(const char* what) {
@@ -777,10 +1109,23 @@ situ_status_t situ_glu_fwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
   a.c = c;
   if (rw_mode == SITU_RW_NONE) a.rw.bf16 = 0;
 
+  if (g_load_path.load(std::memory_order_relaxed) == 0) {
+    StreamArgs sa{};
+    sa.gate_up = a.gate_up;
+    sa.gu_pitch = a.gu_pitch;
+    sa.out = a.out;
+    sa.out_pitch = a.out_pitch;
+    sa.rw = a.rw;
+    sa.tokens = tokens;
+    sa.half_bytes = a.half_bytes;
+    sa.vpr = a.vpr;
+    sa.c = c;
+    return launch_stream<false>(sa, dtype, gate, has_linear_beta != 0, static_cast<cudaStream_t>(stream));
+  }
   FwdKernel k = pick_fwd(dtype, gate, has_linear_beta != 0);
   const int threads = choose_threads(a.vpr);
   int grid = 0;
-  st = launch_grid(reinterpret_cast<const void*>(k), threads, tokens, &grid);
+  st = launch_grid(reinterpret_cast<const void*>(k), threads, 0, tokens, &grid);
   if (st != SITU_OK) return st;
   k<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(a);
   return check_launch("situ_glu_fwd");
@@ -883,14 +1228,34 @@ situ_status_t situ_glu_bwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
   a.vpr = static_cast<int>(inter * es / kVecBytes);
   a.c = c;
 
-  BwdKernel k = pick_bwd(dtype, gate, has_linear_beta != 0);
-  const int threads = choose_threads(a.vpr);
-  int grid = 0;
-  st = launch_grid(reinterpret_cast<const void*>(k), threads, tokens, &grid);
-  if (st != SITU_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  k<<<grid, threads, 0, s>>>(a);
-  st = check_launch("situ_glu_bwd");
+  if (g_load_path.load(std::memory_order_relaxed) == 0) {
+    StreamArgs sa{};
+    sa.gate_up = a.gate_up;
+    sa.gu_pitch = a.gu_pitch;
+    sa.grad_out = a.grad_out;
+    sa.go_pitch = a.go_pitch;
+    sa.out = a.d_gate_up;
+    sa.out_pitch = a.dgu_pitch;
+    sa.rw = a.rw;
+    sa.d_rw = a.d_rw;
+    sa.d_rw_stride = a.d_rw_stride;
+    sa.partials = a.partials;
+    sa.want_drw = a.want_drw;
+    sa.tokens = tokens;
+    sa.half_bytes = a.half_bytes;
+    sa.vpr = a.vpr;
+    sa.c = c;
+    st = launch_stream<true>(sa, dtype, gate, has_linear_beta != 0, s);
+  } else {
+    BwdKernel k = pick_bwd(dtype, gate, has_linear_beta != 0);
+    const int threads = choose_threads(a.vpr);
+    int grid = 0;
+    st = launch_grid(reinterpret_cast<const void*>(k), threads, 0, tokens, &grid);
+    if (st != SITU_OK) return st;
+    k<<<grid, threads, 0, s>>>(a);
+    st = check_launch("situ_glu_bwd");
+  }
   if (st != SITU_OK) return st;
   if (want_drw && rw_mode == SITU_RW_SCALAR) {
     situ_glu_dw_scalar_finalize_kernel<<<1, kFinalizeThreads, 0, s>>>(a.partials, tokens, d_rw, a.rw.bf16);
@@ -913,6 +1278,22 @@ const char* situ_glu_status_string(situ_status_t status) {
 const char* situ_glu_last_error(void) { return tl_last_error; }
 
 int situ_glu_abi_version(void) { return SITU_GLU_ABI_VERSION; }
+
+int situ_glu_set_load_path(int path) {
+  if (path != 0 && path != 1) return -1;
+  return g_load_path.exchange(path);
+}
+
+int situ_glu_device_status(int clear) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof v) != cudaSuccess) return -1;
+  if (clear && v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof zero) != cudaSuccess) return -1;
+  }
+  return v;
+}
 
 int situ_glu_set_max_ctas(int max_ctas) {
   if (max_ctas < 0) return -1;

@@ -169,6 +169,22 @@ int situ_glu_abi_version(void);
  * value, or -1 (and changes nothing) for a negative argument. */
 int situ_glu_set_max_ctas(int max_ctas);
 
+/* How the kernels read HBM.  0 (default): one lane per CTA streams chunks of
+ * rows into a shared-memory ring with TMA bulk copies (cp.async.bulk) and the
+ * other warps compute from it.  1: every thread loads its own 16-byte vectors
+ * into registers.  Both paths run the same arithmetic, so results are bitwise
+ * identical.  Process-wide; returns the previous value, or -1 (and changes
+ * nothing) for any other argument. */
+int situ_glu_set_load_path(int path);
+
+/* Status word the kernels set on the current device when one of their
+ * bounded waits (on a shared-memory stage, 2 s at most) expires: 0 = none
+ * has, 1 = a wait expired and that launch's outputs are not valid.  A kernel
+ * whose wait expires returns instead of hanging.  Synchronises the device
+ * first; a nonzero `clear` resets the word.  Returns -1 if the CUDA runtime
+ * reports an error. */
+int situ_glu_device_status(int clear);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

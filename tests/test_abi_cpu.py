@@ -36,7 +36,8 @@ def declared_functions():
 def test_header_declares_the_abi():
     names = declared_functions()
     assert {"situ_glu_fwd", "situ_glu_bwd", "situ_glu_bwd_workspace_bytes", "situ_glu_status_string",
-            "situ_glu_last_error", "situ_glu_abi_version", "situ_glu_set_max_ctas"} <= names
+            "situ_glu_last_error", "situ_glu_abi_version", "situ_glu_set_max_ctas",
+            "situ_glu_set_load_path", "situ_glu_device_status"} <= names
 
 
 def test_library_exports_every_declared_symbol(native_lib_path):
@@ -70,6 +71,13 @@ def test_workspace_query(native_lib_path):
     assert abi.situ_glu_bwd_workspace_bytes(64, SCALAR, 1) == 256
     assert abi.situ_glu_bwd_workspace_bytes(0, SCALAR, 1) == 0
     assert abi.situ_glu_bwd_workspace_bytes(-5, SCALAR, 1) == 0
+
+
+def test_load_path_knob(native_lib_path):
+    prev = abi.situ_glu_set_load_path(1)
+    assert abi.situ_glu_set_load_path(prev) == 1
+    assert abi.situ_glu_set_load_path(2) == -1
+    assert abi.situ_glu_set_load_path(-1) == -1
 
 
 def test_max_ctas_knob(native_lib_path):

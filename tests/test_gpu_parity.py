@@ -302,3 +302,36 @@ def test_errors_surface_from_the_library(cuda_device):
         pkg.situ_glu_fwd(gu, torch.ones(4, 1, device=dev))
     with pytest.raises(ValueError):
         pkg.situ_glu_fwd(torch.zeros(4, 32, dtype=torch.bfloat16, device=dev), None, beta=0.0)
+
+
+@pytest.mark.parametrize("dtype,T,I,lb", [("bf16", 257, 520, 25.0), ("bf16", 64, 3072, None),
+                                          ("f32", 33, 4096, 25.0), ("bf16", 5, 8, 25.0)])
+def test_load_paths_bitwise_identical(dtype, T, I, lb, cuda_device):
+    """The shared-memory ring (TMA bulk copies) and the direct-load path run the
+    same arithmetic: every output must match bit for bit."""
+    dev = cuda_device
+    gu_h, rw32, go_h = case_inputs(dtype, T, I, seed=31)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    gu, go, rw = to_device(gu_h, dev), to_device(go_h, dev), to_device(rw32, dev)
+    results = []
+    prev = abi.situ_glu_set_load_path(0)
+    try:
+        for path in (0, 1):
+            abi.situ_glu_set_load_path(path)
+            out = Guarded(T, I, I, tdt, dev)
+            dgu = Guarded(T, 2 * I, 2 * I, tdt, dev)
+            d_rw = torch.empty(T, dtype=torch.float32, device=dev)
+            abi.check(call_fwd(gu, I, rw, abi.SITU_RW_ROW, 4.0, lb, out), "fwd")
+            abi.check(call_bwd(gu, I, rw, abi.SITU_RW_ROW, 4.0, lb, go, dgu, d_rw=d_rw), "bwd")
+            torch.cuda.synchronize()
+            out.check(); dgu.check()
+            results.append([to_host(out.view), to_host(dgu.view), to_host(d_rw)])
+    finally:
+        abi.situ_glu_set_load_path(prev)
+    for a, b in zip(*results):
+        assert np.array_equal(a.view(np.uint8), b.view(np.uint8))
+
+
+def test_no_bounded_wait_expired(cuda_device):
+    """No kernel launched by the tests above gave up on a shared-memory stage."""
+    assert abi.situ_glu_device_status(0) == 0
