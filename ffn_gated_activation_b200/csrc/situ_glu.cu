@@ -204,12 +204,35 @@ struct Series<F32> {
   }
 };
 
+// The bf16 backward's up branch feeds T_u only as a relative factor (dG within
+// 2^-8, d_w as a sum of terms with independent rounding), so terms to y^3 for
+// |x| < 1/32 suffice there (truncation below 2^-19.6; 1 - E above it within
+// about 2^-18).
+struct SeriesBf16Up {
+  static constexpr float kYmax = 0.03125f / kLn2;
+  __device__ __forceinline__ static float2 eval(float2 y) {
+    const float c1 = kLn2, c2 = -kLn2 * kLn2 / 2.0f, c3 = kLn2 * kLn2 * kLn2 / 6.0f;
+    float2 p = fma2(y, splat(c3), splat(c2));
+    p = fma2(p, y, splat(c1));
+    return mul2(p, y);
+  }
+};
+
+// Series used for the backward's up branch, per storage type.
 template <typename S>
+struct UpSeries {
+  using type = Series<S>;
+};
+template <>
+struct UpSeries<Bf16> {
+  using type = SeriesBf16Up;
+};
+
+template <typename S, typename P = Series<S>>
 __device__ __forceinline__ float2 one_minus_exp2_neg(float2 y, float2 E) {
-  const float2 series = Series<S>::eval(y);
-  const float2 direct = add2(splat(1.0f), make_float2(-E.x, -E.y));
-  return make_float2(fabsf(y.x) < Series<S>::kYmax ? series.x : direct.x,
-                     fabsf(y.y) < Series<S>::kYmax ? series.y : direct.y);
+  const float2 series = P::eval(y);
+  const float2 direct = fma2(E, splat(-1.0f), splat(1.0f));
+  return make_float2(fabsf(y.x) < P::kYmax ? series.x : direct.x, fabsf(y.y) < P::kYmax ? series.y : direct.y);
 }
 
 // How the two gate exponentials relate for the given beta.
@@ -300,11 +323,11 @@ __device__ __forceinline__ GateAbs gate_abs(Bits2 gb, const Coeffs& c) {
   return r;
 }
 
-template <typename S>
+template <typename S, typename P = Series<S>>
 __device__ __forceinline__ float2 up_emu(Bits2 ub, const Coeffs& c, float2& Eu) {
   const float2 y = mul2(abs_f2(ub), splat(c.ku));
   Eu = ex2_neg2(y);
-  return one_minus_exp2_neg<S>(y, Eu);
+  return one_minus_exp2_neg<S, P>(y, Eu);
 }
 
 // fp32 forward of a pair.  Y = w beta beta_L s_g s_u (1 - E_t) sig (1 - E_u)
@@ -330,40 +353,45 @@ __device__ __forceinline__ float2 fwd_pair_abs(Bits2 gb, Bits2 ub, float2 wbb, c
 }
 
 // Backward of a pair.  With A = (1 + E_t)(1 + E_s), B = 1 + E_u (1 without a
-// linear beta), tb = beta tanh(g/beta) (1 + E_t) and sig as above:
-//   T_g  = tb sig / A
-//   T_g' = [4 E_t sig (1 + E_s) + tb (1 + E_t) E_s] / A^2
-//          (sech^2(g/beta) sigmoid + beta tanh sigmoid (1 - sigmoid), each over A^2)
-//   T_u  = tu / B,  T_u' = 4 E_u / B^2,  tu = beta_L s_u (1 - E_u)
-// and one reciprocal R = 1 / (A B)^2 serves every quotient.  Returns dG, dU;
-// adds go T_g T_u to acc.
+// linear beta), sig as above and
+//   tq  = (beta/4) tanh(g/beta) (1 + E_t)              (= (beta/4) s_g (1 - E_t))
+//   T_g  = 4 tq sig / A
+//   T_g' = 4 [E_t sig (1 + E_s) + tq (1 + E_t) E_s] / A^2
+//          (the sech^2(g/beta) sigmoid and beta tanh sigmoid (1 - sigmoid) terms)
+//   T_u  = beta_L su / B,  su = s_u (1 - E_u),   T_u' = 4 E_u / B^2
+// one reciprocal R = 1 / (A B)^2 serves every quotient.  The per-row factors
+// are folded into two constants: k.x = 4 beta_L w (dG) and k.y = 16 w (dU);
+// the d_w terms are accumulated without their factor 4 beta_L, which the
+// caller applies once per row.  Returns dG, dU; adds go T_g T_u / (4 beta_L)
+// to acc.
 template <int GATE, bool HAS_LB, typename S>
-__device__ __forceinline__ void bwd_pair(Bits2 gb, Bits2 ub, float2 go, float2 gow, const Coeffs& c, float2& dg,
-                                         float2& du, float2& acc) {
+__device__ __forceinline__ void bwd_pair(Bits2 gb, Bits2 ub, float2 go, float2 kdg, float2 kdu, const Coeffs& c,
+                                         float2& dg, float2& du, float2& acc) {
   const GateAbs e = gate_abs<GATE, S>(gb, c);
   const float2 sig = select_neg2(gb, e.Es, splat(1.0f));
   const float2 opt = add2(splat(1.0f), e.Et), ops = add2(splat(1.0f), e.Es);
   const float2 A = mul2(opt, ops);
-  const float2 tb = mul2(xor_sign2(e.emt, gb), splat(c.beta));
-  const float2 tg = mul2(tb, sig);
-  const float2 ng = fma2(mul2(mul2(e.Et, sig), ops), splat(4.0f), mul2(mul2(tb, opt), e.Es));
+  float2 tq = xor_sign2(e.emt, gb);
+  if (GATE != kGateSquare) tq = mul2(tq, splat(0.25f * c.beta));  // beta = 4: the factor is 1
+  const float2 tg = mul2(tq, sig);                                  // T_g A / 4
+  const float2 ng = fma2(mul2(e.Et, sig), ops, mul2(mul2(tq, opt), e.Es));  // T_g' A^2 / 4
+  const float2 gtg = mul2(go, tg);
   if (HAS_LB) {
     float2 Eu;
-    const float2 emu = up_emu<S>(ub, c, Eu);
-    const float2 tu = mul2(xor_sign2(emu, ub), splat(c.lb));
+    const float2 su = xor_sign2(up_emu<S, typename UpSeries<S>::type>(ub, c, Eu), ub);  // T_u B / beta_L
     const float2 B = add2(splat(1.0f), Eu);
     const float2 AB = mul2(A, B);
     const float2 R = rcp2(mul2(AB, AB));
-    dg = mul2(mul2(gow, tu), mul2(ng, mul2(B, R)));
-    du = mul2(mul2(gow, tg), mul2(mul2(Eu, splat(4.0f)), mul2(A, R)));
-    acc = fma2(mul2(go, tg), mul2(tu, mul2(AB, R)), acc);
+    dg = mul2(mul2(go, mul2(su, kdg)), mul2(ng, mul2(B, R)));  // go w T_u T_g'
+    du = mul2(mul2(gtg, mul2(Eu, kdu)), mul2(A, R));           // go w T_g T_u'
+    acc = fma2(gtg, mul2(su, mul2(AB, R)), acc);                // go T_g T_u / (4 beta_L)
   } else {
     const float2 u = as_f2(ub);
     const float2 R = rcp2(mul2(A, A));
     const float2 AR = mul2(A, R);
-    dg = mul2(mul2(gow, u), mul2(ng, R));
-    du = mul2(gow, mul2(tg, AR));
-    acc = fma2(mul2(go, tg), mul2(u, AR), acc);
+    dg = mul2(mul2(go, mul2(u, kdg)), mul2(ng, R));
+    du = mul2(mul2(gtg, kdu), AR);
+    acc = fma2(gtg, mul2(u, AR), acc);
   }
 }
 
@@ -438,9 +466,78 @@ __device__ __forceinline__ uint4 fwd_vec(const uint4& gv, const uint4& uv, float
   return o;
 }
 
+// Whether a direct-load kernel loads the CTA's next row while it computes the
+// current one (measured on B200: faster for every forward and the bf16
+// backward, slower for the fp32 backward, whose extra registers cost more
+// occupancy than the overlap gains).
+template <typename S, bool BWD>
+struct PipelineRows {
+  static constexpr bool value = !BWD || std::is_same<S, Bf16>::value;
+};
+// Register budgets of the direct-load kernels: when set, the resident CTAs of
+// kMaxThreads threads that __launch_bounds__ must allow; unset leaves the
+// choice to the compiler.
+#ifdef SITU_FWD_MIN_CTAS
+#define SITU_FWD_BOUNDS __launch_bounds__(kMaxThreads, SITU_FWD_MIN_CTAS)
+#else
+#define SITU_FWD_BOUNDS __launch_bounds__(kMaxThreads)
+#endif
+#ifdef SITU_BWD_MIN_CTAS
+#define SITU_BWD_BOUNDS __launch_bounds__(kMaxThreads, SITU_BWD_MIN_CTAS)
+#else
+#define SITU_BWD_BOUNDS __launch_bounds__(kMaxThreads)
+#endif
+
 template <typename S, int GATE, bool HAS_LB>
-__global__ void __launch_bounds__(kMaxThreads) situ_glu_fwd_kernel(const FwdArgs a) {
+__global__ void SITU_FWD_BOUNDS situ_glu_fwd_kernel(const FwdArgs a) {
   const int nt = blockDim.x;
+  if (PipelineRows<S, false>::value && a.vpr <= 2 * nt) {
+    // Each thread owns vectors j and j + nt of every row it visits: load the
+    // CTA's next row while computing the current one, so that loads stay in
+    // flight during the arithmetic.
+    const int j = threadIdx.x, j2 = j + nt;
+    const bool one = j < a.vpr, two = j2 < a.vpr;
+    int64_t row = blockIdx.x;
+    if (row >= a.tokens) return;
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    uint4 g0 = z, u0 = z, g1 = z, u1 = z;
+    const char* gu = a.gate_up + row * a.gu_pitch;
+    if (one) {
+      g0 = ld_stream(gu + j * kVecBytes);
+      u0 = ld_stream(gu + a.half_bytes + j * kVecBytes);
+    }
+    if (two) {
+      g1 = ld_stream(gu + j2 * kVecBytes);
+      u1 = ld_stream(gu + a.half_bytes + j2 * kVecBytes);
+    }
+    float w = load_rw(a.rw, row);
+    for (;;) {
+      const int64_t next = row + gridDim.x;
+      const bool more = next < a.tokens;
+      uint4 ng0 = z, nu0 = z, ng1 = z, nu1 = z;
+      float nw = 0.0f;
+      if (more) {
+        const char* ngu = a.gate_up + next * a.gu_pitch;
+        if (one) {
+          ng0 = ld_stream(ngu + j * kVecBytes);
+          nu0 = ld_stream(ngu + a.half_bytes + j * kVecBytes);
+        }
+        if (two) {
+          ng1 = ld_stream(ngu + j2 * kVecBytes);
+          nu1 = ld_stream(ngu + a.half_bytes + j2 * kVecBytes);
+        }
+        nw = load_rw(a.rw, next);
+      }
+      char* out = a.out + row * a.out_pitch;
+      const float2 wbb = splat(w * a.c.bb);
+      if (one) st_stream(out + j * kVecBytes, fwd_vec<S, GATE, HAS_LB>(g0, u0, wbb, a.c));
+      if (two) st_stream(out + j2 * kVecBytes, fwd_vec<S, GATE, HAS_LB>(g1, u1, wbb, a.c));
+      if (!more) break;
+      row = next;
+      g0 = ng0; u0 = nu0; g1 = ng1; u1 = nu1; w = nw;
+    }
+    return;
+  }
   for (int64_t row = blockIdx.x; row < a.tokens; row += gridDim.x) {
     const char* gu = a.gate_up + row * a.gu_pitch;
     char* out = a.out + row * a.out_pitch;
@@ -487,29 +584,111 @@ __device__ __forceinline__ void store_rw_grad(void* base, int64_t idx, int bf16,
   }
 }
 
+// Per-row constants of the backward: k.x = 4 beta_L w (dG); k.y = 16 w (dU:
+// 4 from T_g, 4 from T_u' = 4 E_u / B^2), or 4 w without a linear beta
+// (T_u' = 1); and the d_w scale 4 beta_L (beta_L = 1 without a linear beta).
+template <bool HAS_LB>
+__device__ __forceinline__ float2 bwd_row_consts(float w, const Coeffs& c) {
+  return make_float2(4.0f * c.lb * w, (HAS_LB ? 16.0f : 4.0f) * w);
+}
+__device__ __forceinline__ float bwd_dw_scale(const Coeffs& c) { return 4.0f * c.lb; }
+
 template <typename S, int GATE, bool HAS_LB>
-__device__ __forceinline__ void bwd_vec(const uint4& gv, const uint4& uv, const uint4& gov, float w,
+__device__ __forceinline__ void bwd_vec(const uint4& gv, const uint4& uv, const uint4& gov, float2 k,
                                         const Coeffs& c, uint4& dgv, uint4& duv, float2& acc) {
+  const float2 kdg = splat(k.x), kdu = splat(k.y);
 #pragma unroll
   for (int p = 0; p < S::kPairs; ++p) {
-    const float2 go = as_f2(S::pair(gov, p));
     float2 dg, du;
-    bwd_pair<GATE, HAS_LB, S>(S::pair(gv, p), S::pair(uv, p), go, mul2(go, splat(w)), c, dg, du, acc);
+    bwd_pair<GATE, HAS_LB, S>(S::pair(gv, p), S::pair(uv, p), as_f2(S::pair(gov, p)), kdg, kdu, c, dg, du, acc);
     S::put(dgv, p, dg);
     S::put(duv, p, du);
   }
 }
 
 template <typename S, int GATE, bool HAS_LB>
-__global__ void __launch_bounds__(kMaxThreads) situ_glu_bwd_kernel(const BwdArgs a) {
+__global__ void SITU_BWD_BOUNDS situ_glu_bwd_kernel(const BwdArgs a) {
   __shared__ float red[2][kMaxThreads / 32];
   const int nt = blockDim.x;
   int parity = 0;
+  if (PipelineRows<S, true>::value && a.vpr <= 2 * nt) {
+    // As in the forward: the CTA's next row is loaded while this one computes.
+    const int j = threadIdx.x, j2 = j + nt;
+    const bool one = j < a.vpr, two = j2 < a.vpr;
+    int64_t row = blockIdx.x;
+    if (row >= a.tokens) return;
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    uint4 g0 = z, u0 = z, o0 = z, g1 = z, u1 = z, o1 = z;
+    {
+      const char* gu = a.gate_up + row * a.gu_pitch;
+      const char* go_row = a.grad_out + row * a.go_pitch;
+      if (one) {
+        g0 = ld_stream(gu + j * kVecBytes);
+        u0 = ld_stream(gu + a.half_bytes + j * kVecBytes);
+        o0 = ld_stream(go_row + j * kVecBytes);
+      }
+      if (two) {
+        g1 = ld_stream(gu + j2 * kVecBytes);
+        u1 = ld_stream(gu + a.half_bytes + j2 * kVecBytes);
+        o1 = ld_stream(go_row + j2 * kVecBytes);
+      }
+    }
+    float w = load_rw(a.rw, row);
+    for (;;) {
+      const int64_t next = row + gridDim.x;
+      const bool more = next < a.tokens;
+      uint4 ng0 = z, nu0 = z, no0 = z, ng1 = z, nu1 = z, no1 = z;
+      float nw = 0.0f;
+      if (more) {
+        const char* gu = a.gate_up + next * a.gu_pitch;
+        const char* go_row = a.grad_out + next * a.go_pitch;
+        if (one) {
+          ng0 = ld_stream(gu + j * kVecBytes);
+          nu0 = ld_stream(gu + a.half_bytes + j * kVecBytes);
+          no0 = ld_stream(go_row + j * kVecBytes);
+        }
+        if (two) {
+          ng1 = ld_stream(gu + j2 * kVecBytes);
+          nu1 = ld_stream(gu + a.half_bytes + j2 * kVecBytes);
+          no1 = ld_stream(go_row + j2 * kVecBytes);
+        }
+        nw = load_rw(a.rw, next);
+      }
+      char* dgu = a.d_gate_up + row * a.dgu_pitch;
+      const float2 k = bwd_row_consts<HAS_LB>(w, a.c);
+      float2 acc = make_float2(0.0f, 0.0f);
+      uint4 dg, du;
+      if (one) {
+        bwd_vec<S, GATE, HAS_LB>(g0, u0, o0, k, a.c, dg, du, acc);
+        st_stream(dgu + j * kVecBytes, dg);
+        st_stream(dgu + a.half_bytes + j * kVecBytes, du);
+      }
+      if (two) {
+        bwd_vec<S, GATE, HAS_LB>(g1, u1, o1, k, a.c, dg, du, acc);
+        st_stream(dgu + j2 * kVecBytes, dg);
+        st_stream(dgu + a.half_bytes + j2 * kVecBytes, du);
+      }
+      if (a.want_drw) {  // uniform over the launch
+        const float total = block_sum(acc.x + acc.y, red[parity]) * bwd_dw_scale(a.c);
+        parity ^= 1;
+        if (threadIdx.x == 0) {
+          if (a.rw.mode == SITU_RW_SCALAR)
+            a.partials[row] = total;
+          else
+            store_rw_grad(a.d_rw, row * a.d_rw_stride, a.rw.bf16, total);
+        }
+      }
+      if (!more) break;
+      row = next;
+      g0 = ng0; u0 = nu0; o0 = no0; g1 = ng1; u1 = nu1; o1 = no1; w = nw;
+    }
+    return;
+  }
   for (int64_t row = blockIdx.x; row < a.tokens; row += gridDim.x) {
     const char* gu = a.gate_up + row * a.gu_pitch;
     const char* go_row = a.grad_out + row * a.go_pitch;
     char* dgu = a.d_gate_up + row * a.dgu_pitch;
-    const float w = load_rw(a.rw, row);
+    const float2 k = bwd_row_consts<HAS_LB>(load_rw(a.rw, row), a.c);
     float2 acc = make_float2(0.0f, 0.0f);
     for (int j = threadIdx.x; j < a.vpr; j += 2 * nt) {
       const int j2 = j + nt;
@@ -524,17 +703,17 @@ __global__ void __launch_bounds__(kMaxThreads) situ_glu_bwd_kernel(const BwdArgs
         o1 = ld_stream(go_row + j2 * kVecBytes);
       }
       uint4 dg, du;
-      bwd_vec<S, GATE, HAS_LB>(g0, u0, o0, w, a.c, dg, du, acc);
+      bwd_vec<S, GATE, HAS_LB>(g0, u0, o0, k, a.c, dg, du, acc);
       st_stream(dgu + j * kVecBytes, dg);
       st_stream(dgu + a.half_bytes + j * kVecBytes, du);
       if (two) {  // zero inputs contribute exactly 0 to acc, but skip them anyway
-        bwd_vec<S, GATE, HAS_LB>(g1, u1, o1, w, a.c, dg, du, acc);
+        bwd_vec<S, GATE, HAS_LB>(g1, u1, o1, k, a.c, dg, du, acc);
         st_stream(dgu + j2 * kVecBytes, dg);
         st_stream(dgu + a.half_bytes + j2 * kVecBytes, du);
       }
     }
     if (a.want_drw) {  // uniform over the launch
-      const float total = block_sum(acc.x + acc.y, red[parity]);
+      const float total = block_sum(acc.x + acc.y, red[parity]) * bwd_dw_scale(a.c);
       parity ^= 1;
       if (threadIdx.x == 0) {
         if (a.rw.mode == SITU_RW_SCALAR)
@@ -559,7 +738,7 @@ __global__ void __launch_bounds__(kFinalizeThreads)
 }
 
 // ---------------------------------------------------------------------------
-// TMA-staged kernels (the default path)
+// TMA-staged kernels (load path 1)
 // ---------------------------------------------------------------------------
 // Warp 0 of each CTA is a producer: one lane streams chunks of rows from HBM
 // into a ring of shared-memory stages with 1-D bulk copies (cp.async.bulk,
@@ -718,6 +897,7 @@ __device__ __forceinline__ void tma_stream_body(const StreamArgs& a) {
   for (int64_t row = blockIdx.x; row < a.tokens; row += gridDim.x) {
     const float w = load_rw(a.rw, row);
     const float2 wbb = splat(w * a.c.bb);
+    const float2 kc = bwd_row_consts<HAS_LB>(w, a.c);
     char* out = a.out + row * a.out_pitch;
     float2 acc = make_float2(0.0f, 0.0f);
     for (int ch = 0; ch < a.nchunks; ++ch, ++k) {
@@ -747,11 +927,11 @@ __device__ __forceinline__ void tma_stream_body(const StreamArgs& a) {
           const uint4 q0 = lds16(st + 2 * chunk_bytes + v * kVecBytes);
           const uint4 q1 = two ? lds16(st + 2 * chunk_bytes + v2 * kVecBytes) : make_uint4(0, 0, 0, 0);
           uint4 dg, du;
-          bwd_vec<S, GATE, HAS_LB>(g0, u0, q0, w, a.c, dg, du, acc);
+          bwd_vec<S, GATE, HAS_LB>(g0, u0, q0, kc, a.c, dg, du, acc);
           st_stream(o0, dg);
           st_stream(o0 + a.half_bytes, du);
           if (two) {
-            bwd_vec<S, GATE, HAS_LB>(g1, u1, q1, w, a.c, dg, du, acc);
+            bwd_vec<S, GATE, HAS_LB>(g1, u1, q1, kc, a.c, dg, du, acc);
             st_stream(o1, dg);
             st_stream(o1 + a.half_bytes, du);
           }
@@ -774,6 +954,7 @@ __device__ __forceinline__ void tma_stream_body(const StreamArgs& a) {
         float t = ctid < nc / 32 ? slot[ctid] : 0.0f;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        t *= bwd_dw_scale(a.c);
         if (ctid == 0 && ok) {
           if (a.rw.mode == SITU_RW_SCALAR)
             a.partials[row] = t;
@@ -930,7 +1111,7 @@ situ_status_t launch_grid(const void* kernel, int threads, int smem, int64_t tok
 
 situ_status_t check_launch(const char* what);
 
-std::atomic<int> g_load_path{0};  // 0: TMA ring (default), 1: direct vector loads
+std::atomic<int> g_load_path{0};  // 0: direct vector loads (default), 1: TMA ring
 
 // Ring geometry of the TMA-staged kernels for a half row of `vpr` vectors and
 // `inputs` streamed inputs (2 forward, 3 backward).
@@ -1109,7 +1290,7 @@ situ_status_t situ_glu_fwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
   a.c = c;
   if (rw_mode == SITU_RW_NONE) a.rw.bf16 = 0;
 
-  if (g_load_path.load(std::memory_order_relaxed) == 0) {
+  if (g_load_path.load(std::memory_order_relaxed) == 1) {
     StreamArgs sa{};
     sa.gate_up = a.gate_up;
     sa.gu_pitch = a.gu_pitch;
@@ -1229,7 +1410,7 @@ situ_status_t situ_glu_bwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
   a.c = c;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (g_load_path.load(std::memory_order_relaxed) == 0) {
+  if (g_load_path.load(std::memory_order_relaxed) == 1) {
     StreamArgs sa{};
     sa.gate_up = a.gate_up;
     sa.gu_pitch = a.gu_pitch;
