@@ -474,16 +474,15 @@ template <typename S, bool BWD>
 struct PipelineRows {
   static constexpr bool value = !BWD || std::is_same<S, Bf16>::value;
 };
-// Register budgets of the direct-load kernels: when set, the resident CTAs of
-// kMaxThreads threads that __launch_bounds__ must allow; unset leaves the
-// choice to the compiler.
-#ifdef SITU_FWD_MIN_CTAS
-#define SITU_FWD_BOUNDS __launch_bounds__(kMaxThreads, SITU_FWD_MIN_CTAS)
+// Register budgets of the direct-load kernels (registers per thread); unset
+// leaves the choice to the compiler.
+#ifdef SITU_FWD_MAXNREG
+#define SITU_FWD_BOUNDS __maxnreg__(SITU_FWD_MAXNREG)
 #else
 #define SITU_FWD_BOUNDS __launch_bounds__(kMaxThreads)
 #endif
-#ifdef SITU_BWD_MIN_CTAS
-#define SITU_BWD_BOUNDS __launch_bounds__(kMaxThreads, SITU_BWD_MIN_CTAS)
+#ifdef SITU_BWD_MAXNREG
+#define SITU_BWD_BOUNDS __maxnreg__(SITU_BWD_MAXNREG)
 #else
 #define SITU_BWD_BOUNDS __launch_bounds__(kMaxThreads)
 #endif
