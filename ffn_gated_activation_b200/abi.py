@@ -42,6 +42,8 @@ SIGNATURES = {
     "situ_glu_set_max_ctas": (_INT, [_INT]),
     "situ_glu_set_load_path": (_INT, [_INT]),
     "situ_glu_device_status": (_INT, [_INT]),
+    "situ_glu_bwd_no_alloc": (_INT, [_VP, _INT, _I64, _I64, _I64, _VP, _INT, _INT, _I64, _DBL, _INT, _DBL,
+                                     _VP, _I64, _VP, _I64, _VP, _I64, _VP]),
 }
 
 
@@ -101,6 +103,17 @@ def situ_glu_bwd(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype
                               rw_stride, beta, has_linear_beta, linear_beta, grad_out,
                               grad_out_row_stride, d_gate_up, d_gate_up_row_stride, d_rw, d_rw_stride,
                               workspace, workspace_bytes, stream)
+
+
+def situ_glu_bwd_no_alloc(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride,
+                          beta, has_linear_beta, linear_beta, grad_out, grad_out_row_stride, d_gate_up,
+                          d_gate_up_row_stride, d_rw, d_rw_stride, stream) -> int:
+    """situ_glu_bwd without caller scratch (the library's fixed scratch; see
+    include/situ_glu.h for its row limit and sharing rules)."""
+    return lib().situ_glu_bwd_no_alloc(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode,
+                                       rw_stride, beta, has_linear_beta, linear_beta, grad_out,
+                                       grad_out_row_stride, d_gate_up, d_gate_up_row_stride, d_rw, d_rw_stride,
+                                       stream)
 
 
 def situ_glu_bwd_workspace_bytes(tokens, rw_mode, want_drw) -> int:

@@ -1481,3 +1481,77 @@ int situ_glu_set_max_ctas(int max_ctas) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free backward
+// ---------------------------------------------------------------------------
+// Some callers cannot allocate device memory at the point where they run the
+// backward: engines that reserve all of HBM up front and hand their kernels
+// only the buffers they planned, or plain C callers with no CUDA allocator of
+// their own.  situ_glu_bwd needs caller-owned scratch in one mode (a routing
+// weight broadcast to every row: per-row partial sums, 4 bytes per row).  The
+// entry point below takes that scratch from a fixed array that lives in this
+// library instead, so its caller passes only inputs and outputs.
+
+namespace {
+
+constexpr int64_t kNoAllocMaxTokens = 262144;  // rows the fixed scratch can hold (1 MiB)
+
+}  // namespace
+
+// The fixed scratch: one copy on every GPU that loads this library, held
+// until the process exits.  In host code this name is only a stand-in for the
+// symbol; the device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocMaxTokens];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (with that device current) and cached.
+situ_status_t noalloc_scratch(void** addr) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
+  if (dev < 0 || dev >= kMaxDevices) return fail(SITU_ERR_UNSUPPORTED, "device %d beyond %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (err != cudaSuccess || p == nullptr)
+      return fail(SITU_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(err));
+    g_noalloc_addr[dev] = p;
+  }
+  *addr = g_noalloc_addr[dev];
+  return SITU_OK;
+}
+
+}  // namespace
+
+extern "C" situ_status_t situ_glu_bwd_no_alloc(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
+                                               int64_t inter, int64_t gate_up_row_stride, const void* rw,
+                                               situ_dtype_t rw_dtype, situ_rw_mode_t rw_mode, int64_t rw_stride,
+                                               double beta, int has_linear_beta, double linear_beta,
+                                               const void* grad_out, int64_t grad_out_row_stride, void* d_gate_up,
+                                               int64_t d_gate_up_row_stride, void* d_rw, int64_t d_rw_stride,
+                                               void* stream) {
+  tl_last_error[0] = '\0';
+  const size_t need = situ_glu_bwd_workspace_bytes(tokens, rw_mode, d_rw != nullptr ? 1 : 0);
+  void* ws = nullptr;
+  if (need > 0) {
+    if (tokens > kNoAllocMaxTokens)
+      return fail(SITU_ERR_UNSUPPORTED,
+                  "situ_glu_bwd_no_alloc: %lld rows need %zu bytes of scratch; its fixed scratch holds %lld rows",
+                  (long long)tokens, need, (long long)kNoAllocMaxTokens);
+    const situ_status_t st = noalloc_scratch(&ws);
+    if (st != SITU_OK) return st;
+  }
+  // Every step runs in situ_glu_bwd; the per-row partials it writes to the
+  // scratch are all written before the finishing kernel reads them, so no
+  // part of the array has to start at zero.
+  return situ_glu_bwd(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride, beta,
+                      has_linear_beta, linear_beta, grad_out, grad_out_row_stride, d_gate_up, d_gate_up_row_stride,
+                      d_rw, d_rw_stride, ws, need > 0 ? sizeof(g_noalloc_scratch) : 0, stream);
+}

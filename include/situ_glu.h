@@ -187,6 +187,39 @@ int situ_glu_set_load_path(int path);
  * reports an error. */
 int situ_glu_device_status(int clear);
 
+/*
+ * Backward without caller scratch.  Same arguments and results as
+ * situ_glu_bwd, minus `workspace` and `workspace_bytes`.  The pages describe
+ * no counterpart of this entry point: it exists for callers that cannot
+ * allocate device memory where they run the backward (an engine that
+ * reserves all of HBM at start-up and gives its kernels only planned
+ * buffers, or a C caller without a CUDA allocator), for the one mode that
+ * needs scratch: a routing weight broadcast to every row (SITU_RW_SCALAR with
+ * d_rw != NULL), whose per-row partial sums then go to a fixed 1 MiB array
+ * inside this library instead of a caller workspace.
+ *   - Limit: 262144 rows in that mode; more returns SITU_ERR_UNSUPPORTED
+ *     before anything is launched.  Other modes need no scratch and have no
+ *     row limit beyond situ_glu_bwd's.
+ *   - Allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ *     The array exists once per GPU that loads the library, until exit.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array, and it keeps whatever the last call
+ *     left in it (nothing in it has to start at zero).  Calls whose kernels
+ *     overlap on the GPU -- on different streams, or from different threads
+ *     -- race on it and give undefined results; serialise them.
+ */
+situ_status_t situ_glu_bwd_no_alloc(const void *gate_up, situ_dtype_t dtype, int64_t tokens,
+                                    int64_t inter, int64_t gate_up_row_stride,
+                                    const void *rw, situ_dtype_t rw_dtype, situ_rw_mode_t rw_mode,
+                                    int64_t rw_stride,
+                                    double beta, int has_linear_beta, double linear_beta,
+                                    const void *grad_out, int64_t grad_out_row_stride,
+                                    void *d_gate_up, int64_t d_gate_up_row_stride,
+                                    void *d_rw, int64_t d_rw_stride,
+                                    void *stream);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif
