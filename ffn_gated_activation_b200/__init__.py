@@ -8,7 +8,7 @@ over gate_up[..., 2I] = [G | U], with the fused analytic backward.  The work
 runs in the hand-written CUDA kernels of libsitu_glu.so behind the C ABI in
 include/situ_glu.h; this package only marshals torch tensors into it.
 """
-from . import abi
+from . import abi, distributed
 from .abi import NativeLibraryError, SituError
 from .functional import (
     DEFAULT_BETA,
@@ -22,6 +22,7 @@ from .functional import (
 
 __all__ = [
     "abi",
+    "distributed",
     "NativeLibraryError",
     "SituError",
     "DEFAULT_BETA",

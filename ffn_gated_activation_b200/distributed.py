@@ -1,0 +1,85 @@
+"""Multi-GPU plumbing for SiTU-GLU: one process per GPU over torch.distributed.
+
+Rows are independent (each output row depends on its own gate_up row, weight
+and grad_out row only), so:
+
+* Data parallelism shards rows -- contiguous blocks, ``shard_range`` -- and
+  needs no collective for row-aligned routing weights.
+* A routing weight broadcast to every row has one gradient for all rows: its
+  per-rank partials are summed across ranks (``allreduce_drw``).
+* Tensor parallelism of FC1 (column-parallel: rank r holds gate columns
+  [a_r, b_r) and the matching up columns, see ``tp_local_gate_up``) keeps the
+  forward and dG/dU local; only the routing-weight gradient, a sum over all I
+  columns, needs the sum of the ranks' partial sums over their columns: an
+  all-reduce of T values (``situ_glu_bwd_tp``).
+
+Nothing here computes the method; the kernels run in libsitu_glu.so.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import functional
+
+
+def shard_range(n: int, rank: int, world: int, align: int = 1) -> tuple[int, int]:
+    """Contiguous [start, stop) of ``n`` items for ``rank`` of ``world``: sizes
+    differ by at most ``align`` and every boundary is a multiple of ``align``
+    (except ``n`` itself)."""
+    if world <= 0 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} of world {world}")
+    if align <= 0:
+        raise ValueError("align must be positive")
+    units = -(-n // align)
+    base, extra = divmod(units, world)
+    start_u = rank * base + min(rank, extra)
+    stop_u = start_u + base + (1 if rank < extra else 0)
+    return min(n, start_u * align), min(n, stop_u * align)
+
+
+def vector_width(dtype: torch.dtype) -> int:
+    """Elements per 16-byte vector: the granularity a column shard keeps."""
+    return 16 // torch.empty((), dtype=dtype).element_size()
+
+
+def tp_local_gate_up(gate_up: torch.Tensor, rank: int, world: int) -> torch.Tensor:
+    """The [..., 2 * I_r] gate_up a column-parallel FC1 produces on ``rank``:
+    gate columns [a, b) followed by the same up columns [I + a, I + b)."""
+    inter = gate_up.shape[-1] // 2
+    a, b = shard_range(inter, rank, world, vector_width(gate_up.dtype))
+    return torch.cat([gate_up[..., a:b], gate_up[..., inter + a:inter + b]], dim=-1).contiguous()
+
+
+def tp_local_columns(x: torch.Tensor, rank: int, world: int) -> torch.Tensor:
+    """Columns [a, b) of an [..., I] tensor (grad_out or Y) held by ``rank``."""
+    a, b = shard_range(x.shape[-1], rank, world, vector_width(x.dtype))
+    return x[..., a:b].contiguous()
+
+
+def allreduce_drw(d_rw: torch.Tensor, group=None) -> torch.Tensor:
+    """Sum routing-weight gradient partials over ``group`` in place (NCCL for
+    CUDA tensors, gloo for CPU tensors)."""
+    dist.all_reduce(d_rw, op=dist.ReduceOp.SUM, group=group)
+    return d_rw
+
+
+def situ_glu_bwd_tp(gate_up_local, routing_weights, grad_out_local, beta=functional.DEFAULT_BETA,
+                    linear_beta=functional.DEFAULT_LINEAR_BETA, group=None, want_drw=True, **kw):
+    """Backward of a column-parallel shard: local d_gate_up [..., 2 I_r] and the
+    full routing-weight gradient (partials all-reduced over ``group``)."""
+    d_gate_up, d_rw = functional.situ_glu_bwd(gate_up_local, routing_weights, grad_out_local, beta,
+                                              linear_beta, want_drw=want_drw, **kw)
+    if d_rw is not None:
+        allreduce_drw(d_rw, group)
+    return d_gate_up, d_rw
+
+
+def max_over_ranks(value: float, device=None, group=None) -> float:
+    """Largest ``value`` over the ranks (timing: a step lasts as long as its
+    slowest rank).  Returns ``value`` when no process group is initialised."""
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(t.item())

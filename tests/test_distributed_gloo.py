@@ -1,0 +1,127 @@
+"""The N > 1 plumbing on CPU: world-size-2 gloo process groups.
+
+Each rank computes its share with the fp64 oracle (the CUDA kernels need a
+GPU); the tests check the product's sharding and reduction helpers:
+
+* tensor parallelism: column shards of gate_up / grad_out give local dG, dU
+  equal to the matching columns of the unsharded backward, and the
+  all-reduced per-rank routing-weight partials equal the full-width gradient;
+* data parallelism with a broadcast weight: row shards' partial sums,
+  all-reduced, equal the single-process gradient;
+* max-over-ranks timing and the shard arithmetic.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from ffn_gated_activation_b200 import distributed as D
+
+WORLD = 2
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _run(fn, *args):
+    port = _free_port()
+    mp.spawn(_entry, args=(fn, port, args), nprocs=WORLD, join=True)
+
+
+def _entry(rank, fn, port, args):
+    import datetime
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    for p in (root, os.path.join(root, "tests")):
+        if p not in sys.path:
+            sys.path.insert(0, p)
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=WORLD,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        fn(rank, *args)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def _bf16_tensor(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _tp_check(rank, T, I, seed):
+    import oracle
+    import workloads
+    import dataclasses
+    wl = dataclasses.replace(workloads.workload(2), tokens=T, inter=I, seed=seed, rw_kind="uniform")
+    x = workloads.inputs(wl)
+    o = oracle.load()
+    full = o.bwd(x["gate_up"], x["routing_weights"], x["grad_out"], 4.0, 25.0)
+    gu_local = _bits(D.tp_local_gate_up(_bf16_tensor(x["gate_up"]), rank, WORLD))
+    go_local = _bits(D.tp_local_columns(_bf16_tensor(x["grad_out"]), rank, WORLD))
+    a, b = D.shard_range(I, rank, WORLD, align=8)
+    assert gu_local.shape == (T, 2 * (b - a))
+    loc = o.bwd(gu_local, x["routing_weights"], go_local, 4.0, 25.0)
+    # dG and dU need no exchange: they are the matching columns of the full result
+    assert np.array_equal(loc.dg, full.dg[:, a:b]) and np.array_equal(loc.du, full.du[:, a:b])
+    # the routing-weight gradient is the sum of the ranks' column partials
+    d_rw = torch.tensor(loc.dw, dtype=torch.float64)
+    D.allreduce_drw(d_rw)
+    np.testing.assert_allclose(d_rw.numpy(), full.dw, rtol=1e-12, atol=1e-12 * full.sw.max())
+
+
+def _dp_scalar_check(rank, T, I, seed):
+    import oracle
+    import workloads
+    import dataclasses
+    wl = dataclasses.replace(workloads.workload(0), tokens=T, inter=I, seed=seed)
+    x = workloads.inputs(wl)
+    o = oracle.load()
+    total, mag = o.dw_scalar(x["gate_up"], x["grad_out"], 4.0, 25.0)
+    r0, r1 = D.shard_range(T, rank, WORLD)
+    part, _ = o.dw_scalar(x["gate_up"][r0:r1], x["grad_out"][r0:r1], 4.0, 25.0)
+    t = torch.tensor([part], dtype=torch.float64)
+    D.allreduce_drw(t)
+    assert abs(t.item() - total) <= 1e-12 * mag
+
+
+def _max_check(rank):
+    assert D.max_over_ranks(1.5 + rank) == 2.5
+
+
+def test_tensor_parallel_backward_gloo():
+    _run(_tp_check, 37, 520, 11)
+
+
+def test_data_parallel_broadcast_weight_gloo():
+    _run(_dp_scalar_check, 61, 64, 12)
+
+
+def test_max_over_ranks_gloo():
+    _run(_max_check)
+
+
+@pytest.mark.parametrize("n,world,align", [(10, 3, 1), (520, 2, 8), (7, 4, 1), (4096, 8, 8), (3, 5, 1), (0, 2, 8)])
+def test_shard_range_partitions(n, world, align):
+    spans = [D.shard_range(n, r, world, align) for r in range(world)]
+    assert spans[0][0] == 0 and spans[-1][1] == n
+    for (a0, b0), (a1, b1) in zip(spans, spans[1:]):
+        assert b0 == a1
+    for a, b in spans:
+        assert a <= b and a % align == 0
+    sizes = [b - a for a, b in spans]
+    assert max(sizes) - min(sizes) <= align
+
+
+def test_max_over_ranks_without_group():
+    assert D.max_over_ranks(3.25) == 3.25
