@@ -38,6 +38,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <initializer_list>
 #include <type_traits>
 
 #include "situ_glu.h"
@@ -94,6 +95,26 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
 __device__ __forceinline__ void st_stream(void* p, const uint4& v) {
   asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
                "r"(v.w)
+               : "memory");
+}
+
+// 32-byte forms (sm_100): two adjacent 16-byte vectors in one instruction.
+// The address must be 32-byte aligned.
+struct U8 {
+  uint4 a, b;
+};
+
+__device__ __forceinline__ U8 ld_stream32(const void* p) {
+  U8 r;
+  asm("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r.a.x), "=r"(r.a.y), "=r"(r.a.z), "=r"(r.a.w), "=r"(r.b.x), "=r"(r.b.y), "=r"(r.b.z), "=r"(r.b.w)
+      : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void st_stream32(void* p, const uint4& a, const uint4& b) {
+  asm volatile("st.global.cs.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a.x), "r"(a.y),
+               "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
                : "memory");
 }
 
@@ -355,7 +376,7 @@ __device__ __forceinline__ float2 fwd_pair_abs(Bits2 gb, Bits2 ub, float2 wbb, c
 // Backward of a pair.  With A = (1 + E_t)(1 + E_s), B = 1 + E_u (1 without a
 // linear beta), sig as above and
 //   tq  = (beta/4) tanh(g/beta) (1 + E_t)              (= (beta/4) s_g (1 - E_t))
-//   T_g  = 4 tq sig / A
+//   T_g  = 4 tq sig / A  (tgA = tq sig A = T_g A^2 / 4)
 //   T_g' = 4 [E_t sig (1 + E_s) + tq (1 + E_t) E_s] / A^2
 //          (the sech^2(g/beta) sigmoid and beta tanh sigmoid (1 - sigmoid) terms)
 //   T_u  = beta_L su / B,  su = s_u (1 - E_u),   T_u' = 4 E_u / B^2
@@ -373,25 +394,26 @@ __device__ __forceinline__ void bwd_pair(Bits2 gb, Bits2 ub, float2 go, float2 k
   const float2 A = mul2(opt, ops);
   float2 tq = xor_sign2(e.emt, gb);
   if (GATE != kGateSquare) tq = mul2(tq, splat(0.25f * c.beta));  // beta = 4: the factor is 1
-  const float2 tg = mul2(tq, sig);                                  // T_g A / 4
+  const float2 tgA = mul2(mul2(tq, sig), A);                       // T_g A^2 / 4
   const float2 ng = fma2(mul2(e.Et, sig), ops, mul2(mul2(tq, opt), e.Es));  // T_g' A^2 / 4
-  const float2 gtg = mul2(go, tg);
   if (HAS_LB) {
     float2 Eu;
     const float2 su = xor_sign2(up_emu<S, typename UpSeries<S>::type>(ub, c, Eu), ub);  // T_u B / beta_L
     const float2 B = add2(splat(1.0f), Eu);
     const float2 AB = mul2(A, B);
-    const float2 R = rcp2(mul2(AB, AB));
-    dg = mul2(mul2(go, mul2(su, kdg)), mul2(ng, mul2(B, R)));  // go w T_u T_g'
-    du = mul2(mul2(gtg, mul2(Eu, kdu)), mul2(A, R));           // go w T_g T_u'
-    acc = fma2(gtg, mul2(su, mul2(AB, R)), acc);                // go T_g T_u / (4 beta_L)
+    const float2 gR = mul2(go, rcp2(mul2(AB, AB)));  // go / (A B)^2
+    const float2 sB = mul2(su, B);
+    const float2 gRt = mul2(gR, tgA);
+    dg = mul2(mul2(gR, kdg), mul2(sB, ng));  // go w T_u T_g'
+    du = mul2(gRt, mul2(Eu, kdu));           // go w T_g T_u'
+    acc = fma2(gRt, sB, acc);                // go T_g T_u / (4 beta_L)
   } else {
     const float2 u = as_f2(ub);
-    const float2 R = rcp2(mul2(A, A));
-    const float2 AR = mul2(A, R);
-    dg = mul2(mul2(go, mul2(u, kdg)), mul2(ng, R));
-    du = mul2(mul2(gtg, kdu), AR);
-    acc = fma2(gtg, mul2(u, AR), acc);
+    const float2 gR = mul2(go, rcp2(mul2(A, A)));  // go / A^2
+    const float2 gRt = mul2(gR, tgA);
+    dg = mul2(mul2(gR, kdg), mul2(u, ng));
+    du = mul2(gRt, kdu);
+    acc = fma2(gRt, u, acc);
   }
 }
 
@@ -513,7 +535,7 @@ __global__ void SITU_FWD_BOUNDS situ_glu_fwd_kernel(const FwdArgs a) {
     for (;;) {
       const int64_t next = row + gridDim.x;
       const bool more = next < a.tokens;
-      uint4 ng0 = z, nu0 = z, ng1 = z, nu1 = z;
+      uint4 ng0, nu0, ng1, nu1;  // only the lanes' own vectors are loaded and used
       float nw = 0.0f;
       if (more) {
         const char* ngu = a.gate_up + next * a.gu_pitch;
@@ -636,7 +658,7 @@ __global__ void SITU_BWD_BOUNDS situ_glu_bwd_kernel(const BwdArgs a) {
     for (;;) {
       const int64_t next = row + gridDim.x;
       const bool more = next < a.tokens;
-      uint4 ng0 = z, nu0 = z, no0 = z, ng1 = z, nu1 = z, no1 = z;
+      uint4 ng0, nu0, no0, ng1, nu1, no1;  // only the lanes' own vectors are loaded and used
       float nw = 0.0f;
       if (more) {
         const char* gu = a.gate_up + next * a.gu_pitch;
@@ -734,6 +756,47 @@ __global__ void __launch_bounds__(kFinalizeThreads)
   for (int64_t r = threadIdx.x; r < tokens; r += blockDim.x) s += partials[r];
   const float total = block_sum(s, red);
   if (threadIdx.x == 0) store_rw_grad(d_rw, 0, bf16, total);
+}
+
+// ---------------------------------------------------------------------------
+// Wide direct-load forward (the default whenever the layout allows)
+// ---------------------------------------------------------------------------
+// When a half row holds 64 k 16-byte vectors (k = 1..8) and every base and row
+// pitch is 32-byte aligned, CTA thread t owns the 32 contiguous bytes at 32 t
+// of each half row: one 256-bit load per input and one 256-bit store per
+// output, no lane without work, and half the address arithmetic of the
+// two-vector layout.  Rows are software-pipelined as in the kernels above.
+// (The same layout measured slower for the backward, whose next-row loads it
+// did not keep in flight; the backward keeps the two-vector layout.)
+
+template <typename S, int GATE, bool HAS_LB>
+__global__ void __launch_bounds__(kMaxThreads) situ_glu_fwd_wide_kernel(const FwdArgs a) {
+  const int off = threadIdx.x * 32;
+  int64_t row = blockIdx.x;
+  if (row >= a.tokens) return;
+  const char* gu = a.gate_up + row * a.gu_pitch + off;
+  U8 g = ld_stream32(gu), u = ld_stream32(gu + a.half_bytes);
+  float w = load_rw(a.rw, row);
+  for (;;) {
+    const int64_t next = row + gridDim.x;
+    const bool more = next < a.tokens;
+    U8 ng, nu;
+    float nw = 0.0f;
+    if (more) {
+      const char* ngu = a.gate_up + next * a.gu_pitch + off;
+      ng = ld_stream32(ngu);
+      nu = ld_stream32(ngu + a.half_bytes);
+      nw = load_rw(a.rw, next);
+    }
+    const float2 wbb = splat(w * a.c.bb);
+    st_stream32(a.out + row * a.out_pitch + off, fwd_vec<S, GATE, HAS_LB>(g.a, u.a, wbb, a.c),
+                fwd_vec<S, GATE, HAS_LB>(g.b, u.b, wbb, a.c));
+    if (!more) break;
+    row = next;
+    g = ng;
+    u = nu;
+    w = nw;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -1219,6 +1282,34 @@ FwdKernel pick_fwd_gate(int gate) {
   }
 }
 
+template <typename S, bool LB>
+FwdKernel pick_fwd_wide_gate(int gate) {
+  switch (gate) {
+    case kGateSquare: return situ_glu_fwd_wide_kernel<S, kGateSquare, LB>;
+    case kGateEqual: return situ_glu_fwd_wide_kernel<S, kGateEqual, LB>;
+    case kGateRoot: return situ_glu_fwd_wide_kernel<S, kGateRoot, LB>;
+    default: return situ_glu_fwd_wide_kernel<S, kGateGeneric, LB>;
+  }
+}
+
+FwdKernel pick_fwd_wide(situ_dtype_t dtype, int gate, bool lb) {
+  if (dtype == SITU_DTYPE_BF16)
+    return lb ? pick_fwd_wide_gate<Bf16, true>(gate) : pick_fwd_wide_gate<Bf16, false>(gate);
+  return lb ? pick_fwd_wide_gate<F32, true>(gate) : pick_fwd_wide_gate<F32, false>(gate);
+}
+
+// The wide layout applies when a half row is 64 k vectors (k = 1..8: one
+// 32-byte chunk per thread, at most kMaxThreads threads) and every listed
+// base address and row pitch (bytes) is a multiple of 32.
+bool wide_layout(int vpr, std::initializer_list<const void*> bases, std::initializer_list<int64_t> pitches) {
+  if (vpr % 64 != 0 || vpr / 2 > kMaxThreads) return false;
+  for (const void* b : bases)
+    if (!aligned(b, 32)) return false;
+  for (int64_t p : pitches)
+    if (p % 32 != 0) return false;
+  return true;
+}
+
 FwdKernel pick_fwd(situ_dtype_t dtype, int gate, bool lb) {
   if (dtype == SITU_DTYPE_BF16) return lb ? pick_fwd_gate<Bf16, true>(gate) : pick_fwd_gate<Bf16, false>(gate);
   return lb ? pick_fwd_gate<F32, true>(gate) : pick_fwd_gate<F32, false>(gate);
@@ -1302,8 +1393,9 @@ situ_status_t situ_glu_fwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
     sa.c = c;
     return launch_stream<false>(sa, dtype, gate, has_linear_beta != 0, static_cast<cudaStream_t>(stream));
   }
-  FwdKernel k = pick_fwd(dtype, gate, has_linear_beta != 0);
-  const int threads = choose_threads(a.vpr);
+  const bool wide = wide_layout(a.vpr, {gate_up, out}, {a.gu_pitch, a.out_pitch});
+  FwdKernel k = wide ? pick_fwd_wide(dtype, gate, has_linear_beta != 0) : pick_fwd(dtype, gate, has_linear_beta != 0);
+  const int threads = wide ? a.vpr / 2 : choose_threads(a.vpr);
   int grid = 0;
   st = launch_grid(reinterpret_cast<const void*>(k), threads, 0, tokens, &grid);
   if (st != SITU_OK) return st;

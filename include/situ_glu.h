@@ -135,8 +135,9 @@ situ_status_t situ_glu_fwd(const void *gate_up, situ_dtype_t dtype, int64_t toke
  *                      entry and undefined on exit.  May be NULL when that
  *                      query returns 0.
  * Other arguments as for situ_glu_fwd.  Per-row reductions run in a fixed
- * order, so every output is bitwise reproducible for a given build and shape,
- * whatever the launch size.
+ * order, so every output is bitwise reproducible for a given build, shape and
+ * load path, whatever the launch size.  dG and dU do not depend on the load
+ * path either; d_rw's summation order does, within its rounding.
  */
 situ_status_t situ_glu_bwd(const void *gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
                            int64_t gate_up_row_stride,

@@ -304,11 +304,23 @@ def test_errors_surface_from_the_library(cuda_device):
         pkg.situ_glu_fwd(torch.zeros(4, 32, dtype=torch.bfloat16, device=dev), None, beta=0.0)
 
 
+def assert_same_results(first, second):
+    """[Y, d_gate_up, d_w] of two launch layouts.  Y and d_gate_up are computed
+    element by element with the same arithmetic: bitwise equal.  d_w sums each
+    row in an order fixed by how the layout assigns vectors to threads, so two
+    layouts agree within its tolerance (the order is fixed per layout, which the
+    grid-invariance test checks bitwise)."""
+    for a, b in zip(first[:2], second[:2]):
+        assert np.array_equal(a.view(np.uint8), b.view(np.uint8))
+    da, db = first[2].astype(np.float64), second[2].astype(np.float64)
+    assert np.all(np.abs(da - db) <= parity.DW_REL * np.abs(db) + 1e-6 * np.abs(db).max())
+
+
 @pytest.mark.parametrize("dtype,T,I,lb", [("bf16", 257, 520, 25.0), ("bf16", 64, 3072, None),
                                           ("f32", 33, 4096, 25.0), ("bf16", 5, 8, 25.0)])
-def test_load_paths_bitwise_identical(dtype, T, I, lb, cuda_device):
+def test_load_paths_agree(dtype, T, I, lb, cuda_device):
     """The shared-memory ring (TMA bulk copies) and the direct-load path run the
-    same arithmetic: every output must match bit for bit."""
+    same arithmetic (see assert_same_results)."""
     dev = cuda_device
     gu_h, rw32, go_h = case_inputs(dtype, T, I, seed=31)
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
@@ -328,8 +340,36 @@ def test_load_paths_bitwise_identical(dtype, T, I, lb, cuda_device):
             results.append([to_host(out.view), to_host(dgu.view), to_host(d_rw)])
     finally:
         abi.situ_glu_set_load_path(prev)
-    for a, b in zip(*results):
-        assert np.array_equal(a.view(np.uint8), b.view(np.uint8))
+    assert_same_results(*results)
+
+
+@pytest.mark.parametrize("dtype,T,I", [("bf16", 150, 2048), ("bf16", 33, 512), ("f32", 70, 1024)])
+def test_wide_and_two_vector_layouts_agree(dtype, T, I, cuda_device):
+    """Row pitches that are multiples of 32 bytes take the 256-bit-per-thread
+    kernels; pitches that are only 16-byte multiples take the two-vector ones.
+    Same data, same arithmetic (see assert_same_results)."""
+    dev = cuda_device
+    gu_h, rw32, go_h = case_inputs(dtype, T, I, seed=41)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    es = 2 if dtype == "bf16" else 4
+    pad16 = 16 // es  # one extra 16-byte vector per row: pitch no longer a 32-byte multiple
+    results = []
+    for pad in (0, pad16):
+        gpitch, opitch = 2 * I + pad, I + pad
+        gu_p = np.zeros((T, gpitch), dtype=gu_h.dtype); gu_p[:, :2 * I] = gu_h
+        go_p = np.zeros((T, opitch), dtype=go_h.dtype); go_p[:, :I] = go_h
+        gu, go, rw = to_device(gu_p, dev), to_device(go_p, dev), to_device(rw32, dev)
+        out = Guarded(T, I, opitch, tdt, dev)
+        dgu = Guarded(T, 2 * I, gpitch, tdt, dev)
+        d_rw = torch.empty(T, dtype=torch.float32, device=dev)
+        abi.check(call_fwd(gu, I, rw, abi.SITU_RW_ROW, 4.0, 25.0, out), "fwd")
+        abi.check(call_bwd(gu, I, rw, abi.SITU_RW_ROW, 4.0, 25.0, go, dgu, d_rw=d_rw), "bwd")
+        torch.cuda.synchronize()
+        out.check(); dgu.check()
+        results.append([to_host(out.view), to_host(dgu.view), to_host(d_rw)])
+    assert_same_results(*results)
+    o = oracle.load()
+    check_output("Y", results[0][0], o.fwd(gu_h, rw32, 4.0, 25.0))
 
 
 def test_no_bounded_wait_expired(cuda_device):
