@@ -35,8 +35,10 @@ LIBRARY = os.path.join(_HERE, "libsitu_oracle.so")
 
 DTYPE_BF16 = 0
 DTYPE_F32 = 1
-RW_ROW = 0
-RW_SCALAR = 1
+RW_ROW = 0     # w[T] (or [T, 1]): one weight per row
+RW_SCALAR = 1  # one weight for every element
+RW_COL = 2     # w[I]: one weight per column, every row
+RW_FULL = 3    # w[T, I]: one weight per element
 
 # gcc flags: plain IEEE double, no fast-math, no contraction into FMA, so the
 # arithmetic is exactly what the C source spells out.
@@ -107,6 +109,10 @@ class Oracle:
         lib.situ_oracle_dw_scalar.argtypes = [_INT, _VP, _I64, _I64, _I64, _DBL, _INT, _DBL, _VP, _I64,
                                               ctypes.POINTER(_DBL), ctypes.POINTER(_DBL)]
         lib.situ_oracle_dw_scalar.restype = _INT
+        lib.situ_oracle_dw_columns.argtypes = [_INT, _VP, _I64, _I64, _I64, _DBL, _INT, _DBL, _VP, _I64, _VP, _VP]
+        lib.situ_oracle_dw_columns.restype = _INT
+        lib.situ_oracle_dw_terms.argtypes = [_INT, _VP, _I64, _I64, _VP, _I64, _DBL, _INT, _DBL, _VP, _I64, _VP]
+        lib.situ_oracle_dw_terms.restype = _INT
         lib.situ_oracle_mutant_id.restype = _INT
         self._lib = lib
         self.mutant_id = lib.situ_oracle_mutant_id()
@@ -146,10 +152,11 @@ class Oracle:
         inter = width // 2 if inter is None else int(inter)
         r, n = self._rows(rows, T)
         rw_c = np.ascontiguousarray(rw).reshape(-1)
+        rw_stride = inter if rw_mode == RW_FULL else 1
         y = np.empty((n, inter), dtype=np.float64)
         has = linear_beta is not None
         rc = self._lib.situ_oracle_fwd(_dtype_code(gate_up), _ptr(gate_up), width, inter, _ptr(r), n,
-                                       _dtype_code(rw_c), _ptr(rw_c), int(rw_mode), 1,
+                                       _dtype_code(rw_c), _ptr(rw_c), int(rw_mode), rw_stride,
                                        float(beta), int(has), float(linear_beta if has else 0.0), _ptr(y))
         if rc != 0:
             raise ValueError("oracle fwd rejected its arguments")
@@ -166,17 +173,49 @@ class Oracle:
         inter = width // 2 if inter is None else int(inter)
         r, n = self._rows(rows, T)
         rw_c = np.ascontiguousarray(rw).reshape(-1)
+        rw_stride = inter if rw_mode == RW_FULL else 1
         dg = np.empty((n, inter)); du = np.empty((n, inter)); cg = np.empty((n, inter))
         dw = np.empty(n); sw = np.empty(n)
         has = linear_beta is not None
         rc = self._lib.situ_oracle_bwd(_dtype_code(gate_up), _ptr(gate_up), width, inter, _ptr(r), n,
-                                       _dtype_code(rw_c), _ptr(rw_c), int(rw_mode), 1,
+                                       _dtype_code(rw_c), _ptr(rw_c), int(rw_mode), rw_stride,
                                        float(beta), int(has), float(linear_beta if has else 0.0),
                                        _ptr(grad_out), grad_out.shape[1],
                                        _ptr(dg), _ptr(du), _ptr(dw), _ptr(cg), _ptr(sw))
         if rc != 0:
             raise ValueError("oracle bwd rejected its arguments")
         return BackwardResult(dg=dg, du=du, dw=dw, cg=cg, sw=sw)
+
+    def dw_columns(self, gate_up, grad_out, beta, linear_beta=None, inter=None):
+        """Gradient of a per-column weight w[I]: (sums over rows [I], sums of |terms| [I])."""
+        gate_up = np.ascontiguousarray(gate_up)
+        grad_out = np.ascontiguousarray(grad_out)
+        T, width = gate_up.shape
+        inter = width // 2 if inter is None else int(inter)
+        colsum, colmag = np.empty(inter), np.empty(inter)
+        has = linear_beta is not None
+        rc = self._lib.situ_oracle_dw_columns(_dtype_code(gate_up), _ptr(gate_up), width, inter, T,
+                                              float(beta), int(has), float(linear_beta if has else 0.0),
+                                              _ptr(grad_out), grad_out.shape[1], _ptr(colsum), _ptr(colmag))
+        if rc != 0:
+            raise ValueError("oracle dw_columns rejected its arguments")
+        return colsum, colmag
+
+    def dw_terms(self, gate_up, grad_out, beta, linear_beta=None, rows=None, inter=None):
+        """Gradient of a full [T, I] weight for the selected rows: go T_g T_u, float64."""
+        gate_up = np.ascontiguousarray(gate_up)
+        grad_out = np.ascontiguousarray(grad_out)
+        T, width = gate_up.shape
+        inter = width // 2 if inter is None else int(inter)
+        r, n = self._rows(rows, T)
+        terms = np.empty((n, inter))
+        has = linear_beta is not None
+        rc = self._lib.situ_oracle_dw_terms(_dtype_code(gate_up), _ptr(gate_up), width, inter, _ptr(r), n,
+                                            float(beta), int(has), float(linear_beta if has else 0.0),
+                                            _ptr(grad_out), grad_out.shape[1], _ptr(terms))
+        if rc != 0:
+            raise ValueError("oracle dw_terms rejected its arguments")
+        return terms
 
     def dw_scalar(self, gate_up, grad_out, beta, linear_beta=None, inter=None):
         """Gradient of one routing weight broadcast to all rows: (total, sum of |terms|)."""

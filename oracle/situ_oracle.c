@@ -42,8 +42,10 @@
 
 #define ORACLE_DTYPE_BF16 0
 #define ORACLE_DTYPE_F32 1
-#define ORACLE_RW_ROW 0
-#define ORACLE_RW_SCALAR 1
+#define ORACLE_RW_ROW 0    /* w[row * stride]              ([T, 1])   */
+#define ORACLE_RW_SCALAR 1 /* w[0] on every row            (one value) */
+#define ORACLE_RW_COL 2    /* w[col * stride] on every row ([I])       */
+#define ORACLE_RW_FULL 3   /* w[row * stride + col]        ([T, I])    */
 
 /* ---- exact input conversion ------------------------------------------ */
 
@@ -138,9 +140,21 @@ void situ_oracle_up(double u, int has_linear_beta, double linear_beta, double *t
 
 static int64_t row_index(const int64_t *rows, int64_t k) { return rows ? rows[k] : k; }
 
-static double routing_weight(int rw_dtype, const void *rw, int rw_mode, int64_t rw_stride, int64_t row) {
-  if (rw_mode == ORACLE_RW_SCALAR) return load_value(rw, rw_dtype, 0);
-  return load_value(rw, rw_dtype, row * rw_stride);
+/* Routing weight of element (row, col): the weight tensor broadcast against
+ * the [T, I] output (NeMo `_WeightedSiTUFunction.forward`, parameter
+ * routing_weights: row-aligned [..., 1] or broadcastable). */
+static double routing_weight(int rw_dtype, const void *rw, int rw_mode, int64_t rw_stride, int64_t row,
+                             int64_t col) {
+  switch (rw_mode) {
+    case ORACLE_RW_SCALAR: return load_value(rw, rw_dtype, 0);
+#if SITU_ORACLE_MUTANT == 13
+    case ORACLE_RW_COL: return load_value(rw, rw_dtype, row * rw_stride); /* planted: row for column */
+#else
+    case ORACLE_RW_COL: return load_value(rw, rw_dtype, col * rw_stride);
+#endif
+    case ORACLE_RW_FULL: return load_value(rw, rw_dtype, row * rw_stride + col);
+    default: return load_value(rw, rw_dtype, row * rw_stride);
+  }
 }
 
 /* Gate is the first half of a gate_up row, up the second half
@@ -190,9 +204,9 @@ int situ_oracle_fwd(int dtype, const void *gate_up, int64_t gu_stride, int64_t i
   if (!gate_up || !rw || !y || inter <= 0 || nrows < 0 || gu_stride < 2 * inter) return -1;
   for (int64_t k = 0; k < nrows; ++k) {
     int64_t r = row_index(rows, k);
-    double w = routing_weight(rw_dtype, rw, rw_mode, rw_stride, r);
     for (int64_t i = 0; i < inter; ++i) {
       double g, u, t_g, t_u;
+      double w = routing_weight(rw_dtype, rw, rw_mode, rw_stride, r, i);
       load_pair(dtype, gate_up, gu_stride, inter, r, i, &g, &u);
       situ_oracle_gate(g, beta, &t_g, NULL, NULL);
       situ_oracle_up(u, has_linear_beta, linear_beta, &t_u, NULL);
@@ -230,11 +244,11 @@ int situ_oracle_bwd(int dtype, const void *gate_up, int64_t gu_stride, int64_t i
     return -1;
   for (int64_t k = 0; k < nrows; ++k) {
     int64_t r = row_index(rows, k);
-    double w = routing_weight(rw_dtype, rw, rw_mode, rw_stride, r);
     neumaier_t red = {0.0, 0.0};
     neumaier_t mag = {0.0, 0.0};
     for (int64_t i = 0; i < inter; ++i) {
       double g, u, t_g, dt_g, dt_g_mag, t_u, dt_u;
+      double w = routing_weight(rw_dtype, rw, rw_mode, rw_stride, r, i);
       load_pair(dtype, gate_up, gu_stride, inter, r, i, &g, &u);
       double go = load_value(grad_out, dtype, r * go_stride + i);
       situ_oracle_gate(g, beta, &t_g, &dt_g, &dt_g_mag);
@@ -262,6 +276,56 @@ int situ_oracle_bwd(int dtype, const void *gate_up, int64_t gu_stride, int64_t i
     }
     if (dw) dw[k] = neumaier_value(&red);
     if (sw) sw[k] = neumaier_value(&mag);
+  }
+  return 0;
+}
+
+/* Gradient of a per-column routing weight w[i] (shape [I], broadcast over
+ * the rows): d w[i] = sum over rows r of go * T_g * T_u, for every column,
+ * each in one compensated sum; mag[i] receives the sum of absolute terms
+ * (may be NULL).  For a full [T, I] weight the gradient is the term
+ * go * T_g * T_u itself, element by element: situ_oracle_bwd's per-row sums
+ * are those terms summed over each row. */
+int situ_oracle_dw_columns(int dtype, const void *gate_up, int64_t gu_stride, int64_t inter, int64_t tokens,
+                           double beta, int has_linear_beta, double linear_beta, const void *grad_out,
+                           int64_t go_stride, double *colsum, double *colmag) {
+  if (!gate_up || !grad_out || !colsum || inter <= 0 || tokens < 0 || gu_stride < 2 * inter || go_stride < inter)
+    return -1;
+  for (int64_t i = 0; i < inter; ++i) {
+    neumaier_t red = {0.0, 0.0};
+    neumaier_t mag = {0.0, 0.0};
+    for (int64_t r = 0; r < tokens; ++r) {
+      double g, u, t_g, t_u;
+      load_pair(dtype, gate_up, gu_stride, inter, r, i, &g, &u);
+      double go = load_value(grad_out, dtype, r * go_stride + i);
+      situ_oracle_gate(g, beta, &t_g, NULL, NULL);
+      situ_oracle_up(u, has_linear_beta, linear_beta, &t_u, NULL);
+      neumaier_add(&red, go * t_g * t_u);
+      neumaier_add(&mag, fabs(go * t_g * t_u));
+    }
+    colsum[i] = neumaier_value(&red);
+    if (colmag) colmag[i] = neumaier_value(&mag);
+  }
+  return 0;
+}
+
+/* The weight-gradient terms go * T_g * T_u of each selected row, packed
+ * [nrows, inter]: the gradient of a full [T, I] routing weight. */
+int situ_oracle_dw_terms(int dtype, const void *gate_up, int64_t gu_stride, int64_t inter, const int64_t *rows,
+                         int64_t nrows, double beta, int has_linear_beta, double linear_beta, const void *grad_out,
+                         int64_t go_stride, double *terms) {
+  if (!gate_up || !grad_out || !terms || inter <= 0 || nrows < 0 || gu_stride < 2 * inter || go_stride < inter)
+    return -1;
+  for (int64_t k = 0; k < nrows; ++k) {
+    int64_t r = row_index(rows, k);
+    for (int64_t i = 0; i < inter; ++i) {
+      double g, u, t_g, t_u;
+      load_pair(dtype, gate_up, gu_stride, inter, r, i, &g, &u);
+      double go = load_value(grad_out, dtype, r * go_stride + i);
+      situ_oracle_gate(g, beta, &t_g, NULL, NULL);
+      situ_oracle_up(u, has_linear_beta, linear_beta, &t_u, NULL);
+      terms[k * inter + i] = go * t_g * t_u;
+    }
   }
   return 0;
 }

@@ -225,6 +225,41 @@ def pin_torch_autograd_rows(o):
                     np.testing.assert_allclose(b.dw, dW, rtol=1e-12, atol=1e-13 * b.sw.max())
 
 
+def pin_elementwise_weights(o):
+    """Per-column [I] and per-element [T, I] routing weights against float64
+    autograd of the formula: Y, dG, dU and the weight gradients (column sums
+    over rows for [I]; the elementwise terms for [T, I])."""
+    rng = np.random.default_rng(RNG_SEED + 8)
+    T, I = 6, 24
+    for dtype in ("bf16", "f32"):
+        raw = rng.normal(0, 3, (T, 2 * I)).astype(np.float32)
+        raw_go = rng.normal(0, 1, (T, I)).astype(np.float32)
+        if dtype == "bf16":
+            gu, go = workloads.f32_to_bf16_bits(raw), workloads.f32_to_bf16_bits(raw_go)
+        else:
+            gu, go = raw, raw_go
+        for mode, shape in ((oracle.RW_COL, (I,)), (oracle.RW_FULL, (T, I))):
+            w = rng.uniform(-1.0, 1.0, shape).astype(np.float32)
+            G = torch.tensor(_as_f64(gu)[:, :I], requires_grad=True)
+            U = torch.tensor(_as_f64(gu)[:, I:], requires_grad=True)
+            W = torch.tensor(w.astype(np.float64), requires_grad=True)
+            Y = 4.0 * torch.tanh(G / 4.0) * torch.sigmoid(G) * 25.0 * torch.tanh(U / 25.0) * W
+            (Y * torch.tensor(_as_f64(go))).sum().backward()
+            y = o.fwd(gu, w, 4.0, 25.0, rw_mode=mode)
+            b = o.bwd(gu, w, go, 4.0, 25.0, rw_mode=mode)
+            np.testing.assert_allclose(y, Y.detach().numpy(), rtol=1e-13, atol=1e-300)
+            np.testing.assert_allclose(b.dg, G.grad.numpy(), rtol=1e-12, atol=1e-13 * np.abs(G.grad.numpy()).max())
+            np.testing.assert_allclose(b.du, U.grad.numpy(), rtol=1e-12, atol=1e-13 * np.abs(U.grad.numpy()).max())
+            if mode == oracle.RW_COL:
+                cs, cm = o.dw_columns(gu, go, 4.0, 25.0)
+                np.testing.assert_allclose(cs, W.grad.numpy(), rtol=1e-12, atol=1e-13 * cm.max())
+            else:
+                terms = o.dw_terms(gu, go, 4.0, 25.0)
+                np.testing.assert_allclose(terms, W.grad.numpy(), rtol=1e-13, atol=1e-300)
+                # the per-row sums of the full gradient are the row-aligned gradient
+                np.testing.assert_allclose(terms.sum(axis=1), b.dw, rtol=1e-12, atol=1e-13 * b.sw.max())
+
+
 def pin_special_rows(o):
     """A zero gate column gives Y = 0, dU = 0, dG = go w T_u / 2; a zero up
     column gives Y = 0, dG = 0, dU = go w T_g (sech^2(0) = 1)."""
@@ -297,6 +332,7 @@ PINS = [
     pin_linear_beta_none,
     pin_finite_differences,
     pin_torch_autograd_rows,
+    pin_elementwise_weights,
     pin_special_rows,
     pin_dw_bruteforce,
     pin_bf16_loading,
@@ -323,6 +359,7 @@ MUTANTS = {
     10: "linear beta ignored",
     11: "sech^2 with exp(-|a|) instead of exp(-2|a|)",
     12: "row stride ignored",
+    13: "per-column weight indexed by the row",
 }
 
 
