@@ -25,8 +25,10 @@ SITU_DTYPE_F32 = 1
 SITU_RW_ROW = 0
 SITU_RW_SCALAR = 1
 SITU_RW_NONE = 2
+SITU_RW_COL = 3
+SITU_RW_FULL = 4
 
-ABI_VERSION = 1
+ABI_VERSION = 2
 
 # Entry points declared in include/situ_glu.h: name -> (restype, argtypes).
 _I64, _INT, _DBL, _VP, _SZ = ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_void_p, ctypes.c_size_t
@@ -35,7 +37,7 @@ SIGNATURES = {
                             _VP, _I64, _VP]),
     "situ_glu_bwd": (_INT, [_VP, _INT, _I64, _I64, _I64, _VP, _INT, _INT, _I64, _DBL, _INT, _DBL,
                             _VP, _I64, _VP, _I64, _VP, _I64, _VP, _SZ, _VP]),
-    "situ_glu_bwd_workspace_bytes": (_SZ, [_I64, _INT, _INT]),
+    "situ_glu_bwd_workspace_bytes": (_SZ, [_I64, _I64, _INT, _INT]),
     "situ_glu_status_string": (ctypes.c_char_p, [_INT]),
     "situ_glu_last_error": (ctypes.c_char_p, []),
     "situ_glu_abi_version": (_INT, []),
@@ -116,8 +118,8 @@ def situ_glu_bwd_no_alloc(gate_up, dtype, tokens, inter, gate_up_row_stride, rw,
                                        stream)
 
 
-def situ_glu_bwd_workspace_bytes(tokens, rw_mode, want_drw) -> int:
-    return lib().situ_glu_bwd_workspace_bytes(tokens, rw_mode, want_drw)
+def situ_glu_bwd_workspace_bytes(tokens, inter, rw_mode, want_drw) -> int:
+    return lib().situ_glu_bwd_workspace_bytes(tokens, inter, rw_mode, want_drw)
 
 
 def situ_glu_status_string(status) -> str:

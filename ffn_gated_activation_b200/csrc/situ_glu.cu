@@ -759,6 +759,412 @@ __global__ void __launch_bounds__(kFinalizeThreads)
 }
 
 // ---------------------------------------------------------------------------
+// Element-wise routing weights: one per column ([I]) or per element ([T, I])
+// ---------------------------------------------------------------------------
+// The weight of element (r, i) enters the same pair arithmetic as a per-pair
+// factor.  The [T, I] gradient is the term go T_g T_u itself; the [I] gradient
+// sums it over rows.  The rows are cut into chunks of kColChunk (chunk k holds
+// rows [k kColChunk, (k + 1) kColChunk)); a CTA takes chunks blockIdx.x,
+// blockIdx.x + gridDim.x, ...; each thread adds the terms of its own columns
+// in row order and writes the chunk's column sums to workspace row k; a second
+// kernel adds the chunks in order.  Both orders are fixed by the shape alone,
+// so the results do not depend on the grid.  Small chunks keep the CTAs evenly
+// loaded; the partial sums cost 8 I bytes of traffic per chunk against the
+// 10 I bytes (bf16) every row moves.
+//
+// As in the per-row kernels, a thread owns vectors j and j + blockDim.x of
+// each row and loads the CTA's next row while it computes this one.  The
+// column sums then live in registers; the looped form (rows wider than two
+// vectors per thread) keeps them in shared memory.
+
+constexpr int kColChunk = 16;
+constexpr int kMaxColInter = 16384;  // column sums of the looped form live in shared memory
+
+struct EwArgs {
+  const char* gate_up;
+  int64_t gu_pitch;  // bytes
+  const char* grad_out;  // backward only
+  int64_t go_pitch;
+  char* out;  // forward: Y; backward: d_gate_up
+  int64_t out_pitch;
+  const char* rw;
+  int64_t rw_pitch;  // bytes between rows of a [T, I] weight (0 for [I])
+  char* d_rw;        // backward: gradient shaped like rw (NULL: not wanted)
+  int64_t d_rw_pitch;
+  float* partials;   // backward, [I] weights: [ceil(T / kColChunk)][inter]
+  int rw_bf16;
+  int64_t tokens;
+  int half_bytes;
+  int vpr;
+  int inter;
+  Coeffs c;
+};
+
+__device__ __forceinline__ uint2 ld_stream8(const void* p) {
+  uint2 r;
+  asm("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void st_stream8(void* p, const uint2& v) {
+  asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
+
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t q) {
+  return make_float2(__uint_as_float(q << 16), __uint_as_float(q & 0xffff0000u));
+}
+
+// The kPairs weight pairs of vector j (elements 2 kPairs j ...) from `w_row`:
+// 8 or 16 bytes of bf16, 16 or 32 bytes of fp32.
+template <typename S>
+__device__ __forceinline__ void load_w_pairs(const char* w_row, int j, int bf16, float2 (&w)[S::kPairs]) {
+  constexpr int kElems = 2 * S::kPairs;
+  if (bf16) {
+    const char* p = w_row + j * kElems * 2;
+    if constexpr (kElems == 8) {
+      const uint4 v = ld_stream(p);
+      w[0] = bf16x2_to_f2(v.x); w[1] = bf16x2_to_f2(v.y); w[2] = bf16x2_to_f2(v.z); w[3] = bf16x2_to_f2(v.w);
+    } else {
+      const uint2 v = ld_stream8(p);
+      w[0] = bf16x2_to_f2(v.x); w[1] = bf16x2_to_f2(v.y);
+    }
+  } else {
+    const char* p = w_row + j * kElems * 4;
+#pragma unroll
+    for (int k = 0; k < S::kPairs / 2; ++k) {
+      const uint4 v = ld_stream(p + 16 * k);
+      w[2 * k] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+      w[2 * k + 1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+    }
+  }
+}
+
+template <typename S>
+__device__ __forceinline__ void store_w_pairs(char* d_row, int j, int bf16, const float2 (&d)[S::kPairs]) {
+  constexpr int kElems = 2 * S::kPairs;
+  if (bf16) {
+    char* p = d_row + j * kElems * 2;
+    if constexpr (kElems == 8)
+      st_stream(p, make_uint4(Bf16::pack(d[0]), Bf16::pack(d[1]), Bf16::pack(d[2]), Bf16::pack(d[3])));
+    else
+      st_stream8(p, make_uint2(Bf16::pack(d[0]), Bf16::pack(d[1])));
+  } else {
+    char* p = d_row + j * kElems * 4;
+#pragma unroll
+    for (int k = 0; k < S::kPairs / 2; ++k)
+      st_stream(p + 16 * k, make_uint4(__float_as_uint(d[2 * k].x), __float_as_uint(d[2 * k].y),
+                                       __float_as_uint(d[2 * k + 1].x), __float_as_uint(d[2 * k + 1].y)));
+  }
+}
+
+// One 16-byte vector of Y with per-element weights w.
+template <typename S, int GATE, bool HAS_LB>
+__device__ __forceinline__ uint4 ew_fwd_vec(const uint4& gv, const uint4& uv, const float2 (&w)[S::kPairs],
+                                            const Coeffs& c) {
+  uint4 o;
+#pragma unroll
+  for (int p = 0; p < S::kPairs; ++p) {
+    const float2 wbb = mul2(w[p], splat(c.bb));
+    float2 y;
+    if constexpr (std::is_same<S, Bf16>::value)
+      y = fwd_pair_bf16<GATE, HAS_LB>(S::pair(gv, p), S::pair(uv, p), wbb, c);
+    else
+      y = fwd_pair_abs<GATE, HAS_LB, S>(S::pair(gv, p), S::pair(uv, p), wbb, c);
+    S::put(o, p, y);
+  }
+  return o;
+}
+
+// One 16-byte vector of dG and dU with per-element weights w; t receives the
+// weight-gradient terms go T_g T_u.
+template <typename S, int GATE, bool HAS_LB>
+__device__ __forceinline__ void ew_bwd_vec(const uint4& gv, const uint4& uv, const uint4& ov,
+                                           const float2 (&w)[S::kPairs], const Coeffs& c, uint4& dgv, uint4& duv,
+                                           float2 (&t)[S::kPairs]) {
+  const float kdg = 4.0f * c.lb, kdu = HAS_LB ? 16.0f : 4.0f;
+  const float dws = bwd_dw_scale(c);
+#pragma unroll
+  for (int p = 0; p < S::kPairs; ++p) {
+    float2 dg, du, acc = make_float2(0.0f, 0.0f);
+    bwd_pair<GATE, HAS_LB, S>(S::pair(gv, p), S::pair(uv, p), as_f2(S::pair(ov, p)), mul2(w[p], splat(kdg)),
+                              mul2(w[p], splat(kdu)), c, dg, du, acc);
+    t[p] = mul2(acc, splat(dws));
+    S::put(dgv, p, dg);
+    S::put(duv, p, du);
+  }
+}
+
+template <typename S>
+__device__ __forceinline__ void add_pairs(float2 (&s)[S::kPairs], const float2 (&t)[S::kPairs]) {
+#pragma unroll
+  for (int p = 0; p < S::kPairs; ++p) s[p] = add2(s[p], t[p]);
+}
+
+template <typename S>
+__device__ __forceinline__ void zero_pairs(float2 (&s)[S::kPairs]) {
+#pragma unroll
+  for (int p = 0; p < S::kPairs; ++p) s[p] = make_float2(0.0f, 0.0f);
+}
+
+// Column sums of vector j (kElems floats) to workspace row `chunk`.
+template <typename S>
+__device__ __forceinline__ void store_col_partials(float* partials, int64_t chunk, int inter, int j,
+                                                   const float2 (&s)[S::kPairs]) {
+  float4* p = reinterpret_cast<float4*>(partials + chunk * inter + j * 2 * S::kPairs);
+#pragma unroll
+  for (int k = 0; k < S::kPairs / 2; ++k) p[k] = make_float4(s[2 * k].x, s[2 * k].y, s[2 * k + 1].x, s[2 * k + 1].y);
+}
+
+template <typename S, int GATE, bool HAS_LB, bool FULL>
+__global__ void __launch_bounds__(kMaxThreads) situ_glu_fwd_ew_kernel(const EwArgs a) {
+  constexpr int kP = S::kPairs;
+  const int nt = blockDim.x;
+  if (a.vpr <= 2 * nt) {
+    const int j = threadIdx.x, j2 = j + nt;
+    const bool one = j < a.vpr, two = j2 < a.vpr;
+    int64_t row = blockIdx.x;
+    if (row >= a.tokens) return;
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    uint4 g0 = z, u0 = z, g1 = z, u1 = z;
+    float2 w0[kP], w1[kP];  // [I]: this thread's columns, loaded once; [T, I]: the current row's
+    {
+      const char* gu = a.gate_up + row * a.gu_pitch;
+      const char* wr = a.rw + row * a.rw_pitch;
+      if (one) {
+        g0 = ld_stream(gu + j * kVecBytes);
+        u0 = ld_stream(gu + a.half_bytes + j * kVecBytes);
+        load_w_pairs<S>(wr, j, a.rw_bf16, w0);
+      }
+      if (two) {
+        g1 = ld_stream(gu + j2 * kVecBytes);
+        u1 = ld_stream(gu + a.half_bytes + j2 * kVecBytes);
+        load_w_pairs<S>(wr, j2, a.rw_bf16, w1);
+      }
+    }
+    for (;;) {
+      const int64_t next = row + gridDim.x;
+      const bool more = next < a.tokens;
+      uint4 ng0, nu0, ng1, nu1;
+      float2 nw0[kP], nw1[kP];
+      if (more) {
+        const char* gu = a.gate_up + next * a.gu_pitch;
+        const char* wr = a.rw + next * a.rw_pitch;
+        if (one) {
+          ng0 = ld_stream(gu + j * kVecBytes);
+          nu0 = ld_stream(gu + a.half_bytes + j * kVecBytes);
+          if (FULL) load_w_pairs<S>(wr, j, a.rw_bf16, nw0);
+        }
+        if (two) {
+          ng1 = ld_stream(gu + j2 * kVecBytes);
+          nu1 = ld_stream(gu + a.half_bytes + j2 * kVecBytes);
+          if (FULL) load_w_pairs<S>(wr, j2, a.rw_bf16, nw1);
+        }
+      }
+      char* out = a.out + row * a.out_pitch;
+      if (one) st_stream(out + j * kVecBytes, ew_fwd_vec<S, GATE, HAS_LB>(g0, u0, w0, a.c));
+      if (two) st_stream(out + j2 * kVecBytes, ew_fwd_vec<S, GATE, HAS_LB>(g1, u1, w1, a.c));
+      if (!more) break;
+      row = next;
+      g0 = ng0; u0 = nu0; g1 = ng1; u1 = nu1;
+      if (FULL) {
+#pragma unroll
+        for (int p = 0; p < kP; ++p) { w0[p] = nw0[p]; w1[p] = nw1[p]; }
+      }
+    }
+    return;
+  }
+  for (int64_t row = blockIdx.x; row < a.tokens; row += gridDim.x) {
+    const char* gu = a.gate_up + row * a.gu_pitch;
+    char* out = a.out + row * a.out_pitch;
+    const char* wr = a.rw + row * a.rw_pitch;
+    for (int j = threadIdx.x; j < a.vpr; j += nt) {
+      float2 w[kP];
+      load_w_pairs<S>(wr, j, a.rw_bf16, w);
+      st_stream(out + j * kVecBytes, ew_fwd_vec<S, GATE, HAS_LB>(ld_stream(gu + j * kVecBytes),
+                                                                 ld_stream(gu + a.half_bytes + j * kVecBytes), w, a.c));
+    }
+  }
+}
+
+template <typename S, int GATE, bool HAS_LB, bool FULL>
+__global__ void __launch_bounds__(kMaxThreads) situ_glu_bwd_ew_kernel(const EwArgs a) {
+  extern __shared__ float col_sums[];  // looped form, [I] weights with a wanted gradient: [inter]
+  constexpr int kP = S::kPairs, kElems = 2 * kP;
+  constexpr int64_t kRows = FULL ? 1 : kColChunk;  // rows per chunk
+  const int nt = blockDim.x;
+  const bool want = a.d_rw != nullptr;
+  const int64_t nchunks = (a.tokens + kRows - 1) / kRows;
+  if (a.vpr <= 2 * nt) {
+    const int j = threadIdx.x, j2 = j + nt;
+    const bool one = j < a.vpr, two = j2 < a.vpr;
+    int64_t ch = blockIdx.x;
+    if (ch >= nchunks) return;
+    int64_t row = ch * kRows, end = min(a.tokens, row + kRows);
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    uint4 g0 = z, u0 = z, o0 = z, g1 = z, u1 = z, o1 = z;
+    float2 w0[kP], w1[kP], s0[kP], s1[kP];
+    zero_pairs<S>(s0);
+    zero_pairs<S>(s1);
+    {
+      const char* gu = a.gate_up + row * a.gu_pitch;
+      const char* gor = a.grad_out + row * a.go_pitch;
+      const char* wr = a.rw + row * a.rw_pitch;
+      if (one) {
+        g0 = ld_stream(gu + j * kVecBytes);
+        u0 = ld_stream(gu + a.half_bytes + j * kVecBytes);
+        o0 = ld_stream(gor + j * kVecBytes);
+        load_w_pairs<S>(wr, j, a.rw_bf16, w0);
+      }
+      if (two) {
+        g1 = ld_stream(gu + j2 * kVecBytes);
+        u1 = ld_stream(gu + a.half_bytes + j2 * kVecBytes);
+        o1 = ld_stream(gor + j2 * kVecBytes);
+        load_w_pairs<S>(wr, j2, a.rw_bf16, w1);
+      }
+    }
+    for (;;) {
+      int64_t next = row + 1, nch = ch, nend = end;
+      if (next >= end) {  // the chunk is done: on to the CTA's next chunk
+        nch = ch + gridDim.x;
+        next = nch * kRows;
+        nend = min(a.tokens, next + kRows);
+      }
+      const bool more = nch < nchunks;
+      uint4 ng0, nu0, no0, ng1, nu1, no1;
+      float2 nw0[kP], nw1[kP];
+      if (more) {
+        const char* gu = a.gate_up + next * a.gu_pitch;
+        const char* gor = a.grad_out + next * a.go_pitch;
+        const char* wr = a.rw + next * a.rw_pitch;
+        if (one) {
+          ng0 = ld_stream(gu + j * kVecBytes);
+          nu0 = ld_stream(gu + a.half_bytes + j * kVecBytes);
+          no0 = ld_stream(gor + j * kVecBytes);
+          if (FULL) load_w_pairs<S>(wr, j, a.rw_bf16, nw0);
+        }
+        if (two) {
+          ng1 = ld_stream(gu + j2 * kVecBytes);
+          nu1 = ld_stream(gu + a.half_bytes + j2 * kVecBytes);
+          no1 = ld_stream(gor + j2 * kVecBytes);
+          if (FULL) load_w_pairs<S>(wr, j2, a.rw_bf16, nw1);
+        }
+      }
+      char* dgu = a.out + row * a.out_pitch;
+      char* drw = FULL && want ? a.d_rw + row * a.d_rw_pitch : nullptr;
+      float2 t[kP];
+      uint4 dg, du;
+      if (one) {
+        ew_bwd_vec<S, GATE, HAS_LB>(g0, u0, o0, w0, a.c, dg, du, t);
+        st_stream(dgu + j * kVecBytes, dg);
+        st_stream(dgu + a.half_bytes + j * kVecBytes, du);
+        if (want) {
+          if (FULL) store_w_pairs<S>(drw, j, a.rw_bf16, t);
+          else add_pairs<S>(s0, t);
+        }
+      }
+      if (two) {
+        ew_bwd_vec<S, GATE, HAS_LB>(g1, u1, o1, w1, a.c, dg, du, t);
+        st_stream(dgu + j2 * kVecBytes, dg);
+        st_stream(dgu + a.half_bytes + j2 * kVecBytes, du);
+        if (want) {
+          if (FULL) store_w_pairs<S>(drw, j2, a.rw_bf16, t);
+          else add_pairs<S>(s1, t);
+        }
+      }
+      if (!FULL && want && nch != ch) {
+        if (one) store_col_partials<S>(a.partials, ch, a.inter, j, s0);
+        if (two) store_col_partials<S>(a.partials, ch, a.inter, j2, s1);
+        zero_pairs<S>(s0);
+        zero_pairs<S>(s1);
+      }
+      if (!more) break;
+      row = next;
+      ch = nch;
+      end = nend;
+      g0 = ng0; u0 = nu0; o0 = no0; g1 = ng1; u1 = nu1; o1 = no1;
+      if (FULL) {
+#pragma unroll
+        for (int p = 0; p < kP; ++p) { w0[p] = nw0[p]; w1[p] = nw1[p]; }
+      }
+    }
+    return;
+  }
+  // Looped form.  Thread t owns the columns of its vectors j = t, t + nt, ...:
+  // it alone resets, adds to and exports them, so no barrier is needed.
+  const bool colsum = !FULL && want;
+  for (int64_t ch = blockIdx.x; ch < nchunks; ch += gridDim.x) {
+    if (colsum)
+      for (int j = threadIdx.x; j < a.vpr; j += nt)
+        for (int e = 0; e < kElems; ++e) col_sums[j * kElems + e] = 0.0f;
+    const int64_t r1 = min(a.tokens, (ch + 1) * kRows);
+    for (int64_t row = ch * kRows; row < r1; ++row) {
+      const char* gu = a.gate_up + row * a.gu_pitch;
+      const char* gor = a.grad_out + row * a.go_pitch;
+      char* dgu = a.out + row * a.out_pitch;
+      const char* wr = a.rw + row * a.rw_pitch;
+      for (int j = threadIdx.x; j < a.vpr; j += nt) {
+        float2 w[kP], t[kP];
+        load_w_pairs<S>(wr, j, a.rw_bf16, w);
+        uint4 dg, du;
+        ew_bwd_vec<S, GATE, HAS_LB>(ld_stream(gu + j * kVecBytes), ld_stream(gu + a.half_bytes + j * kVecBytes),
+                                    ld_stream(gor + j * kVecBytes), w, a.c, dg, du, t);
+        st_stream(dgu + j * kVecBytes, dg);
+        st_stream(dgu + a.half_bytes + j * kVecBytes, du);
+        if (want) {
+          if (FULL) {
+            store_w_pairs<S>(a.d_rw + row * a.d_rw_pitch, j, a.rw_bf16, t);
+          } else {
+#pragma unroll
+            for (int p = 0; p < kP; ++p) {
+              col_sums[j * kElems + 2 * p] += t[p].x;
+              col_sums[j * kElems + 2 * p + 1] += t[p].y;
+            }
+          }
+        }
+      }
+    }
+    if (colsum)
+      for (int j = threadIdx.x; j < a.vpr; j += nt)
+        for (int e = 0; e < kElems; ++e) a.partials[ch * a.inter + j * kElems + e] = col_sums[j * kElems + e];
+  }
+}
+
+// Per-column gradient: add the chunks' partial sums.  A CTA takes 32 columns
+// (one warp-wide, coalesced row of partials) and 32 chunk groups: group g adds
+// chunks g, g + 32, ... in eight interleaved running sums (eight loads in
+// flight per thread), and the groups are then added in group order.  The
+// order depends on nchunks alone.
+constexpr int kFinCols = 32, kFinGroups = 32, kFinLanes = 8;
+
+__global__ void __launch_bounds__(kFinCols * kFinGroups)
+    situ_glu_dw_columns_finalize_kernel(const float* partials, int64_t nchunks, int inter, void* d_rw, int bf16) {
+  __shared__ float red[kFinGroups][kFinCols + 1];
+  const int lane = threadIdx.x % kFinCols, grp = threadIdx.x / kFinCols;
+  const int i = blockIdx.x * kFinCols + lane;
+  float s = 0.0f;
+  if (i < inter) {
+    float acc[kFinLanes];
+#pragma unroll
+    for (int q = 0; q < kFinLanes; ++q) acc[q] = 0.0f;
+    int64_t k = grp;
+    for (; k + (kFinLanes - 1) * kFinGroups < nchunks; k += kFinLanes * kFinGroups) {
+#pragma unroll
+      for (int q = 0; q < kFinLanes; ++q) acc[q] += partials[(k + q * kFinGroups) * inter + i];
+    }
+    for (; k < nchunks; k += kFinGroups) acc[0] += partials[k * inter + i];
+#pragma unroll
+    for (int q = 0; q < kFinLanes; ++q) s += acc[q];
+  }
+  red[grp][lane] = s;
+  __syncthreads();
+  if (grp == 0 && i < inter) {
+    float t = red[0][lane];
+    for (int g = 1; g < kFinGroups; ++g) t += red[g][lane];
+    store_rw_grad(d_rw, i, bf16, t);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Wide direct-load forward (the default whenever the layout allows)
 // ---------------------------------------------------------------------------
 // When a half row holds 64 k 16-byte vectors (k = 1..8) and every base and row
@@ -1097,6 +1503,17 @@ Span matrix_span(const void* base, int64_t rows, int64_t pitch_elems, int64_t wi
 
 bool overlap(const Span& a, const Span& b) { return a.lo < b.hi && b.lo < a.hi; }
 
+// Bytes a routing-weight tensor (or its gradient) spans in a given mode.
+Span weight_span(const void* p, situ_rw_mode_t mode, int64_t tokens, int64_t stride, int64_t inter, int es) {
+  switch (mode) {
+    case SITU_RW_ROW: return matrix_span(p, tokens, stride, 1, es);
+    case SITU_RW_SCALAR: return matrix_span(p, 1, 1, 1, es);
+    case SITU_RW_COL: return matrix_span(p, 1, inter, inter, es);
+    case SITU_RW_FULL: return matrix_span(p, tokens, stride, inter, es);
+    default: return {0, 0};
+  }
+}
+
 // rows * pitch + width fits in int64 bytes.
 bool span_fits(int64_t rows, int64_t pitch, int64_t width, int es) {
   const int64_t limit = INT64_MAX / es - width;
@@ -1107,13 +1524,22 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 constexpr int64_t kMaxInter = int64_t(1) << 28;
 
+// Bytes of element-wise weights that go with one 16-byte vector of gate_up
+// (the kernels load them in one piece), at most 16: the alignment that
+// per-column and per-element weights and their gradient rows need.
+int ew_align(situ_dtype_t dtype, situ_dtype_t rw_dtype) {
+  const int a = kVecBytes / elem_size(dtype) * elem_size(rw_dtype);
+  return a < 16 ? a : 16;
+}
+
 // Checks common to fwd and bwd.  Fills coefficients and the gate mode.
 situ_status_t check_common(situ_dtype_t dtype, int64_t tokens, int64_t inter, int64_t gu_stride,
                            const void* rw, situ_dtype_t rw_dtype, situ_rw_mode_t rw_mode,
                            int64_t rw_stride, double beta, int has_lb, double lb, Coeffs* c,
                            int* gate_mode) {
   if (!valid_dtype(dtype)) return fail(SITU_ERR_INVALID_ARG, "dtype %d is not a situ_dtype_t", (int)dtype);
-  if (rw_mode != SITU_RW_ROW && rw_mode != SITU_RW_SCALAR && rw_mode != SITU_RW_NONE)
+  if (rw_mode != SITU_RW_ROW && rw_mode != SITU_RW_SCALAR && rw_mode != SITU_RW_NONE && rw_mode != SITU_RW_COL &&
+      rw_mode != SITU_RW_FULL)
     return fail(SITU_ERR_INVALID_ARG, "rw_mode %d is not a situ_rw_mode_t", (int)rw_mode);
   if (rw_mode != SITU_RW_NONE && !valid_dtype(rw_dtype))
     return fail(SITU_ERR_INVALID_ARG, "rw_dtype %d is not a situ_dtype_t", (int)rw_dtype);
@@ -1131,7 +1557,16 @@ situ_status_t check_common(situ_dtype_t dtype, int64_t tokens, int64_t inter, in
     return fail(SITU_ERR_INVALID_ARG, "rw is NULL");
   }
   if (rw_mode == SITU_RW_ROW && rw_stride < 0) return fail(SITU_ERR_INVALID_ARG, "rw_stride < 0");
+  if (rw_mode == SITU_RW_FULL && rw_stride < inter) return fail(SITU_ERR_INVALID_ARG, "rw_stride < inter (full weights)");
+  if (rw_mode == SITU_RW_COL && inter > kMaxColInter)
+    return fail(SITU_ERR_UNSUPPORTED, "per-column weights support inter <= %d", kMaxColInter);
   const int es = elem_size(dtype);
+  if ((rw_mode == SITU_RW_COL || rw_mode == SITU_RW_FULL) && tokens > 0) {
+    const int a = ew_align(dtype, rw_dtype);
+    if (!aligned(rw, a)) return fail(SITU_ERR_MISALIGNED, "element-wise weights must be %d-byte aligned", a);
+    if (rw_mode == SITU_RW_FULL && (rw_stride * elem_size(rw_dtype)) % a != 0)
+      return fail(SITU_ERR_MISALIGNED, "row pitch of full weights is not a multiple of %d bytes", a);
+  }
   if ((inter * es) % kVecBytes != 0)
     return fail(SITU_ERR_MISALIGNED, "inter * element size (%lld bytes) is not a multiple of 16",
                 (long long)(inter * es));
@@ -1282,6 +1717,33 @@ FwdKernel pick_fwd_gate(int gate) {
   }
 }
 
+using EwKernel = void (*)(EwArgs);
+
+template <typename S, int GATE, bool LB, bool BWD>
+EwKernel ew_kernel(bool full) {
+  if constexpr (BWD)
+    return full ? situ_glu_bwd_ew_kernel<S, GATE, LB, true> : situ_glu_bwd_ew_kernel<S, GATE, LB, false>;
+  else
+    return full ? situ_glu_fwd_ew_kernel<S, GATE, LB, true> : situ_glu_fwd_ew_kernel<S, GATE, LB, false>;
+}
+
+template <typename S, bool LB, bool BWD>
+EwKernel pick_ew_gate(int gate, bool full) {
+  switch (gate) {
+    case kGateSquare: return ew_kernel<S, kGateSquare, LB, BWD>(full);
+    case kGateEqual: return ew_kernel<S, kGateEqual, LB, BWD>(full);
+    case kGateRoot: return ew_kernel<S, kGateRoot, LB, BWD>(full);
+    default: return ew_kernel<S, kGateGeneric, LB, BWD>(full);
+  }
+}
+
+template <bool BWD>
+EwKernel pick_ew(situ_dtype_t dtype, int gate, bool lb, bool full) {
+  if (dtype == SITU_DTYPE_BF16)
+    return lb ? pick_ew_gate<Bf16, true, BWD>(gate, full) : pick_ew_gate<Bf16, false, BWD>(gate, full);
+  return lb ? pick_ew_gate<F32, true, BWD>(gate, full) : pick_ew_gate<F32, false, BWD>(gate, full);
+}
+
 template <typename S, bool LB>
 FwdKernel pick_fwd_wide_gate(int gate) {
   switch (gate) {
@@ -1353,7 +1815,8 @@ situ_status_t situ_glu_fwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
   if (gate_up == nullptr || out == nullptr) return fail(SITU_ERR_INVALID_ARG, "gate_up or out is NULL");
   const int es = elem_size(dtype);
   if (!span_fits(tokens, gate_up_row_stride, 2 * inter, es) || !span_fits(tokens, out_row_stride, inter, es) ||
-      (rw_mode == SITU_RW_ROW && !span_fits(tokens, rw_stride, 1, elem_size(rw_dtype))))
+      (rw_mode == SITU_RW_ROW && !span_fits(tokens, rw_stride, 1, elem_size(rw_dtype))) ||
+      (rw_mode == SITU_RW_FULL && !span_fits(tokens, rw_stride, inter, elem_size(rw_dtype))))
     return fail(SITU_ERR_INVALID_ARG, "tensor extent overflows int64");
   if (!aligned(gate_up, 16) || !aligned(out, 16) || (gate_up_row_stride * es) % 16 != 0 ||
       (out_row_stride * es) % 16 != 0)
@@ -1363,10 +1826,31 @@ situ_status_t situ_glu_fwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
   const Span s_out = matrix_span(out, tokens, out_row_stride, inter, es);
   if (overlap(s_out, matrix_span(gate_up, tokens, gate_up_row_stride, 2 * inter, es)))
     return fail(SITU_ERR_INVALID_ARG, "out overlaps gate_up");
-  if (rw_mode == SITU_RW_ROW && overlap(s_out, matrix_span(rw, tokens, rw_stride, 1, elem_size(rw_dtype))))
+  if (overlap(s_out, weight_span(rw, rw_mode, tokens, rw_stride, inter, elem_size(rw_dtype))))
     return fail(SITU_ERR_INVALID_ARG, "out overlaps rw");
-  if (rw_mode == SITU_RW_SCALAR && overlap(s_out, matrix_span(rw, 1, 1, 1, elem_size(rw_dtype))))
-    return fail(SITU_ERR_INVALID_ARG, "out overlaps rw");
+
+  if (rw_mode == SITU_RW_COL || rw_mode == SITU_RW_FULL) {
+    EwArgs e{};
+    e.gate_up = static_cast<const char*>(gate_up);
+    e.gu_pitch = gate_up_row_stride * es;
+    e.out = static_cast<char*>(out);
+    e.out_pitch = out_row_stride * es;
+    e.rw = static_cast<const char*>(rw);
+    e.rw_pitch = rw_mode == SITU_RW_FULL ? rw_stride * elem_size(rw_dtype) : 0;
+    e.rw_bf16 = rw_dtype == SITU_DTYPE_BF16 ? 1 : 0;
+    e.tokens = tokens;
+    e.half_bytes = static_cast<int>(inter * es);
+    e.vpr = static_cast<int>(inter * es / kVecBytes);
+    e.inter = static_cast<int>(inter);
+    e.c = c;
+    EwKernel k = pick_ew<false>(dtype, gate, has_linear_beta != 0, rw_mode == SITU_RW_FULL);
+    const int threads = choose_threads(e.vpr);
+    int grid = 0;
+    st = launch_grid(reinterpret_cast<const void*>(k), threads, 0, tokens, &grid);
+    if (st != SITU_OK) return st;
+    k<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(e);
+    return check_launch("situ_glu_fwd");
+  }
 
   FwdArgs a;
   a.gate_up = static_cast<const char*>(gate_up);
@@ -1403,9 +1887,12 @@ situ_status_t situ_glu_fwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
   return check_launch("situ_glu_fwd");
 }
 
-size_t situ_glu_bwd_workspace_bytes(int64_t tokens, situ_rw_mode_t rw_mode, int want_drw) {
-  if (tokens <= 0 || rw_mode != SITU_RW_SCALAR || !want_drw) return 0;
-  const uint64_t bytes = static_cast<uint64_t>(tokens) * sizeof(float);
+size_t situ_glu_bwd_workspace_bytes(int64_t tokens, int64_t inter, situ_rw_mode_t rw_mode, int want_drw) {
+  if (tokens <= 0 || inter <= 0 || !want_drw) return 0;
+  uint64_t bytes = 0;
+  if (rw_mode == SITU_RW_SCALAR) bytes = static_cast<uint64_t>(tokens) * sizeof(float);
+  if (rw_mode == SITU_RW_COL)
+    bytes = static_cast<uint64_t>((tokens + kColChunk - 1) / kColChunk) * static_cast<uint64_t>(inter) * sizeof(float);
   return static_cast<size_t>((bytes + 255) / 256 * 256);
 }
 
@@ -1427,13 +1914,16 @@ situ_status_t situ_glu_bwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
     return fail(SITU_ERR_INVALID_ARG, "d_rw must be NULL for SITU_RW_NONE");
   const bool want_drw = d_rw != nullptr;
   if (want_drw && rw_mode == SITU_RW_ROW && d_rw_stride < 1) return fail(SITU_ERR_INVALID_ARG, "d_rw_stride < 1");
-  const size_t ws_needed = situ_glu_bwd_workspace_bytes(tokens, rw_mode, want_drw ? 1 : 0);
+  if (want_drw && rw_mode == SITU_RW_FULL && d_rw_stride < inter)
+    return fail(SITU_ERR_INVALID_ARG, "d_rw_stride < inter (full weights)");
+  const size_t ws_needed = situ_glu_bwd_workspace_bytes(tokens, inter, rw_mode, want_drw ? 1 : 0);
   if (tokens == 0) {
     // The gradient of a broadcast weight over zero rows is zero; nothing else
     // is written.  That store is the one piece of work an empty call does.
-    if (want_drw && rw_mode == SITU_RW_SCALAR) {
+    if (want_drw && (rw_mode == SITU_RW_SCALAR || rw_mode == SITU_RW_COL)) {
       if (!aligned(d_rw, elem_size(rw_dtype))) return fail(SITU_ERR_MISALIGNED, "d_rw not aligned");
-      cudaError_t err = cudaMemsetAsync(d_rw, 0, elem_size(rw_dtype), static_cast<cudaStream_t>(stream));
+      const size_t n = rw_mode == SITU_RW_COL ? static_cast<size_t>(inter) : 1;
+      cudaError_t err = cudaMemsetAsync(d_rw, 0, n * elem_size(rw_dtype), static_cast<cudaStream_t>(stream));
       if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
     }
     return SITU_OK;
@@ -1445,7 +1935,9 @@ situ_status_t situ_glu_bwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
   if (!span_fits(tokens, gate_up_row_stride, 2 * inter, es) || !span_fits(tokens, grad_out_row_stride, inter, es) ||
       !span_fits(tokens, d_gate_up_row_stride, 2 * inter, es) ||
       (rw_mode == SITU_RW_ROW && !span_fits(tokens, rw_stride, 1, rw_es)) ||
-      (want_drw && rw_mode == SITU_RW_ROW && !span_fits(tokens, d_rw_stride, 1, rw_es)))
+      (want_drw && rw_mode == SITU_RW_ROW && !span_fits(tokens, d_rw_stride, 1, rw_es)) ||
+      (rw_mode == SITU_RW_FULL && !span_fits(tokens, rw_stride, inter, rw_es)) ||
+      (want_drw && rw_mode == SITU_RW_FULL && !span_fits(tokens, d_rw_stride, inter, rw_es)))
     return fail(SITU_ERR_INVALID_ARG, "tensor extent overflows int64");
   if (!aligned(gate_up, 16) || !aligned(grad_out, 16) || !aligned(d_gate_up, 16) ||
       (gate_up_row_stride * es) % 16 != 0 || (grad_out_row_stride * es) % 16 != 0 ||
@@ -1453,6 +1945,10 @@ situ_status_t situ_glu_bwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
     return fail(SITU_ERR_MISALIGNED, "gate_up/grad_out/d_gate_up base or row pitch not 16-byte aligned");
   if (rw_mode != SITU_RW_NONE && !aligned(rw, rw_es)) return fail(SITU_ERR_MISALIGNED, "rw not aligned");
   if (want_drw && !aligned(d_rw, rw_es)) return fail(SITU_ERR_MISALIGNED, "d_rw not aligned");
+  if (want_drw && rw_mode == SITU_RW_FULL &&
+      (!aligned(d_rw, ew_align(dtype, rw_dtype)) || (d_rw_stride * rw_es) % ew_align(dtype, rw_dtype) != 0))
+    return fail(SITU_ERR_MISALIGNED, "per-element weight gradient base or row pitch not %d-byte aligned",
+                ew_align(dtype, rw_dtype));
   if (ws_needed > 0) {
     if (workspace == nullptr || workspace_bytes < ws_needed)
       return fail(SITU_ERR_INVALID_ARG, "workspace needs %zu bytes, got %zu", ws_needed,
@@ -1464,15 +1960,12 @@ situ_status_t situ_glu_bwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
   const Span s_gu = matrix_span(gate_up, tokens, gate_up_row_stride, 2 * inter, es);
   const Span s_go = matrix_span(grad_out, tokens, grad_out_row_stride, inter, es);
   const Span s_dgu = matrix_span(d_gate_up, tokens, d_gate_up_row_stride, 2 * inter, es);
-  Span s_rw = {0, 0};
-  if (rw_mode == SITU_RW_ROW) s_rw = matrix_span(rw, tokens, rw_stride, 1, rw_es);
-  if (rw_mode == SITU_RW_SCALAR) s_rw = matrix_span(rw, 1, 1, 1, rw_es);
+  const Span s_rw = weight_span(rw, rw_mode, tokens, rw_stride, inter, rw_es);
   if (overlap(s_dgu, s_gu) || overlap(s_dgu, s_go) || overlap(s_dgu, s_rw))
     return fail(SITU_ERR_INVALID_ARG, "d_gate_up overlaps an input");
   Span s_drw = {0, 0};
   if (want_drw) {
-    s_drw = rw_mode == SITU_RW_ROW ? matrix_span(d_rw, tokens, d_rw_stride, 1, rw_es)
-                                   : matrix_span(d_rw, 1, 1, 1, rw_es);
+    s_drw = weight_span(d_rw, rw_mode, tokens, d_rw_stride, inter, rw_es);
     if (overlap(s_drw, s_gu) || overlap(s_drw, s_go) || overlap(s_drw, s_rw) || overlap(s_drw, s_dgu))
       return fail(SITU_ERR_INVALID_ARG, "d_rw overlaps another tensor");
   }
@@ -1481,6 +1974,48 @@ situ_status_t situ_glu_bwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
     if (overlap(s_ws, s_gu) || overlap(s_ws, s_go) || overlap(s_ws, s_rw) || overlap(s_ws, s_dgu) ||
         overlap(s_ws, s_drw))
       return fail(SITU_ERR_INVALID_ARG, "workspace overlaps a tensor");
+  }
+
+  if (rw_mode == SITU_RW_COL || rw_mode == SITU_RW_FULL) {
+    EwArgs e{};
+    e.gate_up = static_cast<const char*>(gate_up);
+    e.gu_pitch = gate_up_row_stride * es;
+    e.grad_out = static_cast<const char*>(grad_out);
+    e.go_pitch = grad_out_row_stride * es;
+    e.out = static_cast<char*>(d_gate_up);
+    e.out_pitch = d_gate_up_row_stride * es;
+    e.rw = static_cast<const char*>(rw);
+    e.rw_pitch = rw_mode == SITU_RW_FULL ? rw_stride * rw_es : 0;
+    e.d_rw = static_cast<char*>(d_rw);
+    e.d_rw_pitch = rw_mode == SITU_RW_FULL ? d_rw_stride * rw_es : 0;
+    e.partials = static_cast<float*>(workspace);
+    e.rw_bf16 = rw_dtype == SITU_DTYPE_BF16 ? 1 : 0;
+    e.tokens = tokens;
+    e.half_bytes = static_cast<int>(inter * es);
+    e.vpr = static_cast<int>(inter * es / kVecBytes);
+    e.inter = static_cast<int>(inter);
+    e.c = c;
+    const bool full = rw_mode == SITU_RW_FULL;
+    EwKernel k = pick_ew<true>(dtype, gate, has_linear_beta != 0, full);
+    const int threads = choose_threads(e.vpr);
+    // Shared memory only for the column sums of the looped form.
+    const int smem = (!full && want_drw && e.vpr > 2 * threads) ? static_cast<int>(inter * sizeof(float)) : 0;
+    const int64_t nchunks = full ? tokens : (tokens + kColChunk - 1) / kColChunk;
+    if (smem > 48 * 1024) {  // opt in beyond the default dynamic shared-memory limit
+      st = ensure_smem(reinterpret_cast<const void*>(k), smem);
+      if (st != SITU_OK) return st;
+    }
+    int grid = 0;
+    st = launch_grid(reinterpret_cast<const void*>(k), threads, smem, nchunks, &grid);
+    if (st != SITU_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    k<<<grid, threads, smem, s>>>(e);
+    st = check_launch("situ_glu_bwd");
+    if (st != SITU_OK || rw_mode != SITU_RW_COL || !want_drw) return st;
+    const int fin_grid = static_cast<int>((inter + kFinCols - 1) / kFinCols);
+    situ_glu_dw_columns_finalize_kernel<<<fin_grid, kFinCols * kFinGroups, 0, s>>>(e.partials, nchunks, e.inter,
+                                                                                  d_rw, e.rw_bf16);
+    return check_launch("situ_glu_bwd (per-column d_rw)");
   }
 
   BwdArgs a;
@@ -1630,13 +2165,14 @@ extern "C" situ_status_t situ_glu_bwd_no_alloc(const void* gate_up, situ_dtype_t
                                                int64_t d_gate_up_row_stride, void* d_rw, int64_t d_rw_stride,
                                                void* stream) {
   tl_last_error[0] = '\0';
-  const size_t need = situ_glu_bwd_workspace_bytes(tokens, rw_mode, d_rw != nullptr ? 1 : 0);
+  const size_t need = situ_glu_bwd_workspace_bytes(tokens, inter, rw_mode, d_rw != nullptr ? 1 : 0);
   void* ws = nullptr;
   if (need > 0) {
-    if (tokens > kNoAllocMaxTokens)
+    if (need > sizeof(g_noalloc_scratch))
       return fail(SITU_ERR_UNSUPPORTED,
-                  "situ_glu_bwd_no_alloc: %lld rows need %zu bytes of scratch; its fixed scratch holds %lld rows",
-                  (long long)tokens, need, (long long)kNoAllocMaxTokens);
+                  "situ_glu_bwd_no_alloc: %lld rows need %zu bytes of scratch; its fixed scratch holds %zu bytes "
+                  "(%lld rows with a broadcast weight)",
+                  (long long)tokens, need, sizeof(g_noalloc_scratch), (long long)kNoAllocMaxTokens);
     const situ_status_t st = noalloc_scratch(&ws);
     if (st != SITU_OK) return st;
   }

@@ -9,9 +9,13 @@ and grad_out row only), so:
   per-rank partials are summed across ranks (``allreduce_drw``).
 * Tensor parallelism of FC1 (column-parallel: rank r holds gate columns
   [a_r, b_r) and the matching up columns, see ``tp_local_gate_up``) keeps the
-  forward and dG/dU local; only the routing-weight gradient, a sum over all I
-  columns, needs the sum of the ranks' partial sums over their columns: an
-  all-reduce of T values (``situ_glu_bwd_tp``).
+  forward and dG/dU local; a row-aligned or broadcast routing-weight
+  gradient, a sum over all I columns, needs the sum of the ranks' partial
+  sums over their columns: an all-reduce of T values (``situ_glu_bwd_tp``).
+  Per-column ([I]) and per-element ([..., I]) weights are sharded with their
+  columns (``tp_local_columns``); their gradients stay local.
+* Under data parallelism a per-column weight is shared by every row shard,
+  so its [I] gradient is all-reduced like a broadcast weight's.
 
 Nothing here computes the method; the kernels run in libsitu_glu.so.
 """
@@ -67,12 +71,26 @@ def allreduce_drw(d_rw: torch.Tensor, group=None) -> torch.Tensor:
 def situ_glu_bwd_tp(gate_up_local, routing_weights, grad_out_local, beta=functional.DEFAULT_BETA,
                     linear_beta=functional.DEFAULT_LINEAR_BETA, group=None, want_drw=True, **kw):
     """Backward of a column-parallel shard: local d_gate_up [..., 2 I_r] and the
-    full routing-weight gradient (partials all-reduced over ``group``)."""
+    routing-weight gradient.  Row-aligned and broadcast weights span every
+    column, so their partials are all-reduced over ``group``; per-column and
+    per-element weights are passed as this rank's columns and their gradient
+    is already complete."""
+    lead = tuple(gate_up_local.shape[:-1])
+    inter_local = gate_up_local.shape[-1] // 2
     d_gate_up, d_rw = functional.situ_glu_bwd(gate_up_local, routing_weights, grad_out_local, beta,
                                               linear_beta, want_drw=want_drw, **kw)
-    if d_rw is not None:
+    if d_rw is not None and tp_drw_needs_allreduce(lead, inter_local, routing_weights):
         allreduce_drw(d_rw, group)
     return d_gate_up, d_rw
+
+
+def tp_drw_needs_allreduce(lead: tuple, inter_local: int, routing_weights) -> bool:
+    """Whether a column-parallel shard's routing-weight gradient is a partial
+    sum (row-aligned or broadcast weights) rather than this rank's own slice
+    (per-column or per-element weights)."""
+    from . import abi
+    mode = functional.routing_mode(lead, inter_local, routing_weights)[0]
+    return mode in (abi.SITU_RW_ROW, abi.SITU_RW_SCALAR)
 
 
 def max_over_ranks(value: float, device=None, group=None) -> float:

@@ -53,25 +53,34 @@ def _rows(gate_up: torch.Tensor):
     return g2, lead, inter
 
 
-def routing_mode(gate_up_lead: tuple, routing_weights):
-    """Classify routing_weights against gate_up's leading shape (NeMo
-    `_situ_rw_is_row_aligned`): returns (mode, flat view or None).
+def routing_mode(gate_up_lead: tuple, inter: int, routing_weights):
+    """Classify routing_weights against the output [*lead, inter] the way
+    broadcasting aligns them (NeMo `_situ_rw_is_row_aligned` and
+    `_WeightedSiTUFunction.forward`, parameter routing_weights).  Returns
+    (mode, view, stride): the C-ABI mode, the tensor the library reads, and
+    its element stride (rows for row-aligned and full weights).
 
-    None -> unweighted; one element -> broadcast scalar; shape [..., 1] with
-    gate_up's leading dimensions -> row-aligned.  Other broadcastable shapes
-    are not implemented (NotImplementedError)."""
+    None -> unweighted; one element -> broadcast scalar; [*lead, 1] ->
+    row-aligned; inter elements along the last axis ([I], [1, I], ...) -> one
+    weight per column; [*lead, I] -> one weight per element."""
     if routing_weights is None:
-        return abi.SITU_RW_NONE, None
+        return abi.SITU_RW_NONE, None, 1
     rw = routing_weights
     if rw.numel() == 1:
-        return abi.SITU_RW_SCALAR, rw.reshape(1)
-    if rw.dim() >= 1 and tuple(rw.shape[:-1]) == gate_up_lead and rw.shape[-1] == 1:
-        return abi.SITU_RW_ROW, rw.reshape(-1)
-    if tuple(rw.shape) == gate_up_lead:
-        return abi.SITU_RW_ROW, rw.reshape(-1)
+        return abi.SITU_RW_SCALAR, rw.reshape(1), 1
+    if rw.dim() == len(gate_up_lead) + 1 and tuple(rw.shape[:-1]) == gate_up_lead and rw.shape[-1] == 1:
+        flat = rw.reshape(-1)
+        return abi.SITU_RW_ROW, flat, flat.stride(0) if flat.numel() > 1 else 1
+    if rw.dim() >= 1 and rw.shape[-1] == inter and rw.numel() == inter:
+        return abi.SITU_RW_COL, rw.reshape(inter).contiguous(), 1
+    if tuple(rw.shape) == tuple(gate_up_lead) + (inter,):
+        w2 = rw.reshape(-1, inter)
+        if w2.stride(1) != 1 or (w2.shape[0] > 1 and w2.stride(0) < inter):
+            w2 = w2.contiguous()
+        return abi.SITU_RW_FULL, w2, w2.stride(0) if w2.shape[0] > 1 else inter
     raise NotImplementedError(
-        f"routing_weights of shape {tuple(rw.shape)} against gate_up rows {gate_up_lead}: only "
-        "row-aligned [..., 1], a single broadcast value, or None are implemented")
+        f"routing_weights of shape {tuple(rw.shape)} do not broadcast to the output {gate_up_lead + (inter,)} "
+        "as one of: [..., 1] (per row), one value, [I] (per column), [..., I] (per element)")
 
 
 def _stream_handle(stream) -> int:
@@ -86,7 +95,7 @@ def situ_glu_fwd(gate_up: torch.Tensor, routing_weights, beta: float = DEFAULT_B
     _check_beta(beta, linear_beta)
     g2, lead, inter = _rows(gate_up)
     dtype = _dtype_code(g2, "gate_up")
-    mode, rw = routing_mode(lead, routing_weights)
+    mode, rw, rw_stride = routing_mode(lead, inter, routing_weights)
     if rw is not None:
         if rw.device != g2.device:
             raise ValueError("routing_weights must be on gate_up's device")
@@ -98,8 +107,7 @@ def situ_glu_fwd(gate_up: torch.Tensor, routing_weights, beta: float = DEFAULT_B
     o2 = out.view(-1, inter)
     tokens = g2.shape[0]
     st = abi.situ_glu_fwd(g2.data_ptr(), dtype, tokens, inter, g2.stride(0) if tokens > 1 else 2 * inter,
-                          rw.data_ptr() if rw is not None else None, rw_dtype, mode,
-                          rw.stride(0) if rw is not None else 1,
+                          rw.data_ptr() if rw is not None else None, rw_dtype, mode, rw_stride,
                           float(beta), int(linear_beta is not None),
                           float(linear_beta) if linear_beta is not None else 0.0,
                           o2.data_ptr(), o2.stride(0) if tokens > 1 else inter, _stream_handle(stream))
@@ -124,30 +132,33 @@ def situ_glu_bwd(gate_up: torch.Tensor, routing_weights, grad_out: torch.Tensor,
     go2 = grad_out.reshape(-1, inter)
     if go2.stride(1) != 1 or (go2.shape[0] > 1 and go2.stride(0) < inter):
         go2 = go2.contiguous()
-    mode, rw = routing_mode(lead, routing_weights)
+    mode, rw, rw_stride = routing_mode(lead, inter, routing_weights)
     rw_dtype = _dtype_code(rw, "routing_weights") if rw is not None else abi.SITU_DTYPE_F32
     want = bool(want_drw) and rw is not None
     if d_gate_up is None:
         d_gate_up = torch.empty(lead + (2 * inter,), dtype=gate_up.dtype, device=gate_up.device)
     dg2 = d_gate_up.view(-1, 2 * inter)
-    d_rw_flat = None
+    d_rw_flat, d_rw_stride = None, 1
     if want:
         if d_rw is None:
             d_rw = torch.empty(routing_weights.shape, dtype=routing_weights.dtype, device=gate_up.device)
-        d_rw_flat = d_rw.view(-1)
+        if mode == abi.SITU_RW_FULL:
+            d_rw_flat = d_rw.view(-1, inter)
+            d_rw_stride = d_rw_flat.stride(0) if d_rw_flat.shape[0] > 1 else inter
+        else:
+            d_rw_flat = d_rw.view(-1)
+            d_rw_stride = d_rw_flat.stride(0) if d_rw_flat.numel() > 1 else 1
     tokens = g2.shape[0]
-    ws_bytes = abi.situ_glu_bwd_workspace_bytes(tokens, mode, int(want))
+    ws_bytes = abi.situ_glu_bwd_workspace_bytes(tokens, inter, mode, int(want))
     if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=gate_up.device)
     st = abi.situ_glu_bwd(g2.data_ptr(), dtype, tokens, inter, g2.stride(0) if tokens > 1 else 2 * inter,
-                          rw.data_ptr() if rw is not None else None, rw_dtype, mode,
-                          rw.stride(0) if rw is not None else 1,
+                          rw.data_ptr() if rw is not None else None, rw_dtype, mode, rw_stride,
                           float(beta), int(linear_beta is not None),
                           float(linear_beta) if linear_beta is not None else 0.0,
                           go2.data_ptr(), go2.stride(0) if tokens > 1 else inter,
                           dg2.data_ptr(), dg2.stride(0) if tokens > 1 else 2 * inter,
-                          d_rw_flat.data_ptr() if d_rw_flat is not None else None,
-                          d_rw_flat.stride(0) if d_rw_flat is not None else 1,
+                          d_rw_flat.data_ptr() if d_rw_flat is not None else None, d_rw_stride,
                           workspace.data_ptr() if ws_bytes else None, ws_bytes,
                           _stream_handle(stream))
     abi.check(st, "situ_glu_bwd")
@@ -188,7 +199,8 @@ def weighted_situ(gate_up: torch.Tensor, routing_weights, beta: float = DEFAULT_
                   linear_beta: float | None = DEFAULT_LINEAR_BETA) -> torch.Tensor:
     """Apply SiTU-GLU and routing weights to gate_up [..., 2 * intermediate]
     (NeMo `_weighted_situ`): gate in the first half, up in the second.
-    routing_weights: [..., 1] row-aligned, one broadcast value, or None."""
+    routing_weights: [..., 1] row-aligned, one broadcast value, [I] per
+    column, [..., I] per element, or None."""
     return WeightedSiTUFunction.apply(gate_up, routing_weights, beta, linear_beta)
 
 

@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define SITU_GLU_ABI_VERSION 1
+#define SITU_GLU_ABI_VERSION 2
 
 typedef enum situ_status {
   SITU_OK = 0,
@@ -71,8 +71,12 @@ typedef enum situ_dtype {
 typedef enum situ_rw_mode {
   SITU_RW_ROW = 0,    /* one weight per row: w[row * rw_stride], gradient per row   */
   SITU_RW_SCALAR = 1, /* one weight for every row: w[0]                             */
-  SITU_RW_NONE = 2    /* unweighted SiTU-GLU (w = 1; Megatron-LM PR #6673 "Design":
+  SITU_RW_NONE = 2,   /* unweighted SiTU-GLU (w = 1; Megatron-LM PR #6673 "Design":
                          the TE SiTUGLU op / `situlu`).  rw and d_rw must be NULL. */
+  SITU_RW_COL = 3,    /* one weight per column, shared by every row: w[i], contiguous
+                         [inter]; its gradient is the sum over rows (needs workspace) */
+  SITU_RW_FULL = 4    /* one weight per element: w[r * rw_stride + i], [tokens, >= inter]
+                         (rw_stride = row pitch in elements); gradient per element */
 } situ_rw_mode_t;
 
 /*
@@ -89,8 +93,14 @@ typedef enum situ_rw_mode {
  *   inter              I, > 0.  inter * sizeof(dtype) must be a multiple of 16
  *                      (bf16: I % 8 == 0, fp32: I % 4 == 0).
  *   rw, rw_dtype       routing weights (bf16 or fp32), laid out per rw_mode;
- *                      rw_stride (elements, >= 0; 0 repeats w[0] on every row,
- *                      as an expanded tensor does) is used by SITU_RW_ROW only.
+ *                      rw_stride (elements): SITU_RW_ROW >= 0 (0 repeats w[0] on
+ *                      every row, as an expanded tensor does); SITU_RW_FULL the
+ *                      row pitch, >= inter; ignored otherwise.  SITU_RW_COL and
+ *                      SITU_RW_FULL read the weights of one 16-byte vector of
+ *                      gate_up in one piece: rw (and the FULL row pitch) must
+ *                      be aligned to min(16, 16 / sizeof(dtype) * sizeof(rw_dtype))
+ *                      bytes -- 16, or 8 for bf16 weights with fp32 gate_up.
+ *                      SITU_RW_COL supports inter <= 16384.
  *   beta               gate beta, finite and > 0 (Megatron-LM PR #6673
  *                      "Design": finite positive betas).  Kimi-K3 default 4.
  *   has_linear_beta    0: T_u = U.  1: linear_beta is used, finite and > 0
@@ -117,7 +127,9 @@ situ_status_t situ_glu_fwd(const void *gate_up, situ_dtype_t dtype, int64_t toke
  *   d_gate_up[r, I:2I] = go * w * T_g * T_u'
  *   d_rw               = sum over columns of go * T_g * T_u: per row for
  *                        SITU_RW_ROW; summed over every row as well for
- *                        SITU_RW_SCALAR (autograd's sum to the weight's shape).
+ *                        SITU_RW_SCALAR (autograd's sum to the weight's shape);
+ *                        per column, summed over rows, for SITU_RW_COL; the
+ *                        term go * T_g * T_u itself for SITU_RW_FULL.
  * Defined by: NeMo kimi_k3.situ `_situ_bwd_core` (d_g, d_u, red; want_drw)
  * and `_WeightedSiTUFunction.backward` (returns d_gate_up, d_routing_weights).
  *
@@ -126,14 +138,17 @@ situ_status_t situ_glu_fwd(const void *gate_up, situ_dtype_t dtype, int64_t toke
  *                      d_gate_up_row_stride.  Written; must not overlap any input.
  *   d_rw               NULL: the routing-weight gradient is not wanted and no
  *                      reduction runs (`want_drw` = false).  Otherwise in
- *                      rw_dtype: element r at d_rw[r * d_rw_stride] (row mode)
- *                      or one element (scalar mode).  Must be NULL for
+ *                      rw_dtype, shaped like rw: element r at d_rw[r * d_rw_stride]
+ *                      (row mode), one element (scalar mode), [inter] contiguous
+ *                      (column mode, sums over rows), or element (r, i) at
+ *                      d_rw[r * d_rw_stride + i] (full mode; d_rw_stride >= inter,
+ *                      base and row pitch aligned like rw's).  Must be NULL for
  *                      SITU_RW_NONE.
- *   workspace          scratch for SITU_RW_SCALAR with d_rw != NULL: at least
- *                      situ_glu_bwd_workspace_bytes() bytes, 16-byte aligned,
- *                      device memory owned by the caller, contents ignored on
- *                      entry and undefined on exit.  May be NULL when that
- *                      query returns 0.
+ *   workspace          scratch for SITU_RW_SCALAR and SITU_RW_COL with
+ *                      d_rw != NULL: at least situ_glu_bwd_workspace_bytes()
+ *                      bytes, 16-byte aligned, device memory owned by the caller,
+ *                      contents ignored on entry and undefined on exit.  May be
+ *                      NULL when that query returns 0.
  * Other arguments as for situ_glu_fwd.  Per-row reductions run in a fixed
  * order, so every output is bitwise reproducible for a given build, shape and
  * load path, whatever the launch size.  dG and dU do not depend on the load
@@ -150,9 +165,11 @@ situ_status_t situ_glu_bwd(const void *gate_up, situ_dtype_t dtype, int64_t toke
                            void *workspace, size_t workspace_bytes,
                            void *stream);
 
-/* Bytes of workspace situ_glu_bwd needs: tokens * 4 rounded up to 256 for
- * SITU_RW_SCALAR with want_drw != 0, otherwise 0.  Negative tokens give 0. */
-size_t situ_glu_bwd_workspace_bytes(int64_t tokens, situ_rw_mode_t rw_mode, int want_drw);
+/* Bytes of workspace situ_glu_bwd needs with want_drw != 0: tokens * 4 for
+ * SITU_RW_SCALAR (one partial per row), ceil(tokens / 64) * inter * 4 for
+ * SITU_RW_COL (one partial per column per block of 64 rows), each rounded up
+ * to 256; otherwise 0.  Non-positive tokens or inter give 0. */
+size_t situ_glu_bwd_workspace_bytes(int64_t tokens, int64_t inter, situ_rw_mode_t rw_mode, int want_drw);
 
 /* Static, human-readable name of a status code. */
 const char *situ_glu_status_string(situ_status_t status);
@@ -198,9 +215,10 @@ int situ_glu_device_status(int clear);
  * needs scratch: a routing weight broadcast to every row (SITU_RW_SCALAR with
  * d_rw != NULL), whose per-row partial sums then go to a fixed 1 MiB array
  * inside this library instead of a caller workspace.
- *   - Limit: 262144 rows in that mode; more returns SITU_ERR_UNSUPPORTED
- *     before anything is launched.  Other modes need no scratch and have no
- *     row limit beyond situ_glu_bwd's.
+ *   - Limit: 1 MiB of scratch -- 262144 rows in that mode (per-column
+ *     weights, SITU_RW_COL, use it too: ceil(tokens / 64) * inter * 4 bytes);
+ *     more returns SITU_ERR_UNSUPPORTED before anything is launched.  Other
+ *     modes need no scratch and have no limit beyond situ_glu_bwd's.
  *   - Allocates nothing (no cudaMalloc, cudaFree or allocating library call).
  *     The array exists once per GPU that loads the library, until exit.
  *   - The first call on a device looks up the array's device address (with

@@ -107,7 +107,7 @@ def call_bwd(gu: torch.Tensor, inter: int, rw, rw_mode: int, beta: float, lb, go
     tokens = gu.shape[0]
     rw_ptr = rw.data_ptr() if rw is not None else None
     rw_dt = dtype_code(rw) if rw is not None else abi.SITU_DTYPE_F32
-    ws_bytes = abi.situ_glu_bwd_workspace_bytes(tokens, rw_mode, int(d_rw is not None))
+    ws_bytes = abi.situ_glu_bwd_workspace_bytes(tokens, inter, rw_mode, int(d_rw is not None))
     ws_ptr = None
     if ws_bytes:
         if workspace is None:

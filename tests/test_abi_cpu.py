@@ -58,19 +58,26 @@ def test_binding_covers_the_header_exactly():
 
 
 def test_version_and_status_strings(native_lib_path):
-    assert abi.situ_glu_abi_version() == abi.ABI_VERSION == 1
+    assert abi.situ_glu_abi_version() == abi.ABI_VERSION == 2
     assert abi.situ_glu_status_string(OK) == "SITU_OK"
     assert abi.situ_glu_status_string(MISAL) == "SITU_ERR_MISALIGNED"
     assert abi.situ_glu_status_string(99) == "SITU_ERR_UNKNOWN"
 
 
 def test_workspace_query(native_lib_path):
-    assert abi.situ_glu_bwd_workspace_bytes(1000, ROW, 1) == 0
-    assert abi.situ_glu_bwd_workspace_bytes(1000, SCALAR, 0) == 0
-    assert abi.situ_glu_bwd_workspace_bytes(1000, SCALAR, 1) == 4096
-    assert abi.situ_glu_bwd_workspace_bytes(64, SCALAR, 1) == 256
-    assert abi.situ_glu_bwd_workspace_bytes(0, SCALAR, 1) == 0
-    assert abi.situ_glu_bwd_workspace_bytes(-5, SCALAR, 1) == 0
+    COL, FULL = abi.SITU_RW_COL, abi.SITU_RW_FULL
+    assert abi.situ_glu_bwd_workspace_bytes(1000, 64, ROW, 1) == 0
+    assert abi.situ_glu_bwd_workspace_bytes(1000, 64, FULL, 1) == 0
+    assert abi.situ_glu_bwd_workspace_bytes(1000, 64, SCALAR, 0) == 0
+    assert abi.situ_glu_bwd_workspace_bytes(1000, 64, SCALAR, 1) == 4096
+    assert abi.situ_glu_bwd_workspace_bytes(64, 64, SCALAR, 1) == 256
+    assert abi.situ_glu_bwd_workspace_bytes(0, 64, SCALAR, 1) == 0
+    assert abi.situ_glu_bwd_workspace_bytes(-5, 64, SCALAR, 1) == 0
+    # per-column weights: one partial per column per chunk of 16 rows
+    assert abi.situ_glu_bwd_workspace_bytes(1000, 64, COL, 1) == 63 * 64 * 4
+    assert abi.situ_glu_bwd_workspace_bytes(65, 520, COL, 1) == (5 * 520 * 4 + 255) // 256 * 256
+    assert abi.situ_glu_bwd_workspace_bytes(1000, 64, COL, 0) == 0
+    assert abi.situ_glu_bwd_workspace_bytes(1000, 0, COL, 1) == 0
 
 
 def test_load_path_knob(native_lib_path):
@@ -106,6 +113,13 @@ def bwd(**kw):
 FWD_CASES = [
     ("bad dtype", dict(dtype=7), INVALID),
     ("bad rw_mode", dict(rw_mode=9), INVALID),
+    ("full weights: stride short", dict(rw_mode=4, rw_stride=63), INVALID),
+    ("full weights misaligned", dict(rw_mode=4, rw_stride=64, rw=RW + 4), MISAL),
+    ("full weights pitch misaligned", dict(rw_mode=4, rw_stride=65), MISAL),
+    ("full bf16 weights, fp32 gate_up: pitch not 8-byte", dict(dtype=1, rw_dtype=0, rw_mode=4, rw_stride=66), MISAL),
+    ("column weights misaligned", dict(rw_mode=3, rw=RW + 8), MISAL),
+    ("column weights: inter too large", dict(rw_mode=3, inter=1 << 15, gate_up_row_stride=1 << 16,
+                                              out_row_stride=1 << 15), UNSUP),
     ("bad rw_dtype", dict(rw_dtype=3), INVALID),
     ("negative tokens", dict(tokens=-1), INVALID),
     ("zero inter", dict(inter=0), INVALID),
@@ -147,6 +161,9 @@ BWD_CASES = [
     ("d_rw when unweighted", dict(rw=None, rw_mode=NONE), INVALID),
     ("d_rw stride zero", dict(d_rw_stride=0), INVALID),
     ("scalar without workspace", dict(rw_mode=SCALAR), INVALID),
+    ("column weights without workspace", dict(rw_mode=3), INVALID),
+    ("full weights: d_rw stride short", dict(rw_mode=4, rw_stride=64, d_rw_stride=63), INVALID),
+    ("full weights: d_rw overlaps rw", dict(rw_mode=4, rw_stride=64, d_rw_stride=64, d_rw=RW + 256), INVALID),
     ("scalar workspace short", dict(rw_mode=SCALAR, workspace=WS, workspace_bytes=32), INVALID),
     ("scalar workspace misaligned", dict(rw_mode=SCALAR, workspace=WS + 4, workspace_bytes=256), MISAL),
     ("grad_out NULL", dict(grad_out=None), INVALID),
@@ -177,15 +194,23 @@ def test_zero_tokens_launch_nothing(native_lib_path):
 def test_binding_routing_modes():
     import torch
     from ffn_gated_activation_b200.functional import routing_mode
-    lead = (4, 6)
-    assert routing_mode(lead, None)[0] == NONE
-    assert routing_mode(lead, torch.tensor(0.5))[0] == SCALAR
-    assert routing_mode(lead, torch.ones(1, 1, 1))[0] == SCALAR
-    m, flat = routing_mode(lead, torch.ones(4, 6, 1))
-    assert m == ROW and flat.shape == (24,)
-    assert routing_mode(lead, torch.ones(4, 6))[0] == ROW
-    with pytest.raises(NotImplementedError):
-        routing_mode(lead, torch.ones(4, 6, 8))
+    lead, inter = (4, 6), 16
+    COL, FULL = abi.SITU_RW_COL, abi.SITU_RW_FULL
+    assert routing_mode(lead, inter, None)[0] == NONE
+    assert routing_mode(lead, inter, torch.tensor(0.5))[0] == SCALAR
+    assert routing_mode(lead, inter, torch.ones(1, 1, 1))[0] == SCALAR
+    m, flat, stride = routing_mode(lead, inter, torch.ones(4, 6, 1))
+    assert m == ROW and flat.shape == (24,) and stride == 1
+    # a column slice of top-k weights: rows 8 elements apart
+    m, flat, stride = routing_mode(lead, inter, torch.ones(4, 6, 8)[..., 2:3])
+    assert m == ROW and stride == 8
+    assert routing_mode(lead, inter, torch.ones(16))[0] == COL
+    assert routing_mode(lead, inter, torch.ones(1, 1, 16))[0] == COL
+    m, w2, stride = routing_mode(lead, inter, torch.ones(4, 6, 16))
+    assert m == FULL and w2.shape == (24, 16) and stride == 16
+    for bad in (torch.ones(4, 6), torch.ones(4, 6, 8), torch.ones(6, 16)):
+        with pytest.raises(NotImplementedError):  # none of these broadcast as a per-row / column / element weight
+            routing_mode(lead, inter, bad)
 
 
 def test_binding_validates_betas():

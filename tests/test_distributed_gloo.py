@@ -95,6 +95,32 @@ def _dp_scalar_check(rank, T, I, seed):
     assert abs(t.item() - total) <= 1e-12 * mag
 
 
+def _col_weight_check(rank, T, I, seed):
+    """Per-column weights: row shards all-reduce their [I] partials; column
+    shards own their slice of the gradient outright."""
+    import oracle
+    import workloads
+    import dataclasses
+    wl = dataclasses.replace(workloads.workload(0), tokens=T, inter=I, seed=seed)
+    x = workloads.inputs(wl)
+    o = oracle.load()
+    full, mag = o.dw_columns(x["gate_up"], x["grad_out"], 4.0, 25.0)
+    r0, r1 = D.shard_range(T, rank, WORLD)
+    part, _ = o.dw_columns(x["gate_up"][r0:r1], x["grad_out"][r0:r1], 4.0, 25.0)
+    t = torch.tensor(part, dtype=torch.float64)
+    D.allreduce_drw(t)
+    assert np.all(np.abs(t.numpy() - full) <= 1e-12 * mag)
+    # tensor parallel: the rank's columns of gate_up / grad_out give its columns of d_w exactly
+    gu_local = _bits(D.tp_local_gate_up(_bf16_tensor(x["gate_up"]), rank, WORLD))
+    go_local = _bits(D.tp_local_columns(_bf16_tensor(x["grad_out"]), rank, WORLD))
+    a, b = D.shard_range(I, rank, WORLD, align=8)
+    loc, _ = o.dw_columns(gu_local, go_local, 4.0, 25.0)
+    assert np.array_equal(loc, full[a:b])
+    rw_local = torch.ones(b - a)
+    assert not D.tp_drw_needs_allreduce((T,), b - a, rw_local)
+    assert D.tp_drw_needs_allreduce((T,), b - a, torch.ones(T, 1))
+
+
 def _max_check(rank):
     assert D.max_over_ranks(1.5 + rank) == 2.5
 
@@ -105,6 +131,18 @@ def test_tensor_parallel_backward_gloo():
 
 def test_data_parallel_broadcast_weight_gloo():
     _run(_dp_scalar_check, 61, 64, 12)
+
+
+def test_column_weight_gradient_gloo():
+    _run(_col_weight_check, 45, 136, 13)
+
+
+def test_tp_drw_reduction_by_weight_shape():
+    lead, i_local = (6, 5), 24
+    assert D.tp_drw_needs_allreduce(lead, i_local, torch.ones(6, 5, 1))
+    assert D.tp_drw_needs_allreduce(lead, i_local, torch.tensor(2.0))
+    assert not D.tp_drw_needs_allreduce(lead, i_local, torch.ones(i_local))
+    assert not D.tp_drw_needs_allreduce(lead, i_local, torch.ones(6, 5, i_local))
 
 
 def test_max_over_ranks_gloo():

@@ -69,3 +69,14 @@ def test_algorithmic_bytes():
     assert workloads.workload(2).fwd_bytes() == 402_784_256
     assert workloads.workload(3).bwd_bytes() == 1_342_308_352
     assert workloads.workload(4).fwd_bytes() == 3_221_749_760
+
+
+def test_elementwise_weight_generators_are_prefix_stable():
+    wl = workloads.workload(0)
+    a = workloads.element_weights(wl, tokens=130, inter=24)
+    b = workloads.element_weights(wl, tokens=70, inter=24)
+    assert a.dtype == np.float32 and a.shape == (130, 24)
+    assert np.array_equal(a[:70], b)
+    assert np.all((a >= 0) & (a < 1))
+    c = workloads.column_weights(wl, inter=24)
+    assert c.shape == (24,) and np.array_equal(c, workloads.column_weights(wl, inter=24))

@@ -53,6 +53,26 @@ def test_matches_workspace_entry_point_twice(dtype, cuda_device):
         assert da == db  # same kernels, same fixed reduction order
 
 
+def test_per_column_weights_use_the_fixed_scratch(cuda_device):
+    """[I] weights keep one partial per column per 16-row chunk in the scratch."""
+    dev = cuda_device
+    T, I = 300, 520
+    gu_h, _, go_h = case_inputs("bf16", T, I, seed=960)
+    gu, go = to_device(gu_h, dev), to_device(go_h, dev)
+    w = torch.linspace(0.1, 1.0, I, device=dev)
+    ref_dgu = Guarded(T, 2 * I, 2 * I, torch.bfloat16, dev)
+    ref_dw = torch.empty(I, dtype=torch.float32, device=dev)
+    abi.check(call_bwd(gu, I, w, abi.SITU_RW_COL, 4.0, 25.0, go, ref_dgu, d_rw=ref_dw), "situ_glu_bwd")
+    for _ in range(2):
+        out_dgu = Guarded(T, 2 * I, 2 * I, torch.bfloat16, dev)
+        out_dw = torch.full((I,), float("nan"), device=dev)
+        abi.check(no_alloc_bwd(gu, I, w, abi.SITU_RW_COL, 4.0, 25.0, go, out_dgu, out_dw), "situ_glu_bwd_no_alloc")
+        torch.cuda.synchronize()
+        out_dgu.check()
+        assert torch.equal(out_dgu.view.view(torch.int16), ref_dgu.view.view(torch.int16))
+        assert torch.equal(out_dw, ref_dw)
+
+
 def test_row_mode_needs_no_scratch(cuda_device):
     dev = cuda_device
     T, I = 129, 264
@@ -82,3 +102,18 @@ def test_rejects_rows_beyond_the_fixed_scratch(cuda_device):
     assert "fixed scratch" in abi.situ_glu_last_error()
     torch.cuda.synchronize()
     assert d_w.item() == 5.0  # nothing was launched
+
+
+def test_rejects_per_column_partials_beyond_the_fixed_scratch(cuda_device):
+    dev = cuda_device
+    T, I = 16 * 65, 4096  # 65 chunks x 4096 columns x 4 bytes > 1 MiB
+    gu = torch.zeros(T, 2 * I, dtype=torch.bfloat16, device=dev)
+    go = torch.zeros(T, I, dtype=torch.bfloat16, device=dev)
+    w = torch.ones(I, dtype=torch.float32, device=dev)
+    dgu = Guarded(T, 2 * I, 2 * I, torch.bfloat16, dev)
+    d_w = torch.full((I,), 5.0, device=dev)
+    st = no_alloc_bwd(gu, I, w, abi.SITU_RW_COL, 4.0, 25.0, go, dgu, d_w)
+    assert st == abi.SITU_ERR_UNSUPPORTED
+    assert "fixed scratch" in abi.situ_glu_last_error()
+    torch.cuda.synchronize()
+    assert torch.all(d_w == 5.0)

@@ -27,6 +27,8 @@ BLOCK_ROWS = 64
 TENSOR_GATE_UP = 1
 TENSOR_ROUTING = 2
 TENSOR_GRAD_OUT = 3
+TENSOR_COL_WEIGHTS = 4
+TENSOR_ELEM_WEIGHTS = 5
 
 
 @dataclass(frozen=True)
@@ -212,6 +214,29 @@ def routing_weights(wl: Workload, tokens: int | None = None) -> np.ndarray:
             probs[t0:t0 + n] = np.take_along_axis(p, order, axis=1)
         return probs.reshape(-1)[:tokens].astype(np.float32)
     raise ValueError(f"unknown routing-weight kind {wl.rw_kind!r}")
+
+
+def column_weights(wl: Workload, inter: int | None = None) -> np.ndarray:
+    """Per-column routing weights [I] float32 ~ U(0, 1): one weight shared by
+    every row of a column (the [I] broadcast form of routing_weights)."""
+    inter = wl.inter if inter is None else inter
+    return _rng(wl.seed, TENSOR_COL_WEIGHTS, 0).random(inter).astype(np.float32)
+
+
+def element_weights(wl: Workload, tokens: int | None = None, inter: int | None = None) -> np.ndarray:
+    """Per-element routing weights [T, I] float32 ~ U(0, 1), drawn in whole
+    64-row blocks like gate_up."""
+    tokens = wl.tokens if tokens is None else tokens
+    inter = wl.inter if inter is None else inter
+    out = np.empty((tokens, inter), dtype=np.float32)
+
+    def fill(b):
+        r0 = b * BLOCK_ROWS
+        n = min(BLOCK_ROWS, tokens - r0)
+        out[r0:r0 + n] = _rng(wl.seed, TENSOR_ELEM_WEIGHTS, b).random((BLOCK_ROWS, inter))[:n]
+
+    _fill_blocks(tokens, fill)
+    return out
 
 
 def inputs(wl: Workload, tokens: int | None = None, inter: int | None = None) -> dict:
