@@ -5,9 +5,9 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 (``ffn_gated_activation_b200``) never imports it, and it never imports the
 product path: the two share no code.
 
-The arithmetic lives in ``situ_oracle.c`` (plain C, IEEE double, one element
-at a time); this module only builds that file with gcc and marshals numpy
-arrays through ctypes.
+The arithmetic lives in ``situ_oracle.c`` and ``mx_oracle.c`` (plain C, IEEE
+double, one element at a time); this module only builds them with gcc and
+marshals numpy arrays through ctypes.
 
 Sources followed (see the C file for the per-function citations):
   * Megatron-LM PR #6673 "[Dev] Add SiTU-GLU through Transformer Engine",
@@ -16,6 +16,9 @@ Sources followed (see the C file for the per-function citations):
   * NeMo AutoModel API, kimi_k3.situ: `_situ_fwd_core` (Y = situ(g) up(u0) w,
     optional linear beta), `_situ_bwd_core` (analytic d_g, d_u and the
     routing-weight reduction), `_WeightedSiTUFunction` (gate/up halves).
+  * OCP Microscaling Formats (MX) v1.0 for the MXFP8 outputs (E4M3 elements,
+    E8M0 block scales, blocks of 32), the format of the MXFP8 recipe named in
+    Megatron-LM PR #6673 "Test results".
 
 Every function is pinned by tests/test_oracle_pins.py; no function here is
 "parity unpinned".
@@ -31,6 +34,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 SOURCE = os.path.join(_HERE, "situ_oracle.c")
+MX_SOURCE = os.path.join(_HERE, "mx_oracle.c")  # MXFP8 block scaling (OCP MX v1.0)
 LIBRARY = os.path.join(_HERE, "libsitu_oracle.so")
 
 DTYPE_BF16 = 0
@@ -39,6 +43,10 @@ RW_ROW = 0     # w[T] (or [T, 1]): one weight per row
 RW_SCALAR = 1  # one weight for every element
 RW_COL = 2     # w[I]: one weight per column, every row
 RW_FULL = 3    # w[T, I]: one weight per element
+MX_BLOCK = 32         # MXFP8: elements per shared scale
+MX_RULE_OCP = 0       # e = floor(log2 amax) - 8, elements clamped to +-448
+MX_RULE_CEIL = 1      # smallest e with amax <= 448 * 2^e
+MX_SCALE_NAN = 128    # mx_scale_exp's value for a NaN scale (scale byte 255)
 
 # gcc flags: plain IEEE double, no fast-math, no contraction into FMA, so the
 # arithmetic is exactly what the C source spells out.
@@ -50,10 +58,10 @@ def build(output: str = LIBRARY, mutant: int = 0, force: bool = False) -> str:
     copy with the planted mistake number ``mutant`` (used only by the pin tests
     to show the pins reject it).  Rebuilds when the source is newer."""
     if (not force and os.path.exists(output)
-            and os.path.getmtime(output) >= os.path.getmtime(SOURCE)):
+            and os.path.getmtime(output) >= max(os.path.getmtime(SOURCE), os.path.getmtime(MX_SOURCE))):
         return output
     tmp = output + f".tmp{os.getpid()}"
-    cmd = ["gcc", *CFLAGS, f"-DSITU_ORACLE_MUTANT={int(mutant)}", SOURCE, "-o", tmp, "-lm"]
+    cmd = ["gcc", *CFLAGS, f"-DSITU_ORACLE_MUTANT={int(mutant)}", SOURCE, MX_SOURCE, "-o", tmp, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, output)
     return output
@@ -114,6 +122,14 @@ class Oracle:
         lib.situ_oracle_dw_terms.argtypes = [_INT, _VP, _I64, _I64, _VP, _I64, _DBL, _INT, _DBL, _VP, _I64, _VP]
         lib.situ_oracle_dw_terms.restype = _INT
         lib.situ_oracle_mutant_id.restype = _INT
+        lib.situ_oracle_e4m3_encode.argtypes = [_DBL]
+        lib.situ_oracle_e4m3_encode.restype = _INT
+        lib.situ_oracle_e4m3_decode.argtypes = [_INT]
+        lib.situ_oracle_e4m3_decode.restype = _DBL
+        lib.situ_oracle_mx_scale_exp.argtypes = [_DBL, _INT]
+        lib.situ_oracle_mx_scale_exp.restype = _INT
+        lib.situ_oracle_mxfp8_quantize.argtypes = [_VP, _I64, _I64, _I64, _INT, _VP, _VP]
+        lib.situ_oracle_mxfp8_quantize.restype = _INT
         self._lib = lib
         self.mutant_id = lib.situ_oracle_mutant_id()
 
@@ -232,6 +248,35 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle dw_scalar rejected its arguments")
         return total.value, mag.value
+
+
+    # -- MXFP8 block scaling (mx_oracle.c) -------------------------------------
+
+    def e4m3_encode(self, x) -> np.ndarray:
+        """E4M3 codes (uint8) of reals x: nearest-even, clamped to +-448."""
+        x = np.asarray(x, dtype=np.float64)
+        f = self._lib.situ_oracle_e4m3_encode
+        return np.array([f(float(v)) for v in x.reshape(-1)], dtype=np.uint8).reshape(x.shape)
+
+    def e4m3_decode(self, codes) -> np.ndarray:
+        c = np.asarray(codes, dtype=np.uint8)
+        f = self._lib.situ_oracle_e4m3_decode
+        return np.array([f(int(v)) for v in c.reshape(-1)], dtype=np.float64).reshape(c.shape)
+
+    def mx_scale_exp(self, amax: float, rule: int = MX_RULE_OCP) -> int:
+        """Shared exponent of a block with largest magnitude amax (MX_SCALE_NAN for NaN)."""
+        return self._lib.situ_oracle_mx_scale_exp(float(amax), int(rule))
+
+    def mxfp8_quantize(self, v, rule: int = MX_RULE_OCP):
+        """(codes [R, C] uint8, scale bytes [R, C / 32] uint8) of the fp64 matrix v."""
+        v = np.ascontiguousarray(np.asarray(v, dtype=np.float64))
+        rows, cols = v.shape
+        codes = np.empty((rows, cols), dtype=np.uint8)
+        scales = np.empty((rows, cols // MX_BLOCK), dtype=np.uint8)
+        rc = self._lib.situ_oracle_mxfp8_quantize(_ptr(v), rows, cols, cols, int(rule), _ptr(codes), _ptr(scales))
+        if rc != 0:
+            raise ValueError("oracle mxfp8_quantize: columns must be a multiple of 32")
+        return codes, scales
 
 
 _DEFAULT = None

@@ -15,7 +15,9 @@ itself checked here against things other than itself:
   * torch float64 autograd of the formula for whole rows (independent
     derivatives, strided rows, both dtypes, both routing-weight modes);
   * special rows (G = 0, U = 0) whose gradients have closed forms;
-  * brute-force compensated sums for the routing-weight gradient.
+  * brute-force compensated sums for the routing-weight gradient;
+  * MXFP8 (mx_oracle.c): torch's float8_e4m3fn encoding and decoding, the
+    OCP MX format's clamp at 448, and the scale rules' defining inequalities.
 
 Each pin is a plain function of an oracle handle.  ``test_mutant_rejected``
 rebuilds situ_oracle.c with each planted mistake (-DSITU_ORACLE_MUTANT=n: a
@@ -322,6 +324,100 @@ def pin_bf16_loading(o):
     assert _close(y[0, 0], float(_mp_gate(1.0, 4.0) * _mp_up(1.0, 25.0)), 4e-15)
 
 
+# ---- MXFP8 block scaling (mx_oracle.c, OCP MX v1.0) -----------------------------
+
+def pin_e4m3_decode_torch(o):
+    """All 256 E4M3 codes decode to the values torch's float8_e4m3fn gives them."""
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = o.e4m3_decode(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert np.array_equal(np.signbit(got[ok]), np.signbit(ref[ok]))
+
+
+def pin_e4m3_encode_torch(o):
+    """Nearest-even encoding against torch's float32 -> float8_e4m3fn conversion:
+    every finite bf16 value with |x| <= 464 (above that torch overflows to NaN
+    where the MX conversion clamps) and random fp32 values from the subnormals
+    (below 2^-6) to the top binade."""
+    x = workloads.bf16_bits_to_f32(np.arange(1 << 16, dtype=np.uint32).astype(np.uint16))
+    x = x[np.isfinite(x) & (np.abs(x) <= 464.0)]
+    rng = np.random.default_rng(RNG_SEED)
+    y = (rng.standard_normal(20000) * np.exp2(rng.integers(-14, 9, 20000))).astype(np.float32)
+    v = np.concatenate([x, y[np.abs(y) <= 464.0]])
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = o.e4m3_encode(v.astype(np.float64))
+    bad = np.flatnonzero(got != ref)
+    assert bad.size == 0, (v[bad[:5]], got[bad[:5]], ref[bad[:5]])
+
+
+def pin_e4m3_saturation(o):
+    """E4M3 has no infinities: the MX conversion clamps magnitudes at or above
+    its largest normal 448 (code 0x7E) to +-448; NaN stays NaN."""
+    got = o.e4m3_encode([448.0, 449.0, 470.0, 1e9, float("inf"), -500.0, -float("inf")])
+    assert list(got) == [0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE], list(got)
+    assert (int(o.e4m3_encode([float("nan")])[0]) & 0x7F) == 0x7F
+
+
+def pin_mx_scale_rules(o):
+    """Shared exponents.  The spec's rule makes the block maximum land in
+    [2^8, 2^9) after scaling (floor(log2 amax) - 8); the no-clamp rule takes
+    the smallest power of two with amax / X <= 448, so amax / X > 224.  Closed
+    forms at the boundaries; zero, tiny, NaN and infinite blocks."""
+    OCP, CEIL = oracle.MX_RULE_OCP, oracle.MX_RULE_CEIL
+    cases = {1.0: (-8, -8), 448.0: (0, 0), 500.0: (0, 1), 511.0: (0, 1), 512.0: (1, 1), 224.0: (-1, -1),
+             224.5: (-1, 0), 0.0: (-127, -127), 2.0 ** -140: (-127, -127), 1.99 * 2.0 ** 127: (119, 120)}
+    for amax, (e_ocp, e_ceil) in cases.items():
+        assert o.mx_scale_exp(amax, OCP) == e_ocp, (amax, o.mx_scale_exp(amax, OCP))
+        assert o.mx_scale_exp(amax, CEIL) == e_ceil, (amax, o.mx_scale_exp(amax, CEIL))
+    for bad in (float("nan"), float("inf")):
+        assert o.mx_scale_exp(bad, OCP) == oracle.MX_SCALE_NAN
+    rng = np.random.default_rng(RNG_SEED + 1)
+    for amax in np.exp2(rng.uniform(-118.0, 120.0, 4000)):
+        r = amax / 2.0 ** o.mx_scale_exp(amax, OCP)
+        assert 256.0 <= r < 512.0, (amax, r)
+        r = amax / 2.0 ** o.mx_scale_exp(amax, CEIL)
+        assert 224.0 < r <= 448.0, (amax, r)
+
+
+def pin_mxfp8_blocks(o):
+    """Blocks of 32 along each row: scale byte = e + 127 from the block's own
+    largest magnitude (checked by the rules' inequalities), codes = torch's E4M3
+    conversion of v / 2^e, clamped to 448 under the spec's rule.  Rows hold an
+    all-zero block, a NaN, tiny values and an outlier."""
+    rng = np.random.default_rng(RNG_SEED + 2)
+    v = (rng.standard_normal((7, 96)) * np.exp2(rng.integers(-20, 20, (7, 1)))).astype(np.float32)
+    v[1, 32:64] = 0.0
+    v[2, 5] = np.nan
+    v[3, 64:96] *= np.float32(2.0 ** -100)
+    v[4, 7] = 1e4
+    v = v.astype(np.float64)
+    for rule in (oracle.MX_RULE_OCP, oracle.MX_RULE_CEIL):
+        codes, scales = o.mxfp8_quantize(v, rule)
+        assert codes.shape == v.shape and scales.shape == (7, 3)
+        for r in range(7):
+            for b in range(3):
+                blk = v[r, 32 * b:32 * b + 32]
+                s = int(scales[r, b])
+                if np.isnan(blk).any():
+                    assert s == 255
+                    continue
+                amax = np.abs(blk).max()
+                if amax == 0.0:
+                    assert s == 0 and not np.any(codes[r, 32 * b:32 * b + 32] & 0x7F)
+                    continue
+                ratio = amax / 2.0 ** (s - 127)
+                if rule == oracle.MX_RULE_OCP:
+                    assert 256.0 <= ratio < 512.0, (r, b, ratio)
+                else:
+                    assert 224.0 < ratio <= 448.0, (r, b, ratio)
+                scaled = (blk / 2.0 ** (s - 127)).astype(np.float32)
+                ref = torch.from_numpy(np.clip(scaled, -448.0, 448.0)).to(torch.float8_e4m3fn)
+                assert np.array_equal(codes[r, 32 * b:32 * b + 32], ref.view(torch.uint8).numpy()), (r, b)
+
+
 PINS = [
     pin_gate_values_mpmath,
     pin_up_values_mpmath,
@@ -336,6 +432,11 @@ PINS = [
     pin_special_rows,
     pin_dw_bruteforce,
     pin_bf16_loading,
+    pin_e4m3_decode_torch,
+    pin_e4m3_encode_torch,
+    pin_e4m3_saturation,
+    pin_mx_scale_rules,
+    pin_mxfp8_blocks,
 ]
 
 
@@ -360,6 +461,12 @@ MUTANTS = {
     11: "sech^2 with exp(-|a|) instead of exp(-2|a|)",
     12: "row stride ignored",
     13: "per-column weight indexed by the row",
+    14: "MX shared exponent from ceil(log2 amax)",
+    15: "MX shared exponent with E4M3 emax 7",
+    16: "E4M3 overflow to NaN instead of clamping",
+    17: "E4M3 ties rounded away from zero",
+    18: "E4M3 subnormal spacing 2^-10",
+    19: "no-clamp scale rule bumps the exponent at equality",
 }
 
 
