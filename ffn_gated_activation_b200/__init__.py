@@ -15,7 +15,9 @@ from .functional import (
     DEFAULT_LINEAR_BETA,
     WeightedSiTUFunction,
     situ_glu_bwd,
+    situ_glu_bwd_mxfp8,
     situ_glu_fwd,
+    situ_glu_fwd_mxfp8,
     situlu,
     weighted_situ,
 )
@@ -30,6 +32,8 @@ __all__ = [
     "WeightedSiTUFunction",
     "situ_glu_fwd",
     "situ_glu_bwd",
+    "situ_glu_fwd_mxfp8",
+    "situ_glu_bwd_mxfp8",
     "situlu",
     "weighted_situ",
 ]

@@ -29,6 +29,7 @@
 // series of 1 - exp(-x) instead.
 
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -1206,6 +1207,359 @@ __global__ void __launch_bounds__(kMaxThreads) situ_glu_fwd_wide_kernel(const Fw
 }
 
 // ---------------------------------------------------------------------------
+// MXFP8 outputs (OCP Microscaling Formats v1.0)
+// ---------------------------------------------------------------------------
+// Y (forward) or d_gate_up (backward) leave the kernel as FP8 E4M3 codes with
+// one E8M0 scale per 32 consecutive elements of a row, the format of the
+// MXFP8 recipe the SiTU-GLU integration was tested with (Megatron-LM PR #6673,
+// "Test results").  A block is the 32 / kElems adjacent lanes that own its
+// vectors (4 for bf16 inputs, 8 for fp32); its largest magnitude is combined
+// with lane shuffles, so the fp32 values are quantised straight from
+// registers.  Shared exponent e, stored as the byte e + 127:
+//   SITU_MX_RULE_OCP:  floor(log2 amax) - 8 (the exponent of E4M3's largest
+//                      normal), elements clamped to +-448;
+//   SITU_MX_RULE_CEIL: the smallest e with amax <= 448 2^e (nothing clamps);
+// both at least -127.  Both exponents come from the bits of amax, exactly.
+// A block holding a NaN or an infinity gets scale byte 255 (NaN) and NaN codes.
+
+constexpr int kMxBlock = 32;
+
+struct MxOut {
+  char* data;            // E4M3 codes, [tokens, cols]
+  int64_t data_pitch;    // bytes
+  uint8_t* scale;        // E8M0 bytes, [tokens, cols / 32]
+  int64_t scale_pitch;   // bytes
+  int rule;              // situ_mx_rule_t
+};
+
+__device__ __forceinline__ void st_stream_u32(void* p, uint32_t v) {
+  asm volatile("st.global.cs.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Four E4M3 codes (nearest even, clamped to +-448, NaN to NaN) of a.x, a.y,
+// b.x, b.y, in that byte order.  cvt...e4m3x2 puts its first source in the
+// upper byte of the 16-bit result.
+__device__ __forceinline__ uint32_t e4m3x4(float2 a, float2 b) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
+// Where a thread's vector j of a row goes: its codes at byte kElems j of the
+// row, its block's scale byte at j / (32 / kElems) (written by the block's
+// first lane).  Computed once per thread.
+template <typename S>
+struct MxSlot {
+  int code_off;
+  int scale_off;
+  bool lead;
+  __device__ __forceinline__ explicit MxSlot(int j) {
+    constexpr int kElems = 2 * S::kPairs, kLanes = kMxBlock / kElems;
+    code_off = j * kElems;
+    scale_off = j / kLanes;
+    lead = (j % kLanes) == 0;
+  }
+};
+
+// Quantise the kPairs pairs y of one vector of a row.  Every lane of the warp
+// calls this (the block maximum is shuffled); lanes with `active` set store
+// their codes and the first lane of each block the scale byte.  A block is
+// active or inactive as a whole (rows are multiples of 32 elements).
+template <typename S, bool ACTIVE_ALWAYS = false>
+__device__ __forceinline__ void mx_store_vec(const float2 (&y)[S::kPairs], bool active, char* data_row,
+                                             uint8_t* scale_row, const MxSlot<S>& slot, int rule) {
+  constexpr int kElems = 2 * S::kPairs;
+  constexpr int kLanes = kMxBlock / kElems;
+  float amax = 0.0f;
+#pragma unroll
+  for (int p = 0; p < S::kPairs; ++p) amax = max_nan(amax, max_nan(fabsf(y[p].x), fabsf(y[p].y)));
+  if (!ACTIVE_ALWAYS && !active) amax = 0.0f;
+#pragma unroll
+  for (int o = 1; o < kLanes; o <<= 1) amax = max_nan(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const uint32_t ab = __float_as_uint(amax);
+  const int ef = static_cast<int>(ab >> 23);  // amax >= 0 (or NaN with the sign bit clear)
+  // e + 127 = (ef - 127) - 8 + 127, plus one under the no-clamp rule when the
+  // significand of amax exceeds 1.75 (448 = 1.75 2^8); zero and subnormal
+  // blocks land on the smallest scale; ef = 255 (NaN, inf) gives the NaN scale.
+  int sb = ef - 8 + ((rule == SITU_MX_RULE_CEIL && (ab & 0x7fffffu) > 0x600000u) ? 1 : 0);
+  sb = sb < 0 ? 0 : sb;
+  const bool nan_blk = ef >= 255;
+  sb = nan_blk ? 255 : sb;
+  // 2^-e as a normal float (biased exponent 254 - sb in [7, 254] for sb <= 247);
+  // a NaN block scales by NaN, so that its codes come out NaN.
+  const float inv = nan_blk ? __uint_as_float(0x7fc00000u) : __uint_as_float(static_cast<uint32_t>(254 - sb) << 23);
+  uint32_t q[S::kPairs / 2];
+#pragma unroll
+  for (int k = 0; k < S::kPairs / 2; ++k) q[k] = e4m3x4(mul2(y[2 * k], splat(inv)), mul2(y[2 * k + 1], splat(inv)));
+  if (!ACTIVE_ALWAYS && !active) return;
+  char* p = data_row + slot.code_off;
+  if constexpr (kElems == 8)
+    st_stream8(p, make_uint2(q[0], q[1]));
+  else
+    st_stream_u32(p, q[0]);
+  if (slot.lead) scale_row[slot.scale_off] = static_cast<uint8_t>(sb);
+}
+
+template <typename S, int GATE, bool HAS_LB>
+__device__ __forceinline__ void fwd_pairs(const uint4& gv, const uint4& uv, float2 wbb, const Coeffs& c,
+                                          float2 (&y)[S::kPairs]) {
+#pragma unroll
+  for (int p = 0; p < S::kPairs; ++p) {
+    if constexpr (std::is_same<S, Bf16>::value)
+      y[p] = fwd_pair_bf16<GATE, HAS_LB>(S::pair(gv, p), S::pair(uv, p), wbb, c);
+    else
+      y[p] = fwd_pair_abs<GATE, HAS_LB, S>(S::pair(gv, p), S::pair(uv, p), wbb, c);
+  }
+}
+
+template <typename S, int GATE, bool HAS_LB>
+__device__ __forceinline__ void bwd_pairs(const uint4& gv, const uint4& uv, const uint4& gov, float2 k,
+                                          const Coeffs& c, float2 (&dg)[S::kPairs], float2 (&du)[S::kPairs],
+                                          float2& acc) {
+  const float2 kdg = splat(k.x), kdu = splat(k.y);
+#pragma unroll
+  for (int p = 0; p < S::kPairs; ++p)
+    bwd_pair<GATE, HAS_LB, S>(S::pair(gv, p), S::pair(uv, p), as_f2(S::pair(gov, p)), kdg, kdu, c, dg[p], du[p], acc);
+}
+
+template <typename S>
+__device__ __forceinline__ void zero_y(float2 (&y)[S::kPairs]) {
+#pragma unroll
+  for (int p = 0; p < S::kPairs; ++p) y[p] = make_float2(0.0f, 0.0f);
+}
+
+// Rows of the two-vector layout; ALL: every lane owns two vectors (vpr = 2 nt),
+// so no lane is ever inactive.
+template <typename S, int GATE, bool HAS_LB, bool ALL>
+__device__ __forceinline__ void fwd_mx_rows(const FwdArgs& a, const MxOut& m) {
+  constexpr int kP = S::kPairs;
+  const int nt = blockDim.x;
+  const int j = threadIdx.x, j2 = j + nt;
+  const bool one = ALL || j < a.vpr, two = ALL || j2 < a.vpr;
+  const MxSlot<S> s0(j), s1(j2);
+  const int rule = m.rule;
+  int64_t row = blockIdx.x;
+  if (row >= a.tokens) return;
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  uint4 g0 = z, u0 = z, g1 = z, u1 = z;
+  {
+    const char* gu = a.gate_up + row * a.gu_pitch;
+    if (one) {
+      g0 = ld_stream(gu + j * kVecBytes);
+      u0 = ld_stream(gu + a.half_bytes + j * kVecBytes);
+    }
+    if (two) {
+      g1 = ld_stream(gu + j2 * kVecBytes);
+      u1 = ld_stream(gu + a.half_bytes + j2 * kVecBytes);
+    }
+  }
+  float w = load_rw(a.rw, row);
+  for (;;) {
+    const int64_t next = row + gridDim.x;
+    const bool more = next < a.tokens;
+    uint4 ng0, nu0, ng1, nu1;
+    float nw = 0.0f;
+    if (more) {
+      const char* ngu = a.gate_up + next * a.gu_pitch;
+      if (one) {
+        ng0 = ld_stream(ngu + j * kVecBytes);
+        nu0 = ld_stream(ngu + a.half_bytes + j * kVecBytes);
+      }
+      if (two) {
+        ng1 = ld_stream(ngu + j2 * kVecBytes);
+        nu1 = ld_stream(ngu + a.half_bytes + j2 * kVecBytes);
+      }
+      nw = load_rw(a.rw, next);
+    }
+    const float2 wbb = splat(w * a.c.bb);
+    char* drow = m.data + row * m.data_pitch;
+    uint8_t* srow = m.scale + row * m.scale_pitch;
+    float2 y[kP];
+    if (ALL || one) fwd_pairs<S, GATE, HAS_LB>(g0, u0, wbb, a.c, y); else zero_y<S>(y);
+    mx_store_vec<S, ALL>(y, one, drow, srow, s0, rule);
+    if (ALL || two) fwd_pairs<S, GATE, HAS_LB>(g1, u1, wbb, a.c, y); else zero_y<S>(y);
+    mx_store_vec<S, ALL>(y, two, drow, srow, s1, rule);
+    if (!more) break;
+    row = next;
+    g0 = ng0; u0 = nu0; g1 = ng1; u1 = nu1; w = nw;
+  }
+}
+
+template <typename S, int GATE, bool HAS_LB>
+__global__ void __launch_bounds__(kMaxThreads) situ_glu_fwd_mx_kernel(const FwdArgs a, const MxOut m) {
+  constexpr int kP = S::kPairs;
+  const int nt = blockDim.x;
+  if (a.vpr == 2 * nt) {
+    fwd_mx_rows<S, GATE, HAS_LB, true>(a, m);
+    return;
+  }
+  if (a.vpr < 2 * nt) {
+    fwd_mx_rows<S, GATE, HAS_LB, false>(a, m);
+    return;
+  }
+  for (int64_t row = blockIdx.x; row < a.tokens; row += gridDim.x) {
+    const char* gu = a.gate_up + row * a.gu_pitch;
+    const float2 wbb = splat(load_rw(a.rw, row) * a.c.bb);
+    char* drow = m.data + row * m.data_pitch;
+    uint8_t* srow = m.scale + row * m.scale_pitch;
+    for (int jb = 0; jb < a.vpr; jb += nt) {  // uniform trip count: every lane reaches the shuffles
+      const int j = jb + threadIdx.x;
+      const bool act = j < a.vpr;
+      float2 y[kP];
+      if (act)
+        fwd_pairs<S, GATE, HAS_LB>(ld_stream(gu + j * kVecBytes), ld_stream(gu + a.half_bytes + j * kVecBytes), wbb,
+                                   a.c, y);
+      else
+        zero_y<S>(y);
+      mx_store_vec<S>(y, act, drow, srow, MxSlot<S>(j), m.rule);
+    }
+  }
+}
+
+// Backward with MXFP8 d_gate_up: codes [tokens, 2 inter] (dG then dU), scales
+// [tokens, 2 inter / 32]; the routing-weight gradient as in the per-row kernel.
+template <typename S, int GATE, bool HAS_LB>
+__device__ __forceinline__ void bwd_mx_finish_row(const BwdArgs& a, int64_t row, float2 acc, float* red) {
+  if (a.want_drw) {  // uniform over the launch
+    const float total = block_sum(acc.x + acc.y, red) * bwd_dw_scale(a.c);
+    if (threadIdx.x == 0) {
+      if (a.rw.mode == SITU_RW_SCALAR)
+        a.partials[row] = total;
+      else
+        store_rw_grad(a.d_rw, row * a.d_rw_stride, a.rw.bf16, total);
+    }
+  }
+}
+
+// One vector's dG and dU, quantised.  dU's codes and scales sit half a row on.
+template <typename S, int GATE, bool HAS_LB, bool ALL>
+__device__ __forceinline__ void bwd_mx_vec(const uint4& g, const uint4& u, const uint4& o, bool act, float2 k,
+                                           const Coeffs& c, char* drow, uint8_t* srow, int inter,
+                                           const MxSlot<S>& slot, int rule, float2& acc) {
+  constexpr int kP = S::kPairs;
+  float2 dg[kP], du[kP];
+  if (ALL || act) {
+    bwd_pairs<S, GATE, HAS_LB>(g, u, o, k, c, dg, du, acc);
+  } else {
+    zero_y<S>(dg);
+    zero_y<S>(du);
+  }
+  mx_store_vec<S, ALL>(dg, act, drow, srow, slot, rule);
+  mx_store_vec<S, ALL>(du, act, drow + inter, srow + inter / kMxBlock, slot, rule);
+}
+
+template <typename S, int GATE, bool HAS_LB, bool ALL>
+__device__ __forceinline__ void bwd_mx_rows(const BwdArgs& a, const MxOut& m, float (*red)[kMaxThreads / 32]) {
+  constexpr int kP = S::kPairs;
+  const int nt = blockDim.x;
+  const int inter = a.half_bytes / kVecBytes * (2 * kP);  // elements per half row
+  const int j = threadIdx.x, j2 = j + nt;
+  const bool one = ALL || j < a.vpr, two = ALL || j2 < a.vpr;
+  const MxSlot<S> s0(j), s1(j2);
+  const int rule = m.rule;
+  int parity = 0;
+  int64_t row = blockIdx.x;
+  if (row >= a.tokens) return;
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  uint4 g0 = z, u0 = z, o0 = z, g1 = z, u1 = z, o1 = z;
+  {
+    const char* gu = a.gate_up + row * a.gu_pitch;
+    const char* go_row = a.grad_out + row * a.go_pitch;
+    if (one) {
+      g0 = ld_stream(gu + j * kVecBytes);
+      u0 = ld_stream(gu + a.half_bytes + j * kVecBytes);
+      o0 = ld_stream(go_row + j * kVecBytes);
+    }
+    if (two) {
+      g1 = ld_stream(gu + j2 * kVecBytes);
+      u1 = ld_stream(gu + a.half_bytes + j2 * kVecBytes);
+      o1 = ld_stream(go_row + j2 * kVecBytes);
+    }
+  }
+  float w = load_rw(a.rw, row);
+  for (;;) {
+    const int64_t next = row + gridDim.x;
+    const bool more = next < a.tokens;
+    uint4 ng0, nu0, no0, ng1, nu1, no1;
+    float nw = 0.0f;
+    if (more) {
+      const char* gu = a.gate_up + next * a.gu_pitch;
+      const char* go_row = a.grad_out + next * a.go_pitch;
+      if (one) {
+        ng0 = ld_stream(gu + j * kVecBytes);
+        nu0 = ld_stream(gu + a.half_bytes + j * kVecBytes);
+        no0 = ld_stream(go_row + j * kVecBytes);
+      }
+      if (two) {
+        ng1 = ld_stream(gu + j2 * kVecBytes);
+        nu1 = ld_stream(gu + a.half_bytes + j2 * kVecBytes);
+        no1 = ld_stream(go_row + j2 * kVecBytes);
+      }
+      nw = load_rw(a.rw, next);
+    }
+    const float2 k = bwd_row_consts<HAS_LB>(w, a.c);
+    char* drow = m.data + row * m.data_pitch;
+    uint8_t* srow = m.scale + row * m.scale_pitch;
+    float2 acc = make_float2(0.0f, 0.0f);
+    bwd_mx_vec<S, GATE, HAS_LB, ALL>(g0, u0, o0, one, k, a.c, drow, srow, inter, s0, rule, acc);
+    bwd_mx_vec<S, GATE, HAS_LB, ALL>(g1, u1, o1, two, k, a.c, drow, srow, inter, s1, rule, acc);
+    bwd_mx_finish_row<S, GATE, HAS_LB>(a, row, acc, red[parity]);
+    parity ^= 1;
+    if (!more) break;
+    row = next;
+    g0 = ng0; u0 = nu0; o0 = no0; g1 = ng1; u1 = nu1; o1 = no1; w = nw;
+  }
+}
+
+// Three CTAs of 256 threads per SM (at most 85 registers a thread): measured
+// faster on B200 than two, the issue-bound MXFP8 backward gaining more from
+// the extra warps than it loses to the tighter register budget.
+#ifndef SITU_BWD_MX_MIN_CTAS
+#define SITU_BWD_MX_MIN_CTAS 3
+#endif
+#define SITU_BWD_MX_BOUNDS __launch_bounds__(kMaxThreads, SITU_BWD_MX_MIN_CTAS)
+
+template <typename S, int GATE, bool HAS_LB>
+__global__ void SITU_BWD_MX_BOUNDS situ_glu_bwd_mx_kernel(const BwdArgs a, const MxOut m) {
+  __shared__ float red[2][kMaxThreads / 32];
+  const int nt = blockDim.x;
+  if (PipelineRows<S, true>::value && a.vpr == 2 * nt) {
+    bwd_mx_rows<S, GATE, HAS_LB, true>(a, m, red);
+    return;
+  }
+  if (PipelineRows<S, true>::value && a.vpr < 2 * nt) {
+    bwd_mx_rows<S, GATE, HAS_LB, false>(a, m, red);
+    return;
+  }
+  const int inter = a.half_bytes / kVecBytes * (2 * S::kPairs);
+  int parity = 0;
+  for (int64_t row = blockIdx.x; row < a.tokens; row += gridDim.x) {
+    const char* gu = a.gate_up + row * a.gu_pitch;
+    const char* go_row = a.grad_out + row * a.go_pitch;
+    const float2 k = bwd_row_consts<HAS_LB>(load_rw(a.rw, row), a.c);
+    char* drow = m.data + row * m.data_pitch;
+    uint8_t* srow = m.scale + row * m.scale_pitch;
+    float2 acc = make_float2(0.0f, 0.0f);
+    for (int jb = 0; jb < a.vpr; jb += nt) {  // uniform trip count: every lane reaches the shuffles
+      const int j = jb + threadIdx.x;
+      const bool act = j < a.vpr;
+      const uint4 z = make_uint4(0, 0, 0, 0);
+      bwd_mx_vec<S, GATE, HAS_LB, false>(act ? ld_stream(gu + j * kVecBytes) : z,
+                                         act ? ld_stream(gu + a.half_bytes + j * kVecBytes) : z,
+                                         act ? ld_stream(go_row + j * kVecBytes) : z, act, k, a.c, drow, srow,
+                                         inter, MxSlot<S>(j), m.rule, acc);
+    }
+    bwd_mx_finish_row<S, GATE, HAS_LB>(a, row, acc, red[parity]);
+    parity ^= 1;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // TMA-staged kernels (load path 1)
 // ---------------------------------------------------------------------------
 // Warp 0 of each CTA is a producer: one lane streams chunks of rows from HBM
@@ -1792,42 +2146,113 @@ BwdKernel pick_bwd(situ_dtype_t dtype, int gate, bool lb) {
   return lb ? pick_bwd_gate<F32, true>(gate) : pick_bwd_gate<F32, false>(gate);
 }
 
-}  // namespace
+using FwdMxKernel = void (*)(FwdArgs, MxOut);
+using BwdMxKernel = void (*)(BwdArgs, MxOut);
 
-// ---------------------------------------------------------------------------
-// C ABI
-// ---------------------------------------------------------------------------
+template <typename S, bool LB, bool BWD>
+auto pick_mx_gate(int gate) {
+  if constexpr (BWD) {
+    switch (gate) {
+      case kGateSquare: return situ_glu_bwd_mx_kernel<S, kGateSquare, LB>;
+      case kGateEqual: return situ_glu_bwd_mx_kernel<S, kGateEqual, LB>;
+      case kGateRoot: return situ_glu_bwd_mx_kernel<S, kGateRoot, LB>;
+      default: return situ_glu_bwd_mx_kernel<S, kGateGeneric, LB>;
+    }
+  } else {
+    switch (gate) {
+      case kGateSquare: return situ_glu_fwd_mx_kernel<S, kGateSquare, LB>;
+      case kGateEqual: return situ_glu_fwd_mx_kernel<S, kGateEqual, LB>;
+      case kGateRoot: return situ_glu_fwd_mx_kernel<S, kGateRoot, LB>;
+      default: return situ_glu_fwd_mx_kernel<S, kGateGeneric, LB>;
+    }
+  }
+}
 
-extern "C" {
+FwdMxKernel pick_fwd_mx(situ_dtype_t dtype, int gate, bool lb) {
+  if (dtype == SITU_DTYPE_BF16)
+    return lb ? pick_mx_gate<Bf16, true, false>(gate) : pick_mx_gate<Bf16, false, false>(gate);
+  return lb ? pick_mx_gate<F32, true, false>(gate) : pick_mx_gate<F32, false, false>(gate);
+}
 
-situ_status_t situ_glu_fwd(const void* gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
-                           int64_t gate_up_row_stride, const void* rw, situ_dtype_t rw_dtype,
-                           situ_rw_mode_t rw_mode, int64_t rw_stride, double beta, int has_linear_beta,
-                           double linear_beta, void* out, int64_t out_row_stride, void* stream) {
+BwdMxKernel pick_bwd_mx(situ_dtype_t dtype, int gate, bool lb) {
+  if (dtype == SITU_DTYPE_BF16)
+    return lb ? pick_mx_gate<Bf16, true, true>(gate) : pick_mx_gate<Bf16, false, true>(gate);
+  return lb ? pick_mx_gate<F32, true, true>(gate) : pick_mx_gate<F32, false, true>(gate);
+}
+
+// Argument checks of an MXFP8 output of `cols` columns per row.
+situ_status_t check_mx_args(const MxOut& m, int64_t inter, int64_t cols, situ_rw_mode_t rw_mode) {
+  if (m.rule != SITU_MX_RULE_OCP && m.rule != SITU_MX_RULE_CEIL)
+    return fail(SITU_ERR_INVALID_ARG, "rule %d is not a situ_mx_rule_t", m.rule);
+  if (inter % kMxBlock != 0)
+    return fail(SITU_ERR_INVALID_ARG, "MXFP8 outputs need inter a multiple of %d, got %lld", kMxBlock,
+                (long long)inter);
+  if (rw_mode == SITU_RW_COL || rw_mode == SITU_RW_FULL)
+    return fail(SITU_ERR_UNSUPPORTED, "MXFP8 outputs take per-row, broadcast or no routing weights");
+  if (m.data_pitch < cols) return fail(SITU_ERR_INVALID_ARG, "MXFP8 data row pitch < %lld bytes", (long long)cols);
+  if (m.scale_pitch < cols / kMxBlock)
+    return fail(SITU_ERR_INVALID_ARG, "MXFP8 scale row pitch < %lld bytes", (long long)(cols / kMxBlock));
+  return SITU_OK;
+}
+
+// Pointer, extent and alignment checks of an MXFP8 output (tokens > 0).
+situ_status_t check_mx_buffers(const MxOut& m, int64_t tokens, int64_t cols) {
+  if (m.data == nullptr || m.scale == nullptr) return fail(SITU_ERR_INVALID_ARG, "MXFP8 data or scale is NULL");
+  if (!span_fits(tokens, m.data_pitch, cols, 1) || !span_fits(tokens, m.scale_pitch, cols / kMxBlock, 1))
+    return fail(SITU_ERR_INVALID_ARG, "tensor extent overflows int64");
+  if (!aligned(m.data, 16) || m.data_pitch % 16 != 0)
+    return fail(SITU_ERR_MISALIGNED, "MXFP8 data base or row pitch not 16-byte aligned");
+  const Span sd = matrix_span(m.data, tokens, m.data_pitch, cols, 1);
+  const Span ss = matrix_span(m.scale, tokens, m.scale_pitch, cols / kMxBlock, 1);
+  if (overlap(sd, ss)) return fail(SITU_ERR_INVALID_ARG, "MXFP8 data overlaps its scales");
+  return SITU_OK;
+}
+
+// The forward with a native (mx == NULL) or an MXFP8 output.
+situ_status_t fwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
+                        int64_t gate_up_row_stride, const void* rw, situ_dtype_t rw_dtype, situ_rw_mode_t rw_mode,
+                        int64_t rw_stride, double beta, int has_linear_beta, double linear_beta, void* out,
+                        int64_t out_row_stride, const MxOut* mx, void* stream) {
   tl_last_error[0] = '\0';
   Coeffs c;
   int gate = kGateGeneric;
   situ_status_t st = check_common(dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode,
                                   rw_stride, beta, has_linear_beta, linear_beta, &c, &gate);
   if (st != SITU_OK) return st;
-  if (out_row_stride < inter) return fail(SITU_ERR_INVALID_ARG, "out_row_stride < inter");
+  if (mx != nullptr) {
+    st = check_mx_args(*mx, inter, inter, rw_mode);
+    if (st != SITU_OK) return st;
+  } else if (out_row_stride < inter) {
+    return fail(SITU_ERR_INVALID_ARG, "out_row_stride < inter");
+  }
   if (tokens == 0) return SITU_OK;
-  if (gate_up == nullptr || out == nullptr) return fail(SITU_ERR_INVALID_ARG, "gate_up or out is NULL");
+  if (gate_up == nullptr || (mx == nullptr && out == nullptr))
+    return fail(SITU_ERR_INVALID_ARG, "gate_up or out is NULL");
   const int es = elem_size(dtype);
-  if (!span_fits(tokens, gate_up_row_stride, 2 * inter, es) || !span_fits(tokens, out_row_stride, inter, es) ||
+  if (!span_fits(tokens, gate_up_row_stride, 2 * inter, es) ||
+      (mx == nullptr && !span_fits(tokens, out_row_stride, inter, es)) ||
       (rw_mode == SITU_RW_ROW && !span_fits(tokens, rw_stride, 1, elem_size(rw_dtype))) ||
       (rw_mode == SITU_RW_FULL && !span_fits(tokens, rw_stride, inter, elem_size(rw_dtype))))
     return fail(SITU_ERR_INVALID_ARG, "tensor extent overflows int64");
-  if (!aligned(gate_up, 16) || !aligned(out, 16) || (gate_up_row_stride * es) % 16 != 0 ||
-      (out_row_stride * es) % 16 != 0)
+  if (mx != nullptr) {
+    st = check_mx_buffers(*mx, tokens, inter);
+    if (st != SITU_OK) return st;
+  }
+  if (!aligned(gate_up, 16) || (gate_up_row_stride * es) % 16 != 0 ||
+      (mx == nullptr && (!aligned(out, 16) || (out_row_stride * es) % 16 != 0)))
     return fail(SITU_ERR_MISALIGNED, "gate_up/out base or row pitch not 16-byte aligned");
   if (rw_mode != SITU_RW_NONE && !aligned(rw, elem_size(rw_dtype)))
     return fail(SITU_ERR_MISALIGNED, "rw not aligned to its element size");
-  const Span s_out = matrix_span(out, tokens, out_row_stride, inter, es);
-  if (overlap(s_out, matrix_span(gate_up, tokens, gate_up_row_stride, 2 * inter, es)))
-    return fail(SITU_ERR_INVALID_ARG, "out overlaps gate_up");
-  if (overlap(s_out, weight_span(rw, rw_mode, tokens, rw_stride, inter, elem_size(rw_dtype))))
-    return fail(SITU_ERR_INVALID_ARG, "out overlaps rw");
+  const Span s_gu = matrix_span(gate_up, tokens, gate_up_row_stride, 2 * inter, es);
+  const Span s_rw = weight_span(rw, rw_mode, tokens, rw_stride, inter, elem_size(rw_dtype));
+  const Span s_out = mx ? matrix_span(mx->data, tokens, mx->data_pitch, inter, 1)
+                        : matrix_span(out, tokens, out_row_stride, inter, es);
+  if (overlap(s_out, s_gu)) return fail(SITU_ERR_INVALID_ARG, "out overlaps gate_up");
+  if (overlap(s_out, s_rw)) return fail(SITU_ERR_INVALID_ARG, "out overlaps rw");
+  if (mx != nullptr) {
+    const Span s_sc = matrix_span(mx->scale, tokens, mx->scale_pitch, inter / kMxBlock, 1);
+    if (overlap(s_sc, s_gu) || overlap(s_sc, s_rw)) return fail(SITU_ERR_INVALID_ARG, "MXFP8 scales overlap an input");
+  }
 
   if (rw_mode == SITU_RW_COL || rw_mode == SITU_RW_FULL) {
     EwArgs e{};
@@ -1864,6 +2289,15 @@ situ_status_t situ_glu_fwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
   a.c = c;
   if (rw_mode == SITU_RW_NONE) a.rw.bf16 = 0;
 
+  if (mx != nullptr) {
+    FwdMxKernel k = pick_fwd_mx(dtype, gate, has_linear_beta != 0);
+    const int threads = choose_threads(a.vpr);
+    int grid = 0;
+    st = launch_grid(reinterpret_cast<const void*>(k), threads, 0, tokens, &grid);
+    if (st != SITU_OK) return st;
+    k<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(a, *mx);
+    return check_launch("situ_glu_fwd_mxfp8");
+  }
   if (g_load_path.load(std::memory_order_relaxed) == 1) {
     StreamArgs sa{};
     sa.gate_up = a.gate_up;
@@ -1887,6 +2321,33 @@ situ_status_t situ_glu_fwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
   return check_launch("situ_glu_fwd");
 }
 
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// C ABI
+// ---------------------------------------------------------------------------
+
+extern "C" {
+
+situ_status_t situ_glu_fwd(const void* gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
+                           int64_t gate_up_row_stride, const void* rw, situ_dtype_t rw_dtype,
+                           situ_rw_mode_t rw_mode, int64_t rw_stride, double beta, int has_linear_beta,
+                           double linear_beta, void* out, int64_t out_row_stride, void* stream) {
+  return fwd_entry(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride, beta,
+                   has_linear_beta, linear_beta, out, out_row_stride, nullptr, stream);
+}
+
+situ_status_t situ_glu_fwd_mxfp8(const void* gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
+                                 int64_t gate_up_row_stride, const void* rw, situ_dtype_t rw_dtype,
+                                 situ_rw_mode_t rw_mode, int64_t rw_stride, double beta, int has_linear_beta,
+                                 double linear_beta, void* y_data, int64_t y_data_row_stride, void* y_scale,
+                                 int64_t y_scale_row_stride, situ_mx_rule_t rule, void* stream) {
+  const MxOut m{static_cast<char*>(y_data), y_data_row_stride, static_cast<uint8_t*>(y_scale), y_scale_row_stride,
+                static_cast<int>(rule)};
+  return fwd_entry(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride, beta,
+                   has_linear_beta, linear_beta, nullptr, 0, &m, stream);
+}
+
 size_t situ_glu_bwd_workspace_bytes(int64_t tokens, int64_t inter, situ_rw_mode_t rw_mode, int want_drw) {
   if (tokens <= 0 || inter <= 0 || !want_drw) return 0;
   uint64_t bytes = 0;
@@ -1896,12 +2357,17 @@ size_t situ_glu_bwd_workspace_bytes(int64_t tokens, int64_t inter, situ_rw_mode_
   return static_cast<size_t>((bytes + 255) / 256 * 256);
 }
 
-situ_status_t situ_glu_bwd(const void* gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
-                           int64_t gate_up_row_stride, const void* rw, situ_dtype_t rw_dtype,
-                           situ_rw_mode_t rw_mode, int64_t rw_stride, double beta, int has_linear_beta,
-                           double linear_beta, const void* grad_out, int64_t grad_out_row_stride,
-                           void* d_gate_up, int64_t d_gate_up_row_stride, void* d_rw, int64_t d_rw_stride,
-                           void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The backward with a native (mx == NULL) or an MXFP8 d_gate_up.
+situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
+                        int64_t gate_up_row_stride, const void* rw, situ_dtype_t rw_dtype, situ_rw_mode_t rw_mode,
+                        int64_t rw_stride, double beta, int has_linear_beta, double linear_beta,
+                        const void* grad_out, int64_t grad_out_row_stride, void* d_gate_up,
+                        int64_t d_gate_up_row_stride, void* d_rw, int64_t d_rw_stride, void* workspace,
+                        size_t workspace_bytes, const MxOut* mx, void* stream) {
   tl_last_error[0] = '\0';
   Coeffs c;
   int gate = kGateGeneric;
@@ -1909,7 +2375,12 @@ situ_status_t situ_glu_bwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
                                   rw_stride, beta, has_linear_beta, linear_beta, &c, &gate);
   if (st != SITU_OK) return st;
   if (grad_out_row_stride < inter) return fail(SITU_ERR_INVALID_ARG, "grad_out_row_stride < inter");
-  if (d_gate_up_row_stride < 2 * inter) return fail(SITU_ERR_INVALID_ARG, "d_gate_up_row_stride < 2 * inter");
+  if (mx != nullptr) {
+    st = check_mx_args(*mx, inter, 2 * inter, rw_mode);
+    if (st != SITU_OK) return st;
+  } else if (d_gate_up_row_stride < 2 * inter) {
+    return fail(SITU_ERR_INVALID_ARG, "d_gate_up_row_stride < 2 * inter");
+  }
   if (rw_mode == SITU_RW_NONE && d_rw != nullptr)
     return fail(SITU_ERR_INVALID_ARG, "d_rw must be NULL for SITU_RW_NONE");
   const bool want_drw = d_rw != nullptr;
@@ -1928,20 +2399,24 @@ situ_status_t situ_glu_bwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
     }
     return SITU_OK;
   }
-  if (gate_up == nullptr || grad_out == nullptr || d_gate_up == nullptr)
+  if (gate_up == nullptr || grad_out == nullptr || (mx == nullptr && d_gate_up == nullptr))
     return fail(SITU_ERR_INVALID_ARG, "gate_up, grad_out or d_gate_up is NULL");
   const int es = elem_size(dtype);
   const int rw_es = rw_mode == SITU_RW_NONE ? 4 : elem_size(rw_dtype);
+  if (mx != nullptr) {
+    st = check_mx_buffers(*mx, tokens, 2 * inter);
+    if (st != SITU_OK) return st;
+  }
   if (!span_fits(tokens, gate_up_row_stride, 2 * inter, es) || !span_fits(tokens, grad_out_row_stride, inter, es) ||
-      !span_fits(tokens, d_gate_up_row_stride, 2 * inter, es) ||
+      (mx == nullptr && !span_fits(tokens, d_gate_up_row_stride, 2 * inter, es)) ||
       (rw_mode == SITU_RW_ROW && !span_fits(tokens, rw_stride, 1, rw_es)) ||
       (want_drw && rw_mode == SITU_RW_ROW && !span_fits(tokens, d_rw_stride, 1, rw_es)) ||
       (rw_mode == SITU_RW_FULL && !span_fits(tokens, rw_stride, inter, rw_es)) ||
       (want_drw && rw_mode == SITU_RW_FULL && !span_fits(tokens, d_rw_stride, inter, rw_es)))
     return fail(SITU_ERR_INVALID_ARG, "tensor extent overflows int64");
-  if (!aligned(gate_up, 16) || !aligned(grad_out, 16) || !aligned(d_gate_up, 16) ||
-      (gate_up_row_stride * es) % 16 != 0 || (grad_out_row_stride * es) % 16 != 0 ||
-      (d_gate_up_row_stride * es) % 16 != 0)
+  if (!aligned(gate_up, 16) || !aligned(grad_out, 16) || (gate_up_row_stride * es) % 16 != 0 ||
+      (grad_out_row_stride * es) % 16 != 0 ||
+      (mx == nullptr && (!aligned(d_gate_up, 16) || (d_gate_up_row_stride * es) % 16 != 0)))
     return fail(SITU_ERR_MISALIGNED, "gate_up/grad_out/d_gate_up base or row pitch not 16-byte aligned");
   if (rw_mode != SITU_RW_NONE && !aligned(rw, rw_es)) return fail(SITU_ERR_MISALIGNED, "rw not aligned");
   if (want_drw && !aligned(d_rw, rw_es)) return fail(SITU_ERR_MISALIGNED, "d_rw not aligned");
@@ -1959,20 +2434,25 @@ situ_status_t situ_glu_bwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
   // Aliasing: no output may overlap an input or another output.
   const Span s_gu = matrix_span(gate_up, tokens, gate_up_row_stride, 2 * inter, es);
   const Span s_go = matrix_span(grad_out, tokens, grad_out_row_stride, inter, es);
-  const Span s_dgu = matrix_span(d_gate_up, tokens, d_gate_up_row_stride, 2 * inter, es);
+  const Span s_dgu = mx ? matrix_span(mx->data, tokens, mx->data_pitch, 2 * inter, 1)
+                        : matrix_span(d_gate_up, tokens, d_gate_up_row_stride, 2 * inter, es);
   const Span s_rw = weight_span(rw, rw_mode, tokens, rw_stride, inter, rw_es);
   if (overlap(s_dgu, s_gu) || overlap(s_dgu, s_go) || overlap(s_dgu, s_rw))
     return fail(SITU_ERR_INVALID_ARG, "d_gate_up overlaps an input");
+  const Span s_sc = mx ? matrix_span(mx->scale, tokens, mx->scale_pitch, 2 * inter / kMxBlock, 1) : Span{0, 0};
+  if (mx != nullptr && (overlap(s_sc, s_gu) || overlap(s_sc, s_go) || overlap(s_sc, s_rw)))
+    return fail(SITU_ERR_INVALID_ARG, "MXFP8 scales overlap an input");
   Span s_drw = {0, 0};
   if (want_drw) {
     s_drw = weight_span(d_rw, rw_mode, tokens, d_rw_stride, inter, rw_es);
-    if (overlap(s_drw, s_gu) || overlap(s_drw, s_go) || overlap(s_drw, s_rw) || overlap(s_drw, s_dgu))
+    if (overlap(s_drw, s_gu) || overlap(s_drw, s_go) || overlap(s_drw, s_rw) || overlap(s_drw, s_dgu) ||
+        overlap(s_drw, s_sc))
       return fail(SITU_ERR_INVALID_ARG, "d_rw overlaps another tensor");
   }
   if (ws_needed > 0) {
     const Span s_ws = {reinterpret_cast<uintptr_t>(workspace), reinterpret_cast<uintptr_t>(workspace) + ws_needed};
     if (overlap(s_ws, s_gu) || overlap(s_ws, s_go) || overlap(s_ws, s_rw) || overlap(s_ws, s_dgu) ||
-        overlap(s_ws, s_drw))
+        overlap(s_ws, s_drw) || overlap(s_ws, s_sc))
       return fail(SITU_ERR_INVALID_ARG, "workspace overlaps a tensor");
   }
 
@@ -2036,7 +2516,15 @@ situ_status_t situ_glu_bwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
   a.c = c;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (g_load_path.load(std::memory_order_relaxed) == 1) {
+  if (mx != nullptr) {
+    BwdMxKernel k = pick_bwd_mx(dtype, gate, has_linear_beta != 0);
+    const int threads = choose_threads(a.vpr);
+    int grid = 0;
+    st = launch_grid(reinterpret_cast<const void*>(k), threads, 0, tokens, &grid);
+    if (st != SITU_OK) return st;
+    k<<<grid, threads, 0, s>>>(a, *mx);
+    st = check_launch("situ_glu_bwd_mxfp8");
+  } else if (g_load_path.load(std::memory_order_relaxed) == 1) {
     StreamArgs sa{};
     sa.gate_up = a.gate_up;
     sa.gu_pitch = a.gu_pitch;
@@ -2069,6 +2557,35 @@ situ_status_t situ_glu_bwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
     st = check_launch("situ_glu_bwd (scalar d_rw)");
   }
   return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+situ_status_t situ_glu_bwd(const void* gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
+                           int64_t gate_up_row_stride, const void* rw, situ_dtype_t rw_dtype,
+                           situ_rw_mode_t rw_mode, int64_t rw_stride, double beta, int has_linear_beta,
+                           double linear_beta, const void* grad_out, int64_t grad_out_row_stride,
+                           void* d_gate_up, int64_t d_gate_up_row_stride, void* d_rw, int64_t d_rw_stride,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_entry(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride, beta,
+                   has_linear_beta, linear_beta, grad_out, grad_out_row_stride, d_gate_up, d_gate_up_row_stride,
+                   d_rw, d_rw_stride, workspace, workspace_bytes, nullptr, stream);
+}
+
+situ_status_t situ_glu_bwd_mxfp8(const void* gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
+                                 int64_t gate_up_row_stride, const void* rw, situ_dtype_t rw_dtype,
+                                 situ_rw_mode_t rw_mode, int64_t rw_stride, double beta, int has_linear_beta,
+                                 double linear_beta, const void* grad_out, int64_t grad_out_row_stride,
+                                 void* d_gate_up_data, int64_t d_gate_up_data_row_stride, void* d_gate_up_scale,
+                                 int64_t d_gate_up_scale_row_stride, situ_mx_rule_t rule, void* d_rw,
+                                 int64_t d_rw_stride, void* workspace, size_t workspace_bytes, void* stream) {
+  const MxOut m{static_cast<char*>(d_gate_up_data), d_gate_up_data_row_stride,
+                static_cast<uint8_t*>(d_gate_up_scale), d_gate_up_scale_row_stride, static_cast<int>(rule)};
+  return bwd_entry(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride, beta,
+                   has_linear_beta, linear_beta, grad_out, grad_out_row_stride, nullptr, 0, d_rw, d_rw_stride,
+                   workspace, workspace_bytes, &m, stream);
 }
 
 const char* situ_glu_status_string(situ_status_t status) {

@@ -165,6 +165,106 @@ def situ_glu_bwd(gate_up: torch.Tensor, routing_weights, grad_out: torch.Tensor,
     return d_gate_up, (d_rw if want else None)
 
 
+_MX_RULES = {"ocp": abi.SITU_MX_RULE_OCP, "ceil": abi.SITU_MX_RULE_CEIL}
+
+
+def _mx_rule(rule) -> int:
+    if isinstance(rule, str):
+        try:
+            return _MX_RULES[rule]
+        except KeyError:
+            raise ValueError(f"rule must be one of {sorted(_MX_RULES)}, got {rule!r}") from None
+    return int(rule)
+
+
+def _mx_buffers(lead: tuple, cols: int, device, data=None, scale=None):
+    """E4M3 codes [..., cols] (torch.float8_e4m3fn) and E8M0 scale bytes
+    [..., cols / 32] (torch.uint8), allocated when not given; returns the two
+    tensors and their 2-D byte views."""
+    if data is None:
+        data = torch.empty(lead + (cols,), dtype=torch.float8_e4m3fn, device=device)
+    if scale is None:
+        scale = torch.empty(lead + (cols // 32,), dtype=torch.uint8, device=device)
+    if data.element_size() != 1 or scale.element_size() != 1:
+        raise TypeError("MXFP8 data and scale tensors hold one byte per element")
+    d2 = data.view(-1, cols)
+    s2 = scale.view(-1, cols // 32)
+    return data, scale, d2, s2
+
+
+def situ_glu_fwd_mxfp8(gate_up: torch.Tensor, routing_weights, beta: float = DEFAULT_BETA,
+                       linear_beta: float | None = DEFAULT_LINEAR_BETA, rule="ocp", data=None, scale=None,
+                       stream=None):
+    """Forward with an MXFP8 Y (OCP MX v1.0: E4M3 codes, one E8M0 scale per 32
+    elements of a row).  Returns (codes [..., I] as torch.float8_e4m3fn,
+    scale bytes [..., I / 32] as torch.uint8).  rule: "ocp" (shared exponent
+    floor(log2 amax) - 8, elements clamped to +-448) or "ceil" (smallest
+    exponent with no clamping).  I must be a multiple of 32; routing weights
+    per row, broadcast, or None."""
+    _check_beta(beta, linear_beta)
+    g2, lead, inter = _rows(gate_up)
+    dtype = _dtype_code(g2, "gate_up")
+    mode, rw, rw_stride = routing_mode(lead, inter, routing_weights)
+    rw_dtype = _dtype_code(rw, "routing_weights") if rw is not None else abi.SITU_DTYPE_F32
+    data, scale, d2, s2 = _mx_buffers(lead, inter, gate_up.device, data, scale)
+    tokens = g2.shape[0]
+    st = abi.situ_glu_fwd_mxfp8(g2.data_ptr(), dtype, tokens, inter, g2.stride(0) if tokens > 1 else 2 * inter,
+                                rw.data_ptr() if rw is not None else None, rw_dtype, mode, rw_stride,
+                                float(beta), int(linear_beta is not None),
+                                float(linear_beta) if linear_beta is not None else 0.0,
+                                d2.data_ptr(), d2.stride(0) if tokens > 1 else inter,
+                                s2.data_ptr(), s2.stride(0) if tokens > 1 else inter // 32,
+                                _mx_rule(rule), _stream_handle(stream))
+    abi.check(st, "situ_glu_fwd_mxfp8")
+    return data, scale
+
+
+def situ_glu_bwd_mxfp8(gate_up: torch.Tensor, routing_weights, grad_out: torch.Tensor,
+                       beta: float = DEFAULT_BETA, linear_beta: float | None = DEFAULT_LINEAR_BETA,
+                       rule="ocp", want_drw: bool = True, data=None, scale=None, d_rw=None, workspace=None,
+                       stream=None):
+    """Backward with an MXFP8 d_gate_up: returns (codes [..., 2I] as
+    torch.float8_e4m3fn with dG then dU, scale bytes [..., 2I / 32],
+    d_routing_weights or None).  Same rules and restrictions as
+    situ_glu_fwd_mxfp8; the weight gradient is as in situ_glu_bwd."""
+    _check_beta(beta, linear_beta)
+    g2, lead, inter = _rows(gate_up)
+    dtype = _dtype_code(g2, "gate_up")
+    if grad_out.dtype != gate_up.dtype:
+        raise TypeError("grad_out must have gate_up's dtype")
+    if tuple(grad_out.shape) != lead + (inter,):
+        raise ValueError(f"grad_out shape {tuple(grad_out.shape)} != {lead + (inter,)}")
+    go2 = grad_out.reshape(-1, inter)
+    if go2.stride(1) != 1 or (go2.shape[0] > 1 and go2.stride(0) < inter):
+        go2 = go2.contiguous()
+    mode, rw, rw_stride = routing_mode(lead, inter, routing_weights)
+    rw_dtype = _dtype_code(rw, "routing_weights") if rw is not None else abi.SITU_DTYPE_F32
+    want = bool(want_drw) and rw is not None
+    data, scale, d2, s2 = _mx_buffers(lead, 2 * inter, gate_up.device, data, scale)
+    d_rw_flat, d_rw_stride = None, 1
+    if want:
+        if d_rw is None:
+            d_rw = torch.empty(routing_weights.shape, dtype=routing_weights.dtype, device=gate_up.device)
+        d_rw_flat = d_rw.view(-1)
+        d_rw_stride = d_rw_flat.stride(0) if d_rw_flat.numel() > 1 else 1
+    tokens = g2.shape[0]
+    ws_bytes = abi.situ_glu_bwd_workspace_bytes(tokens, inter, mode, int(want))
+    if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=gate_up.device)
+    st = abi.situ_glu_bwd_mxfp8(g2.data_ptr(), dtype, tokens, inter, g2.stride(0) if tokens > 1 else 2 * inter,
+                                rw.data_ptr() if rw is not None else None, rw_dtype, mode, rw_stride,
+                                float(beta), int(linear_beta is not None),
+                                float(linear_beta) if linear_beta is not None else 0.0,
+                                go2.data_ptr(), go2.stride(0) if tokens > 1 else inter,
+                                d2.data_ptr(), d2.stride(0) if tokens > 1 else 2 * inter,
+                                s2.data_ptr(), s2.stride(0) if tokens > 1 else 2 * inter // 32,
+                                _mx_rule(rule), d_rw_flat.data_ptr() if d_rw_flat is not None else None,
+                                d_rw_stride, workspace.data_ptr() if ws_bytes else None, ws_bytes,
+                                _stream_handle(stream))
+    abi.check(st, "situ_glu_bwd_mxfp8")
+    return data, scale, (d_rw if want else None)
+
+
 class WeightedSiTUFunction(torch.autograd.Function):
     """Routing-weighted SiTU-GLU with the analytic fused backward.
 

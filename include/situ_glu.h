@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define SITU_GLU_ABI_VERSION 2
+#define SITU_GLU_ABI_VERSION 3
 
 typedef enum situ_status {
   SITU_OK = 0,
@@ -165,11 +165,69 @@ situ_status_t situ_glu_bwd(const void *gate_up, situ_dtype_t dtype, int64_t toke
                            void *workspace, size_t workspace_bytes,
                            void *stream);
 
-/* Bytes of workspace situ_glu_bwd needs with want_drw != 0: tokens * 4 for
- * SITU_RW_SCALAR (one partial per row), ceil(tokens / 64) * inter * 4 for
- * SITU_RW_COL (one partial per column per block of 64 rows), each rounded up
- * to 256; otherwise 0.  Non-positive tokens or inter give 0. */
+/* Bytes of workspace situ_glu_bwd (and situ_glu_bwd_mxfp8) needs with
+ * want_drw != 0: tokens * 4 for SITU_RW_SCALAR (one partial per row),
+ * ceil(tokens / 16) * inter * 4 for SITU_RW_COL (one partial per column per
+ * chunk of 16 rows), each rounded up to 256; otherwise 0.  Non-positive
+ * tokens or inter give 0. */
 size_t situ_glu_bwd_workspace_bytes(int64_t tokens, int64_t inter, situ_rw_mode_t rw_mode, int want_drw);
+
+/* ---- MXFP8 outputs ---------------------------------------------------------
+ * Block-scaled FP8 outputs in the OCP Microscaling Formats (MX) v1.0 layout,
+ * the format of the MXFP8 recipe the SiTU-GLU integration was tested with
+ * (Megatron-LM PR #6673, "Test results"; the format itself is the public OCP
+ * specification): every 32 consecutive elements of a row share one E8M0
+ * scale byte S (X = 2^(S - 127); S = 255 is NaN) and each element is an FP8
+ * E4M3 code (bias 7, largest normal 448, S.1111.111 NaN) of value / X,
+ * rounded to nearest even.  The values are quantised from the kernel's fp32
+ * results, never rounded to bf16 first.  A block holding a NaN or an
+ * infinity gets S = 255 and NaN codes. */
+typedef enum situ_mx_rule {
+  SITU_MX_RULE_OCP = 0,  /* shared exponent floor(log2 amax) - 8, elements clamped to +-448
+                            (the OCP MX conversion)                                          */
+  SITU_MX_RULE_CEIL = 1  /* smallest exponent e with amax <= 448 * 2^e: no element clamps     */
+} situ_mx_rule_t;        /* both at least -127 (S >= 0); amax = 0 gives S = 0                  */
+
+/*
+ * Forward with an MXFP8 Y: as situ_glu_fwd, but Y is written as
+ *   y_data   [tokens, >= inter] E4M3 codes, row pitch y_data_row_stride BYTES
+ *            (a multiple of 16; y_data 16-byte aligned);
+ *   y_scale  [tokens, >= inter / 32] scale bytes, row pitch y_scale_row_stride
+ *            bytes; byte b of a row scales columns [32 b, 32 b + 32).
+ * inter must be a multiple of 32 (SITU_ERR_INVALID_ARG otherwise).  Routing
+ * weights: SITU_RW_ROW, SITU_RW_SCALAR or SITU_RW_NONE (SITU_ERR_UNSUPPORTED
+ * for the element-wise forms).  Neither output may overlap an input or the
+ * other.  Other arguments and errors as for situ_glu_fwd.
+ */
+situ_status_t situ_glu_fwd_mxfp8(const void *gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
+                                 int64_t gate_up_row_stride,
+                                 const void *rw, situ_dtype_t rw_dtype, situ_rw_mode_t rw_mode,
+                                 int64_t rw_stride,
+                                 double beta, int has_linear_beta, double linear_beta,
+                                 void *y_data, int64_t y_data_row_stride,
+                                 void *y_scale, int64_t y_scale_row_stride,
+                                 situ_mx_rule_t rule, void *stream);
+
+/*
+ * Backward with an MXFP8 d_gate_up: as situ_glu_bwd, but d_gate_up is written
+ * as E4M3 codes d_gate_up_data [tokens, >= 2 inter] (dG in columns [0, I), dU
+ * in [I, 2I); row pitch in BYTES, a multiple of 16, base 16-byte aligned) and
+ * scale bytes d_gate_up_scale [tokens, >= 2 inter / 32] (dG blocks first).
+ * The routing-weight gradient (d_rw, workspace) is exactly as in situ_glu_bwd.
+ * Same restrictions as situ_glu_fwd_mxfp8.
+ */
+situ_status_t situ_glu_bwd_mxfp8(const void *gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
+                                 int64_t gate_up_row_stride,
+                                 const void *rw, situ_dtype_t rw_dtype, situ_rw_mode_t rw_mode,
+                                 int64_t rw_stride,
+                                 double beta, int has_linear_beta, double linear_beta,
+                                 const void *grad_out, int64_t grad_out_row_stride,
+                                 void *d_gate_up_data, int64_t d_gate_up_data_row_stride,
+                                 void *d_gate_up_scale, int64_t d_gate_up_scale_row_stride,
+                                 situ_mx_rule_t rule,
+                                 void *d_rw, int64_t d_rw_stride,
+                                 void *workspace, size_t workspace_bytes,
+                                 void *stream);
 
 /* Static, human-readable name of a status code. */
 const char *situ_glu_status_string(situ_status_t status);

@@ -124,6 +124,8 @@ class Oracle:
         lib.situ_oracle_mutant_id.restype = _INT
         lib.situ_oracle_e4m3_encode.argtypes = [_DBL]
         lib.situ_oracle_e4m3_encode.restype = _INT
+        lib.situ_oracle_e4m3_encode_n.argtypes = [_VP, _I64, _VP]
+        lib.situ_oracle_e4m3_encode_n.restype = None
         lib.situ_oracle_e4m3_decode.argtypes = [_INT]
         lib.situ_oracle_e4m3_decode.restype = _DBL
         lib.situ_oracle_mx_scale_exp.argtypes = [_DBL, _INT]
@@ -254,9 +256,10 @@ class Oracle:
 
     def e4m3_encode(self, x) -> np.ndarray:
         """E4M3 codes (uint8) of reals x: nearest-even, clamped to +-448."""
-        x = np.asarray(x, dtype=np.float64)
-        f = self._lib.situ_oracle_e4m3_encode
-        return np.array([f(float(v)) for v in x.reshape(-1)], dtype=np.uint8).reshape(x.shape)
+        x = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+        out = np.empty(x.shape, dtype=np.uint8)
+        self._lib.situ_oracle_e4m3_encode_n(_ptr(x), x.size, _ptr(out))
+        return out
 
     def e4m3_decode(self, codes) -> np.ndarray:
         c = np.asarray(codes, dtype=np.uint8)

@@ -17,7 +17,7 @@
  *     conversion): shared exponent e = floor(log2(max_i |V_i|)) - emax,
  *     emax = 8 (the exponent of E4M3's largest normal); X = 2^e; each
  *     P_i = V_i / X rounded to nearest-even E4M3, clamped to +-448.
- * A second scale rule (SITU_MX_SCALE_CEIL in the library) takes the smallest
+ * A second scale rule (the no-clamp rule, rule 1 below) takes the smallest
  * e with max_i |V_i| / 2^e <= 448, so that no element is clamped.
  *
  * Readings (where the spec leaves a choice to the implementation): a block
@@ -157,4 +157,9 @@ int situ_oracle_mxfp8_quantize(const double *v, int64_t rows, int64_t cols, int6
     }
   }
   return 0;
+}
+
+/* situ_oracle_e4m3_encode over n values. */
+void situ_oracle_e4m3_encode_n(const double *x, int64_t n, uint8_t *codes) {
+  for (int64_t i = 0; i < n; ++i) codes[i] = (uint8_t)situ_oracle_e4m3_encode(x[i]);
 }

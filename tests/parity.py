@@ -22,6 +22,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
+import oracle
 import workloads
 from ffn_gated_activation_b200 import abi
 
@@ -182,3 +183,58 @@ def check_dw(name: str, got: np.ndarray, ref: np.ndarray, mag: np.ndarray):
                              f"got {y[i]!r}, oracle {ref[i]!r}, sum |terms| {mag[i]!r}")
     strict = np.abs(y - ref) <= DW_REL * np.abs(ref)
     return {"n": int(y.size), "extra_clause": int((~strict).sum())}
+
+
+# ---- MXFP8 outputs ----------------------------------------------------------------------
+
+def e4m3_key(codes: np.ndarray) -> np.ndarray:
+    """E4M3 codes in value order (sign-magnitude; both zeros equal)."""
+    c = codes.astype(np.int32)
+    m = c & 0x7F
+    return np.where(c & 0x80, -m, m)
+
+
+def check_mx(name: str, codes: np.ndarray, scales: np.ndarray, ref: np.ndarray, tol: np.ndarray, rule: int,
+             min_exact: float = 0.9):
+    """MXFP8 codes [R, C] and scale bytes [R, C / 32] against the oracle's
+    exact values ``ref`` when the kernel's fp32 values may differ from ref by
+    up to ``tol`` (elementwise).  Quantisation is monotone, so each block's
+    shared exponent must lie between the oracle's exponents for the smallest
+    and largest block maximum within tol, and, given the kernel's scale X, each
+    code between the oracle's codes for (ref - tol) / X and (ref + tol) / X;
+    at least ``min_exact`` of the codes must equal the oracle's code for
+    ref / X.  Blocks holding NaN or infinity must carry scale byte 255."""
+    o = oracle.load()
+    R, C = ref.shape
+    nb = C // 32
+    assert codes.shape == (R, C) and scales.shape == (R, nb), (codes.shape, scales.shape, ref.shape)
+    refb, tolb = ref.reshape(R, nb, 32), tol.reshape(R, nb, 32)
+    special = ~np.isfinite(refb).all(axis=2)
+    absb = np.where(np.isfinite(refb), np.abs(refb), 0.0)
+    amax_lo = np.maximum(absb - tolb, 0.0).max(axis=2)
+    amax_hi = (absb + tolb).max(axis=2)
+    got_e = scales.astype(np.int64) - 127
+    for r in range(R):
+        for b in range(nb):
+            if special[r, b]:
+                assert scales[r, b] == 255, f"{name}: block ({r}, {b}) holds NaN/inf, scale {scales[r, b]}"
+                continue
+            e_lo, e_hi = o.mx_scale_exp(amax_lo[r, b], rule), o.mx_scale_exp(amax_hi[r, b], rule)
+            assert e_lo <= got_e[r, b] <= e_hi, (f"{name}: block ({r}, {b}) exponent {got_e[r, b]} outside "
+                                                 f"[{e_lo}, {e_hi}] (amax {amax_lo[r, b]}..{amax_hi[r, b]})")
+    Xe = np.repeat(np.exp2(np.where(scales == 255, 0, got_e).astype(np.float64)), 32, axis=1)
+    fin = np.repeat(~special, 32, axis=1) & np.isfinite(ref)
+    with np.errstate(invalid="ignore"):
+        lo = e4m3_key(o.e4m3_encode((ref - tol) / Xe))
+        hi = e4m3_key(o.e4m3_encode((ref + tol) / Xe))
+        mid = e4m3_key(o.e4m3_encode(ref / Xe))
+    g = e4m3_key(codes)
+    bad = np.flatnonzero(fin & ~((lo <= g) & (g <= hi)))
+    if bad.size:
+        i = bad[0]
+        raise AssertionError(f"{name}: {bad.size} codes out of range; first at flat {i}: code {codes.flat[i]:#x}, "
+                             f"oracle value {ref.flat[i]!r} / X {Xe.flat[i]!r}, allowed keys "
+                             f"[{lo.flat[i]}, {hi.flat[i]}]")
+    exact, total = int(np.sum(fin & (g == mid))), int(np.sum(fin))
+    assert total == 0 or exact >= min_exact * total, f"{name}: only {exact} of {total} codes equal the oracle's"
+    return {"codes": total, "exact": exact}

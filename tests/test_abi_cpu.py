@@ -58,7 +58,7 @@ def test_binding_covers_the_header_exactly():
 
 
 def test_version_and_status_strings(native_lib_path):
-    assert abi.situ_glu_abi_version() == abi.ABI_VERSION == 2
+    assert abi.situ_glu_abi_version() == abi.ABI_VERSION == 3
     assert abi.situ_glu_status_string(OK) == "SITU_OK"
     assert abi.situ_glu_status_string(MISAL) == "SITU_ERR_MISALIGNED"
     assert abi.situ_glu_status_string(99) == "SITU_ERR_UNKNOWN"
@@ -227,3 +227,81 @@ def test_defaults_match_the_pages():
     assert pkg.DEFAULT_BETA == golden["beta"]["value"]
     assert pkg.DEFAULT_LINEAR_BETA == golden["linear_beta"]["value"]
     assert golden["moe_intermediate_size"]["value"] == 3072
+
+
+# ---- MXFP8 entry points: argument checks run before any CUDA call --------------
+
+MXD = 0x10000000   # fake 16-byte aligned device addresses for the outputs
+MXS = 0x18000000
+
+
+def fwd_mx(**kw):
+    a = dict(gate_up=GU, dtype=BF16, tokens=16, inter=64, gate_up_row_stride=128, rw=RW, rw_dtype=F32,
+             rw_mode=ROW, rw_stride=1, beta=4.0, has_linear_beta=1, linear_beta=25.0, y_data=MXD,
+             y_data_row_stride=64, y_scale=MXS, y_scale_row_stride=2, rule=abi.SITU_MX_RULE_OCP, stream=None)
+    a.update(kw)
+    return abi.situ_glu_fwd_mxfp8(**a)
+
+
+def bwd_mx(**kw):
+    a = dict(gate_up=GU, dtype=BF16, tokens=16, inter=64, gate_up_row_stride=128, rw=RW, rw_dtype=F32,
+             rw_mode=ROW, rw_stride=1, beta=4.0, has_linear_beta=1, linear_beta=25.0, grad_out=GO,
+             grad_out_row_stride=64, d_gate_up_data=MXD, d_gate_up_data_row_stride=128, d_gate_up_scale=MXS,
+             d_gate_up_scale_row_stride=4, rule=abi.SITU_MX_RULE_OCP, d_rw=DRW, d_rw_stride=1, workspace=None,
+             workspace_bytes=0, stream=None)
+    a.update(kw)
+    return abi.situ_glu_bwd_mxfp8(**a)
+
+
+MX_CASES = [
+    ("inter not a multiple of 32", dict(inter=40, gate_up_row_stride=80), INVALID),
+    ("bad rule", dict(rule=5), INVALID),
+    ("per-column weights", dict(rw_mode=3), UNSUP),
+    ("per-element weights", dict(rw_mode=4, rw_stride=64), UNSUP),
+    ("scale pitch short", dict(scale_short=True), INVALID),
+    ("data pitch short", dict(data_short=True), INVALID),
+    ("data pitch not 16-byte", dict(data_pitch_odd=True), MISAL),
+    ("data misaligned", dict(data_off=8), MISAL),
+    ("data NULL", dict(data_null=True), INVALID),
+    ("data overlaps gate_up", dict(data_at_gu=True), INVALID),
+    ("scale overlaps data", dict(scale_at_data=True), INVALID),
+    ("bad beta", dict(beta=-1.0), INVALID),
+]
+
+
+def _mx_kw(kw, cols, prefix):
+    kw = dict(kw)
+    d, dp, sc, sp = (f"{prefix}data", f"{prefix}data_row_stride", f"{prefix}scale", f"{prefix}scale_row_stride")
+    if kw.pop("scale_short", False):
+        kw[sp] = cols // 32 - 1
+    if kw.pop("data_short", False):
+        kw[dp] = cols - 16
+    if kw.pop("data_pitch_odd", False):
+        kw[dp] = cols + 8
+    off = kw.pop("data_off", 0)
+    if off:
+        kw[d] = MXD + off
+    if kw.pop("data_null", False):
+        kw[d] = None
+    if kw.pop("data_at_gu", False):
+        kw[d] = GU
+    if kw.pop("scale_at_data", False):
+        kw[sc] = MXD + 32
+    return kw
+
+
+@pytest.mark.parametrize("name,kw,want", MX_CASES, ids=[c[0] for c in MX_CASES])
+def test_fwd_mxfp8_argument_errors(name, kw, want, native_lib_path):
+    inter = kw.get("inter", 64)
+    assert fwd_mx(**_mx_kw(kw, inter, "y_")) == want, abi.situ_glu_last_error()
+
+
+@pytest.mark.parametrize("name,kw,want", MX_CASES, ids=[c[0] for c in MX_CASES])
+def test_bwd_mxfp8_argument_errors(name, kw, want, native_lib_path):
+    inter = kw.get("inter", 64)
+    assert bwd_mx(**_mx_kw(kw, 2 * inter, "d_gate_up_")) == want, abi.situ_glu_last_error()
+
+
+def test_mxfp8_zero_tokens_is_a_no_op(native_lib_path):
+    assert fwd_mx(tokens=0, y_data=None, y_scale=None) == OK
+    assert bwd_mx(tokens=0, d_gate_up_data=None, d_gate_up_scale=None, d_rw=None) == OK
