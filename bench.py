@@ -8,6 +8,13 @@ must move: read gate_up and w, write Y; read gate_up, grad_out and w, write
 d_gate_up and d_w), plus rows/s.
 
     python bench.py [--gpus N --steps K --warmup W] [--config 0..4] [--impl reference]
+                    [--variant row|col|full|mxfp8]
+
+--variant picks the form timed (default: per-row routing weights, the routed
+MoE form): per-column [I] or per-element [T, I] weights, or MXFP8 outputs
+(E4M3 codes + E8M0 scales for Y and d_gate_up, OCP rule).  Algorithmic
+bytes follow the form (weights read, weight gradients written, one byte per
+code plus one per 32 codes).
 
 For N > 1 launch one process per GPU with torchrun; every rank runs the same
 per-GPU workload (weak scaling, no collective on the data path), the step
@@ -53,6 +60,8 @@ def parse_args(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-oracle sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--variant", choices=["row", "col", "full", "mxfp8"], default="row",
+                   help="routing-weight form or output format timed (default: per-row weights)")
     p.add_argument("--flush", choices=["auto", "always", "never"], default="auto",
                    help="flush L2 before every step (auto: when the inputs fit in L2)")
     return p.parse_args(argv)
@@ -88,10 +97,17 @@ def recorded_traffic(kernel: str, workload_name: str):
     return float(entry["bytes_per_launch"])
 
 
-def workload_config(wl, beta, l2_note, world):
+def workload_config(wl, beta, l2_note, world, variant="row"):
     rw = {"uniform": "U(0,1) per row", "ones": "1.0 per row",
           "topk_softmax": f"top-{wl.topk} softmax weights of N(0,1) logits over {wl.experts} experts"}[wl.rw_kind]
+    if variant == "col":
+        rw = "U(0,1) per column ([I], shared by every row)"
+    elif variant == "full":
+        rw = "U(0,1) per element ([T, I])"
     return {
+        "variant": {"row": "per-row routing weights, bf16/fp32 outputs",
+                    "col": "per-column routing weights [I]", "full": "per-element routing weights [T, I]",
+                    "mxfp8": "per-row routing weights, MXFP8 Y and d_gate_up (E4M3 + E8M0 per 32, OCP rule)"}[variant],
         "workload": wl.describe(),
         "name": wl.name,
         "tokens": wl.tokens,
@@ -177,19 +193,57 @@ class ClockSampler:
                 "power_w_max": round(max(s[2] for s in self.samples), 1), "source": "nvml"}
 
 
-def cpu_oracle_rate(wl, beta, x, seconds: float):
+def variant_bytes(wl, variant: str):
+    """Algorithmic bytes (forward, backward) of one pass over the workload in
+    the given form.  Per-row weights: read gate_up and w, write Y; read
+    gate_up, grad_out and w, write d_gate_up and d_w.  Per-column weights move
+    I weights and I gradients per pass; per-element weights T I of each.
+    MXFP8 writes one byte per code and one scale byte per 32 codes."""
+    T, I = wl.tokens, wl.inter
+    es = 2 if wl.dtype == "bf16" else 4
+    if variant == "col":
+        return T * 3 * I * es + 4 * I, T * 5 * I * es + 8 * I
+    if variant == "full":
+        return T * (3 * I * es + 4 * I), T * (5 * I * es + 8 * I)
+    if variant == "mxfp8":
+        return T * (2 * I * es + I + I // 32 + 4), T * (3 * I * es + 2 * I + 2 * I // 32 + 8)
+    return wl.fwd_bytes(), wl.bwd_bytes()
+
+
+def variant_weights(wl, x, variant: str):
+    """Host routing weights of the form (float32) and the oracle's mode."""
+    import oracle
+    if variant == "col":
+        return workloads.column_weights(wl), oracle.RW_COL
+    if variant == "full":
+        return workloads.element_weights(wl), oracle.RW_FULL
+    return x["routing_weights"], oracle.RW_ROW
+
+
+def cpu_oracle_rate(wl, beta, x, seconds: float, variant: str = "row"):
     """The fp64 oracle (single thread, as it stands) on the first rows of the
-    workload, fwd then bwd per chunk of rows, until ``seconds`` have passed.
+    workload, fwd then bwd per chunk of rows (MXFP8: plus the oracle's block
+    quantisation of Y and d_gate_up), until ``seconds`` have passed.
     Returns (GB/s of algorithmic bytes, rows done, elapsed)."""
     import oracle
     o = oracle.load()
-    per_row = (wl.fwd_bytes() + wl.bwd_bytes()) / wl.tokens
+    fb, bb = variant_bytes(wl, variant)
+    per_row = (fb + bb) / wl.tokens
+    w, mode = variant_weights(wl, x, variant)
     chunk = max(1, min(64, int(2 ** 20 // wl.inter)))
     done, t0 = 0, time.perf_counter()
     while done < wl.tokens:
-        rows = np.arange(done, min(wl.tokens, done + chunk), dtype=np.int64)
-        o.fwd(x["gate_up"], x["routing_weights"], beta, wl.linear_beta, rows=rows)
-        o.bwd(x["gate_up"], x["routing_weights"], x["grad_out"], beta, wl.linear_beta, rows=rows)
+        stop = min(wl.tokens, done + chunk)
+        rows = np.arange(done, stop, dtype=np.int64)
+        if mode == oracle.RW_FULL:  # the oracle reads [T, I] weights from row 0: pass the chunk's own rows
+            gu, go, wr, rsel = x["gate_up"][done:stop], x["grad_out"][done:stop], w[done:stop], None
+        else:
+            gu, go, wr, rsel = x["gate_up"], x["grad_out"], w, rows
+        y = o.fwd(gu, wr, beta, wl.linear_beta, rows=rsel, rw_mode=mode)
+        r = o.bwd(gu, wr, go, beta, wl.linear_beta, rows=rsel, rw_mode=mode)
+        if variant == "mxfp8":
+            o.mxfp8_quantize(y)
+            o.mxfp8_quantize(np.concatenate([r.dg, r.du], axis=1))
         done += rows.size
         if time.perf_counter() - t0 >= seconds:
             break
@@ -210,11 +264,18 @@ def run_reference(args):
     x = workloads.inputs(wl, tokens=rows_per_step)
     import oracle
     o = oracle.load()
-    per_row = (wl.fwd_bytes() + wl.bwd_bytes()) / wl.tokens
+    fb, bb = variant_bytes(wl, args.variant)
+    per_row = (fb + bb) / wl.tokens
+    w, mode = variant_weights(wl, x, args.variant)
+    if mode == oracle.RW_FULL:
+        w = w[:rows_per_step]
 
     def step():
-        o.fwd(x["gate_up"], x["routing_weights"], beta, wl.linear_beta)
-        o.bwd(x["gate_up"], x["routing_weights"], x["grad_out"], beta, wl.linear_beta)
+        y = o.fwd(x["gate_up"], w, beta, wl.linear_beta, rw_mode=mode)
+        r = o.bwd(x["gate_up"], w, x["grad_out"], beta, wl.linear_beta, rw_mode=mode)
+        if args.variant == "mxfp8":
+            o.mxfp8_quantize(y)
+            o.mxfp8_quantize(np.concatenate([r.dg, r.du], axis=1))
 
     for _ in range(args.warmup):
         step()
@@ -229,7 +290,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(wl, beta, "n/a (host)", 1),
+        "data": "synthetic", "config": workload_config(wl, beta, "n/a (host)", 1, args.variant),
         "rows_per_s": rows_per_step * args.steps / dt,
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -275,14 +336,24 @@ def run_ours(args):
         t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
         return t.pin_memory()
 
+    variant = args.variant
     gu_h, go_h = upload(x["gate_up"]), upload(x["grad_out"])
-    rw_h = torch.from_numpy(x["routing_weights"]).reshape(T, 1).pin_memory()
+    w_np, _ = variant_weights(wl, x, variant)
+    rw_h = torch.from_numpy(w_np).reshape({"col": (I,), "full": (T, I)}.get(variant, (T, 1))).pin_memory()
     gu = gu_h.to(dev)
     go = go_h.to(dev)
     rw = rw_h.to(dev)
-    y = torch.empty(T, I, dtype=tdt, device=dev)
-    d_gu = torch.empty(T, 2 * I, dtype=tdt, device=dev)
-    d_rw = torch.empty(T, 1, dtype=torch.float32, device=dev)
+    d_rw = torch.empty(rw.shape, dtype=torch.float32, device=dev)
+    if variant == "mxfp8":
+        y = torch.empty(T, I, dtype=torch.float8_e4m3fn, device=dev)
+        y_sc = torch.empty(T, I // 32, dtype=torch.uint8, device=dev)
+        d_gu = torch.empty(T, 2 * I, dtype=torch.float8_e4m3fn, device=dev)
+        d_sc = torch.empty(T, 2 * I // 32, dtype=torch.uint8, device=dev)
+        outputs = [y, y_sc, d_gu, d_sc, d_rw]
+    else:
+        y = torch.empty(T, I, dtype=tdt, device=dev)
+        d_gu = torch.empty(T, 2 * I, dtype=tdt, device=dev)
+        outputs = [y, d_gu, d_rw]
 
     input_bytes = gu.numel() * gu.element_size() + go.numel() * go.element_size() + rw.numel() * 4
     flush = args.flush == "always" or (args.flush == "auto" and input_bytes < 2 * L2_BYTES)
@@ -290,11 +361,18 @@ def run_ours(args):
     l2_note = (f"L2 flushed before every step by writing {2 * L2_BYTES >> 20} MB (flush not timed)" if flush
                else f"inputs ({input_bytes / 1e6:.0f} MB) exceed the {L2_BYTES >> 20} MB L2; no flush")
 
-    def fwd():
-        pkg.situ_glu_fwd(gu, rw, beta, lb, out=y)
+    if variant == "mxfp8":
+        def fwd():
+            pkg.situ_glu_fwd_mxfp8(gu, rw, beta, lb, rule="ocp", data=y, scale=y_sc)
 
-    def bwd():
-        pkg.situ_glu_bwd(gu, rw, go, beta, lb, d_gate_up=d_gu, d_rw=d_rw)
+        def bwd():
+            pkg.situ_glu_bwd_mxfp8(gu, rw, go, beta, lb, rule="ocp", data=d_gu, scale=d_sc, d_rw=d_rw)
+    else:
+        def fwd():
+            pkg.situ_glu_fwd(gu, rw, beta, lb, out=y)
+
+        def bwd():
+            pkg.situ_glu_bwd(gu, rw, go, beta, lb, d_gate_up=d_gu, d_rw=d_rw)
 
     stream = torch.cuda.current_stream(dev)
     for _ in range(max(3, args.warmup)):
@@ -332,20 +410,32 @@ def run_ours(args):
         dist.all_reduce(times, op=dist.ReduceOp.MAX)
     total_ms, fwd_sum, bwd_sum = times.tolist()
     ms_per_step = total_ms / K
-    step_bytes = wl.fwd_bytes() + wl.bwd_bytes()
+    fwd_bytes, bwd_bytes = variant_bytes(wl, variant)
+    step_bytes = fwd_bytes + bwd_bytes
     value = step_bytes * world / (ms_per_step / 1e3) / 1e9
     peak, peak_src = measured_peak()
     fwd_us, bwd_us = fwd_sum / K * 1e3, bwd_sum / K * 1e3
-    fwd_gbs, bwd_gbs = wl.fwd_bytes() / fwd_us / 1e3, wl.bwd_bytes() / bwd_us / 1e3
-    traffic = recorded_traffic("situ_glu_bwd_kernel", wl.name)
+    fwd_gbs, bwd_gbs = fwd_bytes / fwd_us / 1e3, bwd_bytes / bwd_us / 1e3
+    # the kernels each pass launches for this form and shape (the forward's
+    # layout follows the library's own choice: 32-byte vectors when a half row
+    # is a multiple of 64 vectors and every pitch is 32-byte aligned)
+    vpr = I * (2 if wl.dtype == "bf16" else 4) // 16
+    fwd_kernel, bwd_kernel = {
+        "row": ("situ_glu_fwd_wide_kernel" if vpr % 64 == 0 and vpr // 2 <= 256 else "situ_glu_fwd_kernel",
+                "situ_glu_bwd_kernel"),
+        "col": ("situ_glu_fwd_ew_kernel", "situ_glu_bwd_ew_kernel"),
+        "full": ("situ_glu_fwd_ew_kernel", "situ_glu_bwd_ew_kernel"),
+        "mxfp8": ("situ_glu_fwd_mx_kernel", "situ_glu_bwd_mx_kernel"),
+    }[variant]
+    launches_per_step = 3 if variant == "col" else 2  # per-column weights: plus the column finalize
+    traffic_key = wl.name if variant == "row" else f"{wl.name}/{variant}"
+    traffic = recorded_traffic(bwd_kernel, traffic_key)
 
     # End to end through the public API with host buffers: every step copies the
     # inputs from pinned host memory, runs both passes and reads all outputs back.
     e2e = None
     if not args.no_e2e:
-        y_h = torch.empty(T, I, dtype=tdt).pin_memory()
-        d_gu_h = torch.empty(T, 2 * I, dtype=tdt).pin_memory()
-        d_rw_h = torch.empty(T, 1, dtype=torch.float32).pin_memory()
+        outputs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outputs]
         K2 = args.e2e_steps or max(1, min(K, 20))
 
         def e2e_step():
@@ -354,9 +444,8 @@ def run_ours(args):
             rw.copy_(rw_h, non_blocking=True)
             fwd()
             bwd()
-            y_h.copy_(y, non_blocking=True)
-            d_gu_h.copy_(d_gu, non_blocking=True)
-            d_rw_h.copy_(d_rw, non_blocking=True)
+            for th, td in zip(outputs_h, outputs):
+                th.copy_(td, non_blocking=True)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -374,37 +463,35 @@ def run_ours(args):
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = t.item() / K2
         h2d = input_bytes
-        d2h = y_h.numel() * y_h.element_size() + d_gu_h.numel() * d_gu_h.element_size() + d_rw_h.numel() * 4
+        d2h = sum(t.numel() * t.element_size() for t in outputs_h)
+        api = "situ_glu_fwd_mxfp8/situ_glu_bwd_mxfp8" if variant == "mxfp8" else "situ_glu_fwd/situ_glu_bwd"
         e2e = {"value": step_bytes * world / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": K2,
-               "api": "ffn_gated_activation_b200.situ_glu_fwd/situ_glu_bwd on pinned host copies"}
+               "api": f"ffn_gated_activation_b200.{api} on pinned host copies"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, rows_done, secs = cpu_oracle_rate(wl, beta, x, args.cpu_seconds)
+        rate, rows_done, secs = cpu_oracle_rate(wl, beta, x, args.cpu_seconds, variant)
         cpu = {"value": rate, "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": f"first {rows_done} of {T} rows, fwd + bwd, {secs:.1f} s, single-threaded fp64"}
 
-    launches_per_step = 2
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": workload_config(wl, beta, l2_note, world),
+            "config": workload_config(wl, beta, l2_note, world, variant),
             "rows_per_s": T * world / (ms_per_step / 1e3),
             "pct_of_nominal_hbm": value / world / NOMINAL_HBM_GBS * 100.0,
             "kernels": {
-                "situ_glu_fwd_kernel": {"us": fwd_us, "bytes": wl.fwd_bytes(), "GB/s": fwd_gbs,
-                                        "pct_of_nominal_8TBs": fwd_gbs / NOMINAL_HBM_GBS * 100,
-                                        "frac_of_measured_copy": fwd_gbs / peak,
-                                        "rows_per_s": T / (fwd_us / 1e6)},
-                "situ_glu_bwd_kernel": {"us": bwd_us, "bytes": wl.bwd_bytes(), "GB/s": bwd_gbs,
-                                        "pct_of_nominal_8TBs": bwd_gbs / NOMINAL_HBM_GBS * 100,
-                                        "frac_of_measured_copy": bwd_gbs / peak,
-                                        "rows_per_s": T / (bwd_us / 1e6)},
+                fwd_kernel: {"us": fwd_us, "bytes": fwd_bytes, "GB/s": fwd_gbs,
+                             "pct_of_nominal_8TBs": fwd_gbs / NOMINAL_HBM_GBS * 100,
+                             "frac_of_measured_copy": fwd_gbs / peak, "rows_per_s": T / (fwd_us / 1e6)},
+                bwd_kernel: {"us": bwd_us, "bytes": bwd_bytes, "GB/s": bwd_gbs,
+                             "pct_of_nominal_8TBs": bwd_gbs / NOMINAL_HBM_GBS * 100,
+                             "frac_of_measured_copy": bwd_gbs / peak, "rows_per_s": T / (bwd_us / 1e6)},
             },
-            "roofline": {"bound": "hbm", "kernel": "situ_glu_bwd_kernel", "achieved": bwd_gbs, "peak": peak,
+            "roofline": {"bound": "hbm", "kernel": bwd_kernel, "achieved": bwd_gbs, "peak": peak,
                          "unit": "GB/s", "frac": bwd_gbs / peak, "peak_source": f"{peak_src} copy bandwidth",
                          "traffic": traffic},
             "cpu_baseline": cpu,
