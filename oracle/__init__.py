@@ -16,6 +16,9 @@ Sources followed (see the C file for the per-function citations):
   * NeMo AutoModel API, kimi_k3.situ: `_situ_fwd_core` (Y = situ(g) up(u0) w,
     optional linear beta), `_situ_bwd_core` (analytic d_g, d_u and the
     routing-weight reduction), `_WeightedSiTUFunction` (gate/up halves).
+  * Megatron-LM PR #6673, "Design": the fused grouped GEMM + SiTU-GLU, taken
+    as FC1 (per-expert grouped GEMM) followed by the activation
+    (fc1_oracle.c).
   * OCP Microscaling Formats (MX) v1.0 for the MXFP8 outputs (E4M3 elements,
     E8M0 block scales, blocks of 32), the format of the MXFP8 recipe named in
     Megatron-LM PR #6673 "Test results".
@@ -35,6 +38,8 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 SOURCE = os.path.join(_HERE, "situ_oracle.c")
 MX_SOURCE = os.path.join(_HERE, "mx_oracle.c")  # MXFP8 block scaling (OCP MX v1.0)
+FC1_SOURCE = os.path.join(_HERE, "fc1_oracle.c")  # FC1 (grouped) followed by SiTU-GLU
+SOURCES = [SOURCE, MX_SOURCE, FC1_SOURCE]
 LIBRARY = os.path.join(_HERE, "libsitu_oracle.so")
 
 DTYPE_BF16 = 0
@@ -58,10 +63,10 @@ def build(output: str = LIBRARY, mutant: int = 0, force: bool = False) -> str:
     copy with the planted mistake number ``mutant`` (used only by the pin tests
     to show the pins reject it).  Rebuilds when the source is newer."""
     if (not force and os.path.exists(output)
-            and os.path.getmtime(output) >= max(os.path.getmtime(SOURCE), os.path.getmtime(MX_SOURCE))):
+            and os.path.getmtime(output) >= max(os.path.getmtime(p) for p in SOURCES)):
         return output
     tmp = output + f".tmp{os.getpid()}"
-    cmd = ["gcc", *CFLAGS, f"-DSITU_ORACLE_MUTANT={int(mutant)}", SOURCE, MX_SOURCE, "-o", tmp, "-lm"]
+    cmd = ["gcc", *CFLAGS, f"-DSITU_ORACLE_MUTANT={int(mutant)}", *SOURCES, "-o", tmp, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, output)
     return output
@@ -132,6 +137,9 @@ class Oracle:
         lib.situ_oracle_mx_scale_exp.restype = _INT
         lib.situ_oracle_mxfp8_quantize.argtypes = [_VP, _I64, _I64, _I64, _INT, _VP, _VP]
         lib.situ_oracle_mxfp8_quantize.restype = _INT
+        lib.situ_oracle_fc1_fwd.argtypes = [_VP, _I64, _I64, _VP, _I64, _I64, _VP, _I64, _VP, _I64, _VP,
+                                            _DBL, _INT, _DBL, _VP, _VP, _VP]
+        lib.situ_oracle_fc1_fwd.restype = _INT
         self._lib = lib
         self.mutant_id = lib.situ_oracle_mutant_id()
 
@@ -280,6 +288,34 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle mxfp8_quantize: columns must be a multiple of 32")
         return codes, scales
+
+
+    # -- FC1 followed by SiTU-GLU (fc1_oracle.c) ------------------------------
+
+    def fc1_fwd(self, x, w1, offsets, inter, rw, beta, linear_beta=None, rows=None):
+        """(Y [nrows, I], error scale [nrows, I], unrounded gate_up [nrows, 2I]),
+        all float64, for token rows of x (bf16 bits [T, H]) routed by
+        ``offsets`` [E + 1] to experts whose FC1 weights are w1 (bf16 bits
+        [E * 2I, H]: per expert I gate rows, then I up rows).  rw: float32 [T]
+        per-row routing weights, or None for w = 1."""
+        x = np.ascontiguousarray(x)
+        w1 = np.ascontiguousarray(w1)
+        if x.dtype != np.uint16 or w1.dtype != np.uint16:
+            raise TypeError("x and w1 are bf16 bit patterns (uint16)")
+        off = np.ascontiguousarray(np.asarray(offsets, dtype=np.int64))
+        T, hidden = x.shape
+        r, n = self._rows(rows, T)
+        rw_c = None if rw is None else np.ascontiguousarray(np.asarray(rw, dtype=np.float32).reshape(-1))
+        y = np.empty((n, inter))
+        err = np.empty((n, inter))
+        gu = np.empty((n, 2 * inter))
+        has = linear_beta is not None
+        rc = self._lib.situ_oracle_fc1_fwd(_ptr(x), x.shape[1], hidden, _ptr(w1), w1.shape[1], int(inter), _ptr(off),
+                                           off.size - 1, _ptr(r), n, _ptr(rw_c), float(beta), int(has),
+                                           float(linear_beta if has else 0.0), _ptr(y), _ptr(err), _ptr(gu))
+        if rc != 0:
+            raise ValueError("oracle fc1_fwd rejected its arguments")
+        return y, err, gu
 
 
 _DEFAULT = None

@@ -17,7 +17,10 @@ itself checked here against things other than itself:
   * special rows (G = 0, U = 0) whose gradients have closed forms;
   * brute-force compensated sums for the routing-weight gradient;
   * MXFP8 (mx_oracle.c): torch's float8_e4m3fn encoding and decoding, the
-    OCP MX format's clamp at 448, and the scale rules' defining inequalities.
+    OCP MX format's clamp at 448, and the scale rules' defining inequalities;
+  * FC1 + SiTU-GLU (fc1_oracle.c): fsum dot products and 50-digit element
+    values, exact agreement with the activation oracle on bf16-exact FC1
+    outputs, and the grouped call against per-expert calls.
 
 Each pin is a plain function of an oracle handle.  ``test_mutant_rejected``
 rebuilds situ_oracle.c with each planted mistake (-DSITU_ORACLE_MUTANT=n: a
@@ -418,6 +421,74 @@ def pin_mxfp8_blocks(o):
                 assert np.array_equal(codes[r, 32 * b:32 * b + 32], ref.view(torch.uint8).numpy()), (r, b)
 
 
+# ---- FC1 followed by SiTU-GLU (fc1_oracle.c) ---------------------------------------
+
+def _bf16(a):
+    return workloads.f32_to_bf16_bits(np.asarray(a, dtype=np.float32))
+
+
+def _widen(bits):
+    return workloads.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def pin_fc1_bruteforce(o):
+    """A tiny grouped case (3 experts, one of them empty): every FC1 output is a
+    math.fsum dot product over the hidden axis with the owning expert's gate or
+    up row, and Y is the 50-digit value of T_g(G) T_u(U) w."""
+    rng = np.random.default_rng(RNG_SEED + 3)
+    E, I, H, T = 3, 8, 24, 11
+    x = _bf16(rng.standard_normal((T, H)))
+    w1 = _bf16(0.3 * rng.standard_normal((E * 2 * I, H)))
+    offsets = [0, 4, 4, 11]
+    rw = rng.random(T).astype(np.float32)
+    y, err, gu = o.fc1_fwd(x, w1, offsets, I, rw, 4.0, 25.0)
+    xf, wf = _widen(x), _widen(w1)
+    for r in range(T):
+        e = 0 if r < 4 else 2
+        for i in range(I):
+            g = math.fsum(xf[r] * wf[e * 2 * I + i])
+            u = math.fsum(xf[r] * wf[e * 2 * I + I + i])
+            assert _close(gu[r, i], g, 1e-14, 1e-14) and _close(gu[r, I + i], u, 1e-14, 1e-14), (r, i)
+            ref = float(_mp_gate(g, 4.0) * _mp_up(u, 25.0)) * float(rw[r])
+            assert _close(y[r, i], ref, 1e-12, 1e-15), (r, i, y[r, i], ref)
+            assert err[r, i] >= 0.0
+
+
+def pin_fc1_matches_activation_oracle(o):
+    """With inputs in {-1/4, 0, 1/4} every FC1 output is k/16, |k| <= 16, a bf16
+    number: the fused oracle then equals the pinned activation oracle applied
+    to that gate_up, exactly, for every beta form."""
+    rng = np.random.default_rng(RNG_SEED + 4)
+    T, H, I = 6, 16, 8
+    x = _bf16(rng.integers(-1, 2, (T, H)) / 4.0)
+    w1 = _bf16(rng.integers(-1, 2, (2 * I, H)) / 4.0)
+    rw = rng.random(T).astype(np.float32)
+    for beta, lb in ((4.0, 25.0), (1.0, None), (16.0, 2.0)):
+        y, _, gu = o.fc1_fwd(x, w1, [0, T], I, rw, beta, lb)
+        gu_bits = _bf16(gu)
+        assert np.array_equal(_widen(gu_bits), gu)
+        assert np.array_equal(y, o.fwd(gu_bits, rw, beta, lb))
+
+
+def pin_fc1_grouped_equals_per_expert(o):
+    """The grouped call equals one call per expert on that expert's rows and weights."""
+    rng = np.random.default_rng(RNG_SEED + 5)
+    E, I, H = 4, 8, 32
+    sizes = [5, 0, 9, 3]
+    offsets = np.concatenate([[0], np.cumsum(sizes)])
+    T = int(offsets[-1])
+    x = _bf16(rng.standard_normal((T, H)))
+    w1 = _bf16(0.2 * rng.standard_normal((E * 2 * I, H)))
+    rw = rng.random(T).astype(np.float32)
+    y, _, _ = o.fc1_fwd(x, w1, offsets, I, rw, 4.0, 25.0)
+    for e in range(E):
+        a, b = offsets[e], offsets[e + 1]
+        if a == b:
+            continue
+        ye, _, _ = o.fc1_fwd(x[a:b], w1[e * 2 * I:(e + 1) * 2 * I], [0, b - a], I, rw[a:b], 4.0, 25.0)
+        assert np.array_equal(y[a:b], ye), e
+
+
 PINS = [
     pin_gate_values_mpmath,
     pin_up_values_mpmath,
@@ -437,6 +508,9 @@ PINS = [
     pin_e4m3_saturation,
     pin_mx_scale_rules,
     pin_mxfp8_blocks,
+    pin_fc1_bruteforce,
+    pin_fc1_matches_activation_oracle,
+    pin_fc1_grouped_equals_per_expert,
 ]
 
 
@@ -467,6 +541,10 @@ MUTANTS = {
     17: "E4M3 ties rounded away from zero",
     18: "E4M3 subnormal spacing 2^-10",
     19: "no-clamp scale rule bumps the exponent at equality",
+    20: "FC1 uses the next expert's weights",
+    21: "FC1 up rows taken from the gate rows",
+    22: "FC1 dot product drops the last product",
+    23: "FC1 boundary row assigned to the earlier expert",
 }
 
 
