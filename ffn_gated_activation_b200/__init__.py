@@ -16,6 +16,7 @@ from .functional import (
     WeightedSiTUFunction,
     situ_glu_bwd,
     situ_glu_bwd_mxfp8,
+    situ_glu_fc1_fwd,
     situ_glu_fwd,
     situ_glu_fwd_mxfp8,
     situlu,
@@ -34,6 +35,7 @@ __all__ = [
     "situ_glu_bwd",
     "situ_glu_fwd_mxfp8",
     "situ_glu_bwd_mxfp8",
+    "situ_glu_fc1_fwd",
     "situlu",
     "weighted_situ",
 ]

@@ -28,6 +28,7 @@
 // relative accuracy as x -> 0; below a threshold it is taken from the Taylor
 // series of 1 - exp(-x) instead.
 
+#include <cuda.h>  // CUtensorMap and its encoder's types (the encoder is fetched at run time)
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
@@ -1799,6 +1800,8 @@ __global__ void __launch_bounds__(kMaxConsumers + 32) situ_glu_bwd_tma_kernel(co
   tma_stream_body<S, GATE, HAS_LB, true>(a);
 }
 
+#include "situ_fc1.cuh"
+
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
@@ -1886,6 +1889,18 @@ int ew_align(situ_dtype_t dtype, situ_dtype_t rw_dtype) {
   return a < 16 ? a : 16;
 }
 
+// Per-call constants of the element arithmetic and the gate's exponent form.
+void fill_coeffs(double beta, int has_lb, double lb, Coeffs* c, int* gate_mode) {
+  const double kLog2eD = 1.4426950408889634;
+  c->beta = static_cast<float>(beta);
+  c->kt = static_cast<float>(2.0 * kLog2eD / beta);
+  c->lb = has_lb ? static_cast<float>(lb) : 1.0f;
+  c->inv_lb = has_lb ? static_cast<float>(1.0 / lb) : 1.0f;
+  c->ku = has_lb ? static_cast<float>(2.0 * kLog2eD / lb) : 0.0f;
+  c->bb = static_cast<float>(has_lb ? beta * lb : beta);
+  *gate_mode = beta == 4.0 ? kGateSquare : beta == 2.0 ? kGateEqual : beta == 1.0 ? kGateRoot : kGateGeneric;
+}
+
 // Checks common to fwd and bwd.  Fills coefficients and the gate mode.
 situ_status_t check_common(situ_dtype_t dtype, int64_t tokens, int64_t inter, int64_t gu_stride,
                            const void* rw, situ_dtype_t rw_dtype, situ_rw_mode_t rw_mode,
@@ -1925,14 +1940,7 @@ situ_status_t check_common(situ_dtype_t dtype, int64_t tokens, int64_t inter, in
     return fail(SITU_ERR_MISALIGNED, "inter * element size (%lld bytes) is not a multiple of 16",
                 (long long)(inter * es));
 
-  const double kLog2eD = 1.4426950408889634;
-  c->beta = static_cast<float>(beta);
-  c->kt = static_cast<float>(2.0 * kLog2eD / beta);
-  c->lb = has_lb ? static_cast<float>(lb) : 1.0f;
-  c->inv_lb = has_lb ? static_cast<float>(1.0 / lb) : 1.0f;
-  c->ku = has_lb ? static_cast<float>(2.0 * kLog2eD / lb) : 0.0f;
-  c->bb = static_cast<float>(has_lb ? beta * lb : beta);
-  *gate_mode = beta == 4.0 ? kGateSquare : beta == 2.0 ? kGateEqual : beta == 1.0 ? kGateRoot : kGateGeneric;
+  fill_coeffs(beta, has_lb, lb, c, gate_mode);
   return SITU_OK;
 }
 
@@ -2321,6 +2329,53 @@ situ_status_t fwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
   return check_launch("situ_glu_fwd");
 }
 
+// ---- FC1 grouped GEMM + SiTU-GLU: tensor maps and launch ----------------------
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map of a row-major [rows, >= inner] matrix read in boxes of
+// 64 x 128 with the 128-byte swizzle the UMMA descriptors expect.
+situ_status_t bf16_tile_map(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t pitch_elems) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr) return fail(SITU_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(pitch_elems) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(fc1::kBK), static_cast<cuuint32_t>(fc1::kBM)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SITU_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return SITU_OK;
+}
+
+using Fc1Kernel = void (*)(const CUtensorMap, const CUtensorMap, const fc1::Args);
+
+template <bool LB>
+Fc1Kernel pick_fc1_gate(int gate) {
+  switch (gate) {
+    case kGateSquare: return fc1::situ_fc1_kernel<kGateSquare, LB>;
+    case kGateEqual: return fc1::situ_fc1_kernel<kGateEqual, LB>;
+    case kGateRoot: return fc1::situ_fc1_kernel<kGateRoot, LB>;
+    default: return fc1::situ_fc1_kernel<kGateGeneric, LB>;
+  }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -2699,4 +2754,95 @@ extern "C" situ_status_t situ_glu_bwd_no_alloc(const void* gate_up, situ_dtype_t
   return situ_glu_bwd(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride, beta,
                       has_linear_beta, linear_beta, grad_out, grad_out_row_stride, d_gate_up, d_gate_up_row_stride,
                       d_rw, d_rw_stride, ws, need > 0 ? sizeof(g_noalloc_scratch) : 0, stream);
+}
+
+
+// ---------------------------------------------------------------------------
+// FC1 grouped GEMM + SiTU-GLU forward
+// ---------------------------------------------------------------------------
+
+extern "C" situ_status_t situ_glu_fc1_fwd(const void* x, int64_t tokens, int64_t hidden, int64_t x_row_stride,
+                                          const void* w1, int64_t experts, int64_t inter, int64_t w1_row_stride,
+                                          const int64_t* offsets, const void* rw, situ_dtype_t rw_dtype,
+                                          situ_rw_mode_t rw_mode, int64_t rw_stride, double beta,
+                                          int has_linear_beta, double linear_beta, void* y, int64_t y_row_stride,
+                                          void* stream) {
+  tl_last_error[0] = '\0';
+  if (!finite_positive(beta)) return fail(SITU_ERR_INVALID_ARG, "beta must be finite and > 0");
+  if (has_linear_beta != 0 && has_linear_beta != 1)
+    return fail(SITU_ERR_INVALID_ARG, "has_linear_beta must be 0 or 1");
+  if (has_linear_beta && !finite_positive(linear_beta))
+    return fail(SITU_ERR_INVALID_ARG, "linear_beta must be finite and > 0");
+  if (rw_mode != SITU_RW_ROW && rw_mode != SITU_RW_SCALAR && rw_mode != SITU_RW_NONE)
+    return fail(rw_mode == SITU_RW_COL || rw_mode == SITU_RW_FULL ? SITU_ERR_UNSUPPORTED : SITU_ERR_INVALID_ARG,
+                "situ_glu_fc1_fwd takes per-row, broadcast or no routing weights");
+  if (rw_mode != SITU_RW_NONE && !valid_dtype(rw_dtype))
+    return fail(SITU_ERR_INVALID_ARG, "rw_dtype %d is not a situ_dtype_t", (int)rw_dtype);
+  if (tokens < 0) return fail(SITU_ERR_INVALID_ARG, "tokens = %lld < 0", (long long)tokens);
+  if (hidden < fc1::kBK || hidden % fc1::kBK != 0)
+    return fail(SITU_ERR_UNSUPPORTED, "hidden must be a positive multiple of %d, got %lld", fc1::kBK,
+                (long long)hidden);
+  if (inter < fc1::kBN || inter % fc1::kBN != 0)
+    return fail(SITU_ERR_UNSUPPORTED, "inter must be a positive multiple of %d, got %lld", fc1::kBN,
+                (long long)inter);
+  if (experts < 1 || experts > fc1::kMaxExperts)
+    return fail(SITU_ERR_UNSUPPORTED, "experts must be in [1, %d], got %lld", fc1::kMaxExperts, (long long)experts);
+  if (tokens > INT32_MAX || experts * 2 * inter > INT32_MAX || hidden > INT32_MAX)
+    return fail(SITU_ERR_UNSUPPORTED, "sizes exceed the 32-bit tensor-map coordinates");
+  if (x_row_stride < hidden || w1_row_stride < hidden || y_row_stride < inter)
+    return fail(SITU_ERR_INVALID_ARG, "a row stride is shorter than its row");
+  if (rw_mode == SITU_RW_ROW && rw_stride < 0) return fail(SITU_ERR_INVALID_ARG, "rw_stride < 0");
+  if (tokens == 0) return SITU_OK;
+  if (x == nullptr || w1 == nullptr || offsets == nullptr || y == nullptr ||
+      (rw_mode != SITU_RW_NONE && rw == nullptr))
+    return fail(SITU_ERR_INVALID_ARG, "x, w1, offsets, y or rw is NULL");
+  if (rw_mode == SITU_RW_NONE && rw != nullptr) return fail(SITU_ERR_INVALID_ARG, "rw must be NULL for SITU_RW_NONE");
+  if (!span_fits(tokens, x_row_stride, hidden, 2) || !span_fits(experts * 2 * inter, w1_row_stride, hidden, 2) ||
+      !span_fits(tokens, y_row_stride, inter, 2) ||
+      (rw_mode == SITU_RW_ROW && !span_fits(tokens, rw_stride, 1, elem_size(rw_dtype))))
+    return fail(SITU_ERR_INVALID_ARG, "tensor extent overflows int64");
+  if (!aligned(x, 16) || !aligned(w1, 16) || !aligned(y, 16) || (x_row_stride * 2) % 16 != 0 ||
+      (w1_row_stride * 2) % 16 != 0 || (y_row_stride * 2) % 16 != 0 || !aligned(offsets, 8) ||
+      (rw_mode != SITU_RW_NONE && !aligned(rw, elem_size(rw_dtype))))
+    return fail(SITU_ERR_MISALIGNED, "x, w1, y (16 bytes), offsets (8) or rw base or row pitch misaligned");
+  const Span s_y = matrix_span(y, tokens, y_row_stride, inter, 2);
+  const Span s_off = {reinterpret_cast<uintptr_t>(offsets),
+                      reinterpret_cast<uintptr_t>(offsets) + static_cast<uintptr_t>(experts + 1) * 8};
+  if (overlap(s_y, matrix_span(x, tokens, x_row_stride, hidden, 2)) ||
+      overlap(s_y, matrix_span(w1, experts * 2 * inter, w1_row_stride, hidden, 2)) || overlap(s_y, s_off) ||
+      overlap(s_y, weight_span(rw, rw_mode, tokens, rw_stride, inter, elem_size(rw_dtype))))
+    return fail(SITU_ERR_INVALID_ARG, "y overlaps an input");
+
+  fc1::Args a{};
+  a.offsets = offsets;
+  a.experts = static_cast<int>(experts);
+  a.tokens = tokens;
+  a.hidden = static_cast<int>(hidden);
+  a.inter = static_cast<int>(inter);
+  a.rw = {rw, rw_stride, static_cast<int>(rw_mode), (rw_mode != SITU_RW_NONE && rw_dtype == SITU_DTYPE_BF16) ? 1 : 0};
+  a.y = static_cast<char*>(y);
+  a.y_pitch = y_row_stride * 2;
+  int gate = kGateGeneric;
+  fill_coeffs(beta, has_linear_beta, linear_beta, &a.c, &gate);
+
+  CUtensorMap mx, mw;
+  situ_status_t st = bf16_tile_map(&mx, x, hidden, tokens, x_row_stride);
+  if (st != SITU_OK) return st;
+  st = bf16_tile_map(&mw, w1, hidden, experts * 2 * inter, w1_row_stride);
+  if (st != SITU_OK) return st;
+
+  Fc1Kernel k = has_linear_beta ? pick_fc1_gate<true>(gate) : pick_fc1_gate<false>(gate);
+  const int smem = fc1::kStages * fc1::kStageBytes + 1024 + fc1::kHeaderBytes +
+                   static_cast<int>(experts) * (8 + 8 + 4) + 8;
+  cudaError_t err = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(err));
+  int sms = 0;
+  st = device_sm_count(&sms);
+  if (st != SITU_OK) return st;
+  int grid = sms;
+  const int cap = g_max_ctas.load(std::memory_order_relaxed);
+  if (cap > 0 && grid > cap) grid = cap;
+  k<<<grid, fc1::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(mx, mw, a);
+  return check_launch("situ_glu_fc1_fwd");
 }

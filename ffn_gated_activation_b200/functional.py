@@ -265,6 +265,53 @@ def situ_glu_bwd_mxfp8(gate_up: torch.Tensor, routing_weights, grad_out: torch.T
     return data, scale, (d_rw if want else None)
 
 
+def situ_glu_fc1_fwd(x: torch.Tensor, w1: torch.Tensor, offsets: torch.Tensor, routing_weights=None,
+                     beta: float = DEFAULT_BETA, linear_beta: float | None = DEFAULT_LINEAR_BETA,
+                     out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """FC1 grouped GEMM with the SiTU-GLU epilogue (Megatron-LM PR #6673
+    "Design": the fused grouped GEMM + SiTU-GLU).
+
+    x: bf16 [T, H] token rows grouped by expert; w1: bf16 [E, 2I, H] (or
+    [E * 2I, H]) -- per expert I gate rows then I up rows; offsets: int64
+    [E + 1] on x's device, rows of expert e = [offsets[e], offsets[e+1]);
+    routing_weights: [T, 1] / [T] per row, one value, or None.  Returns bf16
+    Y [T, I]; rows outside every expert are left as they are in ``out``
+    (uninitialised when out is None)."""
+    _check_beta(beta, linear_beta)
+    if x.dtype != torch.bfloat16 or w1.dtype != torch.bfloat16:
+        raise TypeError("x and w1 must be bfloat16")
+    if x.device.type != "cuda" or w1.device != x.device or offsets.device != x.device:
+        raise ValueError("x, w1 and offsets must be on the same CUDA device")
+    if offsets.dtype != torch.int64 or offsets.dim() != 1:
+        raise TypeError("offsets must be a 1-D int64 tensor")
+    experts = offsets.numel() - 1
+    if x.dim() != 2:
+        raise ValueError("x must be [tokens, hidden]")
+    tokens, hidden = x.shape
+    w2 = w1.reshape(-1, w1.shape[-1])
+    if w2.shape[1] != hidden or w2.shape[0] % (2 * experts):
+        raise ValueError(f"w1 {tuple(w1.shape)} does not match {experts} experts of hidden size {hidden}")
+    inter = w2.shape[0] // (2 * experts)
+    if x.stride(1) != 1:
+        x = x.contiguous()
+    if w2.stride(1) != 1:
+        w2 = w2.contiguous()
+    mode, rw, rw_stride = routing_mode((tokens,), inter, routing_weights)
+    if mode in (abi.SITU_RW_COL, abi.SITU_RW_FULL):
+        raise NotImplementedError("situ_glu_fc1_fwd takes per-row, broadcast or no routing weights")
+    rw_dtype = _dtype_code(rw, "routing_weights") if rw is not None else abi.SITU_DTYPE_F32
+    if out is None:
+        out = torch.empty(tokens, inter, dtype=torch.bfloat16, device=x.device)
+    st = abi.situ_glu_fc1_fwd(x.data_ptr(), tokens, hidden, x.stride(0) if tokens > 1 else hidden,
+                              w2.data_ptr(), experts, inter, w2.stride(0), offsets.data_ptr(),
+                              rw.data_ptr() if rw is not None else None, rw_dtype, mode, rw_stride,
+                              float(beta), int(linear_beta is not None),
+                              float(linear_beta) if linear_beta is not None else 0.0,
+                              out.data_ptr(), out.stride(0) if tokens > 1 else inter, _stream_handle(stream))
+    abi.check(st, "situ_glu_fc1_fwd")
+    return out
+
+
 class WeightedSiTUFunction(torch.autograd.Function):
     """Routing-weighted SiTU-GLU with the analytic fused backward.
 

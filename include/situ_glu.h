@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define SITU_GLU_ABI_VERSION 3
+#define SITU_GLU_ABI_VERSION 4
 
 typedef enum situ_status {
   SITU_OK = 0,
@@ -228,6 +228,42 @@ situ_status_t situ_glu_bwd_mxfp8(const void *gate_up, situ_dtype_t dtype, int64_
                                  void *d_rw, int64_t d_rw_stride,
                                  void *workspace, size_t workspace_bytes,
                                  void *stream);
+
+/* ---- FC1 grouped GEMM + SiTU-GLU --------------------------------------------
+ * Megatron-LM PR #6673, "Design": with a SiTU-capable cuDNN frontend FC1's
+ * grouped GEMM and SiTU-GLU run as one fused operation.  For token row r of
+ * expert e (rows [offsets[e], offsets[e+1]) of x):
+ *   G[r, i] = sum_k x[r, k] w1[e 2I + i, k],  U[r, i] = sum_k x[r, k] w1[e 2I + I + i, k]
+ *   y[r, i] = T_g(G) T_u(U) w[r]                (as situ_glu_fwd, from fp32 G, U)
+ * The products accumulate in fp32 on the tensor cores; G and U are never
+ * written.
+ *
+ *   x         bf16 [tokens, >= hidden], row pitch x_row_stride elements
+ *   w1        bf16 [experts * 2 inter, >= hidden], row pitch w1_row_stride:
+ *             expert e's inter gate rows, then its inter up rows
+ *   offsets   DEVICE int64 [experts + 1], non-decreasing; each value is
+ *             clamped to [0, tokens] (a decreasing pair is an empty expert).
+ *             Rows outside every expert are not written.  Overlapping ranges
+ *             (non-monotone offsets) leave those rows unspecified.
+ *   rw        per-row (SITU_RW_ROW), broadcast (SITU_RW_SCALAR) or no
+ *             (SITU_RW_NONE) routing weights, as for situ_glu_fwd
+ *   y         bf16 [tokens, >= inter], row pitch y_row_stride; must not
+ *             overlap an input
+ * hidden must be a multiple of 64, inter of 128, experts in [1, 1024]
+ * (SITU_ERR_UNSUPPORTED otherwise); x, w1, y 16-byte aligned with row pitches
+ * of a multiple of 16 bytes, offsets 8-byte aligned.  tokens == 0 launches
+ * nothing.  The kernel uses the whole tensor memory and about 200 KiB of
+ * shared memory of each SM it runs on; every internal wait is bounded and an
+ * expired wait is reported by situ_glu_device_status.
+ */
+situ_status_t situ_glu_fc1_fwd(const void *x, int64_t tokens, int64_t hidden, int64_t x_row_stride,
+                               const void *w1, int64_t experts, int64_t inter, int64_t w1_row_stride,
+                               const int64_t *offsets,
+                               const void *rw, situ_dtype_t rw_dtype, situ_rw_mode_t rw_mode,
+                               int64_t rw_stride,
+                               double beta, int has_linear_beta, double linear_beta,
+                               void *y, int64_t y_row_stride,
+                               void *stream);
 
 /* Static, human-readable name of a status code. */
 const char *situ_glu_status_string(situ_status_t status);

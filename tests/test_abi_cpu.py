@@ -58,7 +58,7 @@ def test_binding_covers_the_header_exactly():
 
 
 def test_version_and_status_strings(native_lib_path):
-    assert abi.situ_glu_abi_version() == abi.ABI_VERSION == 3
+    assert abi.situ_glu_abi_version() == abi.ABI_VERSION == 4
     assert abi.situ_glu_status_string(OK) == "SITU_OK"
     assert abi.situ_glu_status_string(MISAL) == "SITU_ERR_MISALIGNED"
     assert abi.situ_glu_status_string(99) == "SITU_ERR_UNKNOWN"
@@ -305,3 +305,49 @@ def test_bwd_mxfp8_argument_errors(name, kw, want, native_lib_path):
 def test_mxfp8_zero_tokens_is_a_no_op(native_lib_path):
     assert fwd_mx(tokens=0, y_data=None, y_scale=None) == OK
     assert bwd_mx(tokens=0, d_gate_up_data=None, d_gate_up_scale=None, d_rw=None) == OK
+
+
+# ---- FC1 grouped GEMM + SiTU-GLU: argument checks run before any CUDA call -------
+
+XP, W1P, OFFP, YP = 0x20000000, 0x28000000, 0x30000000, 0x38000000
+
+
+def fc1(**kw):
+    a = dict(x=XP, tokens=256, hidden=128, x_row_stride=128, w1=W1P, experts=2, inter=128, w1_row_stride=128,
+             offsets=OFFP, rw=RW, rw_dtype=F32, rw_mode=ROW, rw_stride=1, beta=4.0, has_linear_beta=1,
+             linear_beta=25.0, y=YP, y_row_stride=128, stream=None)
+    a.update(kw)
+    return abi.situ_glu_fc1_fwd(**a)
+
+
+FC1_CASES = [
+    ("hidden not a multiple of 64", dict(hidden=96, x_row_stride=96, w1_row_stride=96), UNSUP),
+    ("inter not a multiple of 128", dict(inter=64, y_row_stride=64), UNSUP),
+    ("no experts", dict(experts=0), UNSUP),
+    ("too many experts", dict(experts=1025), UNSUP),
+    ("per-column weights", dict(rw_mode=3), UNSUP),
+    ("bad rw_mode", dict(rw_mode=9), INVALID),
+    ("negative tokens", dict(tokens=-1), INVALID),
+    ("x stride short", dict(x_row_stride=64), INVALID),
+    ("w1 stride short", dict(w1_row_stride=64), INVALID),
+    ("y stride short", dict(y_row_stride=64), INVALID),
+    ("x NULL", dict(x=None), INVALID),
+    ("offsets NULL", dict(offsets=None), INVALID),
+    ("x misaligned", dict(x=XP + 8), MISAL),
+    ("y pitch not 16-byte", dict(y_row_stride=132), MISAL),
+    ("offsets misaligned", dict(offsets=OFFP + 4), MISAL),
+    ("y overlaps x", dict(y=XP + 256), INVALID),
+    ("y overlaps offsets", dict(y=OFFP - 64), INVALID),
+    ("beta nan", dict(beta=float("nan")), INVALID),
+    ("linear beta zero", dict(linear_beta=0.0), INVALID),
+    ("rw with SITU_RW_NONE", dict(rw_mode=2), INVALID),
+]
+
+
+@pytest.mark.parametrize("name,kw,want", FC1_CASES, ids=[c[0] for c in FC1_CASES])
+def test_fc1_argument_errors(name, kw, want, native_lib_path):
+    assert fc1(**kw) == want, abi.situ_glu_last_error()
+
+
+def test_fc1_zero_tokens_is_a_no_op(native_lib_path):
+    assert fc1(tokens=0, x=None, offsets=None, y=None) == OK

@@ -29,6 +29,9 @@ TENSOR_ROUTING = 2
 TENSOR_GRAD_OUT = 3
 TENSOR_COL_WEIGHTS = 4
 TENSOR_ELEM_WEIGHTS = 5
+TENSOR_FC1_X = 6
+TENSOR_FC1_W = 7
+TENSOR_FC1_SPLIT = 8
 
 
 @dataclass(frozen=True)
@@ -246,3 +249,50 @@ def inputs(wl: Workload, tokens: int | None = None, inter: int | None = None) ->
         "routing_weights": routing_weights(wl, tokens),
         "grad_out": grad_out(wl, tokens, inter),
     }
+
+
+# ---- FC1 (grouped GEMM) inputs -----------------------------------------------------
+
+def expert_offsets(tokens: int, experts: int, seed: int, skew: float = 1.0) -> np.ndarray:
+    """Row offsets [E + 1] of ``tokens`` token rows grouped by expert: expert
+    sizes from a Dirichlet(skew) share of the rows (uneven, some possibly
+    empty), rounded so that they add up to ``tokens``."""
+    rng = _rng(seed, TENSOR_FC1_SPLIT, 0)
+    share = rng.dirichlet(np.full(experts, float(skew)))
+    sizes = np.floor(share * tokens).astype(np.int64)
+    sizes[: tokens - int(sizes.sum())] += 1
+    return np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
+
+
+def fc1_inputs(tokens: int, hidden: int, inter: int, experts: int, seed: int, w_std: float | None = None):
+    """x bf16 [T, H] ~ N(0, 1); w1 bf16 [E * 2I, H] ~ N(0, w_std) (default
+    3 / sqrt(H), so that G and U ~ N(0, 3) like the routed-MoE rows); row
+    offsets from expert_offsets; per-row weights U(0, 1) float32.  x is drawn
+    in 64-row blocks, w1 in 64-row blocks of its own."""
+    w_std = 3.0 / np.sqrt(hidden) if w_std is None else w_std
+    x = np.empty((tokens, hidden), dtype=np.uint16)
+
+    def fill_x(b):
+        r0 = b * BLOCK_ROWS
+        n = min(BLOCK_ROWS, tokens - r0)
+        x[r0:r0 + n] = f32_to_bf16_bits(_rng(seed, TENSOR_FC1_X, b).standard_normal((BLOCK_ROWS, hidden))[:n]
+                                        .astype(np.float32))
+
+    _fill_blocks(tokens, fill_x)
+    rows_w = experts * 2 * inter
+    w1 = np.empty((rows_w, hidden), dtype=np.uint16)
+
+    def fill_w(b):
+        r0 = b * BLOCK_ROWS
+        n = min(BLOCK_ROWS, rows_w - r0)
+        v = _rng(seed, TENSOR_FC1_W, b).standard_normal((BLOCK_ROWS, hidden))[:n] * w_std
+        w1[r0:r0 + n] = f32_to_bf16_bits(v.astype(np.float32))
+
+    _fill_blocks(rows_w, fill_w)
+    offsets = expert_offsets(tokens, experts, seed)
+    rw = np.empty(tokens, dtype=np.float32)
+    for b in range((tokens + BLOCK_ROWS - 1) // BLOCK_ROWS):
+        r0 = b * BLOCK_ROWS
+        n = min(BLOCK_ROWS, tokens - r0)
+        rw[r0:r0 + n] = _rng(seed, TENSOR_ROUTING, b).random(BLOCK_ROWS)[:n].astype(np.float32)
+    return {"x": x, "w1": w1, "offsets": offsets, "routing_weights": rw}
