@@ -14,7 +14,10 @@ d_gate_up and d_w), plus rows/s.
 MoE form): per-column [I] or per-element [T, I] weights, or MXFP8 outputs
 (E4M3 codes + E8M0 scales for Y and d_gate_up, OCP rule).  Algorithmic
 bytes follow the form (weights read, weight gradients written, one byte per
-code plus one per 32 codes).
+code plus one per 32 codes).  --variant fc1 times the fused FC1 grouped GEMM
++ SiTU-GLU forward on the routed-MoE rows (hidden 7168, 8 local experts) in
+TFLOP/s against the tensor-core peak, with the unfused cuBLAS GEMMs +
+SiTU-GLU kernel timed beside it.
 
 For N > 1 launch one process per GPU with torchrun; every rank runs the same
 per-GPU workload (weak scaling, no collective on the data path), the step
@@ -60,7 +63,7 @@ def parse_args(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-oracle sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--variant", choices=["row", "col", "full", "mxfp8"], default="row",
+    p.add_argument("--variant", choices=["row", "col", "full", "mxfp8", "fc1"], default="row",
                    help="routing-weight form or output format timed (default: per-row weights)")
     p.add_argument("--flush", choices=["auto", "always", "never"], default="auto",
                    help="flush L2 before every step (auto: when the inputs fit in L2)")
@@ -193,6 +196,49 @@ class ClockSampler:
                 "power_w_max": round(max(s[2] for s in self.samples), 1), "source": "nvml"}
 
 
+# The fused FC1 workload: the routed-MoE token rows (32768 rows, I = 2048) fed
+# by a hidden size of 7168, grouped over 8 local experts with an uneven split.
+FC1_HIDDEN = 7168
+FC1_EXPERTS = 8
+FC1_METRIC = "fused FC1 grouped GEMM + SiTU-GLU forward TFLOP/s"
+
+
+def fc1_workload(wl):
+    """Inputs of the fused FC1 bench: (x, w1, offsets, routing weights) on the
+    host, from the routed-MoE rows' sizes and seed."""
+    d = workloads.fc1_inputs(wl.tokens, FC1_HIDDEN, wl.inter, FC1_EXPERTS, wl.seed)
+    d["offsets"] = workloads.expert_offsets(wl.tokens, FC1_EXPERTS, wl.seed, skew=2.0)
+    d["routing_weights"] = workloads.routing_weights(wl)
+    return d
+
+
+def fc1_flops(wl) -> float:
+    return 2.0 * wl.tokens * FC1_HIDDEN * 2 * wl.inter
+
+
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback"
+
+
+def fc1_cpu_rate(wl, beta, d, seconds: float):
+    """The fp64 FC1 oracle on the first rows until ``seconds`` pass: TFLOP/s."""
+    import oracle
+    o = oracle.load()
+    per_row = 2.0 * FC1_HIDDEN * 2 * wl.inter
+    done, t0 = 0, time.perf_counter()
+    while done < wl.tokens and time.perf_counter() - t0 < seconds:
+        rows = np.arange(done, min(wl.tokens, done + 8), dtype=np.int64)
+        o.fc1_fwd(d["x"], d["w1"], d["offsets"], wl.inter, d["routing_weights"], beta, wl.linear_beta, rows=rows)
+        done += rows.size
+    dt = time.perf_counter() - t0
+    return per_row * done / dt / 1e12, done, dt
+
+
 def variant_bytes(wl, variant: str):
     """Algorithmic bytes (forward, backward) of one pass over the workload in
     the given form.  Per-row weights: read gate_up and w, write Y; read
@@ -260,6 +306,8 @@ def run_reference(args):
     wl = workloads.workload(args.config)
     beta = args.beta if args.beta is not None else wl.betas[0]
     world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.variant == "fc1":
+        return run_reference_fc1(args, wl, beta, world)
     rows_per_step = max(1, min(wl.tokens, (1 << 17) // wl.inter))
     x = workloads.inputs(wl, tokens=rows_per_step)
     import oracle
@@ -300,6 +348,188 @@ def run_reference(args):
     return 0
 
 
+def run_reference_fc1(args, wl, beta, world):
+    d = fc1_workload(wl)
+    import oracle
+    o = oracle.load()
+    rows_per_step = 4
+    per_row = 2.0 * FC1_HIDDEN * 2 * wl.inter
+    rows = np.arange(rows_per_step, dtype=np.int64)
+
+    def step():
+        o.fc1_fwd(d["x"], d["w1"], d["offsets"], wl.inter, d["routing_weights"], beta, wl.linear_beta, rows=rows)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = per_row * rows_per_step * args.steps / dt / 1e12
+    sample = (f"{rows_per_step} of {wl.tokens} rows per step, {args.steps} steps, single-threaded fp64 FC1 oracle "
+              f"(hidden {FC1_HIDDEN}, {FC1_EXPERTS} experts)")
+    line = {
+        "impl": "reference", "metric": FC1_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": fc1_config(wl, beta, "n/a (host)", 1),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def fc1_config(wl, beta, l2_note, world):
+    return {
+        "workload": (f"fused FC1: x bf16 [{wl.tokens}, {FC1_HIDDEN}] ~ N(0,1), w1 bf16 [{FC1_EXPERTS} x {2 * wl.inter},"
+                     f" {FC1_HIDDEN}] ~ N(0, 3/sqrt({FC1_HIDDEN})), {FC1_EXPERTS} experts (Dirichlet(2) split), "
+                     f"Y bf16 [{wl.tokens}, {wl.inter}]"),
+        "name": f"{wl.name}/fc1",
+        "tokens": wl.tokens, "hidden": FC1_HIDDEN, "inter": wl.inter, "experts": FC1_EXPERTS,
+        "beta": beta, "linear_beta": wl.linear_beta,
+        "routing_weights": f"top-{wl.topk} softmax weights per row",
+        "l2": l2_note,
+        "parallelism": f"replicas x{world} (weak scaling; no collective)",
+    }
+
+
+def run_ours_fc1(args, wl, beta, dev, world, rank, local, barrier):
+    import torch
+    import torch.distributed as dist
+
+    import ffn_gated_activation_b200 as pkg
+
+    lb = wl.linear_beta
+    T, I = wl.tokens, wl.inter
+    d = fc1_workload(wl)
+
+    def pinned(a):
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.pin_memory()
+
+    x_h, w1_h = pinned(d["x"]), pinned(d["w1"])
+    off_h = torch.from_numpy(d["offsets"]).pin_memory()
+    rw_h = torch.from_numpy(d["routing_weights"]).reshape(T, 1).pin_memory()
+    x, w1, off, rw = x_h.to(dev), w1_h.to(dev), off_h.to(dev), rw_h.to(dev)
+    y = torch.empty(T, I, dtype=torch.bfloat16, device=dev)
+    flops = fc1_flops(wl)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd():
+        pkg.situ_glu_fc1_fwd(x, w1, off, rw, beta, lb, out=y)
+
+    for _ in range(max(3, args.warmup)):
+        fwd()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for a, b in ev:
+        a.record(stream)
+        fwd()
+        b.record(stream)
+    torch.cuda.synchronize()
+    clocks.stop()
+    barrier()
+    times = torch.tensor([sum(a.elapsed_time(b) for a, b in ev)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    ms = times.item() / K
+    tflops = flops / (ms / 1e3) / 1e12
+    peak, peak_src = measured_tensor_peak()
+
+    # The unfused pipeline on the same data: one cuBLAS GEMM per expert into a
+    # bf16 gate_up buffer, then the SiTU-GLU kernel over all rows.
+    offs = d["offsets"]
+    gu = torch.empty(T, 2 * I, dtype=torch.bfloat16, device=dev)
+    w1e = w1.view(FC1_EXPERTS, 2 * I, FC1_HIDDEN)
+
+    def unfused():
+        for e in range(FC1_EXPERTS):
+            a0, a1 = int(offs[e]), int(offs[e + 1])
+            if a1 > a0:
+                torch.matmul(x[a0:a1], w1e[e].t(), out=gu[a0:a1])
+        pkg.situ_glu_fwd(gu, rw, beta, lb, out=y)
+
+    for _ in range(3):
+        unfused()
+    torch.cuda.synchronize()
+    ue = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(max(3, K // 2))]
+    for a, b in ue:
+        a.record(stream)
+        unfused()
+        b.record(stream)
+    torch.cuda.synchronize()
+    unfused_ms = statistics.median([a.elapsed_time(b) for a, b in ue])
+    del gu
+
+    e2e = None
+    if not args.no_e2e:
+        y_h = torch.empty(T, I, dtype=torch.bfloat16).pin_memory()
+        K2 = args.e2e_steps or max(1, min(K, 10))
+
+        def e2e_step():
+            x.copy_(x_h, non_blocking=True)
+            w1.copy_(w1_h, non_blocking=True)
+            off.copy_(off_h, non_blocking=True)
+            rw.copy_(rw_h, non_blocking=True)
+            fwd()
+            y_h.copy_(y, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(K2):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        t = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item() / K2
+        h2d = sum(t_.numel() * t_.element_size() for t_ in (x_h, w1_h, off_h, rw_h))
+        e2e = {"value": flops * world / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": y_h.numel() * 2, "ms_per_step": e2e_ms, "steps": K2,
+               "api": "ffn_gated_activation_b200.situ_glu_fc1_fwd on pinned host copies"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, rows_done, secs = fc1_cpu_rate(wl, beta, d, args.cpu_seconds)
+        cpu = {"value": rate, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+               "sample": f"first {rows_done} of {T} rows, {secs:.1f} s, single-threaded fp64 FC1 oracle"}
+    if rank == 0:
+        line = {
+            "metric": FC1_METRIC, "value": tflops * world, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": fc1_config(wl, beta, "inputs 940 MB exceed the 126 MB L2; no flush", world),
+            "kernels": {"fc1::situ_fc1_kernel": {"us": ms * 1e3, "TFLOP/s": tflops, "frac_of_measured_bf16": tflops / peak}},
+            "unfused": {"ms": unfused_ms, "TFLOP/s": flops / (unfused_ms / 1e3) / 1e12,
+                        "what": "cuBLAS bf16 GEMM per expert (torch.matmul) into gate_up, then situ_glu_fwd"},
+            "roofline": {"bound": "tensor", "kernel": "fc1::situ_fc1_kernel", "achieved": tflops, "peak": peak,
+                         "unit": "TFLOP/s", "frac": tflops / peak, "peak_source": f"{peak_src} cuBLAS bf16 (burst)",
+                         "traffic": recorded_traffic("situ_fc1_kernel", f"{wl.name}/fc1")},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": K,
+            "clocks": clocks.summary(),
+            "device_status": pkg.abi.situ_glu_device_status(0),
+            "device": torch.cuda.get_device_name(dev),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 # ---- our arm -----------------------------------------------------------------------
 
 def run_ours(args):
@@ -327,6 +557,8 @@ def run_ours(args):
 
     wl = workloads.workload(args.config)
     beta = args.beta if args.beta is not None else wl.betas[0]
+    if args.variant == "fc1":
+        return run_ours_fc1(args, wl, beta, dev, world, rank, local, barrier)
     lb = wl.linear_beta
     T, I = wl.tokens, wl.inter
     x = workloads.inputs(wl)

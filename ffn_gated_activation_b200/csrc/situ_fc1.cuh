@@ -47,7 +47,10 @@ constexpr int kAccBufs = 2;
 constexpr int kTmemCols = kAccCols * kAccBufs;  // 512: the whole TMEM of the SM
 constexpr int kThreads = 192;              // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int kEpiThreads = 128;
-constexpr int kGroupM = 8;
+#ifndef SITU_FC1_GROUP_M
+#define SITU_FC1_GROUP_M 8
+#endif
+constexpr int kGroupM = SITU_FC1_GROUP_M;  // row tiles that sweep the column tiles together
 constexpr int kMaxExperts = 1024;
 // Header after the ring: 12 mbarriers, TMEM base and abort flag, the drain
 // mbarrier; then per-expert tables (row ranges, first tile).
