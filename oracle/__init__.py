@@ -19,6 +19,8 @@ Sources followed (see the C file for the per-function citations):
   * Megatron-LM PR #6673, "Design": the fused grouped GEMM + SiTU-GLU, taken
     as FC1 (per-expert grouped GEMM) followed by the activation
     (fc1_oracle.c).
+  * NeMo AutoModel API, kimi_k3.situ `_attn_res_core` / `_apply_attn_res`:
+    the attention-residual mixing chain (attn_res_oracle.c).
   * OCP Microscaling Formats (MX) v1.0 for the MXFP8 outputs (E4M3 elements,
     E8M0 block scales, blocks of 32), the format of the MXFP8 recipe named in
     Megatron-LM PR #6673 "Test results".
@@ -39,7 +41,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 SOURCE = os.path.join(_HERE, "situ_oracle.c")
 MX_SOURCE = os.path.join(_HERE, "mx_oracle.c")  # MXFP8 block scaling (OCP MX v1.0)
 FC1_SOURCE = os.path.join(_HERE, "fc1_oracle.c")  # FC1 (grouped) followed by SiTU-GLU
-SOURCES = [SOURCE, MX_SOURCE, FC1_SOURCE]
+ATTN_RES_SOURCE = os.path.join(_HERE, "attn_res_oracle.c")  # attention-residual mixing core
+SOURCES = [SOURCE, MX_SOURCE, FC1_SOURCE, ATTN_RES_SOURCE]
 LIBRARY = os.path.join(_HERE, "libsitu_oracle.so")
 
 DTYPE_BF16 = 0
@@ -140,6 +143,9 @@ class Oracle:
         lib.situ_oracle_fc1_fwd.argtypes = [_VP, _I64, _I64, _VP, _I64, _I64, _VP, _I64, _VP, _I64, _VP,
                                             _DBL, _INT, _DBL, _VP, _VP, _VP]
         lib.situ_oracle_fc1_fwd.restype = _INT
+        lib.situ_oracle_attn_res.argtypes = [_VP, _I64, _I64, _I64, _VP, _I64, _INT, _I64, _VP, _INT, _VP, _INT,
+                                             _DBL, _VP, _I64, _VP, _VP, _VP]
+        lib.situ_oracle_attn_res.restype = _INT
         self._lib = lib
         self.mutant_id = lib.situ_oracle_mutant_id()
 
@@ -316,6 +322,39 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle fc1_fwd rejected its arguments")
         return y, err, gu
+
+
+    # -- attention-residual mixing core (attn_res_oracle.c) -------------------
+
+    def attn_res(self, blocks, prefix, norm_weight, proj_weight, eps, rows=None):
+        """(out [nrows, H], combine magnitude [nrows, H], prob [nrows, S]) in
+        float64.  blocks: [T, B, H] stored sums (bf16 bits or float32) or None;
+        prefix: [T, H] current sum (same dtype) or None -- appended as the last
+        source.  norm_weight, proj_weight: [H] float32 or bf16 bits."""
+        if blocks is None and prefix is None:
+            raise ValueError("no sources")
+        ref = blocks if blocks is not None else prefix
+        dtype = _dtype_code(np.asarray(ref))
+        blocks_c = None if blocks is None else np.ascontiguousarray(blocks)
+        prefix_c = None if prefix is None else np.ascontiguousarray(prefix)
+        if blocks_c is not None and prefix_c is not None and blocks_c.dtype != prefix_c.dtype:
+            raise TypeError("blocks and prefix must share a dtype")
+        T = (blocks_c if blocks_c is not None else prefix_c).shape[0]
+        H = (blocks_c if blocks_c is not None else prefix_c).shape[-1]
+        nb = 0 if blocks_c is None else blocks_c.shape[1]
+        nw = np.ascontiguousarray(norm_weight)
+        pw = np.ascontiguousarray(proj_weight)
+        r, n = self._rows(rows, T)
+        S = nb + (prefix_c is not None)
+        out = np.empty((n, H))
+        mag = np.empty((n, H))
+        prob = np.empty((n, S))
+        rc = self._lib.situ_oracle_attn_res(_ptr(blocks_c), nb, nb * H, H, _ptr(prefix_c), H, dtype, H, _ptr(nw),
+                                            _dtype_code(nw), _ptr(pw), _dtype_code(pw), float(eps), _ptr(r), n,
+                                            _ptr(out), _ptr(mag), _ptr(prob))
+        if rc != 0:
+            raise ValueError("oracle attn_res rejected its arguments")
+        return out, mag, prob
 
 
 _DEFAULT = None

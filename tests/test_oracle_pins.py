@@ -20,7 +20,10 @@ itself checked here against things other than itself:
     OCP MX format's clamp at 448, and the scale rules' defining inequalities;
   * FC1 + SiTU-GLU (fc1_oracle.c): fsum dot products and 50-digit element
     values, exact agreement with the activation oracle on bf16-exact FC1
-    outputs, and the grouped call against per-expert calls.
+    outputs, and the grouped call against per-expert calls;
+  * attention-residual core (attn_res_oracle.c): torch's float64 rms_norm and
+    softmax, invariants (identical sources, zero projection, one source,
+    scaling), large logits, and the two-array source layout.
 
 Each pin is a plain function of an oracle handle.  ``test_mutant_rejected``
 rebuilds situ_oracle.c with each planted mistake (-DSITU_ORACLE_MUTANT=n: a
@@ -489,6 +492,86 @@ def pin_fc1_grouped_equals_per_expert(o):
         assert np.array_equal(y[a:b], ye), e
 
 
+# ---- attention-residual mixing core (attn_res_oracle.c) -----------------------------
+
+def _torch_attn_res(x, nw, pw, eps):
+    """float64 torch library routines: rms_norm, a matmul projection, softmax,
+    and the weighted sum of the raw values."""
+    xt = torch.from_numpy(x)
+    k = torch.nn.functional.rms_norm(xt, (x.shape[-1],), weight=torch.from_numpy(nw), eps=eps)
+    logits = k @ torch.from_numpy(pw)
+    prob = torch.softmax(logits, dim=-1)
+    return torch.einsum("tb,tbh->th", prob, xt).numpy(), prob.numpy()
+
+
+def pin_attn_res_torch(o):
+    """Against torch's float64 rms_norm / softmax: stored sums and a current sum
+    (appended last), bf16 values, one source of tiny values (where epsilon
+    matters), fp32 weights."""
+    rng = np.random.default_rng(RNG_SEED + 6)
+    T, B, H = 5, 3, 64
+    blocks = _bf16(rng.standard_normal((T, B, H)) * 2.0)
+    blocks[:, 1] = _bf16(_widen(blocks[:, 1]) * 1e-3)
+    prefix = _bf16(rng.standard_normal((T, H)))
+    nw = (1.0 + 0.1 * rng.standard_normal(H)).astype(np.float32)
+    pw = (0.2 * rng.standard_normal(H)).astype(np.float32)
+    eps = 1e-6
+    out, mag, prob = o.attn_res(blocks, prefix, nw, pw, eps)
+    x = np.concatenate([_widen(blocks), _widen(prefix)[:, None, :]], axis=1)
+    ref, pref = _torch_attn_res(x, nw.astype(np.float64), pw.astype(np.float64), eps)
+    assert np.allclose(out, ref, rtol=1e-12, atol=1e-14), np.abs(out - ref).max()
+    assert np.allclose(prob, pref, rtol=1e-12, atol=1e-15)
+    assert np.all(mag >= np.abs(out) * (1 - 1e-12))
+
+
+def pin_attn_res_invariants(o):
+    """Identical sources give that source back; a zero projection gives the plain
+    average; a single source is returned as is; doubling every value (exact in
+    bf16) with epsilon 0 doubles the output and leaves the weights."""
+    rng = np.random.default_rng(RNG_SEED + 7)
+    T, H = 4, 48
+    v = _bf16(rng.standard_normal((T, H)))
+    nw = rng.random(H).astype(np.float32) + 0.5
+    pw = rng.standard_normal(H).astype(np.float32)
+    same = np.repeat(v[:, None, :], 4, axis=1)
+    out, _, _ = o.attn_res(same, None, nw, pw, 1e-6)
+    assert np.allclose(out, _widen(v), rtol=1e-15, atol=0)
+    blocks = _bf16(rng.standard_normal((T, 3, H)))
+    out, _, prob = o.attn_res(blocks, None, nw, np.zeros(H, np.float32), 1e-6)
+    assert np.allclose(prob, 1.0 / 3.0, rtol=1e-15) and np.allclose(out, _widen(blocks).mean(axis=1), rtol=1e-14)
+    out, _, _ = o.attn_res(None, v, nw, pw, 1e-6)
+    assert np.array_equal(out, _widen(v))
+    o1, _, p1 = o.attn_res(blocks, v, nw, pw, 0.0)
+    o2, _, p2 = o.attn_res(_bf16(_widen(blocks) * 2), _bf16(_widen(v) * 2), nw, pw, 0.0)
+    assert np.allclose(p1, p2, rtol=1e-13) and np.allclose(o2, 2 * o1, rtol=1e-13, atol=1e-300)
+
+
+def pin_attn_res_large_logits(o):
+    """Logits of thousands: the softmax must stay finite and match torch's."""
+    rng = np.random.default_rng(RNG_SEED + 8)
+    T, B, H = 3, 5, 32
+    blocks = _bf16(rng.standard_normal((T, B, H)))
+    nw = np.ones(H, np.float32)
+    pw = (1e3 * rng.standard_normal(H)).astype(np.float32)
+    out, _, prob = o.attn_res(blocks, None, nw, pw, 1e-6)
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(prob))
+    ref, pref = _torch_attn_res(_widen(blocks), nw.astype(np.float64), pw.astype(np.float64), 1e-6)
+    assert np.allclose(prob, pref, rtol=1e-9, atol=1e-300) and np.allclose(out, ref, rtol=1e-9, atol=1e-12)
+
+
+def pin_attn_res_two_arrays(o):
+    """Stored sums plus the current sum equal the same sources stacked in one array."""
+    rng = np.random.default_rng(RNG_SEED + 9)
+    T, B, H = 4, 2, 40
+    blocks = _bf16(rng.standard_normal((T, B, H)))
+    prefix = _bf16(rng.standard_normal((T, H)))
+    nw = rng.random(H).astype(np.float32) + 0.5
+    pw = rng.standard_normal(H).astype(np.float32)
+    a, _, _ = o.attn_res(blocks, prefix, nw, pw, 1e-6)
+    b, _, _ = o.attn_res(np.concatenate([blocks, prefix[:, None, :]], axis=1), None, nw, pw, 1e-6)
+    assert np.array_equal(a, b)
+
+
 PINS = [
     pin_gate_values_mpmath,
     pin_up_values_mpmath,
@@ -511,6 +594,10 @@ PINS = [
     pin_fc1_bruteforce,
     pin_fc1_matches_activation_oracle,
     pin_fc1_grouped_equals_per_expert,
+    pin_attn_res_torch,
+    pin_attn_res_invariants,
+    pin_attn_res_large_logits,
+    pin_attn_res_two_arrays,
 ]
 
 
@@ -545,6 +632,11 @@ MUTANTS = {
     21: "FC1 up rows taken from the gate rows",
     22: "FC1 dot product drops the last product",
     23: "FC1 boundary row assigned to the earlier expert",
+    24: "RMSNorm with the sum instead of the mean of squares",
+    25: "RMSNorm epsilon dropped",
+    26: "RMSNorm weight not applied",
+    27: "softmax without the max shift",
+    28: "a transformed value combined instead of the raw one",
 }
 
 
