@@ -17,7 +17,10 @@ bytes follow the form (weights read, weight gradients written, one byte per
 code plus one per 32 codes).  --variant fc1 times the fused FC1 grouped GEMM
 + SiTU-GLU forward on the routed-MoE rows (hidden 7168, 8 local experts) in
 TFLOP/s against the tensor-core peak, with the unfused cuBLAS GEMMs +
-SiTU-GLU kernel timed beside it.
+SiTU-GLU kernel timed beside it.  --variant attn_res times the
+attention-residual mixing core (16384 tokens, 8 stored sums + the current
+sum, hidden 7168, bf16) in GB/s of algorithmic bytes (every source value read
+once, the output written once).
 
 For N > 1 launch one process per GPU with torchrun; every rank runs the same
 per-GPU workload (weak scaling, no collective on the data path), the step
@@ -63,7 +66,7 @@ def parse_args(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-oracle sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--variant", choices=["row", "col", "full", "mxfp8", "fc1"], default="row",
+    p.add_argument("--variant", choices=["row", "col", "full", "mxfp8", "fc1", "attn_res"], default="row",
                    help="routing-weight form or output format timed (default: per-row weights)")
     p.add_argument("--flush", choices=["auto", "always", "never"], default="auto",
                    help="flush L2 before every step (auto: when the inputs fit in L2)")
@@ -239,6 +242,175 @@ def fc1_cpu_rate(wl, beta, d, seconds: float):
     return per_row * done / dt / 1e12, done, dt
 
 
+# The attention-residual mixing workload: 16384 tokens, 8 stored block sums
+# plus the current sum (Kimi-K3 stores at most 8 sums), hidden 7168, bf16.
+AR_TOKENS, AR_BLOCKS, AR_HIDDEN = 16384, 8, 7168
+AR_METRIC = "attention-residual mixing core achieved HBM GB/s"
+
+
+def ar_bytes() -> int:
+    return AR_TOKENS * (AR_BLOCKS + 1) * AR_HIDDEN * 2 + AR_TOKENS * AR_HIDDEN * 2
+
+
+def ar_config(l2_note, world):
+    return {"workload": (f"attention-residual mix: {AR_BLOCKS} stored sums bf16 [{AR_TOKENS}, {AR_BLOCKS}, "
+                         f"{AR_HIDDEN}] (source b ~ N(0, 1 + b/2)) + the current sum [{AR_TOKENS}, {AR_HIDDEN}], "
+                         f"norm/proj weights fp32 [{AR_HIDDEN}], eps 1e-6, out bf16"),
+            "name": "attn_res", "tokens": AR_TOKENS, "sources": AR_BLOCKS + 1, "hidden": AR_HIDDEN,
+            "l2": l2_note, "parallelism": f"replicas x{world} (weak scaling; no collective)"}
+
+
+def run_reference_attn_res(args, world):
+    import oracle
+    o = oracle.load()
+    rows_per_step = 16
+    d = workloads.attn_res_inputs(rows_per_step, AR_BLOCKS, AR_HIDDEN, seed=2)
+
+    def step():
+        o.attn_res(d["blocks"], d["prefix"], d["norm_weight"], d["proj_weight"], 1e-6)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = ar_bytes() / AR_TOKENS * rows_per_step * args.steps / dt / 1e9
+    line = {"impl": "reference", "metric": AR_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": ar_config("n/a (host)", 1),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{rows_per_step} rows per step, {args.steps} steps, single-threaded fp64"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours_attn_res(args, dev, world, rank, local, barrier):
+    import torch
+    import torch.distributed as dist
+
+    import ffn_gated_activation_b200 as pkg
+
+    d = workloads.attn_res_inputs(AR_TOKENS, AR_BLOCKS, AR_HIDDEN, seed=2)
+
+    def pinned(a):
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.pin_memory()
+
+    blocks_h, prefix_h = pinned(d["blocks"]), pinned(d["prefix"])
+    blocks, prefix = blocks_h.to(dev), prefix_h.to(dev)
+    nw, pw = torch.from_numpy(d["norm_weight"]).to(dev), torch.from_numpy(d["proj_weight"]).to(dev)
+    out = torch.empty(AR_TOKENS, AR_HIDDEN, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd():
+        pkg.apply_attn_res(prefix, blocks, pw, nw, 1e-6, out=out)
+
+    for _ in range(max(3, args.warmup)):
+        fwd()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for a, b in ev:
+        a.record(stream)
+        fwd()
+        b.record(stream)
+    torch.cuda.synchronize()
+    clocks.stop()
+    barrier()
+    t = torch.tensor([sum(a.elapsed_time(b) for a, b in ev)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = t.item() / K
+    gbs = ar_bytes() / (ms / 1e3) / 1e9
+    peak, peak_src = measured_peak()
+
+    # The same chain in plain PyTorch ops (eager, fp32), for context.
+    def torch_chain():
+        x = torch.cat([blocks, prefix.unsqueeze(1)], dim=1).float()
+        k = torch.nn.functional.rms_norm(x, (AR_HIDDEN,), weight=nw, eps=1e-6)
+        prob = torch.softmax(k @ pw, dim=-1)
+        return (prob.unsqueeze(-1) * x).sum(dim=1).to(torch.bfloat16)
+
+    for _ in range(2):
+        torch_chain()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(3):
+        torch_chain()
+    b.record(stream)
+    torch.cuda.synchronize()
+    torch_ms = a.elapsed_time(b) / 3
+
+    e2e = None
+    if not args.no_e2e:
+        out_h = torch.empty(AR_TOKENS, AR_HIDDEN, dtype=torch.bfloat16).pin_memory()
+        K2 = args.e2e_steps or max(1, min(K, 10))
+
+        def e2e_step():
+            blocks.copy_(blocks_h, non_blocking=True)
+            prefix.copy_(prefix_h, non_blocking=True)
+            fwd()
+            out_h.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(K2):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        tt = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = tt.item() / K2
+        e2e = {"value": ar_bytes() * world / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": blocks_h.numel() * 2 + prefix_h.numel() * 2,
+               "d2h_bytes_per_step": out_h.numel() * 2, "ms_per_step": e2e_ms, "steps": K2,
+               "api": "ffn_gated_activation_b200.apply_attn_res on pinned host copies"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        o = oracle.load()
+        done, t0 = 0, time.perf_counter()
+        per_row = ar_bytes() / AR_TOKENS
+        while time.perf_counter() - t0 < args.cpu_seconds and done < AR_TOKENS:
+            rows = np.arange(done, min(AR_TOKENS, done + 8), dtype=np.int64)
+            o.attn_res(d["blocks"], d["prefix"], d["norm_weight"], d["proj_weight"], 1e-6, rows=rows)
+            done += rows.size
+        secs = time.perf_counter() - t0
+        cpu = {"value": per_row * done / secs / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"first {done} of {AR_TOKENS} rows, {secs:.1f} s, single-threaded fp64 oracle"}
+    if rank == 0:
+        line = {"metric": AR_METRIC, "value": gbs * world, "unit": "GB/s", "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": ar_config(f"inputs {ar_bytes() / 1e9:.1f} GB exceed the 126 MB L2; no flush", world),
+                "kernels": {"situ_attn_res_kernel": {"us": ms * 1e3, "GB/s": gbs, "frac_of_measured_copy": gbs / peak}},
+                "torch_eager_fp32_chain": {"ms": torch_ms, "GB/s": ar_bytes() / (torch_ms / 1e3) / 1e9},
+                "roofline": {"bound": "hbm", "kernel": "situ_attn_res_kernel", "achieved": gbs, "peak": peak,
+                             "unit": "GB/s", "frac": gbs / peak, "peak_source": f"{peak_src} copy bandwidth",
+                             "traffic": recorded_traffic("situ_attn_res_kernel", "attn_res")},
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K, "clocks": clocks.summary(),
+                "device_status": pkg.abi.situ_glu_device_status(0), "device": torch.cuda.get_device_name(dev)}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def variant_bytes(wl, variant: str):
     """Algorithmic bytes (forward, backward) of one pass over the workload in
     the given form.  Per-row weights: read gate_up and w, write Y; read
@@ -308,6 +480,8 @@ def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.variant == "fc1":
         return run_reference_fc1(args, wl, beta, world)
+    if args.variant == "attn_res":
+        return run_reference_attn_res(args, world)
     rows_per_step = max(1, min(wl.tokens, (1 << 17) // wl.inter))
     x = workloads.inputs(wl, tokens=rows_per_step)
     import oracle
@@ -559,6 +733,8 @@ def run_ours(args):
     beta = args.beta if args.beta is not None else wl.betas[0]
     if args.variant == "fc1":
         return run_ours_fc1(args, wl, beta, dev, world, rank, local, barrier)
+    if args.variant == "attn_res":
+        return run_ours_attn_res(args, dev, world, rank, local, barrier)
     lb = wl.linear_beta
     T, I = wl.tokens, wl.inter
     x = workloads.inputs(wl)

@@ -12,6 +12,8 @@ from . import abi, distributed
 from .abi import NativeLibraryError, SituError
 from .functional import (
     DEFAULT_BETA,
+    apply_attn_res,
+    attn_res_core,
     DEFAULT_LINEAR_BETA,
     WeightedSiTUFunction,
     situ_glu_bwd,
@@ -30,6 +32,8 @@ __all__ = [
     "SituError",
     "DEFAULT_BETA",
     "DEFAULT_LINEAR_BETA",
+    "apply_attn_res",
+    "attn_res_core",
     "WeightedSiTUFunction",
     "situ_glu_fwd",
     "situ_glu_bwd",

@@ -1800,6 +1800,159 @@ __global__ void __launch_bounds__(kMaxConsumers + 32) situ_glu_bwd_tma_kernel(co
   tma_stream_body<S, GATE, HAS_LB, true>(a);
 }
 
+// ---------------------------------------------------------------------------
+// Attention-residual mixing core
+// ---------------------------------------------------------------------------
+// NeMo AutoModel kimi_k3.situ `_attn_res_core` / `_apply_attn_res`: for token
+// row t with sources b (the stored block sums, then the current prefix sum),
+//   logit[b] = sum_h values[b, h] / sqrt(mean_h values[b]^2 + eps) * norm_w[h] * proj_w[h]
+//   out[h]   = sum_b softmax(logit)[b] values[b, h]
+// in fp32.  The RMSNorm scale is constant over h, so each logit is
+// rsqrt(ss_b / H + eps) * dd_b with two sums per source, ss_b = sum_h x^2 and
+// dd_b = sum_h x c_h, c = norm_w * proj_w (kept in shared memory).  One CTA
+// works on one row at a time: pass 1 streams the row's sources once for the
+// 2 S sums (per-thread partials, warp shuffles, then the warps in order: a
+// fixed order, so results do not depend on the grid); every thread then forms
+// the softmax; pass 2 reads the sources again -- from L2, where pass 1 left
+// them -- and writes the weighted sum.  HBM sees each value once.
+
+constexpr int kArMaxSources = 16;
+constexpr int kArThreads = 256;
+
+struct ArArgs {
+  const char* blocks;        // stored sums: row pitch / source pitch in bytes
+  int64_t block_row_pitch;
+  int64_t block_pitch;
+  const char* prefix;        // current sum (the last source) or NULL
+  int64_t prefix_row_pitch;
+  int nblocks;
+  int sources;
+  int64_t tokens;
+  int hidden;
+  int vpr;                   // 16-byte vectors of one source row
+  const void* norm_w;
+  int norm_bf16;
+  const void* proj_w;
+  int proj_bf16;
+  float eps;
+  float inv_hidden;
+  char* out;
+  int64_t out_pitch;         // bytes
+  int out_bf16;
+};
+
+__device__ __forceinline__ float ar_weight(const void* w, int bf16, int h) {
+  return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(w)[h]) : reinterpret_cast<const float*>(w)[h];
+}
+
+template <typename S>
+__device__ __forceinline__ const char* ar_source(const ArArgs& a, int64_t row, int b) {
+  return b < a.nblocks ? a.blocks + row * a.block_row_pitch + b * a.block_pitch : a.prefix + row * a.prefix_row_pitch;
+}
+
+template <typename S>
+__global__ void __launch_bounds__(kArThreads) situ_attn_res_kernel(const ArArgs a) {
+  constexpr int kElems = 2 * S::kPairs;
+  extern __shared__ float c_sh[];                       // [hidden]: norm_w * proj_w
+  __shared__ float red[kArThreads / 32][2 * kArMaxSources];
+  __shared__ float prob_sh[kArMaxSources];
+  const int nt = blockDim.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int h = threadIdx.x; h < a.hidden; h += nt) c_sh[h] = ar_weight(a.norm_w, a.norm_bf16, h) * ar_weight(a.proj_w, a.proj_bf16, h);
+  __syncthreads();
+  for (int64_t row = blockIdx.x; row < a.tokens; row += gridDim.x) {
+    float ss[kArMaxSources], dd[kArMaxSources];
+#pragma unroll
+    for (int b = 0; b < kArMaxSources; ++b) {
+      ss[b] = 0.0f;
+      dd[b] = 0.0f;
+      if (b < a.sources) {
+        const char* src = ar_source<S>(a, row, b);
+        for (int j = threadIdx.x; j < a.vpr; j += nt) {
+          const uint4 v = ld_stream(src + j * kVecBytes);
+#pragma unroll
+          for (int p = 0; p < S::kPairs; ++p) {
+            const float2 x = as_f2(S::pair(v, p));
+            const float2 c = make_float2(c_sh[j * kElems + 2 * p], c_sh[j * kElems + 2 * p + 1]);
+            ss[b] = fmaf(x.x, x.x, fmaf(x.y, x.y, ss[b]));
+            dd[b] = fmaf(x.x, c.x, fmaf(x.y, c.y, dd[b]));
+          }
+        }
+      }
+    }
+    // CTA sums of the 2 S partials: warp shuffles, then the warps in order.
+#pragma unroll
+    for (int b = 0; b < kArMaxSources; ++b) {
+      if (b < a.sources) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          ss[b] += __shfl_xor_sync(0xffffffffu, ss[b], o);
+          dd[b] += __shfl_xor_sync(0xffffffffu, dd[b], o);
+        }
+        if (lane == 0) {
+          red[warp][2 * b] = ss[b];
+          red[warp][2 * b + 1] = dd[b];
+        }
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < a.sources) {
+      const int b = threadIdx.x;
+      float s2 = 0.0f, d2 = 0.0f;
+      for (int w = 0; w < (nt >> 5); ++w) {
+        s2 += red[w][2 * b];
+        d2 += red[w][2 * b + 1];
+      }
+      prob_sh[b] = d2 * rsqrtf(s2 * a.inv_hidden + a.eps);  // the logit, for now
+    }
+    __syncthreads();
+    float p[kArMaxSources];
+    float mx = prob_sh[0];
+#pragma unroll
+    for (int b = 1; b < kArMaxSources; ++b)
+      if (b < a.sources) mx = fmaxf(mx, prob_sh[b]);
+    float z = 0.0f;
+#pragma unroll
+    for (int b = 0; b < kArMaxSources; ++b) {
+      p[b] = b < a.sources ? __expf(prob_sh[b] - mx) : 0.0f;
+      z += p[b];
+    }
+    const float rz = 1.0f / z;
+#pragma unroll
+    for (int b = 0; b < kArMaxSources; ++b) p[b] *= rz;
+    // pass 2: out = sum_b p_b values[b]
+    char* orow = a.out + row * a.out_pitch;
+    for (int j = threadIdx.x; j < a.vpr; j += nt) {
+      float2 acc[S::kPairs];
+#pragma unroll
+      for (int q = 0; q < S::kPairs; ++q) acc[q] = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int b = 0; b < kArMaxSources; ++b) {
+        if (b < a.sources) {
+          const uint4 v = *reinterpret_cast<const uint4*>(ar_source<S>(a, row, b) + j * kVecBytes);
+#pragma unroll
+          for (int q = 0; q < S::kPairs; ++q) acc[q] = fma2(splat(p[b]), as_f2(S::pair(v, q)), acc[q]);
+        }
+      }
+      if (a.out_bf16) {
+        uint32_t w[S::kPairs];
+#pragma unroll
+        for (int q = 0; q < S::kPairs; ++q) w[q] = Bf16::pack(acc[q]);
+        if constexpr (S::kPairs == 4)
+          st_stream(orow + j * 16, make_uint4(w[0], w[1], w[2], w[3]));
+        else
+          st_stream8(orow + j * 8, make_uint2(w[0], w[1]));
+      } else {
+#pragma unroll
+        for (int q = 0; q < S::kPairs / 2; ++q)
+          st_stream(orow + j * kElems * 4 + q * 16, make_uint4(__float_as_uint(acc[2 * q].x), __float_as_uint(acc[2 * q].y),
+                                                              __float_as_uint(acc[2 * q + 1].x),
+                                                              __float_as_uint(acc[2 * q + 1].y)));
+      }
+    }
+    __syncthreads();  // red and prob_sh are rewritten by the next row
+  }
+}
+
 #include "situ_fc1.cuh"
 
 // ---------------------------------------------------------------------------
@@ -2845,4 +2998,95 @@ extern "C" situ_status_t situ_glu_fc1_fwd(const void* x, int64_t tokens, int64_t
   if (cap > 0 && grid > cap) grid = cap;
   k<<<grid, fc1::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(mx, mw, a);
   return check_launch("situ_glu_fc1_fwd");
+}
+
+
+// ---------------------------------------------------------------------------
+// Attention-residual mixing core
+// ---------------------------------------------------------------------------
+
+extern "C" situ_status_t situ_attn_res_fwd(const void* blocks, int64_t nblocks, int64_t block_row_stride,
+                                           int64_t block_stride, const void* prefix, int64_t prefix_row_stride,
+                                           situ_dtype_t dtype, int64_t tokens, int64_t hidden,
+                                           const void* norm_weight, situ_dtype_t norm_dtype,
+                                           const void* proj_weight, situ_dtype_t proj_dtype, double variance_epsilon,
+                                           void* out, situ_dtype_t out_dtype, int64_t out_row_stride,
+                                           void* stream) {
+  tl_last_error[0] = '\0';
+  if (!valid_dtype(dtype) || !valid_dtype(norm_dtype) || !valid_dtype(proj_dtype) || !valid_dtype(out_dtype))
+    return fail(SITU_ERR_INVALID_ARG, "a dtype is not a situ_dtype_t");
+  if (nblocks < 0) return fail(SITU_ERR_INVALID_ARG, "nblocks < 0");
+  const int64_t sources = nblocks + (prefix != nullptr ? 1 : 0);
+  if (sources < 1 || sources > kArMaxSources)
+    return fail(SITU_ERR_UNSUPPORTED, "sources (blocks plus the prefix sum) must be in [1, %d], got %lld",
+                kArMaxSources, (long long)sources);
+  if (tokens < 0) return fail(SITU_ERR_INVALID_ARG, "tokens = %lld < 0", (long long)tokens);
+  if (hidden <= 0) return fail(SITU_ERR_INVALID_ARG, "hidden = %lld <= 0", (long long)hidden);
+  if (hidden > 32768) return fail(SITU_ERR_UNSUPPORTED, "hidden = %lld exceeds 32768", (long long)hidden);
+  if (!std::isfinite(variance_epsilon) || variance_epsilon < 0.0)
+    return fail(SITU_ERR_INVALID_ARG, "variance_epsilon must be finite and >= 0");
+  if ((nblocks > 0 && (block_row_stride < hidden || block_stride < hidden)) ||
+      (prefix != nullptr && prefix_row_stride < hidden) || out_row_stride < hidden)
+    return fail(SITU_ERR_INVALID_ARG, "a stride is shorter than a row");
+  const int es = elem_size(dtype), oes = elem_size(out_dtype);
+  if ((hidden * es) % 16 != 0)
+    return fail(SITU_ERR_MISALIGNED, "hidden * element size (%lld bytes) is not a multiple of 16",
+                (long long)(hidden * es));
+  if (tokens == 0) return SITU_OK;
+  if ((nblocks > 0 && blocks == nullptr) || norm_weight == nullptr || proj_weight == nullptr || out == nullptr)
+    return fail(SITU_ERR_INVALID_ARG, "blocks, norm_weight, proj_weight or out is NULL");
+  if ((nblocks > 0 && !span_fits(tokens, block_row_stride, nblocks * block_stride, es)) ||
+      (prefix != nullptr && !span_fits(tokens, prefix_row_stride, hidden, es)) ||
+      !span_fits(tokens, out_row_stride, hidden, oes))
+    return fail(SITU_ERR_INVALID_ARG, "tensor extent overflows int64");
+  if ((nblocks > 0 && (!aligned(blocks, 16) || (block_row_stride * es) % 16 != 0 || (block_stride * es) % 16 != 0)) ||
+      (prefix != nullptr && (!aligned(prefix, 16) || (prefix_row_stride * es) % 16 != 0)) || !aligned(out, 16) ||
+      (out_row_stride * oes) % 16 != 0 || !aligned(norm_weight, elem_size(norm_dtype)) ||
+      !aligned(proj_weight, elem_size(proj_dtype)))
+    return fail(SITU_ERR_MISALIGNED, "a base address or row pitch is misaligned");
+  const Span s_out = matrix_span(out, tokens, out_row_stride, hidden, oes);
+  if ((nblocks > 0 && overlap(s_out, matrix_span(blocks, tokens, block_row_stride, (nblocks - 1) * block_stride + hidden,
+                                                  es))) ||
+      (prefix != nullptr && overlap(s_out, matrix_span(prefix, tokens, prefix_row_stride, hidden, es))) ||
+      overlap(s_out, matrix_span(norm_weight, 1, hidden, hidden, elem_size(norm_dtype))) ||
+      overlap(s_out, matrix_span(proj_weight, 1, hidden, hidden, elem_size(proj_dtype))))
+    return fail(SITU_ERR_INVALID_ARG, "out overlaps an input");
+
+  ArArgs a{};
+  a.blocks = static_cast<const char*>(blocks);
+  a.block_row_pitch = block_row_stride * es;
+  a.block_pitch = block_stride * es;
+  a.prefix = static_cast<const char*>(prefix);
+  a.prefix_row_pitch = prefix_row_stride * es;
+  a.nblocks = static_cast<int>(nblocks);
+  a.sources = static_cast<int>(sources);
+  a.tokens = tokens;
+  a.hidden = static_cast<int>(hidden);
+  a.vpr = static_cast<int>(hidden * es / kVecBytes);
+  a.norm_w = norm_weight;
+  a.norm_bf16 = norm_dtype == SITU_DTYPE_BF16;
+  a.proj_w = proj_weight;
+  a.proj_bf16 = proj_dtype == SITU_DTYPE_BF16;
+  a.eps = static_cast<float>(variance_epsilon);
+  a.inv_hidden = static_cast<float>(1.0 / static_cast<double>(hidden));
+  a.out = static_cast<char*>(out);
+  a.out_pitch = out_row_stride * oes;
+  a.out_bf16 = out_dtype == SITU_DTYPE_BF16;
+  const void* k = dtype == SITU_DTYPE_BF16 ? reinterpret_cast<const void*>(situ_attn_res_kernel<Bf16>)
+                                           : reinterpret_cast<const void*>(situ_attn_res_kernel<F32>);
+  const int threads = a.vpr >= kArThreads ? kArThreads : (a.vpr + 31) / 32 * 32;
+  const int smem = static_cast<int>(hidden * sizeof(float));
+  if (smem > 48 * 1024) {
+    situ_status_t st = ensure_smem(k, smem);
+    if (st != SITU_OK) return st;
+  }
+  int grid = 0;
+  situ_status_t st = launch_grid(k, threads, smem, tokens, &grid);
+  if (st != SITU_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == SITU_DTYPE_BF16)
+    situ_attn_res_kernel<Bf16><<<grid, threads, smem, s>>>(a);
+  else
+    situ_attn_res_kernel<F32><<<grid, threads, smem, s>>>(a);
+  return check_launch("situ_attn_res_fwd");
 }

@@ -312,6 +312,66 @@ def situ_glu_fc1_fwd(x: torch.Tensor, w1: torch.Tensor, offsets: torch.Tensor, r
     return out
 
 
+_DTYPE_OF = {torch.bfloat16: abi.SITU_DTYPE_BF16, torch.float32: abi.SITU_DTYPE_F32}
+
+
+def _attn_res_launch(blocks, prefix, norm_weight, proj_weight, variance_epsilon, out_dtype, out):
+    src = blocks if blocks is not None else prefix
+    if src.device.type != "cuda":
+        raise ValueError("the sources must be CUDA tensors")
+    dtype = _dtype_code(src, "values")
+    if blocks is not None and prefix is not None and blocks.dtype != prefix.dtype:
+        raise TypeError("block_residual and prefix_sum must share a dtype")
+    tokens, hidden = src.shape[0], src.shape[-1]
+    nw = norm_weight.reshape(-1)
+    pw = proj_weight.reshape(-1)
+    if nw.numel() != hidden or pw.numel() != hidden:
+        raise ValueError(f"norm_weight and proj_weight must hold {hidden} values")
+    nw, pw = nw.contiguous(), pw.contiguous()
+    out_dtype = src.dtype if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty(tokens, hidden, dtype=out_dtype, device=src.device)
+    nb = 0
+    if blocks is not None:
+        if blocks.stride(-1) != 1:
+            blocks = blocks.contiguous()
+        nb = blocks.shape[1]
+    if prefix is not None and prefix.stride(-1) != 1:
+        prefix = prefix.contiguous()
+    st = abi.situ_attn_res_fwd(blocks.data_ptr() if blocks is not None else None, nb,
+                               blocks.stride(0) if blocks is not None else hidden,
+                               blocks.stride(1) if blocks is not None else hidden,
+                               prefix.data_ptr() if prefix is not None else None,
+                               prefix.stride(0) if prefix is not None else hidden, dtype, tokens, hidden,
+                               nw.data_ptr(), _dtype_code(nw, "norm_weight"), pw.data_ptr(),
+                               _dtype_code(pw, "proj_weight"), float(variance_epsilon), out.data_ptr(),
+                               _dtype_code(out, "out"), out.stride(0) if tokens > 1 else hidden,
+                               _stream_handle(None))
+    abi.check(st, "situ_attn_res_fwd")
+    return out
+
+
+def attn_res_core(values: torch.Tensor, norm_weight: torch.Tensor, proj_weight: torch.Tensor,
+                  variance_epsilon: float, out_dtype: torch.dtype | None = None, out=None) -> torch.Tensor:
+    """NeMo `_attn_res_core`: fp32 attention-residual mixing of values
+    [tokens, sources, hidden] (block residuals with the current prefix sum
+    appended) -> [tokens, hidden] in out_dtype (default: values' dtype)."""
+    if values.dim() != 3:
+        raise ValueError("values must be [tokens, sources, hidden]")
+    return _attn_res_launch(values, None, norm_weight, proj_weight, variance_epsilon, out_dtype, out)
+
+
+def apply_attn_res(prefix_sum: torch.Tensor, block_residual: torch.Tensor, proj_weight: torch.Tensor,
+                   norm_weight: torch.Tensor, variance_epsilon: float, out_dtype: torch.dtype | None = None,
+                   out=None) -> torch.Tensor:
+    """NeMo `_apply_attn_res`: mix prefix_sum [tokens, hidden] with the stored
+    block_residual [tokens, blocks, hidden] without stacking them (the prefix
+    sum is the last source)."""
+    if prefix_sum.dim() != 2 or block_residual.dim() != 3:
+        raise ValueError("prefix_sum must be [tokens, hidden] and block_residual [tokens, blocks, hidden]")
+    return _attn_res_launch(block_residual, prefix_sum, norm_weight, proj_weight, variance_epsilon, out_dtype, out)
+
+
 class WeightedSiTUFunction(torch.autograd.Function):
     """Routing-weighted SiTU-GLU with the analytic fused backward.
 

@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define SITU_GLU_ABI_VERSION 4
+#define SITU_GLU_ABI_VERSION 5
 
 typedef enum situ_status {
   SITU_OK = 0,
@@ -264,6 +264,40 @@ situ_status_t situ_glu_fc1_fwd(const void *x, int64_t tokens, int64_t hidden, in
                                double beta, int has_linear_beta, double linear_beta,
                                void *y, int64_t y_row_stride,
                                void *stream);
+
+/* ---- Attention-residual mixing core -------------------------------------------
+ * NeMo AutoModel API, kimi_k3.situ, `_attn_res_core` ("fp32 attention-residual
+ * mixing chain") and `_apply_attn_res` (mix the current [tokens, hidden] sum
+ * with the stored [tokens, blocks, hidden] sums).  For token t, with sources
+ * b = 0 .. S-1 the nblocks stored sums followed by the prefix sum (if given):
+ *   logit[b] = sum_h x_b[h] / sqrt(mean_h x_b^2 + eps) * norm_weight[h] * proj_weight[h]
+ *   out[h]   = sum_b softmax_b(logit)[b] x_b[h]
+ * in fp32 (RMSNorm in its standard form; the projection is the squeezed
+ * [hidden] weight of a hidden -> 1 linear layer).
+ *
+ *   blocks            stored sums, dtype; element (t, b, h) at
+ *                     blocks[t * block_row_stride + b * block_stride + h];
+ *                     may be NULL when nblocks == 0
+ *   prefix            current sum [tokens, >= hidden] (row pitch
+ *                     prefix_row_stride), the last source; NULL: none
+ *   dtype             storage of blocks and prefix (bf16 or fp32)
+ *   norm_weight, proj_weight  [hidden] in their own dtypes
+ *   variance_epsilon  RMSNorm epsilon, finite and >= 0
+ *   out               [tokens, >= hidden] in out_dtype, row pitch
+ *                     out_row_stride; must not overlap an input
+ * 1 <= S <= 16 and hidden <= 32768 (SITU_ERR_UNSUPPORTED otherwise); hidden *
+ * sizeof(dtype) a multiple of 16; sources and out 16-byte aligned with row
+ * (and source) pitches of a multiple of 16 bytes.  Results do not depend on
+ * the launch size.
+ */
+situ_status_t situ_attn_res_fwd(const void *blocks, int64_t nblocks, int64_t block_row_stride,
+                                int64_t block_stride, const void *prefix, int64_t prefix_row_stride,
+                                situ_dtype_t dtype, int64_t tokens, int64_t hidden,
+                                const void *norm_weight, situ_dtype_t norm_dtype,
+                                const void *proj_weight, situ_dtype_t proj_dtype,
+                                double variance_epsilon,
+                                void *out, situ_dtype_t out_dtype, int64_t out_row_stride,
+                                void *stream);
 
 /* Static, human-readable name of a status code. */
 const char *situ_glu_status_string(situ_status_t status);

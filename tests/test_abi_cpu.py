@@ -29,7 +29,7 @@ def declared_functions():
     for h in HEADERS:
         text = open(h).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-        names |= set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(situ_glu_\w+)\s*\(", text, flags=re.M))
+        names |= set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(situ_(?:glu|attn_res)_\w+)\s*\(", text, flags=re.M))
     return names
 
 
@@ -58,7 +58,7 @@ def test_binding_covers_the_header_exactly():
 
 
 def test_version_and_status_strings(native_lib_path):
-    assert abi.situ_glu_abi_version() == abi.ABI_VERSION == 4
+    assert abi.situ_glu_abi_version() == abi.ABI_VERSION == 5
     assert abi.situ_glu_status_string(OK) == "SITU_OK"
     assert abi.situ_glu_status_string(MISAL) == "SITU_ERR_MISALIGNED"
     assert abi.situ_glu_status_string(99) == "SITU_ERR_UNKNOWN"
@@ -351,3 +351,47 @@ def test_fc1_argument_errors(name, kw, want, native_lib_path):
 
 def test_fc1_zero_tokens_is_a_no_op(native_lib_path):
     assert fc1(tokens=0, x=None, offsets=None, y=None) == OK
+
+
+# ---- attention-residual core: argument checks run before any CUDA call -------------
+
+ARB, ARP, ARNW, ARPW, ARO = 0x40000000, 0x48000000, 0x50000000, 0x58000000, 0x60000000
+
+
+def attn_res(**kw):
+    a = dict(blocks=ARB, nblocks=8, block_row_stride=8 * 256, block_stride=256, prefix=ARP, prefix_row_stride=256,
+             dtype=BF16, tokens=64, hidden=256, norm_weight=ARNW, norm_dtype=F32, proj_weight=ARPW, proj_dtype=F32,
+             variance_epsilon=1e-6, out=ARO, out_dtype=BF16, out_row_stride=256, stream=None)
+    a.update(kw)
+    return abi.situ_attn_res_fwd(**a)
+
+
+AR_CASES = [
+    ("too many sources", dict(nblocks=16), UNSUP),
+    ("no sources", dict(nblocks=0, prefix=None), UNSUP),
+    ("negative blocks", dict(nblocks=-1), INVALID),
+    ("hidden too large", dict(hidden=40000, block_stride=40000, block_row_stride=320000, prefix_row_stride=40000,
+                              out_row_stride=40000), UNSUP),
+    ("hidden not a 16-byte multiple", dict(hidden=100, block_stride=100, block_row_stride=800, prefix_row_stride=100,
+                                           out_row_stride=100), MISAL),
+    ("epsilon negative", dict(variance_epsilon=-1.0), INVALID),
+    ("epsilon nan", dict(variance_epsilon=float("nan")), INVALID),
+    ("source stride short", dict(block_stride=128), INVALID),
+    ("out stride short", dict(out_row_stride=128), INVALID),
+    ("bad dtype", dict(out_dtype=5), INVALID),
+    ("blocks NULL", dict(blocks=None), INVALID),
+    ("blocks misaligned", dict(blocks=ARB + 8), MISAL),
+    ("source pitch not 16-byte", dict(block_stride=260, block_row_stride=8 * 260), MISAL),
+    ("out overlaps blocks", dict(out=ARB + 512), INVALID),
+    ("out overlaps the prefix", dict(out=ARP + 64), INVALID),
+]
+
+
+@pytest.mark.parametrize("name,kw,want", AR_CASES, ids=[c[0] for c in AR_CASES])
+def test_attn_res_argument_errors(name, kw, want, native_lib_path):
+    assert attn_res(**kw) == want, abi.situ_glu_last_error()
+
+
+def test_attn_res_zero_tokens_is_a_no_op(native_lib_path):
+    assert attn_res(tokens=0, blocks=None, prefix=None, nblocks=0) == UNSUP  # still no source
+    assert attn_res(tokens=0, blocks=None, out=None) == OK

@@ -32,6 +32,8 @@ TENSOR_ELEM_WEIGHTS = 5
 TENSOR_FC1_X = 6
 TENSOR_FC1_W = 7
 TENSOR_FC1_SPLIT = 8
+TENSOR_AR_VALUES = 9
+TENSOR_AR_WEIGHTS = 10
 
 
 @dataclass(frozen=True)
@@ -296,3 +298,30 @@ def fc1_inputs(tokens: int, hidden: int, inter: int, experts: int, seed: int, w_
         n = min(BLOCK_ROWS, tokens - r0)
         rw[r0:r0 + n] = _rng(seed, TENSOR_ROUTING, b).random(BLOCK_ROWS)[:n].astype(np.float32)
     return {"x": x, "w1": w1, "offsets": offsets, "routing_weights": rw}
+
+
+# ---- attention-residual mixing inputs -----------------------------------------------
+
+def attn_res_inputs(tokens: int, blocks: int, hidden: int, seed: int, dtype: str = "bf16"):
+    """Stored block sums [T, B, H] and the current prefix sum [T, H] (bf16 bits
+    or float32): source b ~ N(0, s_b) with s_b = 1 + b / 2, as sums over more
+    layers grow; norm_weight ~ 1 + 0.1 N(0, 1) and proj_weight ~ N(0, 1 /
+    sqrt(H)) float32 [H], so that logits are a few units.  64-row blocks."""
+    store = (lambda v: f32_to_bf16_bits(v.astype(np.float32))) if dtype == "bf16" else (lambda v: v.astype(np.float32))
+    kind = np.uint16 if dtype == "bf16" else np.float32
+    blk = np.empty((tokens, blocks, hidden), dtype=kind)
+    pre = np.empty((tokens, hidden), dtype=kind)
+    scale = (1.0 + 0.5 * np.arange(blocks + 1))[None, :, None]
+
+    def fill(b):
+        r0 = b * BLOCK_ROWS
+        n = min(BLOCK_ROWS, tokens - r0)
+        v = _rng(seed, TENSOR_AR_VALUES, b).standard_normal((BLOCK_ROWS, blocks + 1, hidden))[:n] * scale
+        blk[r0:r0 + n] = store(v[:, :blocks])
+        pre[r0:r0 + n] = store(v[:, blocks])
+
+    _fill_blocks(tokens, fill)
+    rng = _rng(seed, TENSOR_AR_WEIGHTS, 0)
+    norm_w = (1.0 + 0.1 * rng.standard_normal(hidden)).astype(np.float32)
+    proj_w = (rng.standard_normal(hidden) / np.sqrt(hidden)).astype(np.float32)
+    return {"blocks": blk, "prefix": pre, "norm_weight": norm_w, "proj_weight": proj_w}
