@@ -1953,6 +1953,186 @@ __global__ void __launch_bounds__(kArThreads) situ_attn_res_kernel(const ArArgs 
   }
 }
 
+// Staged form (the default when every source row is one 16-byte vector per
+// thread, at most kArStagedSources sources, and the row fits in shared
+// memory): one CTA per SM, thread j owns column vector j of every source.
+// A bulk copy brings the CTA's next token row -- each source row is one
+// contiguous run -- into shared memory while the current row is computed from
+// registers, so each value crosses HBM once and the copy of the next row
+// overlaps the reductions, the softmax and the weighted sum of this one.
+// The mbarrier wait is bounded; an expired wait sets the device status word
+// and the CTA stops after letting its own copy land.
+constexpr int kArStagedSources = 9;
+constexpr int kArStagedThreads = 896;  // hidden 7168 in bf16: one 16-byte vector per thread
+
+template <typename S>
+__global__ void __launch_bounds__(kArStagedThreads, 1) situ_attn_res_staged_kernel(const ArArgs a) {
+  constexpr int kElems = 2 * S::kPairs;
+  extern __shared__ __align__(16) unsigned char ar_stage[];  // [sources][row bytes]
+  __shared__ float red[kArStagedThreads / 32][2 * kArStagedSources];
+  __shared__ float logit_sh[kArStagedSources];
+  __shared__ __align__(8) uint64_t bar;
+  const int j = threadIdx.x, warp = j >> 5, lane = j & 31, nwarps = blockDim.x >> 5;
+  const bool col = j < a.vpr;
+  const uint32_t row_bytes = static_cast<uint32_t>(a.vpr) * kVecBytes;
+  // c = norm_w * proj_w for this thread's elements, as pairs
+  float2 c[S::kPairs];
+#pragma unroll
+  for (int p = 0; p < S::kPairs; ++p)
+    c[p] = col ? make_float2(ar_weight(a.norm_w, a.norm_bf16, j * kElems + 2 * p) *
+                                 ar_weight(a.proj_w, a.proj_bf16, j * kElems + 2 * p),
+                             ar_weight(a.norm_w, a.norm_bf16, j * kElems + 2 * p + 1) *
+                                 ar_weight(a.proj_w, a.proj_bf16, j * kElems + 2 * p + 1))
+               : make_float2(0.0f, 0.0f);
+  int64_t row = blockIdx.x;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  auto issue = [&](int64_t r) {  // thread 0: copy token row r into the stage
+    mbar_arrive_expect_tx(&bar, row_bytes * static_cast<uint32_t>(a.sources));
+    for (int b = 0; b < a.sources; ++b)
+      bulk_load(ar_stage + b * row_bytes, ar_source<S>(a, r, b), row_bytes, &bar);
+  };
+  if (threadIdx.x == 0 && row < a.tokens) issue(row);
+  uint32_t phase = 0;
+  bool in_flight = row < a.tokens;
+  while (row < a.tokens) {
+    const bool ok = mbar_wait(&bar, phase);
+    if (__syncthreads_or(!ok)) {
+      if (threadIdx.x == 0) atomicExch(&g_device_status, kStatusWaitExpired);
+      break;
+    }
+    in_flight = false;
+    phase ^= 1u;
+    uint4 x[kArStagedSources];
+#pragma unroll
+    for (int b = 0; b < kArStagedSources; ++b)
+      x[b] = (col && b < a.sources) ? lds16(ar_stage + b * row_bytes + j * kVecBytes) : make_uint4(0, 0, 0, 0);
+    __syncthreads();  // the stage is free: start the next row's copy
+    const int64_t next = row + gridDim.x;
+    if (threadIdx.x == 0 && next < a.tokens) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // our reads before the copy's writes
+      issue(next);
+    }
+    in_flight = next < a.tokens;
+    // Per-source sums of squares and projections (packed pairs).  Sources
+    // 0-7 (16 slots: 2b the sum of squares, 2b + 1 the projection) are
+    // reduced over the warp in one halving pass: at each level a lane keeps
+    // half of its slots and adds its partner's copy of that half (8 + 4 + 2
+    // + 1 exchanges, then one more add across lane pairs, instead of 5 per
+    // slot); source 8 takes plain shuffles.  Every addition order is fixed.
+    auto sums = [&](int b, float& ss, float& dd) {
+      float2 ss2 = make_float2(0.0f, 0.0f), dd2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int p = 0; p < S::kPairs; ++p) {
+        const float2 xv = as_f2(S::pair(x[b], p));
+        ss2 = fma2(xv, xv, ss2);
+        dd2 = fma2(xv, c[p], dd2);
+      }
+      ss = ss2.x + ss2.y;
+      dd = dd2.x + dd2.y;
+    };
+    {
+      float v[16];
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        v[2 * b] = 0.0f;
+        v[2 * b + 1] = 0.0f;
+        if (b < a.sources) sums(b, v[2 * b], v[2 * b + 1]);
+      }
+#pragma unroll
+      for (int o = 16, n = 8; n > 0; o >>= 1, n >>= 1) {
+        const bool upper = (lane & o) != 0;  // keep slots [n, 2n), send [0, n)
+#pragma unroll
+        for (int k = 0; k < n; ++k) {
+          const float send = upper ? v[k] : v[n + k];
+          const float keep = upper ? v[n + k] : v[k];
+          v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+      // Lanes 2s and 2s + 1 now hold the warp's sum of slot s (the halves
+      // kept, level by level, spell out bits 4..1 of the lane).
+      const int slot = lane >> 1;
+      if ((lane & 1) == 0 && slot < 2 * a.sources && slot < 16) red[warp][slot] = v[0];
+    }
+    if (a.sources > 8) {  // uniform
+      float ss = 0.0f, dd = 0.0f;
+      sums(8, ss, dd);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        dd += __shfl_xor_sync(0xffffffffu, dd, o);
+      }
+      if (lane == 0) {
+        red[warp][16] = ss;
+        red[warp][17] = dd;
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < a.sources) {
+      const int b = threadIdx.x;
+      float s2 = 0.0f, d2 = 0.0f;
+      for (int w = 0; w < nwarps; ++w) {
+        s2 += red[w][2 * b];
+        d2 += red[w][2 * b + 1];
+      }
+      logit_sh[b] = d2 * rsqrtf(s2 * a.inv_hidden + a.eps);
+    }
+    __syncthreads();
+    float p[kArStagedSources];
+    float mx = logit_sh[0];
+#pragma unroll
+    for (int b = 1; b < kArStagedSources; ++b)
+      if (b < a.sources) mx = fmaxf(mx, logit_sh[b]);
+    float z = 0.0f;
+#pragma unroll
+    for (int b = 0; b < kArStagedSources; ++b) {
+      p[b] = b < a.sources ? __expf(logit_sh[b] - mx) : 0.0f;
+      z += p[b];
+    }
+    const float rz = 1.0f / z;
+    if (col) {
+      float2 acc[S::kPairs];
+#pragma unroll
+      for (int q = 0; q < S::kPairs; ++q) acc[q] = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int b = 0; b < kArStagedSources; ++b) {
+        if (b < a.sources) {
+#pragma unroll
+          for (int q = 0; q < S::kPairs; ++q) acc[q] = fma2(splat(p[b] * rz), as_f2(S::pair(x[b], q)), acc[q]);
+        }
+      }
+      char* orow = a.out + row * a.out_pitch;
+      if (a.out_bf16) {
+        uint32_t w[S::kPairs];
+#pragma unroll
+        for (int q = 0; q < S::kPairs; ++q) w[q] = Bf16::pack(acc[q]);
+        if constexpr (S::kPairs == 4)
+          st_stream(orow + j * 16, make_uint4(w[0], w[1], w[2], w[3]));
+        else
+          st_stream8(orow + j * 8, make_uint2(w[0], w[1]));
+      } else {
+#pragma unroll
+        for (int q = 0; q < S::kPairs / 2; ++q)
+          st_stream(orow + j * kElems * 4 + q * 16,
+                    make_uint4(__float_as_uint(acc[2 * q].x), __float_as_uint(acc[2 * q].y),
+                               __float_as_uint(acc[2 * q + 1].x), __float_as_uint(acc[2 * q + 1].y)));
+      }
+    }
+    row = next;
+  }
+  // An expired wait leaves a copy possibly in flight: let it land (bounded)
+  // before the CTA's shared memory is released.
+  if (in_flight && threadIdx.x == 0) {
+    const unsigned long long t0 = global_timer_ns();
+    while (!mbar_try_wait(&bar, phase) && global_timer_ns() - t0 < kWaitLimitNs) {
+    }
+  }
+}
+
 #include "situ_fc1.cuh"
 
 // ---------------------------------------------------------------------------
@@ -3072,6 +3252,26 @@ extern "C" situ_status_t situ_attn_res_fwd(const void* blocks, int64_t nblocks, 
   a.out = static_cast<char*>(out);
   a.out_pitch = out_row_stride * oes;
   a.out_bf16 = out_dtype == SITU_DTYPE_BF16;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t stage_bytes = sources * hidden * es;
+  if (a.vpr <= kArStagedThreads && sources <= kArStagedSources && stage_bytes <= 180 * 1024) {
+    const void* ks = dtype == SITU_DTYPE_BF16 ? reinterpret_cast<const void*>(situ_attn_res_staged_kernel<Bf16>)
+                                              : reinterpret_cast<const void*>(situ_attn_res_staged_kernel<F32>);
+    const int threads = (a.vpr + 31) / 32 * 32;
+    const int smem = static_cast<int>(stage_bytes);
+    if (smem > 48 * 1024) {
+      situ_status_t st = ensure_smem(ks, smem);
+      if (st != SITU_OK) return st;
+    }
+    int grid = 0;
+    situ_status_t st = launch_grid(ks, threads, smem, tokens, &grid);
+    if (st != SITU_OK) return st;
+    if (dtype == SITU_DTYPE_BF16)
+      situ_attn_res_staged_kernel<Bf16><<<grid, threads, smem, s>>>(a);
+    else
+      situ_attn_res_staged_kernel<F32><<<grid, threads, smem, s>>>(a);
+    return check_launch("situ_attn_res_fwd");
+  }
   const void* k = dtype == SITU_DTYPE_BF16 ? reinterpret_cast<const void*>(situ_attn_res_kernel<Bf16>)
                                            : reinterpret_cast<const void*>(situ_attn_res_kernel<F32>);
   const int threads = a.vpr >= kArThreads ? kArThreads : (a.vpr + 31) / 32 * 32;
@@ -3083,7 +3283,6 @@ extern "C" situ_status_t situ_attn_res_fwd(const void* blocks, int64_t nblocks, 
   int grid = 0;
   situ_status_t st = launch_grid(k, threads, smem, tokens, &grid);
   if (st != SITU_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == SITU_DTYPE_BF16)
     situ_attn_res_kernel<Bf16><<<grid, threads, smem, s>>>(a);
   else
