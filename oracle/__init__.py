@@ -19,6 +19,9 @@ Sources followed (see the C file for the per-function citations):
   * Megatron-LM PR #6673, "Design": the fused grouped GEMM + SiTU-GLU, taken
     as FC1 (per-expert grouped GEMM) followed by the activation
     (fc1_oracle.c).
+  * Megatron-LM PR #6673, "Test results" (the fused path's backward with a
+    dSiTU correction): FC2's data gradient followed by the SiTU-GLU backward
+    (fc2_oracle.c).
   * NeMo AutoModel API, kimi_k3.situ `_attn_res_core` / `_apply_attn_res`:
     the attention-residual mixing chain (attn_res_oracle.c).
   * OCP Microscaling Formats (MX) v1.0 for the MXFP8 outputs (E4M3 elements,
@@ -42,7 +45,8 @@ SOURCE = os.path.join(_HERE, "situ_oracle.c")
 MX_SOURCE = os.path.join(_HERE, "mx_oracle.c")  # MXFP8 block scaling (OCP MX v1.0)
 FC1_SOURCE = os.path.join(_HERE, "fc1_oracle.c")  # FC1 (grouped) followed by SiTU-GLU
 ATTN_RES_SOURCE = os.path.join(_HERE, "attn_res_oracle.c")  # attention-residual mixing core
-SOURCES = [SOURCE, MX_SOURCE, FC1_SOURCE, ATTN_RES_SOURCE]
+FC2_SOURCE = os.path.join(_HERE, "fc2_oracle.c")  # FC2 data gradient followed by the SiTU-GLU backward
+SOURCES = [SOURCE, MX_SOURCE, FC1_SOURCE, ATTN_RES_SOURCE, FC2_SOURCE]
 LIBRARY = os.path.join(_HERE, "libsitu_oracle.so")
 
 DTYPE_BF16 = 0
@@ -146,6 +150,9 @@ class Oracle:
         lib.situ_oracle_attn_res.argtypes = [_VP, _I64, _I64, _I64, _VP, _I64, _INT, _I64, _VP, _INT, _VP, _INT,
                                              _DBL, _VP, _I64, _VP, _VP, _VP]
         lib.situ_oracle_attn_res.restype = _INT
+        lib.situ_oracle_fc2_dgrad.argtypes = [_VP, _I64, _I64, _VP, _I64, _I64, _VP, _I64, _VP, _I64, _VP, _DBL, _INT,
+                                              _DBL, _VP, _I64, _VP, _VP, _VP, _VP, _VP]
+        lib.situ_oracle_fc2_dgrad.restype = _INT
         self._lib = lib
         self.mutant_id = lib.situ_oracle_mutant_id()
 
@@ -355,6 +362,39 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle attn_res rejected its arguments")
         return out, mag, prob
+
+
+    # -- FC2 data gradient + SiTU-GLU backward (fc2_oracle.c) -----------------
+
+    def fc2_dgrad(self, dout, w2t, offsets, gate_up, rw, beta, linear_beta=None, rows=None):
+        """(d_gate_up [n, 2I], d_w [n], dY [n, I], error scales [n, 2I], d_w error
+        scales [n]) in float64 for token rows of dout (bf16 bits [T, H]) routed by
+        ``offsets`` to experts with transposed FC2 weights w2t (bf16 bits
+        [E * I, H]); gate_up: the saved bf16 bits [T, 2I]; rw: float32 [T] or None."""
+        dout = np.ascontiguousarray(dout)
+        w2t = np.ascontiguousarray(w2t)
+        gate_up = np.ascontiguousarray(gate_up)
+        for a in (dout, w2t, gate_up):
+            if a.dtype != np.uint16:
+                raise TypeError("dout, w2t and gate_up are bf16 bit patterns (uint16)")
+        off = np.ascontiguousarray(np.asarray(offsets, dtype=np.int64))
+        T, hidden = dout.shape
+        inter = gate_up.shape[1] // 2
+        r, n = self._rows(rows, T)
+        rw_c = None if rw is None else np.ascontiguousarray(np.asarray(rw, dtype=np.float32).reshape(-1))
+        dgu = np.empty((n, 2 * inter))
+        dw = np.empty(n)
+        dy = np.empty((n, inter))
+        err = np.empty((n, 2 * inter))
+        dw_err = np.empty(n)
+        has = linear_beta is not None
+        rc = self._lib.situ_oracle_fc2_dgrad(_ptr(dout), dout.shape[1], hidden, _ptr(w2t), w2t.shape[1], inter,
+                                             _ptr(off), off.size - 1, _ptr(gate_up), gate_up.shape[1], _ptr(rw_c),
+                                             float(beta), int(has), float(linear_beta if has else 0.0), _ptr(r), n,
+                                             _ptr(dgu), _ptr(dw), _ptr(dy), _ptr(err), _ptr(dw_err))
+        if rc != 0:
+            raise ValueError("oracle fc2_dgrad rejected its arguments")
+        return dgu, dw, dy, err, dw_err
 
 
 _DEFAULT = None

@@ -21,6 +21,9 @@ itself checked here against things other than itself:
   * FC1 + SiTU-GLU (fc1_oracle.c): fsum dot products and 50-digit element
     values, exact agreement with the activation oracle on bf16-exact FC1
     outputs, and the grouped call against per-expert calls;
+  * FC2 data gradient + SiTU-GLU backward (fc2_oracle.c): fsum dot products
+    with 50-digit derivatives, exact agreement with the activation backward
+    on bf16-exact dY, per-expert calls;
   * attention-residual core (attn_res_oracle.c): torch's float64 rms_norm and
     softmax, invariants (identical sources, zero projection, one source,
     scaling), large logits, and the two-array source layout.
@@ -572,6 +575,74 @@ def pin_attn_res_two_arrays(o):
     assert np.array_equal(a, b)
 
 
+# ---- FC2 data gradient + SiTU-GLU backward (fc2_oracle.c) ---------------------------
+
+def pin_fc2_dgrad_bruteforce(o):
+    """A tiny grouped case: dY as fsum dot products with the owning expert's
+    transposed FC2 rows, dG, dU from 50-digit derivatives of the branch
+    functions, d_w an fsum over the row."""
+    rng = np.random.default_rng(RNG_SEED + 10)
+    E, I, H, T = 2, 8, 24, 9
+    dout = _bf16(rng.standard_normal((T, H)))
+    w2t = _bf16(0.3 * rng.standard_normal((E * I, H)))
+    gu = _bf16(2.0 * rng.standard_normal((T, 2 * I)))
+    offsets = [0, 5, 9]
+    rw = rng.random(T).astype(np.float32)
+    dgu, dw, dy, err, dw_err = o.fc2_dgrad(dout, w2t, offsets, gu, rw, 4.0, 25.0)
+    df, wf, gf = _widen(dout), _widen(w2t), _widen(gu)
+    for r in range(T):
+        e = 0 if r < 5 else 1
+        terms = []
+        for i in range(I):
+            d = math.fsum(df[r] * wf[e * I + i])
+            assert _close(dy[r, i], d, 1e-14, 1e-14), (r, i)
+            g, u = gf[r, i], gf[r, I + i]
+            tg, tu = float(_mp_gate(g, 4.0)), float(_mp_up(u, 25.0))
+            dtg = _mp_diff(lambda v: _mp_gate(v, 4.0), g)
+            dtu = _mp_diff(lambda v: _mp_up(v, 25.0), u)
+            assert _close(dgu[r, i], d * float(rw[r]) * tu * dtg, 1e-12, 1e-14), (r, i)
+            assert _close(dgu[r, I + i], d * float(rw[r]) * tg * dtu, 1e-12, 1e-14), (r, i)
+            terms.append(d * tg * tu)
+        assert _close(dw[r], math.fsum(terms), 1e-12, 1e-14), r
+    assert np.all(err >= 0) and np.all(dw_err >= 0)
+
+
+def pin_fc2_dgrad_matches_activation_backward(o):
+    """With inputs in {-1/4, 0, 1/4} every dY is k/16, a bf16 number: the fused
+    oracle then equals the pinned activation backward with grad_out = dY."""
+    rng = np.random.default_rng(RNG_SEED + 11)
+    T, H, I = 5, 16, 8
+    dout = _bf16(rng.integers(-1, 2, (T, H)) / 4.0)
+    w2t = _bf16(rng.integers(-1, 2, (I, H)) / 4.0)
+    gu = _bf16(rng.standard_normal((T, 2 * I)) * 3.0)
+    rw = rng.random(T).astype(np.float32)
+    for beta, lb in ((4.0, 25.0), (1.0, None)):
+        dgu, dw, dy, _, _ = o.fc2_dgrad(dout, w2t, [0, T], gu, rw, beta, lb)
+        dy_bits = _bf16(dy)
+        assert np.array_equal(_widen(dy_bits), dy)
+        ref = o.bwd(gu, rw, dy_bits, beta, lb)
+        assert np.array_equal(dgu[:, :I], ref.dg) and np.array_equal(dgu[:, I:], ref.du)
+        assert np.allclose(dw, ref.dw, rtol=1e-14, atol=1e-15)
+
+
+def pin_fc2_dgrad_grouped_equals_per_expert(o):
+    rng = np.random.default_rng(RNG_SEED + 12)
+    E, I, H = 3, 8, 32
+    offsets = np.array([0, 4, 4, 11], dtype=np.int64)
+    T = 11
+    dout = _bf16(rng.standard_normal((T, H)))
+    w2t = _bf16(0.2 * rng.standard_normal((E * I, H)))
+    gu = _bf16(rng.standard_normal((T, 2 * I)))
+    rw = rng.random(T).astype(np.float32)
+    dgu, dw, _, _, _ = o.fc2_dgrad(dout, w2t, offsets, gu, rw, 4.0, 25.0)
+    for e in range(E):
+        a, b = offsets[e], offsets[e + 1]
+        if a == b:
+            continue
+        de, we, _, _, _ = o.fc2_dgrad(dout[a:b], w2t[e * I:(e + 1) * I], [0, b - a], gu[a:b], rw[a:b], 4.0, 25.0)
+        assert np.array_equal(dgu[a:b], de) and np.array_equal(dw[a:b], we)
+
+
 PINS = [
     pin_gate_values_mpmath,
     pin_up_values_mpmath,
@@ -598,6 +669,9 @@ PINS = [
     pin_attn_res_invariants,
     pin_attn_res_large_logits,
     pin_attn_res_two_arrays,
+    pin_fc2_dgrad_bruteforce,
+    pin_fc2_dgrad_matches_activation_backward,
+    pin_fc2_dgrad_grouped_equals_per_expert,
 ]
 
 
@@ -637,6 +711,9 @@ MUTANTS = {
     26: "RMSNorm weight not applied",
     27: "softmax without the max shift",
     28: "a transformed value combined instead of the raw one",
+    29: "FC2 weight read untransposed in the data gradient",
+    30: "routing weight dropped from the fused dG",
+    31: "upstream gradient dropped from the fused d_w",
 }
 
 
