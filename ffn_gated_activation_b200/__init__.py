@@ -19,6 +19,7 @@ from .functional import (
     situ_glu_bwd,
     situ_glu_bwd_mxfp8,
     situ_glu_fc1_fwd,
+    situ_glu_fc2_dgrad_bwd,
     situ_glu_fwd,
     situ_glu_fwd_mxfp8,
     situlu,
@@ -40,6 +41,7 @@ __all__ = [
     "situ_glu_fwd_mxfp8",
     "situ_glu_bwd_mxfp8",
     "situ_glu_fc1_fwd",
+    "situ_glu_fc2_dgrad_bwd",
     "situlu",
     "weighted_situ",
 ]

@@ -13,7 +13,7 @@ import subprocess
 PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG_DIR)
 SOURCES = [os.path.join(PKG_DIR, "csrc", "situ_glu.cu")]
-HEADERS = [os.path.join(ROOT, "include", "situ_glu.h"), os.path.join(PKG_DIR, "csrc", "situ_fc1.cuh")]
+HEADERS = [os.path.join(ROOT, "include", "situ_glu.h"), os.path.join(PKG_DIR, "csrc", "situ_fused_gemm.cuh")]
 LIBRARY = os.path.join(PKG_DIR, "libsitu_glu.so")
 
 NVCC_FLAGS = [

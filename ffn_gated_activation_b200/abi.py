@@ -31,7 +31,7 @@ SITU_RW_FULL = 4
 SITU_MX_RULE_OCP = 0
 SITU_MX_RULE_CEIL = 1
 
-ABI_VERSION = 5
+ABI_VERSION = 6
 
 # Entry points declared in include/situ_glu.h: name -> (restype, argtypes).
 _I64, _INT, _DBL, _VP, _SZ = ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_void_p, ctypes.c_size_t
@@ -46,6 +46,9 @@ SIGNATURES = {
                                   _VP, _I64, _VP, _I64, _VP, _I64, _INT, _VP, _I64, _VP, _SZ, _VP]),
     "situ_glu_fc1_fwd": (_INT, [_VP, _I64, _I64, _I64, _VP, _I64, _I64, _I64, _VP, _VP, _INT, _INT, _I64,
                                 _DBL, _INT, _DBL, _VP, _I64, _VP]),
+    "situ_glu_fc2_dgrad_bwd": (_INT, [_VP, _I64, _I64, _I64, _VP, _I64, _I64, _I64, _VP, _VP, _I64, _VP, _INT, _INT,
+                                      _I64, _DBL, _INT, _DBL, _VP, _I64, _VP, _I64, _VP, _SZ, _VP]),
+    "situ_glu_fc2_dgrad_workspace_bytes": (_SZ, [_I64, _I64, _INT]),
     "situ_attn_res_fwd": (_INT, [_VP, _I64, _I64, _I64, _VP, _I64, _INT, _I64, _I64, _VP, _INT, _VP, _INT, _DBL,
                                  _VP, _INT, _I64, _VP]),
     "situ_glu_bwd_workspace_bytes": (_SZ, [_I64, _I64, _INT, _INT]),
@@ -142,6 +145,20 @@ def situ_glu_fc1_fwd(x, tokens, hidden, x_row_stride, w1, experts, inter, w1_row
     return lib().situ_glu_fc1_fwd(x, tokens, hidden, x_row_stride, w1, experts, inter, w1_row_stride, offsets, rw,
                                   rw_dtype, rw_mode, rw_stride, beta, has_linear_beta, linear_beta, y, y_row_stride,
                                   stream)
+
+
+def situ_glu_fc2_dgrad_bwd(dout, tokens, hidden, dout_row_stride, w2t, experts, inter, w2t_row_stride, offsets,
+                           gate_up, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride, beta, has_linear_beta,
+                           linear_beta, d_gate_up, d_gate_up_row_stride, d_rw, d_rw_stride, workspace,
+                           workspace_bytes, stream) -> int:
+    return lib().situ_glu_fc2_dgrad_bwd(dout, tokens, hidden, dout_row_stride, w2t, experts, inter, w2t_row_stride,
+                                        offsets, gate_up, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride, beta,
+                                        has_linear_beta, linear_beta, d_gate_up, d_gate_up_row_stride, d_rw,
+                                        d_rw_stride, workspace, workspace_bytes, stream)
+
+
+def situ_glu_fc2_dgrad_workspace_bytes(tokens, inter, want_drw) -> int:
+    return lib().situ_glu_fc2_dgrad_workspace_bytes(tokens, inter, want_drw)
 
 
 def situ_attn_res_fwd(blocks, nblocks, block_row_stride, block_stride, prefix, prefix_row_stride, dtype, tokens,

@@ -1,35 +1,42 @@
-// FC1 grouped GEMM with the SiTU-GLU epilogue on the sm_100a tensor cores.
+// Grouped GEMMs on the sm_100a tensor cores with a SiTU-GLU epilogue: the
+// fused FC1 forward and the fused FC2 data gradient.
 //
-// Megatron-LM PR #6673, "Design": with a SiTU-capable cuDNN frontend, FC1's
-// grouped GEMM and the SiTU-GLU activation run as one fused operation.  For a
+// FC1 (Megatron-LM PR #6673, "Design": with a SiTU-capable cuDNN frontend,
+// FC1's grouped GEMM and the SiTU-GLU activation run as one operation).  For a
 // token row r routed to expert e,
 //     G[r, i] = sum_k X[r, k] W1_e[i, k],  U[r, i] = sum_k X[r, k] W1_e[I + i, k]
 //     Y[r, i] = T_g(G) T_u(U) w[r]
-// and the fp32 gate/up accumulators never leave the chip: this kernel reads
-// X and W1 once per tile and writes only Y.
+// FC2 data gradient with the SiTU-GLU backward (the "dSiTU" of the fused
+// grouped MLP's backward, Megatron-LM PR #6673, "Test results"):
+//     dY[r, i] = sum_h dOut[r, h] W2_e[h, i]   (W2 passed transposed: W2T_e [I, H])
+//     dG = dY w T_u T_g',  dU = dY w T_g T_u',  d_w[r] = sum_i dY T_g T_u
+// The fp32 accumulators never leave the chip: G and U (or dY) are never
+// written, only Y (or dG, dU and per-tile d_w partials).
 //
 // Included into situ_glu.cu (anonymous namespace): it uses the library's
-// element arithmetic (fwd_pair_abs), storage helpers and bounded mbarriers.
+// element arithmetic (fwd_pair_abs, bwd_pair), storage helpers and bounded
+// mbarriers.
 //
 // Structure (one CTA per SM, persistent over output tiles):
-//   * tile = 128 token rows x 128 output columns; its gate columns
-//     [n0, n0 + 128) and up columns [I + n0, I + n0 + 128) of W1_e are loaded
-//     as one 256-row B operand, so one tcgen05.mma (M = 128, N = 256,
-//     K = 16) accumulates gate and up side by side in 256 TMEM columns;
-//   * warp 0 streams 64-wide K slices of X and W1 with TMA (128-byte swizzle)
-//     into a 4-stage shared-memory ring; warp 1 owns the TMEM allocation and
-//     issues the MMAs from one lane, releasing each stage with tcgen05.commit;
+//   * a tile is 128 token rows; its B operand is 256 rows of the expert's
+//     weight, so one tcgen05.mma (M = 128, N = 256, K = 16) per 16 hidden
+//     elements fills 256 TMEM columns.  FC1 puts gate columns [n0, n0 + 128)
+//     and the matching up columns side by side (128 output columns per tile);
+//     FC2 takes 256 consecutive dY columns;
+//   * warp 0 streams 64-wide K slices with TMA (128-byte swizzle) into a
+//     4-stage shared-memory ring; warp 1 owns the TMEM allocation and issues
+//     the MMAs from one lane, releasing each stage with tcgen05.commit;
 //   * two TMEM accumulators (512 columns) let warps 2-5 run the epilogue of
 //     one tile while the next tile's MMAs run: each epilogue thread owns one
-//     accumulator row (its warp's TMEM lane quarter), reads gate and up
-//     columns with tcgen05.ld, applies SiTU-GLU and the routing weight in
-//     fp32 and stores bf16 Y, then releases the accumulator;
+//     accumulator row (its warp's TMEM lane quarter), reads it with
+//     tcgen05.ld, applies the element arithmetic in fp32 and stores bf16;
 //   * tiles are numbered expert by expert from device-side row offsets; within
 //     an expert, groups of kGroupM row tiles sweep the column tiles so that
-//     the CTAs running together share X and W1 tiles in L2.
+//     the CTAs running together share operand tiles in L2.
 // Every wait is bounded (kWaitLimitNs); a wait that expires sets the device
 // status word and a CTA-wide abort flag, every role then stops issuing work,
-// the producer waits (bounded) for its own copies, and TMEM is freed.
+// the producer waits (bounded) for its own copies, the MMA warp for its own
+// MMAs, and TMEM is freed.
 
 namespace fc1 {
 
@@ -69,8 +76,11 @@ struct Args {
   int hidden;
   int inter;
   RwArgs rw;
-  char* y;                 // bf16 [tokens, >= inter]
+  char* y;                 // FC1: Y bf16 [tokens, >= inter]; FC2: d_gate_up bf16 [tokens, >= 2 inter]
   int64_t y_pitch;         // bytes
+  const char* gate_up;     // FC2: the saved gate_up bf16 [tokens, >= 2 inter]
+  int64_t gu_pitch;        // bytes
+  float* partials;         // FC2: d_w partials [tokens][inter / 256] (NULL: not wanted)
   Coeffs c;
 };
 
@@ -152,7 +162,7 @@ struct Tile {
 // tiles sweep all column tiles).  first_tile[e] is the first tile of expert e,
 // first_tile[experts] the total; [lo[e], hi[e]) its rows.
 __device__ __forceinline__ Tile decode_tile(int t, const int* first_tile, const int64_t* lo, const int64_t* hi,
-                                            int experts, int n_tiles) {
+                                            int experts, int n_tiles, int out_cols) {
   int left = 0, right = experts - 1;  // the last e with first_tile[e] <= t
   while (left < right) {
     const int mid = (left + right + 1) >> 1;
@@ -170,14 +180,102 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* first_tile, const 
   tile.expert = e;
   tile.m0 = r0 + static_cast<int64_t>(first_m + within % group_m) * kBM;
   tile.m_end = r1;
-  tile.n0 = (within / group_m) * kBN;
+  tile.n0 = (within / group_m) * out_cols;
   return tile;
 }
 
-template <int GATE, bool HAS_LB>
+// FC1: B = the expert's gate rows [n0, n0 + 128) then its up rows; the
+// epilogue turns gate column c and up column 128 + c into Y column n0 + c.
+struct Fc1Epilogue {
+  static constexpr int kOutCols = kBN;
+  __device__ __forceinline__ static void b_rows(const Args& a, const Tile& t, int32_t& r0, int32_t& r1) {
+    r0 = t.expert * 2 * a.inter + t.n0;
+    r1 = r0 + a.inter;
+  }
+  template <int GATE, bool HAS_LB>
+  __device__ __forceinline__ static void run(const Args& a, const Tile& tile, int64_t row, bool valid,
+                                             uint32_t taddr) {
+    const float wbb = (valid ? load_rw(a.rw, row) : 0.0f) * a.c.bb;
+    char* yrow = a.y + (valid ? row : 0) * a.y_pitch + static_cast<int64_t>(tile.n0) * 2;
+#pragma unroll 1
+    for (int c = 0; c < kBN; c += 16) {
+      uint32_t g[16], u[16];
+      tmem_ld16(taddr + c, g);
+      tmem_ld16(taddr + kBN + c, u);
+      tmem_ld_wait();
+      uint32_t q[8];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 gv = make_uint4(g[4 * v], g[4 * v + 1], g[4 * v + 2], g[4 * v + 3]);
+        const uint4 uv = make_uint4(u[4 * v], u[4 * v + 1], u[4 * v + 2], u[4 * v + 3]);
+#pragma unroll
+        for (int p = 0; p < 2; ++p)
+          q[2 * v + p] =
+              Bf16::pack(fwd_pair_abs<GATE, HAS_LB, F32>(F32::pair(gv, p), F32::pair(uv, p), splat(wbb), a.c));
+      }
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(yrow + c * 2);
+        dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
+        dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
+      }
+    }
+  }
+};
+
+// FC2 data gradient: B = the expert's transposed FC2 rows [n0, n0 + 256); the
+// epilogue reads G, U of the saved gate_up row, writes dG, dU for columns
+// [n0, n0 + 256) and the tile's share of d_w.
+struct Fc2Epilogue {
+  static constexpr int kOutCols = kUmmaN;
+  __device__ __forceinline__ static void b_rows(const Args& a, const Tile& t, int32_t& r0, int32_t& r1) {
+    r0 = t.expert * a.inter + t.n0;
+    r1 = r0 + kBN;
+  }
+  template <int GATE, bool HAS_LB>
+  __device__ __forceinline__ static void run(const Args& a, const Tile& tile, int64_t row, bool valid,
+                                             uint32_t taddr) {
+    const float w = valid ? load_rw(a.rw, row) : 0.0f;
+    const float2 k = bwd_row_consts<HAS_LB>(w, a.c);
+    const float2 kdg = splat(k.x), kdu = splat(k.y);
+    const int64_t r = valid ? row : 0;
+    const char* grow = a.gate_up + r * a.gu_pitch + static_cast<int64_t>(tile.n0) * 2;
+    const char* urow = grow + static_cast<int64_t>(a.inter) * 2;
+    char* dgrow = a.y + r * a.y_pitch + static_cast<int64_t>(tile.n0) * 2;
+    char* durow = dgrow + static_cast<int64_t>(a.inter) * 2;
+    float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll 1
+    for (int c = 0; c < kUmmaN; c += 16) {
+      uint32_t d[16];
+      tmem_ld16(taddr + c, d);
+      tmem_ld_wait();
+      if (valid) {
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          const uint4 gv = *reinterpret_cast<const uint4*>(grow + c * 2 + v * 16);
+          const uint4 uv = *reinterpret_cast<const uint4*>(urow + c * 2 + v * 16);
+          uint4 dgv, duv;
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            float2 dg, du;
+            const float2 go = make_float2(__uint_as_float(d[8 * v + 2 * p]), __uint_as_float(d[8 * v + 2 * p + 1]));
+            bwd_pair<GATE, HAS_LB, Bf16>(Bf16::pair(gv, p), Bf16::pair(uv, p), go, kdg, kdu, a.c, dg, du, acc);
+            Bf16::put(dgv, p, dg);
+            Bf16::put(duv, p, du);
+          }
+          *reinterpret_cast<uint4*>(dgrow + c * 2 + v * 16) = dgv;
+          *reinterpret_cast<uint4*>(durow + c * 2 + v * 16) = duv;
+        }
+      }
+    }
+    if (valid && a.partials != nullptr)
+      a.partials[row * (a.inter / kUmmaN) + tile.n0 / kUmmaN] = (acc.x + acc.y) * bwd_dw_scale(a.c);
+  }
+};
+
+template <class Epi, int GATE, bool HAS_LB>
 __global__ void __launch_bounds__(kThreads, 1)
-    situ_fc1_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                    const Args a) {
+    situ_fused_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                           const Args a) {
   extern __shared__ unsigned char smem_raw[];
   // The ring needs 1024-byte alignment (128-byte swizzle atoms of 8 rows).
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -195,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* first_tile = reinterpret_cast<int*>(hi + a.experts);                              // [experts + 1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles = a.inter / kBN;
+  const int n_tiles = a.inter / Epi::kOutCols;
   const int k_blocks = a.hidden / kBK;
 
   if (threadIdx.x == 0) {
@@ -258,8 +356,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t issued = 0;  // bit s: stage s holds a copy that may still be in flight
     bool ok = true;
     for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
-      const Tile tile = decode_tile(t, first_tile, lo, hi, a.experts, n_tiles);
-      const int32_t wrow = tile.expert * 2 * a.inter + tile.n0;
+      const Tile tile = decode_tile(t, first_tile, lo, hi, a.experts, n_tiles, Epi::kOutCols);
+      int32_t wrow0, wrow1;
+      Epi::b_rows(a, tile, wrow0, wrow1);
       for (int kb = 0; kb < k_blocks; ++kb) {
         if (!wait_or_abort(&empty[stage], phase ^ 1u, abort_flag)) {
           ok = false;
@@ -269,8 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           unsigned char* st = ring + stage * kStageBytes;
           mbar_arrive_expect_tx(&full[stage], kStageBytes);
           tma_load_2d(st, &tmap_x, kb * kBK, static_cast<int32_t>(tile.m0), &full[stage]);
-          tma_load_2d(st + kABytes, &tmap_w, kb * kBK, wrow, &full[stage]);
-          tma_load_2d(st + kABytes + kBHalfBytes, &tmap_w, kb * kBK, wrow + a.inter, &full[stage]);
+          tma_load_2d(st + kABytes, &tmap_w, kb * kBK, wrow0, &full[stage]);
+          tma_load_2d(st + kABytes + kBHalfBytes, &tmap_w, kb * kBK, wrow1, &full[stage]);
         }
         __syncwarp();
         issued |= 1u << stage;
@@ -349,33 +448,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = it & 1;
       if (!wait_or_abort(&acc_full[b], (acc_phase >> b) & 1u, abort_flag)) break;
       tc_fence_after();
-      const Tile tile = decode_tile(t, first_tile, lo, hi, a.experts, n_tiles);
+      const Tile tile = decode_tile(t, first_tile, lo, hi, a.experts, n_tiles, Epi::kOutCols);
       const int64_t row = tile.m0 + row_in_tile;
-      const bool valid = row < tile.m_end;
-      const float wbb = (valid ? load_rw(a.rw, row) : 0.0f) * a.c.bb;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * kAccCols);
-      char* yrow = a.y + (valid ? row : 0) * a.y_pitch + static_cast<int64_t>(tile.n0) * 2;
-#pragma unroll 1
-      for (int c = 0; c < kBN; c += 16) {
-        uint32_t g[16], u[16];
-        tmem_ld16(taddr + c, g);
-        tmem_ld16(taddr + kBN + c, u);
-        tmem_ld_wait();
-        uint32_t q[8];
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const uint4 gv = make_uint4(g[4 * v], g[4 * v + 1], g[4 * v + 2], g[4 * v + 3]);
-          const uint4 uv = make_uint4(u[4 * v], u[4 * v + 1], u[4 * v + 2], u[4 * v + 3]);
-#pragma unroll
-          for (int p = 0; p < 2; ++p)
-            q[2 * v + p] = Bf16::pack(fwd_pair_abs<GATE, HAS_LB, F32>(F32::pair(gv, p), F32::pair(uv, p), splat(wbb), a.c));
-        }
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(yrow + c * 2);
-          dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
-          dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
-        }
-      }
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * kAccCols);
+      Epi::template run<GATE, HAS_LB>(a, tile, row, row < tile.m_end, taddr);
       tc_fence_before();
       mbar_arrive(&acc_empty[b]);
       acc_phase ^= 1u << b;

@@ -2133,7 +2133,7 @@ __global__ void __launch_bounds__(kArStagedThreads, 1) situ_attn_res_staged_kern
   }
 }
 
-#include "situ_fc1.cuh"
+#include "situ_fused_gemm.cuh"
 
 // ---------------------------------------------------------------------------
 // Host side
@@ -2697,15 +2697,54 @@ situ_status_t bf16_tile_map(CUtensorMap* m, const void* base, int64_t inner, int
   return SITU_OK;
 }
 
-using Fc1Kernel = void (*)(const CUtensorMap, const CUtensorMap, const fc1::Args);
+using FusedGemmKernel = void (*)(const CUtensorMap, const CUtensorMap, const fc1::Args);
 
-template <bool LB>
-Fc1Kernel pick_fc1_gate(int gate) {
+template <class Epi, bool LB>
+FusedGemmKernel pick_fused_gate(int gate) {
   switch (gate) {
-    case kGateSquare: return fc1::situ_fc1_kernel<kGateSquare, LB>;
-    case kGateEqual: return fc1::situ_fc1_kernel<kGateEqual, LB>;
-    case kGateRoot: return fc1::situ_fc1_kernel<kGateRoot, LB>;
-    default: return fc1::situ_fc1_kernel<kGateGeneric, LB>;
+    case kGateSquare: return fc1::situ_fused_gemm_kernel<Epi, kGateSquare, LB>;
+    case kGateEqual: return fc1::situ_fused_gemm_kernel<Epi, kGateEqual, LB>;
+    case kGateRoot: return fc1::situ_fused_gemm_kernel<Epi, kGateRoot, LB>;
+    default: return fc1::situ_fused_gemm_kernel<Epi, kGateGeneric, LB>;
+  }
+}
+
+template <class Epi>
+FusedGemmKernel pick_fused(int gate, bool lb) {
+  return lb ? pick_fused_gate<Epi, true>(gate) : pick_fused_gate<Epi, false>(gate);
+}
+
+// Launch of a fused grouped GEMM: one persistent CTA per SM.
+situ_status_t launch_fused(FusedGemmKernel k, const CUtensorMap& ma, const CUtensorMap& mb, const fc1::Args& a,
+                           int64_t experts, cudaStream_t s, const char* what) {
+  const int smem = fc1::kStages * fc1::kStageBytes + 1024 + fc1::kHeaderBytes + static_cast<int>(experts) * (8 + 8 + 4) + 8;
+  cudaError_t err = cudaFuncSetAttribute(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem);
+  if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(err));
+  int sms = 0;
+  situ_status_t st = device_sm_count(&sms);
+  if (st != SITU_OK) return st;
+  int grid = sms;
+  const int cap = g_max_ctas.load(std::memory_order_relaxed);
+  if (cap > 0 && grid > cap) grid = cap;
+  k<<<grid, fc1::kThreads, smem, s>>>(ma, mb, a);
+  return check_launch(what);
+}
+
+// Per-row d_w of the fused FC2 data gradient: the row's column-tile partials
+// in tile order, for the rows [offsets[0], offsets[experts]) (clamped).
+__global__ void __launch_bounds__(256) situ_fc2_dw_finalize_kernel(const float* partials, int n_tiles,
+                                                                   const int64_t* offsets, int experts,
+                                                                   int64_t tokens, void* d_rw, int64_t d_rw_stride,
+                                                                   int bf16) {
+  int64_t lo = offsets[0], hi = offsets[experts];
+  lo = lo < 0 ? 0 : (lo > tokens ? tokens : lo);
+  hi = hi < lo ? lo : (hi > tokens ? tokens : hi);
+  for (int64_t r = lo + blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; r < hi;
+       r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float sum = 0.0f;
+    for (int k = 0; k < n_tiles; ++k) sum += partials[r * n_tiles + k];
+    store_rw_grad(d_rw, r * d_rw_stride, bf16, sum);
   }
 }
 
@@ -3164,20 +3203,126 @@ extern "C" situ_status_t situ_glu_fc1_fwd(const void* x, int64_t tokens, int64_t
   st = bf16_tile_map(&mw, w1, hidden, experts * 2 * inter, w1_row_stride);
   if (st != SITU_OK) return st;
 
-  Fc1Kernel k = has_linear_beta ? pick_fc1_gate<true>(gate) : pick_fc1_gate<false>(gate);
-  const int smem = fc1::kStages * fc1::kStageBytes + 1024 + fc1::kHeaderBytes +
-                   static_cast<int>(experts) * (8 + 8 + 4) + 8;
-  cudaError_t err = cudaFuncSetAttribute(reinterpret_cast<const void*>(k),
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(err));
+  return launch_fused(pick_fused<fc1::Fc1Epilogue>(gate, has_linear_beta != 0), mx, mw, a, experts,
+                      static_cast<cudaStream_t>(stream), "situ_glu_fc1_fwd");
+}
+
+// ---------------------------------------------------------------------------
+// FC2 data gradient + SiTU-GLU backward
+// ---------------------------------------------------------------------------
+
+extern "C" size_t situ_glu_fc2_dgrad_workspace_bytes(int64_t tokens, int64_t inter, int want_drw) {
+  if (tokens <= 0 || inter <= 0 || !want_drw) return 0;
+  const uint64_t bytes = static_cast<uint64_t>(tokens) * static_cast<uint64_t>(inter / fc1::kUmmaN) * sizeof(float);
+  return static_cast<size_t>((bytes + 255) / 256 * 256);
+}
+
+extern "C" situ_status_t situ_glu_fc2_dgrad_bwd(const void* dout, int64_t tokens, int64_t hidden,
+                                                int64_t dout_row_stride, const void* w2t, int64_t experts,
+                                                int64_t inter, int64_t w2t_row_stride, const int64_t* offsets,
+                                                const void* gate_up, int64_t gate_up_row_stride, const void* rw,
+                                                situ_dtype_t rw_dtype, situ_rw_mode_t rw_mode, int64_t rw_stride,
+                                                double beta, int has_linear_beta, double linear_beta,
+                                                void* d_gate_up, int64_t d_gate_up_row_stride, void* d_rw,
+                                                int64_t d_rw_stride, void* workspace, size_t workspace_bytes,
+                                                void* stream) {
+  tl_last_error[0] = '\0';
+  if (!finite_positive(beta)) return fail(SITU_ERR_INVALID_ARG, "beta must be finite and > 0");
+  if (has_linear_beta != 0 && has_linear_beta != 1)
+    return fail(SITU_ERR_INVALID_ARG, "has_linear_beta must be 0 or 1");
+  if (has_linear_beta && !finite_positive(linear_beta))
+    return fail(SITU_ERR_INVALID_ARG, "linear_beta must be finite and > 0");
+  if (rw_mode != SITU_RW_ROW && rw_mode != SITU_RW_NONE)
+    return fail(rw_mode == SITU_RW_SCALAR || rw_mode == SITU_RW_COL || rw_mode == SITU_RW_FULL ? SITU_ERR_UNSUPPORTED
+                                                                                                : SITU_ERR_INVALID_ARG,
+                "situ_glu_fc2_dgrad_bwd takes per-row or no routing weights");
+  if (rw_mode != SITU_RW_NONE && !valid_dtype(rw_dtype))
+    return fail(SITU_ERR_INVALID_ARG, "rw_dtype %d is not a situ_dtype_t", (int)rw_dtype);
+  if (rw_mode == SITU_RW_NONE && (rw != nullptr || d_rw != nullptr))
+    return fail(SITU_ERR_INVALID_ARG, "rw and d_rw must be NULL for SITU_RW_NONE");
+  if (tokens < 0) return fail(SITU_ERR_INVALID_ARG, "tokens = %lld < 0", (long long)tokens);
+  if (hidden < fc1::kBK || hidden % fc1::kBK != 0)
+    return fail(SITU_ERR_UNSUPPORTED, "hidden must be a positive multiple of %d, got %lld", fc1::kBK,
+                (long long)hidden);
+  if (inter < fc1::kUmmaN || inter % fc1::kUmmaN != 0)
+    return fail(SITU_ERR_UNSUPPORTED, "inter must be a positive multiple of %d, got %lld", fc1::kUmmaN,
+                (long long)inter);
+  if (experts < 1 || experts > fc1::kMaxExperts)
+    return fail(SITU_ERR_UNSUPPORTED, "experts must be in [1, %d], got %lld", fc1::kMaxExperts, (long long)experts);
+  if (tokens > INT32_MAX || experts * inter > INT32_MAX || hidden > INT32_MAX)
+    return fail(SITU_ERR_UNSUPPORTED, "sizes exceed the 32-bit tensor-map coordinates");
+  if (dout_row_stride < hidden || w2t_row_stride < hidden || gate_up_row_stride < 2 * inter ||
+      d_gate_up_row_stride < 2 * inter)
+    return fail(SITU_ERR_INVALID_ARG, "a row stride is shorter than its row");
+  if (rw_mode == SITU_RW_ROW && (rw_stride < 0 || (d_rw != nullptr && d_rw_stride < 1)))
+    return fail(SITU_ERR_INVALID_ARG, "rw_stride < 0 or d_rw_stride < 1");
+  const bool want_drw = d_rw != nullptr;
+  const size_t ws_needed = situ_glu_fc2_dgrad_workspace_bytes(tokens, inter, want_drw ? 1 : 0);
+  if (tokens == 0) return SITU_OK;
+  if (dout == nullptr || w2t == nullptr || offsets == nullptr || gate_up == nullptr || d_gate_up == nullptr ||
+      (rw_mode == SITU_RW_ROW && rw == nullptr))
+    return fail(SITU_ERR_INVALID_ARG, "dout, w2t, offsets, gate_up, d_gate_up or rw is NULL");
+  if (!span_fits(tokens, dout_row_stride, hidden, 2) || !span_fits(experts * inter, w2t_row_stride, hidden, 2) ||
+      !span_fits(tokens, gate_up_row_stride, 2 * inter, 2) || !span_fits(tokens, d_gate_up_row_stride, 2 * inter, 2) ||
+      (rw_mode == SITU_RW_ROW && !span_fits(tokens, rw_stride, 1, elem_size(rw_dtype))) ||
+      (want_drw && !span_fits(tokens, d_rw_stride, 1, elem_size(rw_dtype))))
+    return fail(SITU_ERR_INVALID_ARG, "tensor extent overflows int64");
+  if (!aligned(dout, 16) || !aligned(w2t, 16) || !aligned(gate_up, 16) || !aligned(d_gate_up, 16) ||
+      (dout_row_stride * 2) % 16 != 0 || (w2t_row_stride * 2) % 16 != 0 || (gate_up_row_stride * 2) % 16 != 0 ||
+      (d_gate_up_row_stride * 2) % 16 != 0 || !aligned(offsets, 8) ||
+      (rw_mode == SITU_RW_ROW && !aligned(rw, elem_size(rw_dtype))) ||
+      (want_drw && !aligned(d_rw, elem_size(rw_dtype))))
+    return fail(SITU_ERR_MISALIGNED, "a base address or row pitch is misaligned");
+  if (ws_needed > 0 && (workspace == nullptr || workspace_bytes < ws_needed || !aligned(workspace, 16)))
+    return fail(SITU_ERR_INVALID_ARG, "workspace needs %zu bytes (16-byte aligned), got %zu", ws_needed,
+                workspace == nullptr ? (size_t)0 : workspace_bytes);
+  const Span s_dgu = matrix_span(d_gate_up, tokens, d_gate_up_row_stride, 2 * inter, 2);
+  const Span s_ws = {reinterpret_cast<uintptr_t>(workspace), reinterpret_cast<uintptr_t>(workspace) + ws_needed};
+  const Span s_off = {reinterpret_cast<uintptr_t>(offsets),
+                      reinterpret_cast<uintptr_t>(offsets) + static_cast<uintptr_t>(experts + 1) * 8};
+  const Span ins[] = {matrix_span(dout, tokens, dout_row_stride, hidden, 2),
+                      matrix_span(w2t, experts * inter, w2t_row_stride, hidden, 2),
+                      matrix_span(gate_up, tokens, gate_up_row_stride, 2 * inter, 2), s_off,
+                      weight_span(rw, rw_mode, tokens, rw_stride, inter, elem_size(rw_dtype))};
+  const Span s_drw = want_drw ? weight_span(d_rw, SITU_RW_ROW, tokens, d_rw_stride, inter, elem_size(rw_dtype))
+                              : Span{0, 0};
+  for (const Span& in : ins)
+    if (overlap(s_dgu, in) || overlap(s_drw, in) || (ws_needed && overlap(s_ws, in)))
+      return fail(SITU_ERR_INVALID_ARG, "an output or the workspace overlaps an input");
+  if (overlap(s_dgu, s_drw) || (ws_needed && (overlap(s_ws, s_dgu) || overlap(s_ws, s_drw))))
+    return fail(SITU_ERR_INVALID_ARG, "outputs or the workspace overlap each other");
+
+  fc1::Args a{};
+  a.offsets = offsets;
+  a.experts = static_cast<int>(experts);
+  a.tokens = tokens;
+  a.hidden = static_cast<int>(hidden);
+  a.inter = static_cast<int>(inter);
+  a.rw = {rw, rw_stride, static_cast<int>(rw_mode), (rw_mode != SITU_RW_NONE && rw_dtype == SITU_DTYPE_BF16) ? 1 : 0};
+  a.y = static_cast<char*>(d_gate_up);
+  a.y_pitch = d_gate_up_row_stride * 2;
+  a.gate_up = static_cast<const char*>(gate_up);
+  a.gu_pitch = gate_up_row_stride * 2;
+  a.partials = want_drw ? static_cast<float*>(workspace) : nullptr;
+  int gate = kGateGeneric;
+  fill_coeffs(beta, has_linear_beta, linear_beta, &a.c, &gate);
+
+  CUtensorMap ma, mb;
+  situ_status_t st = bf16_tile_map(&ma, dout, hidden, tokens, dout_row_stride);
+  if (st != SITU_OK) return st;
+  st = bf16_tile_map(&mb, w2t, hidden, experts * inter, w2t_row_stride);
+  if (st != SITU_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_fused(pick_fused<fc1::Fc2Epilogue>(gate, has_linear_beta != 0), ma, mb, a, experts, s,
+                    "situ_glu_fc2_dgrad_bwd");
+  if (st != SITU_OK || !want_drw) return st;
   int sms = 0;
   st = device_sm_count(&sms);
   if (st != SITU_OK) return st;
-  int grid = sms;
-  const int cap = g_max_ctas.load(std::memory_order_relaxed);
-  if (cap > 0 && grid > cap) grid = cap;
-  k<<<grid, fc1::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(mx, mw, a);
-  return check_launch("situ_glu_fc1_fwd");
+  situ_fc2_dw_finalize_kernel<<<sms, 256, 0, s>>>(a.partials, static_cast<int>(inter / fc1::kUmmaN), offsets,
+                                                  static_cast<int>(experts), tokens, d_rw, d_rw_stride,
+                                                  a.rw.bf16);
+  return check_launch("situ_glu_fc2_dgrad_bwd (d_rw)");
 }
 
 

@@ -312,6 +312,59 @@ def situ_glu_fc1_fwd(x: torch.Tensor, w1: torch.Tensor, offsets: torch.Tensor, r
     return out
 
 
+def situ_glu_fc2_dgrad_bwd(dout: torch.Tensor, w2t: torch.Tensor, offsets: torch.Tensor, gate_up: torch.Tensor,
+                           routing_weights=None, beta: float = DEFAULT_BETA,
+                           linear_beta: float | None = DEFAULT_LINEAR_BETA, want_drw: bool = True,
+                           d_gate_up=None, d_rw=None, workspace=None, stream=None):
+    """FC2 data gradient fused with the SiTU-GLU backward.  dout: bf16 [T, H];
+    w2t: bf16 [E, I, H] (or [E * I, H]) -- FC2's weight transposed per expert;
+    offsets: int64 [E + 1] on dout's device; gate_up: the saved bf16 [T, 2I];
+    routing_weights: per-row [T, 1] / [T] or None.  Returns (d_gate_up [T, 2I],
+    d_routing_weights shaped like routing_weights, or None)."""
+    _check_beta(beta, linear_beta)
+    for t, name in ((dout, "dout"), (w2t, "w2t"), (gate_up, "gate_up")):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16")
+    if dout.dim() != 2 or gate_up.dim() != 2:
+        raise ValueError("dout and gate_up must be 2-D")
+    tokens, hidden = dout.shape
+    inter = gate_up.shape[1] // 2
+    experts = offsets.numel() - 1
+    w2 = w2t.reshape(-1, w2t.shape[-1])
+    if w2.shape != (experts * inter, hidden):
+        raise ValueError(f"w2t {tuple(w2t.shape)} does not match {experts} experts x {inter} x {hidden}")
+    dout = dout if dout.stride(1) == 1 else dout.contiguous()
+    w2 = w2 if w2.stride(1) == 1 else w2.contiguous()
+    gate_up = gate_up if gate_up.stride(1) == 1 else gate_up.contiguous()
+    mode, rw, rw_stride = routing_mode((tokens,), inter, routing_weights)
+    if mode not in (abi.SITU_RW_ROW, abi.SITU_RW_NONE):
+        raise NotImplementedError("situ_glu_fc2_dgrad_bwd takes per-row or no routing weights")
+    rw_dtype = _dtype_code(rw, "routing_weights") if rw is not None else abi.SITU_DTYPE_F32
+    want = bool(want_drw) and rw is not None
+    if d_gate_up is None:
+        d_gate_up = torch.empty(tokens, 2 * inter, dtype=torch.bfloat16, device=dout.device)
+    d_rw_flat = None
+    if want:
+        if d_rw is None:
+            d_rw = torch.empty(routing_weights.shape, dtype=routing_weights.dtype, device=dout.device)
+        d_rw_flat = d_rw.view(-1)
+    ws = abi.situ_glu_fc2_dgrad_workspace_bytes(tokens, inter, int(want))
+    if ws and (workspace is None or workspace.numel() * workspace.element_size() < ws):
+        workspace = torch.empty(ws, dtype=torch.uint8, device=dout.device)
+    st = abi.situ_glu_fc2_dgrad_bwd(dout.data_ptr(), tokens, hidden, dout.stride(0) if tokens > 1 else hidden,
+                                    w2.data_ptr(), experts, inter, w2.stride(0), offsets.data_ptr(),
+                                    gate_up.data_ptr(), gate_up.stride(0) if tokens > 1 else 2 * inter,
+                                    rw.data_ptr() if rw is not None else None, rw_dtype, mode, rw_stride,
+                                    float(beta), int(linear_beta is not None),
+                                    float(linear_beta) if linear_beta is not None else 0.0,
+                                    d_gate_up.data_ptr(), d_gate_up.stride(0) if tokens > 1 else 2 * inter,
+                                    d_rw_flat.data_ptr() if d_rw_flat is not None else None,
+                                    d_rw_flat.stride(0) if d_rw_flat is not None and d_rw_flat.numel() > 1 else 1,
+                                    workspace.data_ptr() if ws else None, ws, _stream_handle(stream))
+    abi.check(st, "situ_glu_fc2_dgrad_bwd")
+    return d_gate_up, (d_rw if want else None)
+
+
 _DTYPE_OF = {torch.bfloat16: abi.SITU_DTYPE_BF16, torch.float32: abi.SITU_DTYPE_F32}
 
 

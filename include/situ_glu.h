@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define SITU_GLU_ABI_VERSION 5
+#define SITU_GLU_ABI_VERSION 6
 
 typedef enum situ_status {
   SITU_OK = 0,
@@ -264,6 +264,48 @@ situ_status_t situ_glu_fc1_fwd(const void *x, int64_t tokens, int64_t hidden, in
                                double beta, int has_linear_beta, double linear_beta,
                                void *y, int64_t y_row_stride,
                                void *stream);
+
+/* ---- FC2 data gradient + SiTU-GLU backward --------------------------------------
+ * The backward of the fused grouped MLP at the activation (Megatron-LM PR
+ * #6673, "Test results": the fused path's backward with a dSiTU correction):
+ * FC2's data gradient is the activation's upstream gradient, so for token row
+ * r of expert e
+ *   dY[r, i]            = sum_h dout[r, h] W2_e[h, i]       (fp32 on the tensor cores, never written)
+ *   d_gate_up[r, i]     = dY w[r] T_u(U) T_g'(G)            (as situ_glu_bwd with grad_out = dY)
+ *   d_gate_up[r, I + i] = dY w[r] T_g(G) T_u'(U)
+ *   d_rw[r]             = sum_i dY T_g(G) T_u(U)
+ * with G, U the halves of the saved gate_up row.
+ *
+ *   dout        bf16 [tokens, >= hidden], row pitch dout_row_stride
+ *   w2t         bf16 [experts * inter, >= hidden]: FC2's weight W2_e [hidden,
+ *               inter] TRANSPOSED (row e * inter + i holds W2_e[:, i])
+ *   offsets     DEVICE int64 [experts + 1], as for situ_glu_fc1_fwd
+ *   gate_up     bf16 [tokens, >= 2 inter], the forward's saved FC1 output
+ *   rw, rw_dtype, rw_stride  per-row routing weights (SITU_RW_ROW) or none
+ *               (SITU_RW_NONE: rw and d_rw NULL); other modes SITU_ERR_UNSUPPORTED
+ *   d_gate_up   bf16 [tokens, >= 2 inter]; d_rw (rw_dtype, stride d_rw_stride)
+ *               or NULL when not wanted
+ *   workspace   >= situ_glu_fc2_dgrad_workspace_bytes() bytes (per-row,
+ *               per-256-column-tile d_rw partials, added in tile order)
+ * hidden a multiple of 64, inter of 256, experts in [1, 1024]; alignment and
+ * offsets rules as for situ_glu_fc1_fwd.  Rows outside every expert are not
+ * written.
+ */
+situ_status_t situ_glu_fc2_dgrad_bwd(const void *dout, int64_t tokens, int64_t hidden, int64_t dout_row_stride,
+                                     const void *w2t, int64_t experts, int64_t inter, int64_t w2t_row_stride,
+                                     const int64_t *offsets,
+                                     const void *gate_up, int64_t gate_up_row_stride,
+                                     const void *rw, situ_dtype_t rw_dtype, situ_rw_mode_t rw_mode,
+                                     int64_t rw_stride,
+                                     double beta, int has_linear_beta, double linear_beta,
+                                     void *d_gate_up, int64_t d_gate_up_row_stride,
+                                     void *d_rw, int64_t d_rw_stride,
+                                     void *workspace, size_t workspace_bytes,
+                                     void *stream);
+
+/* Bytes of workspace situ_glu_fc2_dgrad_bwd needs: tokens * (inter / 256) * 4
+ * rounded up to 256 when want_drw != 0, else 0. */
+size_t situ_glu_fc2_dgrad_workspace_bytes(int64_t tokens, int64_t inter, int want_drw);
 
 /* ---- Attention-residual mixing core -------------------------------------------
  * NeMo AutoModel API, kimi_k3.situ, `_attn_res_core` ("fp32 attention-residual

@@ -58,7 +58,7 @@ def test_binding_covers_the_header_exactly():
 
 
 def test_version_and_status_strings(native_lib_path):
-    assert abi.situ_glu_abi_version() == abi.ABI_VERSION == 5
+    assert abi.situ_glu_abi_version() == abi.ABI_VERSION == 6
     assert abi.situ_glu_status_string(OK) == "SITU_OK"
     assert abi.situ_glu_status_string(MISAL) == "SITU_ERR_MISALIGNED"
     assert abi.situ_glu_status_string(99) == "SITU_ERR_UNKNOWN"
@@ -395,3 +395,44 @@ def test_attn_res_argument_errors(name, kw, want, native_lib_path):
 def test_attn_res_zero_tokens_is_a_no_op(native_lib_path):
     assert attn_res(tokens=0, blocks=None, prefix=None, nblocks=0) == UNSUP  # still no source
     assert attn_res(tokens=0, blocks=None, out=None) == OK
+
+
+# ---- FC2 data gradient + SiTU-GLU backward: argument checks ---------------------------
+
+DOP, W2P, GUP, DGUP, DRWP, WSP = (0x70000000 + 0x01000000 * k for k in range(6))
+
+
+def fc2(**kw):
+    a = dict(dout=DOP, tokens=256, hidden=128, dout_row_stride=128, w2t=W2P, experts=2, inter=256,
+             w2t_row_stride=128, offsets=OFFP, gate_up=GUP, gate_up_row_stride=512, rw=RW, rw_dtype=F32,
+             rw_mode=ROW, rw_stride=1, beta=4.0, has_linear_beta=1, linear_beta=25.0, d_gate_up=DGUP,
+             d_gate_up_row_stride=512, d_rw=DRWP, d_rw_stride=1, workspace=WSP, workspace_bytes=1 << 20,
+             stream=None)
+    a.update(kw)
+    return abi.situ_glu_fc2_dgrad_bwd(**a)
+
+
+FC2_CASES = [
+    ("inter not a multiple of 256", dict(inter=128, gate_up_row_stride=256, d_gate_up_row_stride=256), UNSUP),
+    ("hidden not a multiple of 64", dict(hidden=96, dout_row_stride=96, w2t_row_stride=96), UNSUP),
+    ("broadcast weight", dict(rw_mode=SCALAR), UNSUP),
+    ("d_rw with no weights", dict(rw_mode=NONE, rw=None), INVALID),
+    ("workspace missing", dict(workspace=None, workspace_bytes=0), INVALID),
+    ("workspace short", dict(workspace_bytes=16), INVALID),
+    ("gate_up stride short", dict(gate_up_row_stride=256), INVALID),
+    ("d_gate_up overlaps gate_up", dict(d_gate_up=GUP + 1024), INVALID),
+    ("workspace overlaps dout", dict(workspace=DOP + 64), INVALID),
+    ("dout misaligned", dict(dout=DOP + 4), MISAL),
+    ("gate_up NULL", dict(gate_up=None), INVALID),
+]
+
+
+@pytest.mark.parametrize("name,kw,want", FC2_CASES, ids=[c[0] for c in FC2_CASES])
+def test_fc2_argument_errors(name, kw, want, native_lib_path):
+    assert fc2(**kw) == want, abi.situ_glu_last_error()
+
+
+def test_fc2_workspace_query(native_lib_path):
+    assert abi.situ_glu_fc2_dgrad_workspace_bytes(1000, 2048, 1) == (1000 * 8 * 4 + 255) // 256 * 256
+    assert abi.situ_glu_fc2_dgrad_workspace_bytes(1000, 2048, 0) == 0
+    assert abi.situ_glu_fc2_dgrad_workspace_bytes(0, 2048, 1) == 0

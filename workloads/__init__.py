@@ -34,6 +34,9 @@ TENSOR_FC1_W = 7
 TENSOR_FC1_SPLIT = 8
 TENSOR_AR_VALUES = 9
 TENSOR_AR_WEIGHTS = 10
+TENSOR_FC2_DOUT = 11
+TENSOR_FC2_W = 12
+TENSOR_FC2_GU = 13
 
 
 @dataclass(frozen=True)
@@ -325,3 +328,33 @@ def attn_res_inputs(tokens: int, blocks: int, hidden: int, seed: int, dtype: str
     norm_w = (1.0 + 0.1 * rng.standard_normal(hidden)).astype(np.float32)
     proj_w = (rng.standard_normal(hidden) / np.sqrt(hidden)).astype(np.float32)
     return {"blocks": blk, "prefix": pre, "norm_weight": norm_w, "proj_weight": proj_w}
+
+
+# ---- FC2 data-gradient inputs ---------------------------------------------------------
+
+def fc2_inputs(tokens: int, hidden: int, inter: int, experts: int, seed: int):
+    """dout bf16 [T, H] ~ N(0, 1); w2t bf16 [E * I, H] ~ N(0, 1 / sqrt(H)) (FC2's
+    weight transposed per expert, so dY ~ N(0, 1)); gate_up bf16 [T, 2I] ~
+    N(0, 3) (the saved FC1 output); offsets as expert_offsets; per-row
+    weights U(0, 1).  64-row blocks."""
+    def block_fill(out, rows, cols, tensor, std):
+        def fill(b):
+            r0 = b * BLOCK_ROWS
+            n = min(BLOCK_ROWS, rows - r0)
+            v = _rng(seed, tensor, b).standard_normal((BLOCK_ROWS, cols))[:n] * std
+            out[r0:r0 + n] = f32_to_bf16_bits(v.astype(np.float32))
+        _fill_blocks(rows, fill)
+
+    dout = np.empty((tokens, hidden), dtype=np.uint16)
+    block_fill(dout, tokens, hidden, TENSOR_FC2_DOUT, 1.0)
+    w2t = np.empty((experts * inter, hidden), dtype=np.uint16)
+    block_fill(w2t, experts * inter, hidden, TENSOR_FC2_W, 1.0 / np.sqrt(hidden))
+    gu = np.empty((tokens, 2 * inter), dtype=np.uint16)
+    block_fill(gu, tokens, 2 * inter, TENSOR_FC2_GU, 3.0)
+    rw = np.empty(tokens, dtype=np.float32)
+    for b in range((tokens + BLOCK_ROWS - 1) // BLOCK_ROWS):
+        r0 = b * BLOCK_ROWS
+        n = min(BLOCK_ROWS, tokens - r0)
+        rw[r0:r0 + n] = _rng(seed, TENSOR_ROUTING, b).random(BLOCK_ROWS)[:n].astype(np.float32)
+    return {"dout": dout, "w2t": w2t, "gate_up": gu, "offsets": expert_offsets(tokens, experts, seed),
+            "routing_weights": rw}
