@@ -17,7 +17,9 @@ bytes follow the form (weights read, weight gradients written, one byte per
 code plus one per 32 codes).  --variant fc1 times the fused FC1 grouped GEMM
 + SiTU-GLU forward on the routed-MoE rows (hidden 7168, 8 local experts) in
 TFLOP/s against the tensor-core peak, with the unfused cuBLAS GEMMs +
-SiTU-GLU kernel timed beside it.  --variant attn_res times the
+SiTU-GLU kernel timed beside it; --variant fc2 the fused FC2 data gradient
++ SiTU-GLU backward on the same rows (against cuBLAS GEMMs + situ_glu_bwd).
+--variant attn_res times the
 attention-residual mixing core (16384 tokens, 8 stored sums + the current
 sum, hidden 7168, bf16) in GB/s of algorithmic bytes (every source value read
 once, the output written once).
@@ -50,7 +52,8 @@ METRIC = "SiTU-GLU fwd/bwd achieved HBM GB/s (% of B200 peak) and rows/s"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
-KERNEL_SOURCE = os.path.join(ROOT, "ffn_gated_activation_b200", "csrc", "situ_glu.cu")
+KERNEL_SOURCES = [os.path.join(ROOT, "ffn_gated_activation_b200", "csrc", n)
+                  for n in ("situ_glu.cu", "situ_fused_gemm.cuh")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 
 
@@ -66,7 +69,7 @@ def parse_args(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-oracle sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--variant", choices=["row", "col", "full", "mxfp8", "fc1", "attn_res"], default="row",
+    p.add_argument("--variant", choices=["row", "col", "full", "mxfp8", "fc1", "fc2", "attn_res"], default="row",
                    help="routing-weight form or output format timed (default: per-row weights)")
     p.add_argument("--flush", choices=["auto", "always", "never"], default="auto",
                    help="flush L2 before every step (auto: when the inputs fit in L2)")
@@ -85,8 +88,13 @@ def measured_peak():
 
 
 def source_digest() -> str:
-    with open(KERNEL_SOURCE, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
+    """sha256 over the kernel sources, in order: a recorded ncu traffic figure
+    is used only while the kernels are the ones it was taken on."""
+    h = hashlib.sha256()
+    for path in KERNEL_SOURCES:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def recorded_traffic(kernel: str, workload_name: str):
@@ -398,11 +406,12 @@ def run_ours_attn_res(args, dev, world, rank, local, barrier):
                 "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": ar_config(f"inputs {ar_bytes() / 1e9:.1f} GB exceed the 126 MB L2; no flush", world),
-                "kernels": {"situ_attn_res_kernel": {"us": ms * 1e3, "GB/s": gbs, "frac_of_measured_copy": gbs / peak}},
+                "kernels": {"situ_attn_res_staged_kernel": {"us": ms * 1e3, "GB/s": gbs,
+                                                            "frac_of_measured_copy": gbs / peak}},
                 "torch_eager_fp32_chain": {"ms": torch_ms, "GB/s": ar_bytes() / (torch_ms / 1e3) / 1e9},
-                "roofline": {"bound": "hbm", "kernel": "situ_attn_res_kernel", "achieved": gbs, "peak": peak,
+                "roofline": {"bound": "hbm", "kernel": "situ_attn_res_staged_kernel", "achieved": gbs, "peak": peak,
                              "unit": "GB/s", "frac": gbs / peak, "peak_source": f"{peak_src} copy bandwidth",
-                             "traffic": recorded_traffic("situ_attn_res_kernel", "attn_res")},
+                             "traffic": recorded_traffic("situ_attn_res_staged_kernel", "attn_res")},
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K, "clocks": clocks.summary(),
                 "device_status": pkg.abi.situ_glu_device_status(0), "device": torch.cuda.get_device_name(dev)}
         print(json.dumps(line), flush=True)
@@ -480,6 +489,8 @@ def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.variant == "fc1":
         return run_reference_fc1(args, wl, beta, world)
+    if args.variant == "fc2":
+        return run_reference_fc2(args, wl, beta, world)
     if args.variant == "attn_res":
         return run_reference_attn_res(args, world)
     rows_per_step = max(1, min(wl.tokens, (1 << 17) // wl.inter))
@@ -567,6 +578,153 @@ def fc1_config(wl, beta, l2_note, world):
         "l2": l2_note,
         "parallelism": f"replicas x{world} (weak scaling; no collective)",
     }
+
+
+FC2_METRIC = "fused FC2 data-gradient GEMM + SiTU-GLU backward TFLOP/s"
+
+
+def fc2_flops(wl) -> float:
+    return 2.0 * wl.tokens * FC1_HIDDEN * wl.inter
+
+
+def run_reference_fc2(args, wl, beta, world):
+    d = workloads.fc2_inputs(wl.tokens, FC1_HIDDEN, wl.inter, FC1_EXPERTS, wl.seed)
+    import oracle
+    o = oracle.load()
+    rows = np.arange(4, dtype=np.int64)
+
+    def step():
+        o.fc2_dgrad(d["dout"], d["w2t"], d["offsets"], d["gate_up"], d["routing_weights"], beta, wl.linear_beta,
+                    rows=rows)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = 2.0 * FC1_HIDDEN * wl.inter * rows.size * args.steps / dt / 1e12
+    cfg = fc1_config(wl, beta, "n/a (host)", 1)
+    cfg["name"] = f"{wl.name}/fc2"
+    line = {"impl": "reference", "metric": FC2_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": cfg,
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{rows.size} rows per step, {args.steps} steps, single-threaded fp64"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours_fc2(args, wl, beta, dev, world, rank, local, barrier):
+    import torch
+    import torch.distributed as dist
+
+    import ffn_gated_activation_b200 as pkg
+
+    lb = wl.linear_beta
+    T, I, H, E = wl.tokens, wl.inter, FC1_HIDDEN, FC1_EXPERTS
+    d = workloads.fc2_inputs(T, H, I, E, wl.seed)
+    d["offsets"] = workloads.expert_offsets(T, E, wl.seed, skew=2.0)
+
+    def up(a):
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.to(dev)
+
+    dout, w2t, gu = up(d["dout"]), up(d["w2t"]), up(d["gate_up"])
+    off = torch.from_numpy(d["offsets"]).to(dev)
+    rw = up(d["routing_weights"]).reshape(T, 1)
+    dgu = torch.empty(T, 2 * I, dtype=torch.bfloat16, device=dev)
+    d_rw = torch.empty(T, 1, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(1, pkg.abi.situ_glu_fc2_dgrad_workspace_bytes(T, I, 1)), dtype=torch.uint8, device=dev)
+    flops = fc2_flops(wl)
+    stream = torch.cuda.current_stream(dev)
+
+    def bwd():
+        pkg.situ_glu_fc2_dgrad_bwd(dout, w2t, off, gu, rw, beta, lb, d_gate_up=dgu, d_rw=d_rw, workspace=ws)
+
+    for _ in range(max(3, args.warmup)):
+        bwd()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for a, b in ev:
+        a.record(stream)
+        bwd()
+        b.record(stream)
+    torch.cuda.synchronize()
+    clocks.stop()
+    barrier()
+    t = torch.tensor([sum(a.elapsed_time(b) for a, b in ev)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = t.item() / K
+    tflops = flops / (ms / 1e3) / 1e12
+    peak, peak_src = measured_tensor_peak()
+
+    # unfused: cuBLAS dY = dOut W2_e per expert, then situ_glu_bwd
+    offs = d["offsets"]
+    dy = torch.empty(T, I, dtype=torch.bfloat16, device=dev)
+    w2e = w2t.view(E, I, H)
+
+    def unfused():
+        for e in range(E):
+            a0, a1 = int(offs[e]), int(offs[e + 1])
+            if a1 > a0:
+                torch.matmul(dout[a0:a1], w2e[e].t(), out=dy[a0:a1])
+        pkg.situ_glu_bwd(gu, rw, dy, beta, lb, d_gate_up=dgu, d_rw=d_rw)
+
+    for _ in range(3):
+        unfused()
+    torch.cuda.synchronize()
+    ue = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(max(3, K // 2))]
+    for a, b in ue:
+        a.record(stream)
+        unfused()
+        b.record(stream)
+    torch.cuda.synchronize()
+    unfused_ms = statistics.median([a.elapsed_time(b) for a, b in ue])
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        o = oracle.load()
+        done, t0 = 0, time.perf_counter()
+        while done < T and time.perf_counter() - t0 < args.cpu_seconds:
+            rows = np.arange(done, min(T, done + 8), dtype=np.int64)
+            o.fc2_dgrad(d["dout"], d["w2t"], d["offsets"], d["gate_up"], d["routing_weights"], beta, lb, rows=rows)
+            done += rows.size
+        secs = time.perf_counter() - t0
+        cpu = {"value": 2.0 * H * I * done / secs / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+               "sample": f"first {done} of {T} rows, {secs:.1f} s, single-threaded fp64 FC2-dgrad oracle"}
+    if rank == 0:
+        cfg = fc1_config(wl, beta, "inputs 1.1 GB exceed the 126 MB L2; no flush", world)
+        cfg["name"] = f"{wl.name}/fc2"
+        cfg["workload"] = (f"fused FC2 data gradient: dOut bf16 [{T}, {H}] ~ N(0,1), W2 transposed bf16 "
+                           f"[{E} x {I}, {H}] ~ N(0, 1/sqrt({H})), saved gate_up bf16 [{T}, {2 * I}] ~ N(0,3), "
+                           f"{E} experts (Dirichlet(2) split), d_gate_up bf16, d_w fp32")
+        line = {"metric": FC2_METRIC, "value": tflops * world, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+                "kernels": {"fc1::situ_fused_gemm_kernel<Fc2Epilogue>": {"us": ms * 1e3, "TFLOP/s": tflops,
+                                                                         "frac_of_measured_bf16": tflops / peak}},
+                "unfused": {"ms": unfused_ms, "TFLOP/s": flops / (unfused_ms / 1e3) / 1e12,
+                            "what": "cuBLAS bf16 GEMM per expert (torch.matmul) into dY, then situ_glu_bwd"},
+                "roofline": {"bound": "tensor", "kernel": "fc1::situ_fused_gemm_kernel<Fc2Epilogue>", "achieved": tflops,
+                             "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
+                             "peak_source": f"{peak_src} cuBLAS bf16 (burst)",
+                             "traffic": recorded_traffic("situ_fused_gemm_kernel<Fc2Epilogue>", f"{wl.name}/fc2")},
+                "cpu_baseline": cpu, "e2e": None, "gpu_launches": 2 * K, "clocks": clocks.summary(),
+                "device_status": pkg.abi.situ_glu_device_status(0), "device": torch.cuda.get_device_name(dev)}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
 
 
 def run_ours_fc1(args, wl, beta, dev, world, rank, local, barrier):
@@ -685,12 +843,14 @@ def run_ours_fc1(args, wl, beta, dev, world, rank, local, barrier):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": fc1_config(wl, beta, "inputs 940 MB exceed the 126 MB L2; no flush", world),
-            "kernels": {"fc1::situ_fc1_kernel": {"us": ms * 1e3, "TFLOP/s": tflops, "frac_of_measured_bf16": tflops / peak}},
+            "kernels": {"fc1::situ_fused_gemm_kernel<Fc1Epilogue>": {"us": ms * 1e3, "TFLOP/s": tflops,
+                                                                     "frac_of_measured_bf16": tflops / peak}},
             "unfused": {"ms": unfused_ms, "TFLOP/s": flops / (unfused_ms / 1e3) / 1e12,
                         "what": "cuBLAS bf16 GEMM per expert (torch.matmul) into gate_up, then situ_glu_fwd"},
-            "roofline": {"bound": "tensor", "kernel": "fc1::situ_fc1_kernel", "achieved": tflops, "peak": peak,
+            "roofline": {"bound": "tensor", "kernel": "fc1::situ_fused_gemm_kernel<Fc1Epilogue>", "achieved": tflops,
+                         "peak": peak,
                          "unit": "TFLOP/s", "frac": tflops / peak, "peak_source": f"{peak_src} cuBLAS bf16 (burst)",
-                         "traffic": recorded_traffic("situ_fc1_kernel", f"{wl.name}/fc1")},
+                         "traffic": recorded_traffic("situ_fused_gemm_kernel<Fc1Epilogue>", f"{wl.name}/fc1")},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": K,
@@ -733,6 +893,8 @@ def run_ours(args):
     beta = args.beta if args.beta is not None else wl.betas[0]
     if args.variant == "fc1":
         return run_ours_fc1(args, wl, beta, dev, world, rank, local, barrier)
+    if args.variant == "fc2":
+        return run_ours_fc2(args, wl, beta, dev, world, rank, local, barrier)
     if args.variant == "attn_res":
         return run_ours_attn_res(args, dev, world, rank, local, barrier)
     lb = wl.linear_beta
