@@ -144,6 +144,14 @@ class Oracle:
         lib.situ_oracle_mx_scale_exp.restype = _INT
         lib.situ_oracle_mxfp8_quantize.argtypes = [_VP, _I64, _I64, _I64, _INT, _VP, _VP]
         lib.situ_oracle_mxfp8_quantize.restype = _INT
+        lib.situ_oracle_e2m1_encode.argtypes = [_DBL]
+        lib.situ_oracle_e2m1_encode.restype = _INT
+        lib.situ_oracle_e2m1_decode.argtypes = [_INT]
+        lib.situ_oracle_e2m1_decode.restype = _DBL
+        lib.situ_oracle_nvfp4_tensor_scale.argtypes = [_DBL]
+        lib.situ_oracle_nvfp4_tensor_scale.restype = _DBL
+        lib.situ_oracle_nvfp4_quantize.argtypes = [_VP, _I64, _I64, _I64, _DBL, _VP, _VP]
+        lib.situ_oracle_nvfp4_quantize.restype = _INT
         lib.situ_oracle_fc1_fwd.argtypes = [_VP, _I64, _I64, _VP, _I64, _I64, _VP, _I64, _VP, _I64, _VP,
                                             _DBL, _INT, _DBL, _VP, _VP, _VP]
         lib.situ_oracle_fc1_fwd.restype = _INT
@@ -302,6 +310,36 @@ class Oracle:
             raise ValueError("oracle mxfp8_quantize: columns must be a multiple of 32")
         return codes, scales
 
+
+    # -- NVFP4 (mx_oracle.c) ----------------------------------------------------
+
+    def e2m1_encode(self, x) -> np.ndarray:
+        x = np.asarray(x, dtype=np.float64)
+        f = self._lib.situ_oracle_e2m1_encode
+        return np.array([f(float(v)) for v in x.reshape(-1)], dtype=np.uint8).reshape(x.shape)
+
+    def e2m1_decode(self, codes) -> np.ndarray:
+        c = np.asarray(codes, dtype=np.uint8)
+        f = self._lib.situ_oracle_e2m1_decode
+        return np.array([f(int(v)) for v in c.reshape(-1)], dtype=np.float64).reshape(c.shape)
+
+    def nvfp4_tensor_scale(self, amax: float) -> float:
+        return self._lib.situ_oracle_nvfp4_tensor_scale(float(amax))
+
+    def nvfp4_quantize(self, v, s_enc=None):
+        """(codes [R, C] one 4-bit code per byte, block scale codes [R, C / 16]
+        E4M3, s_enc) of the fp64 matrix v; s_enc defaults to the tensor's own."""
+        v = np.ascontiguousarray(np.asarray(v, dtype=np.float64))
+        if s_enc is None:
+            fin = v[np.isfinite(v)]
+            s_enc = self.nvfp4_tensor_scale(float(np.abs(fin).max()) if fin.size else 0.0)
+        rows, cols = v.shape
+        codes = np.empty((rows, cols), dtype=np.uint8)
+        scales = np.empty((rows, cols // 16), dtype=np.uint8)
+        rc = self._lib.situ_oracle_nvfp4_quantize(_ptr(v), rows, cols, cols, float(s_enc), _ptr(codes), _ptr(scales))
+        if rc != 0:
+            raise ValueError("oracle nvfp4_quantize: columns must be a multiple of 16")
+        return codes, scales, s_enc
 
     # -- FC1 followed by SiTU-GLU (fc1_oracle.c) ------------------------------
 

@@ -163,3 +163,91 @@ int situ_oracle_mxfp8_quantize(const double *v, int64_t rows, int64_t cols, int6
 void situ_oracle_e4m3_encode_n(const double *x, int64_t n, uint8_t *codes) {
   for (int64_t i = 0; i < n; ++i) codes[i] = (uint8_t)situ_oracle_e4m3_encode(x[i]);
 }
+
+/* ---- NVFP4 --------------------------------------------------------------
+ * The NVFP4 recipe named beside MXFP8 (Megatron-LM PR #6673, "Test results";
+ * the format is NVIDIA's public NVFP4 definition, not on the pages):
+ *   * elements are FP4 E2M1 codes: sign, 2 exponent bits (bias 1), 1 mantissa
+ *     bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6; no infinities or NaN;
+ *   * every 16 consecutive elements of a row share one FP8 E4M3 scale s_b;
+ *   * the tensor has one fp32 scale: with A = max |V| over the tensor,
+ *     S_enc = 448 * 6 / A (S_enc = 1 when A = 0), and the decoded value of a
+ *     code q in block b is q * s_b / S_enc.
+ * Conversion, read plainly in exact arithmetic with one rounding per stored
+ * number: s_b = E4M3(amax_b * S_enc / 6) (nearest even, clamped to 448);
+ * q_i = E2M1(V_i * S_enc / s_b) (nearest even, clamped to +-6); a block whose
+ * scale code is zero gets zero codes.  A NaN or infinite value gives the NaN
+ * block scale (0x7F) and zero codes (E2M1 has no NaN). */
+
+#define E2M1_MAX 6.0
+
+/* E2M1 code (4 bits: sign << 3 | magnitude code) of x, nearest even, clamped to 6. */
+int situ_oracle_e2m1_encode(double x) {
+  static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  if (isnan(x)) return 0;
+  const int s = signbit(x) ? 8 : 0;
+  double a = fabs(x);
+  if (a >= E2M1_MAX) return s | 7;
+  int best = 0;
+  for (int k = 1; k < 8; ++k) {
+    const double dk = fabs(a - mag[k]), db = fabs(a - mag[best]);
+#if SITU_ORACLE_MUTANT == 32
+    if (dk <= db) best = k; /* planted: ties to the larger magnitude */
+#else
+    if (dk < db || (dk == db && (k & 1) == 0)) best = k; /* ties to the even code */
+#endif
+  }
+  return s | best;
+}
+
+double situ_oracle_e2m1_decode(int code) {
+  static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  const double v = mag[code & 7];
+  return (code & 8) ? -v : v;
+}
+
+/* Per-tensor encode scale S_enc of a tensor with largest magnitude amax. */
+double situ_oracle_nvfp4_tensor_scale(double amax) {
+  if (!(amax > 0.0) || isinf(amax)) return 1.0;
+#if SITU_ORACLE_MUTANT == 34
+  return 1.0; /* planted: no tensor scale */
+#else
+  return E4M3_MAX * E2M1_MAX / amax;
+#endif
+}
+
+/* NVFP4 quantisation of v[rows, cols] (row pitch v_stride): codes[rows, cols]
+ * (one 4-bit code per byte here, unpacked), block scale codes [rows, cols /
+ * 16] (E4M3), with the tensor scale s_enc given.  Returns 0, or -1 when cols
+ * is not a multiple of 16. */
+int situ_oracle_nvfp4_quantize(const double *v, int64_t rows, int64_t cols, int64_t v_stride, double s_enc,
+                               uint8_t *codes, uint8_t *scales) {
+  if (cols % 16 != 0 || rows < 0) return -1;
+  const int64_t nblk = cols / 16;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t b = 0; b < nblk; ++b) {
+      const double *blk = v + r * v_stride + b * 16;
+      double amax = 0.0;
+      int special = 0;
+      for (int i = 0; i < 16; ++i) {
+        if (isnan(blk[i]) || isinf(blk[i])) special = 1;
+        else if (fabs(blk[i]) > amax) amax = fabs(blk[i]);
+      }
+      int sc;
+      if (special) {
+        sc = 0x7F;
+      } else {
+#if SITU_ORACLE_MUTANT == 33
+        sc = situ_oracle_e4m3_encode(amax * s_enc / 4.0); /* planted: divided by 4 instead of 6 */
+#else
+        sc = situ_oracle_e4m3_encode(amax * s_enc / E2M1_MAX);
+#endif
+      }
+      scales[r * nblk + b] = (uint8_t)sc;
+      const double sb = special ? 0.0 : situ_oracle_e4m3_decode(sc);
+      for (int i = 0; i < 16; ++i)
+        codes[r * cols + b * 16 + i] = (uint8_t)((sb > 0.0) ? situ_oracle_e2m1_encode(blk[i] * s_enc / sb) : 0);
+    }
+  }
+  return 0;
+}

@@ -427,6 +427,57 @@ def pin_mxfp8_blocks(o):
                 assert np.array_equal(codes[r, 32 * b:32 * b + 32], ref.view(torch.uint8).numpy()), (r, b)
 
 
+# ---- NVFP4 (mx_oracle.c) ----------------------------------------------------------------
+
+_E2M1 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def pin_e2m1_nearest_even(o):
+    """Every E2M1 code decodes to the format's 8 magnitudes with its sign; the
+    encoding of random values is the nearest of them by brute-force search,
+    ties to the even code (the midpoints 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5),
+    and magnitudes from 6 up clamp to 6."""
+    codes = np.arange(16, dtype=np.uint8)
+    dec = o.e2m1_decode(codes)
+    assert list(np.abs(dec[:8])) == _E2M1 and list(-dec[8:]) == _E2M1 and np.all(np.signbit(dec[8:]))
+    mids = {0.25: 0.0, 0.75: 1.0, 1.25: 1.0, 1.75: 2.0, 2.5: 2.0, 3.5: 4.0, 5.0: 4.0, 6.0: 6.0, 7.0: 6.0, 1e9: 6.0}
+    for x, want in mids.items():
+        assert o.e2m1_decode(o.e2m1_encode([x]))[0] == want, x
+        assert o.e2m1_decode(o.e2m1_encode([-x]))[0] == -want, -x
+    rng = np.random.default_rng(RNG_SEED + 13)
+    x = rng.uniform(-7.0, 7.0, 4000)
+    got = o.e2m1_decode(o.e2m1_encode(x))
+    grid = np.array(_E2M1)
+    for xv, g in zip(x, got):
+        d = np.abs(np.abs(xv) - grid)
+        assert abs(abs(g) - grid[np.argmin(d)]) == 0.0 or abs(xv) >= 6.0, (xv, g)
+        assert np.sign(g) in (0.0, np.sign(xv))
+
+
+def pin_nvfp4_blocks(o):
+    """Tensor scale 2688 / amax; each 16-element block's scale is torch's E4M3
+    conversion of amax_b * S_enc / 6; element codes are the nearest E2M1 of
+    v * S_enc / s_b; decoded values lie within half an E2M1 step (scaled) of v."""
+    rng = np.random.default_rng(RNG_SEED + 14)
+    v = rng.standard_normal((5, 64)) * np.exp2(rng.integers(-6, 6, (5, 1)))
+    v[2, 16:32] = 0.0
+    codes, scales, s_enc = o.nvfp4_quantize(v)
+    assert s_enc == 448.0 * 6.0 / np.abs(v).max()
+    for r in range(5):
+        for b in range(4):
+            blk = v[r, 16 * b:16 * b + 16]
+            want = torch.tensor([np.abs(blk).max() * s_enc / 6.0], dtype=torch.float32).to(torch.float8_e4m3fn)
+            assert scales[r, b] == want.view(torch.uint8).item(), (r, b)
+            sb = o.e4m3_decode(scales[r, b:b + 1])[0]
+            dec = o.e2m1_decode(codes[r, 16 * b:16 * b + 16]) * sb / s_enc
+            if sb == 0:
+                assert not np.any(codes[r, 16 * b:16 * b + 16] & 7)
+                continue
+            y = blk * s_enc / sb
+            step = np.where(np.abs(y) < 2, 0.5, np.where(np.abs(y) < 4, 1.0, 2.0))
+            assert np.all(np.abs(dec - blk) <= 0.5 * step * sb / s_enc * (1 + 1e-12) + (np.abs(y) > 6) * np.abs(blk)), (r, b)
+
+
 # ---- FC1 followed by SiTU-GLU (fc1_oracle.c) ---------------------------------------
 
 def _bf16(a):
@@ -662,6 +713,8 @@ PINS = [
     pin_e4m3_saturation,
     pin_mx_scale_rules,
     pin_mxfp8_blocks,
+    pin_e2m1_nearest_even,
+    pin_nvfp4_blocks,
     pin_fc1_bruteforce,
     pin_fc1_matches_activation_oracle,
     pin_fc1_grouped_equals_per_expert,
@@ -714,6 +767,9 @@ MUTANTS = {
     29: "FC2 weight read untransposed in the data gradient",
     30: "routing weight dropped from the fused dG",
     31: "upstream gradient dropped from the fused d_w",
+    32: "E2M1 ties to the larger magnitude",
+    33: "NVFP4 block scale from amax / 4",
+    34: "NVFP4 tensor scale not applied",
 }
 
 
