@@ -8,11 +8,13 @@ must move: read gate_up and w, write Y; read gate_up, grad_out and w, write
 d_gate_up and d_w), plus rows/s.
 
     python bench.py [--gpus N --steps K --warmup W] [--config 0..4] [--impl reference]
-                    [--variant row|col|full|mxfp8]
+                    [--variant row|col|full|mxfp8|nvfp4|fc1|fc2|attn_res]
 
 --variant picks the form timed (default: per-row routing weights, the routed
 MoE form): per-column [I] or per-element [T, I] weights, or MXFP8 outputs
-(E4M3 codes + E8M0 scales for Y and d_gate_up, OCP rule).  Algorithmic
+(E4M3 codes + E8M0 scales for Y and d_gate_up, OCP rule), or an NVFP4 Y
+(E2M1 codes + E4M3 scales per 16 + the tensor maximum, bf16 backward; the
+quantising kernel is also timed alone for its roofline).  Algorithmic
 bytes follow the form (weights read, weight gradients written, one byte per
 code plus one per 32 codes).  --variant fc1 times the fused FC1 grouped GEMM
 + SiTU-GLU forward on the routed-MoE rows (hidden 7168, 8 local experts) in
@@ -69,7 +71,8 @@ def parse_args(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-oracle sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--variant", choices=["row", "col", "full", "mxfp8", "fc1", "fc2", "attn_res"], default="row",
+    p.add_argument("--variant", choices=["row", "col", "full", "mxfp8", "nvfp4", "fc1", "fc2", "attn_res"],
+                   default="row",
                    help="routing-weight form or output format timed (default: per-row weights)")
     p.add_argument("--flush", choices=["auto", "always", "never"], default="auto",
                    help="flush L2 before every step (auto: when the inputs fit in L2)")
@@ -121,7 +124,9 @@ def workload_config(wl, beta, l2_note, world, variant="row"):
     return {
         "variant": {"row": "per-row routing weights, bf16/fp32 outputs",
                     "col": "per-column routing weights [I]", "full": "per-element routing weights [T, I]",
-                    "mxfp8": "per-row routing weights, MXFP8 Y and d_gate_up (E4M3 + E8M0 per 32, OCP rule)"}[variant],
+                    "mxfp8": "per-row routing weights, MXFP8 Y and d_gate_up (E4M3 + E8M0 per 32, OCP rule)",
+                    "nvfp4": "per-row routing weights, NVFP4 Y (E2M1 + E4M3 per 16, tensor scale from this "
+                             "call's amax pass), bf16 d_gate_up"}[variant],
         "workload": wl.describe(),
         "name": wl.name,
         "tokens": wl.tokens,
@@ -425,7 +430,9 @@ def variant_bytes(wl, variant: str):
     the given form.  Per-row weights: read gate_up and w, write Y; read
     gate_up, grad_out and w, write d_gate_up and d_w.  Per-column weights move
     I weights and I gradients per pass; per-element weights T I of each.
-    MXFP8 writes one byte per code and one scale byte per 32 codes."""
+    MXFP8 writes one byte per code and one scale byte per 32 codes; NVFP4
+    half a byte per code and one scale byte per 16 (the tensor maximum's extra
+    read of gate_up is not algorithmic: it counts against the kernels)."""
     T, I = wl.tokens, wl.inter
     es = 2 if wl.dtype == "bf16" else 4
     if variant == "col":
@@ -434,6 +441,8 @@ def variant_bytes(wl, variant: str):
         return T * (3 * I * es + 4 * I), T * (5 * I * es + 8 * I)
     if variant == "mxfp8":
         return T * (2 * I * es + I + I // 32 + 4), T * (3 * I * es + 2 * I + 2 * I // 32 + 8)
+    if variant == "nvfp4":
+        return T * (2 * I * es + I // 2 + I // 16 + 4), wl.bwd_bytes()
     return wl.fwd_bytes(), wl.bwd_bytes()
 
 
@@ -471,6 +480,8 @@ def cpu_oracle_rate(wl, beta, x, seconds: float, variant: str = "row"):
         if variant == "mxfp8":
             o.mxfp8_quantize(y)
             o.mxfp8_quantize(np.concatenate([r.dg, r.du], axis=1))
+        elif variant == "nvfp4":
+            o.nvfp4_quantize(y)
         done += rows.size
         if time.perf_counter() - t0 >= seconds:
             break
@@ -509,6 +520,8 @@ def run_reference(args):
         if args.variant == "mxfp8":
             o.mxfp8_quantize(y)
             o.mxfp8_quantize(np.concatenate([r.dg, r.du], axis=1))
+        elif args.variant == "nvfp4":
+            o.nvfp4_quantize(y)
 
     for _ in range(args.warmup):
         step()
@@ -920,6 +933,12 @@ def run_ours(args):
         d_gu = torch.empty(T, 2 * I, dtype=torch.float8_e4m3fn, device=dev)
         d_sc = torch.empty(T, 2 * I // 32, dtype=torch.uint8, device=dev)
         outputs = [y, y_sc, d_gu, d_sc, d_rw]
+    elif variant == "nvfp4":
+        y = torch.empty(T, I // 2, dtype=torch.uint8, device=dev)
+        y_sc = torch.empty(T, I // 16, dtype=torch.float8_e4m3fn, device=dev)
+        y_amax = torch.empty(1, dtype=torch.float32, device=dev)
+        d_gu = torch.empty(T, 2 * I, dtype=tdt, device=dev)
+        outputs = [y, y_sc, y_amax, d_gu, d_rw]
     else:
         y = torch.empty(T, I, dtype=tdt, device=dev)
         d_gu = torch.empty(T, 2 * I, dtype=tdt, device=dev)
@@ -937,6 +956,12 @@ def run_ours(args):
 
         def bwd():
             pkg.situ_glu_bwd_mxfp8(gu, rw, go, beta, lb, rule="ocp", data=d_gu, scale=d_sc, d_rw=d_rw)
+    elif variant == "nvfp4":
+        def fwd():
+            pkg.situ_glu_fwd_nvfp4(gu, rw, beta, lb, data=y, scale=y_sc, amax_out=y_amax)
+
+        def bwd():
+            pkg.situ_glu_bwd(gu, rw, go, beta, lb, d_gate_up=d_gu, d_rw=d_rw)
     else:
         def fwd():
             pkg.situ_glu_fwd(gu, rw, beta, lb, out=y)
@@ -979,6 +1004,23 @@ def run_ours(args):
     if world > 1:
         dist.all_reduce(times, op=dist.ReduceOp.MAX)
     total_ms, fwd_sum, bwd_sum = times.tolist()
+    quant_us = None
+    if variant == "nvfp4":
+        # the quantising kernel alone: the same call with the tensor maximum given
+        given = y_amax.clone()
+        qev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        torch.cuda.synchronize()
+        for k in range(K):
+            if flush:
+                flush_buf.zero_()
+            qev[k][0].record(stream)
+            pkg.situ_glu_fwd_nvfp4(gu, rw, beta, lb, data=y, scale=y_sc, amax=given)
+            qev[k][1].record(stream)
+        torch.cuda.synchronize()
+        qt = torch.tensor([sum(e[0].elapsed_time(e[1]) for e in qev)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(qt, op=dist.ReduceOp.MAX)
+        quant_us = qt.item() / K * 1e3
     ms_per_step = total_ms / K
     fwd_bytes, bwd_bytes = variant_bytes(wl, variant)
     step_bytes = fwd_bytes + bwd_bytes
@@ -995,11 +1037,14 @@ def run_ours(args):
                 "situ_glu_bwd_kernel"),
         "col": ("situ_glu_fwd_ew_kernel", "situ_glu_bwd_ew_kernel"),
         "full": ("situ_glu_fwd_ew_kernel", "situ_glu_bwd_ew_kernel"),
-        "mxfp8": ("situ_glu_fwd_mx_kernel", "situ_glu_bwd_mx_kernel"),
+        "mxfp8": ("situ_glu_fwd_quant_kernel<MxQuant>", "situ_glu_bwd_mx_kernel"),
+        "nvfp4": ("situ_glu_amax_kernel+situ_glu_fwd_quant_kernel<Nvfp4Quant>", "situ_glu_bwd_kernel"),
     }[variant]
-    launches_per_step = 3 if variant == "col" else 2  # per-column weights: plus the column finalize
+    # per-column weights: plus the column finalize; NVFP4: the amax pass, the quantising pass, the backward
+    launches_per_step = {"col": 3, "nvfp4": 3}.get(variant, 2)
     traffic_key = wl.name if variant == "row" else f"{wl.name}/{variant}"
-    traffic = recorded_traffic(bwd_kernel, traffic_key)
+    roof_kernel = "situ_glu_fwd_quant_kernel<Nvfp4Quant>" if variant == "nvfp4" else bwd_kernel
+    traffic = recorded_traffic(roof_kernel, traffic_key)
 
     # End to end through the public API with host buffers: every step copies the
     # inputs from pinned host memory, runs both passes and reads all outputs back.
@@ -1034,7 +1079,8 @@ def run_ours(args):
         e2e_ms = t.item() / K2
         h2d = input_bytes
         d2h = sum(t.numel() * t.element_size() for t in outputs_h)
-        api = "situ_glu_fwd_mxfp8/situ_glu_bwd_mxfp8" if variant == "mxfp8" else "situ_glu_fwd/situ_glu_bwd"
+        api = {"mxfp8": "situ_glu_fwd_mxfp8/situ_glu_bwd_mxfp8",
+               "nvfp4": "situ_glu_fwd_nvfp4/situ_glu_bwd"}.get(variant, "situ_glu_fwd/situ_glu_bwd")
         e2e = {"value": step_bytes * world / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": K2,
                "api": f"ffn_gated_activation_b200.{api} on pinned host copies"}
@@ -1045,6 +1091,30 @@ def run_ours(args):
         cpu = {"value": rate, "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": f"first {rows_done} of {T} rows, fwd + bwd, {secs:.1f} s, single-threaded fp64"}
 
+    kernels = {
+        fwd_kernel: {"us": fwd_us, "bytes": fwd_bytes, "GB/s": fwd_gbs,
+                     "pct_of_nominal_8TBs": fwd_gbs / NOMINAL_HBM_GBS * 100,
+                     "frac_of_measured_copy": fwd_gbs / peak, "rows_per_s": T / (fwd_us / 1e6)},
+        bwd_kernel: {"us": bwd_us, "bytes": bwd_bytes, "GB/s": bwd_gbs,
+                     "pct_of_nominal_8TBs": bwd_gbs / NOMINAL_HBM_GBS * 100,
+                     "frac_of_measured_copy": bwd_gbs / peak, "rows_per_s": T / (bwd_us / 1e6)},
+    }
+    roofline = {"bound": "hbm", "kernel": bwd_kernel, "achieved": bwd_gbs, "peak": peak,
+                "unit": "GB/s", "frac": bwd_gbs / peak, "peak_source": f"{peak_src} copy bandwidth",
+                "traffic": traffic}
+    if quant_us is not None:
+        amax_bytes = T * (2 * I * (2 if wl.dtype == "bf16" else 4) + 4)
+        amax_us = max(fwd_us - quant_us, 1e-9)
+        q_gbs = fwd_bytes / quant_us / 1e3
+        kernels["situ_glu_amax_kernel"] = {"us": amax_us, "bytes": amax_bytes, "GB/s": amax_bytes / amax_us / 1e3,
+                                           "frac_of_measured_copy": amax_bytes / amax_us / 1e3 / peak,
+                                           "note": "the NVFP4 call's time less the quantising pass alone"}
+        kernels[roof_kernel] = {"us": quant_us, "bytes": fwd_bytes, "GB/s": q_gbs,
+                                "frac_of_measured_copy": q_gbs / peak,
+                                "note": "timed alone, tensor maximum given"}
+        roofline = {"bound": "hbm", "kernel": roof_kernel, "achieved": q_gbs, "peak": peak, "unit": "GB/s",
+                    "frac": q_gbs / peak, "peak_source": f"{peak_src} copy bandwidth", "traffic": traffic}
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
@@ -1053,17 +1123,8 @@ def run_ours(args):
             "config": workload_config(wl, beta, l2_note, world, variant),
             "rows_per_s": T * world / (ms_per_step / 1e3),
             "pct_of_nominal_hbm": value / world / NOMINAL_HBM_GBS * 100.0,
-            "kernels": {
-                fwd_kernel: {"us": fwd_us, "bytes": fwd_bytes, "GB/s": fwd_gbs,
-                             "pct_of_nominal_8TBs": fwd_gbs / NOMINAL_HBM_GBS * 100,
-                             "frac_of_measured_copy": fwd_gbs / peak, "rows_per_s": T / (fwd_us / 1e6)},
-                bwd_kernel: {"us": bwd_us, "bytes": bwd_bytes, "GB/s": bwd_gbs,
-                             "pct_of_nominal_8TBs": bwd_gbs / NOMINAL_HBM_GBS * 100,
-                             "frac_of_measured_copy": bwd_gbs / peak, "rows_per_s": T / (bwd_us / 1e6)},
-            },
-            "roofline": {"bound": "hbm", "kernel": bwd_kernel, "achieved": bwd_gbs, "peak": peak,
-                         "unit": "GB/s", "frac": bwd_gbs / peak, "peak_source": f"{peak_src} copy bandwidth",
-                         "traffic": traffic},
+            "kernels": kernels,
+            "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches_per_step * K,

@@ -1306,6 +1306,104 @@ __device__ __forceinline__ void mx_store_vec(const float2 (&y)[S::kPairs], bool 
   if (slot.lead) scale_row[slot.scale_off] = static_cast<uint8_t>(sb);
 }
 
+// ---- NVFP4 (E2M1 codes, an E4M3 scale per 16 elements, a per-tensor scale)
+// NVIDIA's NVFP4 format, the other block-scaled recipe the SiTU-GLU path was
+// tested with (Megatron-LM PR #6673, "Test results").  With A the tensor's
+// largest magnitude, S_enc = 448 * 6 / A (1 when A is 0 or not finite); block
+// b of 16 elements stores s_b = E4M3(amax_b * S_enc / 6) and each element the
+// E2M1 code of y * (S_enc / s_b) (nearest even, clamped to +-6); decoding is
+// q * s_b / S_enc.  Codes are packed two per byte, element 2k in the low
+// nibble.  A block holding NaN or infinity gets scale code 0x7F.
+
+struct Nvfp4Out {
+  char* data;            // packed E2M1 codes, [tokens, cols / 2] bytes
+  int64_t data_pitch;    // bytes
+  uint8_t* scale;        // E4M3 block scales, [tokens, cols / 16]
+  int64_t scale_pitch;   // bytes
+  const float* amax;     // device: the tensor's largest magnitude
+};
+
+// Two E2M1 codes of (lo, hi) in one byte, lo in the low nibble (cvt packs its
+// first source into the high nibble); four such bytes per register.
+__device__ __forceinline__ uint32_t e2m1x8(const float2 (&v)[4]) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(v[0].x), "f"(v[0].y), "f"(v[1].x), "f"(v[1].y), "f"(v[2].x), "f"(v[2].y), "f"(v[3].x), "f"(v[3].y));
+  return r;
+}
+__device__ __forceinline__ uint32_t e2m1x4(const float2 (&v)[2]) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 b0, b1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "mov.b16 %0, {b0, b1};\n\t}"
+      : "=h"(r)
+      : "f"(v[0].x), "f"(v[0].y), "f"(v[1].x), "f"(v[1].y));
+  return r;
+}
+
+__device__ __forceinline__ float nvfp4_tensor_scale(float amax) {
+  return (amax > 0.0f && amax <= 3.402823466e38f) ? 2688.0f / amax : 1.0f;  // 448 * 6 / A
+}
+
+// Quantise the kPairs pairs y of vector j of a row into NVFP4.  Every lane of
+// the warp calls this (the block maximum is shuffled over the 16 / kElems
+// lanes of a block); lanes with `active` set store their codes and the first
+// lane of each block its scale code.
+template <typename S, bool ACTIVE_ALWAYS = false>
+__device__ __forceinline__ void nvfp4_store_vec(const float2 (&y)[S::kPairs], bool active, char* data_row,
+                                                uint8_t* scale_row, int j, float s_enc) {
+  constexpr int kElems = 2 * S::kPairs;
+  constexpr int kLanes = 16 / kElems;
+  float amax = 0.0f;
+#pragma unroll
+  for (int p = 0; p < S::kPairs; ++p) amax = max_nan(amax, max_nan(fabsf(y[p].x), fabsf(y[p].y)));
+  if (!ACTIVE_ALWAYS && !active) amax = 0.0f;
+#pragma unroll
+  for (int o = 1; o < kLanes; o <<= 1) amax = max_nan(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const bool special = __float_as_uint(amax) >= 0x7f800000u;
+  const uint8_t sc = special ? static_cast<uint8_t>(0x7f)
+                             : static_cast<uint8_t>(__nv_cvt_float_to_fp8(amax * s_enc / 6.0f, __NV_SATFINITE, __NV_E4M3));
+  const float sb = special ? 0.0f : __half2float(__half(__nv_cvt_fp8_to_halfraw(sc, __NV_E4M3)));
+  const float r = sb > 0.0f ? s_enc / sb : 0.0f;
+  float2 q[S::kPairs];
+#pragma unroll
+  for (int p = 0; p < S::kPairs; ++p) q[p] = mul2(y[p], splat(r));
+  if (!ACTIVE_ALWAYS && !active) return;
+  if constexpr (S::kPairs == 4) {
+    *reinterpret_cast<uint32_t*>(data_row + j * 4) = e2m1x8(q);
+  } else {
+    *reinterpret_cast<uint16_t*>(data_row + j * 2) = static_cast<uint16_t>(e2m1x4(q));
+  }
+  if (j % kLanes == 0) scale_row[j / kLanes] = sc;
+}
+
+// Output policies of the quantising forward: MXFP8 and NVFP4.
+struct MxQuant {
+  using Out = MxOut;
+  template <typename S, bool ALL>
+  __device__ __forceinline__ static void store(const float2 (&y)[S::kPairs], bool active, const Out& m, int64_t row,
+                                               int j, float) {
+    mx_store_vec<S, ALL>(y, active, m.data + row * m.data_pitch, m.scale + row * m.scale_pitch, MxSlot<S>(j), m.rule);
+  }
+  __device__ __forceinline__ static float tensor_param(const Out&) { return 0.0f; }
+};
+struct Nvfp4Quant {
+  using Out = Nvfp4Out;
+  template <typename S, bool ALL>
+  __device__ __forceinline__ static void store(const float2 (&y)[S::kPairs], bool active, const Out& m, int64_t row,
+                                               int j, float s_enc) {
+    nvfp4_store_vec<S, ALL>(y, active, m.data + row * m.data_pitch, m.scale + row * m.scale_pitch, j, s_enc);
+  }
+  __device__ __forceinline__ static float tensor_param(const Out& m) { return nvfp4_tensor_scale(*m.amax); }
+};
+
 template <typename S, int GATE, bool HAS_LB>
 __device__ __forceinline__ void fwd_pairs(const uint4& gv, const uint4& uv, float2 wbb, const Coeffs& c,
                                           float2 (&y)[S::kPairs]) {
@@ -1335,15 +1433,14 @@ __device__ __forceinline__ void zero_y(float2 (&y)[S::kPairs]) {
 }
 
 // Rows of the two-vector layout; ALL: every lane owns two vectors (vpr = 2 nt),
-// so no lane is ever inactive.
-template <typename S, int GATE, bool HAS_LB, bool ALL>
-__device__ __forceinline__ void fwd_mx_rows(const FwdArgs& a, const MxOut& m) {
+// so no lane is ever inactive.  Q: the output format (MXFP8 or NVFP4).
+template <typename S, int GATE, bool HAS_LB, bool ALL, class Q>
+__device__ __forceinline__ void fwd_quant_rows(const FwdArgs& a, const typename Q::Out& m) {
   constexpr int kP = S::kPairs;
   const int nt = blockDim.x;
   const int j = threadIdx.x, j2 = j + nt;
   const bool one = ALL || j < a.vpr, two = ALL || j2 < a.vpr;
-  const MxSlot<S> s0(j), s1(j2);
-  const int rule = m.rule;
+  const float tp = Q::tensor_param(m);
   int64_t row = blockIdx.x;
   if (row >= a.tokens) return;
   const uint4 z = make_uint4(0, 0, 0, 0);
@@ -1378,36 +1475,33 @@ __device__ __forceinline__ void fwd_mx_rows(const FwdArgs& a, const MxOut& m) {
       nw = load_rw(a.rw, next);
     }
     const float2 wbb = splat(w * a.c.bb);
-    char* drow = m.data + row * m.data_pitch;
-    uint8_t* srow = m.scale + row * m.scale_pitch;
     float2 y[kP];
     if (ALL || one) fwd_pairs<S, GATE, HAS_LB>(g0, u0, wbb, a.c, y); else zero_y<S>(y);
-    mx_store_vec<S, ALL>(y, one, drow, srow, s0, rule);
+    Q::template store<S, ALL>(y, one, m, row, j, tp);
     if (ALL || two) fwd_pairs<S, GATE, HAS_LB>(g1, u1, wbb, a.c, y); else zero_y<S>(y);
-    mx_store_vec<S, ALL>(y, two, drow, srow, s1, rule);
+    Q::template store<S, ALL>(y, two, m, row, j2, tp);
     if (!more) break;
     row = next;
     g0 = ng0; u0 = nu0; g1 = ng1; u1 = nu1; w = nw;
   }
 }
 
-template <typename S, int GATE, bool HAS_LB>
-__global__ void __launch_bounds__(kMaxThreads) situ_glu_fwd_mx_kernel(const FwdArgs a, const MxOut m) {
+template <typename S, int GATE, bool HAS_LB, class Q>
+__global__ void __launch_bounds__(kMaxThreads) situ_glu_fwd_quant_kernel(const FwdArgs a, const typename Q::Out m) {
   constexpr int kP = S::kPairs;
   const int nt = blockDim.x;
   if (a.vpr == 2 * nt) {
-    fwd_mx_rows<S, GATE, HAS_LB, true>(a, m);
+    fwd_quant_rows<S, GATE, HAS_LB, true, Q>(a, m);
     return;
   }
   if (a.vpr < 2 * nt) {
-    fwd_mx_rows<S, GATE, HAS_LB, false>(a, m);
+    fwd_quant_rows<S, GATE, HAS_LB, false, Q>(a, m);
     return;
   }
+  const float tp = Q::tensor_param(m);
   for (int64_t row = blockIdx.x; row < a.tokens; row += gridDim.x) {
     const char* gu = a.gate_up + row * a.gu_pitch;
     const float2 wbb = splat(load_rw(a.rw, row) * a.c.bb);
-    char* drow = m.data + row * m.data_pitch;
-    uint8_t* srow = m.scale + row * m.scale_pitch;
     for (int jb = 0; jb < a.vpr; jb += nt) {  // uniform trip count: every lane reaches the shuffles
       const int j = jb + threadIdx.x;
       const bool act = j < a.vpr;
@@ -1417,9 +1511,36 @@ __global__ void __launch_bounds__(kMaxThreads) situ_glu_fwd_mx_kernel(const FwdA
                                    a.c, y);
       else
         zero_y<S>(y);
-      mx_store_vec<S>(y, act, drow, srow, MxSlot<S>(j), m.rule);
+      Q::template store<S, false>(y, act, m, row, j, tp);
     }
   }
+}
+
+// The tensor's largest finite |Y| (NVFP4's tensor scale; NaN and infinite
+// elements only mark their own blocks): per-thread maxima of the fp32
+// results, a warp maximum, one integer atomicMax per warp on the float bits
+// (non-negative floats order as integers), so the result is order-free.
+template <typename S, int GATE, bool HAS_LB>
+__global__ void __launch_bounds__(kMaxThreads) situ_glu_amax_kernel(const FwdArgs a, unsigned int* amax_bits) {
+  constexpr int kP = S::kPairs;
+  float m = 0.0f;
+  for (int64_t row = blockIdx.x; row < a.tokens; row += gridDim.x) {
+    const char* gu = a.gate_up + row * a.gu_pitch;
+    const float2 wbb = splat(load_rw(a.rw, row) * a.c.bb);
+    for (int j = threadIdx.x; j < a.vpr; j += blockDim.x) {
+      float2 y[kP];
+      fwd_pairs<S, GATE, HAS_LB>(ld_stream(gu + j * kVecBytes), ld_stream(gu + a.half_bytes + j * kVecBytes), wbb, a.c,
+                                 y);
+#pragma unroll
+      for (int p = 0; p < kP; ++p) {
+        const float ax = fabsf(y[p].x), ay = fabsf(y[p].y);
+        m = ax <= 3.402823466e38f ? fmaxf(m, ax) : m;  // false for NaN and infinity
+        m = ay <= 3.402823466e38f ? fmaxf(m, ay) : m;
+      }
+    }
+  }
+  const unsigned int bits = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+  if ((threadIdx.x & 31) == 0 && bits != 0u) atomicMax(amax_bits, bits);
 }
 
 // Backward with MXFP8 d_gate_up: codes [tokens, 2 inter] (dG then dU), scales
@@ -2501,12 +2622,42 @@ auto pick_mx_gate(int gate) {
     }
   } else {
     switch (gate) {
-      case kGateSquare: return situ_glu_fwd_mx_kernel<S, kGateSquare, LB>;
-      case kGateEqual: return situ_glu_fwd_mx_kernel<S, kGateEqual, LB>;
-      case kGateRoot: return situ_glu_fwd_mx_kernel<S, kGateRoot, LB>;
-      default: return situ_glu_fwd_mx_kernel<S, kGateGeneric, LB>;
+      case kGateSquare: return situ_glu_fwd_quant_kernel<S, kGateSquare, LB, MxQuant>;
+      case kGateEqual: return situ_glu_fwd_quant_kernel<S, kGateEqual, LB, MxQuant>;
+      case kGateRoot: return situ_glu_fwd_quant_kernel<S, kGateRoot, LB, MxQuant>;
+      default: return situ_glu_fwd_quant_kernel<S, kGateGeneric, LB, MxQuant>;
     }
   }
+}
+
+using FwdNvKernel = void (*)(FwdArgs, Nvfp4Out);
+using AmaxKernel = void (*)(FwdArgs, unsigned int*);
+
+template <typename S, bool LB>
+FwdNvKernel pick_nv_gate(int gate) {
+  switch (gate) {
+    case kGateSquare: return situ_glu_fwd_quant_kernel<S, kGateSquare, LB, Nvfp4Quant>;
+    case kGateEqual: return situ_glu_fwd_quant_kernel<S, kGateEqual, LB, Nvfp4Quant>;
+    case kGateRoot: return situ_glu_fwd_quant_kernel<S, kGateRoot, LB, Nvfp4Quant>;
+    default: return situ_glu_fwd_quant_kernel<S, kGateGeneric, LB, Nvfp4Quant>;
+  }
+}
+template <typename S, bool LB>
+AmaxKernel pick_amax_gate(int gate) {
+  switch (gate) {
+    case kGateSquare: return situ_glu_amax_kernel<S, kGateSquare, LB>;
+    case kGateEqual: return situ_glu_amax_kernel<S, kGateEqual, LB>;
+    case kGateRoot: return situ_glu_amax_kernel<S, kGateRoot, LB>;
+    default: return situ_glu_amax_kernel<S, kGateGeneric, LB>;
+  }
+}
+FwdNvKernel pick_fwd_nv(situ_dtype_t dtype, int gate, bool lb) {
+  if (dtype == SITU_DTYPE_BF16) return lb ? pick_nv_gate<Bf16, true>(gate) : pick_nv_gate<Bf16, false>(gate);
+  return lb ? pick_nv_gate<F32, true>(gate) : pick_nv_gate<F32, false>(gate);
+}
+AmaxKernel pick_amax(situ_dtype_t dtype, int gate, bool lb) {
+  if (dtype == SITU_DTYPE_BF16) return lb ? pick_amax_gate<Bf16, true>(gate) : pick_amax_gate<Bf16, false>(gate);
+  return lb ? pick_amax_gate<F32, true>(gate) : pick_amax_gate<F32, false>(gate);
 }
 
 FwdMxKernel pick_fwd_mx(situ_dtype_t dtype, int gate, bool lb) {
@@ -3433,4 +3584,91 @@ extern "C" situ_status_t situ_attn_res_fwd(const void* blocks, int64_t nblocks, 
   else
     situ_attn_res_kernel<F32><<<grid, threads, smem, s>>>(a);
   return check_launch("situ_attn_res_fwd");
+}
+
+
+// ---------------------------------------------------------------------------
+// NVFP4 forward
+// ---------------------------------------------------------------------------
+
+extern "C" situ_status_t situ_glu_fwd_nvfp4(const void* gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
+                                            int64_t gate_up_row_stride, const void* rw, situ_dtype_t rw_dtype,
+                                            situ_rw_mode_t rw_mode, int64_t rw_stride, double beta,
+                                            int has_linear_beta, double linear_beta, void* y_data,
+                                            int64_t y_data_row_stride, void* y_scale, int64_t y_scale_row_stride,
+                                            float* amax, int amax_given, void* stream) {
+  tl_last_error[0] = '\0';
+  Coeffs c;
+  int gate = kGateGeneric;
+  situ_status_t st = check_common(dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride, beta,
+                                  has_linear_beta, linear_beta, &c, &gate);
+  if (st != SITU_OK) return st;
+  if (inter % 16 != 0)
+    return fail(SITU_ERR_INVALID_ARG, "NVFP4 outputs need inter a multiple of 16, got %lld", (long long)inter);
+  if (rw_mode == SITU_RW_COL || rw_mode == SITU_RW_FULL)
+    return fail(SITU_ERR_UNSUPPORTED, "NVFP4 outputs take per-row, broadcast or no routing weights");
+  if (amax_given != 0 && amax_given != 1) return fail(SITU_ERR_INVALID_ARG, "amax_given must be 0 or 1");
+  if (y_data_row_stride < inter / 2 || y_scale_row_stride < inter / 16)
+    return fail(SITU_ERR_INVALID_ARG, "NVFP4 data or scale row pitch shorter than a row");
+  if (amax == nullptr) return fail(SITU_ERR_INVALID_ARG, "amax is NULL");
+  if (!aligned(amax, 4)) return fail(SITU_ERR_MISALIGNED, "amax not 4-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (tokens == 0) {
+    if (!amax_given) {
+      cudaError_t err = cudaMemsetAsync(amax, 0, sizeof(float), s);
+      if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
+    }
+    return SITU_OK;
+  }
+  if (gate_up == nullptr || y_data == nullptr || y_scale == nullptr)
+    return fail(SITU_ERR_INVALID_ARG, "gate_up, y_data or y_scale is NULL");
+  const int es = elem_size(dtype);
+  if (!span_fits(tokens, gate_up_row_stride, 2 * inter, es) || !span_fits(tokens, y_data_row_stride, inter / 2, 1) ||
+      !span_fits(tokens, y_scale_row_stride, inter / 16, 1) ||
+      (rw_mode == SITU_RW_ROW && !span_fits(tokens, rw_stride, 1, elem_size(rw_dtype))))
+    return fail(SITU_ERR_INVALID_ARG, "tensor extent overflows int64");
+  if (!aligned(gate_up, 16) || (gate_up_row_stride * es) % 16 != 0 || !aligned(y_data, 16) ||
+      y_data_row_stride % 16 != 0 || (rw_mode != SITU_RW_NONE && !aligned(rw, elem_size(rw_dtype))))
+    return fail(SITU_ERR_MISALIGNED, "gate_up / y_data base or row pitch not 16-byte aligned, or rw misaligned");
+  const Span s_gu = matrix_span(gate_up, tokens, gate_up_row_stride, 2 * inter, es);
+  const Span s_rw = weight_span(rw, rw_mode, tokens, rw_stride, inter, elem_size(rw_dtype));
+  const Span s_d = matrix_span(y_data, tokens, y_data_row_stride, inter / 2, 1);
+  const Span s_s = matrix_span(y_scale, tokens, y_scale_row_stride, inter / 16, 1);
+  const Span s_a = {reinterpret_cast<uintptr_t>(amax), reinterpret_cast<uintptr_t>(amax) + 4};
+  const Span outs[] = {s_d, s_s, s_a};
+  for (int i = 0; i < 3; ++i) {
+    if (overlap(outs[i], s_gu) || overlap(outs[i], s_rw)) return fail(SITU_ERR_INVALID_ARG, "an output overlaps an input");
+    for (int k = i + 1; k < 3; ++k)
+      if (overlap(outs[i], outs[k])) return fail(SITU_ERR_INVALID_ARG, "outputs overlap each other");
+  }
+  FwdArgs a;
+  a.gate_up = static_cast<const char*>(gate_up);
+  a.gu_pitch = gate_up_row_stride * es;
+  a.out = nullptr;
+  a.out_pitch = 0;
+  a.rw = {rw, rw_stride, static_cast<int>(rw_mode), (rw_mode != SITU_RW_NONE && rw_dtype == SITU_DTYPE_BF16) ? 1 : 0};
+  a.tokens = tokens;
+  a.half_bytes = static_cast<int>(inter * es);
+  a.vpr = static_cast<int>(inter * es / kVecBytes);
+  a.c = c;
+  const int threads = choose_threads(a.vpr);
+  if (!amax_given) {
+    cudaError_t err = cudaMemsetAsync(amax, 0, sizeof(float), s);
+    if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
+    AmaxKernel ka = pick_amax(dtype, gate, has_linear_beta != 0);
+    int grid = 0;
+    st = launch_grid(reinterpret_cast<const void*>(ka), threads, 0, tokens, &grid);
+    if (st != SITU_OK) return st;
+    ka<<<grid, threads, 0, s>>>(a, reinterpret_cast<unsigned int*>(amax));
+    st = check_launch("situ_glu_fwd_nvfp4 (amax)");
+    if (st != SITU_OK) return st;
+  }
+  const Nvfp4Out m{static_cast<char*>(y_data), y_data_row_stride, static_cast<uint8_t*>(y_scale), y_scale_row_stride,
+                   amax};
+  FwdNvKernel k = pick_fwd_nv(dtype, gate, has_linear_beta != 0);
+  int grid = 0;
+  st = launch_grid(reinterpret_cast<const void*>(k), threads, 0, tokens, &grid);
+  if (st != SITU_OK) return st;
+  k<<<grid, threads, 0, s>>>(a, m);
+  return check_launch("situ_glu_fwd_nvfp4");
 }

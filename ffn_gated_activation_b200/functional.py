@@ -425,6 +425,43 @@ def apply_attn_res(prefix_sum: torch.Tensor, block_residual: torch.Tensor, proj_
     return _attn_res_launch(block_residual, prefix_sum, norm_weight, proj_weight, variance_epsilon, out_dtype, out)
 
 
+def situ_glu_fwd_nvfp4(gate_up: torch.Tensor, routing_weights, beta: float = DEFAULT_BETA,
+                       linear_beta: float | None = DEFAULT_LINEAR_BETA, amax: torch.Tensor | None = None,
+                       data=None, scale=None, amax_out: torch.Tensor | None = None, stream=None):
+    """Forward with an NVFP4 Y: returns (packed E2M1 codes [..., I / 2] uint8,
+    E4M3 block scales [..., I / 16] as torch.float8_e4m3fn, amax: a 1-element
+    fp32 tensor holding the tensor maximum A).  Pass ``amax`` (1 element, on
+    gate_up's device) to use a known A instead of computing it; otherwise A is
+    computed into ``amax_out`` (allocated when None).  Decode code q of block
+    b as q * scale_b * A / 2688."""
+    _check_beta(beta, linear_beta)
+    g2, lead, inter = _rows(gate_up)
+    dtype = _dtype_code(g2, "gate_up")
+    mode, rw, rw_stride = routing_mode(lead, inter, routing_weights)
+    rw_dtype = _dtype_code(rw, "routing_weights") if rw is not None else abi.SITU_DTYPE_F32
+    if data is None:
+        data = torch.empty(lead + (inter // 2,), dtype=torch.uint8, device=gate_up.device)
+    if scale is None:
+        scale = torch.empty(lead + (inter // 16,), dtype=torch.float8_e4m3fn, device=gate_up.device)
+    given = amax is not None
+    if amax is None:
+        amax = amax_out if amax_out is not None else torch.empty(1, dtype=torch.float32, device=gate_up.device)
+    if amax.dtype != torch.float32 or amax.numel() != 1 or amax.device != gate_up.device:
+        raise ValueError("amax must be one float32 element on gate_up's device")
+    d2 = data.view(-1, inter // 2)
+    s2 = scale.view(-1, inter // 16)
+    tokens = g2.shape[0]
+    st = abi.situ_glu_fwd_nvfp4(g2.data_ptr(), dtype, tokens, inter, g2.stride(0) if tokens > 1 else 2 * inter,
+                                rw.data_ptr() if rw is not None else None, rw_dtype, mode, rw_stride,
+                                float(beta), int(linear_beta is not None),
+                                float(linear_beta) if linear_beta is not None else 0.0,
+                                d2.data_ptr(), d2.stride(0) if tokens > 1 else inter // 2,
+                                s2.data_ptr(), s2.stride(0) if tokens > 1 else inter // 16,
+                                amax.data_ptr(), int(given), _stream_handle(stream))
+    abi.check(st, "situ_glu_fwd_nvfp4")
+    return data, scale, amax
+
+
 class WeightedSiTUFunction(torch.autograd.Function):
     """Routing-weighted SiTU-GLU with the analytic fused backward.
 

@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define SITU_GLU_ABI_VERSION 6
+#define SITU_GLU_ABI_VERSION 7
 
 typedef enum situ_status {
   SITU_OK = 0,
@@ -228,6 +228,36 @@ situ_status_t situ_glu_bwd_mxfp8(const void *gate_up, situ_dtype_t dtype, int64_
                                  void *d_rw, int64_t d_rw_stride,
                                  void *workspace, size_t workspace_bytes,
                                  void *stream);
+
+/*
+ * Forward with an NVFP4 Y (NVIDIA's NVFP4 format, the other block-scaled
+ * recipe the integration was tested with -- Megatron-LM PR #6673, "Test
+ * results"; the format is NVIDIA's public definition): with A the largest
+ * finite |Y| of the call and S_enc = 448 * 6 / A (1 when A is 0 or not finite),
+ *   y_scale  [tokens, >= inter / 16] E4M3 codes s_b = E4M3(amax_b S_enc / 6)
+ *            of every 16 consecutive elements of a row (0x7F for a block
+ *            holding NaN or infinity); row pitch y_scale_row_stride bytes
+ *   y_data   [tokens, >= inter / 2] bytes of packed FP4 E2M1 codes of
+ *            Y S_enc / s_b (nearest even, clamped to +-6), element 2k in the
+ *            low nibble of byte k; row pitch y_data_row_stride bytes (a
+ *            multiple of 16, base 16-byte aligned)
+ *   amax     device fp32: A.  amax_given = 0: the library computes it first
+ *            (a pass that reads gate_up once more) and writes it here;
+ *            amax_given = 1: the caller's A is used (e.g. from an earlier
+ *            step); block scales and codes saturate (448, +-6) where it is
+ *            below the call's own maximum.
+ * A consumer decodes code q of block b as q * s_b * A / 2688.  inter must be a
+ * multiple of 16; routing weights per row, broadcast or none.  Other
+ * arguments and errors as for situ_glu_fwd.
+ */
+situ_status_t situ_glu_fwd_nvfp4(const void *gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
+                                 int64_t gate_up_row_stride,
+                                 const void *rw, situ_dtype_t rw_dtype, situ_rw_mode_t rw_mode,
+                                 int64_t rw_stride,
+                                 double beta, int has_linear_beta, double linear_beta,
+                                 void *y_data, int64_t y_data_row_stride,
+                                 void *y_scale, int64_t y_scale_row_stride,
+                                 float *amax, int amax_given, void *stream);
 
 /* ---- FC1 grouped GEMM + SiTU-GLU --------------------------------------------
  * Megatron-LM PR #6673, "Design": with a SiTU-capable cuDNN frontend FC1's

@@ -146,6 +146,8 @@ class Oracle:
         lib.situ_oracle_mxfp8_quantize.restype = _INT
         lib.situ_oracle_e2m1_encode.argtypes = [_DBL]
         lib.situ_oracle_e2m1_encode.restype = _INT
+        lib.situ_oracle_e2m1_encode_n.argtypes = [_VP, _I64, _VP]
+        lib.situ_oracle_e2m1_encode_n.restype = None
         lib.situ_oracle_e2m1_decode.argtypes = [_INT]
         lib.situ_oracle_e2m1_decode.restype = _DBL
         lib.situ_oracle_nvfp4_tensor_scale.argtypes = [_DBL]
@@ -314,9 +316,11 @@ class Oracle:
     # -- NVFP4 (mx_oracle.c) ----------------------------------------------------
 
     def e2m1_encode(self, x) -> np.ndarray:
-        x = np.asarray(x, dtype=np.float64)
-        f = self._lib.situ_oracle_e2m1_encode
-        return np.array([f(float(v)) for v in x.reshape(-1)], dtype=np.uint8).reshape(x.shape)
+        """E2M1 codes (sign << 3 | magnitude code, uint8) of reals x: nearest-even, clamped to +-6."""
+        x = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+        out = np.empty(x.shape, dtype=np.uint8)
+        self._lib.situ_oracle_e2m1_encode_n(_ptr(x), x.size, _ptr(out))
+        return out
 
     def e2m1_decode(self, codes) -> np.ndarray:
         c = np.asarray(codes, dtype=np.uint8)

@@ -200,6 +200,10 @@ int situ_oracle_e2m1_encode(double x) {
   return s | best;
 }
 
+void situ_oracle_e2m1_encode_n(const double *x, int64_t n, uint8_t *codes) {
+  for (int64_t i = 0; i < n; ++i) codes[i] = (uint8_t)situ_oracle_e2m1_encode(x[i]);
+}
+
 double situ_oracle_e2m1_decode(int code) {
   static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
   const double v = mag[code & 7];

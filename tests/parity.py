@@ -238,3 +238,96 @@ def check_mx(name: str, codes: np.ndarray, scales: np.ndarray, ref: np.ndarray, 
     exact, total = int(np.sum(fin & (g == mid))), int(np.sum(fin))
     assert total == 0 or exact >= min_exact * total, f"{name}: only {exact} of {total} codes equal the oracle's"
     return {"codes": total, "exact": exact}
+
+
+# ---- NVFP4 outputs ----------------------------------------------------------------------
+
+def e2m1_key(codes: np.ndarray) -> np.ndarray:
+    """E2M1 codes (one per byte) in value order (sign-magnitude; both zeros equal)."""
+    c = codes.astype(np.int32)
+    m = c & 0x7
+    return np.where(c & 0x8, -m, m)
+
+
+def unpack_e2m1(packed: np.ndarray) -> np.ndarray:
+    """[R, C / 2] bytes -> [R, C] codes, element 2k from the low nibble of byte k."""
+    p = packed.astype(np.uint8)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), dtype=np.uint8)
+    out[..., 0::2] = p & 0xF
+    out[..., 1::2] = p >> 4
+    return out
+
+
+# The kernel forms S_enc, the block-scale argument and the element ratio in
+# fp32 (a few roundings of 2^-24 each): they may sit this far (relative) from
+# the oracle's fp64 values.
+NVFP4_SLACK = 2.0 ** -20
+
+
+def check_nvfp4(name: str, packed: np.ndarray, scales: np.ndarray, amax: float, ref: np.ndarray, tol: np.ndarray,
+                min_exact: float = 0.9, full_tensor: bool = True):
+    """NVFP4 codes (packed [R, C / 2]), E4M3 block scales [R, C / 16] and the
+    tensor maximum ``amax`` the kernel used, against the oracle's exact values
+    ``ref`` [R, C] when the kernel's fp32 values may differ from ref by up to
+    ``tol``.  ``amax`` must lie within the bounds the oracle's values allow
+    (max |ref| -+ tol, when ``ref`` holds the whole tensor, else at least the
+    lower bound); with S = 2688 / amax, each block scale must lie between the
+    oracle's E4M3 codes for the smallest and the largest block maximum within
+    tol, times S / 6; given the kernel's block scale s, each code between the
+    oracle's E2M1 codes for (ref -+ tol) S / s; and at least ``min_exact`` of
+    the codes equal the oracle's code of ref S / s (oracle.nvfp4_quantize with
+    the same S, on the rows it covers).  Blocks holding NaN or infinity must
+    carry scale code 0x7F; a block whose scale decodes to 0 must hold only zero
+    codes."""
+    o = oracle.load()
+    R, C = ref.shape
+    nb = C // 16
+    codes = unpack_e2m1(packed)
+    assert codes.shape == (R, C) and scales.shape == (R, nb), (codes.shape, scales.shape, ref.shape)
+    fin_all = np.isfinite(ref)
+    absr = np.where(fin_all, np.abs(ref), 0.0)
+    a_lo = float(np.maximum(absr - tol, 0.0).max()) if ref.size else 0.0
+    a_hi = float((absr + tol).max()) if ref.size else 0.0
+    assert amax >= a_lo * (1 - NVFP4_SLACK), f"{name}: amax {amax!r} below the oracle's lower bound {a_lo!r}"
+    if full_tensor:
+        assert amax <= a_hi * (1 + NVFP4_SLACK), f"{name}: amax {amax!r} above the oracle's upper bound {a_hi!r}"
+    s = o.nvfp4_tensor_scale(amax)
+    refb, tolb = ref.reshape(R, nb, 16), tol.reshape(R, nb, 16)
+    special = ~np.isfinite(refb).all(axis=2)
+    absb = np.where(np.isfinite(refb), np.abs(refb), 0.0)
+    bmax_lo = np.maximum(absb - tolb, 0.0).max(axis=2) * s / 6.0 * (1 - NVFP4_SLACK)
+    bmax_hi = (absb + tolb).max(axis=2) * s / 6.0 * (1 + NVFP4_SLACK)
+    k_lo, k_hi = e4m3_key(o.e4m3_encode(bmax_lo)), e4m3_key(o.e4m3_encode(bmax_hi))
+    k = e4m3_key(scales)
+    sp = np.flatnonzero(special & (scales != 0x7F))
+    assert sp.size == 0, f"{name}: block {np.unravel_index(sp[0], special.shape)} holds NaN/inf, scale {scales.flat[sp[0]]:#x}"
+    bad = np.flatnonzero(~special & ~((k_lo <= k) & (k <= k_hi)))
+    if bad.size:
+        i = bad[0]
+        raise AssertionError(f"{name}: {bad.size} block scales out of range; first block {np.unravel_index(i, k.shape)}: "
+                             f"code {scales.flat[i]:#x}, allowed keys [{k_lo.flat[i]}, {k_hi.flat[i]}]")
+    sb = np.where(special, 0.0, o.e4m3_decode(np.where(special, 0, scales)))
+    sbe = np.repeat(sb, 16, axis=1)
+    use = np.repeat(~special, 16, axis=1) & fin_all
+    zero_blk = use & (sbe == 0.0)
+    zb = np.flatnonzero(zero_blk & (e2m1_key(codes) != 0))
+    assert zb.size == 0, f"{name}: a block with scale 0 holds a nonzero code at flat {zb[0]}"
+    live = use & (sbe > 0.0)
+    ratio = np.where(live, s / np.where(sbe > 0.0, sbe, 1.0), 0.0)
+    with np.errstate(invalid="ignore"):
+        x_lo, x_hi = (ref - tol) * ratio, (ref + tol) * ratio
+        lo = e2m1_key(o.e2m1_encode(np.where(live, x_lo - np.abs(x_lo) * NVFP4_SLACK, 0.0)))
+        hi = e2m1_key(o.e2m1_encode(np.where(live, x_hi + np.abs(x_hi) * NVFP4_SLACK, 0.0)))
+    oc, osc, _ = o.nvfp4_quantize(np.where(fin_all, ref, np.nan), s_enc=s)
+    g = e2m1_key(codes)
+    bad = np.flatnonzero(live & ~((lo <= g) & (g <= hi)))
+    if bad.size:
+        i = bad[0]
+        raise AssertionError(f"{name}: {bad.size} codes out of range; first at flat {i}: code {codes.flat[i]:#x}, "
+                             f"oracle value {ref.flat[i]!r} x {ratio.flat[i]!r}, allowed keys "
+                             f"[{lo.flat[i]}, {hi.flat[i]}]")
+    same_scale = np.repeat(osc == scales, 16, axis=1)
+    exact = int(np.sum(live & same_scale & (g == e2m1_key(oc))))
+    total = int(np.sum(live))
+    assert total == 0 or exact >= min_exact * total, f"{name}: only {exact} of {total} codes equal the oracle's"
+    return {"codes": total, "exact": exact, "scales_equal": float(np.mean(osc == scales)) if osc.size else 1.0}

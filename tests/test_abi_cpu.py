@@ -58,7 +58,7 @@ def test_binding_covers_the_header_exactly():
 
 
 def test_version_and_status_strings(native_lib_path):
-    assert abi.situ_glu_abi_version() == abi.ABI_VERSION == 6
+    assert abi.situ_glu_abi_version() == abi.ABI_VERSION == 7
     assert abi.situ_glu_status_string(OK) == "SITU_OK"
     assert abi.situ_glu_status_string(MISAL) == "SITU_ERR_MISALIGNED"
     assert abi.situ_glu_status_string(99) == "SITU_ERR_UNKNOWN"
@@ -231,8 +231,8 @@ def test_defaults_match_the_pages():
 
 # ---- MXFP8 entry points: argument checks run before any CUDA call --------------
 
-MXD = 0x10000000   # fake 16-byte aligned device addresses for the outputs
-MXS = 0x18000000
+MXD = 0x80000000   # fake 16-byte aligned device addresses for the outputs, clear of the inputs
+MXS = 0x88000000
 
 
 def fwd_mx(**kw):
@@ -305,6 +305,50 @@ def test_bwd_mxfp8_argument_errors(name, kw, want, native_lib_path):
 def test_mxfp8_zero_tokens_is_a_no_op(native_lib_path):
     assert fwd_mx(tokens=0, y_data=None, y_scale=None) == OK
     assert bwd_mx(tokens=0, d_gate_up_data=None, d_gate_up_scale=None, d_rw=None) == OK
+
+
+# ---- NVFP4 forward: argument checks run before any CUDA call ---------------------
+
+AMX = 0x8C000000
+
+
+def fwd_nv(**kw):
+    a = dict(gate_up=GU, dtype=BF16, tokens=16, inter=64, gate_up_row_stride=128, rw=RW, rw_dtype=F32,
+             rw_mode=ROW, rw_stride=1, beta=4.0, has_linear_beta=1, linear_beta=25.0, y_data=MXD,
+             y_data_row_stride=32, y_scale=MXS, y_scale_row_stride=4, amax=AMX, amax_given=1, stream=None)
+    a.update(kw)
+    return abi.situ_glu_fwd_nvfp4(**a)
+
+
+NV_CASES = [
+    ("inter not a multiple of 16", dict(inter=40, gate_up_row_stride=80, y_data_row_stride=32,
+                                        y_scale_row_stride=4), INVALID),
+    ("per-column weights", dict(rw_mode=3), UNSUP),
+    ("per-element weights", dict(rw_mode=4, rw_stride=64), UNSUP),
+    ("scale pitch short", dict(y_scale_row_stride=3), INVALID),
+    ("data pitch short", dict(y_data_row_stride=16), INVALID),
+    ("data pitch not 16-byte", dict(y_data_row_stride=40), MISAL),
+    ("data misaligned", dict(y_data=MXD + 8), MISAL),
+    ("data NULL", dict(y_data=None), INVALID),
+    ("scale NULL", dict(y_scale=None), INVALID),
+    ("amax NULL", dict(amax=None), INVALID),
+    ("amax misaligned", dict(amax=AMX + 2), MISAL),
+    ("amax_given not 0 or 1", dict(amax_given=2), INVALID),
+    ("data overlaps gate_up", dict(y_data=GU), INVALID),
+    ("amax inside the scales", dict(amax=MXS + 8), INVALID),
+    ("scale overlaps data", dict(y_scale=MXD + 32), INVALID),
+    ("bad beta", dict(beta=-1.0), INVALID),
+    ("bad dtype", dict(dtype=7), INVALID),
+]
+
+
+@pytest.mark.parametrize("name,kw,want", NV_CASES, ids=[c[0] for c in NV_CASES])
+def test_fwd_nvfp4_argument_errors(name, kw, want, native_lib_path):
+    assert fwd_nv(**kw) == want, abi.situ_glu_last_error()
+
+
+def test_nvfp4_zero_tokens_with_given_amax_is_a_no_op(native_lib_path):
+    assert fwd_nv(tokens=0, y_data=None, y_scale=None) == OK
 
 
 # ---- FC1 grouped GEMM + SiTU-GLU: argument checks run before any CUDA call -------
