@@ -1371,37 +1371,70 @@ __device__ __forceinline__ void nvfp4_store_vec(const float2 (&y)[S::kPairs], bo
   const uint8_t sc = special ? static_cast<uint8_t>(0x7f)
                              : static_cast<uint8_t>(__nv_cvt_float_to_fp8(amax * s_enc / 6.0f, __NV_SATFINITE, __NV_E4M3));
   const float sb = special ? 0.0f : __half2float(__half(__nv_cvt_fp8_to_halfraw(sc, __NV_E4M3)));
-  const float r = sb > 0.0f ? s_enc / sb : 0.0f;
+  // S_enc / s_b to 2 ulp (s_b is at most 448): an extra rounding of a few
+  // 2^-24 that can only move an element sitting on an E2M1 midpoint
+  const float r = sb > 0.0f ? __fdividef(s_enc, sb) : 0.0f;
   float2 q[S::kPairs];
 #pragma unroll
   for (int p = 0; p < S::kPairs; ++p) q[p] = mul2(y[p], splat(r));
   if (!ACTIVE_ALWAYS && !active) return;
   if constexpr (S::kPairs == 4) {
-    *reinterpret_cast<uint32_t*>(data_row + j * 4) = e2m1x8(q);
+    st_stream_u32(data_row + j * 4, e2m1x8(q));
   } else {
-    *reinterpret_cast<uint16_t*>(data_row + j * 2) = static_cast<uint16_t>(e2m1x4(q));
+    const uint16_t v = static_cast<uint16_t>(e2m1x4(q));
+    asm volatile("st.global.cs.u16 [%0], %1;" ::"l"(data_row + j * 2), "h"(v) : "memory");
   }
   if (j % kLanes == 0) scale_row[j / kLanes] = sc;
 }
 
-// Output policies of the quantising forward: MXFP8 and NVFP4.
+// Output policies of the row pipeline below: MXFP8 codes, NVFP4 codes, or
+// the tensor maximum only.  State is what a thread carries across its rows
+// (the tensor scale, or its running maximum); finish() runs once per thread
+// at the end, with every lane of the warp present.
 struct MxQuant {
   using Out = MxOut;
+  using State = int;
+  __device__ __forceinline__ static State init(const Out&) { return 0; }
   template <typename S, bool ALL>
   __device__ __forceinline__ static void store(const float2 (&y)[S::kPairs], bool active, const Out& m, int64_t row,
-                                               int j, float) {
+                                               int j, State&) {
     mx_store_vec<S, ALL>(y, active, m.data + row * m.data_pitch, m.scale + row * m.scale_pitch, MxSlot<S>(j), m.rule);
   }
-  __device__ __forceinline__ static float tensor_param(const Out&) { return 0.0f; }
+  __device__ __forceinline__ static void finish(const Out&, const State&) {}
 };
 struct Nvfp4Quant {
   using Out = Nvfp4Out;
+  using State = float;  // S_enc
+  __device__ __forceinline__ static State init(const Out& m) { return nvfp4_tensor_scale(*m.amax); }
   template <typename S, bool ALL>
   __device__ __forceinline__ static void store(const float2 (&y)[S::kPairs], bool active, const Out& m, int64_t row,
-                                               int j, float s_enc) {
+                                               int j, State& s_enc) {
     nvfp4_store_vec<S, ALL>(y, active, m.data + row * m.data_pitch, m.scale + row * m.scale_pitch, j, s_enc);
   }
-  __device__ __forceinline__ static float tensor_param(const Out& m) { return nvfp4_tensor_scale(*m.amax); }
+  __device__ __forceinline__ static void finish(const Out&, const State&) {}
+};
+// The tensor's largest finite |Y| (NVFP4's tensor scale; NaN and infinite
+// elements only mark their own blocks): per-thread maxima of the fp32
+// results, a warp maximum, one integer atomicMax per warp on the float bits
+// (non-negative floats order as integers), so the result is order-free.
+struct AmaxOnly {
+  using Out = unsigned int*;
+  using State = float;
+  __device__ __forceinline__ static State init(const Out&) { return 0.0f; }
+  template <typename S, bool ALL>
+  __device__ __forceinline__ static void store(const float2 (&y)[S::kPairs], bool, const Out&, int64_t, int,
+                                               State& m) {
+#pragma unroll
+    for (int p = 0; p < S::kPairs; ++p) {  // inactive lanes hold zeros
+      const float ax = fabsf(y[p].x), ay = fabsf(y[p].y);
+      m = ax <= 3.402823466e38f ? fmaxf(m, ax) : m;  // false for NaN and infinity
+      m = ay <= 3.402823466e38f ? fmaxf(m, ay) : m;
+    }
+  }
+  __device__ __forceinline__ static void finish(const Out& amax_bits, const State& m) {
+    const unsigned int bits = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+    if ((threadIdx.x & 31) == 0 && bits != 0u) atomicMax(amax_bits, bits);
+  }
 };
 
 template <typename S, int GATE, bool HAS_LB>
@@ -1440,9 +1473,9 @@ __device__ __forceinline__ void fwd_quant_rows(const FwdArgs& a, const typename 
   const int nt = blockDim.x;
   const int j = threadIdx.x, j2 = j + nt;
   const bool one = ALL || j < a.vpr, two = ALL || j2 < a.vpr;
-  const float tp = Q::tensor_param(m);
+  typename Q::State st = Q::init(m);
   int64_t row = blockIdx.x;
-  if (row >= a.tokens) return;
+  if (row >= a.tokens) return;  // the whole block
   const uint4 z = make_uint4(0, 0, 0, 0);
   uint4 g0 = z, u0 = z, g1 = z, u1 = z;
   {
@@ -1477,13 +1510,14 @@ __device__ __forceinline__ void fwd_quant_rows(const FwdArgs& a, const typename 
     const float2 wbb = splat(w * a.c.bb);
     float2 y[kP];
     if (ALL || one) fwd_pairs<S, GATE, HAS_LB>(g0, u0, wbb, a.c, y); else zero_y<S>(y);
-    Q::template store<S, ALL>(y, one, m, row, j, tp);
+    Q::template store<S, ALL>(y, one, m, row, j, st);
     if (ALL || two) fwd_pairs<S, GATE, HAS_LB>(g1, u1, wbb, a.c, y); else zero_y<S>(y);
-    Q::template store<S, ALL>(y, two, m, row, j2, tp);
+    Q::template store<S, ALL>(y, two, m, row, j2, st);
     if (!more) break;
     row = next;
     g0 = ng0; u0 = nu0; g1 = ng1; u1 = nu1; w = nw;
   }
+  Q::finish(m, st);
 }
 
 template <typename S, int GATE, bool HAS_LB, class Q>
@@ -1498,7 +1532,7 @@ __global__ void __launch_bounds__(kMaxThreads) situ_glu_fwd_quant_kernel(const F
     fwd_quant_rows<S, GATE, HAS_LB, false, Q>(a, m);
     return;
   }
-  const float tp = Q::tensor_param(m);
+  typename Q::State st = Q::init(m);
   for (int64_t row = blockIdx.x; row < a.tokens; row += gridDim.x) {
     const char* gu = a.gate_up + row * a.gu_pitch;
     const float2 wbb = splat(load_rw(a.rw, row) * a.c.bb);
@@ -1511,36 +1545,10 @@ __global__ void __launch_bounds__(kMaxThreads) situ_glu_fwd_quant_kernel(const F
                                    a.c, y);
       else
         zero_y<S>(y);
-      Q::template store<S, false>(y, act, m, row, j, tp);
+      Q::template store<S, false>(y, act, m, row, j, st);
     }
   }
-}
-
-// The tensor's largest finite |Y| (NVFP4's tensor scale; NaN and infinite
-// elements only mark their own blocks): per-thread maxima of the fp32
-// results, a warp maximum, one integer atomicMax per warp on the float bits
-// (non-negative floats order as integers), so the result is order-free.
-template <typename S, int GATE, bool HAS_LB>
-__global__ void __launch_bounds__(kMaxThreads) situ_glu_amax_kernel(const FwdArgs a, unsigned int* amax_bits) {
-  constexpr int kP = S::kPairs;
-  float m = 0.0f;
-  for (int64_t row = blockIdx.x; row < a.tokens; row += gridDim.x) {
-    const char* gu = a.gate_up + row * a.gu_pitch;
-    const float2 wbb = splat(load_rw(a.rw, row) * a.c.bb);
-    for (int j = threadIdx.x; j < a.vpr; j += blockDim.x) {
-      float2 y[kP];
-      fwd_pairs<S, GATE, HAS_LB>(ld_stream(gu + j * kVecBytes), ld_stream(gu + a.half_bytes + j * kVecBytes), wbb, a.c,
-                                 y);
-#pragma unroll
-      for (int p = 0; p < kP; ++p) {
-        const float ax = fabsf(y[p].x), ay = fabsf(y[p].y);
-        m = ax <= 3.402823466e38f ? fmaxf(m, ax) : m;  // false for NaN and infinity
-        m = ay <= 3.402823466e38f ? fmaxf(m, ay) : m;
-      }
-    }
-  }
-  const unsigned int bits = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
-  if ((threadIdx.x & 31) == 0 && bits != 0u) atomicMax(amax_bits, bits);
+  Q::finish(m, st);
 }
 
 // Backward with MXFP8 d_gate_up: codes [tokens, 2 inter] (dG then dU), scales
@@ -2631,7 +2639,7 @@ auto pick_mx_gate(int gate) {
 }
 
 using FwdNvKernel = void (*)(FwdArgs, Nvfp4Out);
-using AmaxKernel = void (*)(FwdArgs, unsigned int*);
+using AmaxKernel = void (*)(FwdArgs, unsigned int*);  // situ_glu_fwd_quant_kernel<..., AmaxOnly>
 
 template <typename S, bool LB>
 FwdNvKernel pick_nv_gate(int gate) {
@@ -2645,10 +2653,10 @@ FwdNvKernel pick_nv_gate(int gate) {
 template <typename S, bool LB>
 AmaxKernel pick_amax_gate(int gate) {
   switch (gate) {
-    case kGateSquare: return situ_glu_amax_kernel<S, kGateSquare, LB>;
-    case kGateEqual: return situ_glu_amax_kernel<S, kGateEqual, LB>;
-    case kGateRoot: return situ_glu_amax_kernel<S, kGateRoot, LB>;
-    default: return situ_glu_amax_kernel<S, kGateGeneric, LB>;
+    case kGateSquare: return situ_glu_fwd_quant_kernel<S, kGateSquare, LB, AmaxOnly>;
+    case kGateEqual: return situ_glu_fwd_quant_kernel<S, kGateEqual, LB, AmaxOnly>;
+    case kGateRoot: return situ_glu_fwd_quant_kernel<S, kGateRoot, LB, AmaxOnly>;
+    default: return situ_glu_fwd_quant_kernel<S, kGateGeneric, LB, AmaxOnly>;
   }
 }
 FwdNvKernel pick_fwd_nv(situ_dtype_t dtype, int gate, bool lb) {
@@ -3627,9 +3635,12 @@ extern "C" situ_status_t situ_glu_fwd_nvfp4(const void* gate_up, situ_dtype_t dt
       !span_fits(tokens, y_scale_row_stride, inter / 16, 1) ||
       (rw_mode == SITU_RW_ROW && !span_fits(tokens, rw_stride, 1, elem_size(rw_dtype))))
     return fail(SITU_ERR_INVALID_ARG, "tensor extent overflows int64");
-  if (!aligned(gate_up, 16) || (gate_up_row_stride * es) % 16 != 0 || !aligned(y_data, 16) ||
-      y_data_row_stride % 16 != 0 || (rw_mode != SITU_RW_NONE && !aligned(rw, elem_size(rw_dtype))))
-    return fail(SITU_ERR_MISALIGNED, "gate_up / y_data base or row pitch not 16-byte aligned, or rw misaligned");
+  // a thread stores the codes of one 16-byte input vector: 4 bytes (bf16) or 2 (fp32)
+  if (!aligned(gate_up, 16) || (gate_up_row_stride * es) % 16 != 0 || !aligned(y_data, 4) ||
+      y_data_row_stride % 4 != 0 || (rw_mode != SITU_RW_NONE && !aligned(rw, elem_size(rw_dtype))))
+    return fail(SITU_ERR_MISALIGNED,
+                "gate_up base or row pitch not 16-byte aligned, y_data base or row pitch not 4-byte aligned, or rw "
+                "misaligned");
   const Span s_gu = matrix_span(gate_up, tokens, gate_up_row_stride, 2 * inter, es);
   const Span s_rw = weight_span(rw, rw_mode, tokens, rw_stride, inter, elem_size(rw_dtype));
   const Span s_d = matrix_span(y_data, tokens, y_data_row_stride, inter / 2, 1);

@@ -240,7 +240,7 @@ situ_status_t situ_glu_bwd_mxfp8(const void *gate_up, situ_dtype_t dtype, int64_
  *   y_data   [tokens, >= inter / 2] bytes of packed FP4 E2M1 codes of
  *            Y S_enc / s_b (nearest even, clamped to +-6), element 2k in the
  *            low nibble of byte k; row pitch y_data_row_stride bytes (a
- *            multiple of 16, base 16-byte aligned)
+ *            multiple of 4, base 4-byte aligned)
  *   amax     device fp32: A.  amax_given = 0: the library computes it first
  *            (a pass that reads gate_up once more) and writes it here;
  *            amax_given = 1: the caller's A is used (e.g. from an earlier

@@ -327,8 +327,8 @@ NV_CASES = [
     ("per-element weights", dict(rw_mode=4, rw_stride=64), UNSUP),
     ("scale pitch short", dict(y_scale_row_stride=3), INVALID),
     ("data pitch short", dict(y_data_row_stride=16), INVALID),
-    ("data pitch not 16-byte", dict(y_data_row_stride=40), MISAL),
-    ("data misaligned", dict(y_data=MXD + 8), MISAL),
+    ("data pitch not 4-byte", dict(y_data_row_stride=34), MISAL),
+    ("data misaligned", dict(y_data=MXD + 2), MISAL),
     ("data NULL", dict(y_data=None), INVALID),
     ("scale NULL", dict(y_scale=None), INVALID),
     ("amax NULL", dict(amax=None), INVALID),

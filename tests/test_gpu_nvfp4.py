@@ -53,7 +53,7 @@ def oracle_y(gu_h, rw_h, T, beta, lb):
     return o.fwd(gu_h, rw_h, beta, lb, rw_mode=mode)
 
 
-def run_nv(dev, dtype, T, I, beta, lb, kind, seed, pad=0, gu_h=None, given=None):
+def run_nv(dev, dtype, T, I, beta, lb, kind, seed, pad=0, gu_h=None, given=None, data_pitch=None):
     g_h, rw32 = nv_inputs(dtype, T, I, seed)
     gu_h = g_h if gu_h is None else gu_h
     rw_h, mode = rw_case(kind, rw32)
@@ -62,7 +62,7 @@ def run_nv(dev, dtype, T, I, beta, lb, kind, seed, pad=0, gu_h=None, given=None)
     rw_ptr = rw.data_ptr() if rw is not None else None
     rw_dt = (abi.SITU_DTYPE_BF16 if rw.dtype == torch.bfloat16 else abi.SITU_DTYPE_F32) if rw is not None else 1
     dt = abi.SITU_DTYPE_BF16 if dtype == "bf16" else abi.SITU_DTYPE_F32
-    data = Guarded(T, I // 2, I // 2 + 16 * pad, torch.uint8, dev)
+    data = Guarded(T, I // 2, data_pitch or I // 2 + 16 * pad, torch.uint8, dev)
     scale = Guarded(T, I // 16, I // 16 + pad, torch.uint8, dev)
     amax = torch.full((1,), float("nan") if given is None else given, dtype=torch.float32, device=dev)
     abi.check(abi.situ_glu_fwd_nvfp4(gu.data_ptr(), dt, T, I, gu.stride(0), rw_ptr, rw_dt, mode, 1, beta,
@@ -93,9 +93,11 @@ def test_nvfp4_parity(dtype, T, I, beta, lb, kind, cuda_device):
 
 
 def test_nvfp4_padded_pitches(cuda_device):
-    """Row pitches above the row (data +16 bytes, scales +1): guard bytes catch
-    any write into the padding."""
+    """Row pitches above the row (data +16 bytes, scales +1; and an 8-byte data
+    row, I = 16, with a 12-byte pitch): guard bytes catch any write into the
+    padding."""
     run_nv(cuda_device, "bf16", 67, 256, 4.0, 25.0, "row_f32", seed=5, pad=1)
+    run_nv(cuda_device, "f32", 9, 16, 4.0, 25.0, "row_f32", seed=5, data_pitch=12)
 
 
 def test_nvfp4_given_amax(cuda_device):
