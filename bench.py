@@ -13,8 +13,8 @@ d_gate_up and d_w), plus rows/s.
 --variant picks the form timed (default: per-row routing weights, the routed
 MoE form): per-column [I] or per-element [T, I] weights, or MXFP8 outputs
 (E4M3 codes + E8M0 scales for Y and d_gate_up, OCP rule), or an NVFP4 Y
-(E2M1 codes + E4M3 scales per 16 + the tensor maximum, bf16 backward; the
-quantising kernel is also timed alone for its roofline).  Algorithmic
+and d_gate_up (E2M1 codes + E4M3 scales per 16 + the tensor maximum; the
+quantising kernels are also timed alone, and the backward's is the roofline).  Algorithmic
 bytes follow the form (weights read, weight gradients written, one byte per
 code plus one per 32 codes).  --variant fc1 times the fused FC1 grouped GEMM
 + SiTU-GLU forward on the routed-MoE rows (hidden 7168, 8 local experts) in
@@ -125,8 +125,8 @@ def workload_config(wl, beta, l2_note, world, variant="row"):
         "variant": {"row": "per-row routing weights, bf16/fp32 outputs",
                     "col": "per-column routing weights [I]", "full": "per-element routing weights [T, I]",
                     "mxfp8": "per-row routing weights, MXFP8 Y and d_gate_up (E4M3 + E8M0 per 32, OCP rule)",
-                    "nvfp4": "per-row routing weights, NVFP4 Y (E2M1 + E4M3 per 16, tensor scale from this "
-                             "call's amax pass), bf16 d_gate_up"}[variant],
+                    "nvfp4": "per-row routing weights, NVFP4 Y and d_gate_up (E2M1 + E4M3 per 16, each tensor "
+                             "scale from its call's own amax pass)"}[variant],
         "workload": wl.describe(),
         "name": wl.name,
         "tokens": wl.tokens,
@@ -442,7 +442,7 @@ def variant_bytes(wl, variant: str):
     if variant == "mxfp8":
         return T * (2 * I * es + I + I // 32 + 4), T * (3 * I * es + 2 * I + 2 * I // 32 + 8)
     if variant == "nvfp4":
-        return T * (2 * I * es + I // 2 + I // 16 + 4), wl.bwd_bytes()
+        return T * (2 * I * es + I // 2 + I // 16 + 4), T * (3 * I * es + I + 2 * I // 16 + 8)
     return wl.fwd_bytes(), wl.bwd_bytes()
 
 
@@ -482,6 +482,7 @@ def cpu_oracle_rate(wl, beta, x, seconds: float, variant: str = "row"):
             o.mxfp8_quantize(np.concatenate([r.dg, r.du], axis=1))
         elif variant == "nvfp4":
             o.nvfp4_quantize(y)
+            o.nvfp4_quantize(np.concatenate([r.dg, r.du], axis=1))
         done += rows.size
         if time.perf_counter() - t0 >= seconds:
             break
@@ -522,6 +523,7 @@ def run_reference(args):
             o.mxfp8_quantize(np.concatenate([r.dg, r.du], axis=1))
         elif args.variant == "nvfp4":
             o.nvfp4_quantize(y)
+            o.nvfp4_quantize(np.concatenate([r.dg, r.du], axis=1))
 
     for _ in range(args.warmup):
         step()
@@ -937,8 +939,10 @@ def run_ours(args):
         y = torch.empty(T, I // 2, dtype=torch.uint8, device=dev)
         y_sc = torch.empty(T, I // 16, dtype=torch.float8_e4m3fn, device=dev)
         y_amax = torch.empty(1, dtype=torch.float32, device=dev)
-        d_gu = torch.empty(T, 2 * I, dtype=tdt, device=dev)
-        outputs = [y, y_sc, y_amax, d_gu, d_rw]
+        d_gu = torch.empty(T, I, dtype=torch.uint8, device=dev)
+        d_sc = torch.empty(T, 2 * I // 16, dtype=torch.float8_e4m3fn, device=dev)
+        d_amax = torch.empty(1, dtype=torch.float32, device=dev)
+        outputs = [y, y_sc, y_amax, d_gu, d_sc, d_amax, d_rw]
     else:
         y = torch.empty(T, I, dtype=tdt, device=dev)
         d_gu = torch.empty(T, 2 * I, dtype=tdt, device=dev)
@@ -961,7 +965,7 @@ def run_ours(args):
             pkg.situ_glu_fwd_nvfp4(gu, rw, beta, lb, data=y, scale=y_sc, amax_out=y_amax)
 
         def bwd():
-            pkg.situ_glu_bwd(gu, rw, go, beta, lb, d_gate_up=d_gu, d_rw=d_rw)
+            pkg.situ_glu_bwd_nvfp4(gu, rw, go, beta, lb, data=d_gu, scale=d_sc, amax_out=d_amax, d_rw=d_rw)
     else:
         def fwd():
             pkg.situ_glu_fwd(gu, rw, beta, lb, out=y)
@@ -1006,21 +1010,24 @@ def run_ours(args):
     total_ms, fwd_sum, bwd_sum = times.tolist()
     quant_us = None
     if variant == "nvfp4":
-        # the quantising kernel alone: the same call with the tensor maximum given
-        given = y_amax.clone()
-        qev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        # the quantising kernels alone: the same calls with the tensor maxima given
+        fgiven, bgiven = y_amax.clone(), d_amax.clone()
+        qev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
         torch.cuda.synchronize()
         for k in range(K):
             if flush:
                 flush_buf.zero_()
             qev[k][0].record(stream)
-            pkg.situ_glu_fwd_nvfp4(gu, rw, beta, lb, data=y, scale=y_sc, amax=given)
+            pkg.situ_glu_fwd_nvfp4(gu, rw, beta, lb, data=y, scale=y_sc, amax=fgiven)
             qev[k][1].record(stream)
+            pkg.situ_glu_bwd_nvfp4(gu, rw, go, beta, lb, data=d_gu, scale=d_sc, amax=bgiven, d_rw=d_rw)
+            qev[k][2].record(stream)
         torch.cuda.synchronize()
-        qt = torch.tensor([sum(e[0].elapsed_time(e[1]) for e in qev)], dtype=torch.float64, device=dev)
+        qt = torch.tensor([sum(e[0].elapsed_time(e[1]) for e in qev), sum(e[1].elapsed_time(e[2]) for e in qev)],
+                          dtype=torch.float64, device=dev)
         if world > 1:
             dist.all_reduce(qt, op=dist.ReduceOp.MAX)
-        quant_us = qt.item() / K * 1e3
+        quant_us = [v / K * 1e3 for v in qt.tolist()]
     ms_per_step = total_ms / K
     fwd_bytes, bwd_bytes = variant_bytes(wl, variant)
     step_bytes = fwd_bytes + bwd_bytes
@@ -1037,13 +1044,14 @@ def run_ours(args):
                 "situ_glu_bwd_kernel"),
         "col": ("situ_glu_fwd_ew_kernel", "situ_glu_bwd_ew_kernel"),
         "full": ("situ_glu_fwd_ew_kernel", "situ_glu_bwd_ew_kernel"),
-        "mxfp8": ("situ_glu_fwd_quant_kernel<MxQuant>", "situ_glu_bwd_mx_kernel"),
-        "nvfp4": ("situ_glu_amax_kernel+situ_glu_fwd_quant_kernel<Nvfp4Quant>", "situ_glu_bwd_kernel"),
+        "mxfp8": ("situ_glu_fwd_quant_kernel<MxQuant>", "situ_glu_bwd_quant_kernel<MxQuant>"),
+        "nvfp4": ("situ_glu_fwd_quant_kernel<AmaxOnly>+situ_glu_fwd_quant_kernel<Nvfp4Quant>",
+                  "situ_glu_bwd_quant_kernel<AmaxOnly>+situ_glu_bwd_quant_kernel<Nvfp4Quant>"),
     }[variant]
-    # per-column weights: plus the column finalize; NVFP4: the amax pass, the quantising pass, the backward
-    launches_per_step = {"col": 3, "nvfp4": 3}.get(variant, 2)
+    # per-column weights: plus the column finalize; NVFP4: an amax pass and a quantising pass each way
+    launches_per_step = {"col": 3, "nvfp4": 4}.get(variant, 2)
     traffic_key = wl.name if variant == "row" else f"{wl.name}/{variant}"
-    roof_kernel = "situ_glu_fwd_quant_kernel<Nvfp4Quant>" if variant == "nvfp4" else bwd_kernel
+    roof_kernel = "situ_glu_bwd_quant_kernel<Nvfp4Quant>" if variant == "nvfp4" else bwd_kernel
     traffic = recorded_traffic(roof_kernel, traffic_key)
 
     # End to end through the public API with host buffers: every step copies the
@@ -1080,7 +1088,7 @@ def run_ours(args):
         h2d = input_bytes
         d2h = sum(t.numel() * t.element_size() for t in outputs_h)
         api = {"mxfp8": "situ_glu_fwd_mxfp8/situ_glu_bwd_mxfp8",
-               "nvfp4": "situ_glu_fwd_nvfp4/situ_glu_bwd"}.get(variant, "situ_glu_fwd/situ_glu_bwd")
+               "nvfp4": "situ_glu_fwd_nvfp4/situ_glu_bwd_nvfp4"}.get(variant, "situ_glu_fwd/situ_glu_bwd")
         e2e = {"value": step_bytes * world / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": K2,
                "api": f"ffn_gated_activation_b200.{api} on pinned host copies"}
@@ -1103,15 +1111,19 @@ def run_ours(args):
                 "unit": "GB/s", "frac": bwd_gbs / peak, "peak_source": f"{peak_src} copy bandwidth",
                 "traffic": traffic}
     if quant_us is not None:
-        amax_bytes = T * (2 * I * (2 if wl.dtype == "bf16" else 4) + 4)
-        amax_us = max(fwd_us - quant_us, 1e-9)
-        q_gbs = fwd_bytes / quant_us / 1e3
-        kernels["situ_glu_amax_kernel"] = {"us": amax_us, "bytes": amax_bytes, "GB/s": amax_bytes / amax_us / 1e3,
-                                           "frac_of_measured_copy": amax_bytes / amax_us / 1e3 / peak,
-                                           "note": "the NVFP4 call's time less the quantising pass alone"}
-        kernels[roof_kernel] = {"us": quant_us, "bytes": fwd_bytes, "GB/s": q_gbs,
-                                "frac_of_measured_copy": q_gbs / peak,
-                                "note": "timed alone, tensor maximum given"}
+        es_ = 2 if wl.dtype == "bf16" else 4
+        passes = [("fwd", fwd_us, fwd_bytes, quant_us[0], T * (2 * I * es_ + 4)),
+                  ("bwd", bwd_us, bwd_bytes, quant_us[1], T * (3 * I * es_ + 4))]
+        for d, call_us, q_bytes, q_us, a_bytes in passes:
+            a_us = max(call_us - q_us, 1e-9)
+            kernels[f"situ_glu_{d}_quant_kernel<AmaxOnly>"] = {
+                "us": a_us, "bytes": a_bytes, "GB/s": a_bytes / a_us / 1e3,
+                "frac_of_measured_copy": a_bytes / a_us / 1e3 / peak,
+                "note": "the NVFP4 call's time less its quantising pass alone"}
+            kernels[f"situ_glu_{d}_quant_kernel<Nvfp4Quant>"] = {
+                "us": q_us, "bytes": q_bytes, "GB/s": q_bytes / q_us / 1e3,
+                "frac_of_measured_copy": q_bytes / q_us / 1e3 / peak, "note": "timed alone, tensor maximum given"}
+        q_gbs = bwd_bytes / quant_us[1] / 1e3
         roofline = {"bound": "hbm", "kernel": roof_kernel, "achieved": q_gbs, "peak": peak, "unit": "GB/s",
                     "frac": q_gbs / peak, "peak_source": f"{peak_src} copy bandwidth", "traffic": traffic}
 

@@ -23,6 +23,7 @@ from .functional import (
     situ_glu_fwd,
     situ_glu_fwd_mxfp8,
     situ_glu_fwd_nvfp4,
+    situ_glu_bwd_nvfp4,
     situlu,
     weighted_situ,
 )
@@ -42,6 +43,7 @@ __all__ = [
     "situ_glu_fwd_mxfp8",
     "situ_glu_bwd_mxfp8",
     "situ_glu_fwd_nvfp4",
+    "situ_glu_bwd_nvfp4",
     "situ_glu_fc1_fwd",
     "situ_glu_fc2_dgrad_bwd",
     "situlu",

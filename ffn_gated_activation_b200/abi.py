@@ -31,7 +31,7 @@ SITU_RW_FULL = 4
 SITU_MX_RULE_OCP = 0
 SITU_MX_RULE_CEIL = 1
 
-ABI_VERSION = 7
+ABI_VERSION = 8
 
 # Entry points declared in include/situ_glu.h: name -> (restype, argtypes).
 _I64, _INT, _DBL, _VP, _SZ = ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_void_p, ctypes.c_size_t
@@ -46,6 +46,8 @@ SIGNATURES = {
                                   _VP, _I64, _VP, _I64, _VP, _I64, _INT, _VP, _I64, _VP, _SZ, _VP]),
     "situ_glu_fwd_nvfp4": (_INT, [_VP, _INT, _I64, _I64, _I64, _VP, _INT, _INT, _I64, _DBL, _INT, _DBL,
                                   _VP, _I64, _VP, _I64, _VP, _INT, _VP]),
+    "situ_glu_bwd_nvfp4": (_INT, [_VP, _INT, _I64, _I64, _I64, _VP, _INT, _INT, _I64, _DBL, _INT, _DBL,
+                                  _VP, _I64, _VP, _I64, _VP, _I64, _VP, _INT, _VP, _I64, _VP, _SZ, _VP]),
     "situ_glu_fc1_fwd": (_INT, [_VP, _I64, _I64, _I64, _VP, _I64, _I64, _I64, _VP, _VP, _INT, _INT, _I64,
                                 _DBL, _INT, _DBL, _VP, _I64, _VP]),
     "situ_glu_fc2_dgrad_bwd": (_INT, [_VP, _I64, _I64, _I64, _VP, _I64, _I64, _I64, _VP, _VP, _I64, _VP, _INT, _INT,
@@ -148,6 +150,17 @@ def situ_glu_fwd_nvfp4(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw
     return lib().situ_glu_fwd_nvfp4(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode,
                                     rw_stride, beta, has_linear_beta, linear_beta, y_data, y_data_row_stride, y_scale,
                                     y_scale_row_stride, amax, amax_given, stream)
+
+
+def situ_glu_bwd_nvfp4(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride, beta,
+                       has_linear_beta, linear_beta, grad_out, grad_out_row_stride, d_gate_up_data,
+                       d_gate_up_data_row_stride, d_gate_up_scale, d_gate_up_scale_row_stride, amax, amax_given,
+                       d_rw, d_rw_stride, workspace, workspace_bytes, stream) -> int:
+    return lib().situ_glu_bwd_nvfp4(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode,
+                                    rw_stride, beta, has_linear_beta, linear_beta, grad_out, grad_out_row_stride,
+                                    d_gate_up_data, d_gate_up_data_row_stride, d_gate_up_scale,
+                                    d_gate_up_scale_row_stride, amax, amax_given, d_rw, d_rw_stride, workspace,
+                                    workspace_bytes, stream)
 
 
 def situ_glu_fc1_fwd(x, tokens, hidden, x_row_stride, w1, experts, inter, w1_row_stride, offsets, rw, rw_dtype,

@@ -1320,7 +1320,15 @@ struct Nvfp4Out {
   int64_t data_pitch;    // bytes
   uint8_t* scale;        // E4M3 block scales, [tokens, cols / 16]
   int64_t scale_pitch;   // bytes
-  const float* amax;     // device: the tensor's largest magnitude
+  const float* amax;     // device: the tensor's largest finite magnitude (read by the quantising pass)
+  float* amax_out;       // the same word, written by the amax pass (host-side use)
+};
+
+// An NVFP4 output of the backward: where its codes go, and whether the
+// caller gives the tensor maximum.
+struct Nvfp4Bwd {
+  Nvfp4Out out;
+  int amax_given;
 };
 
 // Two E2M1 codes of (lo, hi) in one byte, lo in the low nibble (cvt packs its
@@ -1387,6 +1395,21 @@ __device__ __forceinline__ void nvfp4_store_vec(const float2 (&y)[S::kPairs], bo
   if (j % kLanes == 0) scale_row[j / kLanes] = sc;
 }
 
+// Register budgets of the block-scaled backward, as CTAs of 256 threads per
+// SM.  MXFP8: three (at most 85 registers a thread), measured faster on B200
+// than two, the issue-bound MXFP8 backward gaining more from the extra warps
+// than it loses to the tighter budget.  The NVFP4 and amax-only passes: two
+// (at most 128 registers), measured faster than three (which spills).
+#ifndef SITU_BWD_MX_MIN_CTAS
+#define SITU_BWD_MX_MIN_CTAS 3
+#endif
+#ifndef SITU_BWD_NV_MIN_CTAS
+#define SITU_BWD_NV_MIN_CTAS 2
+#endif
+#ifndef SITU_BWD_AMAX_MIN_CTAS
+#define SITU_BWD_AMAX_MIN_CTAS 2
+#endif
+
 // Output policies of the row pipeline below: MXFP8 codes, NVFP4 codes, or
 // the tensor maximum only.  State is what a thread carries across its rows
 // (the tensor scale, or its running maximum); finish() runs once per thread
@@ -1394,22 +1417,43 @@ __device__ __forceinline__ void nvfp4_store_vec(const float2 (&y)[S::kPairs], bo
 struct MxQuant {
   using Out = MxOut;
   using State = int;
+  static constexpr int kBwdMinCtas = SITU_BWD_MX_MIN_CTAS;  // CTAs of 256 threads per SM, backward
   __device__ __forceinline__ static State init(const Out&) { return 0; }
   template <typename S, bool ALL>
   __device__ __forceinline__ static void store(const float2 (&y)[S::kPairs], bool active, const Out& m, int64_t row,
                                                int j, State&) {
     mx_store_vec<S, ALL>(y, active, m.data + row * m.data_pitch, m.scale + row * m.scale_pitch, MxSlot<S>(j), m.rule);
   }
+  // Backward: dG's codes and scales, then dU's half a row on.
+  template <typename S, bool ALL>
+  __device__ __forceinline__ static void store2(const float2 (&dg)[S::kPairs], const float2 (&du)[S::kPairs],
+                                                bool active, const Out& m, int64_t row, int j, int inter, State&) {
+    char* d = m.data + row * m.data_pitch;
+    uint8_t* sc = m.scale + row * m.scale_pitch;
+    const MxSlot<S> slot(j);
+    mx_store_vec<S, ALL>(dg, active, d, sc, slot, m.rule);
+    mx_store_vec<S, ALL>(du, active, d + inter, sc + inter / kMxBlock, slot, m.rule);
+  }
   __device__ __forceinline__ static void finish(const Out&, const State&) {}
 };
 struct Nvfp4Quant {
   using Out = Nvfp4Out;
   using State = float;  // S_enc
+  static constexpr int kBwdMinCtas = SITU_BWD_NV_MIN_CTAS;
   __device__ __forceinline__ static State init(const Out& m) { return nvfp4_tensor_scale(*m.amax); }
   template <typename S, bool ALL>
   __device__ __forceinline__ static void store(const float2 (&y)[S::kPairs], bool active, const Out& m, int64_t row,
                                                int j, State& s_enc) {
     nvfp4_store_vec<S, ALL>(y, active, m.data + row * m.data_pitch, m.scale + row * m.scale_pitch, j, s_enc);
+  }
+  template <typename S, bool ALL>
+  __device__ __forceinline__ static void store2(const float2 (&dg)[S::kPairs], const float2 (&du)[S::kPairs],
+                                                bool active, const Out& m, int64_t row, int j, int inter,
+                                                State& s_enc) {
+    char* d = m.data + row * m.data_pitch;
+    uint8_t* sc = m.scale + row * m.scale_pitch;
+    nvfp4_store_vec<S, ALL>(dg, active, d, sc, j, s_enc);
+    nvfp4_store_vec<S, ALL>(du, active, d + inter / 2, sc + inter / 16, j, s_enc);
   }
   __device__ __forceinline__ static void finish(const Out&, const State&) {}
 };
@@ -1420,6 +1464,7 @@ struct Nvfp4Quant {
 struct AmaxOnly {
   using Out = unsigned int*;
   using State = float;
+  static constexpr int kBwdMinCtas = SITU_BWD_AMAX_MIN_CTAS;
   __device__ __forceinline__ static State init(const Out&) { return 0.0f; }
   template <typename S, bool ALL>
   __device__ __forceinline__ static void store(const float2 (&y)[S::kPairs], bool, const Out&, int64_t, int,
@@ -1430,6 +1475,12 @@ struct AmaxOnly {
       m = ax <= 3.402823466e38f ? fmaxf(m, ax) : m;  // false for NaN and infinity
       m = ay <= 3.402823466e38f ? fmaxf(m, ay) : m;
     }
+  }
+  template <typename S, bool ALL>
+  __device__ __forceinline__ static void store2(const float2 (&dg)[S::kPairs], const float2 (&du)[S::kPairs],
+                                                bool active, const Out& o, int64_t row, int j, int, State& m) {
+    store<S, ALL>(dg, active, o, row, j, m);
+    store<S, ALL>(du, active, o, row, j, m);
   }
   __device__ __forceinline__ static void finish(const Out& amax_bits, const State& m) {
     const unsigned int bits = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
@@ -1551,10 +1602,11 @@ __global__ void __launch_bounds__(kMaxThreads) situ_glu_fwd_quant_kernel(const F
   Q::finish(m, st);
 }
 
-// Backward with MXFP8 d_gate_up: codes [tokens, 2 inter] (dG then dU), scales
-// [tokens, 2 inter / 32]; the routing-weight gradient as in the per-row kernel.
+// Backward with a block-scaled d_gate_up (MXFP8 or NVFP4; dG's codes and
+// scales, then dU's), or the tensor maximum of d_gate_up only (the NVFP4
+// amax pass); the routing-weight gradient as in the per-row kernel.
 template <typename S, int GATE, bool HAS_LB>
-__device__ __forceinline__ void bwd_mx_finish_row(const BwdArgs& a, int64_t row, float2 acc, float* red) {
+__device__ __forceinline__ void bwd_quant_finish_row(const BwdArgs& a, int64_t row, float2 acc, float* red) {
   if (a.want_drw) {  // uniform over the launch
     const float total = block_sum(acc.x + acc.y, red) * bwd_dw_scale(a.c);
     if (threadIdx.x == 0) {
@@ -1566,11 +1618,11 @@ __device__ __forceinline__ void bwd_mx_finish_row(const BwdArgs& a, int64_t row,
   }
 }
 
-// One vector's dG and dU, quantised.  dU's codes and scales sit half a row on.
-template <typename S, int GATE, bool HAS_LB, bool ALL>
-__device__ __forceinline__ void bwd_mx_vec(const uint4& g, const uint4& u, const uint4& o, bool act, float2 k,
-                                           const Coeffs& c, char* drow, uint8_t* srow, int inter,
-                                           const MxSlot<S>& slot, int rule, float2& acc) {
+// One vector's dG and dU, handed to the output policy.
+template <typename S, int GATE, bool HAS_LB, bool ALL, class Q>
+__device__ __forceinline__ void bwd_quant_vec(const uint4& g, const uint4& u, const uint4& o, bool act, float2 k,
+                                              const Coeffs& c, const typename Q::Out& m, int64_t row, int j,
+                                              int inter, typename Q::State& st, float2& acc) {
   constexpr int kP = S::kPairs;
   float2 dg[kP], du[kP];
   if (ALL || act) {
@@ -1579,22 +1631,21 @@ __device__ __forceinline__ void bwd_mx_vec(const uint4& g, const uint4& u, const
     zero_y<S>(dg);
     zero_y<S>(du);
   }
-  mx_store_vec<S, ALL>(dg, act, drow, srow, slot, rule);
-  mx_store_vec<S, ALL>(du, act, drow + inter, srow + inter / kMxBlock, slot, rule);
+  Q::template store2<S, ALL>(dg, du, act, m, row, j, inter, st);
 }
 
-template <typename S, int GATE, bool HAS_LB, bool ALL>
-__device__ __forceinline__ void bwd_mx_rows(const BwdArgs& a, const MxOut& m, float (*red)[kMaxThreads / 32]) {
+template <typename S, int GATE, bool HAS_LB, bool ALL, class Q>
+__device__ __forceinline__ void bwd_quant_rows(const BwdArgs& a, const typename Q::Out& m,
+                                               float (*red)[kMaxThreads / 32]) {
   constexpr int kP = S::kPairs;
   const int nt = blockDim.x;
   const int inter = a.half_bytes / kVecBytes * (2 * kP);  // elements per half row
   const int j = threadIdx.x, j2 = j + nt;
   const bool one = ALL || j < a.vpr, two = ALL || j2 < a.vpr;
-  const MxSlot<S> s0(j), s1(j2);
-  const int rule = m.rule;
+  typename Q::State st = Q::init(m);
   int parity = 0;
   int64_t row = blockIdx.x;
-  if (row >= a.tokens) return;
+  if (row >= a.tokens) return;  // the whole block
   const uint4 z = make_uint4(0, 0, 0, 0);
   uint4 g0 = z, u0 = z, o0 = z, g1 = z, u1 = z, o1 = z;
   {
@@ -1633,60 +1684,53 @@ __device__ __forceinline__ void bwd_mx_rows(const BwdArgs& a, const MxOut& m, fl
       nw = load_rw(a.rw, next);
     }
     const float2 k = bwd_row_consts<HAS_LB>(w, a.c);
-    char* drow = m.data + row * m.data_pitch;
-    uint8_t* srow = m.scale + row * m.scale_pitch;
     float2 acc = make_float2(0.0f, 0.0f);
-    bwd_mx_vec<S, GATE, HAS_LB, ALL>(g0, u0, o0, one, k, a.c, drow, srow, inter, s0, rule, acc);
-    bwd_mx_vec<S, GATE, HAS_LB, ALL>(g1, u1, o1, two, k, a.c, drow, srow, inter, s1, rule, acc);
-    bwd_mx_finish_row<S, GATE, HAS_LB>(a, row, acc, red[parity]);
+    bwd_quant_vec<S, GATE, HAS_LB, ALL, Q>(g0, u0, o0, one, k, a.c, m, row, j, inter, st, acc);
+    bwd_quant_vec<S, GATE, HAS_LB, ALL, Q>(g1, u1, o1, two, k, a.c, m, row, j2, inter, st, acc);
+    bwd_quant_finish_row<S, GATE, HAS_LB>(a, row, acc, red[parity]);
     parity ^= 1;
     if (!more) break;
     row = next;
     g0 = ng0; u0 = nu0; o0 = no0; g1 = ng1; u1 = nu1; o1 = no1; w = nw;
   }
+  Q::finish(m, st);
 }
 
-// Three CTAs of 256 threads per SM (at most 85 registers a thread): measured
-// faster on B200 than two, the issue-bound MXFP8 backward gaining more from
-// the extra warps than it loses to the tighter register budget.
-#ifndef SITU_BWD_MX_MIN_CTAS
-#define SITU_BWD_MX_MIN_CTAS 3
-#endif
-#define SITU_BWD_MX_BOUNDS __launch_bounds__(kMaxThreads, SITU_BWD_MX_MIN_CTAS)
 
-template <typename S, int GATE, bool HAS_LB>
-__global__ void SITU_BWD_MX_BOUNDS situ_glu_bwd_mx_kernel(const BwdArgs a, const MxOut m) {
+template <typename S, int GATE, bool HAS_LB, class Q>
+__global__ void __launch_bounds__(kMaxThreads, Q::kBwdMinCtas)
+    situ_glu_bwd_quant_kernel(const BwdArgs a, const typename Q::Out m) {
   __shared__ float red[2][kMaxThreads / 32];
   const int nt = blockDim.x;
   if (PipelineRows<S, true>::value && a.vpr == 2 * nt) {
-    bwd_mx_rows<S, GATE, HAS_LB, true>(a, m, red);
+    bwd_quant_rows<S, GATE, HAS_LB, true, Q>(a, m, red);
     return;
   }
   if (PipelineRows<S, true>::value && a.vpr < 2 * nt) {
-    bwd_mx_rows<S, GATE, HAS_LB, false>(a, m, red);
+    bwd_quant_rows<S, GATE, HAS_LB, false, Q>(a, m, red);
     return;
   }
   const int inter = a.half_bytes / kVecBytes * (2 * S::kPairs);
+  typename Q::State st = Q::init(m);
   int parity = 0;
   for (int64_t row = blockIdx.x; row < a.tokens; row += gridDim.x) {
     const char* gu = a.gate_up + row * a.gu_pitch;
     const char* go_row = a.grad_out + row * a.go_pitch;
     const float2 k = bwd_row_consts<HAS_LB>(load_rw(a.rw, row), a.c);
-    char* drow = m.data + row * m.data_pitch;
-    uint8_t* srow = m.scale + row * m.scale_pitch;
     float2 acc = make_float2(0.0f, 0.0f);
     for (int jb = 0; jb < a.vpr; jb += nt) {  // uniform trip count: every lane reaches the shuffles
       const int j = jb + threadIdx.x;
       const bool act = j < a.vpr;
       const uint4 z = make_uint4(0, 0, 0, 0);
-      bwd_mx_vec<S, GATE, HAS_LB, false>(act ? ld_stream(gu + j * kVecBytes) : z,
-                                         act ? ld_stream(gu + a.half_bytes + j * kVecBytes) : z,
-                                         act ? ld_stream(go_row + j * kVecBytes) : z, act, k, a.c, drow, srow,
-                                         inter, MxSlot<S>(j), m.rule, acc);
+      bwd_quant_vec<S, GATE, HAS_LB, false, Q>(act ? ld_stream(gu + j * kVecBytes) : z,
+                                               act ? ld_stream(gu + a.half_bytes + j * kVecBytes) : z,
+                                               act ? ld_stream(go_row + j * kVecBytes) : z, act, k, a.c, m, row, j,
+                                               inter, st, acc);
     }
-    bwd_mx_finish_row<S, GATE, HAS_LB>(a, row, acc, red[parity]);
+    bwd_quant_finish_row<S, GATE, HAS_LB>(a, row, acc, red[parity]);
     parity ^= 1;
   }
+  Q::finish(m, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -2616,68 +2660,31 @@ BwdKernel pick_bwd(situ_dtype_t dtype, int gate, bool lb) {
   return lb ? pick_bwd_gate<F32, true>(gate) : pick_bwd_gate<F32, false>(gate);
 }
 
-using FwdMxKernel = void (*)(FwdArgs, MxOut);
-using BwdMxKernel = void (*)(BwdArgs, MxOut);
-
-template <typename S, bool LB, bool BWD>
-auto pick_mx_gate(int gate) {
+// Kernel of a block-scaled (or amax-only) pass for the dtype, gate form and
+// linear-beta flag: the forward's or the backward's row loop with policy Q.
+template <typename S, bool LB, class Q, bool BWD>
+auto pick_quant_gate(int gate) {
   if constexpr (BWD) {
     switch (gate) {
-      case kGateSquare: return situ_glu_bwd_mx_kernel<S, kGateSquare, LB>;
-      case kGateEqual: return situ_glu_bwd_mx_kernel<S, kGateEqual, LB>;
-      case kGateRoot: return situ_glu_bwd_mx_kernel<S, kGateRoot, LB>;
-      default: return situ_glu_bwd_mx_kernel<S, kGateGeneric, LB>;
+      case kGateSquare: return situ_glu_bwd_quant_kernel<S, kGateSquare, LB, Q>;
+      case kGateEqual: return situ_glu_bwd_quant_kernel<S, kGateEqual, LB, Q>;
+      case kGateRoot: return situ_glu_bwd_quant_kernel<S, kGateRoot, LB, Q>;
+      default: return situ_glu_bwd_quant_kernel<S, kGateGeneric, LB, Q>;
     }
   } else {
     switch (gate) {
-      case kGateSquare: return situ_glu_fwd_quant_kernel<S, kGateSquare, LB, MxQuant>;
-      case kGateEqual: return situ_glu_fwd_quant_kernel<S, kGateEqual, LB, MxQuant>;
-      case kGateRoot: return situ_glu_fwd_quant_kernel<S, kGateRoot, LB, MxQuant>;
-      default: return situ_glu_fwd_quant_kernel<S, kGateGeneric, LB, MxQuant>;
+      case kGateSquare: return situ_glu_fwd_quant_kernel<S, kGateSquare, LB, Q>;
+      case kGateEqual: return situ_glu_fwd_quant_kernel<S, kGateEqual, LB, Q>;
+      case kGateRoot: return situ_glu_fwd_quant_kernel<S, kGateRoot, LB, Q>;
+      default: return situ_glu_fwd_quant_kernel<S, kGateGeneric, LB, Q>;
     }
   }
 }
-
-using FwdNvKernel = void (*)(FwdArgs, Nvfp4Out);
-using AmaxKernel = void (*)(FwdArgs, unsigned int*);  // situ_glu_fwd_quant_kernel<..., AmaxOnly>
-
-template <typename S, bool LB>
-FwdNvKernel pick_nv_gate(int gate) {
-  switch (gate) {
-    case kGateSquare: return situ_glu_fwd_quant_kernel<S, kGateSquare, LB, Nvfp4Quant>;
-    case kGateEqual: return situ_glu_fwd_quant_kernel<S, kGateEqual, LB, Nvfp4Quant>;
-    case kGateRoot: return situ_glu_fwd_quant_kernel<S, kGateRoot, LB, Nvfp4Quant>;
-    default: return situ_glu_fwd_quant_kernel<S, kGateGeneric, LB, Nvfp4Quant>;
-  }
-}
-template <typename S, bool LB>
-AmaxKernel pick_amax_gate(int gate) {
-  switch (gate) {
-    case kGateSquare: return situ_glu_fwd_quant_kernel<S, kGateSquare, LB, AmaxOnly>;
-    case kGateEqual: return situ_glu_fwd_quant_kernel<S, kGateEqual, LB, AmaxOnly>;
-    case kGateRoot: return situ_glu_fwd_quant_kernel<S, kGateRoot, LB, AmaxOnly>;
-    default: return situ_glu_fwd_quant_kernel<S, kGateGeneric, LB, AmaxOnly>;
-  }
-}
-FwdNvKernel pick_fwd_nv(situ_dtype_t dtype, int gate, bool lb) {
-  if (dtype == SITU_DTYPE_BF16) return lb ? pick_nv_gate<Bf16, true>(gate) : pick_nv_gate<Bf16, false>(gate);
-  return lb ? pick_nv_gate<F32, true>(gate) : pick_nv_gate<F32, false>(gate);
-}
-AmaxKernel pick_amax(situ_dtype_t dtype, int gate, bool lb) {
-  if (dtype == SITU_DTYPE_BF16) return lb ? pick_amax_gate<Bf16, true>(gate) : pick_amax_gate<Bf16, false>(gate);
-  return lb ? pick_amax_gate<F32, true>(gate) : pick_amax_gate<F32, false>(gate);
-}
-
-FwdMxKernel pick_fwd_mx(situ_dtype_t dtype, int gate, bool lb) {
+template <class Q, bool BWD>
+auto pick_quant(situ_dtype_t dtype, int gate, bool lb) {
   if (dtype == SITU_DTYPE_BF16)
-    return lb ? pick_mx_gate<Bf16, true, false>(gate) : pick_mx_gate<Bf16, false, false>(gate);
-  return lb ? pick_mx_gate<F32, true, false>(gate) : pick_mx_gate<F32, false, false>(gate);
-}
-
-BwdMxKernel pick_bwd_mx(situ_dtype_t dtype, int gate, bool lb) {
-  if (dtype == SITU_DTYPE_BF16)
-    return lb ? pick_mx_gate<Bf16, true, true>(gate) : pick_mx_gate<Bf16, false, true>(gate);
-  return lb ? pick_mx_gate<F32, true, true>(gate) : pick_mx_gate<F32, false, true>(gate);
+    return lb ? pick_quant_gate<Bf16, true, Q, BWD>(gate) : pick_quant_gate<Bf16, false, Q, BWD>(gate);
+  return lb ? pick_quant_gate<F32, true, Q, BWD>(gate) : pick_quant_gate<F32, false, Q, BWD>(gate);
 }
 
 // Argument checks of an MXFP8 output of `cols` columns per row.
@@ -2705,6 +2712,35 @@ situ_status_t check_mx_buffers(const MxOut& m, int64_t tokens, int64_t cols) {
   const Span sd = matrix_span(m.data, tokens, m.data_pitch, cols, 1);
   const Span ss = matrix_span(m.scale, tokens, m.scale_pitch, cols / kMxBlock, 1);
   if (overlap(sd, ss)) return fail(SITU_ERR_INVALID_ARG, "MXFP8 data overlaps its scales");
+  return SITU_OK;
+}
+
+// Argument checks of an NVFP4 output of `cols` columns per row.
+situ_status_t check_nv_args(const Nvfp4Bwd& n, int64_t inter, int64_t cols, situ_rw_mode_t rw_mode) {
+  if (inter % 16 != 0)
+    return fail(SITU_ERR_INVALID_ARG, "NVFP4 outputs need inter a multiple of 16, got %lld", (long long)inter);
+  if (rw_mode == SITU_RW_COL || rw_mode == SITU_RW_FULL)
+    return fail(SITU_ERR_UNSUPPORTED, "NVFP4 outputs take per-row, broadcast or no routing weights");
+  if (n.amax_given != 0 && n.amax_given != 1) return fail(SITU_ERR_INVALID_ARG, "amax_given must be 0 or 1");
+  if (n.out.data_pitch < cols / 2 || n.out.scale_pitch < cols / 16)
+    return fail(SITU_ERR_INVALID_ARG, "NVFP4 data or scale row pitch shorter than a row");
+  if (n.out.amax_out == nullptr) return fail(SITU_ERR_INVALID_ARG, "amax is NULL");
+  if (!aligned(n.out.amax_out, 4)) return fail(SITU_ERR_MISALIGNED, "amax not 4-byte aligned");
+  return SITU_OK;
+}
+
+// Pointer, extent and alignment checks of an NVFP4 output (tokens > 0).
+situ_status_t check_nv_buffers(const Nvfp4Bwd& n, int64_t tokens, int64_t cols) {
+  if (n.out.data == nullptr || n.out.scale == nullptr)
+    return fail(SITU_ERR_INVALID_ARG, "NVFP4 data or scale is NULL");
+  if (!span_fits(tokens, n.out.data_pitch, cols / 2, 1) || !span_fits(tokens, n.out.scale_pitch, cols / 16, 1))
+    return fail(SITU_ERR_INVALID_ARG, "tensor extent overflows int64");
+  // a thread stores the codes of one 16-byte input vector: 4 bytes (bf16) or 2 (fp32)
+  if (!aligned(n.out.data, 4) || n.out.data_pitch % 4 != 0)
+    return fail(SITU_ERR_MISALIGNED, "NVFP4 data base or row pitch not 4-byte aligned");
+  const Span sd = matrix_span(n.out.data, tokens, n.out.data_pitch, cols / 2, 1);
+  const Span ss = matrix_span(n.out.scale, tokens, n.out.scale_pitch, cols / 16, 1);
+  if (overlap(sd, ss)) return fail(SITU_ERR_INVALID_ARG, "NVFP4 data overlaps its scales");
   return SITU_OK;
 }
 
@@ -2790,7 +2826,7 @@ situ_status_t fwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
   if (rw_mode == SITU_RW_NONE) a.rw.bf16 = 0;
 
   if (mx != nullptr) {
-    FwdMxKernel k = pick_fwd_mx(dtype, gate, has_linear_beta != 0);
+    auto k = pick_quant<MxQuant, false>(dtype, gate, has_linear_beta != 0);
     const int threads = choose_threads(a.vpr);
     int grid = 0;
     st = launch_grid(reinterpret_cast<const void*>(k), threads, 0, tokens, &grid);
@@ -2953,7 +2989,7 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
                         int64_t rw_stride, double beta, int has_linear_beta, double linear_beta,
                         const void* grad_out, int64_t grad_out_row_stride, void* d_gate_up,
                         int64_t d_gate_up_row_stride, void* d_rw, int64_t d_rw_stride, void* workspace,
-                        size_t workspace_bytes, const MxOut* mx, void* stream) {
+                        size_t workspace_bytes, const MxOut* mx, const Nvfp4Bwd* nv, void* stream) {
   tl_last_error[0] = '\0';
   Coeffs c;
   int gate = kGateGeneric;
@@ -2963,6 +2999,9 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
   if (grad_out_row_stride < inter) return fail(SITU_ERR_INVALID_ARG, "grad_out_row_stride < inter");
   if (mx != nullptr) {
     st = check_mx_args(*mx, inter, 2 * inter, rw_mode);
+    if (st != SITU_OK) return st;
+  } else if (nv != nullptr) {
+    st = check_nv_args(*nv, inter, 2 * inter, rw_mode);
     if (st != SITU_OK) return st;
   } else if (d_gate_up_row_stride < 2 * inter) {
     return fail(SITU_ERR_INVALID_ARG, "d_gate_up_row_stride < 2 * inter");
@@ -2975,8 +3014,12 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
     return fail(SITU_ERR_INVALID_ARG, "d_rw_stride < inter (full weights)");
   const size_t ws_needed = situ_glu_bwd_workspace_bytes(tokens, inter, rw_mode, want_drw ? 1 : 0);
   if (tokens == 0) {
-    // The gradient of a broadcast weight over zero rows is zero; nothing else
-    // is written.  That store is the one piece of work an empty call does.
+    // The gradient of a broadcast weight over zero rows is zero, and so is the
+    // maximum of an empty NVFP4 gradient; nothing else is written.
+    if (nv != nullptr && !nv->amax_given) {
+      cudaError_t err = cudaMemsetAsync(nv->out.amax_out, 0, sizeof(float), static_cast<cudaStream_t>(stream));
+      if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
+    }
     if (want_drw && (rw_mode == SITU_RW_SCALAR || rw_mode == SITU_RW_COL)) {
       if (!aligned(d_rw, elem_size(rw_dtype))) return fail(SITU_ERR_MISALIGNED, "d_rw not aligned");
       const size_t n = rw_mode == SITU_RW_COL ? static_cast<size_t>(inter) : 1;
@@ -2985,7 +3028,8 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
     }
     return SITU_OK;
   }
-  if (gate_up == nullptr || grad_out == nullptr || (mx == nullptr && d_gate_up == nullptr))
+  const bool native = mx == nullptr && nv == nullptr;
+  if (gate_up == nullptr || grad_out == nullptr || (native && d_gate_up == nullptr))
     return fail(SITU_ERR_INVALID_ARG, "gate_up, grad_out or d_gate_up is NULL");
   const int es = elem_size(dtype);
   const int rw_es = rw_mode == SITU_RW_NONE ? 4 : elem_size(rw_dtype);
@@ -2993,8 +3037,12 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
     st = check_mx_buffers(*mx, tokens, 2 * inter);
     if (st != SITU_OK) return st;
   }
+  if (nv != nullptr) {
+    st = check_nv_buffers(*nv, tokens, 2 * inter);
+    if (st != SITU_OK) return st;
+  }
   if (!span_fits(tokens, gate_up_row_stride, 2 * inter, es) || !span_fits(tokens, grad_out_row_stride, inter, es) ||
-      (mx == nullptr && !span_fits(tokens, d_gate_up_row_stride, 2 * inter, es)) ||
+      (native && !span_fits(tokens, d_gate_up_row_stride, 2 * inter, es)) ||
       (rw_mode == SITU_RW_ROW && !span_fits(tokens, rw_stride, 1, rw_es)) ||
       (want_drw && rw_mode == SITU_RW_ROW && !span_fits(tokens, d_rw_stride, 1, rw_es)) ||
       (rw_mode == SITU_RW_FULL && !span_fits(tokens, rw_stride, inter, rw_es)) ||
@@ -3002,7 +3050,7 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
     return fail(SITU_ERR_INVALID_ARG, "tensor extent overflows int64");
   if (!aligned(gate_up, 16) || !aligned(grad_out, 16) || (gate_up_row_stride * es) % 16 != 0 ||
       (grad_out_row_stride * es) % 16 != 0 ||
-      (mx == nullptr && (!aligned(d_gate_up, 16) || (d_gate_up_row_stride * es) % 16 != 0)))
+      (native && (!aligned(d_gate_up, 16) || (d_gate_up_row_stride * es) % 16 != 0)))
     return fail(SITU_ERR_MISALIGNED, "gate_up/grad_out/d_gate_up base or row pitch not 16-byte aligned");
   if (rw_mode != SITU_RW_NONE && !aligned(rw, rw_es)) return fail(SITU_ERR_MISALIGNED, "rw not aligned");
   if (want_drw && !aligned(d_rw, rw_es)) return fail(SITU_ERR_MISALIGNED, "d_rw not aligned");
@@ -3020,25 +3068,34 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
   // Aliasing: no output may overlap an input or another output.
   const Span s_gu = matrix_span(gate_up, tokens, gate_up_row_stride, 2 * inter, es);
   const Span s_go = matrix_span(grad_out, tokens, grad_out_row_stride, inter, es);
-  const Span s_dgu = mx ? matrix_span(mx->data, tokens, mx->data_pitch, 2 * inter, 1)
-                        : matrix_span(d_gate_up, tokens, d_gate_up_row_stride, 2 * inter, es);
+  const Span s_dgu = mx   ? matrix_span(mx->data, tokens, mx->data_pitch, 2 * inter, 1)
+                    : nv ? matrix_span(nv->out.data, tokens, nv->out.data_pitch, inter, 1)
+                         : matrix_span(d_gate_up, tokens, d_gate_up_row_stride, 2 * inter, es);
   const Span s_rw = weight_span(rw, rw_mode, tokens, rw_stride, inter, rw_es);
   if (overlap(s_dgu, s_gu) || overlap(s_dgu, s_go) || overlap(s_dgu, s_rw))
     return fail(SITU_ERR_INVALID_ARG, "d_gate_up overlaps an input");
-  const Span s_sc = mx ? matrix_span(mx->scale, tokens, mx->scale_pitch, 2 * inter / kMxBlock, 1) : Span{0, 0};
-  if (mx != nullptr && (overlap(s_sc, s_gu) || overlap(s_sc, s_go) || overlap(s_sc, s_rw)))
-    return fail(SITU_ERR_INVALID_ARG, "MXFP8 scales overlap an input");
+  const Span s_sc = mx   ? matrix_span(mx->scale, tokens, mx->scale_pitch, 2 * inter / kMxBlock, 1)
+                    : nv ? matrix_span(nv->out.scale, tokens, nv->out.scale_pitch, 2 * inter / 16, 1)
+                         : Span{0, 0};
+  if (!native && (overlap(s_sc, s_gu) || overlap(s_sc, s_go) || overlap(s_sc, s_rw)))
+    return fail(SITU_ERR_INVALID_ARG, "block scales overlap an input");
+  const Span s_am = nv ? Span{reinterpret_cast<uintptr_t>(nv->out.amax_out),
+                              reinterpret_cast<uintptr_t>(nv->out.amax_out) + sizeof(float)}
+                       : Span{0, 0};
+  if (nv != nullptr && (overlap(s_am, s_gu) || overlap(s_am, s_go) || overlap(s_am, s_rw) ||
+                        overlap(s_am, s_dgu) || overlap(s_am, s_sc)))
+    return fail(SITU_ERR_INVALID_ARG, "amax overlaps another tensor");
   Span s_drw = {0, 0};
   if (want_drw) {
     s_drw = weight_span(d_rw, rw_mode, tokens, d_rw_stride, inter, rw_es);
     if (overlap(s_drw, s_gu) || overlap(s_drw, s_go) || overlap(s_drw, s_rw) || overlap(s_drw, s_dgu) ||
-        overlap(s_drw, s_sc))
+        overlap(s_drw, s_sc) || overlap(s_drw, s_am))
       return fail(SITU_ERR_INVALID_ARG, "d_rw overlaps another tensor");
   }
   if (ws_needed > 0) {
     const Span s_ws = {reinterpret_cast<uintptr_t>(workspace), reinterpret_cast<uintptr_t>(workspace) + ws_needed};
     if (overlap(s_ws, s_gu) || overlap(s_ws, s_go) || overlap(s_ws, s_rw) || overlap(s_ws, s_dgu) ||
-        overlap(s_ws, s_drw) || overlap(s_ws, s_sc))
+        overlap(s_ws, s_drw) || overlap(s_ws, s_sc) || overlap(s_ws, s_am))
       return fail(SITU_ERR_INVALID_ARG, "workspace overlaps a tensor");
   }
 
@@ -3103,13 +3160,34 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (mx != nullptr) {
-    BwdMxKernel k = pick_bwd_mx(dtype, gate, has_linear_beta != 0);
+    auto k = pick_quant<MxQuant, true>(dtype, gate, has_linear_beta != 0);
     const int threads = choose_threads(a.vpr);
     int grid = 0;
     st = launch_grid(reinterpret_cast<const void*>(k), threads, 0, tokens, &grid);
     if (st != SITU_OK) return st;
     k<<<grid, threads, 0, s>>>(a, *mx);
     st = check_launch("situ_glu_bwd_mxfp8");
+  } else if (nv != nullptr) {
+    const int threads = choose_threads(a.vpr);
+    if (!nv->amax_given) {  // the tensor maximum of d_gate_up first: a pass without stores or d_w
+      cudaError_t err = cudaMemsetAsync(nv->out.amax_out, 0, sizeof(float), s);
+      if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
+      auto ka = pick_quant<AmaxOnly, true>(dtype, gate, has_linear_beta != 0);
+      BwdArgs am = a;
+      am.want_drw = 0;
+      int grid = 0;
+      st = launch_grid(reinterpret_cast<const void*>(ka), threads, 0, tokens, &grid);
+      if (st != SITU_OK) return st;
+      ka<<<grid, threads, 0, s>>>(am, reinterpret_cast<unsigned int*>(nv->out.amax_out));
+      st = check_launch("situ_glu_bwd_nvfp4 (amax)");
+      if (st != SITU_OK) return st;
+    }
+    auto k = pick_quant<Nvfp4Quant, true>(dtype, gate, has_linear_beta != 0);
+    int grid = 0;
+    st = launch_grid(reinterpret_cast<const void*>(k), threads, 0, tokens, &grid);
+    if (st != SITU_OK) return st;
+    k<<<grid, threads, 0, s>>>(a, nv->out);
+    st = check_launch("situ_glu_bwd_nvfp4");
   } else if (g_load_path.load(std::memory_order_relaxed) == 1) {
     StreamArgs sa{};
     sa.gate_up = a.gate_up;
@@ -3157,7 +3235,7 @@ situ_status_t situ_glu_bwd(const void* gate_up, situ_dtype_t dtype, int64_t toke
                            void* workspace, size_t workspace_bytes, void* stream) {
   return bwd_entry(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride, beta,
                    has_linear_beta, linear_beta, grad_out, grad_out_row_stride, d_gate_up, d_gate_up_row_stride,
-                   d_rw, d_rw_stride, workspace, workspace_bytes, nullptr, stream);
+                   d_rw, d_rw_stride, workspace, workspace_bytes, nullptr, nullptr, stream);
 }
 
 situ_status_t situ_glu_bwd_mxfp8(const void* gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
@@ -3171,7 +3249,22 @@ situ_status_t situ_glu_bwd_mxfp8(const void* gate_up, situ_dtype_t dtype, int64_
                 static_cast<uint8_t*>(d_gate_up_scale), d_gate_up_scale_row_stride, static_cast<int>(rule)};
   return bwd_entry(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride, beta,
                    has_linear_beta, linear_beta, grad_out, grad_out_row_stride, nullptr, 0, d_rw, d_rw_stride,
-                   workspace, workspace_bytes, &m, stream);
+                   workspace, workspace_bytes, &m, nullptr, stream);
+}
+
+situ_status_t situ_glu_bwd_nvfp4(const void* gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
+                                 int64_t gate_up_row_stride, const void* rw, situ_dtype_t rw_dtype,
+                                 situ_rw_mode_t rw_mode, int64_t rw_stride, double beta, int has_linear_beta,
+                                 double linear_beta, const void* grad_out, int64_t grad_out_row_stride,
+                                 void* d_gate_up_data, int64_t d_gate_up_data_row_stride, void* d_gate_up_scale,
+                                 int64_t d_gate_up_scale_row_stride, float* amax, int amax_given, void* d_rw,
+                                 int64_t d_rw_stride, void* workspace, size_t workspace_bytes, void* stream) {
+  const Nvfp4Bwd nv{{static_cast<char*>(d_gate_up_data), d_gate_up_data_row_stride,
+                     static_cast<uint8_t*>(d_gate_up_scale), d_gate_up_scale_row_stride, amax, amax},
+                    amax_given};
+  return bwd_entry(gate_up, dtype, tokens, inter, gate_up_row_stride, rw, rw_dtype, rw_mode, rw_stride, beta,
+                   has_linear_beta, linear_beta, grad_out, grad_out_row_stride, nullptr, 0, d_rw, d_rw_stride,
+                   workspace, workspace_bytes, nullptr, &nv, stream);
 }
 
 const char* situ_glu_status_string(situ_status_t status) {
@@ -3666,7 +3759,7 @@ extern "C" situ_status_t situ_glu_fwd_nvfp4(const void* gate_up, situ_dtype_t dt
   if (!amax_given) {
     cudaError_t err = cudaMemsetAsync(amax, 0, sizeof(float), s);
     if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
-    AmaxKernel ka = pick_amax(dtype, gate, has_linear_beta != 0);
+    auto ka = pick_quant<AmaxOnly, false>(dtype, gate, has_linear_beta != 0);
     int grid = 0;
     st = launch_grid(reinterpret_cast<const void*>(ka), threads, 0, tokens, &grid);
     if (st != SITU_OK) return st;
@@ -3675,8 +3768,8 @@ extern "C" situ_status_t situ_glu_fwd_nvfp4(const void* gate_up, situ_dtype_t dt
     if (st != SITU_OK) return st;
   }
   const Nvfp4Out m{static_cast<char*>(y_data), y_data_row_stride, static_cast<uint8_t*>(y_scale), y_scale_row_stride,
-                   amax};
-  FwdNvKernel k = pick_fwd_nv(dtype, gate, has_linear_beta != 0);
+                   amax, amax};
+  auto k = pick_quant<Nvfp4Quant, false>(dtype, gate, has_linear_beta != 0);
   int grid = 0;
   st = launch_grid(reinterpret_cast<const void*>(k), threads, 0, tokens, &grid);
   if (st != SITU_OK) return st;

@@ -462,6 +462,64 @@ def situ_glu_fwd_nvfp4(gate_up: torch.Tensor, routing_weights, beta: float = DEF
     return data, scale, amax
 
 
+def situ_glu_bwd_nvfp4(gate_up: torch.Tensor, routing_weights, grad_out: torch.Tensor,
+                       beta: float = DEFAULT_BETA, linear_beta: float | None = DEFAULT_LINEAR_BETA,
+                       want_drw: bool = True, amax: torch.Tensor | None = None, data=None, scale=None,
+                       amax_out: torch.Tensor | None = None, d_rw=None, workspace=None, stream=None):
+    """Backward with an NVFP4 d_gate_up: returns (packed E2M1 codes [..., I]
+    uint8 with dG's I / 2 bytes then dU's, E4M3 block scales [..., 2I / 16] as
+    torch.float8_e4m3fn, amax: a 1-element fp32 tensor holding d_gate_up's
+    tensor maximum A, d_routing_weights or None).  ``amax`` gives A instead
+    of computing it; otherwise it is computed into ``amax_out``.  The weight
+    gradient is as in situ_glu_bwd."""
+    _check_beta(beta, linear_beta)
+    g2, lead, inter = _rows(gate_up)
+    dtype = _dtype_code(g2, "gate_up")
+    if grad_out.dtype != gate_up.dtype:
+        raise TypeError("grad_out must have gate_up's dtype")
+    if tuple(grad_out.shape) != lead + (inter,):
+        raise ValueError(f"grad_out shape {tuple(grad_out.shape)} != {lead + (inter,)}")
+    go2 = grad_out.reshape(-1, inter)
+    if go2.stride(1) != 1 or (go2.shape[0] > 1 and go2.stride(0) < inter):
+        go2 = go2.contiguous()
+    mode, rw, rw_stride = routing_mode(lead, inter, routing_weights)
+    rw_dtype = _dtype_code(rw, "routing_weights") if rw is not None else abi.SITU_DTYPE_F32
+    want = bool(want_drw) and rw is not None
+    if data is None:
+        data = torch.empty(lead + (inter,), dtype=torch.uint8, device=gate_up.device)
+    if scale is None:
+        scale = torch.empty(lead + (2 * inter // 16,), dtype=torch.float8_e4m3fn, device=gate_up.device)
+    given = amax is not None
+    if amax is None:
+        amax = amax_out if amax_out is not None else torch.empty(1, dtype=torch.float32, device=gate_up.device)
+    if amax.dtype != torch.float32 or amax.numel() != 1 or amax.device != gate_up.device:
+        raise ValueError("amax must be one float32 element on gate_up's device")
+    d2 = data.view(-1, inter)
+    s2 = scale.view(-1, 2 * inter // 16)
+    d_rw_flat, d_rw_stride = None, 1
+    if want:
+        if d_rw is None:
+            d_rw = torch.empty(routing_weights.shape, dtype=routing_weights.dtype, device=gate_up.device)
+        d_rw_flat = d_rw.view(-1)
+        d_rw_stride = d_rw_flat.stride(0) if d_rw_flat.numel() > 1 else 1
+    tokens = g2.shape[0]
+    ws_bytes = abi.situ_glu_bwd_workspace_bytes(tokens, inter, mode, int(want))
+    if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=gate_up.device)
+    st = abi.situ_glu_bwd_nvfp4(g2.data_ptr(), dtype, tokens, inter, g2.stride(0) if tokens > 1 else 2 * inter,
+                                rw.data_ptr() if rw is not None else None, rw_dtype, mode, rw_stride,
+                                float(beta), int(linear_beta is not None),
+                                float(linear_beta) if linear_beta is not None else 0.0,
+                                go2.data_ptr(), go2.stride(0) if tokens > 1 else inter,
+                                d2.data_ptr(), d2.stride(0) if tokens > 1 else inter,
+                                s2.data_ptr(), s2.stride(0) if tokens > 1 else 2 * inter // 16,
+                                amax.data_ptr(), int(given),
+                                d_rw_flat.data_ptr() if d_rw_flat is not None else None, d_rw_stride,
+                                workspace.data_ptr() if ws_bytes else None, ws_bytes, _stream_handle(stream))
+    abi.check(st, "situ_glu_bwd_nvfp4")
+    return data, scale, amax, (d_rw if want else None)
+
+
 class WeightedSiTUFunction(torch.autograd.Function):
     """Routing-weighted SiTU-GLU with the analytic fused backward.
 

@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define SITU_GLU_ABI_VERSION 7
+#define SITU_GLU_ABI_VERSION 8
 
 typedef enum situ_status {
   SITU_OK = 0,
@@ -258,6 +258,32 @@ situ_status_t situ_glu_fwd_nvfp4(const void *gate_up, situ_dtype_t dtype, int64_
                                  void *y_data, int64_t y_data_row_stride,
                                  void *y_scale, int64_t y_scale_row_stride,
                                  float *amax, int amax_given, void *stream);
+
+/*
+ * Backward with an NVFP4 d_gate_up (format as for situ_glu_fwd_nvfp4; the
+ * NVFP4 recipe's backward, Megatron-LM PR #6673, "Test results"): with A the
+ * largest finite |dG|, |dU| of the call (one tensor scale S_enc = 2688 / A for
+ * the whole d_gate_up),
+ *   d_gate_up_data   [tokens, >= inter] bytes: dG's packed E2M1 codes
+ *                    (inter / 2 bytes), then dU's; row pitch a multiple of 4,
+ *                    base 4-byte aligned
+ *   d_gate_up_scale  [tokens, >= 2 inter / 16] E4M3 block scales: dG's, then dU's
+ *   amax / amax_given as for situ_glu_fwd_nvfp4 (amax_given = 0: a first pass
+ *                    over gate_up and grad_out computes A)
+ * d_rw, workspace and every other argument and error as for situ_glu_bwd
+ * (per-row, broadcast or no routing weights); inter a multiple of 16.
+ */
+situ_status_t situ_glu_bwd_nvfp4(const void *gate_up, situ_dtype_t dtype, int64_t tokens, int64_t inter,
+                                 int64_t gate_up_row_stride,
+                                 const void *rw, situ_dtype_t rw_dtype, situ_rw_mode_t rw_mode,
+                                 int64_t rw_stride,
+                                 double beta, int has_linear_beta, double linear_beta,
+                                 const void *grad_out, int64_t grad_out_row_stride,
+                                 void *d_gate_up_data, int64_t d_gate_up_data_row_stride,
+                                 void *d_gate_up_scale, int64_t d_gate_up_scale_row_stride,
+                                 float *amax, int amax_given,
+                                 void *d_rw, int64_t d_rw_stride,
+                                 void *workspace, size_t workspace_bytes, void *stream);
 
 /* ---- FC1 grouped GEMM + SiTU-GLU --------------------------------------------
  * Megatron-LM PR #6673, "Design": with a SiTU-capable cuDNN frontend FC1's

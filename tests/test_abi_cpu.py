@@ -58,7 +58,7 @@ def test_binding_covers_the_header_exactly():
 
 
 def test_version_and_status_strings(native_lib_path):
-    assert abi.situ_glu_abi_version() == abi.ABI_VERSION == 7
+    assert abi.situ_glu_abi_version() == abi.ABI_VERSION == 8
     assert abi.situ_glu_status_string(OK) == "SITU_OK"
     assert abi.situ_glu_status_string(MISAL) == "SITU_ERR_MISALIGNED"
     assert abi.situ_glu_status_string(99) == "SITU_ERR_UNKNOWN"
@@ -349,6 +349,44 @@ def test_fwd_nvfp4_argument_errors(name, kw, want, native_lib_path):
 
 def test_nvfp4_zero_tokens_with_given_amax_is_a_no_op(native_lib_path):
     assert fwd_nv(tokens=0, y_data=None, y_scale=None) == OK
+    assert bwd_nv(tokens=0, d_gate_up_data=None, d_gate_up_scale=None, d_rw=None) == OK
+
+
+def bwd_nv(**kw):
+    a = dict(gate_up=GU, dtype=BF16, tokens=16, inter=64, gate_up_row_stride=128, rw=RW, rw_dtype=F32,
+             rw_mode=ROW, rw_stride=1, beta=4.0, has_linear_beta=1, linear_beta=25.0, grad_out=GO,
+             grad_out_row_stride=64, d_gate_up_data=MXD, d_gate_up_data_row_stride=64, d_gate_up_scale=MXS,
+             d_gate_up_scale_row_stride=8, amax=AMX, amax_given=1, d_rw=DRW, d_rw_stride=1, workspace=None,
+             workspace_bytes=0, stream=None)
+    a.update(kw)
+    return abi.situ_glu_bwd_nvfp4(**a)
+
+
+NV_BWD_CASES = [
+    ("inter not a multiple of 16", dict(inter=40, gate_up_row_stride=80, grad_out_row_stride=40), INVALID),
+    ("per-column weights", dict(rw_mode=3), UNSUP),
+    ("per-element weights", dict(rw_mode=4, rw_stride=64), UNSUP),
+    ("scale pitch short", dict(d_gate_up_scale_row_stride=7), INVALID),
+    ("data pitch short", dict(d_gate_up_data_row_stride=60), INVALID),
+    ("data pitch not 4-byte", dict(d_gate_up_data_row_stride=66), MISAL),
+    ("data misaligned", dict(d_gate_up_data=MXD + 2), MISAL),
+    ("data NULL", dict(d_gate_up_data=None), INVALID),
+    ("scale NULL", dict(d_gate_up_scale=None), INVALID),
+    ("amax NULL", dict(amax=None), INVALID),
+    ("amax misaligned", dict(amax=AMX + 2), MISAL),
+    ("amax_given not 0 or 1", dict(amax_given=3), INVALID),
+    ("data overlaps grad_out", dict(d_gate_up_data=GO), INVALID),
+    ("scales overlap gate_up", dict(d_gate_up_scale=GU + 64), INVALID),
+    ("amax inside the data", dict(amax=MXD + 16), INVALID),
+    ("d_rw overlaps amax", dict(d_rw=AMX), INVALID),
+    ("grad_out pitch short", dict(grad_out_row_stride=32), INVALID),
+    ("bad linear beta", dict(linear_beta=0.0), INVALID),
+]
+
+
+@pytest.mark.parametrize("name,kw,want", NV_BWD_CASES, ids=[c[0] for c in NV_BWD_CASES])
+def test_bwd_nvfp4_argument_errors(name, kw, want, native_lib_path):
+    assert bwd_nv(**kw) == want, abi.situ_glu_last_error()
 
 
 # ---- FC1 grouped GEMM + SiTU-GLU: argument checks run before any CUDA call -------
