@@ -52,7 +52,7 @@ extern "C" {
 typedef enum situ_status {
   SITU_OK = 0,
   SITU_ERR_INVALID_ARG = 1, /* NULL pointer, bad size, stride, beta, enum or aliasing */
-  SITU_ERR_UNSUPPORTED = 2, /* a valid request this build does not implement          */
+  SITU_ERR_UNSUPPORTED = 2, /* a valid request the library does not implement         */
   SITU_ERR_MISALIGNED = 3,  /* a base address or row pitch is not 16-byte aligned     */
   SITU_ERR_CUDA = 4         /* the CUDA runtime reported an error at launch           */
 } situ_status_t;
