@@ -2721,8 +2721,8 @@ situ_status_t check_nv_args(const Nvfp4Bwd& n, int64_t inter, int64_t cols, situ
     return fail(SITU_ERR_INVALID_ARG, "NVFP4 outputs need inter a multiple of 16, got %lld", (long long)inter);
   if (rw_mode == SITU_RW_COL || rw_mode == SITU_RW_FULL)
     return fail(SITU_ERR_UNSUPPORTED, "NVFP4 outputs take per-row, broadcast or no routing weights");
-  if (n.amax_given != 0 && n.amax_given != 1) return fail(SITU_ERR_INVALID_ARG, "amax_given must be 0 or 1");
-  if (n.out.data_pitch < cols / 2 || n.out.scale_pitch < cols / 16)
+  if (n.amax_given < 0 || n.amax_given > 2) return fail(SITU_ERR_INVALID_ARG, "amax_given must be 0, 1 or 2");
+  if (n.amax_given != 2 && (n.out.data_pitch < cols / 2 || n.out.scale_pitch < cols / 16))
     return fail(SITU_ERR_INVALID_ARG, "NVFP4 data or scale row pitch shorter than a row");
   if (n.out.amax_out == nullptr) return fail(SITU_ERR_INVALID_ARG, "amax is NULL");
   if (!aligned(n.out.amax_out, 4)) return fail(SITU_ERR_MISALIGNED, "amax not 4-byte aligned");
@@ -3008,6 +3008,8 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
   }
   if (rw_mode == SITU_RW_NONE && d_rw != nullptr)
     return fail(SITU_ERR_INVALID_ARG, "d_rw must be NULL for SITU_RW_NONE");
+  if (nv != nullptr && nv->amax_given == 2 && d_rw != nullptr)
+    return fail(SITU_ERR_INVALID_ARG, "d_rw must be NULL when only the tensor maximum is computed");
   const bool want_drw = d_rw != nullptr;
   if (want_drw && rw_mode == SITU_RW_ROW && d_rw_stride < 1) return fail(SITU_ERR_INVALID_ARG, "d_rw_stride < 1");
   if (want_drw && rw_mode == SITU_RW_FULL && d_rw_stride < inter)
@@ -3016,7 +3018,7 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
   if (tokens == 0) {
     // The gradient of a broadcast weight over zero rows is zero, and so is the
     // maximum of an empty NVFP4 gradient; nothing else is written.
-    if (nv != nullptr && !nv->amax_given) {
+    if (nv != nullptr && nv->amax_given != 1) {
       cudaError_t err = cudaMemsetAsync(nv->out.amax_out, 0, sizeof(float), static_cast<cudaStream_t>(stream));
       if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
     }
@@ -3037,7 +3039,7 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
     st = check_mx_buffers(*mx, tokens, 2 * inter);
     if (st != SITU_OK) return st;
   }
-  if (nv != nullptr) {
+  if (nv != nullptr && nv->amax_given != 2) {
     st = check_nv_buffers(*nv, tokens, 2 * inter);
     if (st != SITU_OK) return st;
   }
@@ -3069,13 +3071,16 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
   const Span s_gu = matrix_span(gate_up, tokens, gate_up_row_stride, 2 * inter, es);
   const Span s_go = matrix_span(grad_out, tokens, grad_out_row_stride, inter, es);
   const Span s_dgu = mx   ? matrix_span(mx->data, tokens, mx->data_pitch, 2 * inter, 1)
-                    : nv ? matrix_span(nv->out.data, tokens, nv->out.data_pitch, inter, 1)
+                    : nv ? (nv->amax_given == 2 ? Span{0, 0}
+                                                : matrix_span(nv->out.data, tokens, nv->out.data_pitch, inter, 1))
                          : matrix_span(d_gate_up, tokens, d_gate_up_row_stride, 2 * inter, es);
   const Span s_rw = weight_span(rw, rw_mode, tokens, rw_stride, inter, rw_es);
   if (overlap(s_dgu, s_gu) || overlap(s_dgu, s_go) || overlap(s_dgu, s_rw))
     return fail(SITU_ERR_INVALID_ARG, "d_gate_up overlaps an input");
   const Span s_sc = mx   ? matrix_span(mx->scale, tokens, mx->scale_pitch, 2 * inter / kMxBlock, 1)
-                    : nv ? matrix_span(nv->out.scale, tokens, nv->out.scale_pitch, 2 * inter / 16, 1)
+                    : nv ? (nv->amax_given == 2
+                                ? Span{0, 0}
+                                : matrix_span(nv->out.scale, tokens, nv->out.scale_pitch, 2 * inter / 16, 1))
                          : Span{0, 0};
   if (!native && (overlap(s_sc, s_gu) || overlap(s_sc, s_go) || overlap(s_sc, s_rw)))
     return fail(SITU_ERR_INVALID_ARG, "block scales overlap an input");
@@ -3169,7 +3174,7 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
     st = check_launch("situ_glu_bwd_mxfp8");
   } else if (nv != nullptr) {
     const int threads = choose_threads(a.vpr);
-    if (!nv->amax_given) {  // the tensor maximum of d_gate_up first: a pass without stores or d_w
+    if (nv->amax_given != 1) {  // the tensor maximum of d_gate_up first: a pass without stores or d_w
       cudaError_t err = cudaMemsetAsync(nv->out.amax_out, 0, sizeof(float), s);
       if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
       auto ka = pick_quant<AmaxOnly, true>(dtype, gate, has_linear_beta != 0);
@@ -3180,7 +3185,7 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
       if (st != SITU_OK) return st;
       ka<<<grid, threads, 0, s>>>(am, reinterpret_cast<unsigned int*>(nv->out.amax_out));
       st = check_launch("situ_glu_bwd_nvfp4 (amax)");
-      if (st != SITU_OK) return st;
+      if (st != SITU_OK || nv->amax_given == 2) return st;
     }
     auto k = pick_quant<Nvfp4Quant, true>(dtype, gate, has_linear_beta != 0);
     int grid = 0;
@@ -3708,36 +3713,39 @@ extern "C" situ_status_t situ_glu_fwd_nvfp4(const void* gate_up, situ_dtype_t dt
     return fail(SITU_ERR_INVALID_ARG, "NVFP4 outputs need inter a multiple of 16, got %lld", (long long)inter);
   if (rw_mode == SITU_RW_COL || rw_mode == SITU_RW_FULL)
     return fail(SITU_ERR_UNSUPPORTED, "NVFP4 outputs take per-row, broadcast or no routing weights");
-  if (amax_given != 0 && amax_given != 1) return fail(SITU_ERR_INVALID_ARG, "amax_given must be 0 or 1");
-  if (y_data_row_stride < inter / 2 || y_scale_row_stride < inter / 16)
+  if (amax_given < 0 || amax_given > 2) return fail(SITU_ERR_INVALID_ARG, "amax_given must be 0, 1 or 2");
+  const bool amax_only = amax_given == 2;  // the tensor maximum alone: no codes, no scales
+  if (!amax_only && (y_data_row_stride < inter / 2 || y_scale_row_stride < inter / 16))
     return fail(SITU_ERR_INVALID_ARG, "NVFP4 data or scale row pitch shorter than a row");
   if (amax == nullptr) return fail(SITU_ERR_INVALID_ARG, "amax is NULL");
   if (!aligned(amax, 4)) return fail(SITU_ERR_MISALIGNED, "amax not 4-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (tokens == 0) {
-    if (!amax_given) {
+    if (amax_given != 1) {
       cudaError_t err = cudaMemsetAsync(amax, 0, sizeof(float), s);
       if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
     }
     return SITU_OK;
   }
-  if (gate_up == nullptr || y_data == nullptr || y_scale == nullptr)
+  if (gate_up == nullptr || (!amax_only && (y_data == nullptr || y_scale == nullptr)))
     return fail(SITU_ERR_INVALID_ARG, "gate_up, y_data or y_scale is NULL");
   const int es = elem_size(dtype);
-  if (!span_fits(tokens, gate_up_row_stride, 2 * inter, es) || !span_fits(tokens, y_data_row_stride, inter / 2, 1) ||
-      !span_fits(tokens, y_scale_row_stride, inter / 16, 1) ||
+  if (!span_fits(tokens, gate_up_row_stride, 2 * inter, es) ||
+      (!amax_only && (!span_fits(tokens, y_data_row_stride, inter / 2, 1) ||
+                      !span_fits(tokens, y_scale_row_stride, inter / 16, 1))) ||
       (rw_mode == SITU_RW_ROW && !span_fits(tokens, rw_stride, 1, elem_size(rw_dtype))))
     return fail(SITU_ERR_INVALID_ARG, "tensor extent overflows int64");
   // a thread stores the codes of one 16-byte input vector: 4 bytes (bf16) or 2 (fp32)
-  if (!aligned(gate_up, 16) || (gate_up_row_stride * es) % 16 != 0 || !aligned(y_data, 4) ||
-      y_data_row_stride % 4 != 0 || (rw_mode != SITU_RW_NONE && !aligned(rw, elem_size(rw_dtype))))
+  if (!aligned(gate_up, 16) || (gate_up_row_stride * es) % 16 != 0 ||
+      (!amax_only && (!aligned(y_data, 4) || y_data_row_stride % 4 != 0)) ||
+      (rw_mode != SITU_RW_NONE && !aligned(rw, elem_size(rw_dtype))))
     return fail(SITU_ERR_MISALIGNED,
                 "gate_up base or row pitch not 16-byte aligned, y_data base or row pitch not 4-byte aligned, or rw "
                 "misaligned");
   const Span s_gu = matrix_span(gate_up, tokens, gate_up_row_stride, 2 * inter, es);
   const Span s_rw = weight_span(rw, rw_mode, tokens, rw_stride, inter, elem_size(rw_dtype));
-  const Span s_d = matrix_span(y_data, tokens, y_data_row_stride, inter / 2, 1);
-  const Span s_s = matrix_span(y_scale, tokens, y_scale_row_stride, inter / 16, 1);
+  const Span s_d = amax_only ? Span{0, 0} : matrix_span(y_data, tokens, y_data_row_stride, inter / 2, 1);
+  const Span s_s = amax_only ? Span{0, 0} : matrix_span(y_scale, tokens, y_scale_row_stride, inter / 16, 1);
   const Span s_a = {reinterpret_cast<uintptr_t>(amax), reinterpret_cast<uintptr_t>(amax) + 4};
   const Span outs[] = {s_d, s_s, s_a};
   for (int i = 0; i < 3; ++i) {
@@ -3756,7 +3764,7 @@ extern "C" situ_status_t situ_glu_fwd_nvfp4(const void* gate_up, situ_dtype_t dt
   a.vpr = static_cast<int>(inter * es / kVecBytes);
   a.c = c;
   const int threads = choose_threads(a.vpr);
-  if (!amax_given) {
+  if (amax_given != 1) {
     cudaError_t err = cudaMemsetAsync(amax, 0, sizeof(float), s);
     if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
     auto ka = pick_quant<AmaxOnly, false>(dtype, gate, has_linear_beta != 0);
@@ -3765,7 +3773,7 @@ extern "C" situ_status_t situ_glu_fwd_nvfp4(const void* gate_up, situ_dtype_t dt
     if (st != SITU_OK) return st;
     ka<<<grid, threads, 0, s>>>(a, reinterpret_cast<unsigned int*>(amax));
     st = check_launch("situ_glu_fwd_nvfp4 (amax)");
-    if (st != SITU_OK) return st;
+    if (st != SITU_OK || amax_only) return st;
   }
   const Nvfp4Out m{static_cast<char*>(y_data), y_data_row_stride, static_cast<uint8_t*>(y_scale), y_scale_row_stride,
                    amax, amax};

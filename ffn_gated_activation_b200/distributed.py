@@ -16,6 +16,14 @@ and grad_out row only), so:
   columns (``tp_local_columns``); their gradients stay local.
 * Under data parallelism a per-column weight is shared by every row shard,
   so its [I] gradient is all-reduced like a broadcast weight's.
+* An NVFP4 output has one per-tensor scale.  When a tensor is split over the
+  ranks of a tensor-parallel group (column shards of Y or d_gate_up), every
+  shard must be coded with the maximum of the whole tensor: each rank
+  computes its shard's maximum, the maxima are all-reduced (MAX), and each
+  rank codes its shard with the result (``situ_glu_fwd_nvfp4_tp``,
+  ``situ_glu_bwd_nvfp4_tp``).  Column shards of a block-scaled tensor keep
+  whole blocks (``align`` = 16 for NVFP4, 32 for MXFP8).  Row shards under
+  data parallelism are separate tensors and keep their own scales.
 
 Nothing here computes the method; the kernels run in libsitu_glu.so.
 """
@@ -47,17 +55,18 @@ def vector_width(dtype: torch.dtype) -> int:
     return 16 // torch.empty((), dtype=dtype).element_size()
 
 
-def tp_local_gate_up(gate_up: torch.Tensor, rank: int, world: int) -> torch.Tensor:
+def tp_local_gate_up(gate_up: torch.Tensor, rank: int, world: int, align: int | None = None) -> torch.Tensor:
     """The [..., 2 * I_r] gate_up a column-parallel FC1 produces on ``rank``:
-    gate columns [a, b) followed by the same up columns [I + a, I + b)."""
+    gate columns [a, b) followed by the same up columns [I + a, I + b).
+    Shard boundaries are multiples of ``align`` (default: one 16-byte vector)."""
     inter = gate_up.shape[-1] // 2
-    a, b = shard_range(inter, rank, world, vector_width(gate_up.dtype))
+    a, b = shard_range(inter, rank, world, align or vector_width(gate_up.dtype))
     return torch.cat([gate_up[..., a:b], gate_up[..., inter + a:inter + b]], dim=-1).contiguous()
 
 
-def tp_local_columns(x: torch.Tensor, rank: int, world: int) -> torch.Tensor:
+def tp_local_columns(x: torch.Tensor, rank: int, world: int, align: int | None = None) -> torch.Tensor:
     """Columns [a, b) of an [..., I] tensor (grad_out or Y) held by ``rank``."""
-    a, b = shard_range(x.shape[-1], rank, world, vector_width(x.dtype))
+    a, b = shard_range(x.shape[-1], rank, world, align or vector_width(x.dtype))
     return x[..., a:b].contiguous()
 
 
@@ -82,6 +91,41 @@ def situ_glu_bwd_tp(gate_up_local, routing_weights, grad_out_local, beta=functio
     if d_rw is not None and tp_drw_needs_allreduce(lead, inter_local, routing_weights):
         allreduce_drw(d_rw, group)
     return d_gate_up, d_rw
+
+
+def allreduce_amax(amax: torch.Tensor, group=None) -> torch.Tensor:
+    """Largest of the ranks' tensor maxima, in place (the per-tensor scale of a
+    tensor whose shards live on the ranks of ``group``)."""
+    dist.all_reduce(amax, op=dist.ReduceOp.MAX, group=group)
+    return amax
+
+
+def situ_glu_fwd_nvfp4_tp(gate_up_local, routing_weights, beta=functional.DEFAULT_BETA,
+                          linear_beta=functional.DEFAULT_LINEAR_BETA, group=None, **kw):
+    """NVFP4 forward of a column-parallel shard (gate_up_local from
+    ``tp_local_gate_up(..., align=16)``): the shard's maximum, the group's
+    maximum, then the shard's codes under the whole tensor's scale.  Returns
+    (data, scale, amax) as situ_glu_fwd_nvfp4."""
+    _, _, amax = functional.situ_glu_fwd_nvfp4(gate_up_local, routing_weights, beta, linear_beta, amax_only=True)
+    allreduce_amax(amax, group)
+    return functional.situ_glu_fwd_nvfp4(gate_up_local, routing_weights, beta, linear_beta, amax=amax, **kw)
+
+
+def situ_glu_bwd_nvfp4_tp(gate_up_local, routing_weights, grad_out_local, beta=functional.DEFAULT_BETA,
+                          linear_beta=functional.DEFAULT_LINEAR_BETA, group=None, want_drw=True, **kw):
+    """NVFP4 backward of a column-parallel shard: d_gate_up's codes under the
+    whole tensor's scale (the group's maximum of the shards' maxima), and the
+    routing-weight gradient all-reduced as in ``situ_glu_bwd_tp``.  Returns
+    (data, scale, amax, d_rw) as situ_glu_bwd_nvfp4."""
+    _, _, amax, _ = functional.situ_glu_bwd_nvfp4(gate_up_local, routing_weights, grad_out_local, beta,
+                                                  linear_beta, amax_only=True)
+    allreduce_amax(amax, group)
+    data, scale, amax, d_rw = functional.situ_glu_bwd_nvfp4(gate_up_local, routing_weights, grad_out_local, beta,
+                                                            linear_beta, want_drw=want_drw, amax=amax, **kw)
+    lead = tuple(gate_up_local.shape[:-1])
+    if d_rw is not None and tp_drw_needs_allreduce(lead, gate_up_local.shape[-1] // 2, routing_weights):
+        allreduce_drw(d_rw, group)
+    return data, scale, amax, d_rw
 
 
 def tp_drw_needs_allreduce(lead: tuple, inter_local: int, routing_weights) -> bool:

@@ -427,51 +427,62 @@ def apply_attn_res(prefix_sum: torch.Tensor, block_residual: torch.Tensor, proj_
 
 def situ_glu_fwd_nvfp4(gate_up: torch.Tensor, routing_weights, beta: float = DEFAULT_BETA,
                        linear_beta: float | None = DEFAULT_LINEAR_BETA, amax: torch.Tensor | None = None,
-                       data=None, scale=None, amax_out: torch.Tensor | None = None, stream=None):
+                       data=None, scale=None, amax_out: torch.Tensor | None = None, amax_only: bool = False,
+                       stream=None):
     """Forward with an NVFP4 Y: returns (packed E2M1 codes [..., I / 2] uint8,
     E4M3 block scales [..., I / 16] as torch.float8_e4m3fn, amax: a 1-element
     fp32 tensor holding the tensor maximum A).  Pass ``amax`` (1 element, on
     gate_up's device) to use a known A instead of computing it; otherwise A is
-    computed into ``amax_out`` (allocated when None).  Decode code q of block
-    b as q * scale_b * A / 2688."""
+    computed into ``amax_out`` (allocated when None).  ``amax_only``: compute
+    A alone and return (None, None, amax).  Decode code q of block b as
+    q * scale_b * A / 2688."""
     _check_beta(beta, linear_beta)
     g2, lead, inter = _rows(gate_up)
     dtype = _dtype_code(g2, "gate_up")
     mode, rw, rw_stride = routing_mode(lead, inter, routing_weights)
     rw_dtype = _dtype_code(rw, "routing_weights") if rw is not None else abi.SITU_DTYPE_F32
-    if data is None:
-        data = torch.empty(lead + (inter // 2,), dtype=torch.uint8, device=gate_up.device)
-    if scale is None:
-        scale = torch.empty(lead + (inter // 16,), dtype=torch.float8_e4m3fn, device=gate_up.device)
+    if amax_only and amax is not None:
+        raise ValueError("amax_only computes the tensor maximum: do not pass one")
+    if not amax_only:
+        if data is None:
+            data = torch.empty(lead + (inter // 2,), dtype=torch.uint8, device=gate_up.device)
+        if scale is None:
+            scale = torch.empty(lead + (inter // 16,), dtype=torch.float8_e4m3fn, device=gate_up.device)
     given = amax is not None
     if amax is None:
         amax = amax_out if amax_out is not None else torch.empty(1, dtype=torch.float32, device=gate_up.device)
     if amax.dtype != torch.float32 or amax.numel() != 1 or amax.device != gate_up.device:
         raise ValueError("amax must be one float32 element on gate_up's device")
-    d2 = data.view(-1, inter // 2)
-    s2 = scale.view(-1, inter // 16)
     tokens = g2.shape[0]
+    if amax_only:
+        d_ptr, d_pitch, s_ptr, s_pitch = None, inter // 2, None, inter // 16
+    else:
+        d2 = data.view(-1, inter // 2)
+        s2 = scale.view(-1, inter // 16)
+        d_ptr, d_pitch = d2.data_ptr(), d2.stride(0) if tokens > 1 else inter // 2
+        s_ptr, s_pitch = s2.data_ptr(), s2.stride(0) if tokens > 1 else inter // 16
     st = abi.situ_glu_fwd_nvfp4(g2.data_ptr(), dtype, tokens, inter, g2.stride(0) if tokens > 1 else 2 * inter,
                                 rw.data_ptr() if rw is not None else None, rw_dtype, mode, rw_stride,
                                 float(beta), int(linear_beta is not None),
                                 float(linear_beta) if linear_beta is not None else 0.0,
-                                d2.data_ptr(), d2.stride(0) if tokens > 1 else inter // 2,
-                                s2.data_ptr(), s2.stride(0) if tokens > 1 else inter // 16,
-                                amax.data_ptr(), int(given), _stream_handle(stream))
+                                d_ptr, d_pitch, s_ptr, s_pitch, amax.data_ptr(), 2 if amax_only else int(given),
+                                _stream_handle(stream))
     abi.check(st, "situ_glu_fwd_nvfp4")
-    return data, scale, amax
+    return (None, None, amax) if amax_only else (data, scale, amax)
 
 
 def situ_glu_bwd_nvfp4(gate_up: torch.Tensor, routing_weights, grad_out: torch.Tensor,
                        beta: float = DEFAULT_BETA, linear_beta: float | None = DEFAULT_LINEAR_BETA,
                        want_drw: bool = True, amax: torch.Tensor | None = None, data=None, scale=None,
-                       amax_out: torch.Tensor | None = None, d_rw=None, workspace=None, stream=None):
+                       amax_out: torch.Tensor | None = None, d_rw=None, workspace=None, amax_only: bool = False,
+                       stream=None):
     """Backward with an NVFP4 d_gate_up: returns (packed E2M1 codes [..., I]
     uint8 with dG's I / 2 bytes then dU's, E4M3 block scales [..., 2I / 16] as
     torch.float8_e4m3fn, amax: a 1-element fp32 tensor holding d_gate_up's
     tensor maximum A, d_routing_weights or None).  ``amax`` gives A instead
-    of computing it; otherwise it is computed into ``amax_out``.  The weight
-    gradient is as in situ_glu_bwd."""
+    of computing it; otherwise it is computed into ``amax_out``.
+    ``amax_only``: compute A alone (no codes, no weight gradient) and return
+    (None, None, amax, None).  The weight gradient is as in situ_glu_bwd."""
     _check_beta(beta, linear_beta)
     g2, lead, inter = _rows(gate_up)
     dtype = _dtype_code(g2, "gate_up")
@@ -484,25 +495,33 @@ def situ_glu_bwd_nvfp4(gate_up: torch.Tensor, routing_weights, grad_out: torch.T
         go2 = go2.contiguous()
     mode, rw, rw_stride = routing_mode(lead, inter, routing_weights)
     rw_dtype = _dtype_code(rw, "routing_weights") if rw is not None else abi.SITU_DTYPE_F32
-    want = bool(want_drw) and rw is not None
-    if data is None:
-        data = torch.empty(lead + (inter,), dtype=torch.uint8, device=gate_up.device)
-    if scale is None:
-        scale = torch.empty(lead + (2 * inter // 16,), dtype=torch.float8_e4m3fn, device=gate_up.device)
+    want = bool(want_drw) and rw is not None and not amax_only
+    if amax_only and amax is not None:
+        raise ValueError("amax_only computes the tensor maximum: do not pass one")
+    if not amax_only:
+        if data is None:
+            data = torch.empty(lead + (inter,), dtype=torch.uint8, device=gate_up.device)
+        if scale is None:
+            scale = torch.empty(lead + (2 * inter // 16,), dtype=torch.float8_e4m3fn, device=gate_up.device)
     given = amax is not None
     if amax is None:
         amax = amax_out if amax_out is not None else torch.empty(1, dtype=torch.float32, device=gate_up.device)
     if amax.dtype != torch.float32 or amax.numel() != 1 or amax.device != gate_up.device:
         raise ValueError("amax must be one float32 element on gate_up's device")
-    d2 = data.view(-1, inter)
-    s2 = scale.view(-1, 2 * inter // 16)
+    tokens = g2.shape[0]
+    if amax_only:
+        d_ptr, d_pitch, s_ptr, s_pitch = None, inter, None, 2 * inter // 16
+    else:
+        d2 = data.view(-1, inter)
+        s2 = scale.view(-1, 2 * inter // 16)
+        d_ptr, d_pitch = d2.data_ptr(), d2.stride(0) if tokens > 1 else inter
+        s_ptr, s_pitch = s2.data_ptr(), s2.stride(0) if tokens > 1 else 2 * inter // 16
     d_rw_flat, d_rw_stride = None, 1
     if want:
         if d_rw is None:
             d_rw = torch.empty(routing_weights.shape, dtype=routing_weights.dtype, device=gate_up.device)
         d_rw_flat = d_rw.view(-1)
         d_rw_stride = d_rw_flat.stride(0) if d_rw_flat.numel() > 1 else 1
-    tokens = g2.shape[0]
     ws_bytes = abi.situ_glu_bwd_workspace_bytes(tokens, inter, mode, int(want))
     if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=gate_up.device)
@@ -511,12 +530,12 @@ def situ_glu_bwd_nvfp4(gate_up: torch.Tensor, routing_weights, grad_out: torch.T
                                 float(beta), int(linear_beta is not None),
                                 float(linear_beta) if linear_beta is not None else 0.0,
                                 go2.data_ptr(), go2.stride(0) if tokens > 1 else inter,
-                                d2.data_ptr(), d2.stride(0) if tokens > 1 else inter,
-                                s2.data_ptr(), s2.stride(0) if tokens > 1 else 2 * inter // 16,
-                                amax.data_ptr(), int(given),
+                                d_ptr, d_pitch, s_ptr, s_pitch, amax.data_ptr(), 2 if amax_only else int(given),
                                 d_rw_flat.data_ptr() if d_rw_flat is not None else None, d_rw_stride,
                                 workspace.data_ptr() if ws_bytes else None, ws_bytes, _stream_handle(stream))
     abi.check(st, "situ_glu_bwd_nvfp4")
+    if amax_only:
+        return None, None, amax, None
     return data, scale, amax, (d_rw if want else None)
 
 

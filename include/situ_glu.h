@@ -244,8 +244,11 @@ situ_status_t situ_glu_bwd_mxfp8(const void *gate_up, situ_dtype_t dtype, int64_
  *   amax     device fp32: A.  amax_given = 0: the library computes it first
  *            (a pass that reads gate_up once more) and writes it here;
  *            amax_given = 1: the caller's A is used (e.g. from an earlier
- *            step); block scales and codes saturate (448, +-6) where it is
- *            below the call's own maximum.
+ *            step, or a maximum reduced over the ranks that hold the shards
+ *            of one tensor); block scales and codes saturate (448, +-6) where
+ *            it is below the call's own maximum; amax_given = 2: only A is
+ *            computed and written (y_data and y_scale may be NULL), the first
+ *            half of a sharded tensor's two-step coding.
  * A consumer decodes code q of block b as q * s_b * A / 2688.  inter must be a
  * multiple of 16; routing weights per row, broadcast or none.  Other
  * arguments and errors as for situ_glu_fwd.
@@ -269,7 +272,8 @@ situ_status_t situ_glu_fwd_nvfp4(const void *gate_up, situ_dtype_t dtype, int64_
  *                    base 4-byte aligned
  *   d_gate_up_scale  [tokens, >= 2 inter / 16] E4M3 block scales: dG's, then dU's
  *   amax / amax_given as for situ_glu_fwd_nvfp4 (amax_given = 0: a first pass
- *                    over gate_up and grad_out computes A)
+ *                    over gate_up and grad_out computes A; 2: only A, with
+ *                    d_rw NULL)
  * d_rw, workspace and every other argument and error as for situ_glu_bwd
  * (per-row, broadcast or no routing weights); inter a multiple of 16.
  */

@@ -333,7 +333,7 @@ NV_CASES = [
     ("scale NULL", dict(y_scale=None), INVALID),
     ("amax NULL", dict(amax=None), INVALID),
     ("amax misaligned", dict(amax=AMX + 2), MISAL),
-    ("amax_given not 0 or 1", dict(amax_given=2), INVALID),
+    ("amax_given not 0, 1 or 2", dict(amax_given=3), INVALID),
     ("data overlaps gate_up", dict(y_data=GU), INVALID),
     ("amax inside the scales", dict(amax=MXS + 8), INVALID),
     ("scale overlaps data", dict(y_scale=MXD + 32), INVALID),
@@ -374,7 +374,8 @@ NV_BWD_CASES = [
     ("scale NULL", dict(d_gate_up_scale=None), INVALID),
     ("amax NULL", dict(amax=None), INVALID),
     ("amax misaligned", dict(amax=AMX + 2), MISAL),
-    ("amax_given not 0 or 1", dict(amax_given=3), INVALID),
+    ("amax_given not 0, 1 or 2", dict(amax_given=3), INVALID),
+    ("amax only with d_rw", dict(amax_given=2), INVALID),
     ("data overlaps grad_out", dict(d_gate_up_data=GO), INVALID),
     ("scales overlap gate_up", dict(d_gate_up_scale=GU + 64), INVALID),
     ("amax inside the data", dict(amax=MXD + 16), INVALID),

@@ -121,12 +121,53 @@ def _col_weight_check(rank, T, I, seed):
     assert D.tp_drw_needs_allreduce((T,), b - a, torch.ones(T, 1))
 
 
+def _tp_nvfp4_check(rank, T, I, seed):
+    """Column shards of an NVFP4 Y and d_gate_up (whole 16-element blocks per
+    rank): the all-reduced maximum of the shards' maxima is the whole
+    tensor's, and each shard's codes and block scales under it are the
+    matching columns of the whole tensor's coding."""
+    import oracle
+    import workloads
+    import dataclasses
+    wl = dataclasses.replace(workloads.workload(2), tokens=T, inter=I, seed=seed, rw_kind="uniform")
+    x = workloads.inputs(wl)
+    o = oracle.load()
+    rw = x["routing_weights"]
+    gu_local = _bits(D.tp_local_gate_up(_bf16_tensor(x["gate_up"]), rank, WORLD, align=16))
+    go_local = _bits(D.tp_local_columns(_bf16_tensor(x["grad_out"]), rank, WORLD, align=16))
+    a, b = D.shard_range(I, rank, WORLD, align=16)
+    assert a % 16 == 0 and b % 16 == 0 and b > a
+    y_full = o.fwd(x["gate_up"], rw, 4.0, 25.0)
+    full = o.bwd(x["gate_up"], rw, x["grad_out"], 4.0, 25.0)
+    d_full = np.concatenate([full.dg, full.du], axis=1)
+    y_loc = o.fwd(gu_local, rw, 4.0, 25.0)
+    loc = o.bwd(gu_local, rw, go_local, 4.0, 25.0)
+    d_loc = np.concatenate([loc.dg, loc.du], axis=1)
+    for whole, part, cols in ((y_full, y_loc, [(a, b)]), (d_full, d_loc, [(a, b), (I + a, I + b)])):
+        amax = torch.tensor([np.abs(part).max()], dtype=torch.float64)
+        D.allreduce_amax(amax)
+        assert amax.item() == np.abs(whole).max()
+        codes_w, scales_w, s_enc = o.nvfp4_quantize(whole)
+        codes_p, scales_p, s_p = o.nvfp4_quantize(part, s_enc=o.nvfp4_tensor_scale(amax.item()))
+        assert s_p == s_enc
+        want_c = np.concatenate([codes_w[:, c0:c1] for c0, c1 in cols], axis=1)
+        want_s = np.concatenate([scales_w[:, c0 // 16:c1 // 16] for c0, c1 in cols], axis=1)
+        assert np.array_equal(codes_p, want_c) and np.array_equal(scales_p, want_s)
+        # a shard coded with its own maximum instead would differ from the whole tensor's coding
+        if amax.item() != np.abs(part).max():
+            assert not np.array_equal(o.nvfp4_quantize(part)[1], want_s)
+
+
 def _max_check(rank):
     assert D.max_over_ranks(1.5 + rank) == 2.5
 
 
 def test_tensor_parallel_backward_gloo():
     _run(_tp_check, 37, 520, 11)
+
+
+def test_tensor_parallel_nvfp4_scale_gloo():
+    _run(_tp_nvfp4_check, 29, 512, 12)
 
 
 def test_data_parallel_broadcast_weight_gloo():

@@ -363,3 +363,27 @@ def test_nvfp4_bwd_routed_moe_size_sampled_rows(cuda_device):
     check_nvfp4("d_gate_up (sampled rows)", d[rows.tolist()].cpu().numpy(),
                 s.view(torch.uint8)[rows.tolist()].cpu().numpy(), a, dd, tol, full_tensor=False)
     check_dw("d_w (sampled rows)", d_rw.reshape(-1)[rows.tolist()].cpu().numpy(), ref.dw, ref.sw)
+
+
+def test_nvfp4_amax_only(cuda_device):
+    """amax_given = 2 computes the tensor maximum alone (no codes, scales or
+    weight gradient: their pointers are NULL) and agrees with the maximum the
+    full calls compute; the sharded two-step coding (the maximum, then codes
+    under a given maximum) gives the same bytes as one call."""
+    dev = cuda_device
+    T, I = 90, 512
+    g_h, rw32, go_h = nv_inputs("bf16", T, I, seed=12)
+    gu, go = to_device(g_h, dev), to_device(go_h, dev)
+    rw = to_device(rw32, dev).reshape(T, 1)
+    d, s, a = pkg.situ_glu_fwd_nvfp4(gu, rw, 4.0, 25.0)
+    _, _, a_only = pkg.situ_glu_fwd_nvfp4(gu, rw, 4.0, 25.0, amax_only=True)
+    d2, s2, _ = pkg.situ_glu_fwd_nvfp4(gu, rw, 4.0, 25.0, amax=a_only)
+    bd, bs, ba, bdrw = pkg.situ_glu_bwd_nvfp4(gu, rw, go, 4.0, 25.0)
+    _, _, ba_only, none = pkg.situ_glu_bwd_nvfp4(gu, rw, go, 4.0, 25.0, amax_only=True)
+    bd2, bs2, _, bdrw2 = pkg.situ_glu_bwd_nvfp4(gu, rw, go, 4.0, 25.0, amax=ba_only)
+    torch.cuda.synchronize()
+    assert none is None
+    assert float(a_only.item()) == float(a.item()) and float(ba_only.item()) == float(ba.item())
+    assert torch.equal(d2, d) and torch.equal(s2.view(torch.uint8), s.view(torch.uint8))
+    assert torch.equal(bd2, bd) and torch.equal(bs2.view(torch.uint8), bs.view(torch.uint8))
+    assert torch.equal(bdrw2, bdrw)
