@@ -69,6 +69,11 @@ constexpr int kHeaderBytes = 128;
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kUmmaN >> 3) << 17) |
                             (static_cast<uint32_t>(kBM >> 4) << 24);
 
+// The epilogues' global accesses (plain, L1-cached: measured faster here than
+// the streaming forms).
+__device__ __forceinline__ uint4 epi_ld(const char* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ void epi_st(char* p, const uint4& v) { *reinterpret_cast<uint4*>(p) = v; }
+
 struct Args {
   const int64_t* offsets;  // device [experts + 1]
   int experts;
@@ -133,7 +138,24 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// The wait, with the loaded registers passed through it: their uses cannot be
+// scheduled above the point where the asynchronous load has landed.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[16], uint32_t (&q)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+                 "+r"(q[0]), "+r"(q[1]), "+r"(q[2]), "+r"(q[3]), "+r"(q[4]), "+r"(q[5]), "+r"(q[6]), "+r"(q[7]),
+                 "+r"(q[8]), "+r"(q[9]), "+r"(q[10]), "+r"(q[11]), "+r"(q[12]), "+r"(q[13]), "+r"(q[14]), "+r"(q[15])
+               :
+               : "memory");
+}
 
 // Bounded wait that also gives up once another role has aborted.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -202,7 +224,7 @@ struct Fc1Epilogue {
       uint32_t g[16], u[16];
       tmem_ld16(taddr + c, g);
       tmem_ld16(taddr + kBN + c, u);
-      tmem_ld_wait();
+      tmem_ld_wait(g, u);
       uint32_t q[8];
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
@@ -214,9 +236,8 @@ struct Fc1Epilogue {
               Bf16::pack(fwd_pair_abs<GATE, HAS_LB, F32>(F32::pair(gv, p), F32::pair(uv, p), splat(wbb), a.c));
       }
       if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(yrow + c * 2);
-        dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
-        dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
+        epi_st(yrow + c * 2, make_uint4(q[0], q[1], q[2], q[3]));
+        epi_st(yrow + c * 2 + 16, make_uint4(q[4], q[5], q[6], q[7]));
       }
     }
   }
@@ -243,27 +264,51 @@ struct Fc2Epilogue {
     char* dgrow = a.y + r * a.y_pitch + static_cast<int64_t>(tile.n0) * 2;
     char* durow = dgrow + static_cast<int64_t>(a.inter) * 2;
     float2 acc = make_float2(0.0f, 0.0f);
+    // Chunk c + 16's accumulator columns (TMEM) and saved gate_up values
+    // (global) are requested before chunk c is computed, so their latency
+    // overlaps the arithmetic: this warp is alone on its scheduler.
+    uint32_t d[16];
+    uint4 gn[2], un[2];
+    tmem_ld16(taddr, d);
+    if (valid) {
+#pragma unroll
+      for (int v = 0; v < 2; ++v) {
+        gn[v] = epi_ld(grow + v * 16);
+        un[v] = epi_ld(urow + v * 16);
+      }
+    }
 #pragma unroll 1
     for (int c = 0; c < kUmmaN; c += 16) {
-      uint32_t d[16];
-      tmem_ld16(taddr + c, d);
-      tmem_ld_wait();
+      tmem_ld_wait(d);
+      uint32_t dc[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) dc[i] = d[i];
+      const uint4 gc[2] = {gn[0], gn[1]}, uc[2] = {un[0], un[1]};
+      if (c + 16 < kUmmaN) {  // uniform over the warp
+        tmem_ld16(taddr + c + 16, d);
+        if (valid) {
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            gn[v] = epi_ld(grow + (c + 16) * 2 + v * 16);
+            un[v] = epi_ld(urow + (c + 16) * 2 + v * 16);
+          }
+        }
+      }
       if (valid) {
 #pragma unroll
         for (int v = 0; v < 2; ++v) {
-          const uint4 gv = *reinterpret_cast<const uint4*>(grow + c * 2 + v * 16);
-          const uint4 uv = *reinterpret_cast<const uint4*>(urow + c * 2 + v * 16);
+          const uint4 gv = gc[v], uv = uc[v];
           uint4 dgv, duv;
 #pragma unroll
           for (int p = 0; p < 4; ++p) {
             float2 dg, du;
-            const float2 go = make_float2(__uint_as_float(d[8 * v + 2 * p]), __uint_as_float(d[8 * v + 2 * p + 1]));
+            const float2 go = make_float2(__uint_as_float(dc[8 * v + 2 * p]), __uint_as_float(dc[8 * v + 2 * p + 1]));
             bwd_pair<GATE, HAS_LB, Bf16>(Bf16::pair(gv, p), Bf16::pair(uv, p), go, kdg, kdu, a.c, dg, du, acc);
             Bf16::put(dgv, p, dg);
             Bf16::put(duv, p, du);
           }
-          *reinterpret_cast<uint4*>(dgrow + c * 2 + v * 16) = dgv;
-          *reinterpret_cast<uint4*>(durow + c * 2 + v * 16) = duv;
+          epi_st(dgrow + c * 2 + v * 16, dgv);
+          epi_st(durow + c * 2 + v * 16, duv);
         }
       }
     }
