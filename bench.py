@@ -100,6 +100,9 @@ def source_digest() -> str:
     return h.hexdigest()
 
 
+E2E_CHUNK_ROWS = 2048  # rows per chunk of the host pipeline in the end-to-end measurement
+
+
 def recorded_traffic(kernel: str, workload_name: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel source; None otherwise."""
@@ -1061,14 +1064,23 @@ def run_ours(args):
         outputs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outputs]
         K2 = args.e2e_steps or max(1, min(K, 20))
 
-        def e2e_step():
-            gu.copy_(gu_h, non_blocking=True)
-            go.copy_(go_h, non_blocking=True)
-            rw.copy_(rw_h, non_blocking=True)
-            fwd()
-            bwd()
-            for th, td in zip(outputs_h, outputs):
-                th.copy_(td, non_blocking=True)
+        if variant == "row":
+            # the public host-tensor API: row chunks streamed through the GPU,
+            # uploads, kernels and downloads of successive chunks overlapped
+            pipe = pkg.HostPipeline(I, tdt, chunk_rows=E2E_CHUNK_ROWS, device=dev)
+            y_h, dgu_h, drw_h = outputs_h
+
+            def e2e_step():
+                pipe.run(gu_h, rw_h, go_h, beta, lb, y=y_h, d_gate_up=dgu_h, d_rw=drw_h)
+        else:
+            def e2e_step():
+                gu.copy_(gu_h, non_blocking=True)
+                go.copy_(go_h, non_blocking=True)
+                rw.copy_(rw_h, non_blocking=True)
+                fwd()
+                bwd()
+                for th, td in zip(outputs_h, outputs):
+                    th.copy_(td, non_blocking=True)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -1087,11 +1099,14 @@ def run_ours(args):
         e2e_ms = t.item() / K2
         h2d = input_bytes
         d2h = sum(t.numel() * t.element_size() for t in outputs_h)
-        api = {"mxfp8": "situ_glu_fwd_mxfp8/situ_glu_bwd_mxfp8",
-               "nvfp4": "situ_glu_fwd_nvfp4/situ_glu_bwd_nvfp4"}.get(variant, "situ_glu_fwd/situ_glu_bwd")
+        api = {"mxfp8": "situ_glu_fwd_mxfp8/situ_glu_bwd_mxfp8 on pinned host copies",
+               "nvfp4": "situ_glu_fwd_nvfp4/situ_glu_bwd_nvfp4 on pinned host copies",
+               "row": f"HostPipeline.run on pinned host tensors (chunks of {E2E_CHUNK_ROWS} rows; uploads, "
+                      f"kernels and downloads of successive chunks overlapped on three streams)"}.get(
+                   variant, "situ_glu_fwd/situ_glu_bwd on pinned host copies")
         e2e = {"value": step_bytes * world / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": K2,
-               "api": f"ffn_gated_activation_b200.{api} on pinned host copies"}
+               "api": f"ffn_gated_activation_b200.{api}"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -9,6 +9,7 @@ runs in the hand-written CUDA kernels of libsitu_glu.so behind the C ABI in
 include/situ_glu.h; this package only marshals torch tensors into it.
 """
 from . import abi, distributed
+from .host_pipeline import HostPipeline
 from .abi import NativeLibraryError, SituError
 from .functional import (
     DEFAULT_BETA,
@@ -31,6 +32,7 @@ from .functional import (
 __all__ = [
     "abi",
     "distributed",
+    "HostPipeline",
     "NativeLibraryError",
     "SituError",
     "DEFAULT_BETA",
