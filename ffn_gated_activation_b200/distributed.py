@@ -86,11 +86,18 @@ def situ_glu_bwd_tp(gate_up_local, routing_weights, grad_out_local, beta=functio
     is already complete."""
     lead = tuple(gate_up_local.shape[:-1])
     inter_local = gate_up_local.shape[-1] // 2
-    d_gate_up, d_rw = functional.situ_glu_bwd(gate_up_local, routing_weights, grad_out_local, beta,
-                                              linear_beta, want_drw=want_drw, **kw)
-    if d_rw is not None and tp_drw_needs_allreduce(lead, inter_local, routing_weights):
-        allreduce_drw(d_rw, group)
+    with _on_stream(kw.pop("stream", None)):  # the kernel, then the all-reduce of its result, on one stream
+        d_gate_up, d_rw = functional.situ_glu_bwd(gate_up_local, routing_weights, grad_out_local, beta,
+                                                  linear_beta, want_drw=want_drw, **kw)
+        if d_rw is not None and tp_drw_needs_allreduce(lead, inter_local, routing_weights):
+            allreduce_drw(d_rw, group)
     return d_gate_up, d_rw
+
+
+def _on_stream(stream):
+    """Context that makes ``stream`` current (no-op for None)."""
+    import contextlib
+    return torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
 
 
 def allreduce_amax(amax: torch.Tensor, group=None) -> torch.Tensor:
@@ -106,9 +113,11 @@ def situ_glu_fwd_nvfp4_tp(gate_up_local, routing_weights, beta=functional.DEFAUL
     ``tp_local_gate_up(..., align=16)``): the shard's maximum, the group's
     maximum, then the shard's codes under the whole tensor's scale.  Returns
     (data, scale, amax) as situ_glu_fwd_nvfp4."""
-    _, _, amax = functional.situ_glu_fwd_nvfp4(gate_up_local, routing_weights, beta, linear_beta, amax_only=True)
-    allreduce_amax(amax, group)
-    return functional.situ_glu_fwd_nvfp4(gate_up_local, routing_weights, beta, linear_beta, amax=amax, **kw)
+    with _on_stream(kw.pop("stream", None)):  # the three steps in order on one stream
+        _, _, amax = functional.situ_glu_fwd_nvfp4(gate_up_local, routing_weights, beta, linear_beta,
+                                                   amax_only=True)
+        allreduce_amax(amax, group)
+        return functional.situ_glu_fwd_nvfp4(gate_up_local, routing_weights, beta, linear_beta, amax=amax, **kw)
 
 
 def situ_glu_bwd_nvfp4_tp(gate_up_local, routing_weights, grad_out_local, beta=functional.DEFAULT_BETA,
@@ -117,14 +126,15 @@ def situ_glu_bwd_nvfp4_tp(gate_up_local, routing_weights, grad_out_local, beta=f
     whole tensor's scale (the group's maximum of the shards' maxima), and the
     routing-weight gradient all-reduced as in ``situ_glu_bwd_tp``.  Returns
     (data, scale, amax, d_rw) as situ_glu_bwd_nvfp4."""
-    _, _, amax, _ = functional.situ_glu_bwd_nvfp4(gate_up_local, routing_weights, grad_out_local, beta,
-                                                  linear_beta, amax_only=True)
-    allreduce_amax(amax, group)
-    data, scale, amax, d_rw = functional.situ_glu_bwd_nvfp4(gate_up_local, routing_weights, grad_out_local, beta,
-                                                            linear_beta, want_drw=want_drw, amax=amax, **kw)
-    lead = tuple(gate_up_local.shape[:-1])
-    if d_rw is not None and tp_drw_needs_allreduce(lead, gate_up_local.shape[-1] // 2, routing_weights):
-        allreduce_drw(d_rw, group)
+    with _on_stream(kw.pop("stream", None)):
+        _, _, amax, _ = functional.situ_glu_bwd_nvfp4(gate_up_local, routing_weights, grad_out_local, beta,
+                                                      linear_beta, amax_only=True)
+        allreduce_amax(amax, group)
+        data, scale, amax, d_rw = functional.situ_glu_bwd_nvfp4(gate_up_local, routing_weights, grad_out_local,
+                                                                beta, linear_beta, want_drw=want_drw, amax=amax, **kw)
+        lead = tuple(gate_up_local.shape[:-1])
+        if d_rw is not None and tp_drw_needs_allreduce(lead, gate_up_local.shape[-1] // 2, routing_weights):
+            allreduce_drw(d_rw, group)
     return data, scale, amax, d_rw
 
 
