@@ -2381,6 +2381,7 @@ Span weight_span(const void* p, situ_rw_mode_t mode, int64_t tokens, int64_t str
 
 // rows * pitch + width fits in int64 bytes.
 bool span_fits(int64_t rows, int64_t pitch, int64_t width, int es) {
+  if (width > INT64_MAX / es) return false;  // one row alone
   const int64_t limit = INT64_MAX / es - width;
   return rows <= 1 || (pitch <= limit / (rows - 1));
 }
@@ -3619,7 +3620,10 @@ extern "C" situ_status_t situ_attn_res_fwd(const void* blocks, int64_t nblocks, 
   if (tokens == 0) return SITU_OK;
   if ((nblocks > 0 && blocks == nullptr) || norm_weight == nullptr || proj_weight == nullptr || out == nullptr)
     return fail(SITU_ERR_INVALID_ARG, "blocks, norm_weight, proj_weight or out is NULL");
-  if ((nblocks > 0 && !span_fits(tokens, block_row_stride, nblocks * block_stride, es)) ||
+  // a token's sources span (nblocks - 1) block strides plus one row; the
+  // tokens then add (tokens - 1) row strides to that
+  if ((nblocks > 0 && (!span_fits(nblocks, block_stride, hidden, es) ||
+                       !span_fits(tokens, block_row_stride, (nblocks - 1) * block_stride + hidden, es))) ||
       (prefix != nullptr && !span_fits(tokens, prefix_row_stride, hidden, es)) ||
       !span_fits(tokens, out_row_stride, hidden, oes))
     return fail(SITU_ERR_INVALID_ARG, "tensor extent overflows int64");

@@ -467,6 +467,9 @@ AR_CASES = [
     ("source pitch not 16-byte", dict(block_stride=260, block_row_stride=8 * 260), MISAL),
     ("out overlaps blocks", dict(out=ARB + 512), INVALID),
     ("out overlaps the prefix", dict(out=ARP + 64), INVALID),
+    # 8 sources 2^62 elements apart: nblocks * block_stride wraps in int64 (found by the randomised test)
+    ("source extent overflows int64", dict(block_stride=2 ** 62), INVALID),
+    ("row extent overflows int64", dict(block_row_stride=2 ** 62), INVALID),
 ]
 
 

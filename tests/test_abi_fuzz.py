@@ -77,7 +77,7 @@ REQUIRED = {"fwd": ["gate_up", "out"], "bwd": ["gate_up", "grad_out", "d_gate_up
             "fc1": ["x", "w1", "offsets", "y"], "fc2": ["dout", "w2t", "offsets", "gate_up", "d_gate_up"],
             "attn_res": ["norm_weight", "proj_weight", "out"]}
 # entry points whose byte extents the overflow property below models
-EXTENTS_MODELLED = {"fwd", "bwd", "fwd_mxfp8", "fwd_nvfp4", "bwd_nvfp4"}
+EXTENTS_MODELLED = {"fwd", "bwd", "fwd_mxfp8", "fwd_nvfp4", "bwd_nvfp4", "bwd_mxfp8", "fc1", "fc2", "attn_res"}
 
 
 def field_strategy(name):
@@ -98,18 +98,50 @@ def field_strategy(name):
 def extent_overflows(entry, a, amax_only):
     """Whether the byte extent (rows - 1) * pitch + row of a tensor the call
     uses exceeds int64 -- exact integer arithmetic."""
-    T, I = a["tokens"], a["inter"]
-    es = 2 if a["dtype"] == 0 else 4
+    limit = 2 ** 63 - 1
+    T = a["tokens"]
+    if entry == "attn_res":  # sources [T, B, H] at (row, source) strides, prefix and out [T, H]
+        H, B = a["hidden"], a["nblocks"]
+        es = 2 if a["dtype"] == 0 else 4
+        oes = 2 if a["out_dtype"] == 0 else 4
+        ext = []
+        if a["blocks"] is not None and B > 0 and a["block_row_stride"] >= 0 and a["block_stride"] >= 0:
+            ext.append(((T - 1) * a["block_row_stride"] + (B - 1) * a["block_stride"] + H) * es)
+        if a["prefix"] is not None and a["prefix_row_stride"] >= H:
+            ext.append(((T - 1) * a["prefix_row_stride"] + H) * es)
+        if a["out_row_stride"] >= H:
+            ext.append(((T - 1) * a["out_row_stride"] + H) * oes)
+        return H > 0 and any(e > limit for e in ext)
+    I = a["inter"]
+    es = 2 if a.get("dtype", 0) == 0 else 4
     rw_es = 2 if a["rw_dtype"] == 0 else 4
+    if entry in ("fc1", "fc2"):  # bf16 only; weights [E * 2I or E * I, H]
+        H, E = a["hidden"], a["experts"]
+        if entry == "fc1":
+            spans = [(a["x_row_stride"], H, 2), (a["y_row_stride"], I, 2)]
+            w_rows, w_pitch = E * 2 * I, a["w1_row_stride"]
+        else:
+            spans = [(a["dout_row_stride"], H, 2), (a["gate_up_row_stride"], 2 * I, 2),
+                     (a["d_gate_up_row_stride"], 2 * I, 2)]
+            w_rows, w_pitch = E * I, a["w2t_row_stride"]
+        if w_pitch >= H >= 0 and E > 0 and ((w_rows - 1) * w_pitch + H) * 2 > limit:
+            return True
+        if a["rw_mode"] == abi.SITU_RW_ROW and a["rw"] is not None:
+            spans.append((a["rw_stride"], 1, rw_es))
+            if entry == "fc2" and a.get("d_rw") is not None:
+                spans.append((a["d_rw_stride"], 1, rw_es))
+        return any(w * e > limit or ((T - 1) * p + w) * e > limit for p, w, e in spans if p >= w >= 0)
     spans = [(a["gate_up_row_stride"], 2 * I, es)]
     if entry == "fwd":
         spans.append((a["out_row_stride"], I, es))
-    if entry in ("bwd", "bwd_nvfp4"):
+    if entry in ("bwd", "bwd_nvfp4", "bwd_mxfp8"):
         spans.append((a["grad_out_row_stride"], I, es))
     if entry == "bwd":
         spans.append((a["d_gate_up_row_stride"], 2 * I, es))
     if entry == "fwd_mxfp8":
         spans += [(a["y_data_row_stride"], I, 1), (a["y_scale_row_stride"], I // 32, 1)]
+    if entry == "bwd_mxfp8":
+        spans += [(a["d_gate_up_data_row_stride"], 2 * I, 1), (a["d_gate_up_scale_row_stride"], 2 * I // 32, 1)]
     if entry == "fwd_nvfp4" and not amax_only:
         spans += [(a["y_data_row_stride"], I // 2, 1), (a["y_scale_row_stride"], I // 16, 1)]
     if entry == "bwd_nvfp4" and not amax_only:
@@ -118,7 +150,6 @@ def extent_overflows(entry, a, amax_only):
         spans.append((a["rw_stride"], 1, rw_es))
         if a.get("d_rw") is not None:
             spans.append((a["d_rw_stride"], 1, rw_es))
-    limit = 2 ** 63 - 1
     return any(w * e > limit or ((T - 1) * p + w) * e > limit for p, w, e in spans if p >= w >= 0)
 
 
