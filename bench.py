@@ -33,6 +33,7 @@ time is the max over ranks, and rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -65,7 +66,12 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--config", type=int, default=2, help="workload index (default: routed MoE rows)")
+    p.add_argument("--config", type=int, default=4,
+                   help="workload index (default: the large one, bf16 [131072, 8192])")
+    p.add_argument("--tokens", type=int, default=None,
+                   help="rows of the workload (default: its own); for small profiler captures")
+    p.add_argument("--no-sub", action="store_true",
+                   help="skip the per-workload records of the other target workloads")
     p.add_argument("--beta", type=float, default=None, help="gate beta (default: the workload's first)")
     p.add_argument("--e2e-steps", type=int, default=None)
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-oracle sample budget")
@@ -88,6 +94,30 @@ def measured_peak():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def host_info() -> dict:
+    """The host the CPU figures were taken on: CPU model and core counts."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        avail = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        avail = os.cpu_count()
+    return {"cpu_model": model, "host_cores": os.cpu_count(), "cores_available": avail}
+
+
+def cpu_record(value, unit, sample, cores=1, **extra) -> dict:
+    """A cpu_baseline object: the oracle's rate on ``cores`` threads, with the host it ran on."""
+    return {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample, **host_info(),
+            **extra}
 
 
 def source_digest() -> str:
@@ -296,8 +326,8 @@ def run_reference_attn_res(args, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": ar_config("n/a (host)", 1),
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{rows_per_step} rows per step, {args.steps} steps, single-threaded fp64"},
+            "cpu_baseline": cpu_record(value, "GB/s", f"{rows_per_step} rows per step, {args.steps} steps, "
+                                                      f"single-threaded fp64"),
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)
@@ -407,8 +437,8 @@ def run_ours_attn_res(args, dev, world, rank, local, barrier):
             o.attn_res(d["blocks"], d["prefix"], d["norm_weight"], d["proj_weight"], 1e-6, rows=rows)
             done += rows.size
         secs = time.perf_counter() - t0
-        cpu = {"value": per_row * done / secs / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": f"first {done} of {AR_TOKENS} rows, {secs:.1f} s, single-threaded fp64 oracle"}
+        cpu = cpu_record(per_row * done / secs / 1e9, "GB/s",
+                         f"first {done} of {AR_TOKENS} rows, {secs:.1f} s, single-threaded fp64 oracle")
     if rank == 0:
         line = {"metric": AR_METRIC, "value": gbs * world, "unit": "GB/s", "n_gpus": world, "steps": K,
                 "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -500,6 +530,8 @@ def run_reference(args):
     if rank != 0:
         return 0  # the CPU arm runs once, on rank 0
     wl = workloads.workload(args.config)
+    if args.tokens:
+        wl = dataclasses.replace(wl, tokens=args.tokens)
     beta = args.beta if args.beta is not None else wl.betas[0]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.variant == "fc1":
@@ -543,7 +575,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(wl, beta, "n/a (host)", 1, args.variant),
         "rows_per_s": rows_per_step * args.steps / dt,
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": cpu_record(value, "GB/s", sample),
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -576,7 +608,7 @@ def run_reference_fc1(args, wl, beta, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": fc1_config(wl, beta, "n/a (host)", 1),
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": cpu_record(value, "TFLOP/s", sample),
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -628,8 +660,8 @@ def run_reference_fc2(args, wl, beta, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": cfg,
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{rows.size} rows per step, {args.steps} steps, single-threaded fp64"},
+            "cpu_baseline": cpu_record(value, "TFLOP/s", f"{rows.size} rows per step, {args.steps} steps, "
+                                                         f"single-threaded fp64"),
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)
@@ -718,8 +750,8 @@ def run_ours_fc2(args, wl, beta, dev, world, rank, local, barrier):
             o.fc2_dgrad(d["dout"], d["w2t"], d["offsets"], d["gate_up"], d["routing_weights"], beta, lb, rows=rows)
             done += rows.size
         secs = time.perf_counter() - t0
-        cpu = {"value": 2.0 * H * I * done / secs / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-               "sample": f"first {done} of {T} rows, {secs:.1f} s, single-threaded fp64 FC2-dgrad oracle"}
+        cpu = cpu_record(2.0 * H * I * done / secs / 1e12, "TFLOP/s",
+                         f"first {done} of {T} rows, {secs:.1f} s, single-threaded fp64 FC2-dgrad oracle")
     if rank == 0:
         cfg = fc1_config(wl, beta, "inputs 1.1 GB exceed the 126 MB L2; no flush", world)
         cfg["name"] = f"{wl.name}/fc2"
@@ -853,8 +885,7 @@ def run_ours_fc1(args, wl, beta, dev, world, rank, local, barrier):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, rows_done, secs = fc1_cpu_rate(wl, beta, d, args.cpu_seconds)
-        cpu = {"value": rate, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-               "sample": f"first {rows_done} of {T} rows, {secs:.1f} s, single-threaded fp64 FC1 oracle"}
+        cpu = cpu_record(rate, "TFLOP/s", f"first {rows_done} of {T} rows, {secs:.1f} s, single-threaded fp64 FC1 oracle")
     if rank == 0:
         line = {
             "metric": FC1_METRIC, "value": tflops * world, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
@@ -884,6 +915,126 @@ def run_ours_fc1(args, wl, beta, dev, world, rank, local, barrier):
 
 # ---- our arm -----------------------------------------------------------------------
 
+# The other workloads the 80 %-of-peak target names, each timed on its own
+# after the headline workload: (workload index, gate beta).
+SUB_WORKLOADS = ((2, 4.0), (3, 1.0), (3, 4.0), (3, 16.0), (4, 4.0))
+
+
+def step_stats(ms_list) -> dict:
+    """Mean, median and minimum of per-launch times (microseconds)."""
+    us = [v * 1e3 for v in ms_list]
+    return {"us": sum(us) / len(us), "us_median": statistics.median(us), "us_min": min(us)}
+
+
+def kernel_record(stats: dict, nbytes: int, rows: int, peak: float) -> dict:
+    """Per-kernel figures: GB/s from the mean (the roofline's), the median and
+    the fastest launch, each as a fraction of the measured copy and of 8 TB/s."""
+    gbs = nbytes / stats["us"] / 1e3
+    gbs_med = nbytes / stats["us_median"] / 1e3
+    gbs_best = nbytes / stats["us_min"] / 1e3
+    return {**stats, "bytes": nbytes, "GB/s": gbs, "GB/s_median": gbs_med, "GB/s_best": gbs_best,
+            "pct_of_nominal_8TBs": gbs / NOMINAL_HBM_GBS * 100,
+            "pct_of_nominal_8TBs_median": gbs_med / NOMINAL_HBM_GBS * 100,
+            "frac_of_measured_copy": gbs / peak, "frac_of_measured_copy_median": gbs_med / peak,
+            "rows_per_s": rows / (stats["us"] / 1e6)}
+
+
+def row_kernels(wl):
+    """The kernels the per-row forward and backward launch for this shape (the
+    forward takes 32-byte vectors when a half row is a multiple of 64 vectors
+    and at most 256 threads' worth, every pitch being 32-byte aligned here)."""
+    vpr = wl.inter * wl.elem_bytes // 16
+    fwd = "situ_glu_fwd_wide_kernel" if vpr % 64 == 0 and vpr // 2 <= 256 else "situ_glu_fwd_kernel"
+    return fwd, "situ_glu_bwd_kernel"
+
+
+def measure_workload(pkg, wl, beta, dev, K, warmup, local, allreduce_max):
+    """One workload's forward and backward (per-row weights, native outputs),
+    timed alone: K steps with CUDA events on the launching stream around each
+    pass.  Returns the workload's record."""
+    import torch
+    x = workloads.inputs(wl)
+    T, I = wl.tokens, wl.inter
+    up = lambda a: (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16
+                    else torch.from_numpy(a)).to(dev)
+    gu, go = up(x["gate_up"]), up(x["grad_out"])
+    rw = torch.from_numpy(x["routing_weights"]).reshape(T, 1).to(dev)
+    del x
+    tdt = gu.dtype
+    y = torch.empty(T, I, dtype=tdt, device=dev)
+    d_gu = torch.empty(T, 2 * I, dtype=tdt, device=dev)
+    d_rw = torch.empty(T, 1, dtype=torch.float32, device=dev)
+    input_bytes = (gu.numel() + go.numel()) * gu.element_size() + T * 4
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if input_bytes < 2 * L2_BYTES else None
+    lb = wl.linear_beta
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, warmup)):
+        if flush_buf is not None:
+            flush_buf.zero_()
+        pkg.situ_glu_fwd(gu, rw, beta, lb, out=y)
+        pkg.situ_glu_bwd(gu, rw, go, beta, lb, d_gate_up=d_gu, d_rw=d_rw)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    for k in range(K):
+        if flush_buf is not None:
+            flush_buf.zero_()
+        ev[k][0].record(stream)
+        pkg.situ_glu_fwd(gu, rw, beta, lb, out=y)
+        ev[k][1].record(stream)
+        pkg.situ_glu_bwd(gu, rw, go, beta, lb, d_gate_up=d_gu, d_rw=d_rw)
+        ev[k][2].record(stream)
+    torch.cuda.synchronize()
+    clocks.stop()
+    f = step_stats([e[0].elapsed_time(e[1]) for e in ev])
+    b = step_stats([e[1].elapsed_time(e[2]) for e in ev])
+    vals = allreduce_max([f["us"], f["us_median"], f["us_min"], b["us"], b["us_median"], b["us_min"]])
+    f = dict(zip(("us", "us_median", "us_min"), vals[:3]))
+    b = dict(zip(("us", "us_median", "us_min"), vals[3:]))
+    peak, _ = measured_peak()
+    fk, bk = row_kernels(wl)
+    return {"workload": wl.describe(), "beta": beta, "steps": K,
+            "l2": ("L2 flushed before every step" if flush_buf is not None
+                   else f"inputs ({input_bytes / 1e6:.0f} MB) exceed the {L2_BYTES >> 20} MB L2; no flush"),
+            "fwd": {"kernel": fk, **kernel_record(f, wl.fwd_bytes(), T, peak)},
+            "bwd": {"kernel": bk, **kernel_record(b, wl.bwd_bytes(), T, peak)},
+            "clocks": clocks.summary()}
+
+
+def cpu_oracle_rate_threads(wl, beta, x, seconds: float, threads: int):
+    """The same oracle code as cpu_oracle_rate, with the rows split across
+    ``threads`` threads (each takes the next chunk of rows; the C oracle
+    releases the GIL), until ``seconds`` have passed.  Returns (GB/s, rows)."""
+    from concurrent.futures import ThreadPoolExecutor
+    import oracle
+    o = oracle.load()
+    per_row = (wl.fwd_bytes() + wl.bwd_bytes()) / wl.tokens
+    chunk = max(1, min(64, int(2 ** 20 // wl.inter)))
+    nxt, lock, rows_done = [0], threading.Lock(), [0]
+    t0 = time.perf_counter()
+
+    def worker():
+        while time.perf_counter() - t0 < seconds:
+            with lock:
+                r0 = nxt[0]
+                if r0 >= wl.tokens:
+                    return
+                nxt[0] = min(wl.tokens, r0 + chunk)
+            r1 = min(wl.tokens, r0 + chunk)
+            rows = np.arange(r0, r1, dtype=np.int64)
+            o.fwd(x["gate_up"], x["routing_weights"], beta, wl.linear_beta, rows=rows)
+            o.bwd(x["gate_up"], x["routing_weights"], x["grad_out"], beta, wl.linear_beta, rows=rows)
+            with lock:
+                rows_done[0] += r1 - r0
+
+    with ThreadPoolExecutor(max_workers=threads) as pool:
+        for fut in [pool.submit(worker) for _ in range(threads)]:
+            fut.result()
+    dt = time.perf_counter() - t0
+    return per_row * rows_done[0] / dt / 1e9, rows_done[0], dt
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -907,7 +1058,15 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
+    def allreduce_max(vals):
+        t = torch.tensor(list(vals), dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return t.tolist()
+
     wl = workloads.workload(args.config)
+    if args.tokens:
+        wl = dataclasses.replace(wl, tokens=args.tokens)
     beta = args.beta if args.beta is not None else wl.betas[0]
     if args.variant == "fc1":
         return run_ours_fc1(args, wl, beta, dev, world, rank, local, barrier)
@@ -1038,13 +1197,14 @@ def run_ours(args):
     peak, peak_src = measured_peak()
     fwd_us, bwd_us = fwd_sum / K * 1e3, bwd_sum / K * 1e3
     fwd_gbs, bwd_gbs = fwd_bytes / fwd_us / 1e3, bwd_bytes / bwd_us / 1e3
-    # the kernels each pass launches for this form and shape (the forward's
-    # layout follows the library's own choice: 32-byte vectors when a half row
-    # is a multiple of 64 vectors and every pitch is 32-byte aligned)
-    vpr = I * (2 if wl.dtype == "bf16" else 4) // 16
+    # median and fastest launch of each pass, max over ranks
+    fs, bs = step_stats(fwd_ms), step_stats(bwd_ms)
+    mm = allreduce_max([fs["us_median"], fs["us_min"], bs["us_median"], bs["us_min"]])
+    fs = {"us": fwd_us, "us_median": mm[0], "us_min": mm[1]}
+    bs = {"us": bwd_us, "us_median": mm[2], "us_min": mm[3]}
+    # the kernels each pass launches for this form and shape
     fwd_kernel, bwd_kernel = {
-        "row": ("situ_glu_fwd_wide_kernel" if vpr % 64 == 0 and vpr // 2 <= 256 else "situ_glu_fwd_kernel",
-                "situ_glu_bwd_kernel"),
+        "row": row_kernels(wl),
         "col": ("situ_glu_fwd_ew_kernel", "situ_glu_bwd_ew_kernel"),
         "full": ("situ_glu_fwd_ew_kernel", "situ_glu_bwd_ew_kernel"),
         "mxfp8": ("situ_glu_fwd_quant_kernel<MxQuant>", "situ_glu_bwd_quant_kernel<MxQuant>"),
@@ -1111,17 +1271,31 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, rows_done, secs = cpu_oracle_rate(wl, beta, x, args.cpu_seconds, variant)
-        cpu = {"value": rate, "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": f"first {rows_done} of {T} rows, fwd + bwd, {secs:.1f} s, single-threaded fp64"}
+        extra = {}
+        if variant == "row":
+            threads = host_info()["cores_available"] or 1
+            prate, prows, psecs = cpu_oracle_rate_threads(wl, beta, x, args.cpu_seconds, threads)
+            extra["all_cores"] = {"value": prate, "unit": "GB/s", "cores": threads,
+                                  "sample": f"first {prows} of {T} rows, fwd + bwd, {psecs:.1f} s, the same fp64 "
+                                            f"oracle code with the rows split across {threads} threads"}
+        cpu = cpu_record(rate, "GB/s", f"first {rows_done} of {T} rows, fwd + bwd, {secs:.1f} s, "
+                                       f"single-threaded fp64", **extra)
+    del x
 
-    kernels = {
-        fwd_kernel: {"us": fwd_us, "bytes": fwd_bytes, "GB/s": fwd_gbs,
-                     "pct_of_nominal_8TBs": fwd_gbs / NOMINAL_HBM_GBS * 100,
-                     "frac_of_measured_copy": fwd_gbs / peak, "rows_per_s": T / (fwd_us / 1e6)},
-        bwd_kernel: {"us": bwd_us, "bytes": bwd_bytes, "GB/s": bwd_gbs,
-                     "pct_of_nominal_8TBs": bwd_gbs / NOMINAL_HBM_GBS * 100,
-                     "frac_of_measured_copy": bwd_gbs / peak, "rows_per_s": T / (bwd_us / 1e6)},
-    }
+    # The other target workloads, each timed alone after the headline one.
+    subs = None
+    if variant == "row" and not args.no_sub and not args.tokens:
+        del outputs, gu, go, rw, y, d_gu, d_rw, flush_buf
+        torch.cuda.empty_cache()
+        subs = {}
+        for idx, b_ in SUB_WORKLOADS:
+            if idx == args.config and b_ == beta:
+                continue
+            w_ = workloads.workload(idx)
+            subs[f"{w_.name} beta={b_:g}"] = measure_workload(pkg, w_, b_, dev, K, args.warmup, local, allreduce_max)
+            torch.cuda.empty_cache()
+
+    kernels = {fwd_kernel: kernel_record(fs, fwd_bytes, T, peak), bwd_kernel: kernel_record(bs, bwd_bytes, T, peak)}
     roofline = {"bound": "hbm", "kernel": bwd_kernel, "achieved": bwd_gbs, "peak": peak,
                 "unit": "GB/s", "frac": bwd_gbs / peak, "peak_source": f"{peak_src} copy bandwidth",
                 "traffic": traffic}
@@ -1159,6 +1333,8 @@ def run_ours(args):
             "device_status": pkg.abi.situ_glu_device_status(0),
             "device": torch.cuda.get_device_name(dev),
         }
+        if subs is not None:
+            line["workloads"] = subs
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -3319,10 +3319,12 @@ int situ_glu_set_max_ctas(int max_ctas) {
 // Some callers cannot allocate device memory at the point where they run the
 // backward: engines that reserve all of HBM up front and hand their kernels
 // only the buffers they planned, or plain C callers with no CUDA allocator of
-// their own.  situ_glu_bwd needs caller-owned scratch in one mode (a routing
-// weight broadcast to every row: per-row partial sums, 4 bytes per row).  The
-// entry point below takes that scratch from a fixed array that lives in this
-// library instead, so its caller passes only inputs and outputs.
+// their own.  situ_glu_bwd needs caller-owned scratch in two modes when the
+// weight gradient is wanted (a routing weight broadcast to every row: one
+// fp32 partial per row; a per-column weight: one fp32 partial per column per
+// 16-row chunk).  The entry point below takes that scratch from a fixed array
+// that lives in this library instead, so its caller passes only inputs and
+// outputs.  The cached address is valid until the device is reset.
 
 namespace {
 

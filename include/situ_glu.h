@@ -441,19 +441,25 @@ int situ_glu_device_status(int clear);
  * no counterpart of this entry point: it exists for callers that cannot
  * allocate device memory where they run the backward (an engine that
  * reserves all of HBM at start-up and gives its kernels only planned
- * buffers, or a C caller without a CUDA allocator), for the one mode that
- * needs scratch: a routing weight broadcast to every row (SITU_RW_SCALAR with
- * d_rw != NULL), whose per-row partial sums then go to a fixed 1 MiB array
- * inside this library instead of a caller workspace.
- *   - Limit: 1 MiB of scratch -- 262144 rows in that mode (per-column
- *     weights, SITU_RW_COL, use it too: ceil(tokens / 64) * inter * 4 bytes);
- *     more returns SITU_ERR_UNSUPPORTED before anything is launched.  Other
- *     modes need no scratch and have no limit beyond situ_glu_bwd's.
+ * buffers, or a C caller without a CUDA allocator).  Two modes need
+ * scratch when d_rw != NULL, and in both it comes from a fixed 1 MiB array
+ * inside this library instead of a caller workspace: a routing weight
+ * broadcast to every row (SITU_RW_SCALAR: one fp32 partial per row) and a
+ * per-column weight (SITU_RW_COL: one fp32 partial per column per chunk of
+ * 16 rows).
+ *   - Limit: the bytes situ_glu_bwd_workspace_bytes reports must not exceed
+ *     1 MiB (1048576): tokens * 4 for SITU_RW_SCALAR, i.e. at most 262144
+ *     rows; ceil(tokens / 16) * inter * 4 for SITU_RW_COL, each rounded up
+ *     to 256 (at inter = 4096: at most 1024 rows).  More returns
+ *     SITU_ERR_UNSUPPORTED before anything is launched.  Other modes need no
+ *     scratch and have no limit beyond situ_glu_bwd's.
  *   - Allocates nothing (no cudaMalloc, cudaFree or allocating library call).
  *     The array exists once per GPU that loads the library, until exit.
  *   - The first call on a device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture.
+ *     that device current) and caches it for the life of the process; make
+ *     that first call before any stream capture.  cudaDeviceReset discards
+ *     the device's copy of the array, and the cached address with it: do not
+ *     call this entry point on a device after resetting it.
  *   - Every call shares the one array, and it keeps whatever the last call
  *     left in it (nothing in it has to start at zero).  Calls whose kernels
  *     overlap on the GPU -- on different streams, or from different threads

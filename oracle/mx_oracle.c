@@ -215,6 +215,10 @@ double situ_oracle_nvfp4_tensor_scale(double amax) {
   if (!(amax > 0.0) || isinf(amax)) return 1.0;
 #if SITU_ORACLE_MUTANT == 34
   return 1.0; /* planted: no tensor scale */
+#elif SITU_ORACLE_MUTANT == 35
+  return E4M3_MAX / amax; /* planted: the E2M1 range left out */
+#elif SITU_ORACLE_MUTANT == 36
+  return amax / (E4M3_MAX * E2M1_MAX); /* planted: inverted */
 #else
   return E4M3_MAX * E2M1_MAX / amax;
 #endif

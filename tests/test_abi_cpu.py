@@ -522,3 +522,37 @@ def test_fc2_workspace_query(native_lib_path):
     assert abi.situ_glu_fc2_dgrad_workspace_bytes(1000, 2048, 1) == (1000 * 8 * 4 + 255) // 256 * 256
     assert abi.situ_glu_fc2_dgrad_workspace_bytes(1000, 2048, 0) == 0
     assert abi.situ_glu_fc2_dgrad_workspace_bytes(0, 2048, 1) == 0
+
+
+def _no_alloc_limit_from_header():
+    text = open(os.path.join(ROOT, "include", "situ_glu.h")).read()
+    doc = text[:text.index("situ_status_t situ_glu_bwd_no_alloc(")]
+    doc = doc[doc.rindex("/*"):]
+    flat = " ".join(re.sub(r"^\s*\*", " ", doc, flags=re.M).split())
+    limit = int(re.search(r"1 MiB \((\d+)\)", flat).group(1))
+    rows_scalar = int(re.search(r"at most (\d+) rows; ceil\(tokens / 16\) \* inter \* 4", flat).group(1))
+    col_inter, col_rows = map(int, re.search(r"at inter = (\d+): at most (\d+) rows", flat).groups())
+    return limit, rows_scalar, col_inter, col_rows
+
+
+def test_no_alloc_limit_matches_the_workspace_query(native_lib_path):
+    """The allocation-free backward's documented limit is exactly the bytes the
+    workspace query reports at the boundary rows of both scratch modes, and one
+    row more is rejected on the host (SITU_ERR_UNSUPPORTED, nothing launched)."""
+    COL = abi.SITU_RW_COL
+    limit, rows_scalar, col_inter, col_rows = _no_alloc_limit_from_header()
+    assert limit == 1 << 20
+    ws = abi.situ_glu_bwd_workspace_bytes
+    assert ws(rows_scalar, 64, SCALAR, 1) == limit < ws(rows_scalar + 1, 64, SCALAR, 1)
+    assert ws(col_rows, col_inter, COL, 1) == limit < ws(col_rows + 1, col_inter, COL, 1)
+    assert col_rows == 16 * (limit // (col_inter * 4))
+
+    def call(tokens, inter, mode):
+        return abi.situ_glu_bwd_no_alloc(GU, BF16, tokens, inter, 2 * inter, RW, F32, mode, 1, 4.0, 1, 25.0,
+                                         GO, inter, DGU, 2 * inter, DRW, 1, 0)
+
+    # Only the rejected side is called: a size within the limit would go on to
+    # the device.
+    assert call(rows_scalar + 1, 64, SCALAR) == UNSUP
+    assert "262144" in abi.situ_glu_last_error()
+    assert call(col_rows + 1, col_inter, COL) == UNSUP

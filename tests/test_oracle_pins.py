@@ -455,14 +455,25 @@ def pin_e2m1_nearest_even(o):
 
 
 def pin_nvfp4_blocks(o):
-    """Tensor scale 2688 / amax; each 16-element block's scale is torch's E4M3
-    conversion of amax_b * S_enc / 6; element codes are the nearest E2M1 of
-    v * S_enc / s_b; decoded values lie within half an E2M1 step (scaled) of v."""
+    """The two scaling levels of NVFP4 as consequences of their definition:
+    the tensor scale maps the tensor's largest magnitude onto the top of both
+    formats at once, so the block holding it gets the largest E4M3 scale (448)
+    and that element the largest E2M1 code (6), and no block scale saturates;
+    each 16-element block's scale is torch's E4M3 conversion of
+    amax_b * S_enc / 6; decoded codes times s_b / S_enc lie within half an
+    E2M1 step (scaled) of v."""
     rng = np.random.default_rng(RNG_SEED + 14)
     v = rng.standard_normal((5, 64)) * np.exp2(rng.integers(-6, 6, (5, 1)))
     v[2, 16:32] = 0.0
     codes, scales, s_enc = o.nvfp4_quantize(v)
-    assert s_enc == 448.0 * 6.0 / np.abs(v).max()
+    top = np.unravel_index(np.argmax(np.abs(v)), v.shape)
+    assert o.e4m3_decode(scales[top[0], top[1] // 16:top[1] // 16 + 1])[0] == 448.0
+    assert o.e2m1_decode(codes[top[0], top[1]:top[1] + 1])[0] == np.sign(v[top]) * 6.0
+    assert o.e4m3_decode(scales).max() == 448.0
+    # so the largest element decodes back to itself: code x block scale / S_enc
+    top_dec = (o.e2m1_decode(codes[top[0], top[1]:top[1] + 1])[0]
+               * o.e4m3_decode(scales[top[0], top[1] // 16:top[1] // 16 + 1])[0] / s_enc)
+    assert abs(top_dec - v[top]) <= 1e-15 * abs(v[top])
     for r in range(5):
         for b in range(4):
             blk = v[r, 16 * b:16 * b + 16]
@@ -770,6 +781,8 @@ MUTANTS = {
     32: "E2M1 ties to the larger magnitude",
     33: "NVFP4 block scale from amax / 4",
     34: "NVFP4 tensor scale not applied",
+    35: "NVFP4 tensor scale 448 / amax (the E2M1 range left out)",
+    36: "NVFP4 tensor scale inverted (amax / 2688)",
 }
 
 
