@@ -181,8 +181,9 @@ struct Tile {
 };
 
 // Tile t (numbered expert by expert; inside an expert, groups of kGroupM row
-// tiles sweep all column tiles).  first_tile[e] is the first tile of expert e,
-// first_tile[experts] the total; [lo[e], hi[e]) its rows.
+// tiles of BM rows sweep all column tiles).  first_tile[e] is the first tile
+// of expert e, first_tile[experts] the total; [lo[e], hi[e]) its rows.
+template <int BM = kBM>
 __device__ __forceinline__ Tile decode_tile(int t, const int* first_tile, const int64_t* lo, const int64_t* hi,
                                             int experts, int n_tiles, int out_cols) {
   int left = 0, right = experts - 1;  // the last e with first_tile[e] <= t
@@ -193,17 +194,49 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* first_tile, const 
   const int e = left;
   const int local = t - first_tile[e];
   const int64_t r0 = lo[e], r1 = hi[e];
-  const int m_tiles = static_cast<int>((r1 - r0 + kBM - 1) / kBM);
+  const int m_tiles = static_cast<int>((r1 - r0 + BM - 1) / BM);
   const int group = local / (kGroupM * n_tiles);
   const int first_m = group * kGroupM;
   const int group_m = min(kGroupM, m_tiles - first_m);
   const int within = local - group * kGroupM * n_tiles;
   Tile tile;
   tile.expert = e;
-  tile.m0 = r0 + static_cast<int64_t>(first_m + within % group_m) * kBM;
+  tile.m0 = r0 + static_cast<int64_t>(first_m + within % group_m) * BM;
   tile.m_end = r1;
   tile.n0 = (within / group_m) * out_cols;
   return tile;
+}
+
+// Row range [lo_e, hi_e) of each expert (offsets clamped to [0, tokens], a
+// decreasing pair read as empty) and its first tile of BM rows: lane l of the
+// calling warp takes a contiguous run of experts, a warp scan adds the runs'
+// tile counts.
+template <int BM>
+__device__ __forceinline__ void scan_experts(const Args& a, int n_tiles, int lane, int64_t* lo, int64_t* hi,
+                                             int* first_tile) {
+  const int per = (a.experts + 31) / 32;
+  const int e0 = min(a.experts, lane * per), e1 = min(a.experts, e0 + per);
+  int count = 0;
+  for (int e = e0; e < e1; ++e) {
+    int64_t r0 = a.offsets[e], r1 = a.offsets[e + 1];
+    r0 = r0 < 0 ? 0 : (r0 > a.tokens ? a.tokens : r0);
+    r1 = r1 < r0 ? r0 : (r1 > a.tokens ? a.tokens : r1);
+    lo[e] = r0;
+    hi[e] = r1;
+    count += static_cast<int>((r1 - r0 + BM - 1) / BM) * n_tiles;
+  }
+  int incl = count;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  int run = incl - count;
+  for (int e = e0; e < e1; ++e) {
+    first_tile[e] = run;
+    run += static_cast<int>((hi[e] - lo[e] + BM - 1) / BM) * n_tiles;
+  }
+  if (lane == 31) first_tile[a.experts] = incl;
 }
 
 // FC1: B = the expert's gate rows [n0, n0 + 128) then its up rows; the
@@ -354,34 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 0) {
-    // Row range [lo_e, hi_e) of each expert (offsets clamped to [0, tokens],
-    // a decreasing pair read as empty) and its first tile: lane l takes a
-    // contiguous run of experts, a warp scan adds the runs' tile counts.
-    const int per = (a.experts + 31) / 32;
-    const int e0 = min(a.experts, lane * per), e1 = min(a.experts, e0 + per);
-    int count = 0;
-    for (int e = e0; e < e1; ++e) {
-      int64_t r0 = a.offsets[e], r1 = a.offsets[e + 1];
-      r0 = r0 < 0 ? 0 : (r0 > a.tokens ? a.tokens : r0);
-      r1 = r1 < r0 ? r0 : (r1 > a.tokens ? a.tokens : r1);
-      lo[e] = r0;
-      hi[e] = r1;
-      count += static_cast<int>((r1 - r0 + kBM - 1) / kBM) * n_tiles;
-    }
-    int incl = count;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    int run = incl - count;
-    for (int e = e0; e < e1; ++e) {
-      first_tile[e] = run;
-      run += static_cast<int>((hi[e] - lo[e] + kBM - 1) / kBM) * n_tiles;
-    }
-    if (lane == 31) first_tile[a.experts] = incl;
-  }
+  if (warp == 0) scan_experts<kBM>(a, n_tiles, lane, lo, hi, first_tile);
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(kTmemCols)
@@ -509,6 +515,287 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if (warp == 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols) : "memory");
+}
+
+// ---- Two-SM form (tcgen05 cta_group::2) ---------------------------------------
+// A cluster of two CTAs on two SMs computes a 256-row tile: CTA r of the pair
+// stages token rows [m0 + 128 r, m0 + 128 r + 128) of A and half of B (FC1:
+// the gate rows for r = 0, the up rows for r = 1; FC2: B rows [n0 + 128 r,
+// n0 + 128 r + 128)) in its own shared memory, and one thread of CTA 0 issues
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16), which reads both CTAs'
+// halves and leaves each CTA's 128 accumulator rows (all 256 columns) in that
+// CTA's TMEM.  Each SM so reads half of B per K slice instead of all of it:
+// a third fewer operand bytes per FLOP from L2.  The epilogue is the one-SM
+// kernel's, per CTA.  No load is multicast: every CTA loads its own tiles,
+// whose completion bytes both count on CTA 0's stage barrier (the loads'
+// cta_group::2 form), and CTA 0's MMA commits arrive on both CTAs' barriers.
+constexpr int kBM2 = 2 * kBM;                      // token rows per cluster tile
+constexpr int kStages2 = 6;
+constexpr int kStageBytes2 = kABytes + kBHalfBytes;  // 32 KiB per CTA
+// Header after the ring: 17 mbarriers, the TMEM base and the abort flag; then
+// the per-expert tables.
+constexpr int kHeaderBytes2 = 256;
+// kind::f16, fp32 accumulator, bf16 A and B, K-major, N = 256, M = 256.
+constexpr uint32_t kIdesc2 = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kUmmaN >> 3) << 17) |
+                             (static_cast<uint32_t>(kBM2 >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_index() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_count() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// The shared::cluster address of the same shared-memory location in CTA `rank`.
+__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Arrive on an mbarrier of either CTA of the cluster (shared::cluster address).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA load into this CTA's shared memory whose completion bytes count on the
+// mbarrier at `bar` (a shared::cluster address; here CTA 0's).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                                 uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8, %9, %10, %11, %12}, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc2), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u),
+      "r"(0u), "r"(0u));
+}
+// Arrive on the mbarrier at this offset in both CTAs once every MMA issued so
+// far by this thread is done.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+// Arrive on this CTA's own mbarrier once this thread's MMAs are done.
+__device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ bool wait_or_abort_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  while (!mbar_try_wait_cluster(bar, parity)) {
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      atomicExch(&g_device_status, kStatusWaitExpired);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+static_assert((2 * kStages2 + 4 * kAccBufs / 2 + 1) * 8 + 8 <= kHeaderBytes2, "2-SM header overflows");
+
+template <class Epi, int GATE, bool HAS_LB>
+__global__ void __launch_bounds__(kThreads, 1)
+    situ_fused_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                               const Args a) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  unsigned char* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  unsigned char* ring = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages2 * kStageBytes2);
+  uint64_t* empty = full + kStages2;
+  uint64_t* acc_full = empty + kStages2;
+  uint64_t* acc_empty = acc_full + kAccBufs;
+  uint64_t* drain = acc_empty + kAccBufs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int64_t* lo = reinterpret_cast<int64_t*>(smem + kStages2 * kStageBytes2 + kHeaderBytes2);  // [experts]
+  int64_t* hi = lo + a.experts;                                                            // [experts]
+  int* first_tile = reinterpret_cast<int*>(hi + a.experts);                                // [experts + 1]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int cl = static_cast<int>(cluster_index()), ncl = static_cast<int>(cluster_count());
+  const int n_tiles = a.inter / Epi::kOutCols;
+  const int k_blocks = a.hidden / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages2; ++s) {
+      mbar_init(&full[s], 1);   // CTA 0's producer arrives; both CTAs' copies add bytes
+      mbar_init(&empty[s], 1);  // CTA 0's MMA commit
+    }
+    for (int b = 0; b < kAccBufs; ++b) {
+      mbar_init(&acc_full[b], 1);                 // CTA 0's MMA commit
+      mbar_init(&acc_empty[b], 2 * kEpiThreads);  // every epilogue thread of both CTAs
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0) scan_experts<kBM2>(a, n_tiles, lane, lo, hi, first_tile);
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = first_tile[a.experts];
+
+  if (warp == 0) {
+    // ---- TMA producer (both CTAs) ----
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued = 0;
+    bool ok = true;
+    for (int t = cl; ok && t < total; t += ncl) {
+      const Tile tile = decode_tile<kBM2>(t, first_tile, lo, hi, a.experts, n_tiles, Epi::kOutCols);
+      int32_t wrow0, wrow1;
+      Epi::b_rows(a, tile, wrow0, wrow1);
+      const int32_t wrow = leader ? wrow0 : wrow1;
+      const int32_t arow = static_cast<int32_t>(tile.m0 + static_cast<int64_t>(rank) * kBM);
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        if (!wait_or_abort_cluster(&empty[stage], phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          unsigned char* st = ring + stage * kStageBytes2;
+          const uint32_t bar = peer_addr(&full[stage], 0);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes2);
+          tma_load_2d_pair(st, &tmap_x, kb * kBK, arow, bar);
+          tma_load_2d_pair(st + kABytes, &tmap_w, kb * kBK, wrow, bar);
+        }
+        __syncwarp();
+        issued |= 1u << stage;
+        if (++stage == kStages2) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && leader) {
+      // Aborted: let the copies of both CTAs land (they count on CTA 0's
+      // barriers) before the cluster exits; bounded.
+      for (int s = 0; s < kStages2; ++s) {
+        if (!(issued & (1u << s))) continue;
+        const uint32_t ph = (s < stage) ? phase : (phase ^ 1u);
+        const unsigned long long t0 = global_timer_ns();
+        while (!mbar_try_wait_cluster(&full[s], ph) && global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (leader) {
+      // ---- MMA issuer (CTA 0 only) ----
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t acc_phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = cl; ok && t < total; t += ncl, ++it) {
+        const int b = it & 1;
+        if (!wait_or_abort_cluster(&acc_empty[b], ((acc_phase >> b) & 1u) ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * kAccCols);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!wait_or_abort_cluster(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t a_addr = smem_u32(ring + stage * kStageBytes2);
+            const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+            for (int kk = 0; kk < kBK / kUmmaK; ++kk)
+              umma_bf16_pair(d_tmem, smem_desc_sw128(a_addr + kk * kUmmaK * 2),
+                             smem_desc_sw128(b_addr + kk * kUmmaK * 2), (kb | kk) != 0 ? 1u : 0u);
+            umma_commit_pair(&empty[stage]);  // both CTAs' stage is free once these MMAs have read it
+          }
+          __syncwarp();
+          if (++stage == kStages2) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (lane == 0) umma_commit_pair(&acc_full[b]);  // both CTAs' accumulator rows are complete
+        __syncwarp();
+        acc_phase ^= 1u << b;
+      }
+      if (!ok || *abort_flag) {
+        if (lane == 0) umma_commit_pair_local(drain);
+        __syncwarp();
+        const unsigned long long t0 = global_timer_ns();
+        while (!mbar_try_wait_cluster(drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else {
+    // ---- epilogue: warps 2-5 of both CTAs, one accumulator row per thread ----
+    const int quarter = warp & 3;
+    const int row_in_tile = static_cast<int>(rank) * kBM + quarter * 32 + lane;
+    uint32_t acc_phase = 0;
+    int it = 0;
+    for (int t = cl; t < total; t += ncl, ++it) {
+      const int b = it & 1;
+      if (!wait_or_abort_cluster(&acc_full[b], (acc_phase >> b) & 1u, abort_flag)) break;
+      tc_fence_after();
+      const Tile tile = decode_tile<kBM2>(t, first_tile, lo, hi, a.experts, n_tiles, Epi::kOutCols);
+      const int64_t row = tile.m0 + row_in_tile;
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * kAccCols);
+      Epi::template run<GATE, HAS_LB>(a, tile, row, row < tile.m_end, taddr);
+      tc_fence_before();
+      mbar_arrive_remote(peer_addr(&acc_empty[b], 0));
+      acc_phase ^= 1u << b;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while the pair's MMAs or copies may touch its memory
+  tc_fence_after();
+  if (warp == 1)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols) : "memory");
 }
 
 }  // namespace fc1

@@ -375,6 +375,15 @@ __device__ __forceinline__ float2 fwd_pair_abs(Bits2 gb, Bits2 ub, float2 wbb, c
   return xor_sign2(mul2(num, mul2(rcp2(den), wbb)), s);
 }
 
+// Whether the backward of a pair takes the signed gate form: bf16 outputs at
+// beta = 4 (measured on B200: 5 % less time for the bf16 backward, the same
+// results within the tolerance).  fp32 outputs need the |g| form's accuracy
+// for tiny results; other betas keep it too.
+template <int GATE, typename S>
+struct SignedBwd {
+  static constexpr bool value = GATE == kGateSquare && std::is_same<S, Bf16>::value;
+};
+
 // Backward of a pair.  With A = (1 + E_t)(1 + E_s), B = 1 + E_u (1 without a
 // linear beta), sig as above and
 //   tq  = (beta/4) tanh(g/beta) (1 + E_t)              (= (beta/4) s_g (1 - E_t))
@@ -390,14 +399,34 @@ __device__ __forceinline__ float2 fwd_pair_abs(Bits2 gb, Bits2 ub, float2 wbb, c
 template <int GATE, bool HAS_LB, typename S>
 __device__ __forceinline__ void bwd_pair(Bits2 gb, Bits2 ub, float2 go, float2 kdg, float2 kdu, const Coeffs& c,
                                          float2& dg, float2& du, float2& acc) {
-  const GateAbs e = gate_abs<GATE, S>(gb, c);
-  const float2 sig = select_neg2(gb, e.Es, splat(1.0f));
-  const float2 opt = add2(splat(1.0f), e.Et), ops = add2(splat(1.0f), e.Es);
-  const float2 A = mul2(opt, ops);
-  float2 tq = xor_sign2(e.emt, gb);
-  if (GATE != kGateSquare) tq = mul2(tq, splat(0.25f * c.beta));  // beta = 4: the factor is 1
-  const float2 tgA = mul2(mul2(tq, sig), A);                       // T_g A^2 / 4
-  const float2 ng = fma2(mul2(e.Et, sig), ops, mul2(mul2(tq, opt), e.Es));  // T_g' A^2 / 4
+  float2 A, tgA, ng;
+  if constexpr (SignedBwd<GATE, S>::value) {
+    // Signed form (beta = 4, bf16 outputs), as in the bf16 forward: with
+    // H = exp(-g/2) and Hs = H^2 = exp(-g) for g of either sign,
+    //   T_g  = 4 (1 - H) / A,                 A = (1 + H)(1 + Hs),
+    //   T_g' = 4 [H (1 + Hs) + (1 - H)(1 + H) Hs] / A^2,
+    // so no |g|, sign flip or select is needed.  The exponent argument is
+    // clamped at 20 (g >= -27.7: H <= 2^20, A <= 2^60, (A B)^2 <= 2^122), where
+    // |T_g| < 4e-12 and |T_g'| < 1e-11: far below a bf16 output's absolute
+    // resolution of the tolerance.
+    float2 y = mul2(as_f2(gb), splat(c.kt));
+    y = make_float2(max_nan(y.x, -20.0f), max_nan(y.y, -20.0f));
+    const float2 H = ex2_neg2(y), Hs = mul2(H, H);
+    const float2 em = one_minus_exp2_neg<S>(y, H);  // 1 - H
+    const float2 opH = add2(splat(1.0f), H), opHs = add2(splat(1.0f), Hs);
+    A = mul2(opH, opHs);
+    tgA = mul2(em, A);                                // T_g A^2 / 4
+    ng = fma2(H, opHs, mul2(mul2(em, opH), Hs));      // T_g' A^2 / 4
+  } else {
+    const GateAbs e = gate_abs<GATE, S>(gb, c);
+    const float2 sig = select_neg2(gb, e.Es, splat(1.0f));
+    const float2 opt = add2(splat(1.0f), e.Et), ops = add2(splat(1.0f), e.Es);
+    A = mul2(opt, ops);
+    float2 tq = xor_sign2(e.emt, gb);
+    if (GATE != kGateSquare) tq = mul2(tq, splat(0.25f * c.beta));  // beta = 4: the factor is 1
+    tgA = mul2(mul2(tq, sig), A);                                    // T_g A^2 / 4
+    ng = fma2(mul2(e.Et, sig), ops, mul2(mul2(tq, opt), e.Es));      // T_g' A^2 / 4
+  }
   if (HAS_LB) {
     float2 Eu;
     const float2 su = xor_sign2(up_emu<S, typename UpSeries<S>::type>(ub, c, Eu), ub);  // T_u B / beta_L
@@ -746,6 +775,120 @@ __global__ void SITU_BWD_BOUNDS situ_glu_bwd_kernel(const BwdArgs a) {
       }
     }
   }
+}
+
+// ---- Backward with a shared-memory row ring (cp.async) ----------------------
+// The same per-row work as situ_glu_bwd_kernel's pipelined path, but the rows
+// ahead travel into a shared-memory ring by per-thread asynchronous copies
+// instead of registers: kBwdDepth rows are in flight per CTA without holding
+// a register for them.  Each thread copies and reads back only its own
+// 16-byte slots, so its own cp.async.wait_group is the only synchronisation
+// the data needs.  Stage (i + depth) mod (depth + 1) receives row i + depth
+// while row i is read from stage i mod (depth + 1): the stage refilled was
+// read one iteration earlier, and those values have been consumed since.
+#ifndef SITU_BWD_ASYNC
+#define SITU_BWD_ASYNC 0
+#endif
+constexpr int kBwdDepth = SITU_BWD_ASYNC;  // rows in flight per CTA; 0 selects the register-prefetch kernel
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem))),
+               "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds16(const unsigned char* p) { return *reinterpret_cast<const uint4*>(p); }
+
+template <typename S, int GATE, bool HAS_LB>
+__global__ void __launch_bounds__(kMaxThreads) situ_glu_bwd_async_kernel(const BwdArgs a) {
+  constexpr int kDepth = kBwdDepth > 0 ? kBwdDepth : 1;
+  constexpr int kStagesRing = kDepth + 1;
+  extern __shared__ __align__(16) unsigned char bwd_ring[];  // [stage][6 slots][nt][16 bytes]
+  __shared__ float red[2][kMaxThreads / 32];
+  const int nt = blockDim.x;
+  const int j = threadIdx.x, j2 = j + nt;
+  const bool one = j < a.vpr, two = j2 < a.vpr;
+  const int64_t step = gridDim.x;
+  int64_t row = blockIdx.x;
+  if (row >= a.tokens) return;
+  auto slot = [&](int stage, int k) -> unsigned char* {
+    return bwd_ring + (static_cast<size_t>(stage * 6 + k) * nt + j) * kVecBytes;
+  };
+  auto issue = [&](int64_t r, int stage) {
+    if (r < a.tokens) {
+      const char* gu = a.gate_up + r * a.gu_pitch;
+      const char* go_row = a.grad_out + r * a.go_pitch;
+      if (one) {
+        cp_async16(slot(stage, 0), gu + j * kVecBytes);
+        cp_async16(slot(stage, 1), gu + a.half_bytes + j * kVecBytes);
+        cp_async16(slot(stage, 2), go_row + j * kVecBytes);
+      }
+      if (two) {
+        cp_async16(slot(stage, 3), gu + j2 * kVecBytes);
+        cp_async16(slot(stage, 4), gu + a.half_bytes + j2 * kVecBytes);
+        cp_async16(slot(stage, 5), go_row + j2 * kVecBytes);
+      }
+    }
+    cp_async_commit();  // one group per row, empty past the end: the wait counts stay uniform
+  };
+#pragma unroll
+  for (int d = 0; d < kDepth; ++d) issue(row + d * step, d);
+  float w = load_rw(a.rw, row);
+  int parity = 0, stage = 0, fill = kDepth;
+  for (;;) {
+    const int64_t next = row + step;
+    const bool more = next < a.tokens;
+    issue(row + kDepth * step, fill);
+    const float nw = more ? load_rw(a.rw, next) : 0.0f;
+    cp_async_wait<kDepth>();  // this thread's copies of `row` have landed
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    uint4 g0 = z, u0 = z, o0 = z, g1 = z, u1 = z, o1 = z;
+    if (one) {
+      g0 = lds16(slot(stage, 0));
+      u0 = lds16(slot(stage, 1));
+      o0 = lds16(slot(stage, 2));
+    }
+    if (two) {
+      g1 = lds16(slot(stage, 3));
+      u1 = lds16(slot(stage, 4));
+      o1 = lds16(slot(stage, 5));
+    }
+    char* dgu = a.d_gate_up + row * a.dgu_pitch;
+    const float2 k = bwd_row_consts<HAS_LB>(w, a.c);
+    float2 acc = make_float2(0.0f, 0.0f);
+    uint4 dg, du;
+    if (one) {
+      bwd_vec<S, GATE, HAS_LB>(g0, u0, o0, k, a.c, dg, du, acc);
+      st_stream(dgu + j * kVecBytes, dg);
+      st_stream(dgu + a.half_bytes + j * kVecBytes, du);
+    }
+    if (two) {
+      bwd_vec<S, GATE, HAS_LB>(g1, u1, o1, k, a.c, dg, du, acc);
+      st_stream(dgu + j2 * kVecBytes, dg);
+      st_stream(dgu + a.half_bytes + j2 * kVecBytes, du);
+    }
+    if (a.want_drw) {  // uniform over the launch
+      const float total = block_sum(acc.x + acc.y, red[parity]) * bwd_dw_scale(a.c);
+      parity ^= 1;
+      if (threadIdx.x == 0) {
+        if (a.rw.mode == SITU_RW_SCALAR)
+          a.partials[row] = total;
+        else
+          store_rw_grad(a.d_rw, row * a.d_rw_stride, a.rw.bf16, total);
+      }
+    }
+    if (!more) break;
+    row = next;
+    w = nw;
+    stage = stage + 1 == kStagesRing ? 0 : stage + 1;
+    fill = fill + 1 == kStagesRing ? 0 : fill + 1;
+  }
+  cp_async_wait<0>();
 }
 
 // Broadcast routing weight: sum the per-row partials in a fixed order.
@@ -1808,7 +1951,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
-__device__ __forceinline__ uint4 lds16(const unsigned char* p) { return *reinterpret_cast<const uint4*>(p); }
 __device__ __forceinline__ void consumer_bar(int n) { asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory"); }
 
 struct StreamArgs {
@@ -2658,6 +2800,22 @@ BwdKernel pick_bwd_gate(int gate) {
   }
 }
 
+template <typename S, bool LB>
+BwdKernel pick_bwd_async_gate(int gate) {
+  switch (gate) {
+    case kGateSquare: return situ_glu_bwd_async_kernel<S, kGateSquare, LB>;
+    case kGateEqual: return situ_glu_bwd_async_kernel<S, kGateEqual, LB>;
+    case kGateRoot: return situ_glu_bwd_async_kernel<S, kGateRoot, LB>;
+    default: return situ_glu_bwd_async_kernel<S, kGateGeneric, LB>;
+  }
+}
+
+BwdKernel pick_bwd_async(situ_dtype_t dtype, int gate, bool lb) {
+  if (dtype == SITU_DTYPE_BF16)
+    return lb ? pick_bwd_async_gate<Bf16, true>(gate) : pick_bwd_async_gate<Bf16, false>(gate);
+  return lb ? pick_bwd_async_gate<F32, true>(gate) : pick_bwd_async_gate<F32, false>(gate);
+}
+
 BwdKernel pick_bwd(situ_dtype_t dtype, int gate, bool lb) {
   if (dtype == SITU_DTYPE_BF16) return lb ? pick_bwd_gate<Bf16, true>(gate) : pick_bwd_gate<Bf16, false>(gate);
   return lb ? pick_bwd_gate<F32, true>(gate) : pick_bwd_gate<F32, false>(gate);
@@ -2897,25 +3055,43 @@ situ_status_t bf16_tile_map(CUtensorMap* m, const void* base, int64_t inner, int
 
 using FusedGemmKernel = void (*)(const CUtensorMap, const CUtensorMap, const fc1::Args);
 
-template <class Epi, bool LB>
+// Whether the fused GEMMs run as two-SM clusters (tcgen05 cta_group::2).
+#ifndef SITU_FC_2SM
+#define SITU_FC_2SM 0
+#endif
+constexpr bool kFused2Sm = SITU_FC_2SM != 0;
+
+template <class Epi, bool LB, bool PAIR>
 FusedGemmKernel pick_fused_gate(int gate) {
-  switch (gate) {
-    case kGateSquare: return fc1::situ_fused_gemm_kernel<Epi, kGateSquare, LB>;
-    case kGateEqual: return fc1::situ_fused_gemm_kernel<Epi, kGateEqual, LB>;
-    case kGateRoot: return fc1::situ_fused_gemm_kernel<Epi, kGateRoot, LB>;
-    default: return fc1::situ_fused_gemm_kernel<Epi, kGateGeneric, LB>;
+  if constexpr (PAIR) {
+    switch (gate) {
+      case kGateSquare: return fc1::situ_fused_gemm_2sm_kernel<Epi, kGateSquare, LB>;
+      case kGateEqual: return fc1::situ_fused_gemm_2sm_kernel<Epi, kGateEqual, LB>;
+      case kGateRoot: return fc1::situ_fused_gemm_2sm_kernel<Epi, kGateRoot, LB>;
+      default: return fc1::situ_fused_gemm_2sm_kernel<Epi, kGateGeneric, LB>;
+    }
+  } else {
+    switch (gate) {
+      case kGateSquare: return fc1::situ_fused_gemm_kernel<Epi, kGateSquare, LB>;
+      case kGateEqual: return fc1::situ_fused_gemm_kernel<Epi, kGateEqual, LB>;
+      case kGateRoot: return fc1::situ_fused_gemm_kernel<Epi, kGateRoot, LB>;
+      default: return fc1::situ_fused_gemm_kernel<Epi, kGateGeneric, LB>;
+    }
   }
 }
 
 template <class Epi>
 FusedGemmKernel pick_fused(int gate, bool lb) {
-  return lb ? pick_fused_gate<Epi, true>(gate) : pick_fused_gate<Epi, false>(gate);
+  return lb ? pick_fused_gate<Epi, true, kFused2Sm>(gate) : pick_fused_gate<Epi, false, kFused2Sm>(gate);
 }
 
-// Launch of a fused grouped GEMM: one persistent CTA per SM.
+// Launch of a fused grouped GEMM: one persistent CTA per SM (in two-SM
+// clusters for the pair form: as many clusters as fit at once).
 situ_status_t launch_fused(FusedGemmKernel k, const CUtensorMap& ma, const CUtensorMap& mb, const fc1::Args& a,
                            int64_t experts, cudaStream_t s, const char* what) {
-  const int smem = fc1::kStages * fc1::kStageBytes + 1024 + fc1::kHeaderBytes + static_cast<int>(experts) * (8 + 8 + 4) + 8;
+  const int tables = static_cast<int>(experts) * (8 + 8 + 4) + 8;
+  const int smem = kFused2Sm ? fc1::kStages2 * fc1::kStageBytes2 + 1024 + fc1::kHeaderBytes2 + tables
+                             : fc1::kStages * fc1::kStageBytes + 1024 + fc1::kHeaderBytes + tables;
   cudaError_t err = cudaFuncSetAttribute(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          smem);
   if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(err));
@@ -2925,8 +3101,32 @@ situ_status_t launch_fused(FusedGemmKernel k, const CUtensorMap& ma, const CUten
   int grid = sms;
   const int cap = g_max_ctas.load(std::memory_order_relaxed);
   if (cap > 0 && grid > cap) grid = cap;
-  k<<<grid, fc1::kThreads, smem, s>>>(ma, mb, a);
-  return check_launch(what);
+  if constexpr (kFused2Sm) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(fc1::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(2, 1, 1);
+    int clusters = 0;
+    err = cudaOccupancyMaxActiveClusters(&clusters, reinterpret_cast<const void*>(k), &cfg);
+    if (err != cudaSuccess || clusters <= 0)
+      return fail(SITU_ERR_CUDA, "cluster occupancy query: %s", cudaGetErrorString(err));
+    if (2 * clusters > grid) clusters = grid / 2 > 0 ? grid / 2 : 1;
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    err = cudaLaunchKernelEx(&cfg, k, ma, mb, a);
+    if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(err));
+    return check_launch(what);
+  } else {
+    k<<<grid, fc1::kThreads, smem, s>>>(ma, mb, a);
+    return check_launch(what);
+  }
 }
 
 // Per-row d_w of the fused FC2 data gradient: the row's column-tile partials
@@ -3214,6 +3414,17 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
     sa.vpr = a.vpr;
     sa.c = c;
     st = launch_stream<true>(sa, dtype, gate, has_linear_beta != 0, s);
+  } else if (kBwdDepth > 0 && a.vpr <= 2 * choose_threads(a.vpr)) {
+    BwdKernel k = pick_bwd_async(dtype, gate, has_linear_beta != 0);
+    const int threads = choose_threads(a.vpr);
+    const int smem = (kBwdDepth + 1) * 6 * threads * kVecBytes;
+    st = ensure_smem(reinterpret_cast<const void*>(k), smem);
+    if (st != SITU_OK) return st;
+    int grid = 0;
+    st = launch_grid(reinterpret_cast<const void*>(k), threads, smem, tokens, &grid);
+    if (st != SITU_OK) return st;
+    k<<<grid, threads, smem, s>>>(a);
+    st = check_launch("situ_glu_bwd");
   } else {
     BwdKernel k = pick_bwd(dtype, gate, has_linear_beta != 0);
     const int threads = choose_threads(a.vpr);

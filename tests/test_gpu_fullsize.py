@@ -48,9 +48,12 @@ CHUNK_ELEMS = 1 << 17  # oracle elements per task: a few MB of fp64 per thread
 # is far above that rate and far below what a wrong rounding mode gives (a
 # quarter or more).
 FAITHFUL_ONLY_MAX = 1e-2
-# dG needs the cancellation term only where the two terms of T_g' cancel:
-# there |dG| is a small fraction of the uncancelled magnitude C_G.
-CANCEL_RATIO_MAX = 2.0 ** -6
+# dG needs the cancellation term only where the two terms of T_g' cancel.
+# The kernel's dG error is a few fp32 roundings of the uncancelled magnitude
+# C_G (at most 32 * 2^-24 C_G), so an element can exceed the relative bound
+# rel |dG| only where |dG| / C_G < 32 * 2^-24 / rel: 2^-11 for bf16
+# (rel = 2^-8) and 0.19 for fp32 (rel = 1e-5).
+CANCEL_RATIO_MAX = {"bf16": 32 * 2.0 ** -24 / 2.0 ** -8, "f32": 32 * 2.0 ** -24 / 1e-5}
 # A d_w row needs the 2^-18 S term only where its sum cancels.
 DW_RATIO_MAX = 2.0 ** -4
 
@@ -143,7 +146,7 @@ def test_fullsize_every_element(index, cuda_device):
             assert c["n"] == T * I, (name, c["n"])
             assert c["faithful_only"] <= FAITHFUL_ONLY_MAX * c["n"], (tag, name, c)
         assert counts["Y"]["cancel_only"] == 0 and counts["dU"]["cancel_only"] == 0, (tag, counts)
-        assert counts["dG"]["cancel_ratio_max"] <= CANCEL_RATIO_MAX, (tag, counts["dG"])
+        assert counts["dG"]["cancel_ratio_max"] <= CANCEL_RATIO_MAX[wl.dtype], (tag, counts["dG"])
         assert counts["d_w"]["n"] == T
         assert counts["d_w"]["cancel_ratio_max"] <= DW_RATIO_MAX, (tag, counts["d_w"])
         del y_h, dgu_h, drw_h
