@@ -187,6 +187,7 @@ class ClockSampler:
 
     def __init__(self, device_index: int):
         self.samples, self.reasons, self.max_mhz, self.err = [], set(), None, None
+        self.power_limit_w = None
         self._stop = threading.Event()
         self._thread = None
         try:
@@ -201,6 +202,10 @@ class ClockSampler:
             except Exception:
                 self.handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            try:
+                self.power_limit_w = pynvml.nvmlDeviceGetEnforcedPowerLimit(self.handle) / 1000.0
+            except Exception:
+                self.power_limit_w = None
         except Exception as e:  # NVML unavailable: record why
             self.nvml, self.err = None, f"{type(e).__name__}: {e}"
 
@@ -242,7 +247,8 @@ class ClockSampler:
         names = sorted(v for k, v in self.REASONS.items() if mask & k and v != "gpu_idle")
         return {"sm_mhz": statistics.median(s[0] for s in self.samples), "sm_max_mhz": self.max_mhz,
                 "reasons": names, "samples": len(self.samples),
-                "power_w_max": round(max(s[2] for s in self.samples), 1), "source": "nvml"}
+                "power_w_max": round(max(s[2] for s in self.samples), 1), "power_limit_w": self.power_limit_w,
+                "source": "nvml"}
 
 
 # The fused FC1 workload: the routed-MoE token rows (32768 rows, I = 2048) fed

@@ -336,7 +336,7 @@ struct Fc2Epilogue {
           for (int p = 0; p < 4; ++p) {
             float2 dg, du;
             const float2 go = make_float2(__uint_as_float(dc[8 * v + 2 * p]), __uint_as_float(dc[8 * v + 2 * p + 1]));
-            bwd_pair<GATE, HAS_LB, Bf16>(Bf16::pair(gv, p), Bf16::pair(uv, p), go, kdg, kdu, a.c, dg, du, acc);
+            bwd_pair<GATE, HAS_LB, Bf16, true>(Bf16::pair(gv, p), Bf16::pair(uv, p), go, kdg, kdu, a.c, dg, du, acc);
             Bf16::put(dgv, p, dg);
             Bf16::put(duv, p, du);
           }

@@ -375,13 +375,17 @@ __device__ __forceinline__ float2 fwd_pair_abs(Bits2 gb, Bits2 ub, float2 wbb, c
   return xor_sign2(mul2(num, mul2(rcp2(den), wbb)), s);
 }
 
-// Whether the backward of a pair takes the signed gate form: bf16 outputs at
-// beta = 4 (measured on B200: 5 % less time for the bf16 backward, the same
-// results within the tolerance).  fp32 outputs need the |g| form's accuracy
-// for tiny results; other betas keep it too.
-template <int GATE, typename S>
+// Whether the backward of a pair takes the signed gate form: beta = 4, bf16
+// dG and dU, and a caller whose every output derived from them tolerates the
+// clamp below (CLAMPED): the native-output kernels, whose bf16 gradients
+// carry an absolute tolerance far above the clamped values and whose weight
+// gradients are sums.  Outputs that keep relative accuracy for tiny values --
+// block-scaled codes, whose scale follows the block, and per-element weight
+// gradients -- take the |g| form.  Measured on B200: 5 % less time for the
+// bf16 backward.
+template <int GATE, typename S, bool CLAMPED>
 struct SignedBwd {
-  static constexpr bool value = GATE == kGateSquare && std::is_same<S, Bf16>::value;
+  static constexpr bool value = CLAMPED && GATE == kGateSquare && std::is_same<S, Bf16>::value;
 };
 
 // Backward of a pair.  With A = (1 + E_t)(1 + E_s), B = 1 + E_u (1 without a
@@ -396,11 +400,11 @@ struct SignedBwd {
 // the d_w terms are accumulated without their factor 4 beta_L, which the
 // caller applies once per row.  Returns dG, dU; adds go T_g T_u / (4 beta_L)
 // to acc.
-template <int GATE, bool HAS_LB, typename S>
+template <int GATE, bool HAS_LB, typename S, bool CLAMPED = false>
 __device__ __forceinline__ void bwd_pair(Bits2 gb, Bits2 ub, float2 go, float2 kdg, float2 kdu, const Coeffs& c,
                                          float2& dg, float2& du, float2& acc) {
   float2 A, tgA, ng;
-  if constexpr (SignedBwd<GATE, S>::value) {
+  if constexpr (SignedBwd<GATE, S, CLAMPED>::value) {
     // Signed form (beta = 4, bf16 outputs), as in the bf16 forward: with
     // H = exp(-g/2) and Hs = H^2 = exp(-g) for g of either sign,
     //   T_g  = 4 (1 - H) / A,                 A = (1 + H)(1 + Hs),
@@ -652,7 +656,8 @@ __device__ __forceinline__ void bwd_vec(const uint4& gv, const uint4& uv, const 
 #pragma unroll
   for (int p = 0; p < S::kPairs; ++p) {
     float2 dg, du;
-    bwd_pair<GATE, HAS_LB, S>(S::pair(gv, p), S::pair(uv, p), as_f2(S::pair(gov, p)), kdg, kdu, c, dg, du, acc);
+    bwd_pair<GATE, HAS_LB, S, true>(S::pair(gv, p), S::pair(uv, p), as_f2(S::pair(gov, p)), kdg, kdu, c, dg, du,
+                                    acc);
     S::put(dgv, p, dg);
     S::put(duv, p, du);
   }
@@ -775,120 +780,6 @@ __global__ void SITU_BWD_BOUNDS situ_glu_bwd_kernel(const BwdArgs a) {
       }
     }
   }
-}
-
-// ---- Backward with a shared-memory row ring (cp.async) ----------------------
-// The same per-row work as situ_glu_bwd_kernel's pipelined path, but the rows
-// ahead travel into a shared-memory ring by per-thread asynchronous copies
-// instead of registers: kBwdDepth rows are in flight per CTA without holding
-// a register for them.  Each thread copies and reads back only its own
-// 16-byte slots, so its own cp.async.wait_group is the only synchronisation
-// the data needs.  Stage (i + depth) mod (depth + 1) receives row i + depth
-// while row i is read from stage i mod (depth + 1): the stage refilled was
-// read one iteration earlier, and those values have been consumed since.
-#ifndef SITU_BWD_ASYNC
-#define SITU_BWD_ASYNC 0
-#endif
-constexpr int kBwdDepth = SITU_BWD_ASYNC;  // rows in flight per CTA; 0 selects the register-prefetch kernel
-
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem))),
-               "l"(gmem)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ uint4 lds16(const unsigned char* p) { return *reinterpret_cast<const uint4*>(p); }
-
-template <typename S, int GATE, bool HAS_LB>
-__global__ void __launch_bounds__(kMaxThreads) situ_glu_bwd_async_kernel(const BwdArgs a) {
-  constexpr int kDepth = kBwdDepth > 0 ? kBwdDepth : 1;
-  constexpr int kStagesRing = kDepth + 1;
-  extern __shared__ __align__(16) unsigned char bwd_ring[];  // [stage][6 slots][nt][16 bytes]
-  __shared__ float red[2][kMaxThreads / 32];
-  const int nt = blockDim.x;
-  const int j = threadIdx.x, j2 = j + nt;
-  const bool one = j < a.vpr, two = j2 < a.vpr;
-  const int64_t step = gridDim.x;
-  int64_t row = blockIdx.x;
-  if (row >= a.tokens) return;
-  auto slot = [&](int stage, int k) -> unsigned char* {
-    return bwd_ring + (static_cast<size_t>(stage * 6 + k) * nt + j) * kVecBytes;
-  };
-  auto issue = [&](int64_t r, int stage) {
-    if (r < a.tokens) {
-      const char* gu = a.gate_up + r * a.gu_pitch;
-      const char* go_row = a.grad_out + r * a.go_pitch;
-      if (one) {
-        cp_async16(slot(stage, 0), gu + j * kVecBytes);
-        cp_async16(slot(stage, 1), gu + a.half_bytes + j * kVecBytes);
-        cp_async16(slot(stage, 2), go_row + j * kVecBytes);
-      }
-      if (two) {
-        cp_async16(slot(stage, 3), gu + j2 * kVecBytes);
-        cp_async16(slot(stage, 4), gu + a.half_bytes + j2 * kVecBytes);
-        cp_async16(slot(stage, 5), go_row + j2 * kVecBytes);
-      }
-    }
-    cp_async_commit();  // one group per row, empty past the end: the wait counts stay uniform
-  };
-#pragma unroll
-  for (int d = 0; d < kDepth; ++d) issue(row + d * step, d);
-  float w = load_rw(a.rw, row);
-  int parity = 0, stage = 0, fill = kDepth;
-  for (;;) {
-    const int64_t next = row + step;
-    const bool more = next < a.tokens;
-    issue(row + kDepth * step, fill);
-    const float nw = more ? load_rw(a.rw, next) : 0.0f;
-    cp_async_wait<kDepth>();  // this thread's copies of `row` have landed
-    const uint4 z = make_uint4(0, 0, 0, 0);
-    uint4 g0 = z, u0 = z, o0 = z, g1 = z, u1 = z, o1 = z;
-    if (one) {
-      g0 = lds16(slot(stage, 0));
-      u0 = lds16(slot(stage, 1));
-      o0 = lds16(slot(stage, 2));
-    }
-    if (two) {
-      g1 = lds16(slot(stage, 3));
-      u1 = lds16(slot(stage, 4));
-      o1 = lds16(slot(stage, 5));
-    }
-    char* dgu = a.d_gate_up + row * a.dgu_pitch;
-    const float2 k = bwd_row_consts<HAS_LB>(w, a.c);
-    float2 acc = make_float2(0.0f, 0.0f);
-    uint4 dg, du;
-    if (one) {
-      bwd_vec<S, GATE, HAS_LB>(g0, u0, o0, k, a.c, dg, du, acc);
-      st_stream(dgu + j * kVecBytes, dg);
-      st_stream(dgu + a.half_bytes + j * kVecBytes, du);
-    }
-    if (two) {
-      bwd_vec<S, GATE, HAS_LB>(g1, u1, o1, k, a.c, dg, du, acc);
-      st_stream(dgu + j2 * kVecBytes, dg);
-      st_stream(dgu + a.half_bytes + j2 * kVecBytes, du);
-    }
-    if (a.want_drw) {  // uniform over the launch
-      const float total = block_sum(acc.x + acc.y, red[parity]) * bwd_dw_scale(a.c);
-      parity ^= 1;
-      if (threadIdx.x == 0) {
-        if (a.rw.mode == SITU_RW_SCALAR)
-          a.partials[row] = total;
-        else
-          store_rw_grad(a.d_rw, row * a.d_rw_stride, a.rw.bf16, total);
-      }
-    }
-    if (!more) break;
-    row = next;
-    w = nw;
-    stage = stage + 1 == kStagesRing ? 0 : stage + 1;
-    fill = fill + 1 == kStagesRing ? 0 : fill + 1;
-  }
-  cp_async_wait<0>();
 }
 
 // Broadcast routing weight: sum the per-row partials in a fixed order.
@@ -1951,6 +1842,7 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+__device__ __forceinline__ uint4 lds16(const unsigned char* p) { return *reinterpret_cast<const uint4*>(p); }
 __device__ __forceinline__ void consumer_bar(int n) { asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory"); }
 
 struct StreamArgs {
@@ -2800,22 +2692,6 @@ BwdKernel pick_bwd_gate(int gate) {
   }
 }
 
-template <typename S, bool LB>
-BwdKernel pick_bwd_async_gate(int gate) {
-  switch (gate) {
-    case kGateSquare: return situ_glu_bwd_async_kernel<S, kGateSquare, LB>;
-    case kGateEqual: return situ_glu_bwd_async_kernel<S, kGateEqual, LB>;
-    case kGateRoot: return situ_glu_bwd_async_kernel<S, kGateRoot, LB>;
-    default: return situ_glu_bwd_async_kernel<S, kGateGeneric, LB>;
-  }
-}
-
-BwdKernel pick_bwd_async(situ_dtype_t dtype, int gate, bool lb) {
-  if (dtype == SITU_DTYPE_BF16)
-    return lb ? pick_bwd_async_gate<Bf16, true>(gate) : pick_bwd_async_gate<Bf16, false>(gate);
-  return lb ? pick_bwd_async_gate<F32, true>(gate) : pick_bwd_async_gate<F32, false>(gate);
-}
-
 BwdKernel pick_bwd(situ_dtype_t dtype, int gate, bool lb) {
   if (dtype == SITU_DTYPE_BF16) return lb ? pick_bwd_gate<Bf16, true>(gate) : pick_bwd_gate<Bf16, false>(gate);
   return lb ? pick_bwd_gate<F32, true>(gate) : pick_bwd_gate<F32, false>(gate);
@@ -3414,17 +3290,6 @@ situ_status_t bwd_entry(const void* gate_up, situ_dtype_t dtype, int64_t tokens,
     sa.vpr = a.vpr;
     sa.c = c;
     st = launch_stream<true>(sa, dtype, gate, has_linear_beta != 0, s);
-  } else if (kBwdDepth > 0 && a.vpr <= 2 * choose_threads(a.vpr)) {
-    BwdKernel k = pick_bwd_async(dtype, gate, has_linear_beta != 0);
-    const int threads = choose_threads(a.vpr);
-    const int smem = (kBwdDepth + 1) * 6 * threads * kVecBytes;
-    st = ensure_smem(reinterpret_cast<const void*>(k), smem);
-    if (st != SITU_OK) return st;
-    int grid = 0;
-    st = launch_grid(reinterpret_cast<const void*>(k), threads, smem, tokens, &grid);
-    if (st != SITU_OK) return st;
-    k<<<grid, threads, smem, s>>>(a);
-    st = check_launch("situ_glu_bwd");
   } else {
     BwdKernel k = pick_bwd(dtype, gate, has_linear_beta != 0);
     const int threads = choose_threads(a.vpr);
