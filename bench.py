@@ -767,14 +767,14 @@ def run_ours_fc2(args, wl, beta, dev, world, rank, local, barrier):
         line = {"metric": FC2_METRIC, "value": tflops * world, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
                 "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
-                "kernels": {"fc1::situ_fused_gemm_kernel<Fc2Epilogue>": {"us": ms * 1e3, "TFLOP/s": tflops,
+                "kernels": {"fc1::situ_fused_gemm_2sm_kernel<Fc2Epilogue>": {"us": ms * 1e3, "TFLOP/s": tflops,
                                                                          "frac_of_measured_bf16": tflops / peak}},
                 "unfused": {"ms": unfused_ms, "TFLOP/s": flops / (unfused_ms / 1e3) / 1e12,
                             "what": "cuBLAS bf16 GEMM per expert (torch.matmul) into dY, then situ_glu_bwd"},
-                "roofline": {"bound": "tensor", "kernel": "fc1::situ_fused_gemm_kernel<Fc2Epilogue>", "achieved": tflops,
+                "roofline": {"bound": "tensor", "kernel": "fc1::situ_fused_gemm_2sm_kernel<Fc2Epilogue>", "achieved": tflops,
                              "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
                              "peak_source": f"{peak_src} cuBLAS bf16 (burst)",
-                             "traffic": recorded_traffic("situ_fused_gemm_kernel<Fc2Epilogue>", f"{wl.name}/fc2")},
+                             "traffic": recorded_traffic("situ_fused_gemm_2sm_kernel<Fc2Epilogue>", f"{wl.name}/fc2")},
                 "cpu_baseline": cpu, "e2e": None, "gpu_launches": 2 * K, "clocks": clocks.summary(),
                 "device_status": pkg.abi.situ_glu_device_status(0), "device": torch.cuda.get_device_name(dev)}
         print(json.dumps(line), flush=True)
@@ -898,14 +898,14 @@ def run_ours_fc1(args, wl, beta, dev, world, rank, local, barrier):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": fc1_config(wl, beta, "inputs 940 MB exceed the 126 MB L2; no flush", world),
-            "kernels": {"fc1::situ_fused_gemm_kernel<Fc1Epilogue>": {"us": ms * 1e3, "TFLOP/s": tflops,
+            "kernels": {"fc1::situ_fused_gemm_2sm_kernel<Fc1Epilogue>": {"us": ms * 1e3, "TFLOP/s": tflops,
                                                                      "frac_of_measured_bf16": tflops / peak}},
             "unfused": {"ms": unfused_ms, "TFLOP/s": flops / (unfused_ms / 1e3) / 1e12,
                         "what": "cuBLAS bf16 GEMM per expert (torch.matmul) into gate_up, then situ_glu_fwd"},
-            "roofline": {"bound": "tensor", "kernel": "fc1::situ_fused_gemm_kernel<Fc1Epilogue>", "achieved": tflops,
+            "roofline": {"bound": "tensor", "kernel": "fc1::situ_fused_gemm_2sm_kernel<Fc1Epilogue>", "achieved": tflops,
                          "peak": peak,
                          "unit": "TFLOP/s", "frac": tflops / peak, "peak_source": f"{peak_src} cuBLAS bf16 (burst)",
-                         "traffic": recorded_traffic("situ_fused_gemm_kernel<Fc1Epilogue>", f"{wl.name}/fc1")},
+                         "traffic": recorded_traffic("situ_fused_gemm_2sm_kernel<Fc1Epilogue>", f"{wl.name}/fc1")},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": K,

@@ -37,6 +37,10 @@
 // status word and a CTA-wide abort flag, every role then stops issuing work,
 // the producer waits (bounded) for its own copies, the MMA warp for its own
 // MMAs, and TMEM is freed.
+//
+// The library launches the two-SM form at the end of this file (clusters of
+// two CTAs sharing 256-row tiles through tcgen05 cta_group::2) whenever the
+// device can hold such clusters, and this one-SM kernel otherwise.
 
 namespace fc1 {
 

@@ -2342,6 +2342,197 @@ __global__ void __launch_bounds__(kArStagedThreads, 1) situ_attn_res_staged_kern
   }
 }
 
+// Ring form (the default when half a token row of every source fits three
+// times in shared memory): the token row travels as two halves along the
+// hidden axis, each half of every source in one stage of a three-stage ring,
+// so that while a row is computed the copies of the next row and of the first
+// half of the row after it are in flight -- one and a half rows, against one
+// in the staged form, whose single stage only refills once a row has been
+// read.  Thread j owns column vector j: threads below vpr / 2 read the first
+// half's stage, the others the second's.  The per-source sums are reduced
+// over the warps by one warp per source (a fixed shuffle tree), so that the
+// cross-warp step takes one round trip instead of a serial loop.
+template <typename S>
+__global__ void __launch_bounds__(kArStagedThreads, 1) situ_attn_res_ring_kernel(const ArArgs a) {
+  constexpr int kElems = 2 * S::kPairs;
+  constexpr int kStagesRing = 3;
+  extern __shared__ __align__(16) unsigned char ar_ring[];  // [stage][sources][half row bytes]
+  __shared__ float red[kArStagedThreads / 32][2 * kArStagedSources];
+  __shared__ float logit_sh[kArStagedSources];
+  __shared__ __align__(8) uint64_t bar[kStagesRing];
+  const int j = threadIdx.x, warp = j >> 5, lane = j & 31, nwarps = blockDim.x >> 5;
+  const int half_v = a.vpr / 2;
+  const bool col = j < a.vpr;
+  const int hj = j < half_v ? 0 : 1;
+  const int jj = j - hj * half_v;
+  const uint32_t half_bytes = static_cast<uint32_t>(half_v) * kVecBytes;
+  const uint32_t stage_bytes = half_bytes * static_cast<uint32_t>(a.sources);
+  float2 c[S::kPairs];
+#pragma unroll
+  for (int p = 0; p < S::kPairs; ++p)
+    c[p] = col ? make_float2(ar_weight(a.norm_w, a.norm_bf16, j * kElems + 2 * p) *
+                                 ar_weight(a.proj_w, a.proj_bf16, j * kElems + 2 * p),
+                             ar_weight(a.norm_w, a.norm_bf16, j * kElems + 2 * p + 1) *
+                                 ar_weight(a.proj_w, a.proj_bf16, j * kElems + 2 * p + 1))
+               : make_float2(0.0f, 0.0f);
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < kStagesRing; ++k) mbar_init(&bar[k], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  const int64_t step = gridDim.x;
+  // Copy q of this CTA: half q & 1 of its row q >> 1, into stage q mod 3 (the
+  // (q / 3)-th use of that stage).  Copies are issued in order of q.
+  int last_q = -1;  // the last copy issued (thread 0)
+  auto issue = [&](int q) {
+    const int64_t r = blockIdx.x + static_cast<int64_t>(q >> 1) * step;
+    if (r >= a.tokens) return;
+    const int st = q % kStagesRing;
+    const uint32_t off = static_cast<uint32_t>(q & 1) * half_bytes;
+    mbar_arrive_expect_tx(&bar[st], stage_bytes);
+    for (int b = 0; b < a.sources; ++b)
+      bulk_load(ar_ring + st * stage_bytes + b * half_bytes, ar_source<S>(a, r, b) + off, half_bytes, &bar[st]);
+    last_q = q;
+  };
+  if (threadIdx.x == 0)
+    for (int q = 0; q < kStagesRing; ++q) issue(q);
+  bool aborted = false;
+  int64_t row = blockIdx.x;
+  for (int i = 0; row < a.tokens; ++i, row += step) {
+    // this thread's half: copy 2 i + hj, the (2 i + hj) / 3 -th use of its stage
+    const int q = 2 * i + hj;
+    const int st = q % kStagesRing;
+    const bool ok = !col || mbar_wait(&bar[st], static_cast<uint32_t>(q / kStagesRing) & 1u);
+    if (__syncthreads_or(!ok)) {
+      if (threadIdx.x == 0) atomicExch(&g_device_status, kStatusWaitExpired);
+      aborted = true;
+      break;
+    }
+    uint4 x[kArStagedSources];
+#pragma unroll
+    for (int b = 0; b < kArStagedSources; ++b)
+      x[b] = (col && b < a.sources) ? lds16(ar_ring + st * stage_bytes + b * half_bytes + jj * kVecBytes)
+                                    : make_uint4(0, 0, 0, 0);
+    __syncthreads();  // both of this row's stages are free
+    if (threadIdx.x == 0) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // our reads before the copies' writes
+      issue(2 * i + 3);
+      issue(2 * i + 4);
+    }
+    auto sums = [&](int b, float& ss, float& dd) {
+      float2 ss2 = make_float2(0.0f, 0.0f), dd2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int p = 0; p < S::kPairs; ++p) {
+        const float2 xv = as_f2(S::pair(x[b], p));
+        ss2 = fma2(xv, xv, ss2);
+        dd2 = fma2(xv, c[p], dd2);
+      }
+      ss = ss2.x + ss2.y;
+      dd = dd2.x + dd2.y;
+    };
+    {
+      float v[16];
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        v[2 * b] = 0.0f;
+        v[2 * b + 1] = 0.0f;
+        if (b < a.sources) sums(b, v[2 * b], v[2 * b + 1]);
+      }
+#pragma unroll
+      for (int o = 16, n = 8; n > 0; o >>= 1, n >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int k = 0; k < n; ++k) {
+          const float send = upper ? v[k] : v[n + k];
+          const float keep = upper ? v[n + k] : v[k];
+          v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+      const int slot = lane >> 1;
+      if ((lane & 1) == 0 && slot < 2 * a.sources && slot < 16) red[warp][slot] = v[0];
+    }
+    if (a.sources > 8) {  // uniform
+      float ss = 0.0f, dd = 0.0f;
+      sums(8, ss, dd);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        dd += __shfl_xor_sync(0xffffffffu, dd, o);
+      }
+      if (lane == 0) {
+        red[warp][16] = ss;
+        red[warp][17] = dd;
+      }
+    }
+    __syncthreads();
+    if (warp < a.sources) {  // warp b: source b's two sums over the warps, one shuffle tree each
+      float s2 = lane < nwarps ? red[lane][2 * warp] : 0.0f;
+      float d2 = lane < nwarps ? red[lane][2 * warp + 1] : 0.0f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+        d2 += __shfl_xor_sync(0xffffffffu, d2, o);
+      }
+      if (lane == 0) logit_sh[warp] = d2 * rsqrtf(s2 * a.inv_hidden + a.eps);
+    }
+    __syncthreads();
+    float p[kArStagedSources];
+    float mx = logit_sh[0];
+#pragma unroll
+    for (int b = 1; b < kArStagedSources; ++b)
+      if (b < a.sources) mx = fmaxf(mx, logit_sh[b]);
+    float z = 0.0f;
+#pragma unroll
+    for (int b = 0; b < kArStagedSources; ++b) {
+      p[b] = b < a.sources ? __expf(logit_sh[b] - mx) : 0.0f;
+      z += p[b];
+    }
+    const float rz = 1.0f / z;
+    if (col) {
+      float2 acc[S::kPairs];
+#pragma unroll
+      for (int q2 = 0; q2 < S::kPairs; ++q2) acc[q2] = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int b = 0; b < kArStagedSources; ++b) {
+        if (b < a.sources) {
+#pragma unroll
+          for (int q2 = 0; q2 < S::kPairs; ++q2) acc[q2] = fma2(splat(p[b] * rz), as_f2(S::pair(x[b], q2)), acc[q2]);
+        }
+      }
+      char* orow = a.out + row * a.out_pitch;
+      if (a.out_bf16) {
+        uint32_t w[S::kPairs];
+#pragma unroll
+        for (int q2 = 0; q2 < S::kPairs; ++q2) w[q2] = Bf16::pack(acc[q2]);
+        if constexpr (S::kPairs == 4)
+          st_stream(orow + j * 16, make_uint4(w[0], w[1], w[2], w[3]));
+        else
+          st_stream8(orow + j * 8, make_uint2(w[0], w[1]));
+      } else {
+#pragma unroll
+        for (int q2 = 0; q2 < S::kPairs / 2; ++q2)
+          st_stream(orow + j * kElems * 4 + q2 * 16,
+                    make_uint4(__float_as_uint(acc[2 * q2].x), __float_as_uint(acc[2 * q2].y),
+                               __float_as_uint(acc[2 * q2 + 1].x), __float_as_uint(acc[2 * q2 + 1].y)));
+      }
+    }
+    // logit_sh and red are rewritten by the next row only after its first
+    // barrier, which every thread reaches after finishing this row.
+  }
+  // After an expired wait, let every copy this CTA issued land (bounded)
+  // before its shared memory is released: the latest copy q into each stage
+  // completes that stage's phase q / 3.
+  if (aborted && threadIdx.x == 0) {
+    for (int q = last_q; q >= 0 && q > last_q - kStagesRing; --q) {
+      const unsigned long long t0 = global_timer_ns();
+      while (!mbar_try_wait(&bar[q % kStagesRing], static_cast<uint32_t>(q / kStagesRing) & 1u) &&
+             global_timer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+  }
+}
+
 #include "situ_fused_gemm.cuh"
 
 // ---------------------------------------------------------------------------
@@ -2931,12 +3122,6 @@ situ_status_t bf16_tile_map(CUtensorMap* m, const void* base, int64_t inner, int
 
 using FusedGemmKernel = void (*)(const CUtensorMap, const CUtensorMap, const fc1::Args);
 
-// Whether the fused GEMMs run as two-SM clusters (tcgen05 cta_group::2).
-#ifndef SITU_FC_2SM
-#define SITU_FC_2SM 0
-#endif
-constexpr bool kFused2Sm = SITU_FC_2SM != 0;
-
 template <class Epi, bool LB, bool PAIR>
 FusedGemmKernel pick_fused_gate(int gate) {
   if constexpr (PAIR) {
@@ -2956,53 +3141,68 @@ FusedGemmKernel pick_fused_gate(int gate) {
   }
 }
 
+// The one-SM and two-SM kernels of a fused GEMM.
+struct FusedKernels {
+  FusedGemmKernel one, pair;
+};
+
 template <class Epi>
-FusedGemmKernel pick_fused(int gate, bool lb) {
-  return lb ? pick_fused_gate<Epi, true, kFused2Sm>(gate) : pick_fused_gate<Epi, false, kFused2Sm>(gate);
+FusedKernels pick_fused(int gate, bool lb) {
+  if (lb) return {pick_fused_gate<Epi, true, false>(gate), pick_fused_gate<Epi, true, true>(gate)};
+  return {pick_fused_gate<Epi, false, false>(gate), pick_fused_gate<Epi, false, true>(gate)};
 }
 
-// Launch of a fused grouped GEMM: one persistent CTA per SM (in two-SM
-// clusters for the pair form: as many clusters as fit at once).
-situ_status_t launch_fused(FusedGemmKernel k, const CUtensorMap& ma, const CUtensorMap& mb, const fc1::Args& a,
-                           int64_t experts, cudaStream_t s, const char* what) {
+// Launch of a fused grouped GEMM, persistent over the output tiles.  The
+// two-SM form (clusters of two CTAs, tcgen05 cta_group::2) runs whenever the
+// device can keep at least one such cluster resident, as many clusters as fit
+// at once; it measured 1.5 % (FC1) and 4 % (FC2) faster than the one-SM form
+// on B200.  Otherwise one CTA per SM runs the one-SM kernel.
+situ_status_t launch_fused(const FusedKernels& ks, const CUtensorMap& ma, const CUtensorMap& mb,
+                           const fc1::Args& a, int64_t experts, cudaStream_t s, const char* what) {
   const int tables = static_cast<int>(experts) * (8 + 8 + 4) + 8;
-  const int smem = kFused2Sm ? fc1::kStages2 * fc1::kStageBytes2 + 1024 + fc1::kHeaderBytes2 + tables
-                             : fc1::kStages * fc1::kStageBytes + 1024 + fc1::kHeaderBytes + tables;
-  cudaError_t err = cudaFuncSetAttribute(reinterpret_cast<const void*>(k), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem);
-  if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(err));
   int sms = 0;
   situ_status_t st = device_sm_count(&sms);
   if (st != SITU_OK) return st;
   int grid = sms;
   const int cap = g_max_ctas.load(std::memory_order_relaxed);
   if (cap > 0 && grid > cap) grid = cap;
-  if constexpr (kFused2Sm) {
+  if (grid >= 2) {
+    const int smem = fc1::kStages2 * fc1::kStageBytes2 + 1024 + fc1::kHeaderBytes2 + tables;
+    cudaError_t err = cudaFuncSetAttribute(reinterpret_cast<const void*>(ks.pair),
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(err));
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(fc1::kThreads, 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cfg.gridDim = dim3(2, 1, 1);
     int clusters = 0;
-    err = cudaOccupancyMaxActiveClusters(&clusters, reinterpret_cast<const void*>(k), &cfg);
-    if (err != cudaSuccess || clusters <= 0)
-      return fail(SITU_ERR_CUDA, "cluster occupancy query: %s", cudaGetErrorString(err));
-    if (2 * clusters > grid) clusters = grid / 2 > 0 ? grid / 2 : 1;
-    cfg.gridDim = dim3(2 * clusters, 1, 1);
-    err = cudaLaunchKernelEx(&cfg, k, ma, mb, a);
-    if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(err));
-    return check_launch(what);
-  } else {
-    k<<<grid, fc1::kThreads, smem, s>>>(ma, mb, a);
-    return check_launch(what);
+    err = cudaOccupancyMaxActiveClusters(&clusters, reinterpret_cast<const void*>(ks.pair), &cfg);
+    if (err != cudaSuccess) {
+      (void)cudaGetLastError();  // the query's error is not sticky: fall back to the one-SM form
+      clusters = 0;
+    }
+    if (clusters > 0) {
+      if (2 * clusters > grid) clusters = grid / 2;
+      cfg.gridDim = dim3(2 * clusters, 1, 1);
+      err = cudaLaunchKernelEx(&cfg, ks.pair, ma, mb, a);
+      if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(err));
+      return check_launch(what);
+    }
   }
+  const int smem = fc1::kStages * fc1::kStageBytes + 1024 + fc1::kHeaderBytes + tables;
+  cudaError_t err = cudaFuncSetAttribute(reinterpret_cast<const void*>(ks.one),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return fail(SITU_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(err));
+  ks.one<<<grid, fc1::kThreads, smem, s>>>(ma, mb, a);
+  return check_launch(what);
 }
 
 // Per-row d_w of the fused FC2 data gradient: the row's column-tile partials
@@ -3740,6 +3940,28 @@ extern "C" situ_status_t situ_attn_res_fwd(const void* blocks, int64_t nblocks, 
   a.out_bf16 = out_dtype == SITU_DTYPE_BF16;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t stage_bytes = sources * hidden * es;
+#ifndef SITU_AR_RING
+#define SITU_AR_RING 1
+#endif
+  if (SITU_AR_RING && a.vpr % 2 == 0 && a.vpr <= kArStagedThreads && sources <= kArStagedSources &&
+      3 * (stage_bytes / 2) <= 200 * 1024) {
+    const void* ks = dtype == SITU_DTYPE_BF16 ? reinterpret_cast<const void*>(situ_attn_res_ring_kernel<Bf16>)
+                                              : reinterpret_cast<const void*>(situ_attn_res_ring_kernel<F32>);
+    const int threads = (a.vpr + 31) / 32 * 32;
+    const int smem = static_cast<int>(3 * (stage_bytes / 2));
+    if (smem > 48 * 1024) {
+      situ_status_t st = ensure_smem(ks, smem);
+      if (st != SITU_OK) return st;
+    }
+    int grid = 0;
+    situ_status_t st = launch_grid(ks, threads, smem, tokens, &grid);
+    if (st != SITU_OK) return st;
+    if (dtype == SITU_DTYPE_BF16)
+      situ_attn_res_ring_kernel<Bf16><<<grid, threads, smem, s>>>(a);
+    else
+      situ_attn_res_ring_kernel<F32><<<grid, threads, smem, s>>>(a);
+    return check_launch("situ_attn_res_fwd");
+  }
   if (a.vpr <= kArStagedThreads && sources <= kArStagedSources && stage_bytes <= 180 * 1024) {
     const void* ks = dtype == SITU_DTYPE_BF16 ? reinterpret_cast<const void*>(situ_attn_res_staged_kernel<Bf16>)
                                               : reinterpret_cast<const void*>(situ_attn_res_staged_kernel<F32>);
