@@ -400,7 +400,19 @@ struct SignedBwd {
 // the d_w terms are accumulated without their factor 4 beta_L, which the
 // caller applies once per row.  Returns dG, dU; adds go T_g T_u / (4 beta_L)
 // to acc.
-template <int GATE, bool HAS_LB, typename S, bool CLAMPED = false>
+// The signed backward's clamp applied to packed bf16 gate values: g >= -27.75
+// (a bf16 number; y = g kt >= -20.02 for beta = 4), NaN kept, one
+// instruction per pair of elements.
+__device__ __forceinline__ uint4 clamp_gate_bf16x8(uint4 v) {
+  const uint32_t lo = 0xC1DEC1DEu;  // -27.75 in both halves
+  asm("max.NaN.bf16x2 %0, %0, %4;\n\tmax.NaN.bf16x2 %1, %1, %4;\n\t"
+      "max.NaN.bf16x2 %2, %2, %4;\n\tmax.NaN.bf16x2 %3, %3, %4;"
+      : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w)
+      : "r"(lo));
+  return v;
+}
+
+template <int GATE, bool HAS_LB, typename S, bool CLAMPED = false, bool PRECLAMPED = false>
 __device__ __forceinline__ void bwd_pair(Bits2 gb, Bits2 ub, float2 go, float2 kdg, float2 kdu, const Coeffs& c,
                                          float2& dg, float2& du, float2& acc) {
   float2 A, tgA, ng;
@@ -412,11 +424,15 @@ __device__ __forceinline__ void bwd_pair(Bits2 gb, Bits2 ub, float2 go, float2 k
     // so no |g|, sign flip or select is needed.  The exponent argument is
     // clamped at 20 (g >= -27.7: H <= 2^20, A <= 2^60, (A B)^2 <= 2^122), where
     // |T_g| < 4e-12 and |T_g'| < 1e-11: far below a bf16 output's absolute
-    // resolution of the tolerance.
+    // resolution of the tolerance.  PRECLAMPED: the caller clamped the packed
+    // bf16 gate values at -27.75 instead (y >= -20.02, (A B)^2 <= 2^122.1).
     float2 y = mul2(as_f2(gb), splat(c.kt));
-    y = make_float2(max_nan(y.x, -20.0f), max_nan(y.y, -20.0f));
+    if constexpr (!PRECLAMPED) y = make_float2(max_nan(y.x, -20.0f), max_nan(y.y, -20.0f));
     const float2 H = ex2_neg2(y), Hs = mul2(H, H);
-    const float2 em = one_minus_exp2_neg<S>(y, H);  // 1 - H
+    // 1 - H: below |x| = 1/32 from the series to x^3 (truncation under
+    // 2^-19.6), above it 1 - H (MUFU error under 2^-17 relative there): both
+    // far below what a bf16 output and a per-row sum of terms need.
+    const float2 em = one_minus_exp2_neg<S, SeriesBf16Up>(y, H);
     const float2 opH = add2(splat(1.0f), H), opHs = add2(splat(1.0f), Hs);
     A = mul2(opH, opHs);
     tgA = mul2(em, A);                                // T_g A^2 / 4
@@ -653,11 +669,13 @@ template <typename S, int GATE, bool HAS_LB>
 __device__ __forceinline__ void bwd_vec(const uint4& gv, const uint4& uv, const uint4& gov, float2 k,
                                         const Coeffs& c, uint4& dgv, uint4& duv, float2& acc) {
   const float2 kdg = splat(k.x), kdu = splat(k.y);
+  constexpr bool kPre = SignedBwd<GATE, S, true>::value;  // clamp the packed gate values, one instruction a pair
+  const uint4 gc = kPre ? clamp_gate_bf16x8(gv) : gv;
 #pragma unroll
   for (int p = 0; p < S::kPairs; ++p) {
     float2 dg, du;
-    bwd_pair<GATE, HAS_LB, S, true>(S::pair(gv, p), S::pair(uv, p), as_f2(S::pair(gov, p)), kdg, kdu, c, dg, du,
-                                    acc);
+    bwd_pair<GATE, HAS_LB, S, true, kPre>(S::pair(gc, p), S::pair(uv, p), as_f2(S::pair(gov, p)), kdg, kdu, c, dg,
+                                          du, acc);
     S::put(dgv, p, dg);
     S::put(duv, p, du);
   }
@@ -2342,196 +2360,6 @@ __global__ void __launch_bounds__(kArStagedThreads, 1) situ_attn_res_staged_kern
   }
 }
 
-// Ring form (the default when half a token row of every source fits three
-// times in shared memory): the token row travels as two halves along the
-// hidden axis, each half of every source in one stage of a three-stage ring,
-// so that while a row is computed the copies of the next row and of the first
-// half of the row after it are in flight -- one and a half rows, against one
-// in the staged form, whose single stage only refills once a row has been
-// read.  Thread j owns column vector j: threads below vpr / 2 read the first
-// half's stage, the others the second's.  The per-source sums are reduced
-// over the warps by one warp per source (a fixed shuffle tree), so that the
-// cross-warp step takes one round trip instead of a serial loop.
-template <typename S>
-__global__ void __launch_bounds__(kArStagedThreads, 1) situ_attn_res_ring_kernel(const ArArgs a) {
-  constexpr int kElems = 2 * S::kPairs;
-  constexpr int kStagesRing = 3;
-  extern __shared__ __align__(16) unsigned char ar_ring[];  // [stage][sources][half row bytes]
-  __shared__ float red[kArStagedThreads / 32][2 * kArStagedSources];
-  __shared__ float logit_sh[kArStagedSources];
-  __shared__ __align__(8) uint64_t bar[kStagesRing];
-  const int j = threadIdx.x, warp = j >> 5, lane = j & 31, nwarps = blockDim.x >> 5;
-  const int half_v = a.vpr / 2;
-  const bool col = j < a.vpr;
-  const int hj = j < half_v ? 0 : 1;
-  const int jj = j - hj * half_v;
-  const uint32_t half_bytes = static_cast<uint32_t>(half_v) * kVecBytes;
-  const uint32_t stage_bytes = half_bytes * static_cast<uint32_t>(a.sources);
-  float2 c[S::kPairs];
-#pragma unroll
-  for (int p = 0; p < S::kPairs; ++p)
-    c[p] = col ? make_float2(ar_weight(a.norm_w, a.norm_bf16, j * kElems + 2 * p) *
-                                 ar_weight(a.proj_w, a.proj_bf16, j * kElems + 2 * p),
-                             ar_weight(a.norm_w, a.norm_bf16, j * kElems + 2 * p + 1) *
-                                 ar_weight(a.proj_w, a.proj_bf16, j * kElems + 2 * p + 1))
-               : make_float2(0.0f, 0.0f);
-  if (threadIdx.x == 0) {
-    for (int k = 0; k < kStagesRing; ++k) mbar_init(&bar[k], 1);
-    mbar_fence_init();
-  }
-  __syncthreads();
-  const int64_t step = gridDim.x;
-  // Copy q of this CTA: half q & 1 of its row q >> 1, into stage q mod 3 (the
-  // (q / 3)-th use of that stage).  Copies are issued in order of q.
-  int last_q = -1;  // the last copy issued (thread 0)
-  auto issue = [&](int q) {
-    const int64_t r = blockIdx.x + static_cast<int64_t>(q >> 1) * step;
-    if (r >= a.tokens) return;
-    const int st = q % kStagesRing;
-    const uint32_t off = static_cast<uint32_t>(q & 1) * half_bytes;
-    mbar_arrive_expect_tx(&bar[st], stage_bytes);
-    for (int b = 0; b < a.sources; ++b)
-      bulk_load(ar_ring + st * stage_bytes + b * half_bytes, ar_source<S>(a, r, b) + off, half_bytes, &bar[st]);
-    last_q = q;
-  };
-  if (threadIdx.x == 0)
-    for (int q = 0; q < kStagesRing; ++q) issue(q);
-  bool aborted = false;
-  int64_t row = blockIdx.x;
-  for (int i = 0; row < a.tokens; ++i, row += step) {
-    // this thread's half: copy 2 i + hj, the (2 i + hj) / 3 -th use of its stage
-    const int q = 2 * i + hj;
-    const int st = q % kStagesRing;
-    const bool ok = !col || mbar_wait(&bar[st], static_cast<uint32_t>(q / kStagesRing) & 1u);
-    if (__syncthreads_or(!ok)) {
-      if (threadIdx.x == 0) atomicExch(&g_device_status, kStatusWaitExpired);
-      aborted = true;
-      break;
-    }
-    uint4 x[kArStagedSources];
-#pragma unroll
-    for (int b = 0; b < kArStagedSources; ++b)
-      x[b] = (col && b < a.sources) ? lds16(ar_ring + st * stage_bytes + b * half_bytes + jj * kVecBytes)
-                                    : make_uint4(0, 0, 0, 0);
-    __syncthreads();  // both of this row's stages are free
-    if (threadIdx.x == 0) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // our reads before the copies' writes
-      issue(2 * i + 3);
-      issue(2 * i + 4);
-    }
-    auto sums = [&](int b, float& ss, float& dd) {
-      float2 ss2 = make_float2(0.0f, 0.0f), dd2 = make_float2(0.0f, 0.0f);
-#pragma unroll
-      for (int p = 0; p < S::kPairs; ++p) {
-        const float2 xv = as_f2(S::pair(x[b], p));
-        ss2 = fma2(xv, xv, ss2);
-        dd2 = fma2(xv, c[p], dd2);
-      }
-      ss = ss2.x + ss2.y;
-      dd = dd2.x + dd2.y;
-    };
-    {
-      float v[16];
-#pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        v[2 * b] = 0.0f;
-        v[2 * b + 1] = 0.0f;
-        if (b < a.sources) sums(b, v[2 * b], v[2 * b + 1]);
-      }
-#pragma unroll
-      for (int o = 16, n = 8; n > 0; o >>= 1, n >>= 1) {
-        const bool upper = (lane & o) != 0;
-#pragma unroll
-        for (int k = 0; k < n; ++k) {
-          const float send = upper ? v[k] : v[n + k];
-          const float keep = upper ? v[n + k] : v[k];
-          v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-      }
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
-      const int slot = lane >> 1;
-      if ((lane & 1) == 0 && slot < 2 * a.sources && slot < 16) red[warp][slot] = v[0];
-    }
-    if (a.sources > 8) {  // uniform
-      float ss = 0.0f, dd = 0.0f;
-      sums(8, ss, dd);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        dd += __shfl_xor_sync(0xffffffffu, dd, o);
-      }
-      if (lane == 0) {
-        red[warp][16] = ss;
-        red[warp][17] = dd;
-      }
-    }
-    __syncthreads();
-    if (warp < a.sources) {  // warp b: source b's two sums over the warps, one shuffle tree each
-      float s2 = lane < nwarps ? red[lane][2 * warp] : 0.0f;
-      float d2 = lane < nwarps ? red[lane][2 * warp + 1] : 0.0f;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-        d2 += __shfl_xor_sync(0xffffffffu, d2, o);
-      }
-      if (lane == 0) logit_sh[warp] = d2 * rsqrtf(s2 * a.inv_hidden + a.eps);
-    }
-    __syncthreads();
-    float p[kArStagedSources];
-    float mx = logit_sh[0];
-#pragma unroll
-    for (int b = 1; b < kArStagedSources; ++b)
-      if (b < a.sources) mx = fmaxf(mx, logit_sh[b]);
-    float z = 0.0f;
-#pragma unroll
-    for (int b = 0; b < kArStagedSources; ++b) {
-      p[b] = b < a.sources ? __expf(logit_sh[b] - mx) : 0.0f;
-      z += p[b];
-    }
-    const float rz = 1.0f / z;
-    if (col) {
-      float2 acc[S::kPairs];
-#pragma unroll
-      for (int q2 = 0; q2 < S::kPairs; ++q2) acc[q2] = make_float2(0.0f, 0.0f);
-#pragma unroll
-      for (int b = 0; b < kArStagedSources; ++b) {
-        if (b < a.sources) {
-#pragma unroll
-          for (int q2 = 0; q2 < S::kPairs; ++q2) acc[q2] = fma2(splat(p[b] * rz), as_f2(S::pair(x[b], q2)), acc[q2]);
-        }
-      }
-      char* orow = a.out + row * a.out_pitch;
-      if (a.out_bf16) {
-        uint32_t w[S::kPairs];
-#pragma unroll
-        for (int q2 = 0; q2 < S::kPairs; ++q2) w[q2] = Bf16::pack(acc[q2]);
-        if constexpr (S::kPairs == 4)
-          st_stream(orow + j * 16, make_uint4(w[0], w[1], w[2], w[3]));
-        else
-          st_stream8(orow + j * 8, make_uint2(w[0], w[1]));
-      } else {
-#pragma unroll
-        for (int q2 = 0; q2 < S::kPairs / 2; ++q2)
-          st_stream(orow + j * kElems * 4 + q2 * 16,
-                    make_uint4(__float_as_uint(acc[2 * q2].x), __float_as_uint(acc[2 * q2].y),
-                               __float_as_uint(acc[2 * q2 + 1].x), __float_as_uint(acc[2 * q2 + 1].y)));
-      }
-    }
-    // logit_sh and red are rewritten by the next row only after its first
-    // barrier, which every thread reaches after finishing this row.
-  }
-  // After an expired wait, let every copy this CTA issued land (bounded)
-  // before its shared memory is released: the latest copy q into each stage
-  // completes that stage's phase q / 3.
-  if (aborted && threadIdx.x == 0) {
-    for (int q = last_q; q >= 0 && q > last_q - kStagesRing; --q) {
-      const unsigned long long t0 = global_timer_ns();
-      while (!mbar_try_wait(&bar[q % kStagesRing], static_cast<uint32_t>(q / kStagesRing) & 1u) &&
-             global_timer_ns() - t0 < kWaitLimitNs) {
-      }
-    }
-  }
-}
 
 #include "situ_fused_gemm.cuh"
 
@@ -3940,28 +3768,6 @@ extern "C" situ_status_t situ_attn_res_fwd(const void* blocks, int64_t nblocks, 
   a.out_bf16 = out_dtype == SITU_DTYPE_BF16;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t stage_bytes = sources * hidden * es;
-#ifndef SITU_AR_RING
-#define SITU_AR_RING 1
-#endif
-  if (SITU_AR_RING && a.vpr % 2 == 0 && a.vpr <= kArStagedThreads && sources <= kArStagedSources &&
-      3 * (stage_bytes / 2) <= 200 * 1024) {
-    const void* ks = dtype == SITU_DTYPE_BF16 ? reinterpret_cast<const void*>(situ_attn_res_ring_kernel<Bf16>)
-                                              : reinterpret_cast<const void*>(situ_attn_res_ring_kernel<F32>);
-    const int threads = (a.vpr + 31) / 32 * 32;
-    const int smem = static_cast<int>(3 * (stage_bytes / 2));
-    if (smem > 48 * 1024) {
-      situ_status_t st = ensure_smem(ks, smem);
-      if (st != SITU_OK) return st;
-    }
-    int grid = 0;
-    situ_status_t st = launch_grid(ks, threads, smem, tokens, &grid);
-    if (st != SITU_OK) return st;
-    if (dtype == SITU_DTYPE_BF16)
-      situ_attn_res_ring_kernel<Bf16><<<grid, threads, smem, s>>>(a);
-    else
-      situ_attn_res_ring_kernel<F32><<<grid, threads, smem, s>>>(a);
-    return check_launch("situ_attn_res_fwd");
-  }
   if (a.vpr <= kArStagedThreads && sources <= kArStagedSources && stage_bytes <= 180 * 1024) {
     const void* ks = dtype == SITU_DTYPE_BF16 ? reinterpret_cast<const void*>(situ_attn_res_staged_kernel<Bf16>)
                                               : reinterpret_cast<const void*>(situ_attn_res_staged_kernel<F32>);
