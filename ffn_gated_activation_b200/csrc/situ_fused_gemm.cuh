@@ -534,7 +534,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 // whose completion bytes both count on CTA 0's stage barrier (the loads'
 // cta_group::2 form), and CTA 0's MMA commits arrive on both CTAs' barriers.
 constexpr int kBM2 = 2 * kBM;                      // token rows per cluster tile
-constexpr int kStages2 = 6;
+#ifndef SITU_FC2SM_STAGES
+#define SITU_FC2SM_STAGES 6
+#endif
+constexpr int kStages2 = SITU_FC2SM_STAGES;
 constexpr int kStageBytes2 = kABytes + kBHalfBytes;  // 32 KiB per CTA
 // Header after the ring: 17 mbarriers, the TMEM base and the abort flag; then
 // the per-expert tables.
