@@ -65,7 +65,7 @@ def test_attn_res_bf16(T, B, H, cuda_device):
     run_ar(cuda_device, T, B, H, seed=T + B)
 
 
-@pytest.mark.parametrize("T,B,H", [(33, 4, 256), (70, 8, 4096)])
+@pytest.mark.parametrize("T,B,H", [(33, 4, 256), (70, 8, 4096), (40, 8, 2048)])
 def test_attn_res_fp32_values_and_output(T, B, H, cuda_device):
     run_ar(cuda_device, T, B, H, dtype="f32", out_dtype=torch.float32, seed=7)
 
