@@ -1554,11 +1554,39 @@ __device__ __forceinline__ void fwd_pairs(const uint4& gv, const uint4& uv, floa
   }
 }
 
+// Whether any of 8 packed bf16 gate values lies below -27.75, the signed
+// backward's clamp (NaN pairs count as below: they take the |g| form).
+__device__ __forceinline__ bool gate_below_clamp_bf16x8(const uint4& v) {
+  uint32_t m, cl;
+  asm("{\n\t.reg .b32 t0, t1;\n\t"
+      "min.bf16x2 t0, %2, %3;\n\t"
+      "min.bf16x2 t1, %4, %5;\n\t"
+      "min.bf16x2 %0, t0, t1;\n\t"
+      "max.bf16x2 %1, %0, %6;\n\t}"
+      : "=r"(m), "=r"(cl)
+      : "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(0xC1DEC1DEu));
+  return cl != m;
+}
+
+// dG and dU of one vector for the block-scaled outputs.  Their codes keep
+// relative accuracy for tiny values, so the clamped signed form is out; but
+// where no gate value of the warp's vectors lies below the clamp (`extreme`
+// false, the caller's vote) the clamp changes nothing and the signed form
+// runs without it.  Otherwise the |g| form, exact for every g.
 template <typename S, int GATE, bool HAS_LB>
 __device__ __forceinline__ void bwd_pairs(const uint4& gv, const uint4& uv, const uint4& gov, float2 k,
                                           const Coeffs& c, float2 (&dg)[S::kPairs], float2 (&du)[S::kPairs],
-                                          float2& acc) {
+                                          float2& acc, bool extreme) {
   const float2 kdg = splat(k.x), kdu = splat(k.y);
+  if constexpr (SignedBwd<GATE, S, true>::value) {
+    if (!extreme) {
+#pragma unroll
+      for (int p = 0; p < S::kPairs; ++p)
+        bwd_pair<GATE, HAS_LB, S, true, true>(S::pair(gv, p), S::pair(uv, p), as_f2(S::pair(gov, p)), kdg, kdu, c,
+                                              dg[p], du[p], acc);
+      return;
+    }
+  }
 #pragma unroll
   for (int p = 0; p < S::kPairs; ++p)
     bwd_pair<GATE, HAS_LB, S>(S::pair(gv, p), S::pair(uv, p), as_f2(S::pair(gov, p)), kdg, kdu, c, dg[p], du[p], acc);
@@ -1679,8 +1707,10 @@ __device__ __forceinline__ void bwd_quant_vec(const uint4& g, const uint4& u, co
                                               int inter, typename Q::State& st, float2& acc) {
   constexpr int kP = S::kPairs;
   float2 dg[kP], du[kP];
+  // Every lane of the warp is here (inactive lanes hold zero vectors).
+  const bool extreme = !SignedBwd<GATE, S, true>::value || __any_sync(0xffffffffu, gate_below_clamp_bf16x8(g));
   if (ALL || act) {
-    bwd_pairs<S, GATE, HAS_LB>(g, u, o, k, c, dg, du, acc);
+    bwd_pairs<S, GATE, HAS_LB>(g, u, o, k, c, dg, du, acc, extreme);
   } else {
     zero_y<S>(dg);
     zero_y<S>(du);
