@@ -28,8 +28,13 @@ def ew_inputs(dtype: str, T: int, I: int, seed: int):
     return (x["gate_up"], x["grad_out"], workloads.column_weights(wl), workloads.element_weights(wl))
 
 
-def run_ew(dev, dtype, T, I, beta, lb, full, rw_dtype, seed, rw_pad=0, d_rw_pad=0, want_drw=True):
+def run_ew(dev, dtype, T, I, beta, lb, full, rw_dtype, seed, rw_pad=0, d_rw_pad=0, want_drw=True, gate_values=None):
     gu_h, go_h, wc, wf = ew_inputs(dtype, T, I, seed)
+    if gate_values is not None:  # row r's first gate columns: the values rotated by r
+        vals = np.array(gate_values, dtype=np.float32)
+        vals = workloads.f32_to_bf16_bits(vals) if dtype == "bf16" else vals
+        for r in range(T):
+            gu_h[r, :len(vals)] = np.roll(vals, r)
     w32 = wf if full else wc
     w_h = workloads.f32_to_bf16_bits(w32) if rw_dtype == "bf16" else w32
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
@@ -94,6 +99,19 @@ COMBOS = [(4.0, 25.0, "f32"), (1.0, None, "bf16"), (2.0, 1.5, "f32"), (16.0, Non
 @pytest.mark.parametrize("beta,lb,rw_dtype", COMBOS, ids=[f"b{b}-lb{l}-w{w}" for b, l, w in COMBOS])
 def test_elementwise_parity(dtype, T, I, beta, lb, rw_dtype, full, cuda_device):
     run_ew(cuda_device, dtype, T, I, beta, lb, full, rw_dtype, seed=T * 5 + I)
+
+
+# Gate values around and beyond the bf16 backward's clamp at -27.75 (where the
+# per-column form's signed gate arithmetic stops following g) and the usual
+# special values.
+GATE_SPECIALS = [0.0, -0.0, np.inf, -np.inf, 3e38, -3e38, -1e-30, 1e-39, -1.21875, 60.0, -27.5, -27.75, -28.0,
+                 -30.0, -40.0, -60.0, -88.0, -100.0, 1e-3, -1e-3]
+
+
+@pytest.mark.parametrize("full", [False, True], ids=["per_column", "per_element"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_elementwise_special_gate_values(dtype, full, cuda_device):
+    run_ew(cuda_device, dtype, 40, 64, 4.0, 25.0, full, "f32", seed=11, gate_values=GATE_SPECIALS)
 
 
 @pytest.mark.parametrize("dtype,rw_dtype", [("bf16", "f32"), ("bf16", "bf16"), ("f32", "f32")])
