@@ -96,6 +96,37 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def copy_bandwidth(torch, dev, stream, nbytes: int = 1 << 31, reps: int = 10) -> dict:
+    """A device-to-device copy measured in this run: ``dst.copy_(src)`` of
+    ``nbytes`` (one read and one write of every byte) on ``stream``, 3 untimed
+    copies, then ``reps`` timed one by one with CUDA events.  GB/s count
+    2 * nbytes; the median is the figure, the best beside it."""
+    src = torch.ones(nbytes // 2, dtype=torch.bfloat16, device=dev)
+    dst = torch.empty_like(src)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            dst.copy_(src)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for e0, e1 in evs:
+            e0.record(stream)
+            dst.copy_(src)
+            e1.record(stream)
+    torch.cuda.synchronize()
+    ms = sorted(e0.elapsed_time(e1) for e0, e1 in evs)
+    del src, dst
+    torch.cuda.empty_cache()
+    rate = lambda m: 2 * nbytes / (m / 1e3) / 1e9
+    return {"GB/s": rate(ms[len(ms) // 2]), "GB/s_best": rate(ms[0]), "bytes_per_copy": nbytes, "copies": reps,
+            "how": "torch copy_ between two device buffers (read + write counted), CUDA events, median of the copies"}
+
+
+def add_copy_fractions(copy: dict, *records) -> None:
+    """Each record with a GB/s figure gains its fraction of the same-run copy."""
+    for rec in records:
+        if isinstance(rec, dict) and "GB/s" in rec:
+            rec["frac_of_copy_same_run"] = rec["GB/s"] / copy["GB/s"]
+
+
 def host_info() -> dict:
     """The host the CPU figures were taken on: CPU model and core counts."""
     model = None
@@ -445,18 +476,21 @@ def run_ours_attn_res(args, dev, world, rank, local, barrier):
         secs = time.perf_counter() - t0
         cpu = cpu_record(per_row * done / secs / 1e9, "GB/s",
                          f"first {done} of {AR_TOKENS} rows, {secs:.1f} s, single-threaded fp64 oracle")
+    copy = copy_bandwidth(torch, dev, stream)
     if rank == 0:
         line = {"metric": AR_METRIC, "value": gbs * world, "unit": "GB/s", "n_gpus": world, "steps": K,
                 "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": ar_config(f"inputs {ar_bytes() / 1e9:.1f} GB exceed the 126 MB L2; no flush", world),
                 "kernels": {"situ_attn_res_staged_kernel": {"us": ms * 1e3, "GB/s": gbs,
-                                                            "frac_of_measured_copy": gbs / peak}},
+                                                            "frac_of_measured_copy": gbs / peak,
+                                                            "frac_of_copy_same_run": gbs / copy["GB/s"]}},
                 "torch_eager_fp32_chain": {"ms": torch_ms, "GB/s": ar_bytes() / (torch_ms / 1e3) / 1e9},
                 "roofline": {"bound": "hbm", "kernel": "situ_attn_res_staged_kernel", "achieved": gbs, "peak": peak,
                              "unit": "GB/s", "frac": gbs / peak, "peak_source": f"{peak_src} copy bandwidth",
-                             "traffic": recorded_traffic("situ_attn_res_staged_kernel", "attn_res")},
-                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K, "clocks": clocks.summary(),
+                             "traffic": recorded_traffic("situ_attn_res_staged_kernel", "attn_res"),
+                             "copy_same_run_gbs": copy["GB/s"], "frac_of_copy_same_run": gbs / copy["GB/s"]},
+                "copy_same_run": copy, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K, "clocks": clocks.summary(),
                 "device_status": pkg.abi.situ_glu_device_status(0), "device": torch.cuda.get_device_name(dev)}
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -1301,6 +1335,7 @@ def run_ours(args):
             subs[f"{w_.name} beta={b_:g}"] = measure_workload(pkg, w_, b_, dev, K, args.warmup, local, allreduce_max)
             torch.cuda.empty_cache()
 
+    copy = copy_bandwidth(torch, dev, stream)
     kernels = {fwd_kernel: kernel_record(fs, fwd_bytes, T, peak), bwd_kernel: kernel_record(bs, bwd_bytes, T, peak)}
     roofline = {"bound": "hbm", "kernel": bwd_kernel, "achieved": bwd_gbs, "peak": peak,
                 "unit": "GB/s", "frac": bwd_gbs / peak, "peak_source": f"{peak_src} copy bandwidth",
@@ -1322,6 +1357,11 @@ def run_ours(args):
         roofline = {"bound": "hbm", "kernel": roof_kernel, "achieved": q_gbs, "peak": peak, "unit": "GB/s",
                     "frac": q_gbs / peak, "peak_source": f"{peak_src} copy bandwidth", "traffic": traffic}
 
+    roofline["copy_same_run_gbs"] = copy["GB/s"]
+    roofline["frac_of_copy_same_run"] = roofline["achieved"] / copy["GB/s"]
+    add_copy_fractions(copy, *kernels.values())
+    for sub in (subs or {}).values():
+        add_copy_fractions(copy, sub.get("fwd"), sub.get("bwd"))
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
@@ -1332,6 +1372,7 @@ def run_ours(args):
             "pct_of_nominal_hbm": value / world / NOMINAL_HBM_GBS * 100.0,
             "kernels": kernels,
             "roofline": roofline,
+            "copy_same_run": copy,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches_per_step * K,
