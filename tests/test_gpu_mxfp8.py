@@ -148,6 +148,28 @@ def test_mxfp8_special_blocks(rule, cuda_device):
     assert np.all(ys[2] == 0) and not np.any(yc[2] & 0x7F)
 
 
+def gates_beyond_clamp(g_bits, I, seed):
+    """Gate values below -27.75, where the bf16 backward's signed form would need
+    its clamp: row 0 all of them (T_g down to 1e-26: blocks that keep their own
+    small scales), row 1 a band of them in the middle, row 2 one among ordinary
+    values (its warp takes the |g| form, the others the signed form), row 3
+    values just above the clamp."""
+    gu = workloads.bf16_bits_to_f32(g_bits).copy()
+    rng = np.random.default_rng(seed)
+    gu[0, :I] = -rng.uniform(28.0, 60.0, I)
+    gu[1, I // 4:3 * I // 4] = -rng.uniform(27.8, 40.0, I // 2)
+    gu[2, 17] = -40.0
+    gu[3, :I] = -rng.uniform(26.0, 27.7, I)
+    return workloads.f32_to_bf16_bits(gu.astype(np.float32))
+
+
+@pytest.mark.parametrize("rule", ["ocp", "ceil"])
+def test_mxfp8_gates_beyond_the_signed_clamp(rule, cuda_device):
+    T, I = 8, 256
+    g_h, _, _ = mx_inputs("bf16", T, I, seed=81)
+    run_mx(cuda_device, "bf16", T, I, 4.0, 25.0, "row_f32", rule, seed=81, gu_h=gates_beyond_clamp(g_h, I, 81))
+
+
 def test_mxfp8_grid_invariant(cuda_device):
     """Codes and scales do not depend on the launch size."""
     outs = []

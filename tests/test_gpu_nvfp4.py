@@ -292,6 +292,15 @@ def test_nvfp4_bwd_special_blocks(cuda_device):
     assert not np.any(unpack_e2m1(d[2:3]) & 7)
 
 
+def test_nvfp4_bwd_gates_beyond_the_signed_clamp(cuda_device):
+    """Gate values below the bf16 backward's clamp at -27.75 (tiny T_g) in
+    whole rows, a band, a single element, and just above it."""
+    from test_gpu_mxfp8 import gates_beyond_clamp
+    T, I = 8, 256
+    g_h, _, _ = nv_inputs("bf16", T, I, seed=83)
+    run_nv_bwd(cuda_device, "bf16", T, I, 4.0, 25.0, "row_f32", seed=83, gu_h=gates_beyond_clamp(g_h, I, 83))
+
+
 def test_nvfp4_bwd_grid_invariant(cuda_device):
     outs = []
     for ctas in (0, 1, 7):
