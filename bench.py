@@ -96,6 +96,41 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def link_bandwidth(torch, dev, host_in, dev_in, dev_out, host_out, reps: int = 2) -> dict:
+    """PCIe between pinned host memory and the device, measured in this run
+    with the bench's own buffers: host_in -> dev_in alone, dev_out -> host_out
+    alone, then both at once on two streams (CUDA events; the best of
+    ``reps``; GB/s per direction)."""
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    nb_up = host_in.numel() * host_in.element_size()
+    nb_down = host_out.numel() * host_out.element_size()
+
+    def timed(streams_ops):
+        torch.cuda.synchronize()
+        marks = []
+        for s, op in streams_ops:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            with torch.cuda.stream(s):
+                op()
+            b.record(s)
+            marks.append((a, b))
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in marks]
+
+    h2d = lambda: dev_in.copy_(host_in, non_blocking=True)
+    d2h = lambda: host_out.copy_(dev_out, non_blocking=True)
+    alone_up = min(timed([(up, h2d)])[0] for _ in range(reps))
+    alone_down = min(timed([(down, d2h)])[0] for _ in range(reps))
+    both = [timed([(up, h2d), (down, d2h)]) for _ in range(reps)]
+    both_up, both_down = min(b[0] for b in both), min(b[1] for b in both)
+    rate = lambda nb, ms: nb / (ms / 1e3) / 1e9
+    return {"h2d_GB/s": rate(nb_up, alone_up), "d2h_GB/s": rate(nb_down, alone_down),
+            "both_h2d_GB/s": rate(nb_up, both_up), "both_d2h_GB/s": rate(nb_down, both_down),
+            "bytes_h2d": nb_up, "bytes_d2h": nb_down,
+            "how": "copy_ between pinned host and device buffers of this run, CUDA events, best of %d" % reps}
+
+
 class L2Flush:
     """Leaves the L2 cold and clean before a timed kernel: writes a buffer of
     twice the L2 (which evicts whatever the last kernel left there), then reads
@@ -1338,6 +1373,15 @@ def run_ours(args):
         e2e = {"value": step_bytes * world / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": K2,
                "api": f"ffn_gated_activation_b200.{api}"}
+        if variant == "row":
+            # the link the end-to-end step is bound by, measured with its own buffers
+            link = link_bandwidth(torch, dev, gu_h, gu, d_gu, outputs_h[1])
+            e2e["link_same_run"] = link
+            e2e["h2d_GB/s"] = h2d / (e2e_ms / 1e3) / 1e9
+            e2e["d2h_GB/s"] = d2h / (e2e_ms / 1e3) / 1e9
+            # the time the link needs for the step's bytes at its both-ways rates, over the step's time
+            link_ms = max(h2d / link["both_h2d_GB/s"], d2h / link["both_d2h_GB/s"]) / 1e6
+            e2e["frac_of_link_both_ways"] = link_ms / e2e_ms
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
