@@ -196,6 +196,30 @@ def host_info() -> dict:
     return {"cpu_model": model, "host_cores": os.cpu_count(), "cores_available": avail}
 
 
+class PinnedCore:
+    """Runs the calling thread on one core of its affinity set (the first),
+    and puts the set back on exit; ``core`` is None where affinity cannot be
+    set."""
+
+    def __enter__(self):
+        self.saved, self.core = None, None
+        try:
+            self.saved = os.sched_getaffinity(0)
+            self.core = min(self.saved)
+            os.sched_setaffinity(0, {self.core})
+        except (AttributeError, OSError):
+            self.core = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.saved is not None:
+            try:
+                os.sched_setaffinity(0, self.saved)
+            except OSError:
+                pass
+        return False
+
+
 def cpu_record(value, unit, sample, cores=1, **extra) -> dict:
     """A cpu_baseline object: the oracle's rate on ``cores`` threads, with the host it ran on."""
     return {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample, **host_info(),
@@ -584,13 +608,21 @@ def cpu_oracle_rate(wl, beta, x, seconds: float, variant: str = "row"):
     """The fp64 oracle (single thread, as it stands) on the first rows of the
     workload, fwd then bwd per chunk of rows (MXFP8: plus the oracle's block
     quantisation of Y and d_gate_up), until ``seconds`` have passed.
-    Returns (GB/s of algorithmic bytes, rows done, elapsed)."""
+    Returns (GB/s of algorithmic bytes, rows done, elapsed, the core it was
+    pinned to or None)."""
     import oracle
     o = oracle.load()
     fb, bb = variant_bytes(wl, variant)
     per_row = (fb + bb) / wl.tokens
     w, mode = variant_weights(wl, x, variant)
     chunk = max(1, min(64, int(2 ** 20 // wl.inter)))
+    with PinnedCore() as pin:
+        rate, done, dt = _oracle_loop(o, wl, beta, x, w, mode, chunk, seconds, variant, per_row)
+    return rate, done, dt, pin.core
+
+
+def _oracle_loop(o, wl, beta, x, w, mode, chunk, seconds, variant, per_row):
+    import oracle
     done, t0 = 0, time.perf_counter()
     while done < wl.tokens:
         stop = min(wl.tokens, done + chunk)
@@ -651,12 +683,13 @@ def run_reference(args):
             o.nvfp4_quantize(y)
             o.nvfp4_quantize(np.concatenate([r.dg, r.du], axis=1))
 
-    for _ in range(args.warmup):
-        step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
-    dt = time.perf_counter() - t0
+    with PinnedCore() as pin:
+        for _ in range(args.warmup):
+            step()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            step()
+        dt = time.perf_counter() - t0
     value = per_row * rows_per_step * args.steps / dt / 1e9
     sample = (f"{rows_per_step} of {wl.tokens} rows per step (fwd + bwd), {args.steps} steps, "
               f"single-threaded fp64 oracle")
@@ -666,7 +699,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(wl, beta, "n/a (host)", 1, args.variant),
         "rows_per_s": rows_per_step * args.steps / dt,
-        "cpu_baseline": cpu_record(value, "GB/s", sample),
+        "cpu_baseline": cpu_record(value, "GB/s", sample, pinned_core=pin.core),
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -1008,7 +1041,8 @@ def run_ours_fc1(args, wl, beta, dev, world, rank, local, barrier):
 
 # The other workloads the 80 %-of-peak target names, each timed on its own
 # after the headline workload: (workload index, gate beta).
-SUB_WORKLOADS = ((2, 4.0), (3, 1.0), (3, 4.0), (3, 16.0), (4, 4.0))
+SUB_CPU_SECONDS = 2.0  # oracle sample per sub-workload (one pinned core)
+SUB_WORKLOADS = ((1, 4.0), (2, 4.0), (3, 1.0), (3, 4.0), (3, 16.0), (4, 4.0))
 
 
 def step_stats(ms_list) -> dict:
@@ -1039,13 +1073,19 @@ def row_kernels(wl):
     return fwd, "situ_glu_bwd_kernel"
 
 
-def measure_workload(pkg, wl, beta, dev, K, warmup, local, allreduce_max):
+def measure_workload(pkg, wl, beta, dev, K, warmup, local, allreduce_max, cpu_seconds=0.0):
     """One workload's forward and backward (per-row weights, native outputs),
     timed alone: K steps with CUDA events on the launching stream around each
-    pass.  Returns the workload's record."""
+    pass; with ``cpu_seconds`` > 0 also the fp64 oracle on one pinned core over
+    the workload's first rows.  Returns the workload's record."""
     import torch
     x = workloads.inputs(wl)
     T, I = wl.tokens, wl.inter
+    cpu = None
+    if cpu_seconds > 0:
+        rate, rows_done, secs, core = cpu_oracle_rate(wl, beta, x, cpu_seconds)
+        cpu = cpu_record(rate, "GB/s", f"first {rows_done} of {T} rows, fwd + bwd, {secs:.1f} s, single-threaded "
+                                       f"fp64", pinned_core=core)
     up = lambda a: (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16
                     else torch.from_numpy(a)).to(dev)
     gu, go = up(x["gate_up"]), up(x["grad_out"])
@@ -1096,7 +1136,7 @@ def measure_workload(pkg, wl, beta, dev, K, warmup, local, allreduce_max):
                    else f"inputs ({input_bytes / 1e6:.0f} MB) exceed the {L2_BYTES >> 20} MB L2; no flush"),
             "fwd": {"kernel": fk, **kernel_record(f, wl.fwd_bytes(), T, peak)},
             "bwd": {"kernel": bk, **kernel_record(b, wl.bwd_bytes(), T, peak)},
-            "clocks": clocks.summary()}
+            "clocks": clocks.summary(), "cpu_baseline": cpu}
 
 
 def cpu_oracle_rate_threads(wl, beta, x, seconds: float, threads: int):
@@ -1385,8 +1425,8 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, rows_done, secs = cpu_oracle_rate(wl, beta, x, args.cpu_seconds, variant)
-        extra = {}
+        rate, rows_done, secs, core = cpu_oracle_rate(wl, beta, x, args.cpu_seconds, variant)
+        extra = {"pinned_core": core}
         if variant == "row":
             threads = host_info()["cores_available"] or 1
             prate, prows, psecs = cpu_oracle_rate_threads(wl, beta, x, args.cpu_seconds, threads)
@@ -1407,7 +1447,9 @@ def run_ours(args):
             if idx == args.config and b_ == beta:
                 continue
             w_ = workloads.workload(idx)
-            subs[f"{w_.name} beta={b_:g}"] = measure_workload(pkg, w_, b_, dev, K, args.warmup, local, allreduce_max)
+            sub_cpu = SUB_CPU_SECONDS if rank == 0 and world == 1 and not args.no_cpu_baseline else 0.0
+            subs[f"{w_.name} beta={b_:g}"] = measure_workload(pkg, w_, b_, dev, K, args.warmup, local, allreduce_max,
+                                                              sub_cpu)
             torch.cuda.empty_cache()
 
     copy = copy_bandwidth(torch, dev, stream)
