@@ -264,14 +264,23 @@ def check_mx(name: str, codes: np.ndarray, scales: np.ndarray, ref: np.ndarray, 
     amax_lo = np.maximum(absb - tolb, 0.0).max(axis=2)
     amax_hi = (absb + tolb).max(axis=2)
     got_e = scales.astype(np.int64) - 127
-    for r in range(R):
-        for b in range(nb):
-            if special[r, b]:
-                assert scales[r, b] == 255, f"{name}: block ({r}, {b}) holds NaN/inf, scale {scales[r, b]}"
-                continue
-            e_lo, e_hi = o.mx_scale_exp(amax_lo[r, b], rule), o.mx_scale_exp(amax_hi[r, b], rule)
-            assert e_lo <= got_e[r, b] <= e_hi, (f"{name}: block ({r}, {b}) exponent {got_e[r, b]} outside "
-                                                 f"[{e_lo}, {e_hi}] (amax {amax_lo[r, b]}..{amax_hi[r, b]})")
+    sp = np.flatnonzero(special & (scales != 255))
+    assert sp.size == 0, f"{name}: block {np.unravel_index(sp[0], special.shape)} holds NaN/inf, scale {scales.flat[sp[0]]}"
+
+    def oracle_exp(amax):
+        # the oracle's shared exponent of every block maximum at once: a block
+        # holding just that maximum, through the oracle's own quantiser
+        m = np.zeros((R, C))
+        m[:, ::32] = np.where(special, 0.0, amax)
+        return o.mxfp8_quantize(m, rule)[1].astype(np.int64) - 127
+
+    e_lo, e_hi = oracle_exp(amax_lo), oracle_exp(amax_hi)
+    bad = np.flatnonzero(~special & ~((e_lo <= got_e) & (got_e <= e_hi)))
+    if bad.size:
+        r, b = np.unravel_index(bad[0], special.shape)
+        raise AssertionError(f"{name}: {bad.size} block exponents out of range; first block ({r}, {b}) exponent "
+                             f"{got_e[r, b]} outside [{e_lo[r, b]}, {e_hi[r, b]}] "
+                             f"(amax {amax_lo[r, b]}..{amax_hi[r, b]})")
     Xe = np.repeat(np.exp2(np.where(scales == 255, 0, got_e).astype(np.float64)), 32, axis=1)
     fin = np.repeat(~special, 32, axis=1) & np.isfinite(ref)
     with np.errstate(invalid="ignore"):
