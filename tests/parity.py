@@ -158,6 +158,20 @@ def bf16_faithful(bits: np.ndarray, ref: np.ndarray) -> np.ndarray:
     return (y == ref) | (up & (toward >= ref)) | (down & (toward <= ref))
 
 
+def by_row_chunks(fn, rows: np.ndarray, chunk: int = 16):
+    """``fn(rows_chunk)`` -- an oracle call returning an array, or a tuple of
+    arrays, with one leading entry per row -- evaluated on chunks of ``rows``
+    over the host's threads (the C oracle releases the GIL) and joined in row
+    order."""
+    from concurrent.futures import ThreadPoolExecutor
+    parts = [rows[i:i + chunk] for i in range(0, rows.size, chunk)] or [rows]
+    with ThreadPoolExecutor(max_workers=max(1, min(96, os.cpu_count() or 1))) as pool:
+        outs = list(pool.map(fn, parts))
+    if isinstance(outs[0], tuple):
+        return tuple(np.concatenate([o[k] for o in outs], axis=0) for k in range(len(outs[0])))
+    return np.concatenate(outs, axis=0)
+
+
 def check_output(name: str, got: np.ndarray, ref: np.ndarray, cancel_scale: np.ndarray | None = None):
     """Assert the tolerance rule elementwise.  Returns counts: ``n``;
     ``faithful_only``, the bf16 elements that pass only as a neighbour of ref;

@@ -8,6 +8,9 @@ probabilities by a few 1e-7 relative, ten times below 2^-18), or be a
 faithful bf16 rounding of it; an fp32 output within 1e-5 |ref| + 2^-18 M.  The probabilities enter every element of a
 row, so a wrong norm, epsilon, weight or source order fails whole rows.
 """
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import pytest
 import torch
@@ -112,3 +115,27 @@ def test_attn_res_full_size_sampled_rows(cuda_device):
     """16384 tokens, 8 stored sums + the current sum, hidden 7168: 64 sampled rows."""
     rows = np.random.default_rng(3).choice(16384, 64, replace=False)
     run_ar(cuda_device, 16384, 8, 7168, seed=11, rows=np.sort(rows))
+
+
+def test_attn_res_full_size_every_element(cuda_device):
+    """The bench's workload (16384 tokens, 8 stored sums + the current sum,
+    hidden 7168, bf16) in the bench's launch configuration: every output
+    element against the oracle, in row chunks over the host's threads."""
+    dev = cuda_device
+    T, B, H = 16384, 8, 7168
+    d = workloads.attn_res_inputs(T, B, H, 2)
+    blocks, prefix = to_device(d["blocks"], dev), to_device(d["prefix"], dev)
+    nw, pw = to_device(d["norm_weight"], dev), to_device(d["proj_weight"], dev)
+    out = pkg.apply_attn_res(prefix, blocks, pw, nw, 1e-6)
+    torch.cuda.synchronize()
+    got = to_host(out)
+    del out, blocks, prefix
+    o = oracle.load()
+
+    def chunk(r0):
+        rows = np.arange(r0, min(T, r0 + 256), dtype=np.int64)
+        ref, mag, _ = o.attn_res(d["blocks"], d["prefix"], d["norm_weight"], d["proj_weight"], 1e-6, rows=rows)
+        check_ar(f"out rows {r0}..{rows[-1]}", got[rows], ref, mag)
+
+    with ThreadPoolExecutor(max_workers=max(1, min(96, os.cpu_count() or 1))) as pool:
+        list(pool.map(chunk, range(0, T, 256)))
