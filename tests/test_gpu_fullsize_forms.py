@@ -1,6 +1,8 @@
-"""GPU parity at the routed-MoE workload's full size (gate_up bf16 [32768, 4096],
-I = 2048, beta = 4, linear_beta = 25, 1 % outliers) for the other output forms,
-through the public tensor API in the bench's launch configuration:
+"""GPU parity at full size for the other output forms, through the public
+tensor API in the bench's launch configuration: the routed-MoE workload
+(gate_up bf16 [32768, 4096], I = 2048, beta = 4, linear_beta = 25, 1 %
+outliers) for every form, and the large workload (gate_up bf16 [131072, 8192])
+for the element-wise weights and MXFP8:
 
   * per-column routing weights [I] and per-element routing weights [T, I]:
     every element of Y and d_gate_up against the fp64 oracle, and every
@@ -45,16 +47,19 @@ def _pool(fn, T):
         return list(pool.map(fn, range(0, T, ROWS)))
 
 
-def _inputs(dev):
-    wl = workloads.workload(2)
+def _inputs(dev, index=2):
+    wl = workloads.workload(index)
     x = workloads.inputs(wl)
     return wl, x, to_device(x["gate_up"], dev), to_device(x["grad_out"], dev)
 
 
+@pytest.mark.parametrize("index", [2, 4], ids=["routed_moe", "large"])
 @pytest.mark.parametrize("form", ["per_column", "per_element"])
-def test_routed_moe_elementwise_weights_every_element(form, cuda_device):
-    wl, x, gu, go = _inputs(cuda_device)
+def test_elementwise_weights_every_element(form, index, cuda_device):
+    wl, x, gu, go = _inputs(cuda_device, index)
     T, I = wl.tokens, wl.inter
+    beta, lb = wl.betas[0], wl.linear_beta
+    assert (beta, lb) == (BETA, LB)
     col = form == "per_column"
     w = workloads.column_weights(wl) if col else workloads.element_weights(wl)
     rw = torch.from_numpy(np.ascontiguousarray(w)).reshape((I,) if col else (T, I)).to(cuda_device)
@@ -86,8 +91,9 @@ def test_routed_moe_elementwise_weights_every_element(form, cuda_device):
         check_dw("d_w (per column)", drw_h.reshape(-1), colsum, colmag)
 
 
-def test_routed_moe_mxfp8_every_code(cuda_device):
-    wl, x, gu, go = _inputs(cuda_device)
+@pytest.mark.parametrize("index", [2, 4], ids=["routed_moe", "large"])
+def test_mxfp8_every_code(index, cuda_device):
+    wl, x, gu, go = _inputs(cuda_device, index)
     T, I = wl.tokens, wl.inter
     rw = to_device(x["routing_weights"], cuda_device).reshape(T, 1)
     yc, ys = pkg.situ_glu_fwd_mxfp8(gu, rw, BETA, LB, rule="ocp")
