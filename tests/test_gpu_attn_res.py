@@ -63,12 +63,13 @@ def run_ar(dev, T, B, H, with_prefix=True, dtype="bf16", out_dtype=torch.bfloat1
     return got
 
 
-@pytest.mark.parametrize("T,B,H", [(1, 1, 8), (3, 2, 64), (257, 8, 512), (130, 3, 7168), (64, 15, 1024)])
+@pytest.mark.parametrize("T,B,H", [(1, 1, 8), (3, 2, 64), (257, 8, 512), (130, 3, 7168), (64, 15, 1024),
+                                   (37, 5, 1032)])  # 129 vectors a row: two per thread, the last thread one
 def test_attn_res_bf16(T, B, H, cuda_device):
     run_ar(cuda_device, T, B, H, seed=T + B)
 
 
-@pytest.mark.parametrize("T,B,H", [(33, 4, 256), (70, 8, 4096), (40, 8, 2048)])
+@pytest.mark.parametrize("T,B,H", [(33, 4, 256), (70, 8, 4096), (40, 8, 2048), (21, 4, 1028)])
 def test_attn_res_fp32_values_and_output(T, B, H, cuda_device):
     run_ar(cuda_device, T, B, H, dtype="f32", out_dtype=torch.float32, seed=7)
 
