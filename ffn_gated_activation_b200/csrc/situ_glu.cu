@@ -2251,9 +2251,9 @@ __global__ void __launch_bounds__(kArThreads) situ_attn_res_kernel(const ArArgs 
   }
 }
 
-// Staged form (the default when a source row is at most kArStagedThreads
-// 16-byte vectors, there are at most kArStagedSources sources, and the row
-// fits in shared memory): one CTA per SM; thread j owns column vectors j,
+// Staged form (the default when a source row is at most 1024 16-byte
+// vectors, there are at most kArStagedSources sources, and the row fits in
+// shared memory): one CTA per SM; thread j owns column vectors j,
 // j + nt, ... (V of them, nt threads) of every source.  Bulk copies bring the
 // CTA's next token row -- the stored sums as one run when they lie back to
 // back, else one run per source, and the current sum -- into shared memory
@@ -2379,10 +2379,14 @@ __device__ __forceinline__ void ar_combine_store(const ArArgs& a, const uint4 (&
   }
 }
 
-template <typename S, int V>
-__global__ void __launch_bounds__(kArStagedThreads / V, 1) situ_attn_res_staged_kernel(const ArArgs a) {
+// NT: the most threads a launch may have.  Two vectors a thread take 448
+// threads for rows of up to 896 vectors and 512 beyond (up to 1024: hidden
+// 8192 in bf16, 4096 in fp32); the 448-thread bound keeps the register
+// allocation that measured 2 % faster at hidden 7168.
+template <typename S, int V, int NT>
+__global__ void __launch_bounds__(NT, 1) situ_attn_res_staged_kernel(const ArArgs a) {
   extern __shared__ __align__(16) unsigned char ar_stage[];  // [sources][row bytes]
-  __shared__ float red[kArStagedThreads / V / 32][2 * kArStagedSources];
+  __shared__ float red[NT / 32][2 * kArStagedSources];
   __shared__ float logit_sh[kArStagedSources];
   __shared__ float prob_sh[kArStagedSources];
   __shared__ __align__(8) uint64_t bar;
@@ -3894,7 +3898,7 @@ extern "C" situ_status_t situ_attn_res_fwd(const void* blocks, int64_t nblocks, 
   a.out_bf16 = out_dtype == SITU_DTYPE_BF16;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t stage_bytes = sources * hidden * es;
-  if (a.vpr <= kArStagedThreads && sources <= kArStagedSources && stage_bytes <= 180 * 1024) {
+  if (a.vpr <= 1024 && sources <= kArStagedSources && stage_bytes <= 180 * 1024) {
     auto staged = [&](auto kb, auto kf, int vecs) -> situ_status_t {
       const void* ks = dtype == SITU_DTYPE_BF16 ? reinterpret_cast<const void*>(kb) : reinterpret_cast<const void*>(kf);
       const int threads = ((a.vpr + vecs - 1) / vecs + 31) / 32 * 32;
@@ -3916,9 +3920,12 @@ extern "C" situ_status_t situ_attn_res_fwd(const void* blocks, int64_t nblocks, 
     // than one at hidden 7168 (the per-row reductions and the softmax
     // broadcast are paid once per two vectors); four were 7 % slower (seven
     // warps per SM leave the row's dependent steps exposed).
+    if (a.vpr > 2 * 448)
+      return staged(situ_attn_res_staged_kernel<Bf16, 2, 512>, situ_attn_res_staged_kernel<F32, 2, 512>, 2);
     if (a.vpr >= 128)
-      return staged(situ_attn_res_staged_kernel<Bf16, 2>, situ_attn_res_staged_kernel<F32, 2>, 2);
-    return staged(situ_attn_res_staged_kernel<Bf16, 1>, situ_attn_res_staged_kernel<F32, 1>, 1);
+      return staged(situ_attn_res_staged_kernel<Bf16, 2, 448>, situ_attn_res_staged_kernel<F32, 2, 448>, 2);
+    return staged(situ_attn_res_staged_kernel<Bf16, 1, kArStagedThreads>,
+                  situ_attn_res_staged_kernel<F32, 1, kArStagedThreads>, 1);
   }
   const void* k = dtype == SITU_DTYPE_BF16 ? reinterpret_cast<const void*>(situ_attn_res_kernel<Bf16>)
                                            : reinterpret_cast<const void*>(situ_attn_res_kernel<F32>);

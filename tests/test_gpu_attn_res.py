@@ -64,7 +64,8 @@ def run_ar(dev, T, B, H, with_prefix=True, dtype="bf16", out_dtype=torch.bfloat1
 
 
 @pytest.mark.parametrize("T,B,H", [(1, 1, 8), (3, 2, 64), (257, 8, 512), (130, 3, 7168), (64, 15, 1024),
-                                   (37, 5, 1032)])  # 129 vectors a row: two per thread, the last thread one
+                                   (37, 5, 1032),  # 129 vectors a row: two per thread, the last thread one
+                                   (50, 8, 8192), (33, 8, 7176)])  # 1024 and 897 vectors: 512 and 480 threads
 def test_attn_res_bf16(T, B, H, cuda_device):
     run_ar(cuda_device, T, B, H, seed=T + B)
 
