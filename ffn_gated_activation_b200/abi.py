@@ -62,6 +62,7 @@ SIGNATURES = {
     "situ_glu_set_max_ctas": (_INT, [_INT]),
     "situ_glu_set_load_path": (_INT, [_INT]),
     "situ_glu_device_status": (_INT, [_INT]),
+    "situ_glu_wait_probe": (_INT, [_I64, _VP]),
     "situ_glu_bwd_no_alloc": (_INT, [_VP, _INT, _I64, _I64, _I64, _VP, _INT, _INT, _I64, _DBL, _INT, _DBL,
                                      _VP, _I64, _VP, _I64, _VP, _I64, _VP]),
 }
@@ -221,6 +222,10 @@ def situ_glu_abi_version() -> int:
 
 def situ_glu_set_max_ctas(max_ctas) -> int:
     return lib().situ_glu_set_max_ctas(max_ctas)
+
+
+def situ_glu_wait_probe(limit_ns, stream=None) -> int:
+    return lib().situ_glu_wait_probe(int(limit_ns), stream)
 
 
 def situ_glu_set_load_path(path) -> int:

@@ -1882,13 +1882,28 @@ __device__ __forceinline__ unsigned long long global_timer_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// Wait for the phase of parity `parity` to complete; false once the limit expires.
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
+// Wait for the phase of parity `parity` to complete; false once `limit_ns`
+// (the kernels': kWaitLimitNs) has passed.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* b, uint32_t parity, unsigned long long limit_ns) {
   if (mbar_try_wait(b, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   while (!mbar_try_wait(b, parity))
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
   return true;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
+  return mbar_wait_for(b, parity, kWaitLimitNs);
+}
+
+// One thread waiting on an mbarrier that nothing completes (situ_glu_wait_probe):
+// the expiry path every staged kernel takes when a copy never lands.
+__global__ void situ_wait_probe_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+    if (!mbar_wait_for(&bar, 0, limit_ns)) atomicExch(&g_device_status, kStatusWaitExpired);
+  }
 }
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -3538,6 +3553,13 @@ int situ_glu_device_status(int clear) {
     if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof zero) != cudaSuccess) return -1;
   }
   return v;
+}
+
+situ_status_t situ_glu_wait_probe(int64_t limit_ns, void* stream) {
+  if (limit_ns < 1 || limit_ns > 10000000000LL)
+    return fail(SITU_ERR_INVALID_ARG, "limit_ns %lld outside [1, 1e10]", (long long)limit_ns);
+  situ_wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<unsigned long long>(limit_ns));
+  return check_launch("situ_glu_wait_probe");
 }
 
 int situ_glu_set_max_ctas(int max_ctas) {

@@ -435,6 +435,15 @@ int situ_glu_set_load_path(int path);
  * reports an error. */
 int situ_glu_device_status(int clear);
 
+/* Test hook for the bounded waits above: enqueues on `stream` one thread
+ * block that waits, with the limit `limit_ns` (1 to 10^10 ns) instead of the
+ * kernels' 2 s, on a shared-memory mbarrier that nothing completes.  The wait
+ * runs out, the block sets the status word to 1 and returns, as a kernel
+ * whose staged copy never lands would; nothing faults and the context stays
+ * usable.  SITU_ERR_INVALID_ARG (nothing enqueued) for a limit outside that
+ * range. */
+situ_status_t situ_glu_wait_probe(int64_t limit_ns, void *stream);
+
 /*
  * Backward without caller scratch.  Same arguments and results as
  * situ_glu_bwd, minus `workspace` and `workspace_bytes`.  The pages describe

@@ -93,6 +93,12 @@ def test_max_ctas_knob(native_lib_path):
     assert abi.situ_glu_set_max_ctas(-1) == -1
 
 
+@pytest.mark.parametrize("limit_ns", [0, -1, 10_000_000_001])
+def test_wait_probe_rejects_the_limit_before_any_launch(limit_ns, native_lib_path):
+    assert abi.situ_glu_wait_probe(limit_ns) == INVALID
+    assert "limit_ns" in abi.situ_glu_last_error()
+
+
 def fwd(**kw):
     a = dict(gate_up=GU, dtype=BF16, tokens=16, inter=64, gate_up_row_stride=128, rw=RW, rw_dtype=F32,
              rw_mode=ROW, rw_stride=1, beta=4.0, has_linear_beta=1, linear_beta=25.0, out=OUT,

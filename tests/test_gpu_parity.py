@@ -375,3 +375,23 @@ def test_wide_and_two_vector_layouts_agree(dtype, T, I, cuda_device):
 def test_no_bounded_wait_expired(cuda_device):
     """No kernel launched by the tests above gave up on a shared-memory stage."""
     assert abi.situ_glu_device_status(0) == 0
+
+
+def test_expired_wait_sets_the_status_and_the_context_survives(cuda_device):
+    """A bounded wait that runs out: the probe waits 5 ms on an mbarrier that
+    nothing completes, gives up, sets the status word and returns.  The host
+    reads 1, clears it, and the next launches on the same context still match
+    the oracle."""
+    assert abi.situ_glu_device_status(1) == 0
+    stream = torch.cuda.current_stream(cuda_device).cuda_stream
+    abi.check(abi.situ_glu_wait_probe(5_000_000, stream), "wait probe")
+    assert abi.situ_glu_device_status(1) == 1
+    assert abi.situ_glu_device_status(0) == 0
+    wl = workloads.workload(0)
+    x = workloads.inputs(wl, tokens=64)
+    gu = to_device(x["gate_up"], cuda_device)
+    rw = to_device(x["routing_weights"], cuda_device).reshape(64, 1)
+    y = pkg.situ_glu_fwd(gu, rw, 4.0, 25.0)
+    torch.cuda.synchronize()
+    check_output("Y after an expired wait", to_host(y), oracle.load().fwd(x["gate_up"], x["routing_weights"], 4.0, 25.0))
+    assert abi.situ_glu_device_status(0) == 0
