@@ -175,6 +175,46 @@ def test_special_values(cuda_device):
             check_dw(f"d_w {dtype} beta={beta}", to_host(d_rw), ref.dw, ref.sw)
 
 
+@pytest.mark.parametrize("lb", [25.0, None])
+def test_small_gate_values_around_the_series_threshold(lb, cuda_device):
+    """Gate values of magnitude 2^-13 to 2^-4, log-uniform with random signs,
+    where 1 - exp(-2g/beta) is small and its relative accuracy decides the
+    outputs' relative accuracy.  Even rows hold only |g| >= 2^-9 (whole
+    vectors that need no series); odd rows span the full range, with
+    2^-9 and the bf16 value just below it planted at vector boundaries.
+    Every element of Y, dG, dU and d_w against the oracle (bf16, beta = 4)."""
+    dev = cuda_device
+    T, I = 96, 2048
+    gu_h, rw32, go_h = case_inputs("bf16", T, I, seed=91)
+    rng = np.random.default_rng(91)
+    mag = np.where((np.arange(T) % 2 == 0)[:, None], rng.uniform(-9.0, -4.0, (T, I)), rng.uniform(-13.0, -4.0, (T, I)))
+    g = (np.exp2(mag) * rng.choice([-1.0, 1.0], (T, I))).astype(np.float32)
+    g[1::2, 0::8] = np.float32(2.0 ** -9)
+    g[1::2, 7::16] = -np.float32(2.0 ** -9)
+    below = workloads.f32_to_bf16_bits(np.array([2.0 ** -9], dtype=np.float32)) - 1  # 0x3AFF
+    gu_h = gu_h.copy()
+    gu_h[:, :I] = workloads.f32_to_bf16_bits(g)
+    gu_h[1::4, 8::32] = below
+    gu_h[3::4, 15::32] = below | 0x8000
+    gu, go, rw = to_device(gu_h, dev), to_device(go_h, dev), to_device(rw32, dev)
+    out = Guarded(T, I, I, torch.bfloat16, dev)
+    dgu = Guarded(T, 2 * I, 2 * I, torch.bfloat16, dev)
+    d_rw = torch.empty(T, dtype=torch.float32, device=dev)
+    abi.check(call_fwd(gu, I, rw, abi.SITU_RW_ROW, 4.0, lb, out), "fwd")
+    abi.check(call_bwd(gu, I, rw, abi.SITU_RW_ROW, 4.0, lb, go, dgu, d_rw=d_rw), "bwd")
+    torch.cuda.synchronize()
+    out.check()
+    dgu.check()
+    o = oracle.load()
+    check_output("Y", to_host(out.view), o.fwd(gu_h, rw32, 4.0, lb))
+    ref = o.bwd(gu_h, rw32, go_h, 4.0, lb)
+    d = to_host(dgu.view)
+    check_output("dG", d[:, :I], ref.dg, ref.cg)
+    rep = check_output("dU", d[:, I:], ref.du)
+    assert rep["faithful_only"] <= 1e-2 * rep["n"], rep
+    check_dw("d_w", to_host(d_rw), ref.dw, ref.sw)
+
+
 def test_drw_not_wanted_leaves_gradients_identical(cuda_device):
     dev = cuda_device
     T, I = 97, 1024
