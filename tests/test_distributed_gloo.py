@@ -8,7 +8,8 @@ GPU); the tests check the product's sharding and reduction helpers:
   all-reduced per-rank routing-weight partials equal the full-width gradient;
 * data parallelism with a broadcast weight: row shards' partial sums,
   all-reduced, equal the single-process gradient;
-* max-over-ranks timing and the shard arithmetic.
+* max-over-ranks timing and the shard arithmetic;
+* a rank that leaves: the other rank's next collective ends with an error.
 """
 import os
 import socket
@@ -200,6 +201,44 @@ def test_shard_range_partitions(n, world, align):
         assert a <= b and a % align == 0
     sizes = [b - a for a, b in spans]
     assert max(sizes) - min(sizes) <= align
+
+
+def _leave_entry(rank, port, result_path, how):
+    """Rank 1 leaves between steps, before its weight-gradient all-reduce
+    (`exit`: its process ends; `stall`: it stays alive but never joins);
+    rank 0 enters that all-reduce and records how it ended."""
+    import datetime
+    import json
+    import time
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=WORLD,
+                            timeout=datetime.timedelta(seconds=3))
+    if rank == 1:
+        if how == "stall":
+            time.sleep(10)
+        os._exit(0)  # gone, with no collective in flight and no teardown
+    t0 = time.monotonic()
+    try:
+        D.allreduce_drw(torch.ones(4, dtype=torch.float64))
+        outcome = "completed"
+    except Exception as e:  # gloo reports the lost peer or the timeout
+        outcome = f"error: {type(e).__name__}: {str(e)[:200]}"
+    with open(result_path, "w") as f:
+        json.dump({"outcome": outcome, "seconds": time.monotonic() - t0}, f)
+    os._exit(0)  # the group has lost a member: skip its teardown
+
+
+@pytest.mark.parametrize("how", ["exit", "stall"])
+def test_a_rank_that_leaves_ends_the_others_collective_with_an_error(how, tmp_path):
+    """Failure detection on the host: with a short process-group timeout (3 s),
+    the surviving rank's next collective (the routing-weight gradient's
+    all-reduce) raises instead of waiting for the rank that left, whether
+    that rank's process ended or it stopped taking part."""
+    import json
+    result = tmp_path / "rank0.json"
+    mp.spawn(_leave_entry, args=(_free_port(), str(result), how), nprocs=WORLD, join=True)
+    rec = json.loads(result.read_text())
+    assert rec["outcome"].startswith("error"), rec
+    assert rec["seconds"] < 9, rec  # before the stalled rank would have gone
 
 
 def test_max_over_ranks_without_group():
