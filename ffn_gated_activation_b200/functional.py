@@ -47,10 +47,41 @@ def _rows(gate_up: torch.Tensor):
         raise ValueError(f"gate_up's last dimension must be 2 * intermediate, got {tuple(gate_up.shape)}")
     inter = gate_up.shape[-1] // 2
     lead = tuple(gate_up.shape[:-1])
-    g2 = gate_up.reshape(-1, 2 * inter)
+    g2 = gate_up if gate_up.dim() == 2 else gate_up.reshape(-1, 2 * inter)  # 2-D: no view to build
     if g2.stride(1) != 1 or (g2.shape[0] > 1 and g2.stride(0) < 2 * inter):
         g2 = g2.contiguous()
     return g2, lead, inter
+
+
+def _given(t: torch.Tensor, shape: tuple, device, what: str, dtype=None) -> torch.Tensor:
+    """A caller's output buffer, checked before the library writes to it (the
+    library sees a pointer and a row pitch only, so a smaller or strided
+    buffer would be written past): exactly ``shape``, ``dtype`` (None: any
+    one-byte dtype, for code and scale bytes), on ``device``, elements of a
+    row adjacent and rows apart by at least a row.  Returns the 2-D view
+    [rows, shape[-1]] the library is given."""
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{what} shape {tuple(t.shape)} != {tuple(shape)}")
+    if (t.element_size() != 1) if dtype is None else (t.dtype != dtype):
+        raise TypeError(f"{what} must be {dtype if dtype is not None else 'a one-byte dtype'}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{what} must be on {device}, got {t.device}")
+    cols = shape[-1]
+    t2 = t if t.dim() == 2 else t.reshape(-1, cols)
+    if t2.numel() and (t2.data_ptr() != t.data_ptr() or t2.stride(1) != 1
+                       or (t2.shape[0] > 1 and t2.stride(0) < cols)):
+        raise ValueError(f"{what} must hold each row's elements adjacent, rows not overlapping")
+    return t2
+
+
+def _given_drw(d_rw: torch.Tensor, routing_weights: torch.Tensor, device) -> torch.Tensor:
+    """A caller's routing-weight gradient buffer: the weights' shape and dtype."""
+    if tuple(d_rw.shape) != tuple(routing_weights.shape) or d_rw.dtype != routing_weights.dtype:
+        raise ValueError(f"d_rw must have routing_weights' shape {tuple(routing_weights.shape)} and dtype "
+                         f"{routing_weights.dtype}, got {tuple(d_rw.shape)} {d_rw.dtype}")
+    if d_rw.device != device:
+        raise ValueError(f"d_rw must be on {device}, got {d_rw.device}")
+    return d_rw
 
 
 def routing_mode(gate_up_lead: tuple, inter: int, routing_weights):
@@ -68,6 +99,8 @@ def routing_mode(gate_up_lead: tuple, inter: int, routing_weights):
     rw = routing_weights
     if rw.numel() == 1:
         return abi.SITU_RW_SCALAR, rw.reshape(1), 1
+    if rw.dim() == 2 and len(gate_up_lead) == 1 and rw.shape[0] == gate_up_lead[0] and rw.shape[1] == 1:
+        return abi.SITU_RW_ROW, rw, rw.stride(0)  # [T, 1]: row r at rw.stride(0) * r, as in its flat view
     if rw.dim() == len(gate_up_lead) + 1 and tuple(rw.shape[:-1]) == gate_up_lead and rw.shape[-1] == 1:
         flat = rw.reshape(-1)
         return abi.SITU_RW_ROW, flat, flat.stride(0) if flat.numel() > 1 else 1
@@ -104,7 +137,9 @@ def situ_glu_fwd(gate_up: torch.Tensor, routing_weights, beta: float = DEFAULT_B
         rw_dtype = abi.SITU_DTYPE_F32
     if out is None:
         out = torch.empty(lead + (inter,), dtype=gate_up.dtype, device=gate_up.device)
-    o2 = out.view(-1, inter)
+        o2 = out if out.dim() == 2 else out.view(-1, inter)
+    else:
+        o2 = _given(out, lead + (inter,), gate_up.device, "out", gate_up.dtype)
     tokens = g2.shape[0]
     st = abi.situ_glu_fwd(g2.data_ptr(), dtype, tokens, inter, g2.stride(0) if tokens > 1 else 2 * inter,
                           rw.data_ptr() if rw is not None else None, rw_dtype, mode, rw_stride,
@@ -129,7 +164,7 @@ def situ_glu_bwd(gate_up: torch.Tensor, routing_weights, grad_out: torch.Tensor,
         raise TypeError("grad_out must have gate_up's dtype")
     if tuple(grad_out.shape) != lead + (inter,):
         raise ValueError(f"grad_out shape {tuple(grad_out.shape)} != {lead + (inter,)}")
-    go2 = grad_out.reshape(-1, inter)
+    go2 = grad_out if grad_out.dim() == 2 else grad_out.reshape(-1, inter)
     if go2.stride(1) != 1 or (go2.shape[0] > 1 and go2.stride(0) < inter):
         go2 = go2.contiguous()
     mode, rw, rw_stride = routing_mode(lead, inter, routing_weights)
@@ -137,19 +172,27 @@ def situ_glu_bwd(gate_up: torch.Tensor, routing_weights, grad_out: torch.Tensor,
     want = bool(want_drw) and rw is not None
     if d_gate_up is None:
         d_gate_up = torch.empty(lead + (2 * inter,), dtype=gate_up.dtype, device=gate_up.device)
-    dg2 = d_gate_up.view(-1, 2 * inter)
+        dg2 = d_gate_up if d_gate_up.dim() == 2 else d_gate_up.view(-1, 2 * inter)
+    else:
+        dg2 = _given(d_gate_up, lead + (2 * inter,), gate_up.device, "d_gate_up", gate_up.dtype)
     d_rw_flat, d_rw_stride = None, 1
     if want:
         if d_rw is None:
             d_rw = torch.empty(routing_weights.shape, dtype=routing_weights.dtype, device=gate_up.device)
+        else:
+            _given_drw(d_rw, routing_weights, gate_up.device)
         if mode == abi.SITU_RW_FULL:
             d_rw_flat = d_rw.view(-1, inter)
             d_rw_stride = d_rw_flat.stride(0) if d_rw_flat.shape[0] > 1 else inter
+        elif d_rw.dim() == 2 and d_rw.shape[1] == 1 and d_rw.shape[0] > 1:
+            d_rw_flat, d_rw_stride = d_rw, d_rw.stride(0)  # [T, 1]: as its flat view
         else:
             d_rw_flat = d_rw.view(-1)
             d_rw_stride = d_rw_flat.stride(0) if d_rw_flat.numel() > 1 else 1
     tokens = g2.shape[0]
-    ws_bytes = abi.situ_glu_bwd_workspace_bytes(tokens, inter, mode, int(want))
+    # Only a broadcast or per-column weight's gradient takes scratch.
+    ws_bytes = (abi.situ_glu_bwd_workspace_bytes(tokens, inter, mode, int(want))
+                if want and mode in (abi.SITU_RW_SCALAR, abi.SITU_RW_COL) else 0)
     if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=gate_up.device)
     st = abi.situ_glu_bwd(g2.data_ptr(), dtype, tokens, inter, g2.stride(0) if tokens > 1 else 2 * inter,
@@ -183,12 +226,14 @@ def _mx_buffers(lead: tuple, cols: int, device, data=None, scale=None):
     tensors and their 2-D byte views."""
     if data is None:
         data = torch.empty(lead + (cols,), dtype=torch.float8_e4m3fn, device=device)
+        d2 = data.view(-1, cols)
+    else:
+        d2 = _given(data, lead + (cols,), device, "MXFP8 data")
     if scale is None:
         scale = torch.empty(lead + (cols // 32,), dtype=torch.uint8, device=device)
-    if data.element_size() != 1 or scale.element_size() != 1:
-        raise TypeError("MXFP8 data and scale tensors hold one byte per element")
-    d2 = data.view(-1, cols)
-    s2 = scale.view(-1, cols // 32)
+        s2 = scale.view(-1, cols // 32)
+    else:
+        s2 = _given(scale, lead + (cols // 32,), device, "MXFP8 scale")
     return data, scale, d2, s2
 
 
@@ -234,7 +279,7 @@ def situ_glu_bwd_mxfp8(gate_up: torch.Tensor, routing_weights, grad_out: torch.T
         raise TypeError("grad_out must have gate_up's dtype")
     if tuple(grad_out.shape) != lead + (inter,):
         raise ValueError(f"grad_out shape {tuple(grad_out.shape)} != {lead + (inter,)}")
-    go2 = grad_out.reshape(-1, inter)
+    go2 = grad_out if grad_out.dim() == 2 else grad_out.reshape(-1, inter)
     if go2.stride(1) != 1 or (go2.shape[0] > 1 and go2.stride(0) < inter):
         go2 = go2.contiguous()
     mode, rw, rw_stride = routing_mode(lead, inter, routing_weights)
@@ -245,6 +290,8 @@ def situ_glu_bwd_mxfp8(gate_up: torch.Tensor, routing_weights, grad_out: torch.T
     if want:
         if d_rw is None:
             d_rw = torch.empty(routing_weights.shape, dtype=routing_weights.dtype, device=gate_up.device)
+        else:
+            _given_drw(d_rw, routing_weights, gate_up.device)
         d_rw_flat = d_rw.view(-1)
         d_rw_stride = d_rw_flat.stride(0) if d_rw_flat.numel() > 1 else 1
     tokens = g2.shape[0]
@@ -302,6 +349,8 @@ def situ_glu_fc1_fwd(x: torch.Tensor, w1: torch.Tensor, offsets: torch.Tensor, r
     rw_dtype = _dtype_code(rw, "routing_weights") if rw is not None else abi.SITU_DTYPE_F32
     if out is None:
         out = torch.empty(tokens, inter, dtype=torch.bfloat16, device=x.device)
+    else:
+        _given(out, (tokens, inter), x.device, "out", torch.bfloat16)
     st = abi.situ_glu_fc1_fwd(x.data_ptr(), tokens, hidden, x.stride(0) if tokens > 1 else hidden,
                               w2.data_ptr(), experts, inter, w2.stride(0), offsets.data_ptr(),
                               rw.data_ptr() if rw is not None else None, rw_dtype, mode, rw_stride,
@@ -343,10 +392,14 @@ def situ_glu_fc2_dgrad_bwd(dout: torch.Tensor, w2t: torch.Tensor, offsets: torch
     want = bool(want_drw) and rw is not None
     if d_gate_up is None:
         d_gate_up = torch.empty(tokens, 2 * inter, dtype=torch.bfloat16, device=dout.device)
+    else:
+        _given(d_gate_up, (tokens, 2 * inter), dout.device, "d_gate_up", torch.bfloat16)
     d_rw_flat = None
     if want:
         if d_rw is None:
             d_rw = torch.empty(routing_weights.shape, dtype=routing_weights.dtype, device=dout.device)
+        else:
+            _given_drw(d_rw, routing_weights, dout.device)
         d_rw_flat = d_rw.view(-1)
     ws = abi.situ_glu_fc2_dgrad_workspace_bytes(tokens, inter, int(want))
     if ws and (workspace is None or workspace.numel() * workspace.element_size() < ws):
@@ -384,6 +437,8 @@ def _attn_res_launch(blocks, prefix, norm_weight, proj_weight, variance_epsilon,
     out_dtype = src.dtype if out_dtype is None else out_dtype
     if out is None:
         out = torch.empty(tokens, hidden, dtype=out_dtype, device=src.device)
+    else:
+        _given(out, (tokens, hidden), src.device, "out", out.dtype)
     nb = 0
     if blocks is not None:
         if blocks.stride(-1) != 1:
@@ -446,8 +501,12 @@ def situ_glu_fwd_nvfp4(gate_up: torch.Tensor, routing_weights, beta: float = DEF
     if not amax_only:
         if data is None:
             data = torch.empty(lead + (inter // 2,), dtype=torch.uint8, device=gate_up.device)
+        else:
+            _given(data, lead + (inter // 2,), gate_up.device, "NVFP4 data")
         if scale is None:
             scale = torch.empty(lead + (inter // 16,), dtype=torch.float8_e4m3fn, device=gate_up.device)
+        else:
+            _given(scale, lead + (inter // 16,), gate_up.device, "NVFP4 scale")
     given = amax is not None
     if amax is None:
         amax = amax_out if amax_out is not None else torch.empty(1, dtype=torch.float32, device=gate_up.device)
@@ -490,7 +549,7 @@ def situ_glu_bwd_nvfp4(gate_up: torch.Tensor, routing_weights, grad_out: torch.T
         raise TypeError("grad_out must have gate_up's dtype")
     if tuple(grad_out.shape) != lead + (inter,):
         raise ValueError(f"grad_out shape {tuple(grad_out.shape)} != {lead + (inter,)}")
-    go2 = grad_out.reshape(-1, inter)
+    go2 = grad_out if grad_out.dim() == 2 else grad_out.reshape(-1, inter)
     if go2.stride(1) != 1 or (go2.shape[0] > 1 and go2.stride(0) < inter):
         go2 = go2.contiguous()
     mode, rw, rw_stride = routing_mode(lead, inter, routing_weights)
@@ -501,8 +560,12 @@ def situ_glu_bwd_nvfp4(gate_up: torch.Tensor, routing_weights, grad_out: torch.T
     if not amax_only:
         if data is None:
             data = torch.empty(lead + (inter,), dtype=torch.uint8, device=gate_up.device)
+        else:
+            _given(data, lead + (inter,), gate_up.device, "NVFP4 data")
         if scale is None:
             scale = torch.empty(lead + (2 * inter // 16,), dtype=torch.float8_e4m3fn, device=gate_up.device)
+        else:
+            _given(scale, lead + (2 * inter // 16,), gate_up.device, "NVFP4 scale")
     given = amax is not None
     if amax is None:
         amax = amax_out if amax_out is not None else torch.empty(1, dtype=torch.float32, device=gate_up.device)
@@ -520,6 +583,8 @@ def situ_glu_bwd_nvfp4(gate_up: torch.Tensor, routing_weights, grad_out: torch.T
     if want:
         if d_rw is None:
             d_rw = torch.empty(routing_weights.shape, dtype=routing_weights.dtype, device=gate_up.device)
+        else:
+            _given_drw(d_rw, routing_weights, gate_up.device)
         d_rw_flat = d_rw.view(-1)
         d_rw_stride = d_rw_flat.stride(0) if d_rw_flat.numel() > 1 else 1
     ws_bytes = abi.situ_glu_bwd_workspace_bytes(tokens, inter, mode, int(want))
