@@ -236,7 +236,7 @@ def source_digest() -> str:
     return h.hexdigest()
 
 
-E2E_CHUNK_ROWS = 2048  # rows per chunk of the host pipeline in the end-to-end measurement
+E2E_CHUNK_ROWS = 4096  # rows per chunk of the host pipeline in the end-to-end measurement
 
 
 def recorded_traffic(kernel: str, workload_name: str):

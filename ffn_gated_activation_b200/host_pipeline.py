@@ -28,7 +28,7 @@ class HostPipeline:
     chunk; buffers: chunks in flight (3: one uploading, one computing, one
     downloading)."""
 
-    def __init__(self, inter: int, dtype: torch.dtype, chunk_rows: int = 2048, device=None, buffers: int = 3,
+    def __init__(self, inter: int, dtype: torch.dtype, chunk_rows: int = 4096, device=None, buffers: int = 3,
                  rw_dtype: torch.dtype = torch.float32):
         if chunk_rows <= 0 or buffers < 1:
             raise ValueError("chunk_rows and buffers must be positive")
