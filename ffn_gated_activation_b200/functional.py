@@ -67,9 +67,11 @@ def _given(t: torch.Tensor, shape: tuple, device, what: str, dtype=None) -> torc
     if t.device != device:
         raise ValueError(f"{what} must be on {device}, got {t.device}")
     cols = shape[-1]
-    t2 = t if t.dim() == 2 else t.reshape(-1, cols)
-    if t2.numel() and (t2.data_ptr() != t.data_ptr() or t2.stride(1) != 1
-                       or (t2.shape[0] > 1 and t2.stride(0) < cols)):
+    try:
+        t2 = t if t.dim() == 2 else t.view(-1, cols)  # a view or nothing: never a copy
+    except RuntimeError:
+        raise ValueError(f"{what} must be viewable as [rows, {cols}]") from None
+    if t2.numel() and (t2.stride(1) != 1 or (t2.shape[0] > 1 and t2.stride(0) < cols)):
         raise ValueError(f"{what} must hold each row's elements adjacent, rows not overlapping")
     return t2
 
