@@ -172,6 +172,23 @@ def by_row_chunks(fn, rows: np.ndarray, chunk: int = 16):
     return np.concatenate(outs, axis=0)
 
 
+def check_ar(name, got, ref, mag):
+    """The attention-residual core's output against the oracle: bf16 by the
+    2^-8 relative rule (or a faithful neighbour), fp32 within 1e-5, each plus
+    2^-18 of the oracle's accumulation magnitude."""
+    y = as_f64(got)
+    err = np.abs(y - ref)
+    if got.dtype == np.uint16:
+        ok = (err <= 2.0 ** -8 * np.abs(ref) + 1e-6 + 2.0 ** -18 * mag) | bf16_faithful(got, ref)
+    else:
+        ok = err <= 1e-5 * np.abs(ref) + 2.0 ** -18 * mag + 1e-30
+    bad = np.flatnonzero(~ok)
+    if bad.size:
+        i = bad[0]
+        raise AssertionError(f"{name}: {bad.size} of {ok.size} out of tolerance; first at flat {i}: got "
+                             f"{y.flat[i]!r}, oracle {ref.flat[i]!r}, scale {mag.flat[i]!r}")
+
+
 def check_output(name: str, got: np.ndarray, ref: np.ndarray, cancel_scale: np.ndarray | None = None):
     """Assert the tolerance rule elementwise.  Returns counts: ``n``;
     ``faithful_only``, the bf16 elements that pass only as a neighbour of ref;

@@ -20,23 +20,9 @@ import workloads
 from ffn_gated_activation_b200 import abi
 import ffn_gated_activation_b200 as pkg
 
-from parity import as_f64, bf16_faithful, to_device, to_host
+from parity import check_ar, to_device, to_host
 
 pytestmark = pytest.mark.gpu
-
-
-def check_ar(name, got, ref, mag):
-    y = as_f64(got)
-    err = np.abs(y - ref)
-    if got.dtype == np.uint16:
-        ok = (err <= 2.0 ** -8 * np.abs(ref) + 1e-6 + 2.0 ** -18 * mag) | bf16_faithful(got, ref)
-    else:
-        ok = err <= 1e-5 * np.abs(ref) + 2.0 ** -18 * mag + 1e-30
-    bad = np.flatnonzero(~ok)
-    if bad.size:
-        i = bad[0]
-        raise AssertionError(f"{name}: {bad.size} of {ok.size} out of tolerance; first at flat {i}: got "
-                             f"{y.flat[i]!r}, oracle {ref.flat[i]!r}, scale {mag.flat[i]!r}")
 
 
 def run_ar(dev, T, B, H, with_prefix=True, dtype="bf16", out_dtype=torch.bfloat16, weights_bf16=False, seed=0,

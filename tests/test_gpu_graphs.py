@@ -19,7 +19,7 @@ import oracle
 import workloads
 import ffn_gated_activation_b200 as pkg
 
-from parity import check_dw, check_output, to_device, to_host
+from parity import check_ar, check_dw, check_output, to_device, to_host
 
 pytestmark = pytest.mark.gpu
 
@@ -145,6 +145,5 @@ def test_mixed_graph_replay(cuda_device):
     # the replayed attention mix against the oracle on the new sums (the
     # norm and projection weights are the captured ones)
     ref, mag, _ = oracle.load().attn_res(ar2["blocks"], ar2["prefix"], ar["norm_weight"], ar["proj_weight"], 1e-6)
-    from test_gpu_attn_res import check_ar
     check_ar("attention mix replay", got[5], ref, mag)
     del g
